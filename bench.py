@@ -1,0 +1,439 @@
+#!/usr/bin/env python3
+"""Benchmark: implicit-GEMM convolution forward on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one convolution forward pass (the whole hot path: one kernel
+launch) over one batch of the workload, inputs already resident in HBM.
+Between timed steps the inputs rotate over enough independent buffer sets to
+exceed twice the L2 cache, so every step reads x and w from DRAM.
+
+Metric: conv fwd TFLOP/s, FLOPs = 2 * N * Do * Ho * Wo * O * kD * kH * kW * C/groups
+(the "Convolutions" tutorial's count, section 4, extended to batch, depth and
+groups); also the fraction of the B200's dense fp16/bf16 tensor peak.
+
+With N > 1 GPUs (torchrun, one process per GPU) every rank runs the same
+workload on its own device (independent batches: weak scaling, no data-path
+collective); the time is the maximum over ranks and the value counts the
+FLOPs of all ranks.
+
+--impl reference times the CPU oracle (fp64 direct loop, the test-suite's
+checker) on the host cores over a bounded sample of the workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as WL  # noqa: E402
+
+METRIC = "conv fwd TFLOP/s (fp16/bf16) and % of B200 dense tensor peak, 1 GPU"
+SPEC_DENSE_TFLOPS = 2250.0          # B200 dense fp16/bf16, datasheet
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+# ---------------------------------------------------------------- counting
+
+def out_dims(wl):
+    import implicit_gemm_convolution_conv2d_b200 as C
+    return C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil)
+
+
+def conv_flops(wl, dims=None):
+    """Algorithmic FLOPs: 2 * N * Do*Ho*Wo * O * kD*kH*kW * C/groups (padding taps counted)."""
+    Do, Ho, Wo = dims if dims is not None else out_dims(wl)
+    return 2 * wl.N * Do * Ho * Wo * wl.O * wl.k[0] * wl.k[1] * wl.k[2] * (wl.C // wl.groups)
+
+
+def conv_bytes(wl, dims=None):
+    """Algorithmic bytes: x, w and y each moved once (the tutorial's intensity convention)."""
+    Do, Ho, Wo = dims if dims is not None else out_dims(wl)
+    e = WL.ELEM_BYTES[wl.dtype]
+    nx = wl.N * wl.D * wl.H * wl.W * wl.C
+    nw = wl.O * wl.k[0] * wl.k[1] * wl.k[2] * (wl.C // wl.groups)
+    ny = wl.N * Do * Ho * Wo * wl.O
+    return e * nx, e * nw, e * ny
+
+
+# ---------------------------------------------------------------- peaks / profiles
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "implicit_gemm_convolution_conv2d_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(workload, variant_name):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    if not os.path.isdir(PROFILE_DIR):
+        return None
+    src = kernel_source_hash()
+    for name in sorted(os.listdir(PROFILE_DIR)):
+        if not name.endswith((".txt", ".md")):
+            continue
+        with open(os.path.join(PROFILE_DIR, name)) as f:
+            text = f.read()
+        m = re.search(r"^traffic_record:\s*(\{.*\})\s*$", text, re.M)
+        if not m:
+            continue
+        try:
+            rec = json.loads(m.group(1))
+        except ValueError:
+            continue
+        if rec.get("workload") == workload and rec.get("kernel") == variant_name and rec.get("source") == src:
+            return rec.get("dram_bytes_per_launch_full")
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+        time.sleep(0.25)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(ws, backend):
+    import datetime
+    import torch.distributed as dist
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if ws > 1 else None
+
+
+def aggregate(dist, local_ms, device=None):
+    """(max time over ranks, number of ranks) -- the job's time is the slowest rank's."""
+    if dist is None:
+        return local_ms, 1
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item()), dist.get_world_size()
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------- our arm
+
+def bench_ours(args):
+    import implicit_gemm_convolution_conv2d_b200 as C
+
+    ws, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the CUDA path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(ws, "nccl")
+
+    wl = WL.WORKLOADS[args.workload]
+    dims = out_dims(wl)
+    flops = conv_flops(wl, dims)
+    xb, wb, yb = conv_bytes(wl, dims)
+    variant, bn, stages, ctas = C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil,
+                                       wl.groups, wl.dtype)
+    vname = C.VARIANT_NAMES[variant]
+
+    # inputs: seeded on the host (rank-dependent seed), copied once
+    x_h, w_h = WL.make_inputs(wl, seed=wl.seed + 1000 * rank)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per_set = xb + wb + yb
+    nsets = max(2, min(64, math.ceil(2 * l2 / per_set) + 1))
+    xs = [x_h.to(dev) for _ in range(nsets)]
+    wts = [w_h.to(dev) for _ in range(nsets)]
+    Do, Ho, Wo = dims
+    ys = [torch.empty((wl.N, Do, Ho, Wo, wl.O), dtype=x_h.dtype, device=dev) for _ in range(nsets)]
+    stream = torch.cuda.current_stream(dev)
+    geo = lambda i: (wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, *wl.k, wl.stride, wl.pad, wl.dil, wl.groups)
+    dcode = {"f32": 0, "f16": 1, "bf16": 2}[wl.dtype]
+    launches = 0
+
+    def step(i):
+        nonlocal launches
+        s = i % nsets
+        rc = C.conv_fwd_raw(xs[s].data_ptr(), wts[s].data_ptr(), ys[s].data_ptr(), geo(s), dcode,
+                            C.VARIANT_AUTO, stream.cuda_stream)
+        if rc:
+            raise C.ConvError(rc, "conv_fwd")
+        launches += 1
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if C.last_status() != 0:
+        raise SystemExit("bench.py: device status word set during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    launches = 0
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    clk = clocks.stop()
+    local_ms = ev0.elapsed_time(ev1)
+    timed_launches = launches
+    status = C.last_status()
+    if status != 0:
+        raise SystemExit("bench.py: device status word set during the timed region")
+    ms, nranks = aggregate(dist, local_ms, dev)
+    ms_per_step = ms / args.steps
+    value = nranks * flops * args.steps / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the host-buffer C entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        xp = x_h.pin_memory()
+        wp = w_h.pin_memory()
+        yp = torch.empty(ys[0].shape, dtype=x_h.dtype).pin_memory()
+        e_steps = max(3, min(args.steps, 20))
+        for _ in range(2):
+            C.conv_fwd_host(xp, wp, yp, xs[0], wts[0], ys[0], stride=wl.stride, padding=wl.pad,
+                            dilation=wl.dil, groups=wl.groups, stream=stream)
+        barrier(dist, dev)
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            C.conv_fwd_host(xp, wp, yp, xs[0], wts[0], ys[0], stride=wl.stride, padding=wl.pad,
+                            dilation=wl.dil, groups=wl.groups, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems, _ = aggregate(dist, e0.elapsed_time(e1), dev)
+        e2e = {"value": round(nranks * flops * e_steps / (ems * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": xb + wb, "d2h_bytes_per_step": yb, "steps": e_steps,
+               "ms_per_step": round(ems / e_steps, 5), "path": "conv_fwd_host (C ABI, pinned host buffers)"}
+
+    # ---- roofline of the (single) kernel
+    peaks, peak_src = measured_peaks()
+    kern_ms = local_ms / timed_launches
+    achieved_tflops = flops / (kern_ms * 1e-3) / 1e12
+    tensor_bound = wl.dtype in ("f16", "bf16") and flops / (xb + wb + yb) > 300
+    if wl.dtype == "f32":
+        sm_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
+        props = torch.cuda.get_device_properties(dev)
+        peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": round(achieved_tflops, 3), "peak": round(peak, 2),
+                "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
+    elif tensor_bound:
+        peak = float(peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": round(achieved_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved_tflops / peak, 4),
+                "peak_source": f"{peak_src} cuBLAS bf16 burst (MEASURED_PEAKS.json bf16_tflops)"}
+    else:
+        gbs = (xb + wb + yb) / (kern_ms * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(gbs / peak, 4), "peak_source": f"{peak_src} copy bandwidth (hbm_gbs)"}
+    roof["traffic"] = profiled_traffic(args.workload, vname)
+    roof["kernel"] = vname
+    roof["ms_per_launch"] = round(kern_ms, 5)
+
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": nranks, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "frac_of_dense_peak": round(value / nranks / SPEC_DENSE_TFLOPS, 4),
+        "config": {"workload": wl.name, "N": wl.N, "DHW": [wl.D, wl.H, wl.W], "C": wl.C, "O": wl.O,
+                   "kernel": list(wl.k), "stride": list(wl.stride), "pad": list(wl.pad), "dil": list(wl.dil),
+                   "groups": wl.groups, "out_DHW": list(dims), "gflop_per_step": round(flops / 1e9, 4),
+                   "global_batch": wl.N * nranks, "parallelism": f"independent batches x{nranks}",
+                   "variant": vname, "tile": [128, bn], "stages": stages, "ctas": ctas,
+                   "l2": f"inputs rotate over {nsets} buffer sets ({nsets * per_set / 2**20:.0f} MiB > 2x L2)"},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": timed_launches,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def _oracle_sample_step(wl, x, w, n_img):
+    import oracle
+    xs = x[:n_img].contiguous()
+    y, _ = oracle.conv_fwd(xs, w, wl.stride, wl.pad, wl.dil, wl.groups)
+    return y
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    """The oracle as it stands, on the host cores, over the first images of the
+    workload (as many as fit the time budget)."""
+    import oracle
+    x, w = WL.make_inputs(wl)
+    one = wl.with_(N=1)
+    f1 = conv_flops(one)
+    t0 = time.perf_counter()
+    _oracle_sample_step(wl, x, w, 1)
+    t1 = time.perf_counter() - t0
+    n_img = 1
+    total_t, total_f = t1, f1
+    while total_t < budget_s and n_img < wl.N:
+        k = min(wl.N - n_img, max(1, int((budget_s - total_t) / max(t1, 1e-3))))
+        t0 = time.perf_counter()
+        _oracle_sample_step(wl, x[n_img:], w, k)
+        total_t += time.perf_counter() - t0
+        total_f += f1 * k
+        n_img += k
+    return {"value": round(total_f / total_t / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+            "kind": "oracle", "sample": f"first {n_img} of {wl.N} images of {wl.name} ({total_t:.1f} s)"}
+
+
+def bench_reference(args):
+    """The reference arm for this build is the CPU oracle (fp64 direct loop)."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    wl = WL.WORKLOADS[args.workload]
+    x, w = WL.make_inputs(wl)
+    one = wl.with_(N=1)
+    f1 = conv_flops(one)
+    # one step = the oracle on one image of the workload (a bounded sample)
+    for i in range(args.warmup):
+        _oracle_sample_step(wl, x[i % wl.N:], w, 1)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        _oracle_sample_step(wl, x[i % wl.N:], w, 1)
+    dt = time.perf_counter() - t0
+    value = f1 * args.steps / dt / 1e12
+    out = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 0, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": wl.name, "sample": "one image per step"},
+           "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+                            "kind": "oracle", "sample": f"one image of {wl.name} per step, {args.steps} steps"},
+           "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=WL.HEADLINE, choices=sorted(WL.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
+    if args.impl == "reference":
+        bench_reference(args)
+    else:
+        bench_ours(args)
+
+
+if __name__ == "__main__":
+    main()

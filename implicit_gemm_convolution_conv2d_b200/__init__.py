@@ -1,0 +1,200 @@
+"""Implicit-GEMM convolution forward for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/conv_fwd.h``
+(``libconvfwd.so``, built in-tree from ``csrc/``).  This module only marshals
+arguments: shapes, pointers and the current CUDA stream.  Every step of the
+convolution runs in the library's CUDA kernels; there is no CPU path, and the
+module raises if the library is missing or the tensors are not on a CUDA
+device.
+
+Layouts are channels-last: x [N, D, H, W, C] (or [N, H, W, C] for 2-D),
+w [O, kD, kH, kW, C/groups] (or [O, kH, kW, C/groups]), y [N, Do, Ho, Wo, O].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["conv_fwd", "conv_fwd_host", "out_dims", "plan", "last_status", "strerror", "lib",
+           "CONV_F32", "CONV_F16", "CONV_BF16", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC_TMA",
+           "VARIANT_TC_GATHER", "ConvError"]
+
+CONV_F32, CONV_F16, CONV_BF16 = 0, 1, 2
+VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC_TMA, VARIANT_TC_GATHER = -1, 0, 1, 2
+VARIANT_NAMES = {VARIANT_SIMT: "simt_ffma", VARIANT_TC_TMA: "tcgen05_tma_im2col",
+                 VARIANT_TC_GATHER: "tcgen05_gather"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libconvfwd.so")
+_lib = None
+
+
+class ConvError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} ({code})" if what else f"{strerror(code)} ({code})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m implicit_gemm_convolution_conv2d_b200._build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i3 = ctypes.POINTER(ctypes.c_int)
+        vp, ci = ctypes.c_void_p, ctypes.c_int
+        geo = [ci] * 9 + [i3, i3, i3, ci, ci]
+        L.conv_out_dims.argtypes = [ci] * 6 + [i3, i3, i3, i3]
+        L.conv_fwd.argtypes = [vp, vp, vp] + geo + [vp]
+        L.conv_fwd_variant.argtypes = [vp, vp, vp] + geo + [ci, vp]
+        L.conv_fwd_host.argtypes = [vp] * 6 + geo + [vp]
+        L.conv_plan.argtypes = geo + [i3, i3, i3]
+        L.conv_last_status.argtypes = [vp]
+        L.conv_strerror.argtypes = [ci]
+        L.conv_strerror.restype = ctypes.c_char_p
+        for f in ("conv_out_dims", "conv_fwd", "conv_fwd_variant", "conv_fwd_host", "conv_plan",
+                  "conv_last_status", "conv_version"):
+            getattr(L, f).restype = ci
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().conv_strerror(int(code)).decode()
+
+
+def _i3(v):
+    return (ctypes.c_int * 3)(*[int(a) for a in v])
+
+
+def _triple(v, name, spatial_default=None):
+    if isinstance(v, int):
+        return (v, v, v) if spatial_default is None else (spatial_default, v, v)
+    v = tuple(int(a) for a in v)
+    if len(v) == 2:
+        return (spatial_default if spatial_default is not None else 1,) + v
+    if len(v) != 3:
+        raise ValueError(f"{name} must have 2 or 3 entries")
+    return v
+
+
+def _dtype_code(t):
+    import torch
+    code = {torch.float32: CONV_F32, torch.float16: CONV_F16, torch.bfloat16: CONV_BF16}.get(t.dtype)
+    if code is None:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return code
+
+
+def out_dims(D, H, W, kD, kH, kW, stride, pad, dil):
+    """(Do, Ho, Wo) as computed by the library (host only)."""
+    out = (ctypes.c_int * 3)()
+    rc = lib().conv_out_dims(D, H, W, kD, kH, kW, _i3(stride), _i3(pad), _i3(dil), out)
+    if rc:
+        raise ConvError(rc, "conv_out_dims")
+    return tuple(out)
+
+
+def _geometry(x, w, stride, padding, dilation):
+    two_d = x.dim() == 4
+    if two_d:
+        if w.dim() != 4:
+            raise ValueError("2-D input needs a [O, kH, kW, C/groups] weight")
+        N, H, W, C = x.shape
+        D = 1
+        O, kH, kW, Cg = w.shape
+        kD = 1
+        s = _triple(stride, "stride", 1)
+        p = _triple(padding, "padding", 0)
+        d = _triple(dilation, "dilation", 1)
+        if isinstance(stride, int):
+            s = (1, stride, stride)
+        if isinstance(padding, int):
+            p = (0, padding, padding)
+        if isinstance(dilation, int):
+            d = (1, dilation, dilation)
+    else:
+        if x.dim() != 5 or w.dim() != 5:
+            raise ValueError("x must be [N,D,H,W,C] and w [O,kD,kH,kW,C/groups]")
+        N, D, H, W, C = x.shape
+        O, kD, kH, kW, Cg = w.shape
+        s, p, d = _triple(stride, "stride"), _triple(padding, "padding"), _triple(dilation, "dilation")
+    return two_d, (int(N), int(D), int(H), int(W), int(C), int(O), int(kD), int(kH), int(kW), int(Cg)), s, p, d
+
+
+def conv_fwd(x, w, stride=1, padding=0, dilation=1, groups=1, *, out=None, variant=VARIANT_AUTO, stream=None):
+    """y = conv(x, w) on the current CUDA stream (or `stream`).  Returns y.
+
+    x, w: contiguous CUDA tensors of one dtype (float16, bfloat16 or float32).
+    `out` may supply a preallocated contiguous y.  `variant` forces a kernel
+    (VARIANT_*); the default lets the library choose.
+    """
+    import torch
+    if not (x.is_cuda and w.is_cuda):
+        raise ValueError("conv_fwd runs on CUDA tensors only")
+    if x.dtype != w.dtype:
+        raise TypeError("x and w must share a dtype")
+    two_d, (N, D, H, W, C, O, kD, kH, kW, Cg), s, p, d = _geometry(x, w, stride, padding, dilation)
+    if Cg * groups != C:
+        raise ValueError(f"weight has {Cg} channels per group but C={C}, groups={groups}")
+    Do, Ho, Wo = out_dims(D, H, W, kD, kH, kW, s, p, d)
+    shape = (N, Ho, Wo, O) if two_d else (N, Do, Ho, Wo, O)
+    if out is None:
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+    elif tuple(out.shape) != shape or out.dtype != x.dtype or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {x.dtype} tensor of shape {shape}")
+    x = x.contiguous()
+    w = w.contiguous()
+    st = stream if stream is not None else torch.cuda.current_stream(x.device)
+    with torch.cuda.device(x.device):
+        rc = lib().conv_fwd_variant(x.data_ptr(), w.data_ptr(), out.data_ptr(), N, D, H, W, C, O, kD, kH, kW,
+                                    _i3(s), _i3(p), _i3(d), int(groups), _dtype_code(x), int(variant),
+                                    st.cuda_stream)
+    if rc:
+        raise ConvError(rc, "conv_fwd")
+    return out
+
+
+def conv_fwd_raw(x_ptr, w_ptr, y_ptr, geom, dtype, variant=VARIANT_AUTO, stream_handle=0):
+    """The C entry point on raw device pointers: geom = (N,D,H,W,C,O,kD,kH,kW,stride,pad,dil,groups)."""
+    N, D, H, W, C, O, kD, kH, kW, s, p, d, g = geom
+    return lib().conv_fwd_variant(x_ptr, w_ptr, y_ptr, N, D, H, W, C, O, kD, kH, kW, _i3(s), _i3(p), _i3(d),
+                                  int(g), int(dtype), int(variant), stream_handle)
+
+
+def conv_fwd_host(x_host, w_host, y_host, x_dev, w_dev, y_dev, stride=1, padding=0, dilation=1, groups=1,
+                  stream=None):
+    """Host-buffer entry point: copies x, w in, runs, copies y out, waits.
+
+    x_host/w_host/y_host: CPU tensors (pinned for asynchronous copies);
+    x_dev/w_dev/y_dev: CUDA tensors of the same shapes (caller-owned scratch).
+    """
+    import torch
+    two_d, (N, D, H, W, C, O, kD, kH, kW, Cg), s, p, d = _geometry(x_host, w_host, stride, padding, dilation)
+    st = stream if stream is not None else torch.cuda.current_stream(x_dev.device)
+    with torch.cuda.device(x_dev.device):
+        rc = lib().conv_fwd_host(x_host.data_ptr(), w_host.data_ptr(), y_host.data_ptr(), x_dev.data_ptr(),
+                                 w_dev.data_ptr(), y_dev.data_ptr(), N, D, H, W, C, O, kD, kH, kW, _i3(s), _i3(p),
+                                 _i3(d), int(groups), _dtype_code(x_host), st.cuda_stream)
+    if rc:
+        raise ConvError(rc, "conv_fwd_host")
+    return y_host
+
+
+def plan(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype):
+    """(variant, BN, stages, ctas) the library would use; dtype is 'f32' | 'f16' | 'bf16'."""
+    code = {"f32": CONV_F32, "f16": CONV_F16, "bf16": CONV_BF16}[dtype]
+    bn, st, ct = (ctypes.c_int * 1)(), (ctypes.c_int * 1)(), (ctypes.c_int * 1)()
+    v = lib().conv_plan(N, D, H, W, C, O, *k, _i3(stride), _i3(pad), _i3(dil), int(groups), code, bn, st, ct)
+    if v < 0:
+        raise ConvError(v, "conv_plan")
+    return v, bn[0], st[0], ct[0]
+
+
+def last_status(stream=None) -> int:
+    """Wait for the stream, then read and clear the device status word (0 = ok)."""
+    import torch
+    st = stream if stream is not None else torch.cuda.current_stream()
+    return int(lib().conv_last_status(st.cuda_stream))

@@ -1,0 +1,514 @@
+// conv_fwd.cu -- the C ABI (include/conv_fwd.h): argument checks, kernel
+// choice and tiling, TMA tensor-map encoding, launches.  Nothing here touches
+// tensor data; every step of the convolution runs in the kernels of
+// conv_tc.cuh (f16/bf16, tcgen05 tensor cores) and conv_simt.cuh (f32).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/conv_fwd.h"
+#include "conv_simt.cuh"
+#include "conv_tc.cuh"
+
+namespace convfwd {
+namespace {
+
+constexpr int kVersion = 100;                       // 0.1.0
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per pipeline wait
+constexpr uint32_t kSmemBudget = 227 * 1024;        // max dynamic smem per CTA on sm_100
+constexpr int kMaxDevices = 64;
+
+struct Problem {
+  int N, D, H, W, C, O, kD, kH, kW;
+  int s[3], p[3], d[3];
+  int G, Cg, Og;
+  int Do, Ho, Wo;
+  long long M;
+  long long K;
+  int dtype;
+  size_t esize;
+  size_t x_bytes, w_bytes, y_bytes;
+};
+
+long long extent(long long in, int k, int s, int p, int d) {
+  const long long num = in + 2LL * p - static_cast<long long>(d) * (k - 1) - 1;
+  if (num < 0) return 0;
+  return num / s + 1;
+}
+
+int out_dims_impl(int D, int H, int W, int kD, int kH, int kW, const int stride[3], const int pad[3],
+                  const int dil[3], int out[3]) {
+  if (!stride || !pad || !dil || !out) return CONV_EINVAL;
+  const int in[3] = {D, H, W};
+  const int k[3] = {kD, kH, kW};
+  for (int i = 0; i < 3; ++i) {
+    if (in[i] <= 0 || k[i] <= 0 || stride[i] <= 0 || dil[i] <= 0 || pad[i] < 0) return CONV_EINVAL;
+    const long long e = extent(in[i], k[i], stride[i], pad[i], dil[i]);
+    if (e <= 0 || e > 0x7fffffffLL) return CONV_EINVAL;
+    out[i] = static_cast<int>(e);
+  }
+  return CONV_OK;
+}
+
+bool mul_ok(long long a, long long b, long long& r) {
+  if (a < 0 || b < 0) return false;
+  if (a != 0 && b > (1LL << 62) / a) return false;
+  r = a * b;
+  return true;
+}
+
+int make_problem(Problem& P, int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
+                 const int stride[3], const int pad[3], const int dil[3], int groups, int dtype) {
+  if (dtype != CONV_F32 && dtype != CONV_F16 && dtype != CONV_BF16) return CONV_EDTYPE;
+  if (N <= 0 || C <= 0 || O <= 0 || groups <= 0) return CONV_EINVAL;
+  if (C % groups != 0 || O % groups != 0) return CONV_EINVAL;
+  int out[3];
+  const int rc = out_dims_impl(D, H, W, kD, kH, kW, stride, pad, dil, out);
+  if (rc != CONV_OK) return rc;
+  P.N = N; P.D = D; P.H = H; P.W = W; P.C = C; P.O = O; P.kD = kD; P.kH = kH; P.kW = kW;
+  for (int i = 0; i < 3; ++i) { P.s[i] = stride[i]; P.p[i] = pad[i]; P.d[i] = dil[i]; }
+  P.G = groups; P.Cg = C / groups; P.Og = O / groups;
+  P.Do = out[0]; P.Ho = out[1]; P.Wo = out[2];
+  P.dtype = dtype;
+  P.esize = dtype == CONV_F32 ? 4 : 2;
+  long long nx, nw, ny, t;
+  if (!mul_ok(N, D, t) || !mul_ok(t, H, t) || !mul_ok(t, W, t) || !mul_ok(t, C, nx)) return CONV_EINVAL;
+  if (!mul_ok(kD, kH, t) || !mul_ok(t, kW, t) || !mul_ok(t, P.Cg, P.K)) return CONV_EINVAL;
+  if (!mul_ok(O, P.K, nw)) return CONV_EINVAL;
+  if (!mul_ok(N, P.Do, t) || !mul_ok(t, P.Ho, t) || !mul_ok(t, P.Wo, P.M) || !mul_ok(P.M, O, ny))
+    return CONV_EINVAL;
+  // kernel-side limits: K, per-row counts and tile counts are 32-bit
+  if (P.K > 0x7fffffffLL || P.M > (1LL << 46)) return CONV_EINVAL;
+  if (!mul_ok(nx, static_cast<long long>(P.esize), t) || !mul_ok(nw, static_cast<long long>(P.esize), t) ||
+      !mul_ok(ny, static_cast<long long>(P.esize), t))
+    return CONV_EINVAL;
+  P.x_bytes = static_cast<size_t>(nx) * P.esize;
+  P.w_bytes = static_cast<size_t>(nw) * P.esize;
+  P.y_bytes = static_cast<size_t>(ny) * P.esize;
+  return CONV_OK;
+}
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bn && b0 < a0 + an;
+}
+
+int check_pointers(const Problem& P, const void* x, const void* w, const void* y) {
+  if (!x || !w || !y) return CONV_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(y)) & 15)
+    return CONV_EALIGN;
+  if (overlaps(y, P.y_bytes, x, P.x_bytes) || overlaps(y, P.y_bytes, w, P.w_bytes)) return CONV_EALIAS;
+  return CONV_OK;
+}
+
+// ---------------------------------------------------------------- device info
+
+struct DeviceInfo {
+  bool init = false;
+  int sms = 0;
+  bool attrs_set = false;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+int current_device(int& dev) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CONV_ELAUNCH;
+  return CONV_OK;
+}
+
+int device_sms(int dev, int& sms) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_dev[dev].init) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return CONV_ELAUNCH;
+    g_dev[dev].sms = v;
+    g_dev[dev].init = true;
+  }
+  sms = g_dev[dev].sms;
+  return CONV_OK;
+}
+
+int set_kernel_attrs(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_dev[dev].attrs_set) return CONV_OK;
+  const int bytes = static_cast<int>(kSmemBudget);
+  cudaError_t e = cudaSuccess;
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_TMA, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_TMA, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return CONV_ELAUNCH;
+  g_dev[dev].attrs_set = true;
+  return CONV_OK;
+}
+
+// ---------------------------------------------------------------- driver API
+
+typedef CUresult (*PfnEncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+typedef CUresult (*PfnEncodeIm2col)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const int*, const int*, cuuint32_t, cuuint32_t,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DriverFns {
+  bool tried = false;
+  PfnEncodeTiled tiled = nullptr;
+  PfnEncodeIm2col im2col = nullptr;
+  int driver_version = 0;
+};
+DriverFns g_drv;
+
+const DriverFns& driver_fns() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_drv.tried) {
+    g_drv.tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_drv.tiled = reinterpret_cast<PfnEncodeTiled>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeIm2col", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_drv.im2col = reinterpret_cast<PfnEncodeIm2col>(f);
+    cudaDriverGetVersion(&g_drv.driver_version);
+  }
+  return g_drv;
+}
+
+// Drivers up to 13.1 mis-encode one descriptor field for tensors under
+// 128 KiB; clearing bit 21 of the second 64-bit word is the documented
+// remedy used by NVIDIA's CUTLASS (cute/atom/copy_traits_sm90_tma.hpp).
+void small_tensor_fixup(CUtensorMap& m, size_t tensor_bytes, int driver_version) {
+  if (driver_version <= 13010 && tensor_bytes < 131072) {
+    uint64_t* words = reinterpret_cast<uint64_t*>(&m);
+    words[1] &= ~(1ull << 21);
+  }
+}
+
+// ---------------------------------------------------------------- planning
+
+struct TcPlan {
+  int variant;
+  TcArgs args;
+  int ctas;
+  size_t smem;
+};
+
+int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+uint32_t next_pow2_cols(uint32_t v) {
+  uint32_t c = 32;
+  while (c < v) c <<= 1;
+  return c;
+}
+
+// Can the TMA im2col producer describe this problem?  The corner offsets of
+// the pixel bounding box and the per-tap offsets must fit the ranges of the
+// tensor rank (rank 4: [-128, 127]; rank 5: [-16, 15]); traversal strides
+// are at most 8; the pixel rows must be 16-byte strided (C % 8 == 0) and the
+// channel chunk a multiple of 16 elements for the MMA K step.
+bool tma_fits(const Problem& P, bool& rank5) {
+  if (P.dtype == CONV_F32) return false;
+  if (P.Cg % 16 != 0) return false;
+  rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
+  const int lo = rank5 ? -16 : -128, hi = rank5 ? 15 : 127;
+  const int ks[3] = {P.kD, P.kH, P.kW};
+  for (int i = rank5 ? 0 : 1; i < 3; ++i) {
+    if (P.s[i] > 8) return false;
+    const int lower = -P.p[i];
+    const long long upper = static_cast<long long>(P.p[i]) - static_cast<long long>(P.d[i]) * (ks[i] - 1);
+    const long long off = static_cast<long long>(P.d[i]) * (ks[i] - 1);
+    if (lower < lo || lower > hi || upper < lo || upper > hi || off > hi) return false;
+  }
+  if (P.N > 0x7fffffff / 2) return false;
+  return true;
+}
+
+int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
+  if (P.dtype == CONV_F32) return CONV_EUNSUPPORTED;
+  TcArgs& a = plan.args;
+  std::memset(&a, 0, sizeof(a));
+  a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.C = P.C; a.O = P.O;
+  a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
+  a.sd = P.s[0]; a.sh = P.s[1]; a.sw = P.s[2];
+  a.pd = P.p[0]; a.ph = P.p[1]; a.pw = P.p[2];
+  a.dd = P.d[0]; a.dh = P.d[1]; a.dw = P.d[2];
+  a.G = P.G; a.Cg = P.Cg; a.Og = P.Og;
+  a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
+  a.M = P.M;
+  a.K = static_cast<int>(P.K);
+  a.BN = std::min(256, round_up(P.Og, 32));
+  a.n_tiles = (P.Og + a.BN - 1) / a.BN;
+  const long long mt = (P.M + kBM - 1) / kBM;
+  const long long tt = mt * a.n_tiles * P.G;
+  if (tt > 0x7fffffffLL) return CONV_EINVAL;
+  a.m_tiles = static_cast<int>(mt);
+  a.total_tiles = static_cast<int>(tt);
+  bool rank5 = false;
+  if (variant == CONV_VARIANT_TC_TMA) {
+    if (!tma_fits(P, rank5)) return CONV_EUNSUPPORTED;
+    a.kc = (P.Cg % 64 == 0) ? 64 : (P.Cg % 32 == 0 ? 32 : 16);
+    a.cchunks = P.Cg / a.kc;
+    a.kblocks = P.kD * P.kH * P.kW * a.cchunks;
+    a.rank5 = rank5 ? 1 : 0;
+  } else {
+    a.kc = 64;
+    a.cchunks = 0;
+    a.kblocks = static_cast<int>((P.K + 63) / 64);
+    a.rank5 = 0;
+  }
+  a.layout_type = a.kc == 64 ? 2u : (a.kc == 32 ? 4u : 6u);
+  a.sbo = static_cast<uint32_t>(8 * a.kc * 2);
+  a.a_bytes = static_cast<uint32_t>(kBM * a.kc * 2);
+  a.b_bytes = static_cast<uint32_t>(a.BN * a.kc * 2);
+  a.stage_bytes = a.a_bytes + a.b_bytes;
+  const uint32_t avail = kSmemBudget - 1024 - static_cast<uint32_t>(sizeof(TcSmemTail)) - 64;
+  int stages = static_cast<int>(avail / a.stage_bytes);
+  stages = std::min(stages, 8);
+  if (stages < 2) return CONV_EUNSUPPORTED;
+  a.stages = stages;
+  const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
+  a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(a.BN >> 3) << 17) |
+            (static_cast<uint32_t>(kBM >> 4) << 24);
+  a.tmem_cols = next_pow2_cols(static_cast<uint32_t>(2 * a.BN));
+  a.timeout_ns = kWaitTimeoutNs;
+  plan.variant = variant;
+  plan.ctas = std::min(a.total_tiles, sms);
+  plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + 1024 + sizeof(TcSmemTail) + 64;
+  return CONV_OK;
+}
+
+int choose_variant(const Problem& P) {
+  if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
+  bool r5;
+  return tma_fits(P, r5) ? CONV_VARIANT_TC_TMA : CONV_VARIANT_TC_GATHER;
+}
+
+// ---------------------------------------------------------------- launches
+
+int encode_maps(const Problem& P, const TcArgs& a, const void* x, const void* w, CUtensorMap& mx,
+                CUtensorMap& mw) {
+  std::memset(&mx, 0, sizeof(mx));
+  std::memset(&mw, 0, sizeof(mw));
+  if (a.cchunks == 0) return CONV_OK;  // gather mode: maps unused
+  const DriverFns& drv = driver_fns();
+  if (!drv.tiled || !drv.im2col) return CONV_EDRIVER;
+  const CUtensorMapDataType dt =
+      P.dtype == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapSwizzle swz = a.kc == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                            : (a.kc == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  // x: dims innermost first (C, W, H[, D], N)
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t estr[5];
+  int lower[3], upper[3];
+  const int rank = a.rank5 ? 5 : 4;
+  const cuuint64_t eb = 2;
+  gdim[0] = P.C; gdim[1] = P.W; gdim[2] = P.H;
+  gstr[0] = eb * P.C;
+  gstr[1] = gstr[0] * P.W;
+  gstr[2] = gstr[1] * P.H;
+  estr[0] = 1; estr[1] = P.s[2]; estr[2] = P.s[1];
+  lower[0] = -P.p[2]; upper[0] = P.p[2] - P.d[2] * (P.kW - 1);
+  lower[1] = -P.p[1]; upper[1] = P.p[1] - P.d[1] * (P.kH - 1);
+  if (rank == 5) {
+    gdim[3] = P.D; gdim[4] = P.N;
+    gstr[3] = gstr[2] * P.D;
+    estr[3] = P.s[0]; estr[4] = 1;
+    lower[2] = -P.p[0]; upper[2] = P.p[0] - P.d[0] * (P.kD - 1);
+  } else {
+    gdim[3] = P.N;
+    estr[3] = 1;
+  }
+  CUresult r = drv.im2col(&mx, dt, rank, const_cast<void*>(x), gdim, gstr, lower, upper,
+                          static_cast<cuuint32_t>(a.kc), static_cast<cuuint32_t>(kBM), estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  small_tensor_fixup(mx, P.x_bytes, drv.driver_version);
+  // w viewed as [O, K] (K innermost)
+  cuuint64_t wdim[2] = {static_cast<cuuint64_t>(P.K), static_cast<cuuint64_t>(P.O)};
+  cuuint64_t wstr[1] = {static_cast<cuuint64_t>(P.K) * eb};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(a.kc), static_cast<cuuint32_t>(a.BN)};
+  cuuint32_t west[2] = {1, 1};
+  r = drv.tiled(&mw, dt, 2, const_cast<void*>(w), wdim, wstr, box, west, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  small_tensor_fixup(mw, P.w_bytes, drv.driver_version);
+  return CONV_OK;
+}
+
+int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w, void* y, cudaStream_t st,
+              int dev) {
+  int rc = set_kernel_attrs(dev);
+  if (rc != CONV_OK) return rc;
+  TcArgs a = plan.args;
+  a.x = x; a.w = w; a.y = y;
+  CUtensorMap mx, mw;
+  rc = encode_maps(P, a, x, w, mx, mw);
+  if (rc != CONV_OK) return rc;
+  const dim3 grid(plan.ctas), block(plan.variant == CONV_VARIANT_TC_TMA ? tc_threads<MODE_TMA>()
+                                                                         : tc_threads<MODE_GATHER>());
+  const bool bf = P.dtype == CONV_BF16;
+  if (plan.variant == CONV_VARIANT_TC_TMA) {
+    if (bf) conv_fwd_tc_kernel<MODE_TMA, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
+    else    conv_fwd_tc_kernel<MODE_TMA, false><<<grid, block, plan.smem, st>>>(mx, mw, a);
+  } else {
+    if (bf) conv_fwd_tc_kernel<MODE_GATHER, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
+    else    conv_fwd_tc_kernel<MODE_GATHER, false><<<grid, block, plan.smem, st>>>(mx, mw, a);
+  }
+  return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+}
+
+int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st) {
+  SimtArgs a;
+  a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.C = P.C; a.O = P.O;
+  a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
+  a.sd = P.s[0]; a.sh = P.s[1]; a.sw = P.s[2];
+  a.pd = P.p[0]; a.ph = P.p[1]; a.pw = P.p[2];
+  a.dd = P.d[0]; a.dh = P.d[1]; a.dw = P.d[2];
+  a.G = P.G; a.Cg = P.Cg; a.Og = P.Og;
+  a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
+  a.M = P.M; a.K = static_cast<int>(P.K);
+  a.x = x; a.w = w; a.y = y;
+  const long long mt = (P.M + kSimtBM - 1) / kSimtBM;
+  const int nt = (P.Og + kSimtBN - 1) / kSimtBN;
+  if (mt > 0x7fffffffLL || nt > 65535 || P.G > 65535) return CONV_EUNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>(mt), nt, P.G), block(kSimtThreads);
+  if (P.dtype == CONV_F32) conv_fwd_simt_kernel<float><<<grid, block, 0, st>>>(a);
+  else if (P.dtype == CONV_F16) conv_fwd_simt_kernel<__half><<<grid, block, 0, st>>>(a);
+  else conv_fwd_simt_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+}
+
+int run(const Problem& P, const void* x, const void* w, void* y, int variant, cudaStream_t st) {
+  int dev;
+  int rc = current_device(dev);
+  if (rc != CONV_OK) return rc;
+  if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P);
+  if (variant == CONV_VARIANT_SIMT) return launch_simt(P, x, w, y, st);
+  if (variant != CONV_VARIANT_TC_TMA && variant != CONV_VARIANT_TC_GATHER) return CONV_EINVAL;
+  int sms;
+  rc = device_sms(dev, sms);
+  if (rc != CONV_OK) return rc;
+  TcPlan plan;
+  rc = plan_tc(P, variant, sms, plan);
+  if (rc != CONV_OK) return rc;
+  return launch_tc(P, plan, x, w, y, st, dev);
+}
+
+}  // namespace
+}  // namespace convfwd
+
+using namespace convfwd;
+
+extern "C" {
+
+int conv_out_dims(int D, int H, int W, int kD, int kH, int kW, const int stride[3], const int pad[3],
+                  const int dil[3], int out[3]) {
+  return out_dims_impl(D, H, W, kD, kH, kW, stride, pad, dil, out);
+}
+
+int conv_fwd_variant(const void* x, const void* w, void* y, int N, int D, int H, int W, int C, int O, int kD,
+                     int kH, int kW, const int stride[3], const int pad[3], const int dil[3], int groups,
+                     int dtype, int variant, conv_stream_t stream) {
+  Problem P;
+  int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
+  if (rc != CONV_OK) return rc;
+  rc = check_pointers(P, x, w, y);
+  if (rc != CONV_OK) return rc;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_GATHER) return CONV_EINVAL;
+  return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int conv_fwd(const void* x, const void* w, void* y, int N, int D, int H, int W, int C, int O, int kD, int kH,
+             int kW, const int stride[3], const int pad[3], const int dil[3], int groups, int dtype,
+             conv_stream_t stream) {
+  return conv_fwd_variant(x, w, y, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype,
+                          CONV_VARIANT_AUTO, stream);
+}
+
+int conv_fwd_host(const void* x_host, const void* w_host, void* y_host, void* x_dev, void* w_dev, void* y_dev,
+                  int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
+                  const int pad[3], const int dil[3], int groups, int dtype, conv_stream_t stream) {
+  Problem P;
+  int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
+  if (rc != CONV_OK) return rc;
+  if (!x_host || !w_host || !y_host) return CONV_EINVAL;
+  rc = check_pointers(P, x_dev, w_dev, y_dev);
+  if (rc != CONV_OK) return rc;
+  if (overlaps(x_dev, P.x_bytes, w_dev, P.w_bytes)) return CONV_EALIAS;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(x_dev, x_host, P.x_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return CONV_ELAUNCH;
+  if (cudaMemcpyAsync(w_dev, w_host, P.w_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return CONV_ELAUNCH;
+  rc = run(P, x_dev, w_dev, y_dev, CONV_VARIANT_AUTO, st);
+  if (rc != CONV_OK) return rc;
+  if (cudaMemcpyAsync(y_host, y_dev, P.y_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return CONV_ELAUNCH;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return CONV_ELAUNCH;
+  return CONV_OK;
+}
+
+int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
+              const int pad[3], const int dil[3], int groups, int dtype, int* bn, int* stages, int* ctas) {
+  Problem P;
+  int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
+  if (rc != CONV_OK) return rc;
+  const int variant = choose_variant(P);
+  if (variant == CONV_VARIANT_SIMT) {
+    if (bn) *bn = kSimtBN;
+    if (stages) *stages = 1;
+    if (ctas) {
+      const long long mt = (P.M + kSimtBM - 1) / kSimtBM;
+      const long long c = mt * ((P.Og + kSimtBN - 1) / kSimtBN) * P.G;
+      *ctas = static_cast<int>(std::min<long long>(c, 0x7fffffffLL));
+    }
+    return variant;
+  }
+  int dev, sms = 148;
+  if (current_device(dev) == CONV_OK) device_sms(dev, sms);
+  TcPlan plan;
+  rc = plan_tc(P, variant, sms, plan);
+  if (rc != CONV_OK) return rc;
+  if (bn) *bn = plan.args.BN;
+  if (stages) *stages = plan.args.stages;
+  if (ctas) *ctas = plan.ctas;
+  return variant;
+}
+
+int conv_last_status(conv_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return CONV_ELAUNCH;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_conv_status, sizeof(v)) != cudaSuccess) return CONV_ELAUNCH;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_conv_status, &zero, sizeof(zero)) != cudaSuccess) return CONV_ELAUNCH;
+    return CONV_ETIMEOUT;
+  }
+  return CONV_OK;
+}
+
+const char* conv_strerror(int code) {
+  switch (code) {
+    case CONV_OK: return "ok";
+    case CONV_EINVAL: return "invalid argument";
+    case CONV_EDTYPE: return "unknown element type";
+    case CONV_EALIGN: return "buffer not 16-byte aligned";
+    case CONV_EALIAS: return "output overlaps an input";
+    case CONV_ELAUNCH: return "CUDA launch or copy failed";
+    case CONV_ETIMEOUT: return "kernel pipeline wait timed out";
+    case CONV_EUNSUPPORTED: return "variant cannot run this shape or type";
+    case CONV_EDRIVER: return "TMA tensor map encoding failed";
+    default: return "unknown error";
+  }
+}
+
+int conv_version(void) { return kVersion; }
+
+}  // extern "C"

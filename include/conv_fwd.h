@@ -1,0 +1,143 @@
+/*
+ * conv_fwd.h -- C ABI of the B200 (sm_100a) implicit-GEMM convolution forward.
+ *
+ * The operation (the "Convolutions" tutorial, sections 1 and 4, and its
+ * variants table in section 5; the MLX pull request "Add implicit matmul
+ * pathway for mx.conv3d", its description and benchmark table):
+ *
+ *   y[n,od,oh,ow,o] = sum_{kd,kh,kw,c} x[n, od*sd-pd+kd*dd, oh*sh-ph+kh*dh,
+ *                                        ow*sw-pw+kw*dw, g*C/G + c]
+ *                                     * w[o, kd, kh, kw, c]
+ *
+ * a cross-correlation (the filter is not flipped, as the tutorial's worked
+ * example fixes), with zero padding of pad[i] on both sides of spatial
+ * dimension i, g = o / (O/G), and output extents
+ *   Do = floor((D + 2*pd - dd*(kD-1) - 1) / sd) + 1   (likewise Ho, Wo).
+ * It is computed as an implicit GEMM (tutorial section 5, "Implicit GEMM"):
+ * M = N*Do*Ho*Wo output pixels by O/G output channels per group, reduced over
+ * K = kD*kH*kW*C/G, with the patch ("im2col") indices computed inside the
+ * kernel so that no patch matrix is ever stored.
+ *
+ * Layouts (all contiguous, row-major, channels last):
+ *   x  [N, D, H, W, C]            (NDHWC; a 2-D convolution is D = kD = 1)
+ *   w  [O, kD, kH, kW, C/groups]
+ *   y  [N, Do, Ho, Wo, O]
+ * Spatial parameter arrays are ordered (depth, height, width).
+ *
+ * Element types: CONV_F16 and CONV_BF16 run on the tcgen05 tensor cores with
+ * fp32 accumulation in tensor memory and round-to-nearest-even output;
+ * CONV_F32 runs an fp32 FFMA kernel (no TF32).  x, w and y share one type.
+ *
+ * Ownership: the caller owns every buffer.  conv_fwd allocates nothing, does
+ * not synchronise, and returns after queueing its work on `stream`.
+ * Thread safety: calls may come from several host threads.
+ *
+ * Errors: every entry point returns CONV_OK (0) or a negative code and never
+ * aborts the process; argument errors are found on the host before anything is
+ * queued.  Device-side failures (a pipeline wait that timed out) are recorded
+ * in a per-device status word read by conv_last_status().
+ */
+#ifndef CONV_FWD_H_
+#define CONV_FWD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (identical to cudaStream_t / CUstream). NULL is the
+ * legacy default stream. */
+typedef struct CUstream_st* conv_stream_t;
+
+typedef enum { CONV_F32 = 0, CONV_F16 = 1, CONV_BF16 = 2 } conv_dtype_t;
+
+enum {
+  CONV_OK = 0,
+  CONV_EINVAL = -1,      /* a non-positive size, stride or dilation, a negative
+                            pad, C or O not divisible by groups, an empty
+                            output, a NULL pointer, or sizes beyond 2^31-1
+                            elements per dimension product limits */
+  CONV_EDTYPE = -2,      /* unknown element type */
+  CONV_EALIGN = -3,      /* x, w or y not 16-byte aligned */
+  CONV_EALIAS = -4,      /* y overlaps x or w */
+  CONV_ELAUNCH = -5,     /* the CUDA runtime refused the launch or a copy */
+  CONV_ETIMEOUT = -6,    /* a kernel's pipeline wait ran out (device status) */
+  CONV_EUNSUPPORTED = -7,/* the requested kernel variant cannot run this shape */
+  CONV_EDRIVER = -8      /* the driver could not encode a TMA tensor map */
+};
+
+/* Kernel variants (for conv_fwd_variant and conv_plan). */
+enum {
+  CONV_VARIANT_AUTO = -1,
+  CONV_VARIANT_SIMT = 0,       /* fp32 FFMA implicit GEMM (any shape, any type) */
+  CONV_VARIANT_TC_TMA = 1,     /* tcgen05 + TMA im2col loads (C/G % 16 == 0) */
+  CONV_VARIANT_TC_GATHER = 2   /* tcgen05 + in-kernel gather (any C, any geometry) */
+};
+
+/* Output extents.  stride/pad/dil: 3 ints (d, h, w).  out: 3 ints (Do, Ho, Wo).
+ * Returns CONV_OK or CONV_EINVAL (non-positive input, kernel, stride or
+ * dilation, negative pad, or an empty output).  Host-only; needs no GPU. */
+int conv_out_dims(int D, int H, int W, int kD, int kH, int kW,
+                  const int stride[3], const int pad[3], const int dil[3],
+                  int out[3]);
+
+/* Forward convolution on device buffers x, w, y (see the layouts above).
+ * Queues the kernel on `stream`; returns CONV_OK or an error code (nothing is
+ * queued on an error).  The variant is chosen from the type and shape:
+ * f32 -> SIMT; f16/bf16 -> TC_TMA when C/G % 16 == 0 and the geometry fits a
+ * TMA im2col tensor map, else TC_GATHER. */
+int conv_fwd(const void* x, const void* w, void* y,
+             int N, int D, int H, int W, int C, int O,
+             int kD, int kH, int kW,
+             const int stride[3], const int pad[3], const int dil[3],
+             int groups, int dtype, conv_stream_t stream);
+
+/* conv_fwd with an explicit kernel variant (CONV_VARIANT_*).  Returns
+ * CONV_EUNSUPPORTED when that variant cannot run the shape or type
+ * (TC_TMA and TC_GATHER need f16/bf16; TC_TMA needs C/G % 16 == 0). */
+int conv_fwd_variant(const void* x, const void* w, void* y,
+                     int N, int D, int H, int W, int C, int O,
+                     int kD, int kH, int kW,
+                     const int stride[3], const int pad[3], const int dil[3],
+                     int groups, int dtype, int variant, conv_stream_t stream);
+
+/* The same computation on HOST buffers x_host, w_host, y_host.  The caller
+ * also provides device buffers x_dev, w_dev, y_dev of the matching sizes
+ * (the library allocates nothing).  Queues, on `stream`: the two host->device
+ * copies, the kernel, the device->host copy of y; then waits for the stream,
+ * so y_host holds the result on return.  Host buffers should be page-locked
+ * for the copies to be asynchronous. */
+int conv_fwd_host(const void* x_host, const void* w_host, void* y_host,
+                  void* x_dev, void* w_dev, void* y_dev,
+                  int N, int D, int H, int W, int C, int O,
+                  int kD, int kH, int kW,
+                  const int stride[3], const int pad[3], const int dil[3],
+                  int groups, int dtype, conv_stream_t stream);
+
+/* The variant conv_fwd would run for this shape and type (CONV_VARIANT_*), or
+ * a negative error code.  Also reports the output-tile width BN, the number of
+ * pipeline stages and the number of CTAs it would launch (any may be NULL).
+ * Queries the current device's SM count; queues nothing. */
+int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
+              const int stride[3], const int pad[3], const int dil[3],
+              int groups, int dtype, int* bn, int* stages, int* ctas);
+
+/* Waits for `stream`, then reads and clears the current device's status word.
+ * Returns CONV_OK, or CONV_ETIMEOUT if a kernel since the last call gave up on
+ * a pipeline wait (the kernel then wrote no further output and returned), or
+ * CONV_ELAUNCH if the stream itself reports an error. */
+int conv_last_status(conv_stream_t stream);
+
+/* Human-readable text for a return code (static storage). */
+const char* conv_strerror(int code);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int conv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONV_FWD_H_ */

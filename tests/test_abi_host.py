@@ -1,0 +1,125 @@
+"""The C ABI's host side (no GPU needed): symbols, extents, argument checks, planning."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "conv_fwd.h")
+
+
+@pytest.fixture(scope="module")
+def C():
+    from implicit_gemm_convolution_conv2d_b200 import _build
+    _build.build()
+    import implicit_gemm_convolution_conv2d_b200 as mod
+    mod.lib()
+    return mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(conv_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("conv_fwd", "conv_fwd_variant", "conv_fwd_host", "conv_out_dims", "conv_plan",
+              "conv_last_status", "conv_strerror", "conv_version"):
+        assert n in names, n
+
+
+def test_library_exports_every_declared_symbol(C):
+    nm = subprocess.run(["nm", "-D", "--defined-only", C.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = {ln.split()[-1] for ln in nm.stdout.splitlines() if ln.strip()}
+    for n in declared_functions():
+        assert n in exported, f"{n} declared in conv_fwd.h but not exported"
+        assert hasattr(C.lib(), n)
+
+
+def test_out_dims_match_oracle(C):
+    rng = np.random.default_rng(0)
+    n = 0
+    while n < 400:
+        dims = rng.integers(1, 40, 3)
+        k = rng.integers(1, 8, 3)
+        s = rng.integers(1, 4, 3)
+        p = rng.integers(0, 4, 3)
+        d = rng.integers(1, 4, 3)
+        try:
+            ref = oracle.out_dims(*dims, *k, s, p, d)
+        except ValueError:
+            with pytest.raises(C.ConvError):
+                C.out_dims(*dims, *k, s, p, d)
+            continue
+        assert C.out_dims(*dims, *k, s, p, d) == ref
+        n += 1
+
+
+def test_out_dims_pinned_values(C):
+    # tutorial: 224x224, 7x7, stride 2 -> 112x112 (pad 3)
+    assert C.out_dims(1, 224, 224, 1, 7, 7, (1, 2, 2), (0, 3, 3), (1, 1, 1)) == (1, 112, 112)
+
+
+def test_invalid_arguments_rejected_on_host(C):
+    L = C.lib()
+    i3 = lambda *v: (ctypes.c_int * 3)(*v)
+    s, p, d = i3(1, 1, 1), i3(0, 1, 1), i3(1, 1, 1)
+    X, Wt, Y = 0x10000, 0x20000, 0x40000       # never dereferenced: checks come first
+    call = lambda *a: L.conv_fwd(*a)
+    # non-positive sizes, empty batch
+    assert call(X, Wt, Y, 0, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
+    assert call(X, Wt, Y, 1, 1, 4, 4, 0, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
+    # C % groups, O % groups
+    assert call(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 3, 1, None) == -1
+    assert call(X, Wt, Y, 1, 1, 4, 4, 16, 18, 1, 3, 3, s, p, d, 4, 1, None) == -1
+    # empty output (kernel larger than padded input)
+    assert call(X, Wt, Y, 1, 1, 2, 2, 16, 16, 1, 5, 5, s, i3(0, 0, 0), d, 1, 1, None) == -1
+    # bad stride / dilation / pad
+    assert call(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, i3(1, 0, 1), p, d, 1, 1, None) == -1
+    assert call(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, i3(0, -1, 1), d, 1, 1, None) == -1
+    assert call(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, i3(1, 1, 0), 1, 1, None) == -1
+    # dtype
+    assert call(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 9, None) == -2
+    # NULL, misaligned, aliasing
+    assert call(0, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
+    assert call(X + 8, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -3
+    assert call(X, Wt, X + 16, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -4
+    assert call(X, Wt, Wt, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -4
+    # overflow of the element count
+    big = 1 << 30
+    assert call(X, Wt, Y, big, big, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
+    # unknown variant
+    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 5, None) == -1
+
+
+def test_strerror_covers_codes(C):
+    for code in range(0, -9, -1):
+        assert C.strerror(code) and C.strerror(code) != "unknown error"
+    assert C.strerror(-99) == "unknown error"
+
+
+def test_variant_plan(C):
+    plan = lambda *a: C.plan(*a)
+    v, bn, st, _ = plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")
+    assert v == C.VARIANT_TC_TMA and bn == 256 and st >= 3
+    v, bn, _, _ = plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
+    assert v == C.VARIANT_TC_GATHER and bn == 64
+    v, bn, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
+    assert v == C.VARIANT_TC_GATHER and bn == 96
+    v, _, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f32")
+    assert v == C.VARIANT_SIMT
+    # 3-D with pad beyond the rank-5 corner range goes to the gather kernel
+    v, _, _, _ = plan(1, 40, 8, 8, 64, 64, (3, 3, 3), (1, 1, 1), (17, 1, 1), (1, 1, 1), 1, "f16")
+    assert v == C.VARIANT_TC_GATHER
+    # channel chunks of 32 and 16
+    assert plan(2, 64, 64, 64, 32, 64, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA
+    assert plan(1, 1, 9, 9, 48, 96, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 3, "f16")[0] == C.VARIANT_TC_TMA

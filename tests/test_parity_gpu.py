@@ -1,0 +1,215 @@
+"""CUDA path vs oracle, element by element, through the C ABI (needs a B200)."""
+from __future__ import annotations
+
+import json
+import os
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as WL
+from tests.parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+C = pytest.importorskip("implicit_gemm_convolution_conv2d_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    assert os.path.exists(C.LIB_PATH), "CUDA library not built"
+    yield
+    assert C.last_status() == 0
+
+
+def run_gpu(x, w, wl, variant, guard=64):
+    """Run through the C ABI into a guard-banded output; check the guards."""
+    xd, wd = x.cuda(), w.cuda()
+    Do, Ho, Wo = C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil)
+    n = wl.N * Do * Ho * Wo * wl.O
+    buf = torch.full((n + 2 * guard,), 0, dtype=torch.int16 if x.element_size() == 2 else torch.int32,
+                     device="cuda")
+    buf.fill_(0x5A5A if x.element_size() == 2 else 0x5A5A5A5A)
+    y = buf[guard:guard + n].view(x.dtype).view(wl.N, Do, Ho, Wo, wl.O)
+    rc = C.conv_fwd_raw(xd.data_ptr(), wd.data_ptr(), y.data_ptr(),
+                        (wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, *wl.k, wl.stride, wl.pad, wl.dil, wl.groups),
+                        {"f32": 0, "f16": 1, "bf16": 2}[wl.dtype], variant,
+                        torch.cuda.current_stream().cuda_stream)
+    assert rc == 0, C.strerror(rc)
+    torch.cuda.synchronize()
+    assert C.last_status() == 0, "device status word set (pipeline timeout)"
+    g = buf.cpu()
+    pat = 0x5A5A if x.element_size() == 2 else 0x5A5A5A5A
+    assert torch.all(g[:guard] == pat) and torch.all(g[guard + n:] == pat), "write outside y"
+    return y.cpu()
+
+
+def variants_for(wl):
+    vs = []
+    if wl.dtype == "f32":
+        return [C.VARIANT_SIMT]
+    vs.append(C.VARIANT_TC_GATHER)
+    if (wl.C // wl.groups) % 16 == 0:
+        vs.append(C.VARIANT_TC_TMA)
+    return vs
+
+
+# Small geometries: several 128-row tiles with a ragged tail, every stride /
+# pad / dilation / groups combination the kernels branch on.
+SMALL = [
+    WL.case(2, 1, 13, 11, 16, 32, (1, 3, 3), pad=(0, 1, 1), name="2d_c16_o32"),
+    WL.case(1, 1, 17, 19, 64, 64, (1, 3, 3), (1, 2, 2), (0, 1, 1), name="2d_s2"),
+    WL.case(3, 1, 9, 10, 32, 48, (1, 3, 3), dil=(1, 2, 2), name="2d_dil2_o48"),
+    WL.case(2, 1, 15, 15, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), name="stem_like"),
+    WL.case(2, 1, 8, 8, 21, 21, (1, 3, 3), pad=(0, 1, 1), name="c21"),
+    WL.case(2, 1, 10, 10, 64, 64, (1, 3, 3), pad=(0, 1, 1), groups=2, name="groups2"),
+    WL.case(2, 1, 10, 10, 48, 96, (1, 3, 3), pad=(0, 1, 1), groups=3, name="groups3_cg16"),
+    WL.case(2, 1, 9, 9, 32, 32, (1, 3, 3), pad=(0, 1, 1), groups=32, name="depthwise"),
+    WL.case(1, 1, 12, 12, 32, 300, (1, 1, 1), name="o300_two_ntiles"),
+    WL.case(2, 1, 9, 9, 64, 96, (1, 1, 1), name="pointwise"),
+    WL.case(1, 1, 3, 4, 16, 16, (1, 5, 5), pad=(0, 2, 2), name="kernel_larger_than_input"),
+    WL.case(1, 1, 5, 5, 16, 16, (1, 3, 3), pad=(0, 1, 1), name="m_below_tile"),
+    WL.case(1, 1, 11, 7, 256, 64, (1, 3, 3), pad=(0, 1, 1), name="k2304"),
+    WL.case(2, 5, 6, 7, 16, 32, (3, 3, 3), pad=(1, 1, 1), name="3d_c16"),
+    WL.case(1, 6, 7, 8, 64, 128, (3, 3, 3), (2, 2, 2), (1, 1, 1), name="3d_s2"),
+    WL.case(1, 6, 7, 8, 64, 128, (3, 1, 1), pad=(1, 0, 0), name="3d_k311"),
+    WL.case(1, 6, 7, 8, 64, 128, (1, 3, 3), pad=(0, 1, 1), name="3d_k133"),
+    WL.case(1, 5, 6, 5, 32, 64, (3, 3, 3), pad=(1, 1, 1), name="3d_c32"),
+    WL.case(1, 4, 5, 6, 65, 65, (3, 3, 3), pad=(1, 1, 1), name="3d_c65"),
+    WL.case(2, 4, 5, 6, 3, 32, (3, 3, 3), pad=(1, 1, 1), name="3d_c3"),
+    WL.case(1, 7, 6, 9, 16, 16, (2, 3, 2), (2, 2, 1), (1, 0, 2), (2, 1, 3), name="3d_mixed"),
+    WL.case(1, 1, 8, 8, 8, 8, (1, 3, 3), (1, 3, 3), (0, 3, 3), (1, 3, 3), name="s3_d3_p3"),
+]
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_small_sweep(wl, dtype):
+    wl = wl.with_(dtype=dtype, seed=zlib.crc32(wl.name.encode()) % 1000)
+    x, w = WL.make_inputs(wl)
+    y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups)
+    for v in variants_for(wl):
+        y = run_gpu(x, w, wl, v)
+        assert_parity(y, y_ref, s_ref, dtype, f"{wl.name}/{dtype}/{C.VARIANT_NAMES[v]}")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_tutorial_example_on_gpu(dtype):
+    """The tutorial's worked example through the CUDA path: exactly -4 everywhere."""
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "tutorial_tiny_example.json")))
+    dt = WL.TORCH_DTYPE[dtype]
+    x = torch.tensor(g["x_hw"], dtype=dt).reshape(1, 1, 3, 3, 1)
+    w = torch.tensor(g["k_hw"], dtype=dt).reshape(1, 1, 2, 2, 1)
+    wl = WL.case(1, 1, 3, 3, 1, 1, (1, 2, 2), dtype=dtype)
+    for v in ([C.VARIANT_SIMT] if dtype == "f32" else [C.VARIANT_TC_GATHER, C.VARIANT_SIMT]):
+        y = run_gpu(x, w, wl, v)
+        assert torch.equal(y.double().reshape(2, 2), torch.tensor(g["y_hw"], dtype=torch.float64)), (v, y)
+
+
+def test_auto_variant_choice():
+    assert C.plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_TMA
+    assert C.plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
+    assert C.plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f32")[0] == C.VARIANT_SIMT
+
+
+def test_python_api_2d_and_3d():
+    wl = WL.case(2, 1, 12, 10, 64, 64, (1, 3, 3), pad=(0, 1, 1), dtype="bf16", seed=5)
+    x, w = WL.make_inputs(wl)
+    y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups)
+    y2 = C.conv_fwd(x[:, 0].cuda(), w[:, 0].cuda(), stride=1, padding=1)
+    assert y2.shape == (2, 12, 10, 64)
+    assert_parity(y2.cpu(), y_ref[:, 0], s_ref[:, 0], "bf16", "2-D api")
+    y3 = C.conv_fwd(x.cuda(), w.cuda(), stride=(1, 1, 1), padding=(0, 1, 1))
+    assert torch.equal(y3[:, 0].cpu(), y2.cpu())
+
+
+def test_host_buffer_entry_point():
+    wl = WL.case(2, 1, 14, 14, 64, 128, (1, 3, 3), pad=(0, 1, 1), dtype="f16", seed=6)
+    x, w = WL.make_inputs(wl)
+    xh, wh = x.pin_memory(), w.pin_memory()
+    Do, Ho, Wo = C.out_dims(1, 14, 14, 1, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    yh = torch.empty((2, Do, Ho, Wo, 128), dtype=x.dtype).pin_memory()
+    xd, wd = torch.empty_like(x, device="cuda"), torch.empty_like(w, device="cuda")
+    yd = torch.empty(yh.shape, dtype=x.dtype, device="cuda")
+    C.conv_fwd_host(xh, wh, yh, xd, wd, yd, stride=(1, 1, 1), padding=(0, 1, 1))
+    ydev = C.conv_fwd(x.cuda(), w.cuda(), stride=(1, 1, 1), padding=(0, 1, 1))
+    assert torch.equal(yh, ydev.cpu())
+
+
+def test_errors_queue_nothing():
+    x = torch.zeros(1, 1, 4, 4, 16, dtype=torch.float16, device="cuda")
+    w = torch.zeros(16, 1, 3, 3, 16, dtype=torch.float16, device="cuda")
+    geom = (1, 1, 4, 4, 16, 16, 1, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1), 1)
+    y = torch.zeros(1, 1, 4, 4, 16, dtype=torch.float16, device="cuda")
+    assert C.conv_fwd_raw(x.data_ptr(), w.data_ptr(), x.data_ptr(), geom, 1) == -4       # alias
+    assert C.conv_fwd_raw(x.data_ptr() + 2, w.data_ptr(), y.data_ptr(), geom, 1) == -3   # align
+    assert C.conv_fwd_raw(x.data_ptr(), w.data_ptr(), y.data_ptr(), geom, 7) == -2       # dtype
+    assert C.conv_fwd_raw(x.data_ptr(), w.data_ptr(), y.data_ptr(), geom, 0, C.VARIANT_TC_TMA) == -7
+    bad = (1, 1, 4, 4, 16, 16, 1, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1), 3)               # C % groups
+    assert C.conv_fwd_raw(x.data_ptr(), w.data_ptr(), y.data_ptr(), bad, 1) == -1
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(y) == 0
+
+
+# ---------------------------------------------------------------------------
+# The named workloads.  Reduced batch: full oracle, every element.  Full size
+# (the benchmark's launch configuration): sampled elements from the oracle,
+# including the first and last output tile and image borders.
+# ---------------------------------------------------------------------------
+
+def _reduced(wl, max_macs=3e9):
+    """Cut the batch to one image, then the depth (3-D) until the oracle's
+    multiply-adds fit the budget; spatial tiling and channels are kept."""
+    wl = wl.with_(N=1)
+
+    def macs(w):
+        Do, Ho, Wo = oracle.out_dims(w.D, w.H, w.W, *w.k, w.stride, w.pad, w.dil)
+        return Do * Ho * Wo * w.O * w.k[0] * w.k[1] * w.k[2] * (w.C // w.groups)
+
+    while macs(wl) > max_macs and wl.D > 4:
+        wl = wl.with_(D=wl.D // 2)
+    return wl
+
+
+@pytest.mark.parametrize("name", list(WL.WORKLOADS))
+def test_workload_reduced_batch(name):
+    wl = _reduced(WL.WORKLOADS[name])
+    x, w = WL.make_inputs(wl)
+    y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups)
+    y = run_gpu(x, w, wl, C.VARIANT_AUTO)
+    assert_parity(y, y_ref, s_ref, wl.dtype, name)
+
+
+def _sample_indices(shape, rng, n_random=6000):
+    N, Do, Ho, Wo, O = shape
+    total = N * Do * Ho * Wo * O
+    idx = [rng.integers(0, total, n_random)]
+    M = N * Do * Ho * Wo
+    # first and last 128-row tiles, all channels
+    for m0 in (0, max(0, M - 128)):
+        rows = np.arange(m0, min(M, m0 + 128))
+        idx.append((rows[:, None] * O + np.arange(O)[None, :]).ravel())
+    # border row of the last image
+    rows = ((N - 1) * Do * Ho * Wo) + np.arange(Wo)
+    idx.append((rows[:, None] * O + rng.integers(0, O, (Wo, 4))).ravel())
+    return np.unique(np.concatenate(idx))
+
+
+@pytest.mark.parametrize("name", list(WL.WORKLOADS))
+def test_workload_full_size_sampled(name):
+    wl = WL.WORKLOADS[name]
+    x, w = WL.make_inputs(wl)
+    y = C.conv_fwd(x.cuda(), w.cuda(), stride=wl.stride, padding=wl.pad, dilation=wl.dil, groups=wl.groups)
+    torch.cuda.synchronize()
+    assert C.last_status() == 0
+    rng = np.random.default_rng(0)
+    idx = _sample_indices(tuple(y.shape), rng)
+    y_ref, s_ref = oracle.conv_fwd_points(x, w, idx, wl.stride, wl.pad, wl.dil, wl.groups)
+    yv = y.reshape(-1)[torch.as_tensor(idx, device="cuda")].cpu()
+    assert_parity(yv, y_ref, s_ref, wl.dtype, name)
+    assert torch.isfinite(y.float()).all()
