@@ -149,7 +149,9 @@ def test_errors_queue_nothing():
     assert C.conv_fwd_raw(x.data_ptr(), w.data_ptr(), x.data_ptr(), geom, 1) == -4       # alias
     assert C.conv_fwd_raw(x.data_ptr() + 2, w.data_ptr(), y.data_ptr(), geom, 1) == -3   # align
     assert C.conv_fwd_raw(x.data_ptr(), w.data_ptr(), y.data_ptr(), geom, 7) == -2       # dtype
-    assert C.conv_fwd_raw(x.data_ptr(), w.data_ptr(), y.data_ptr(), geom, 0, C.VARIANT_TC_TMA) == -7
+    x32, w32, y32 = x.float(), w.float(), y.float()
+    assert C.conv_fwd_raw(x32.data_ptr(), w32.data_ptr(), y32.data_ptr(), geom, 0, C.VARIANT_TC_TMA) == -7
+    assert C.conv_fwd_raw(x32.data_ptr(), w32.data_ptr(), y32.data_ptr(), geom, 0, C.VARIANT_TC_GATHER) == -7
     bad = (1, 1, 4, 4, 16, 16, 1, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1), 3)               # C % groups
     assert C.conv_fwd_raw(x.data_ptr(), w.data_ptr(), y.data_ptr(), bad, 1) == -1
     torch.cuda.synchronize()
