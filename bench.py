@@ -247,8 +247,9 @@ def bench_ours(args):
     def step(i):
         nonlocal launches
         s = i % nsets
+        # the launch goes to the current stream (the capture stream while a graph is recorded)
         rc = C.conv_fwd_raw(xs[s].data_ptr(), wts[s].data_ptr(), ys[s].data_ptr(), geo(s), dcode,
-                            C.VARIANT_AUTO, stream.cuda_stream)
+                            C.VARIANT_AUTO, torch.cuda.current_stream(dev).cuda_stream)
         if rc:
             raise C.ConvError(rc, "conv_fwd")
         launches += 1
@@ -259,6 +260,29 @@ def bench_ours(args):
     if C.last_status() != 0:
         raise SystemExit("bench.py: device status word set during warm-up")
 
+    # eager launches (host overhead included) -- reported beside the graph time
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n_eager = min(args.steps, 20)
+    e0.record(stream)
+    for i in range(n_eager):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    eager_ms = e0.elapsed_time(e1) / n_eager
+
+    # the K timed launches, recorded once through the same C-ABI calls into a
+    # CUDA graph, so that the timed region measures the kernels rather than
+    # the Python/ctypes call overhead of each launch
+    graph = None
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(args.steps):
+                step(args.warmup + i)
+        graph.replay()  # untimed: one more warm-up pass over every buffer set
+        torch.cuda.synchronize(dev)
+
     clocks = ClockSampler(local)
     clocks.start()
     barrier(dist, dev)
@@ -267,8 +291,12 @@ def bench_ours(args):
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    for i in range(args.steps):
-        step(args.warmup + i)
+    if graph is not None:
+        graph.replay()
+        launches = args.steps
+    else:
+        for i in range(args.steps):
+            step(args.warmup + i)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(dist, dev)
@@ -345,6 +373,8 @@ def bench_ours(args):
                    "variant": vname, "tile": [128, bn], "stages": stages, "ctas": ctas,
                    "l2": f"inputs rotate over {nsets} buffer sets ({nsets * per_set / 2**20:.0f} MiB > 2x L2)"},
         "roofline": roof,
+        "launch": "cuda_graph_of_steps" if graph is not None else "eager",
+        "eager_ms_per_step": round(eager_ms, 5),
         "e2e": e2e,
         "gpu_launches": timed_launches,
         "clocks": clk,
@@ -426,6 +456,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps

@@ -17,12 +17,14 @@ import os
 
 __all__ = ["conv_fwd", "conv_fwd_host", "out_dims", "plan", "last_status", "strerror", "lib",
            "CONV_F32", "CONV_F16", "CONV_BF16", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC_TMA",
-           "VARIANT_TC_GATHER", "ConvError"]
+           "VARIANT_TC_GATHER", "VARIANT_TC_TMA_PAIR", "VARIANT_TC_HALO", "VARIANT_TC_HALO_PAIR", "ConvError"]
 
 CONV_F32, CONV_F16, CONV_BF16 = 0, 1, 2
-VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC_TMA, VARIANT_TC_GATHER = -1, 0, 1, 2
+VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC_TMA, VARIANT_TC_GATHER, VARIANT_TC_TMA_PAIR = -1, 0, 1, 2, 3
+VARIANT_TC_HALO, VARIANT_TC_HALO_PAIR = 4, 5
 VARIANT_NAMES = {VARIANT_SIMT: "simt_ffma", VARIANT_TC_TMA: "tcgen05_tma_im2col",
-                 VARIANT_TC_GATHER: "tcgen05_gather"}
+                 VARIANT_TC_GATHER: "tcgen05_gather", VARIANT_TC_TMA_PAIR: "tcgen05_tma_im2col_pair",
+                 VARIANT_TC_HALO: "tcgen05_tma_halo", VARIANT_TC_HALO_PAIR: "tcgen05_tma_halo_pair"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libconvfwd.so")
@@ -52,10 +54,11 @@ def lib() -> ctypes.CDLL:
         L.conv_fwd_host.argtypes = [vp] * 6 + geo + [vp]
         L.conv_plan.argtypes = geo + [i3, i3, i3]
         L.conv_last_status.argtypes = [vp]
+        L.conv_debug_inject_stall.argtypes = [ctypes.c_ulonglong]
         L.conv_strerror.argtypes = [ci]
         L.conv_strerror.restype = ctypes.c_char_p
         for f in ("conv_out_dims", "conv_fwd", "conv_fwd_variant", "conv_fwd_host", "conv_plan",
-                  "conv_last_status", "conv_version"):
+                  "conv_last_status", "conv_version", "conv_debug_inject_stall"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
@@ -191,6 +194,13 @@ def plan(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype):
     if v < 0:
         raise ConvError(v, "conv_plan")
     return v, bn[0], st[0], ct[0]
+
+
+def inject_stall(timeout_ns: int) -> None:
+    """Test hook: the next tensor-core launch times out after `timeout_ns` on purpose."""
+    rc = lib().conv_debug_inject_stall(int(timeout_ns))
+    if rc:
+        raise ConvError(rc, "conv_debug_inject_stall")
 
 
 def last_status(stream=None) -> int:

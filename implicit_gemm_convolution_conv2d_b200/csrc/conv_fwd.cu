@@ -6,11 +6,13 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/conv_fwd.h"
+#include "conv_halo.cuh"
 #include "conv_simt.cuh"
 #include "conv_tc.cuh"
 
@@ -21,6 +23,7 @@ constexpr int kVersion = 100;                       // 0.1.0
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per pipeline wait
 constexpr uint32_t kSmemBudget = 227 * 1024;        // max dynamic smem per CTA on sm_100
 constexpr int kMaxDevices = 64;
+constexpr long long kMaxResidentB = 96 * 1024;              // weights kept in smem by the gather kernel
 
 struct Problem {
   int N, D, H, W, C, O, kD, kH, kW;
@@ -111,6 +114,8 @@ struct DeviceInfo {
   bool init = false;
   int sms = 0;
   bool attrs_set = false;
+  size_t pair_smem = 0;     // dynamic smem the cached cluster count was measured for
+  int pair_clusters = 0;    // CTA pairs that fit on the device at once
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
@@ -142,6 +147,12 @@ int set_kernel_attrs(int dev) {
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_TMA, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return CONV_ELAUNCH;
   g_dev[dev].attrs_set = true;
   return CONV_OK;
@@ -197,6 +208,7 @@ void small_tensor_fixup(CUtensorMap& m, size_t tensor_bytes, int driver_version)
 
 struct TcPlan {
   int variant;
+  bool pair;      // CTA-pair (cta_group::2) tiles of 256 rows
   TcArgs args;
   int ctas;
   size_t smem;
@@ -232,7 +244,81 @@ bool tma_fits(const Problem& P, bool& rank5) {
   return true;
 }
 
+// Can the halo kernel run this problem?  Stride 1, 64-channel chunks, the
+// halo box inside the TMA box limits (256 per dimension), rank 4 or 5.
+constexpr int kHaloTileH = 16, kHaloTileW = 8;
+
+bool halo_fits(const Problem& P, bool& rank5) {
+  if (P.dtype == CONV_F32 || P.Cg % 64 != 0) return false;
+  if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1) return false;
+  rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
+  const long long hw = kHaloTileW + static_cast<long long>(P.d[2]) * (P.kW - 1);
+  const long long hh = kHaloTileH + static_cast<long long>(P.d[1]) * (P.kH - 1);
+  if (hw > 256 || hh > 256) return false;
+  if (hw * hh * 128 > 64 * 1024) return false;  // two slots must leave room for the weight ring
+  if (P.N > 0x3fffffff) return false;
+  return true;
+}
+
+int plan_halo(const Problem& P, bool pair, int sms, TcPlan& plan) {
+  bool rank5 = false;
+  if (!halo_fits(P, rank5)) return CONV_EUNSUPPORTED;
+  TcArgs& a = plan.args;
+  std::memset(&a, 0, sizeof(a));
+  a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.C = P.C; a.O = P.O;
+  a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
+  a.sd = P.s[0]; a.sh = P.s[1]; a.sw = P.s[2];
+  a.pd = P.p[0]; a.ph = P.p[1]; a.pw = P.p[2];
+  a.dd = P.d[0]; a.dh = P.d[1]; a.dw = P.d[2];
+  a.G = P.G; a.Cg = P.Cg; a.Og = P.Og;
+  a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
+  a.M = P.M;
+  a.K = static_cast<int>(P.K);
+  a.BN = std::min(256, round_up(P.Og, 32));
+  a.n_tiles = (P.Og + a.BN - 1) / a.BN;
+  a.tile_h = kHaloTileH;
+  a.tile_w = kHaloTileW;
+  a.tiles_h = (P.Ho + (pair ? 2 : 1) * kHaloTileH - 1) / ((pair ? 2 : 1) * kHaloTileH);
+  a.tiles_w = (P.Wo + kHaloTileW - 1) / kHaloTileW;
+  const long long tt = static_cast<long long>(P.G) * P.N * P.Do * a.tiles_h * a.tiles_w * a.n_tiles;
+  if (tt > 0x7fffffffLL) return CONV_EINVAL;
+  a.total_tiles = static_cast<int>(tt);
+  a.m_tiles = 0;
+  a.halo_w = kHaloTileW + P.d[2] * (P.kW - 1);
+  a.halo_h = kHaloTileH + P.d[1] * (P.kH - 1);
+  a.halo_bytes = static_cast<uint32_t>(a.halo_w * a.halo_h * 128);
+  a.halo_slot_bytes = (a.halo_bytes + 1023u) & ~1023u;
+  a.a_slots = 2;
+  a.kc = 64;
+  a.cchunks = P.Cg / 64;
+  a.kblocks = P.kD * P.kH * P.kW * a.cchunks;
+  a.rank5 = rank5 ? 1 : 0;
+  a.layout_type = 2u;
+  a.sbo = 1024u;
+  a.a_bytes = 0;
+  a.b_bytes = static_cast<uint32_t>((pair ? a.BN / 2 : a.BN) * 128);
+  a.stage_bytes = a.b_bytes;
+  const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64 -
+                          static_cast<long long>(a.a_slots) * a.halo_slot_bytes;
+  int stages = static_cast<int>(std::min<long long>(8, avail / a.b_bytes));
+  if (stages < 2) return CONV_EUNSUPPORTED;
+  a.stages = stages;
+  const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
+  const uint32_t mma_m = pair ? 2 * kBM : kBM;
+  a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(a.BN >> 3) << 17) | ((mma_m >> 4) << 24);
+  a.tmem_cols = next_pow2_cols(static_cast<uint32_t>(2 * a.BN));
+  a.timeout_ns = kWaitTimeoutNs;
+  plan.variant = pair ? CONV_VARIANT_TC_HALO_PAIR : CONV_VARIANT_TC_HALO;
+  plan.pair = pair;
+  plan.ctas = pair ? 2 * std::min(a.total_tiles, sms / 2) : std::min(a.total_tiles, sms);
+  plan.smem = static_cast<size_t>(a.a_slots) * a.halo_slot_bytes + static_cast<size_t>(a.stages) * a.b_bytes +
+              1024 + sizeof(TcSmemTail) + 64;
+  return CONV_OK;
+}
+
 int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
+  if (variant == CONV_VARIANT_TC_HALO || variant == CONV_VARIANT_TC_HALO_PAIR)
+    return plan_halo(P, variant == CONV_VARIANT_TC_HALO_PAIR, sms, plan);
   if (P.dtype == CONV_F32) return CONV_EUNSUPPORTED;
   TcArgs& a = plan.args;
   std::memset(&a, 0, sizeof(a));
@@ -247,13 +333,16 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
   a.K = static_cast<int>(P.K);
   a.BN = std::min(256, round_up(P.Og, 32));
   a.n_tiles = (P.Og + a.BN - 1) / a.BN;
-  const long long mt = (P.M + kBM - 1) / kBM;
+  // CTA pairs (256-row tiles) for the TMA path once there are enough tiles to
+  // keep every SM pair busy; single CTAs (128-row tiles) otherwise.
+  plan.pair = variant == CONV_VARIANT_TC_TMA_PAIR;
+  const long long mt = plan.pair ? (P.M + 2 * kBM - 1) / (2 * kBM) : (P.M + kBM - 1) / kBM;
   const long long tt = mt * a.n_tiles * P.G;
   if (tt > 0x7fffffffLL) return CONV_EINVAL;
   a.m_tiles = static_cast<int>(mt);
   a.total_tiles = static_cast<int>(tt);
   bool rank5 = false;
-  if (variant == CONV_VARIANT_TC_TMA) {
+  if (variant == CONV_VARIANT_TC_TMA || variant == CONV_VARIANT_TC_TMA_PAIR) {
     if (!tma_fits(P, rank5)) return CONV_EUNSUPPORTED;
     a.kc = (P.Cg % 64 == 0) ? 64 : (P.Cg % 32 == 0 ? 32 : 16);
     a.cchunks = P.Cg / a.kc;
@@ -262,40 +351,76 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
   } else {
     a.kc = 64;
     a.cchunks = 0;
-    a.kblocks = static_cast<int>((P.K + 63) / 64);
     a.rank5 = 0;
+    // gather layout of K: natural weight order (kd, kh, kw, c), except in span
+    // layout where each filter row (kd, kh) is padded to Lp = roundup(kW*C, 8)
+    if (P.Cg % 8 == 0) {
+      a.gather_mode = GATHER_VEC8;
+    } else if (P.G == 1 && P.d[2] == 1) {
+      a.gather_mode = GATHER_SPAN;
+    } else {
+      a.gather_mode = GATHER_SCALAR;
+    }
+    a.Lp = round_up(P.kW * P.C, 8);
+    const long long kp = a.gather_mode == GATHER_SPAN ? static_cast<long long>(P.kD) * P.kH * a.Lp : P.K;
+    if (kp > 0x7fffffffLL - 64) return CONV_EINVAL;
+    a.Kp = static_cast<int>(kp);
+    a.kblocks = static_cast<int>((kp + 63) / 64);
   }
+  a.x_elems = static_cast<long long>(P.x_bytes / P.esize);
   a.layout_type = a.kc == 64 ? 2u : (a.kc == 32 ? 4u : 6u);
   a.sbo = static_cast<uint32_t>(8 * a.kc * 2);
   a.a_bytes = static_cast<uint32_t>(kBM * a.kc * 2);
-  a.b_bytes = static_cast<uint32_t>(a.BN * a.kc * 2);
-  a.stage_bytes = a.a_bytes + a.b_bytes;
-  const uint32_t avail = kSmemBudget - 1024 - static_cast<uint32_t>(sizeof(TcSmemTail)) - 64;
+  a.b_bytes = static_cast<uint32_t>((plan.pair ? a.BN / 2 : a.BN) * a.kc * 2);  // per CTA
+  a.b_resident = 0;
+  a.bres_bytes = 0;
+  if (variant == CONV_VARIANT_TC_GATHER) {
+    const long long bres = static_cast<long long>(a.kblocks) * a.BN * 128;
+    if (P.G == 1 && a.n_tiles == 1 && bres <= kMaxResidentB) {
+      a.b_resident = 1;
+      a.bres_bytes = static_cast<uint32_t>(bres);
+    }
+  }
+  a.stage_bytes = a.a_bytes + (a.b_resident ? 0u : a.b_bytes);
+  const uint32_t avail =
+      kSmemBudget - 1024 - static_cast<uint32_t>(sizeof(TcSmemTail)) - 64 - a.bres_bytes;
   int stages = static_cast<int>(avail / a.stage_bytes);
   stages = std::min(stages, 8);
   if (stages < 2) return CONV_EUNSUPPORTED;
   a.stages = stages;
   const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
+  const uint32_t mma_m = plan.pair ? 2 * kBM : kBM;
   a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(a.BN >> 3) << 17) |
-            (static_cast<uint32_t>(kBM >> 4) << 24);
+            ((mma_m >> 4) << 24);
   a.tmem_cols = next_pow2_cols(static_cast<uint32_t>(2 * a.BN));
   a.timeout_ns = kWaitTimeoutNs;
   plan.variant = variant;
-  plan.ctas = std::min(a.total_tiles, sms);
-  plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + 1024 + sizeof(TcSmemTail) + 64;
+  plan.ctas = plan.pair ? 2 * std::min(a.total_tiles, sms / 2) : std::min(a.total_tiles, sms);
+  plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + a.bres_bytes + 1024 + sizeof(TcSmemTail) + 64;
   return CONV_OK;
 }
 
-int choose_variant(const Problem& P) {
+// f32 -> SIMT.  f16/bf16 -> TMA im2col when it can describe the problem
+// (CTA pairs once there are at least as many 256-row tiles as SM pairs),
+// else the in-kernel gather.
+int choose_variant(const Problem& P, int sms) {
   if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
   bool r5;
-  return tma_fits(P, r5) ? CONV_VARIANT_TC_TMA : CONV_VARIANT_TC_GATHER;
+  const long long og_tiles = (P.Og + 255) / 256;
+  if (halo_fits(P, r5)) {
+    const long long pair_tiles = static_cast<long long>(P.N) * P.Do * ((P.Ho + 31) / 32) * ((P.Wo + 7) / 8) *
+                                 og_tiles * P.G;
+    return pair_tiles >= sms / 2 ? CONV_VARIANT_TC_HALO_PAIR : CONV_VARIANT_TC_HALO;
+  }
+  if (!tma_fits(P, r5)) return CONV_VARIANT_TC_GATHER;
+  const long long pair_tiles = (P.M + 2 * kBM - 1) / (2 * kBM) * og_tiles * P.G;
+  return pair_tiles >= sms / 2 ? CONV_VARIANT_TC_TMA_PAIR : CONV_VARIANT_TC_TMA;
 }
 
 // ---------------------------------------------------------------- launches
 
-int encode_maps(const Problem& P, const TcArgs& a, const void* x, const void* w, CUtensorMap& mx,
-                CUtensorMap& mw) {
+int encode_maps(const Problem& P, const TcArgs& a, bool pair, bool halo, const void* x, const void* w,
+                CUtensorMap& mx, CUtensorMap& mw) {
   std::memset(&mx, 0, sizeof(mx));
   std::memset(&mw, 0, sizeof(mw));
   if (a.cchunks == 0) return CONV_OK;  // gather mode: maps unused
@@ -327,16 +452,24 @@ int encode_maps(const Problem& P, const TcArgs& a, const void* x, const void* w,
     gdim[3] = P.N;
     estr[3] = 1;
   }
-  CUresult r = drv.im2col(&mx, dt, rank, const_cast<void*>(x), gdim, gstr, lower, upper,
-                          static_cast<cuuint32_t>(a.kc), static_cast<cuuint32_t>(kBM), estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r;
+  if (halo) {
+    // a tiled box of 64 channels x halo_w x halo_h pixels (x 1 depth) x 1 image
+    cuuint32_t hbox[5] = {64u, static_cast<cuuint32_t>(a.halo_w), static_cast<cuuint32_t>(a.halo_h), 1u, 1u};
+    cuuint32_t hest[5] = {1u, 1u, 1u, 1u, 1u};
+    r = drv.tiled(&mx, dt, rank, const_cast<void*>(x), gdim, gstr, hbox, hest, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    r = drv.im2col(&mx, dt, rank, const_cast<void*>(x), gdim, gstr, lower, upper, static_cast<cuuint32_t>(a.kc),
+                   static_cast<cuuint32_t>(kBM), estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
   if (r != CUDA_SUCCESS) return CONV_EDRIVER;
   small_tensor_fixup(mx, P.x_bytes, drv.driver_version);
   // w viewed as [O, K] (K innermost)
   cuuint64_t wdim[2] = {static_cast<cuuint64_t>(P.K), static_cast<cuuint64_t>(P.O)};
   cuuint64_t wstr[1] = {static_cast<cuuint64_t>(P.K) * eb};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(a.kc), static_cast<cuuint32_t>(a.BN)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(a.kc), static_cast<cuuint32_t>(pair ? a.BN / 2 : a.BN)};
   cuuint32_t west[2] = {1, 1};
   r = drv.tiled(&mw, dt, 2, const_cast<void*>(w), wdim, wstr, box, west, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -345,18 +478,72 @@ int encode_maps(const Problem& P, const TcArgs& a, const void* x, const void* w,
   return CONV_OK;
 }
 
+// Test hook (conv_debug_inject_stall): when non-zero, the next tensor-core
+// launch makes its MMA thread wait on a barrier that nothing arrives at, with
+// this limit in nanoseconds, so the kernel's timeout path runs.  One-shot.
+std::atomic<unsigned long long> g_inject_stall_ns{0};
+
 int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w, void* y, cudaStream_t st,
               int dev) {
   int rc = set_kernel_attrs(dev);
   if (rc != CONV_OK) return rc;
   TcArgs a = plan.args;
   a.x = x; a.w = w; a.y = y;
+  const unsigned long long stall_ns = g_inject_stall_ns.exchange(0);
+  if (stall_ns != 0) {
+    a.inject_stall = 1;
+    a.timeout_ns = stall_ns;
+  }
   CUtensorMap mx, mw;
-  rc = encode_maps(P, a, x, w, mx, mw);
+  const bool halo = plan.variant == CONV_VARIANT_TC_HALO || plan.variant == CONV_VARIANT_TC_HALO_PAIR;
+  rc = encode_maps(P, a, plan.pair, halo, x, w, mx, mw);
   if (rc != CONV_OK) return rc;
   const dim3 grid(plan.ctas), block(plan.variant == CONV_VARIANT_TC_TMA ? tc_threads<MODE_TMA>()
                                                                          : tc_threads<MODE_GATHER>());
   const bool bf = P.dtype == CONV_BF16;
+  if (halo && !plan.pair) {
+    if (bf) conv_fwd_tc_halo_kernel<true, false><<<grid, 192, plan.smem, st>>>(mx, mw, a);
+    else    conv_fwd_tc_halo_kernel<false, false><<<grid, 192, plan.smem, st>>>(mx, mw, a);
+    return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+  }
+  if (plan.pair) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(plan.ctas);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // never launch more pairs than can be resident together (a second,
+    // partial wave of pairs would double the tail)
+    int clusters = 0;
+    {
+      std::lock_guard<std::mutex> lk(g_mu);
+      if (g_dev[dev].pair_smem != plan.smem) {
+        int c = 0;
+        const cudaError_t oe = halo ? cudaOccupancyMaxActiveClusters(&c, conv_fwd_tc_halo_kernel<false, true>, &cfg)
+                                    : cudaOccupancyMaxActiveClusters(&c, conv_fwd_tc_pair_kernel<false>, &cfg);
+        if (oe != cudaSuccess || c <= 0) return CONV_ELAUNCH;
+        g_dev[dev].pair_smem = plan.smem;
+        g_dev[dev].pair_clusters = c;
+      }
+      clusters = g_dev[dev].pair_clusters;
+    }
+    cfg.gridDim = dim3(2 * std::min(plan.ctas / 2, clusters));
+    cudaError_t e;
+    if (halo)
+      e = bf ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_halo_kernel<true, true>, mx, mw, a)
+             : cudaLaunchKernelEx(&cfg, conv_fwd_tc_halo_kernel<false, true>, mx, mw, a);
+    else
+      e = bf ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_pair_kernel<true>, mx, mw, a)
+             : cudaLaunchKernelEx(&cfg, conv_fwd_tc_pair_kernel<false>, mx, mw, a);
+    return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+  }
   if (plan.variant == CONV_VARIANT_TC_TMA) {
     if (bf) conv_fwd_tc_kernel<MODE_TMA, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
     else    conv_fwd_tc_kernel<MODE_TMA, false><<<grid, block, plan.smem, st>>>(mx, mw, a);
@@ -392,12 +579,11 @@ int run(const Problem& P, const void* x, const void* w, void* y, int variant, cu
   int dev;
   int rc = current_device(dev);
   if (rc != CONV_OK) return rc;
-  if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P);
-  if (variant == CONV_VARIANT_SIMT) return launch_simt(P, x, w, y, st);
-  if (variant != CONV_VARIANT_TC_TMA && variant != CONV_VARIANT_TC_GATHER) return CONV_EINVAL;
   int sms;
   rc = device_sms(dev, sms);
   if (rc != CONV_OK) return rc;
+  if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
+  if (variant == CONV_VARIANT_SIMT) return launch_simt(P, x, w, y, st);
   TcPlan plan;
   rc = plan_tc(P, variant, sms, plan);
   if (rc != CONV_OK) return rc;
@@ -424,7 +610,7 @@ int conv_fwd_variant(const void* x, const void* w, void* y, int N, int D, int H,
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_GATHER) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_PAIR) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -460,7 +646,9 @@ int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, 
   Problem P;
   int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
   if (rc != CONV_OK) return rc;
-  const int variant = choose_variant(P);
+  int dev, sms = 148;
+  if (current_device(dev) == CONV_OK) device_sms(dev, sms);
+  const int variant = choose_variant(P, sms);
   if (variant == CONV_VARIANT_SIMT) {
     if (bn) *bn = kSimtBN;
     if (stages) *stages = 1;
@@ -471,8 +659,6 @@ int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, 
     }
     return variant;
   }
-  int dev, sms = 148;
-  if (current_device(dev) == CONV_OK) device_sms(dev, sms);
   TcPlan plan;
   rc = plan_tc(P, variant, sms, plan);
   if (rc != CONV_OK) return rc;
@@ -510,5 +696,11 @@ const char* conv_strerror(int code) {
 }
 
 int conv_version(void) { return kVersion; }
+
+int conv_debug_inject_stall(unsigned long long timeout_ns) {
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return CONV_EINVAL;
+  g_inject_stall_ns.store(timeout_ns);
+  return CONV_OK;
+}
 
 }  // extern "C"

@@ -1,0 +1,318 @@
+// conv_halo.cuh -- tcgen05 implicit-GEMM convolution forward with input-halo
+// reuse (stride 1, C/G a multiple of 64, f16/bf16).
+//
+// A CTA owns a block of 16 x 8 output pixels (h x w) of one (n, od) output
+// plane: GEMM rows m = r*8 + c for r < 16, c < 8.  For each 64-channel chunk
+// and each depth tap kd, ONE tiled TMA box brings the input halo of that block
+// -- (16 + dh*(kH-1)) x (8 + dw*(kW-1)) pixels x 64 channels -- into shared
+// memory (zero-filled outside the image).  Every (kh, kw) tap is then a view
+// of that box: output row r reads halo row r + kh*dh, output column c reads
+// halo column c + kw*dw.  Because the block is 8 pixels wide, each group of 8
+// GEMM rows is 8 consecutive halo pixels, and successive groups are one halo
+// row apart, so the view is a standard K-major 128B-swizzled UMMA operand with
+// stride (SBO) = halo width x 128 bytes, starting at tap offset
+// (kh*dh*halo_w + kw*dw) x 128 bytes.  Each input pixel of the block is
+// fetched once per (chunk, kd) instead of once per tap.
+//
+// The weights stream through their own ring: one [BN x 64] tile per
+// (chunk, tap).  Roles and the accumulator double-buffer are those of the
+// other tensor-core kernels.  With PAIR, two CTAs of a cluster stack their
+// blocks (32 x 8 output pixels), issue tcgen05.mma.cta_group::2 (M = 256) from
+// the leader, and each loads half of every weight tile.
+#pragma once
+
+#include "conv_tc.cuh"
+
+namespace convfwd {
+
+struct HaloTile {
+  int g, n, od, h0, w0, nt;
+};
+
+__device__ __forceinline__ HaloTile decode_halo_tile(const TcArgs& a, int tile, int rank, bool pair) {
+  HaloTile t;
+  t.nt = tile % a.n_tiles;
+  int q = tile / a.n_tiles;
+  const int tw = q % a.tiles_w;
+  q /= a.tiles_w;
+  const int th = q % a.tiles_h;
+  q /= a.tiles_h;
+  const int plane = q % (a.N * a.Do);
+  t.g = q / (a.N * a.Do);
+  t.od = plane % a.Do;
+  t.n = plane / a.Do;
+  t.h0 = th * (pair ? 2 * a.tile_h : a.tile_h) + rank * a.tile_h;
+  t.w0 = tw * a.tile_w;
+  return t;
+}
+
+template <bool BF16, bool PAIR>
+__global__ void __launch_bounds__(192, 1)
+    conv_fwd_tc_halo_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                            const __grid_constant__ CUtensorMap tmap_w, const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* halo = smem;                                        // a_slots x halo_slot_bytes
+  uint8_t* bring = smem + a.a_slots * a.halo_slot_bytes;       // stages x b_bytes
+  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(bring + a.stages * a.b_bytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const uint16_t both = 3;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&tail->full[s]), 1u);
+      ptx::mbar_init(ptx::smem_u32(&tail->empty[s]), 1u);
+    }
+    for (int s = 0; s < a.a_slots; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&tail->afull[s]), 1u);
+      ptx::mbar_init(ptx::smem_u32(&tail->aempty[s]), 1u);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(ptx::smem_u32(&tail->acc_full[b]), 1u);
+      ptx::mbar_init(ptx::smem_u32(&tail->acc_empty[b]), PAIR ? 8u : 4u);
+    }
+    ptx::mbar_init(ptx::smem_u32(&tail->drain), 1u);
+    ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
+    tail->abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (threadIdx.x == 32) {
+    ptx::prefetch_tmap(&tmap_x);
+    ptx::prefetch_tmap(&tmap_w);
+  }
+  if (warp == 1) {
+    if constexpr (PAIR) {
+      ptx::tmem_alloc_pair(ptx::smem_u32(&tail->tmem_base), a.tmem_cols);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(ptx::smem_u32(&tail->tmem_base), a.tmem_cols);
+      ptx::tmem_relinquish();
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if constexpr (PAIR) ptx::cluster_sync();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = tail->tmem_base;
+  volatile int* abort_flag = &tail->abort_flag;
+  const int unit = PAIR ? (blockIdx.x >> 1) : blockIdx.x;
+  const int nunits = PAIR ? (gridDim.x >> 1) : gridDim.x;
+  const int taps_hw = a.kH * a.kW;
+  const uint32_t mult = PAIR ? 2u : 1u;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int bst = 0, ast = 0;
+      uint32_t bph = 0, aph = 0;
+      long long bfills = 0, afills = 0;
+      bool ok = true;
+      for (int tile = unit; ok && tile < a.total_tiles; tile += nunits) {
+        const HaloTile ht = decode_halo_tile(a, tile, static_cast<int>(rank), PAIR);
+        const int brow = ht.g * a.Og + ht.nt * a.BN + (PAIR ? static_cast<int>(rank) * (a.BN >> 1) : 0);
+        for (int cc = 0; ok && cc < a.cchunks; ++cc) {
+          const int c0 = ht.g * a.Cg + cc * 64;
+          for (int kd = 0; ok && kd < a.kD; ++kd) {
+            // the halo box of this (chunk, kd)
+            if (!wait_bounded(ptx::smem_u32(&tail->aempty[ast]), aph ^ 1u, abort_flag, a.timeout_ns,
+                              kSiteProducerEmpty)) {
+              ok = false;
+              break;
+            }
+            const uint32_t afb = ptx::smem_u32(&tail->afull[ast]);
+            if (leader) ptx::mbar_arrive_expect_tx(afb, mult * a.halo_bytes);
+            const uint32_t afb_l = PAIR ? ptx::mapa_shared(afb, 0) : afb;
+            const uint32_t dst = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
+            const int wc = ht.w0 - a.pw, hc = ht.h0 - a.ph, dc = ht.od - a.pd + kd * a.dd;
+            if (a.rank5) {
+              if constexpr (PAIR) ptx::tma_load_5d_pair(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
+              else ptx::tma_load_5d(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
+            } else {
+              if constexpr (PAIR) ptx::tma_load_4d_pair(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
+              else ptx::tma_load_4d(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
+            }
+            ++afills;
+            if (++ast == a.a_slots) {
+              ast = 0;
+              aph ^= 1u;
+            }
+            // the weight tiles of its taps
+            for (int t = 0; t < taps_hw; ++t) {
+              if (!wait_bounded(ptx::smem_u32(&tail->empty[bst]), bph ^ 1u, abort_flag, a.timeout_ns,
+                                kSiteProducerEmpty)) {
+                ok = false;
+                break;
+              }
+              const uint32_t fb = ptx::smem_u32(&tail->full[bst]);
+              if (leader) ptx::mbar_arrive_expect_tx(fb, mult * a.b_bytes);
+              const uint32_t fb_l = PAIR ? ptx::mapa_shared(fb, 0) : fb;
+              const uint32_t sb = ptx::smem_u32(bring + bst * a.b_bytes);
+              const int tap = kd * taps_hw + t;
+              if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, brow);
+              else ptx::tma_load_2d(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, brow);
+              ++bfills;
+              if (++bst == a.stages) {
+                bst = 0;
+                bph ^= 1u;
+              }
+            }
+          }
+        }
+      }
+      if (!ok && leader) {
+        for (int s = 0; s < a.stages; ++s) {
+          const long long arms = bfills / a.stages + (s < bfills % a.stages ? 1 : 0);
+          if (arms > 0) wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
+        }
+        for (int s = 0; s < a.a_slots; ++s) {
+          const long long arms = afills / a.a_slots + (s < afills % a.a_slots ? 1 : 0);
+          if (arms > 0) wait_drain(ptx::smem_u32(&tail->afull[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (leader && lane == 0) {
+      int bst = 0, ast = 0;
+      uint32_t bph = 0, aph = 0;
+      bool ok = true;
+      int t = 0;
+      if (a.inject_stall)
+        ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
+      const uint32_t sbo = static_cast<uint32_t>(a.halo_w) * 128u;
+      for (int tile = unit; ok && tile < a.total_tiles; tile += nunits, ++t) {
+        const int acc = t & 1;
+        const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
+        if (!wait_bounded(ptx::smem_u32(&tail->acc_empty[acc]), acc_phase ^ 1u, abort_flag, a.timeout_ns,
+                          kSiteMmaAccEmpty)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
+        uint32_t accumulate = 0;
+        for (int cc = 0; ok && cc < a.cchunks; ++cc) {
+          for (int kd = 0; ok && kd < a.kD; ++kd) {
+            if (!wait_bounded(ptx::smem_u32(&tail->afull[ast]), aph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t hbase = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
+            for (int tp = 0; tp < taps_hw; ++tp) {
+              if (!wait_bounded(ptx::smem_u32(&tail->full[bst]), bph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
+                ok = false;
+                break;
+              }
+              ptx::tc_fence_after();
+              const int kh = tp / a.kW, kw = tp - (tp / a.kW) * a.kW;
+              const uint32_t view = hbase + static_cast<uint32_t>(kh * a.dh * a.halo_w + kw * a.dw) * 128u;
+              const uint32_t sb = ptx::smem_u32(bring + bst * a.b_bytes);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t da = ptx::smem_desc_sw128_view(view + k * 32, sbo, 0);
+                const uint64_t db = ptx::smem_desc(sb + k * 32, 16, 1024, 2);
+                if constexpr (PAIR) ptx::mma_f16_pair(d_tmem, da, db, a.idesc, accumulate);
+                else ptx::mma_f16(d_tmem, da, db, a.idesc, accumulate);
+                accumulate = 1;
+              }
+              if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[bst]), both);
+              else ptx::mma_commit(ptx::smem_u32(&tail->empty[bst]));
+              if (++bst == a.stages) {
+                bst = 0;
+                bph ^= 1u;
+              }
+            }
+            if (!ok) break;
+            if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->aempty[ast]), both);
+            else ptx::mma_commit(ptx::smem_u32(&tail->aempty[ast]));
+            if (++ast == a.a_slots) {
+              ast = 0;
+              aph ^= 1u;
+            }
+          }
+        }
+        if (ok) {
+          if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->acc_full[acc]), both);
+          else ptx::mma_commit(ptx::smem_u32(&tail->acc_full[acc]));
+        }
+      }
+      if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->drain), 1);
+      else ptx::mma_commit(ptx::smem_u32(&tail->drain));
+      wait_drain(ptx::smem_u32(&tail->drain), 0, a.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int r = row >> 3, c = row & 7;
+    uint16_t* __restrict__ y = static_cast<uint16_t*>(a.y);
+    int t = 0;
+    for (int tile = unit; tile < a.total_tiles; tile += nunits, ++t) {
+      const int acc = t & 1;
+      const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
+      if (!wait_bounded_warp(ptx::smem_u32(&tail->acc_full[acc]), acc_phase, abort_flag, a.timeout_ns,
+                             kSiteEpiAccFull))
+        break;
+      ptx::tc_fence_after();
+      const HaloTile ht = decode_halo_tile(a, tile, static_cast<int>(rank), PAIR);
+      const int h = ht.h0 + r, w = ht.w0 + c;
+      const bool valid = h < a.Ho && w < a.Wo;
+      const long long m = ((static_cast<long long>(ht.n) * a.Do + ht.od) * a.Ho + h) * a.Wo + w;
+      const int n0 = ht.nt * a.BN;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
+      const long long ybase = m * a.O + static_cast<long long>(ht.g) * a.Og;
+      for (int cb = 0; cb < a.BN; cb += 32) {
+        uint32_t v[32];
+        ptx::tmem_ld_32x32b_x32(taddr + cb, v);
+        ptx::tmem_ld_wait();
+        const int col0 = n0 + cb;
+        const int nvalid = min(32, a.Og - col0);
+        if (valid && nvalid > 0) {
+          uint16_t* dst = y + ybase + col0;
+          if (nvalid == 32 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 o;
+              o.x = pack2<BF16>(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+              o.y = pack2<BF16>(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+              o.z = pack2<BF16>(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+              o.w = pack2<BF16>(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+              d4[j] = o;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) dst[j] = cvt1<BF16>(__uint_as_float(v[j]));
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t ae = ptx::smem_u32(&tail->acc_empty[acc]);
+        if constexpr (PAIR) ptx::mbar_arrive_cluster(ptx::mapa_shared(ae, 0));
+        else ptx::mbar_arrive(ae);
+      }
+    }
+    __syncwarp();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if constexpr (PAIR) ptx::cluster_sync();
+  ptx::tc_fence_after();
+  if (warp == 1) {
+    if constexpr (PAIR) ptx::tmem_dealloc_pair(tmem_base, a.tmem_cols);
+    else ptx::tmem_dealloc(tmem_base, a.tmem_cols);
+  }
+}
+
+}  // namespace convfwd

@@ -52,6 +52,7 @@ enum WaitSite : unsigned {
   kSiteMmaAccEmpty = 3,
   kSiteEpiAccFull = 4,
   kSiteDrain = 5,
+  kSiteInjected = 6,
 };
 
 struct TcArgs {
@@ -74,10 +75,23 @@ struct TcArgs {
   uint32_t idesc;        // tcgen05 instruction descriptor
   uint32_t tmem_cols;
   int rank5;
+  int tile_h, tile_w; // halo kernel: output block per CTA (16 x 8)
+  int tiles_h, tiles_w;  // halo kernel: blocks per output plane (pair blocks are 2*tile_h high)
+  int halo_h, halo_w;    // halo kernel: input block per (channel chunk, kd)
+  uint32_t halo_slot_bytes;  // its shared-memory slot (1024-aligned)
+  uint32_t halo_bytes;       // bytes one halo load delivers
+  int a_slots;               // halo slots in the ring
+  int gather_mode;    // GATHER_SCALAR / GATHER_VEC8 / GATHER_SPAN
+  int Lp;             // span layout: filter-row length kW*C rounded up to 8
+  int Kp;             // K as laid out in shared memory (>= K in span layout)
+  long long x_elems;  // elements of x (bounds of the unaligned 16-byte loads)
+  int b_resident;     // gather: the whole B matrix stays in shared memory
+  uint32_t bres_bytes;  // its size (kblocks * BN * 128), 0 when not resident
   const void* x;
   const void* w;
   void* y;
   unsigned long long timeout_ns;
+  int inject_stall;   // test hook: the MMA thread first waits on a barrier nothing arrives at
 };
 
 struct __align__(8) TcSmemTail {
@@ -86,6 +100,10 @@ struct __align__(8) TcSmemTail {
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;
+  uint64_t stall;     // never arrived on (the injected-timeout test waits here)
+  uint64_t bres;      // resident weights loaded
+  uint64_t afull[4];  // halo kernel: input halo slots
+  uint64_t aempty[4];
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -209,7 +227,7 @@ struct TcRoles<MODE_TMA> {
 };
 template <>
 struct TcRoles<MODE_GATHER> {
-  static constexpr int kProducerWarps = 4;
+  static constexpr int kProducerWarps = 8;
 };
 
 template <int MODE>
@@ -218,93 +236,232 @@ constexpr int tc_threads() {
 }
 
 // ----------------------------------------------------------------------------
-// Gather producer: 128 threads fill one stage (A rows = threads, B rows =
-// threads and threads + 128) from plain global loads with zero fill.
-// Element k of a row decodes to (kd, kh, kw, c) in weight order; the decode
-// is carried incrementally from element to element.
+// Gather producer: 256 threads fill one stage from plain global loads with
+// zero fill.  Thread t owns A row t % 128 and half t / 128 of the 64 K
+// elements of each stage; element k of a row is (kd, kh, kw, c) in weight
+// order.  B is either resident (loaded once per CTA) or gathered per stage.
 // ----------------------------------------------------------------------------
 struct GatherRow {
   bool valid;
-  long long xbase;  // element offset of x[n, 0, 0, 0, g*Cg]
+  long long nbase;  // element offset of x[n, 0, 0, 0, g*Cg]
   int id0, ih0, iw0;
-  // carried decode of the next k
-  int kd, kh, kw, c;
+  int jlo, jhi;     // span mode: valid offsets within a filter row
 };
 
-__device__ __forceinline__ void gather_fill_a(const TcArgs& a, GatherRow& st, int kbase,
-                                              uint8_t* a_tile, int r) {
-  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
-#pragma unroll 1
-  for (int ch = 0; ch < 8; ++ch) {
-    uint32_t v[4];
-#pragma unroll
-    for (int e2 = 0; e2 < 4; ++e2) {
-      uint32_t lohi[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int k = kbase + ch * 8 + e2 * 2 + h;
-        uint16_t val = 0;
-        if (st.valid && k < a.K) {
-          const int id = st.id0 + st.kd * a.dd;
-          const int ih = st.ih0 + st.kh * a.dh;
-          const int iw = st.iw0 + st.kw * a.dw;
-          if (static_cast<unsigned>(id) < static_cast<unsigned>(a.D) &&
-              static_cast<unsigned>(ih) < static_cast<unsigned>(a.H) &&
-              static_cast<unsigned>(iw) < static_cast<unsigned>(a.W)) {
-            const long long off =
-                st.xbase + ((static_cast<long long>(id) * a.H + ih) * a.W + iw) * a.C + st.c;
-            val = __ldg(x + off);
-          }
-        }
-        lohi[h] = val;
-        // advance the carried decode to k + 1
-        if (++st.c == a.Cg) {
-          st.c = 0;
-          if (++st.kw == a.kW) {
-            st.kw = 0;
-            if (++st.kh == a.kH) {
-              st.kh = 0;
-              ++st.kd;
-            }
-          }
-        }
-      }
-      v[e2] = lohi[0] | (lohi[1] << 16);
-    }
-    *reinterpret_cast<uint4*>(a_tile + sw128_offset(r, ch)) = make_uint4(v[0], v[1], v[2], v[3]);
-  }
+// One filter row (kd, kh) of one output pixel: offset of x[n, id, ih, 0, g*Cg]
+// and whether that input row exists.
+__device__ __forceinline__ bool gather_span(const TcArgs& a, const GatherRow& st, int kd, int kh,
+                                            long long& rowptr) {
+  const int id = st.id0 + kd * a.dd;
+  const int ih = st.ih0 + kh * a.dh;
+  const bool ok = st.valid && kd < a.kD && static_cast<unsigned>(id) < static_cast<unsigned>(a.D) &&
+                  static_cast<unsigned>(ih) < static_cast<unsigned>(a.H);
+  rowptr = st.nbase + (static_cast<long long>(id) * a.H + ih) * static_cast<long long>(a.W) * a.C;
+  return ok;
 }
 
-__device__ __forceinline__ void gather_fill_b(const TcArgs& a, int g, int n0, int kbase,
-                                              uint8_t* b_tile, int tid) {
-  const uint16_t* __restrict__ w = static_cast<const uint16_t*>(a.w);
-  const bool vec = (a.K & 7) == 0;
-#pragma unroll 1
-  for (int o = tid; o < a.BN; o += 128) {
-    const int oc = n0 + o;
-    const bool ovalid = oc < a.Og;
-    const long long rowoff = static_cast<long long>(g * a.Og + oc) * a.K;
-#pragma unroll 1
-    for (int ch = 0; ch < 8; ++ch) {
-      const int k0 = kbase + ch * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (ovalid && k0 < a.K) {
-        if (vec) {
-          v = __ldg(reinterpret_cast<const uint4*>(w + rowoff + k0));
-        } else {
-          uint32_t p[4];
+__device__ __forceinline__ void store_chunk(uint8_t* a_tile, int r, int ch, uint4 v) {
+  *reinterpret_cast<uint4*>(a_tile + sw128_offset(r, ch)) = v;
+}
+
+// Scalar gather of the 8 elements p[e] for e in [e_lo, e_hi), zeros elsewhere.
+__device__ __forceinline__ uint4 load8_masked(const uint16_t* p, int e_lo, int e_hi) {
+  uint32_t v[8];
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const int k = k0 + e2 * 2;
-            const uint32_t lo = (k < a.K) ? __ldg(w + rowoff + k) : 0u;
-            const uint32_t hi = (k + 1 < a.K) ? __ldg(w + rowoff + k + 1) : 0u;
-            p[e2] = lo | (hi << 16);
-          }
-          v = make_uint4(p[0], p[1], p[2], p[3]);
+  for (int e = 0; e < 8; ++e) v[e] = (e >= e_lo && e < e_hi) ? __ldg(p + e) : 0u;
+  return make_uint4(v[0] | (v[1] << 16), v[2] | (v[3] << 16), v[4] | (v[5] << 16), v[6] | (v[7] << 16));
+}
+
+// Four 8-element chunks (K elements k0 .. k0+31) of one A row.
+//
+// GATHER_VEC8 (C/G % 8 == 0): a chunk is 8 channels of one input pixel, one
+// aligned 16-byte load, or zeros when the pixel is in the padding.
+// GATHER_SPAN (one group, dilation_w == 1): K is laid out per filter row
+// (kd, kh) as the kW*C contiguous elements of that row, zero-padded to Lp (a
+// multiple of 8), so a chunk never crosses a row; element j of row (kd, kh) is
+// x[n, id, ih, iw0, 0] + j and exists for j in [jlo, jhi).
+// GATHER_SCALAR: element-wise (kw, c) walk with its own bounds check.
+enum { GATHER_SCALAR = 0, GATHER_VEC8 = 1, GATHER_SPAN = 2 };
+
+__device__ __forceinline__ void gather_a_vec8(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
+                                              int r, int chunk0) {
+  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
+  const int tap = k0 / a.Cg;
+  int c = k0 - tap * a.Cg;
+  int kw = tap % a.kW;
+  const int t2 = tap / a.kW;
+  int kh = t2 % a.kH;
+  int kd = t2 / a.kH;
+  long long rowptr;
+  bool rok = gather_span(a, st, kd, kh, rowptr);
+  uint4 v[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int iw = st.iw0 + kw * a.dw;
+    v[q] = make_uint4(0, 0, 0, 0);
+    if (rok && static_cast<unsigned>(iw) < static_cast<unsigned>(a.W))
+      v[q] = __ldg(reinterpret_cast<const uint4*>(x + rowptr + static_cast<long long>(iw) * a.C + c));
+    c += 8;
+    if (c == a.Cg) {
+      c = 0;
+      if (++kw == a.kW) {
+        kw = 0;
+        if (++kh == a.kH) {
+          kh = 0;
+          ++kd;
         }
+        rok = gather_span(a, st, kd, kh, rowptr);
       }
-      *reinterpret_cast<uint4*>(b_tile + sw128_offset(o, ch)) = v;
     }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) store_chunk(a_tile, r, chunk0 + q, v[q]);
+}
+
+// Halfwords h .. h+7 of the 16 halfwords in (b0, b1), h in 0..7.
+__device__ __forceinline__ uint4 extract8(const uint4& b0, const uint4& b1, unsigned h) {
+  const uint32_t w[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+  const unsigned sh = h >> 1;
+  uint32_t u[5];
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    const uint32_t lo = (sh & 1) ? w[(k + 1) & 7] : w[k];
+    const uint32_t hi = (sh & 1) ? w[(k + 3) & 7] : w[(k + 2) & 7];
+    u[k] = (sh & 2) ? hi : lo;  // w[k + sh]
+  }
+  uint32_t r[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r[i] = (h & 1) ? __funnelshift_r(u[i], u[i + 1], 16) : u[i];
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// Zero the halfwords of v whose bit in the 8-bit mask is clear.
+__device__ __forceinline__ uint4 mask8(uint4 v, unsigned m) {
+  const auto keep = [m](int i) -> uint32_t {
+    return ((m >> (2 * i)) & 1 ? 0x0000FFFFu : 0u) | ((m >> (2 * i + 1)) & 1 ? 0xFFFF0000u : 0u);
+  };
+  v.x &= keep(0);
+  v.y &= keep(1);
+  v.z &= keep(2);
+  v.w &= keep(3);
+  return v;
+}
+
+__device__ __forceinline__ void gather_a_span(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
+                                              int r, int chunk0) {
+  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
+  const int span = k0 / a.Lp;
+  int j = k0 - span * a.Lp;
+  int kh = span % a.kH;
+  int kd = span / a.kH;
+  long long rowptr;
+  bool rok = gather_span(a, st, kd, kh, rowptr);
+  rowptr += static_cast<long long>(st.iw0) * a.C;
+  // phase 1: issue every load of the four chunks (aligned 16-byte blocks that
+  // cover the chunk; the halo and the row ends are masked afterwards)
+  uint4 b0[4], b1[4];
+  unsigned hsh[4], msk[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    b0[q] = make_uint4(0, 0, 0, 0);
+    b1[q] = make_uint4(0, 0, 0, 0);
+    hsh[q] = 0;
+    msk[q] = 0;
+    if (rok && j + 8 > st.jlo && j < st.jhi) {
+      const int lo = max(st.jlo - j, 0), hi = min(st.jhi - j, 8);
+      const long long e0 = rowptr + j;
+      const long long a0 = e0 & ~7LL;
+      if (a0 >= 0 && a0 + 16 <= a.x_elems) {
+        hsh[q] = static_cast<unsigned>(e0 - a0);
+        msk[q] = ((1u << hi) - 1u) & ~((1u << lo) - 1u);
+        b0[q] = __ldg(reinterpret_cast<const uint4*>(x + a0));
+        if (hsh[q] != 0) b1[q] = __ldg(reinterpret_cast<const uint4*>(x + a0 + 8));
+      } else {
+        b0[q] = load8_masked(x + e0, lo, hi);  // at the tensor's ends: element loads
+        msk[q] = 0xFFu;
+      }
+    }
+    j += 8;
+    if (j == a.Lp) {
+      j = 0;
+      if (++kh == a.kH) {
+        kh = 0;
+        ++kd;
+      }
+      rok = gather_span(a, st, kd, kh, rowptr);
+      rowptr += static_cast<long long>(st.iw0) * a.C;
+    }
+  }
+  // phase 2: shift into place, mask, store
+#pragma unroll
+  for (int q = 0; q < 4; ++q) store_chunk(a_tile, r, chunk0 + q, mask8(extract8(b0[q], b1[q], hsh[q]), msk[q]));
+}
+
+__device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
+                                                int r, int chunk0) {
+  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
+  uint32_t v[32];
+  const int tap = k0 / a.Cg;
+  int c = k0 - tap * a.Cg;
+  int kw = tap % a.kW;
+  const int t2 = tap / a.kW;
+  int kh = t2 % a.kH;
+  int kd = t2 / a.kH;
+  long long rowptr;
+  bool ok = gather_span(a, st, kd, kh, rowptr);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const int iw = st.iw0 + kw * a.dw;
+    v[e] = (ok && static_cast<unsigned>(iw) < static_cast<unsigned>(a.W))
+               ? __ldg(x + rowptr + static_cast<long long>(iw) * a.C + c)
+               : 0u;
+    if (++c == a.Cg) {
+      c = 0;
+      if (++kw == a.kW) {
+        kw = 0;
+        if (++kh == a.kH) {
+          kh = 0;
+          ++kd;
+        }
+        ok = gather_span(a, st, kd, kh, rowptr);
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    store_chunk(a_tile, r, chunk0 + q,
+                make_uint4(v[8 * q] | (v[8 * q + 1] << 16), v[8 * q + 2] | (v[8 * q + 3] << 16),
+                           v[8 * q + 4] | (v[8 * q + 5] << 16), v[8 * q + 6] | (v[8 * q + 7] << 16)));
+}
+
+// B rows [0, BN) x K elements [kbase, kbase+64) of group g, output channels
+// starting at n0, into a swizzled BN x 128-byte tile.  `nthreads` threads
+// share the 8*BN chunks.  In span layout, padded K element kp of filter row
+// s = kp / Lp, offset j = kp % Lp, is w[o, s*kW*C + j] for j < kW*C, else 0.
+__device__ __forceinline__ void gather_b_block(const TcArgs& a, int g, int n0, int kbase, uint8_t* b_tile,
+                                               int tid, int nthreads) {
+  const uint16_t* __restrict__ w = static_cast<const uint16_t*>(a.w);
+  const bool vec = (a.K & 7) == 0 && a.gather_mode != GATHER_SPAN;
+  const int L = a.kW * a.C;
+#pragma unroll 1
+  for (int q = tid; q < a.BN * 8; q += nthreads) {
+    const int o = q >> 3, ch = q & 7;
+    const int oc = n0 + o;
+    const int kp0 = kbase + ch * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (oc < a.Og && kp0 < a.Kp) {
+      const long long rowoff = static_cast<long long>(g * a.Og + oc) * a.K;
+      if (a.gather_mode == GATHER_SPAN) {
+        const int sp = kp0 / a.Lp;
+        const int j0 = kp0 - sp * a.Lp;
+        v = load8_masked(w + rowoff + static_cast<long long>(sp) * L + j0, 0, L - j0);
+      } else if (vec) {
+        v = __ldg(reinterpret_cast<const uint4*>(w + rowoff + kp0));
+      } else {
+        v = load8_masked(w + rowoff + kp0, 0, a.K - kp0);
+      }
+    }
+    *reinterpret_cast<uint4*>(b_tile + sw128_offset(o, ch)) = v;
   }
 }
 
@@ -321,14 +478,16 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(smem + a.stages * a.stage_bytes);
+  uint8_t* bres = smem + a.stages * a.stage_bytes;  // resident B (gather mode), 1024-aligned
+  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(bres + a.bres_bytes);
+  constexpr uint32_t kProdThreads = kProdWarps * 32;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
-      ptx::mbar_init(ptx::smem_u32(&tail->full[s]), MODE == MODE_TMA ? 1u : 128u);
+      ptx::mbar_init(ptx::smem_u32(&tail->full[s]), MODE == MODE_TMA ? 1u : kProdThreads);
       ptx::mbar_init(ptx::smem_u32(&tail->empty[s]), 1u);
     }
     for (int b = 0; b < 2; ++b) {
@@ -336,6 +495,8 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
       ptx::mbar_init(ptx::smem_u32(&tail->acc_empty[b]), 4u);
     }
     ptx::mbar_init(ptx::smem_u32(&tail->drain), 1u);
+    ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
+    ptx::mbar_init(ptx::smem_u32(&tail->bres), kProdThreads);
     tail->abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -416,22 +577,34 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
       }
       __syncwarp();
     } else {
-      const int tid = threadIdx.x;  // 0..127
+      const int tid = threadIdx.x;  // 0 .. kProdThreads-1
+      const int r = tid & 127;      // A row
+      const int half = tid >> 7;    // which 32 of the 64 K elements of a stage
+      if (a.b_resident) {
+        // the whole B matrix, once per CTA: [kblock][BN rows][128 B]
+        for (int kb = 0; kb < a.kblocks; ++kb)
+          gather_b_block(a, 0, 0, kb * 64, bres + static_cast<uint32_t>(kb) * a.BN * 128u, tid,
+                         kProdThreads);
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(ptx::smem_u32(&tail->bres));
+      }
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x) {
         const TileCoord tc = decode_tile(a, tile);
         GatherRow st;
-        const long long m = static_cast<long long>(tc.mt) * kBM + tid;
+        const long long m = static_cast<long long>(tc.mt) * kBM + r;
         st.valid = m < a.M;
         int n = 0, od = 0, oh = 0, ow = 0;
         if (st.valid) decode_pixel(a, m, n, od, oh, ow);
-        st.xbase = static_cast<long long>(n) * a.D * a.H * a.W * a.C + static_cast<long long>(tc.g) * a.Cg;
+        st.nbase = static_cast<long long>(n) * a.D * a.H * a.W * a.C + static_cast<long long>(tc.g) * a.Cg;
         st.id0 = od * a.sd - a.pd;
         st.ih0 = oh * a.sh - a.ph;
         st.iw0 = ow * a.sw - a.pw;
-        st.kd = st.kh = st.kw = st.c = 0;
+        st.jlo = max(0, -st.iw0) * a.C;
+        st.jhi = min(a.kW, a.W - st.iw0) * a.C;
+        if (st.jhi < st.jlo) st.jhi = st.jlo;
         const int n0 = tc.nt * a.BN;
         for (int kb = 0; kb < a.kblocks; ++kb) {
           if (!wait_bounded(ptx::smem_u32(&tail->empty[stage]), phase ^ 1u, abort_flag, a.timeout_ns,
@@ -440,8 +613,14 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
             break;
           }
           uint8_t* sa = smem + stage * a.stage_bytes;
-          gather_fill_a(a, st, kb * 64, sa, tid);
-          gather_fill_b(a, tc.g, n0, kb * 64, sa + a.a_bytes, tid);
+          const int k0 = kb * 64 + half * 32;
+          if (a.gather_mode == GATHER_VEC8)
+            gather_a_vec8(a, st, k0, sa, r, half * 4);
+          else if (a.gather_mode == GATHER_SPAN)
+            gather_a_span(a, st, k0, sa, r, half * 4);
+          else
+            gather_a_scalar(a, st, k0, sa, r, half * 4);
+          if (!a.b_resident) gather_b_block(a, tc.g, n0, kb * 64, sa + a.a_bytes, tid, kProdThreads);
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(ptx::smem_u32(&tail->full[stage]));
           if (++stage == a.stages) {
@@ -459,6 +638,11 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
       uint32_t phase = 0;
       bool ok = true;
       int t = 0;
+      if (a.inject_stall)
+        ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
+      if (ok && a.b_resident)
+        ok = wait_bounded(ptx::smem_u32(&tail->bres), 0u, abort_flag, a.timeout_ns, kSiteMmaFull);
+      const uint32_t bres_addr = ptx::smem_u32(bres);
       for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++t) {
         const int acc = t & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -477,7 +661,8 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
           }
           ptx::tc_fence_after();
           const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes);
-          const uint32_t sb = sa + a.a_bytes;
+          const uint32_t sb =
+              a.b_resident ? bres_addr + static_cast<uint32_t>(kb) * a.BN * 128u : sa + a.a_bytes;
           const int ksteps = a.kc >> 4;
           for (int k = 0; k < ksteps; ++k) {
             const uint64_t da = ptx::smem_desc(sa + k * 32, 16, a.sbo, a.layout_type);
@@ -553,6 +738,224 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == kMmaWarp) ptx::tmem_dealloc(tmem_base, a.tmem_cols);
+}
+
+}  // namespace convfwd
+
+namespace convfwd {
+
+// ----------------------------------------------------------------------------
+// CTA-pair variant of the TMA kernel: a cluster of two CTAs on two SMs owns a
+// 256 x BN output tile and issues tcgen05.mma.cta_group::2 (M = 256).  Each CTA
+// loads its own 128 rows of A and its own BN/2 rows of B, so per K stage a CTA
+// pulls half the weight bytes of a 128 x BN single-CTA tile for the same MMA
+// work.  Both CTAs' TMA loads complete on the leader's (rank 0) `full`
+// barrier; the leader's single MMA thread issues for the pair and its commits
+// arrive on `empty` / `acc_full` in both CTAs; each CTA's epilogue drains its
+// own 128 accumulator rows and arrives on the leader's `acc_empty`.
+// ----------------------------------------------------------------------------
+template <bool BF16>
+__global__ void __launch_bounds__(192, 1)
+    conv_fwd_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                            const __grid_constant__ CUtensorMap tmap_w, const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(smem + a.stages * a.stage_bytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int half_bn = a.BN >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&tail->full[s]), 1u);
+      ptx::mbar_init(ptx::smem_u32(&tail->empty[s]), 1u);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(ptx::smem_u32(&tail->acc_full[b]), 1u);
+      ptx::mbar_init(ptx::smem_u32(&tail->acc_empty[b]), 8u);  // 4 epilogue warps x 2 CTAs
+    }
+    ptx::mbar_init(ptx::smem_u32(&tail->drain), 1u);
+    ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
+    tail->abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (threadIdx.x == 32) {
+    ptx::prefetch_tmap(&tmap_x);
+    ptx::prefetch_tmap(&tmap_w);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(ptx::smem_u32(&tail->tmem_base), a.tmem_cols);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // barriers of both CTAs initialised before any remote use
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = tail->tmem_base;
+  volatile int* abort_flag = &tail->abort_flag;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long fills = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < a.total_tiles; tile += npairs) {
+        const TileCoord tc = decode_tile(a, tile);
+        int n, od, oh, ow;
+        decode_pixel(a, static_cast<long long>(tc.mt) * (2 * kBM) + rank * kBM, n, od, oh, ow);
+        const int cw = ow * a.sw - a.pw, chh = oh * a.sh - a.ph, cd = od * a.sd - a.pd;
+        const int brow = tc.g * a.Og + tc.nt * a.BN + static_cast<int>(rank) * half_bn;
+        int tap = 0, cchunk = 0;
+        for (int kb = 0; kb < a.kblocks; ++kb) {
+          if (!wait_bounded(ptx::smem_u32(&tail->empty[stage]), phase ^ 1u, abort_flag, a.timeout_ns,
+                            kSiteProducerEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb_local = ptx::smem_u32(&tail->full[stage]);
+          if (leader) ptx::mbar_arrive_expect_tx(fb_local, 2u * (a.a_bytes + a.b_bytes));
+          const uint32_t fb = ptx::mapa_shared(fb_local, 0);
+          const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes);
+          const uint32_t sb = sa + a.a_bytes;
+          const int kw = tap % a.kW;
+          const int kh = (tap / a.kW) % a.kH;
+          const int kd = tap / (a.kW * a.kH);
+          const int c0 = tc.g * a.Cg + cchunk * a.kc;
+          if (a.rank5)
+            ptx::tma_load_im2col_5d_pair(sa, &tmap_x, fb, c0, cw, chh, cd, n, static_cast<uint16_t>(kw * a.dw),
+                                         static_cast<uint16_t>(kh * a.dh), static_cast<uint16_t>(kd * a.dd));
+          else
+            ptx::tma_load_im2col_4d_pair(sa, &tmap_x, fb, c0, cw, chh, n, static_cast<uint16_t>(kw * a.dw),
+                                         static_cast<uint16_t>(kh * a.dh));
+          ptx::tma_load_2d_pair(sb, &tmap_w, fb, tap * a.Cg + cchunk * a.kc, brow);
+          ++fills;
+          if (++cchunk == a.cchunks) {
+            cchunk = 0;
+            ++tap;
+          }
+          if (++stage == a.stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && leader) {
+        for (int s = 0; s < a.stages; ++s) {
+          const long long arms = fills / a.stages + (s < fills % a.stages ? 1 : 0);
+          if (arms > 0)
+            wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int t = 0;
+      if (a.inject_stall)
+        ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
+      for (int tile = pair; ok && tile < a.total_tiles; tile += npairs, ++t) {
+        const int acc = t & 1;
+        const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
+        if (!wait_bounded(ptx::smem_u32(&tail->acc_empty[acc]), acc_phase ^ 1u, abort_flag, a.timeout_ns,
+                          kSiteMmaAccEmpty)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
+        for (int kb = 0; kb < a.kblocks; ++kb) {
+          if (!wait_bounded(ptx::smem_u32(&tail->full[stage]), phase, abort_flag, a.timeout_ns, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes);
+          const uint32_t sb = sa + a.a_bytes;
+          const int ksteps = a.kc >> 4;
+          for (int k = 0; k < ksteps; ++k) {
+            const uint64_t da = ptx::smem_desc(sa + k * 32, 16, a.sbo, a.layout_type);
+            const uint64_t db = ptx::smem_desc(sb + k * 32, 16, a.sbo, a.layout_type);
+            ptx::mma_f16_pair(d_tmem, da, db, a.idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[stage]), 3);
+          if (++stage == a.stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) ptx::mma_commit_pair(ptx::smem_u32(&tail->acc_full[acc]), 3);
+      }
+      ptx::mma_commit_pair(ptx::smem_u32(&tail->drain), 1);
+      wait_drain(ptx::smem_u32(&tail->drain), 0, a.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    uint16_t* __restrict__ y = static_cast<uint16_t*>(a.y);
+    int t = 0;
+    for (int tile = pair; tile < a.total_tiles; tile += npairs, ++t) {
+      const int acc = t & 1;
+      const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
+      if (!wait_bounded_warp(ptx::smem_u32(&tail->acc_full[acc]), acc_phase, abort_flag, a.timeout_ns,
+                             kSiteEpiAccFull))
+        break;
+      ptx::tc_fence_after();
+      const TileCoord tc = decode_tile(a, tile);
+      const long long m = static_cast<long long>(tc.mt) * (2 * kBM) + rank * kBM + row;
+      const int n0 = tc.nt * a.BN;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
+      const long long ybase = m * a.O + static_cast<long long>(tc.g) * a.Og;
+      for (int c = 0; c < a.BN; c += 32) {
+        uint32_t r[32];
+        ptx::tmem_ld_32x32b_x32(taddr + c, r);
+        ptx::tmem_ld_wait();
+        const int col0 = n0 + c;
+        const int nvalid = min(32, a.Og - col0);
+        if (m < a.M && nvalid > 0) {
+          uint16_t* dst = y + ybase + col0;
+          if (nvalid == 32 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 v;
+              v.x = pack2<BF16>(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+              v.y = pack2<BF16>(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+              v.z = pack2<BF16>(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+              v.w = pack2<BF16>(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+              d4[j] = v;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) dst[j] = cvt1<BF16>(__uint_as_float(r[j]));
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(&tail->acc_empty[acc]), 0));
+    }
+    __syncwarp();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // the leader's MMAs (which read this CTA's smem) are complete
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc_pair(tmem_base, a.tmem_cols);
 }
 
 }  // namespace convfwd

@@ -73,7 +73,11 @@ enum {
   CONV_VARIANT_AUTO = -1,
   CONV_VARIANT_SIMT = 0,       /* fp32 FFMA implicit GEMM (any shape, any type) */
   CONV_VARIANT_TC_TMA = 1,     /* tcgen05 + TMA im2col loads (C/G % 16 == 0) */
-  CONV_VARIANT_TC_GATHER = 2   /* tcgen05 + in-kernel gather (any C, any geometry) */
+  CONV_VARIANT_TC_GATHER = 2, /* tcgen05 + in-kernel gather (any C, any geometry) */
+  CONV_VARIANT_TC_TMA_PAIR = 3, /* TC_TMA with CTA pairs: 256-row tiles, cta_group::2 */
+  CONV_VARIANT_TC_HALO = 4,     /* tcgen05, one TMA box of input halo per 16x8 output block
+                                   reused by every filter tap (stride 1, C/G % 64 == 0) */
+  CONV_VARIANT_TC_HALO_PAIR = 5 /* TC_HALO with CTA pairs (32x8 blocks, cta_group::2) */
 };
 
 /* Output extents.  stride/pad/dil: 3 ints (d, h, w).  out: 3 ints (Do, Ho, Wo).
@@ -86,8 +90,10 @@ int conv_out_dims(int D, int H, int W, int kD, int kH, int kW,
 /* Forward convolution on device buffers x, w, y (see the layouts above).
  * Queues the kernel on `stream`; returns CONV_OK or an error code (nothing is
  * queued on an error).  The variant is chosen from the type and shape:
- * f32 -> SIMT; f16/bf16 -> TC_TMA when C/G % 16 == 0 and the geometry fits a
- * TMA im2col tensor map, else TC_GATHER. */
+ * f32 -> SIMT; f16/bf16 -> TC_HALO_PAIR / TC_HALO for stride 1 and
+ * C/G % 64 == 0; otherwise TC_TMA_PAIR / TC_TMA when C/G % 16 == 0 and the
+ * geometry fits a TMA im2col tensor map; otherwise TC_GATHER.  The pair
+ * forms are chosen when there are at least as many pair tiles as SM pairs. */
 int conv_fwd(const void* x, const void* w, void* y,
              int N, int D, int H, int W, int C, int O,
              int kD, int kH, int kW,
@@ -96,7 +102,9 @@ int conv_fwd(const void* x, const void* w, void* y,
 
 /* conv_fwd with an explicit kernel variant (CONV_VARIANT_*).  Returns
  * CONV_EUNSUPPORTED when that variant cannot run the shape or type
- * (TC_TMA and TC_GATHER need f16/bf16; TC_TMA needs C/G % 16 == 0). */
+ * (the tensor-core variants need f16/bf16; TC_TMA and TC_TMA_PAIR need
+ * C/G % 16 == 0 and a geometry inside the TMA im2col limits; TC_HALO and
+ * TC_HALO_PAIR need stride 1 and C/G % 64 == 0). */
 int conv_fwd_variant(const void* x, const void* w, void* y,
                      int N, int D, int H, int W, int C, int O,
                      int kD, int kH, int kW,
@@ -135,6 +143,16 @@ const char* conv_strerror(int code);
 
 /* Library version as major*10000 + minor*100 + patch. */
 int conv_version(void);
+
+/* Failure-detection test hook.  The next tensor-core launch on this process
+ * makes its MMA thread wait on a pipeline barrier that nothing arrives at,
+ * with a limit of `timeout_ns` (1 ns .. 10 s) instead of the usual 2 s: the
+ * wait runs out, the kernel raises its abort flag, every role drains what it
+ * has in flight, tensor memory is freed, the kernel returns without writing
+ * further output, and conv_last_status() then reports CONV_ETIMEOUT.  Nothing
+ * faults or hangs; the context stays usable.  One-shot.  Returns CONV_OK or
+ * CONV_EINVAL. */
+int conv_debug_inject_stall(unsigned long long timeout_ns);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,69 @@
+"""Failure detection on the GPU without a fault: an injected pipeline stall.
+
+`conv_debug_inject_stall` makes the next tensor-core launch's MMA thread wait
+on a barrier that nothing arrives at, with a short limit.  The kernel must
+give up, drain, free its tensor memory and return; the host must read
+CONV_ETIMEOUT from the status word; and the context must stay usable: the
+very next launch is checked against the oracle.
+"""
+from __future__ import annotations
+
+import time
+
+import pytest
+import torch
+
+import oracle
+import workloads as WL
+from tests.parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+C = pytest.importorskip("implicit_gemm_convolution_conv2d_b200")
+ETIMEOUT = -6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    yield
+
+
+def _geom(wl):
+    return (wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, *wl.k, wl.stride, wl.pad, wl.dil, wl.groups)
+
+
+@pytest.mark.parametrize("variant", ["TC_GATHER", "TC_TMA", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR"])
+def test_injected_stall_times_out_and_recovers(variant):
+    v = getattr(C, "VARIANT_" + variant)
+    wl = WL.case(2, 1, 20, 20, 64, 64, (1, 3, 3), pad=(0, 1, 1), dtype="f16", seed=21)
+    x, w = WL.make_inputs(wl)
+    xd, wd = x.cuda(), w.cuda()
+    y = torch.zeros((2, 1, 20, 20, 64), dtype=torch.float16, device="cuda")
+    assert C.last_status() == 0
+    C.inject_stall(50_000_000)  # 50 ms
+    t0 = time.perf_counter()
+    rc = C.conv_fwd_raw(xd.data_ptr(), wd.data_ptr(), y.data_ptr(), _geom(wl), 1, v,
+                        torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert C.last_status() == ETIMEOUT
+    assert C.last_status() == 0          # read-and-clear
+    assert elapsed < 10.0, f"the stalled kernel took {elapsed:.1f} s to give up"
+    # the context is still usable: a normal launch gives the right answer
+    rc = C.conv_fwd_raw(xd.data_ptr(), wd.data_ptr(), y.data_ptr(), _geom(wl), 1, v,
+                        torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert C.last_status() == 0
+    y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups)
+    assert_parity(y.cpu(), y_ref, s_ref, "f16", f"after stall/{variant}")
+
+
+def test_inject_rejects_bad_limits():
+    with pytest.raises(C.ConvError):
+        C.inject_stall(0)
+    with pytest.raises(C.ConvError):
+        C.inject_stall(20_000_000_000)

@@ -55,7 +55,9 @@ def variants_for(wl):
         return [C.VARIANT_SIMT]
     vs.append(C.VARIANT_TC_GATHER)
     if (wl.C // wl.groups) % 16 == 0:
-        vs.append(C.VARIANT_TC_TMA)
+        vs += [C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR]
+    if (wl.C // wl.groups) % 64 == 0 and tuple(wl.stride) == (1, 1, 1):
+        vs += [C.VARIANT_TC_HALO, C.VARIANT_TC_HALO_PAIR]
     return vs
 
 
@@ -84,6 +86,15 @@ SMALL = [
     WL.case(2, 4, 5, 6, 3, 32, (3, 3, 3), pad=(1, 1, 1), name="3d_c3"),
     WL.case(1, 7, 6, 9, 16, 16, (2, 3, 2), (2, 2, 1), (1, 0, 2), (2, 1, 3), name="3d_mixed"),
     WL.case(1, 1, 8, 8, 8, 8, (1, 3, 3), (1, 3, 3), (0, 3, 3), (1, 3, 3), name="s3_d3_p3"),
+    WL.case(2, 1, 9, 11, 5, 8, (1, 3, 3), pad=(0, 1, 2), dil=(1, 1, 2), name="c5_dilw2_scalar"),
+    WL.case(2, 1, 8, 8, 6, 4, (1, 3, 3), pad=(0, 1, 1), groups=2, name="groups2_cg3_scalar"),
+    WL.case(3, 1, 7, 9, 24, 40, (1, 3, 3), pad=(0, 1, 1), name="c24_vec8"),
+    WL.case(1, 2, 9, 200, 3, 16, (1, 1, 7), (1, 1, 3), (0, 0, 3), name="wide_row_span"),
+    WL.case(2, 1, 20, 19, 128, 96, (1, 3, 3), pad=(0, 1, 1), name="halo_c128_o96"),
+    WL.case(1, 3, 9, 13, 64, 64, (3, 3, 3), pad=(1, 1, 1), dil=(1, 2, 1), name="halo_3d_dil"),
+    WL.case(2, 1, 17, 9, 128, 128, (1, 3, 3), pad=(0, 2, 2), dil=(1, 2, 2), groups=2, name="halo_groups2_dil2"),
+    WL.case(1, 1, 12, 12, 64, 320, (1, 3, 3), pad=(0, 1, 1), name="halo_o320"),
+    WL.case(3, 1, 33, 17, 64, 32, (1, 5, 5), pad=(0, 2, 2), name="halo_k5_ragged"),
 ]
 
 
@@ -112,7 +123,10 @@ def test_tutorial_example_on_gpu(dtype):
 
 
 def test_auto_variant_choice():
-    assert C.plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_TMA
+    assert C.plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_HALO_PAIR
+    assert C.plan(1, 1, 56, 56, 64, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_HALO
+    assert C.plan(4, 32, 32, 32, 64, 128, (3, 3, 3), (2, 2, 2), (1, 1, 1), (1, 1, 1), 1, "f16")[0] in (
+        C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR)
     assert C.plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
     assert C.plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f32")[0] == C.VARIANT_SIMT
 
