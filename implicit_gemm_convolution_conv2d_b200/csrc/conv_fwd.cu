@@ -216,6 +216,20 @@ struct TcPlan {
 
 int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
+// K sub-blocks per pipeline stage.  Every stage costs a fixed barrier-wait /
+// MMA-issue / commit round trip (measured on B200 at roughly 700-900 SM
+// cycles), which the tensor pipe hides only if one stage carries about as much
+// MMA work; one sub-block of kc K-elements is kc/16 MMAs of BN/2 cycles each
+// (per SM, M = 128 rows).  Take enough sub-blocks for ~1024 cycles, then
+// shrink until at least two stages fit in `avail` bytes.
+int choose_kbs(int BN, int kc, uint32_t sub_bytes, long long avail, int max_kbs, int& stages) {
+  const int cycles_per_sub = (kc / 16) * (BN / 2);
+  int kbs = std::max(1, std::min(max_kbs, (1024 + cycles_per_sub - 1) / cycles_per_sub));
+  while (kbs > 1 && avail / (static_cast<long long>(kbs) * sub_bytes) < 2) --kbs;
+  stages = static_cast<int>(std::min<long long>(8, avail / (static_cast<long long>(kbs) * sub_bytes)));
+  return kbs;
+}
+
 uint32_t next_pow2_cols(uint32_t v) {
   uint32_t c = 32;
   while (c < v) c <<= 1;
@@ -251,6 +265,7 @@ constexpr int kHaloTileH = 16, kHaloTileW = 8;
 bool halo_fits(const Problem& P, bool& rank5) {
   if (P.dtype == CONV_F32 || P.Cg % 64 != 0) return false;
   if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1) return false;
+  if (P.kH * P.kW < 4) return false;  // too few taps share a halo box to pay for it
   rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
   const long long hw = kHaloTileW + static_cast<long long>(P.d[2]) * (P.kW - 1);
   const long long hh = kHaloTileH + static_cast<long long>(P.d[1]) * (P.kH - 1);
@@ -297,12 +312,15 @@ int plan_halo(const Problem& P, bool pair, int sms, TcPlan& plan) {
   a.sbo = 1024u;
   a.a_bytes = 0;
   a.b_bytes = static_cast<uint32_t>((pair ? a.BN / 2 : a.BN) * 128);
-  a.stage_bytes = a.b_bytes;
+  a.sub_bytes = a.b_bytes;
   const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64 -
                           static_cast<long long>(a.a_slots) * a.halo_slot_bytes;
-  int stages = static_cast<int>(std::min<long long>(8, avail / a.b_bytes));
+  int stages = 0;
+  // a stage may span at most two (chunk, kd) halo groups: kbs <= kH*kW
+  a.kbs = choose_kbs(a.BN, 64, a.b_bytes, avail, std::min(8, P.kH * P.kW), stages);
   if (stages < 2) return CONV_EUNSUPPORTED;
   a.stages = stages;
+  a.stage_bytes = static_cast<uint32_t>(a.kbs) * a.b_bytes;
   const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
   const uint32_t mma_m = pair ? 2 * kBM : kBM;
   a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(a.BN >> 3) << 17) | ((mma_m >> 4) << 24);
@@ -311,7 +329,7 @@ int plan_halo(const Problem& P, bool pair, int sms, TcPlan& plan) {
   plan.variant = pair ? CONV_VARIANT_TC_HALO_PAIR : CONV_VARIANT_TC_HALO;
   plan.pair = pair;
   plan.ctas = pair ? 2 * std::min(a.total_tiles, sms / 2) : std::min(a.total_tiles, sms);
-  plan.smem = static_cast<size_t>(a.a_slots) * a.halo_slot_bytes + static_cast<size_t>(a.stages) * a.b_bytes +
+  plan.smem = static_cast<size_t>(a.a_slots) * a.halo_slot_bytes + static_cast<size_t>(a.stages) * a.stage_bytes +
               1024 + sizeof(TcSmemTail) + 64;
   return CONV_OK;
 }
@@ -381,13 +399,14 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
       a.bres_bytes = static_cast<uint32_t>(bres);
     }
   }
-  a.stage_bytes = a.a_bytes + (a.b_resident ? 0u : a.b_bytes);
-  const uint32_t avail =
-      kSmemBudget - 1024 - static_cast<uint32_t>(sizeof(TcSmemTail)) - 64 - a.bres_bytes;
-  int stages = static_cast<int>(avail / a.stage_bytes);
-  stages = std::min(stages, 8);
+  a.sub_bytes = a.a_bytes + (a.b_resident ? 0u : a.b_bytes);
+  const long long avail =
+      static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64 - a.bres_bytes;
+  int stages = 0;
+  a.kbs = choose_kbs(a.BN, a.kc, a.sub_bytes, avail, 8, stages);
   if (stages < 2) return CONV_EUNSUPPORTED;
   a.stages = stages;
+  a.stage_bytes = static_cast<uint32_t>(a.kbs) * a.sub_bytes;
   const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
   const uint32_t mma_m = plan.pair ? 2 * kBM : kBM;
   a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(a.BN >> 3) << 17) |
@@ -402,17 +421,13 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
 
 // f32 -> SIMT.  f16/bf16 -> TMA im2col when it can describe the problem
 // (CTA pairs once there are at least as many 256-row tiles as SM pairs),
-// else the in-kernel gather.
+// else the in-kernel gather.  The halo kernels are explicit-only: on B200
+// they measure slower than im2col at every shape of the workload set.
 int choose_variant(const Problem& P, int sms) {
   if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
   bool r5;
-  const long long og_tiles = (P.Og + 255) / 256;
-  if (halo_fits(P, r5)) {
-    const long long pair_tiles = static_cast<long long>(P.N) * P.Do * ((P.Ho + 31) / 32) * ((P.Wo + 7) / 8) *
-                                 og_tiles * P.G;
-    return pair_tiles >= sms / 2 ? CONV_VARIANT_TC_HALO_PAIR : CONV_VARIANT_TC_HALO;
-  }
   if (!tma_fits(P, r5)) return CONV_VARIANT_TC_GATHER;
+  const long long og_tiles = (P.Og + 255) / 256;
   const long long pair_tiles = (P.M + 2 * kBM - 1) / (2 * kBM) * og_tiles * P.G;
   return pair_tiles >= sms / 2 ? CONV_VARIANT_TC_TMA_PAIR : CONV_VARIANT_TC_TMA;
 }

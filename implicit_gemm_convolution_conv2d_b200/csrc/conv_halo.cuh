@@ -15,7 +15,8 @@
 // fetched once per (chunk, kd) instead of once per tap.
 //
 // The weights stream through their own ring: one [BN x 64] tile per
-// (chunk, tap).  Roles and the accumulator double-buffer are those of the
+// (chunk, tap), kbs of them per pipeline stage so that one stage carries
+// enough tensor work (>= ~1000 cycles) to hide the wait/commit round trip.  Roles and the accumulator double-buffer are those of the
 // other tensor-core kernels.  With PAIR, two CTAs of a cluster stack their
 // blocks (32 x 8 output pixels), issue tcgen05.mma.cta_group::2 (M = 256) from
 // the leader, and each loads half of every weight tile.
@@ -54,8 +55,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* halo = smem;                                        // a_slots x halo_slot_bytes
-  uint8_t* bring = smem + a.a_slots * a.halo_slot_bytes;       // stages x b_bytes
-  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(bring + a.stages * a.b_bytes);
+  uint8_t* bring = smem + a.a_slots * a.halo_slot_bytes;       // stages x (kbs x b_bytes)
+  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(bring + a.stages * a.stage_bytes);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
@@ -104,6 +105,11 @@ __global__ void __launch_bounds__(192, 1)
   const int taps_hw = a.kH * a.kW;
   const uint32_t mult = PAIR ? 2u : 1u;
 
+  // K-blocks of a tile in issue order: q = (cc * kD + kd) * taps_hw + tap.  A
+  // pipeline stage holds up to kbs consecutive K-blocks (weight tiles); each
+  // (cc, kd) group has one halo box, loaded before its first K-block.  With
+  // taps_hw >= kbs a stage spans at most two groups, so two halo slots suffice.
+  const int Q = a.cchunks * a.kD * taps_hw;
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -114,52 +120,56 @@ __global__ void __launch_bounds__(192, 1)
       for (int tile = unit; ok && tile < a.total_tiles; tile += nunits) {
         const HaloTile ht = decode_halo_tile(a, tile, static_cast<int>(rank), PAIR);
         const int brow = ht.g * a.Og + ht.nt * a.BN + (PAIR ? static_cast<int>(rank) * (a.BN >> 1) : 0);
-        for (int cc = 0; ok && cc < a.cchunks; ++cc) {
-          const int c0 = ht.g * a.Cg + cc * 64;
-          for (int kd = 0; ok && kd < a.kD; ++kd) {
-            // the halo box of this (chunk, kd)
-            if (!wait_bounded(ptx::smem_u32(&tail->aempty[ast]), aph ^ 1u, abort_flag, a.timeout_ns,
-                              kSiteProducerEmpty)) {
-              ok = false;
-              break;
-            }
-            const uint32_t afb = ptx::smem_u32(&tail->afull[ast]);
-            if (leader) ptx::mbar_arrive_expect_tx(afb, mult * a.halo_bytes);
-            const uint32_t afb_l = PAIR ? ptx::mapa_shared(afb, 0) : afb;
-            const uint32_t dst = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
-            const int wc = ht.w0 - a.pw, hc = ht.h0 - a.ph, dc = ht.od - a.pd + kd * a.dd;
-            if (a.rank5) {
-              if constexpr (PAIR) ptx::tma_load_5d_pair(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
-              else ptx::tma_load_5d(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
-            } else {
-              if constexpr (PAIR) ptx::tma_load_4d_pair(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
-              else ptx::tma_load_4d(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
-            }
-            ++afills;
-            if (++ast == a.a_slots) {
-              ast = 0;
-              aph ^= 1u;
-            }
-            // the weight tiles of its taps
-            for (int t = 0; t < taps_hw; ++t) {
-              if (!wait_bounded(ptx::smem_u32(&tail->empty[bst]), bph ^ 1u, abort_flag, a.timeout_ns,
+        for (int q0 = 0; ok && q0 < Q; q0 += a.kbs) {
+          const int nsub = min(a.kbs, Q - q0);
+          if (!wait_bounded(ptx::smem_u32(&tail->empty[bst]), bph ^ 1u, abort_flag, a.timeout_ns,
+                            kSiteProducerEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = ptx::smem_u32(&tail->full[bst]);
+          if (leader) ptx::mbar_arrive_expect_tx(fb, mult * static_cast<uint32_t>(nsub) * a.b_bytes);
+          const uint32_t fb_l = PAIR ? ptx::mapa_shared(fb, 0) : fb;
+          for (int j = 0; j < nsub; ++j) {
+            const int q = q0 + j;
+            const int t = q % taps_hw;
+            const int grp = q / taps_hw;
+            const int kd = grp % a.kD, cc = grp / a.kD;
+            if (t == 0) {
+              // the halo box of group (cc, kd)
+              if (!wait_bounded(ptx::smem_u32(&tail->aempty[ast]), aph ^ 1u, abort_flag, a.timeout_ns,
                                 kSiteProducerEmpty)) {
                 ok = false;
                 break;
               }
-              const uint32_t fb = ptx::smem_u32(&tail->full[bst]);
-              if (leader) ptx::mbar_arrive_expect_tx(fb, mult * a.b_bytes);
-              const uint32_t fb_l = PAIR ? ptx::mapa_shared(fb, 0) : fb;
-              const uint32_t sb = ptx::smem_u32(bring + bst * a.b_bytes);
-              const int tap = kd * taps_hw + t;
-              if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, brow);
-              else ptx::tma_load_2d(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, brow);
-              ++bfills;
-              if (++bst == a.stages) {
-                bst = 0;
-                bph ^= 1u;
+              const uint32_t afb = ptx::smem_u32(&tail->afull[ast]);
+              if (leader) ptx::mbar_arrive_expect_tx(afb, mult * a.halo_bytes);
+              const uint32_t afb_l = PAIR ? ptx::mapa_shared(afb, 0) : afb;
+              const uint32_t dst = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
+              const int c0 = ht.g * a.Cg + cc * 64;
+              const int wc = ht.w0 - a.pw, hc = ht.h0 - a.ph, dc = ht.od - a.pd + kd * a.dd;
+              if (a.rank5) {
+                if constexpr (PAIR) ptx::tma_load_5d_pair(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
+                else ptx::tma_load_5d(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
+              } else {
+                if constexpr (PAIR) ptx::tma_load_4d_pair(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
+                else ptx::tma_load_4d(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
+              }
+              ++afills;
+              if (++ast == a.a_slots) {
+                ast = 0;
+                aph ^= 1u;
               }
             }
+            const uint32_t sb = ptx::smem_u32(bring + bst * a.stage_bytes + j * a.b_bytes);
+            const int tap = kd * taps_hw + t;
+            if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, brow);
+            else ptx::tma_load_2d(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, brow);
+          }
+          ++bfills;
+          if (++bst == a.stages) {
+            bst = 0;
+            bph ^= 1u;
           }
         }
       }
@@ -196,45 +206,52 @@ __global__ void __launch_bounds__(192, 1)
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
         uint32_t accumulate = 0;
-        for (int cc = 0; ok && cc < a.cchunks; ++cc) {
-          for (int kd = 0; ok && kd < a.kD; ++kd) {
-            if (!wait_bounded(ptx::smem_u32(&tail->afull[ast]), aph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
-              ok = false;
-              break;
-            }
-            ptx::tc_fence_after();
-            const uint32_t hbase = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
-            for (int tp = 0; tp < taps_hw; ++tp) {
-              if (!wait_bounded(ptx::smem_u32(&tail->full[bst]), bph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
+        uint32_t hbase = 0;
+        for (int q0 = 0; ok && q0 < Q; q0 += a.kbs) {
+          const int nsub = min(a.kbs, Q - q0);
+          if (!wait_bounded(ptx::smem_u32(&tail->full[bst]), bph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          for (int j = 0; j < nsub; ++j) {
+            const int q = q0 + j;
+            const int tp = q % taps_hw;
+            if (tp == 0) {
+              if (!wait_bounded(ptx::smem_u32(&tail->afull[ast]), aph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
                 ok = false;
                 break;
               }
               ptx::tc_fence_after();
-              const int kh = tp / a.kW, kw = tp - (tp / a.kW) * a.kW;
-              const uint32_t view = hbase + static_cast<uint32_t>(kh * a.dh * a.halo_w + kw * a.dw) * 128u;
-              const uint32_t sb = ptx::smem_u32(bring + bst * a.b_bytes);
+              hbase = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
+            }
+            const int kh = tp / a.kW, kw = tp - (tp / a.kW) * a.kW;
+            const uint32_t view = hbase + static_cast<uint32_t>(kh * a.dh * a.halo_w + kw * a.dw) * 128u;
+            const uint32_t sb = ptx::smem_u32(bring + bst * a.stage_bytes + j * a.b_bytes);
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const uint64_t da = ptx::smem_desc_sw128_view(view + k * 32, sbo, 0);
-                const uint64_t db = ptx::smem_desc(sb + k * 32, 16, 1024, 2);
-                if constexpr (PAIR) ptx::mma_f16_pair(d_tmem, da, db, a.idesc, accumulate);
-                else ptx::mma_f16(d_tmem, da, db, a.idesc, accumulate);
-                accumulate = 1;
-              }
-              if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[bst]), both);
-              else ptx::mma_commit(ptx::smem_u32(&tail->empty[bst]));
-              if (++bst == a.stages) {
-                bst = 0;
-                bph ^= 1u;
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t da = ptx::smem_desc_sw128_view(view + k * 32, sbo, 0);
+              const uint64_t db = ptx::smem_desc(sb + k * 32, 16, 1024, 2);
+              if constexpr (PAIR) ptx::mma_f16_pair(d_tmem, da, db, a.idesc, accumulate);
+              else ptx::mma_f16(d_tmem, da, db, a.idesc, accumulate);
+              accumulate = 1;
+            }
+            if (tp == taps_hw - 1) {
+              // last tap of this (cc, kd): its halo slot is free once these MMAs complete
+              if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->aempty[ast]), both);
+              else ptx::mma_commit(ptx::smem_u32(&tail->aempty[ast]));
+              if (++ast == a.a_slots) {
+                ast = 0;
+                aph ^= 1u;
               }
             }
-            if (!ok) break;
-            if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->aempty[ast]), both);
-            else ptx::mma_commit(ptx::smem_u32(&tail->aempty[ast]));
-            if (++ast == a.a_slots) {
-              ast = 0;
-              aph ^= 1u;
-            }
+          }
+          if (!ok) break;
+          if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[bst]), both);
+          else ptx::mma_commit(ptx::smem_u32(&tail->empty[bst]));
+          if (++bst == a.stages) {
+            bst = 0;
+            bph ^= 1u;
           }
         }
         if (ok) {

@@ -70,6 +70,8 @@ struct TcArgs {
   int cchunks;        // Cg / kc (TMA mode)
   int m_tiles, n_tiles, total_tiles;
   uint32_t a_bytes, b_bytes, stage_bytes;
+  int kbs;              // K sub-blocks (of kc elements) per pipeline stage
+  uint32_t sub_bytes;   // bytes of one sub-block (A and, unless resident, B)
   uint32_t layout_type;  // UMMA smem layout: 2 = 128B swizzle, 4 = 64B, 6 = 32B
   uint32_t sbo;          // bytes between 8-row groups (8 * kc * 2)
   uint32_t idesc;        // tcgen05 instruction descriptor
@@ -529,36 +531,39 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
           const int cw = ow * a.sw - a.pw, chh = oh * a.sh - a.ph, cd = od * a.sd - a.pd;
           const int orow = tc.g * a.Og + tc.nt * a.BN;
           int tap = 0, cchunk = 0;
-          for (int kb = 0; kb < a.kblocks; ++kb) {
+          for (int kb = 0; kb < a.kblocks; kb += a.kbs) {
+            const int nsub = min(a.kbs, a.kblocks - kb);
             if (!wait_bounded(ptx::smem_u32(&tail->empty[stage]), phase ^ 1u, abort_flag,
                               a.timeout_ns, kSiteProducerEmpty)) {
               ok = false;
               break;
             }
             const uint32_t fb = ptx::smem_u32(&tail->full[stage]);
-            ptx::mbar_arrive_expect_tx(fb, a.a_bytes + a.b_bytes);
-            const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes);
-            const uint32_t sb = sa + a.a_bytes;
-            const int kw = tap % a.kW;
-            const int kh = (tap / a.kW) % a.kH;
-            const int kd = tap / (a.kW * a.kH);
-            const int c0 = tc.g * a.Cg + cchunk * a.kc;
-            if (a.rank5) {
-              ptx::tma_load_im2col_5d(sa, &tmap_x, fb, c0, cw, chh, cd, n,
-                                      static_cast<uint16_t>(kw * a.dw),
-                                      static_cast<uint16_t>(kh * a.dh),
-                                      static_cast<uint16_t>(kd * a.dd));
-            } else {
-              ptx::tma_load_im2col_4d(sa, &tmap_x, fb, c0, cw, chh, n,
-                                      static_cast<uint16_t>(kw * a.dw),
-                                      static_cast<uint16_t>(kh * a.dh));
+            ptx::mbar_arrive_expect_tx(fb, static_cast<uint32_t>(nsub) * (a.a_bytes + a.b_bytes));
+            for (int j = 0; j < nsub; ++j) {
+              const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes + j * a.sub_bytes);
+              const uint32_t sb = sa + a.a_bytes;
+              const int kw = tap % a.kW;
+              const int kh = (tap / a.kW) % a.kH;
+              const int kd = tap / (a.kW * a.kH);
+              const int c0 = tc.g * a.Cg + cchunk * a.kc;
+              if (a.rank5) {
+                ptx::tma_load_im2col_5d(sa, &tmap_x, fb, c0, cw, chh, cd, n,
+                                        static_cast<uint16_t>(kw * a.dw),
+                                        static_cast<uint16_t>(kh * a.dh),
+                                        static_cast<uint16_t>(kd * a.dd));
+              } else {
+                ptx::tma_load_im2col_4d(sa, &tmap_x, fb, c0, cw, chh, n,
+                                        static_cast<uint16_t>(kw * a.dw),
+                                        static_cast<uint16_t>(kh * a.dh));
+              }
+              ptx::tma_load_2d(sb, &tmap_w, fb, tap * a.Cg + cchunk * a.kc, orow);
+              if (++cchunk == a.cchunks) {
+                cchunk = 0;
+                ++tap;
+              }
             }
-            ptx::tma_load_2d(sb, &tmap_w, fb, tap * a.Cg + cchunk * a.kc, orow);
             ++fills;
-            if (++cchunk == a.cchunks) {
-              cchunk = 0;
-              ++tap;
-            }
             if (++stage == a.stages) {
               stage = 0;
               phase ^= 1u;
@@ -606,21 +611,24 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
         st.jhi = min(a.kW, a.W - st.iw0) * a.C;
         if (st.jhi < st.jlo) st.jhi = st.jlo;
         const int n0 = tc.nt * a.BN;
-        for (int kb = 0; kb < a.kblocks; ++kb) {
+        for (int kb = 0; kb < a.kblocks; kb += a.kbs) {
+          const int nsub = min(a.kbs, a.kblocks - kb);
           if (!wait_bounded(ptx::smem_u32(&tail->empty[stage]), phase ^ 1u, abort_flag, a.timeout_ns,
                             kSiteProducerEmpty)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + stage * a.stage_bytes;
-          const int k0 = kb * 64 + half * 32;
-          if (a.gather_mode == GATHER_VEC8)
-            gather_a_vec8(a, st, k0, sa, r, half * 4);
-          else if (a.gather_mode == GATHER_SPAN)
-            gather_a_span(a, st, k0, sa, r, half * 4);
-          else
-            gather_a_scalar(a, st, k0, sa, r, half * 4);
-          if (!a.b_resident) gather_b_block(a, tc.g, n0, kb * 64, sa + a.a_bytes, tid, kProdThreads);
+          for (int j = 0; j < nsub; ++j) {
+            uint8_t* sa = smem + stage * a.stage_bytes + j * a.sub_bytes;
+            const int k0 = (kb + j) * 64 + half * 32;
+            if (a.gather_mode == GATHER_VEC8)
+              gather_a_vec8(a, st, k0, sa, r, half * 4);
+            else if (a.gather_mode == GATHER_SPAN)
+              gather_a_span(a, st, k0, sa, r, half * 4);
+            else
+              gather_a_scalar(a, st, k0, sa, r, half * 4);
+            if (!a.b_resident) gather_b_block(a, tc.g, n0, (kb + j) * 64, sa + a.a_bytes, tid, kProdThreads);
+          }
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(ptx::smem_u32(&tail->full[stage]));
           if (++stage == a.stages) {
@@ -653,21 +661,24 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
-        for (int kb = 0; kb < a.kblocks; ++kb) {
+        for (int kb = 0; kb < a.kblocks; kb += a.kbs) {
+          const int nsub = min(a.kbs, a.kblocks - kb);
           if (!wait_bounded(ptx::smem_u32(&tail->full[stage]), phase, abort_flag, a.timeout_ns,
                             kSiteMmaFull)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes);
-          const uint32_t sb =
-              a.b_resident ? bres_addr + static_cast<uint32_t>(kb) * a.BN * 128u : sa + a.a_bytes;
           const int ksteps = a.kc >> 4;
-          for (int k = 0; k < ksteps; ++k) {
-            const uint64_t da = ptx::smem_desc(sa + k * 32, 16, a.sbo, a.layout_type);
-            const uint64_t db = ptx::smem_desc(sb + k * 32, 16, a.sbo, a.layout_type);
-            ptx::mma_f16(d_tmem, da, db, a.idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int j = 0; j < nsub; ++j) {
+            const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes + j * a.sub_bytes);
+            const uint32_t sb = a.b_resident ? bres_addr + static_cast<uint32_t>(kb + j) * a.BN * 128u
+                                             : sa + a.a_bytes;
+            for (int k = 0; k < ksteps; ++k) {
+              const uint64_t da = ptx::smem_desc(sa + k * 32, 16, a.sbo, a.layout_type);
+              const uint64_t db = ptx::smem_desc(sb + k * 32, 16, a.sbo, a.layout_type);
+              ptx::mma_f16(d_tmem, da, db, a.idesc, ((kb + j) | k) != 0 ? 1u : 0u);
+            }
           }
           ptx::mma_commit(ptx::smem_u32(&tail->empty[stage]));
           if (++stage == a.stages) {
@@ -813,33 +824,37 @@ __global__ void __launch_bounds__(192, 1)
         const int cw = ow * a.sw - a.pw, chh = oh * a.sh - a.ph, cd = od * a.sd - a.pd;
         const int brow = tc.g * a.Og + tc.nt * a.BN + static_cast<int>(rank) * half_bn;
         int tap = 0, cchunk = 0;
-        for (int kb = 0; kb < a.kblocks; ++kb) {
+        for (int kb = 0; kb < a.kblocks; kb += a.kbs) {
+          const int nsub = min(a.kbs, a.kblocks - kb);
           if (!wait_bounded(ptx::smem_u32(&tail->empty[stage]), phase ^ 1u, abort_flag, a.timeout_ns,
                             kSiteProducerEmpty)) {
             ok = false;
             break;
           }
           const uint32_t fb_local = ptx::smem_u32(&tail->full[stage]);
-          if (leader) ptx::mbar_arrive_expect_tx(fb_local, 2u * (a.a_bytes + a.b_bytes));
+          if (leader)
+            ptx::mbar_arrive_expect_tx(fb_local, 2u * static_cast<uint32_t>(nsub) * (a.a_bytes + a.b_bytes));
           const uint32_t fb = ptx::mapa_shared(fb_local, 0);
-          const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes);
-          const uint32_t sb = sa + a.a_bytes;
-          const int kw = tap % a.kW;
-          const int kh = (tap / a.kW) % a.kH;
-          const int kd = tap / (a.kW * a.kH);
-          const int c0 = tc.g * a.Cg + cchunk * a.kc;
-          if (a.rank5)
-            ptx::tma_load_im2col_5d_pair(sa, &tmap_x, fb, c0, cw, chh, cd, n, static_cast<uint16_t>(kw * a.dw),
-                                         static_cast<uint16_t>(kh * a.dh), static_cast<uint16_t>(kd * a.dd));
-          else
-            ptx::tma_load_im2col_4d_pair(sa, &tmap_x, fb, c0, cw, chh, n, static_cast<uint16_t>(kw * a.dw),
-                                         static_cast<uint16_t>(kh * a.dh));
-          ptx::tma_load_2d_pair(sb, &tmap_w, fb, tap * a.Cg + cchunk * a.kc, brow);
-          ++fills;
-          if (++cchunk == a.cchunks) {
-            cchunk = 0;
-            ++tap;
+          for (int j = 0; j < nsub; ++j) {
+            const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes + j * a.sub_bytes);
+            const uint32_t sb = sa + a.a_bytes;
+            const int kw = tap % a.kW;
+            const int kh = (tap / a.kW) % a.kH;
+            const int kd = tap / (a.kW * a.kH);
+            const int c0 = tc.g * a.Cg + cchunk * a.kc;
+            if (a.rank5)
+              ptx::tma_load_im2col_5d_pair(sa, &tmap_x, fb, c0, cw, chh, cd, n, static_cast<uint16_t>(kw * a.dw),
+                                           static_cast<uint16_t>(kh * a.dh), static_cast<uint16_t>(kd * a.dd));
+            else
+              ptx::tma_load_im2col_4d_pair(sa, &tmap_x, fb, c0, cw, chh, n, static_cast<uint16_t>(kw * a.dw),
+                                           static_cast<uint16_t>(kh * a.dh));
+            ptx::tma_load_2d_pair(sb, &tmap_w, fb, tap * a.Cg + cchunk * a.kc, brow);
+            if (++cchunk == a.cchunks) {
+              cchunk = 0;
+              ++tap;
+            }
           }
+          ++fills;
           if (++stage == a.stages) {
             stage = 0;
             phase ^= 1u;
@@ -874,19 +889,22 @@ __global__ void __launch_bounds__(192, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
-        for (int kb = 0; kb < a.kblocks; ++kb) {
+        for (int kb = 0; kb < a.kblocks; kb += a.kbs) {
+          const int nsub = min(a.kbs, a.kblocks - kb);
           if (!wait_bounded(ptx::smem_u32(&tail->full[stage]), phase, abort_flag, a.timeout_ns, kSiteMmaFull)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes);
-          const uint32_t sb = sa + a.a_bytes;
           const int ksteps = a.kc >> 4;
-          for (int k = 0; k < ksteps; ++k) {
-            const uint64_t da = ptx::smem_desc(sa + k * 32, 16, a.sbo, a.layout_type);
-            const uint64_t db = ptx::smem_desc(sb + k * 32, 16, a.sbo, a.layout_type);
-            ptx::mma_f16_pair(d_tmem, da, db, a.idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int j = 0; j < nsub; ++j) {
+            const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes + j * a.sub_bytes);
+            const uint32_t sb = sa + a.a_bytes;
+            for (int k = 0; k < ksteps; ++k) {
+              const uint64_t da = ptx::smem_desc(sa + k * 32, 16, a.sbo, a.layout_type);
+              const uint64_t db = ptx::smem_desc(sb + k * 32, 16, a.sbo, a.layout_type);
+              ptx::mma_f16_pair(d_tmem, da, db, a.idesc, ((kb + j) | k) != 0 ? 1u : 0u);
+            }
           }
           ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[stage]), 3);
           if (++stage == a.stages) {

@@ -90,10 +90,10 @@ int conv_out_dims(int D, int H, int W, int kD, int kH, int kW,
 /* Forward convolution on device buffers x, w, y (see the layouts above).
  * Queues the kernel on `stream`; returns CONV_OK or an error code (nothing is
  * queued on an error).  The variant is chosen from the type and shape:
- * f32 -> SIMT; f16/bf16 -> TC_HALO_PAIR / TC_HALO for stride 1 and
- * C/G % 64 == 0; otherwise TC_TMA_PAIR / TC_TMA when C/G % 16 == 0 and the
- * geometry fits a TMA im2col tensor map; otherwise TC_GATHER.  The pair
- * forms are chosen when there are at least as many pair tiles as SM pairs. */
+ * f32 -> SIMT; f16/bf16 -> TC_TMA_PAIR (or TC_TMA when there are fewer
+ * 256-row output tiles than SM pairs) when C/G % 16 == 0 and the geometry fits
+ * a TMA im2col tensor map; otherwise TC_GATHER.  TC_HALO and TC_HALO_PAIR run
+ * only when requested through conv_fwd_variant. */
 int conv_fwd(const void* x, const void* w, void* y,
              int N, int D, int H, int W, int C, int O,
              int kD, int kH, int kW,

@@ -111,9 +111,9 @@ def test_strerror_covers_codes(C):
 def test_variant_plan(C):
     plan = lambda *a: C.plan(*a)
     v, bn, st, _ = plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")
-    assert v == C.VARIANT_TC_HALO_PAIR and bn == 256 and st >= 3
+    assert v == C.VARIANT_TC_TMA_PAIR and bn == 256 and st >= 2
     v, bn, _, _ = plan(1, 1, 56, 56, 64, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "f16")
-    assert v == C.VARIANT_TC_HALO and bn == 64
+    assert v == C.VARIANT_TC_TMA and bn == 64
     v, bn, _, _ = plan(4, 32, 32, 32, 64, 128, (3, 3, 3), (2, 2, 2), (1, 1, 1), (1, 1, 1), 1, "f16")
     assert v in (C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR) and bn == 128
     v, bn, _, _ = plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
@@ -122,14 +122,10 @@ def test_variant_plan(C):
     assert v == C.VARIANT_TC_GATHER and bn == 96
     v, _, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f32")
     assert v == C.VARIANT_SIMT
-    # 3-D with pad beyond the rank-5 im2col corner range: the halo kernel (tiled
-    # boxes take any offset) at stride 1, the gather kernel at stride 2
+    # 3-D with pad beyond the rank-5 im2col corner range goes to the gather kernel
     v, _, _, _ = plan(1, 40, 8, 8, 64, 64, (3, 3, 3), (1, 1, 1), (17, 1, 1), (1, 1, 1), 1, "f16")
-    assert v == C.VARIANT_TC_HALO
-    v, _, _, _ = plan(1, 40, 8, 8, 64, 64, (3, 3, 3), (2, 1, 1), (17, 1, 1), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_GATHER
     # channel chunks of 32 and 16
     assert plan(2, 64, 64, 64, 32, 64, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA_PAIR
     assert plan(1, 1, 9, 9, 48, 96, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 3, "f16")[0] == C.VARIANT_TC_TMA
-    # 64-channel groups at stride 1 take the halo kernel
-    assert plan(1, 1, 9, 9, 128, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 2, "f16")[0] == C.VARIANT_TC_HALO
+    assert plan(1, 1, 9, 9, 128, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 2, "f16")[0] == C.VARIANT_TC_TMA

@@ -56,7 +56,7 @@ def variants_for(wl):
     vs.append(C.VARIANT_TC_GATHER)
     if (wl.C // wl.groups) % 16 == 0:
         vs += [C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR]
-    if (wl.C // wl.groups) % 64 == 0 and tuple(wl.stride) == (1, 1, 1):
+    if (wl.C // wl.groups) % 64 == 0 and tuple(wl.stride) == (1, 1, 1) and wl.k[1] * wl.k[2] >= 4:
         vs += [C.VARIANT_TC_HALO, C.VARIANT_TC_HALO_PAIR]
     return vs
 
@@ -123,8 +123,8 @@ def test_tutorial_example_on_gpu(dtype):
 
 
 def test_auto_variant_choice():
-    assert C.plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_HALO_PAIR
-    assert C.plan(1, 1, 56, 56, 64, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_HALO
+    assert C.plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_TMA_PAIR
+    assert C.plan(1, 1, 56, 56, 64, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA
     assert C.plan(4, 32, 32, 32, 64, 128, (3, 3, 3), (2, 2, 2), (1, 1, 1), (1, 1, 1), 1, "f16")[0] in (
         C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR)
     assert C.plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
