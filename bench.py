@@ -118,62 +118,94 @@ def profiled_traffic(workload, variant_name):
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples (200 ms) during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons sampled DURING the timed region.
+
+    Uses NVML (the library nvidia-smi reads) every ~5 ms from a thread, so that
+    a timed region of a few milliseconds still gets samples; falls back to
+    `nvidia-smi -lms 200` where NVML cannot be loaded."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.samples = []      # (sm_mhz, max_mhz, reasons bitmask)
+        self._stop = threading.Event()
         self._t = None
+        self._nvml = None
+        self._smi = None
+        self._lines = []
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, ValueError):
-            self.proc = None
-            return
-        self._t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self._nvml = (pynvml, h)
+            self._t = threading.Thread(target=self._poll_nvml, daemon=True)
+        except Exception:
+            self._nvml = None
+            try:
+                fields = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+                self._smi = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={fields}", "--format=csv,noheader,nounits",
+                     "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self._t = threading.Thread(target=self._read_smi, daemon=True)
+            except (OSError, ValueError):
+                return
         self._t.start()
-        time.sleep(0.25)
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _poll_nvml(self):
+        pynvml, h = self._nvml
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            try:
+                t = time.perf_counter()
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), int(rs), t))
+            except Exception:
+                break
+            time.sleep(0.005)
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        if self._t:
-            self._t.join(timeout=2)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
+    def _read_smi(self):
+        for line in self._smi.stdout:
+            parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                bits = 0
+                for name, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                   parts[5:9]):
+                    if v.lower().startswith("active"):
+                        bits |= self.REASONS[name]
+                self.samples.append((float(parts[1]), float(parts[2]), bits, time.perf_counter()))
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
+
+    def stop(self, t0=None, t1=None):
+        """Stop sampling; summarise the samples taken inside [t0, t1] (the timed
+        region's wall clock) when there are any, else all of them."""
+        self._stop.set()
+        if self._smi is not None:
+            self._smi.terminate()
+            try:
+                self._smi.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._smi.kill()
+        if self._t is not None:
+            self._t.join(timeout=5)
+        if t0 is not None:
+            inside = [x for x in self.samples if t0 <= x[3] <= t1]
+            if inside:
+                self.samples = inside
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = sorted(n for n, b in self.REASONS.items() if any(s[2] & b for s in self.samples))
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": max(s[1] for s in self.samples),
+                "sm_min_mhz": min(s[0] for s in self.samples), "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml" if self._nvml else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------- distributed
@@ -285,11 +317,13 @@ def bench_ours(args):
 
     clocks = ClockSampler(local)
     clocks.start()
+    time.sleep(0.01)
     barrier(dist, dev)
     torch.cuda.synchronize(dev)
     launches = 0
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.perf_counter()
     ev0.record(stream)
     if graph is not None:
         graph.replay()
@@ -299,8 +333,9 @@ def bench_ours(args):
             step(args.warmup + i)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
+    t_wall1 = time.perf_counter()
     barrier(dist, dev)
-    clk = clocks.stop()
+    clk = clocks.stop(t_wall0, t_wall1)
     local_ms = ev0.elapsed_time(ev1)
     timed_launches = launches
     status = C.last_status()
@@ -370,7 +405,9 @@ def bench_ours(args):
                    "kernel": list(wl.k), "stride": list(wl.stride), "pad": list(wl.pad), "dil": list(wl.dil),
                    "groups": wl.groups, "out_DHW": list(dims), "gflop_per_step": round(flops / 1e9, 4),
                    "global_batch": wl.N * nranks, "parallelism": f"independent batches x{nranks}",
-                   "variant": vname, "tile": [128, bn], "stages": stages, "ctas": ctas,
+                   "variant": vname,
+                   "tile": [64, 64] if variant == C.VARIANT_SIMT else [256 if "pair" in vname else 128, bn],
+                   "stages": stages, "ctas": ctas,
                    "l2": f"inputs rotate over {nsets} buffer sets ({nsets * per_set / 2**20:.0f} MiB > 2x L2)"},
         "roofline": roof,
         "launch": "cuda_graph_of_steps" if graph is not None else "eager",
@@ -450,7 +487,7 @@ def bench_reference(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=WL.HEADLINE, choices=sorted(WL.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

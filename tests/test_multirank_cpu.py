@@ -1,0 +1,92 @@
+"""The benchmark's multi-rank plumbing on CPU (gloo, world size 2).
+
+The forward convolution shards over independent batches with no data-path
+collective; what ranks share is only the timing: a barrier around the timed
+region and the maximum of the per-rank device times.  This checks that logic
+with two gloo processes.
+"""
+from __future__ import annotations
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import bench
+    ws, r, local = bench.dist_env()
+    assert (ws, r, local) == (world, rank, rank)
+    d = bench.init_dist(ws, "gloo")
+    bench.barrier(d)
+    local_ms = 10.0 * (rank + 1)                 # rank 1 is the slow one
+    ms, n = bench.aggregate(d, local_ms)
+    out[rank] = (ms, n)
+    d.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_two_rank_max_time_gloo():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(100)
+        assert p.exitcode == 0
+    assert out[0] == (20.0, 2) and out[1] == (20.0, 2)
+
+
+def test_single_rank_needs_no_process_group():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.init_dist(1, "gloo") is None
+    assert bench.aggregate(None, 3.5) == (3.5, 1)
+
+
+def test_flop_and_byte_counters_match_the_tutorial():
+    """The bench's FLOP and byte counters against the printed figures of the
+    "Convolutions" tutorial (golden fixture): 236 MFLOP for the ResNet-50 stem,
+    3.7 GFLOP / 4.4 MB / 841 FLOP per byte for the 3x3 256->256 layer."""
+    import json
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as WL
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "tutorial_counts.json")))
+    st = g["stem"]
+    wl = WL.case(1, 1, st["H"], st["W"], st["C"], st["O"], (1, st["k"], st["k"]), (1, st["stride"], st["stride"]),
+                 (0, st["pad"], st["pad"]), dtype="bf16")
+    dims = (1, st["H_out"], st["W_out"])
+    f = bench.conv_flops(wl, dims)
+    assert f == 2 * 112 * 112 * 3 * 64 * 7 * 7
+    assert abs(f / st["flops_printed"] - 1) < st["flops_rel_tol"]
+    c3 = g["conv3x3_256"]
+    wl = WL.case(1, 1, c3["H"], c3["W"], c3["C"], c3["O"], (1, 3, 3), pad=(0, 1, 1), dtype="bf16")
+    dims = (1, 56, 56)
+    f = bench.conv_flops(wl, dims)
+    xb, wb, yb = bench.conv_bytes(wl, dims)
+    assert abs(f / c3["flops_printed"] - 1) < c3["flops_rel_tol"]
+    for got, key in ((xb, "x_bytes_printed"), (wb, "w_bytes_printed"), (yb, "y_bytes_printed"),
+                     (xb + wb + yb, "bytes_printed")):
+        assert abs(got / c3[key] - 1) < c3["bytes_rel_tol"], (key, got)
+    assert abs(f / (xb + wb + yb) / c3["intensity_printed"] - 1) < c3["intensity_rel_tol"]
