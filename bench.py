@@ -259,7 +259,7 @@ def bench_ours(args):
     flops = conv_flops(wl, dims)
     xb, wb, yb = conv_bytes(wl, dims)
     variant, bn, stages, ctas = C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil,
-                                       wl.groups, wl.dtype)
+                                       wl.groups, wl.dtype, getattr(C, "VARIANT_" + args.variant))
     vname = C.VARIANT_NAMES[variant]
 
     # inputs: seeded on the host (rank-dependent seed), copied once
@@ -281,7 +281,7 @@ def bench_ours(args):
         s = i % nsets
         # the launch goes to the current stream (the capture stream while a graph is recorded)
         rc = C.conv_fwd_raw(xs[s].data_ptr(), wts[s].data_ptr(), ys[s].data_ptr(), geo(s), dcode,
-                            C.VARIANT_AUTO, torch.cuda.current_stream(dev).cuda_stream)
+                            variant, torch.cuda.current_stream(dev).cuda_stream)
         if rc:
             raise C.ConvError(rc, "conv_fwd")
         launches += 1
@@ -406,7 +406,8 @@ def bench_ours(args):
                    "groups": wl.groups, "out_DHW": list(dims), "gflop_per_step": round(flops / 1e9, 4),
                    "global_batch": wl.N * nranks, "parallelism": f"independent batches x{nranks}",
                    "variant": vname,
-                   "tile": [64, 64] if variant == C.VARIANT_SIMT else [256 if "pair" in vname else 128, bn],
+                   "tile": ([64, 64] if variant == C.VARIANT_SIMT else
+                            [bn, 128] if variant == C.VARIANT_TC_TMA_T else [256 if "pair" in vname else 128, bn]),
                    "stages": stages, "ctas": ctas,
                    "l2": f"inputs rotate over {nsets} buffer sets ({nsets * per_set / 2**20:.0f} MiB > 2x L2)"},
         "roofline": roof,
@@ -494,6 +495,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
+    ap.add_argument("--variant", default="AUTO",
+                    choices=["AUTO", "SIMT", "TC_TMA", "TC_GATHER", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T"],
+                    help="kernel variant (default: the library's own choice)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps

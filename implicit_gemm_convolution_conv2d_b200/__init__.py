@@ -17,14 +17,16 @@ import os
 
 __all__ = ["conv_fwd", "conv_fwd_host", "out_dims", "plan", "last_status", "strerror", "lib",
            "CONV_F32", "CONV_F16", "CONV_BF16", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC_TMA",
-           "VARIANT_TC_GATHER", "VARIANT_TC_TMA_PAIR", "VARIANT_TC_HALO", "VARIANT_TC_HALO_PAIR", "ConvError"]
+           "VARIANT_TC_GATHER", "VARIANT_TC_TMA_PAIR", "VARIANT_TC_HALO", "VARIANT_TC_HALO_PAIR",
+           "VARIANT_TC_TMA_T", "ConvError"]
 
 CONV_F32, CONV_F16, CONV_BF16 = 0, 1, 2
 VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC_TMA, VARIANT_TC_GATHER, VARIANT_TC_TMA_PAIR = -1, 0, 1, 2, 3
-VARIANT_TC_HALO, VARIANT_TC_HALO_PAIR = 4, 5
+VARIANT_TC_HALO, VARIANT_TC_HALO_PAIR, VARIANT_TC_TMA_T = 4, 5, 6
 VARIANT_NAMES = {VARIANT_SIMT: "simt_ffma", VARIANT_TC_TMA: "tcgen05_tma_im2col",
                  VARIANT_TC_GATHER: "tcgen05_gather", VARIANT_TC_TMA_PAIR: "tcgen05_tma_im2col_pair",
-                 VARIANT_TC_HALO: "tcgen05_tma_halo", VARIANT_TC_HALO_PAIR: "tcgen05_tma_halo_pair"}
+                 VARIANT_TC_HALO: "tcgen05_tma_halo", VARIANT_TC_HALO_PAIR: "tcgen05_tma_halo_pair",
+                 VARIANT_TC_TMA_T: "tcgen05_tma_im2col_t"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libconvfwd.so")
@@ -53,12 +55,13 @@ def lib() -> ctypes.CDLL:
         L.conv_fwd_variant.argtypes = [vp, vp, vp] + geo + [ci, vp]
         L.conv_fwd_host.argtypes = [vp] * 6 + geo + [vp]
         L.conv_plan.argtypes = geo + [i3, i3, i3]
+        L.conv_plan_variant.argtypes = geo + [ci, i3, i3, i3]
         L.conv_last_status.argtypes = [vp]
         L.conv_debug_inject_stall.argtypes = [ctypes.c_ulonglong]
         L.conv_strerror.argtypes = [ci]
         L.conv_strerror.restype = ctypes.c_char_p
         for f in ("conv_out_dims", "conv_fwd", "conv_fwd_variant", "conv_fwd_host", "conv_plan",
-                  "conv_last_status", "conv_version", "conv_debug_inject_stall"):
+                  "conv_plan_variant", "conv_last_status", "conv_version", "conv_debug_inject_stall"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
@@ -186,13 +189,15 @@ def conv_fwd_host(x_host, w_host, y_host, x_dev, w_dev, y_dev, stride=1, padding
     return y_host
 
 
-def plan(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype):
-    """(variant, BN, stages, ctas) the library would use; dtype is 'f32' | 'f16' | 'bf16'."""
+def plan(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype, variant=VARIANT_AUTO):
+    """(variant, BN, stages, ctas) the library would use; dtype is 'f32' | 'f16' | 'bf16'.
+    With an explicit `variant`, the plan of that variant (ConvError if it cannot run)."""
     code = {"f32": CONV_F32, "f16": CONV_F16, "bf16": CONV_BF16}[dtype]
     bn, st, ct = (ctypes.c_int * 1)(), (ctypes.c_int * 1)(), (ctypes.c_int * 1)()
-    v = lib().conv_plan(N, D, H, W, C, O, *k, _i3(stride), _i3(pad), _i3(dil), int(groups), code, bn, st, ct)
+    v = lib().conv_plan_variant(N, D, H, W, C, O, *k, _i3(stride), _i3(pad), _i3(dil), int(groups), code,
+                                int(variant), bn, st, ct)
     if v < 0:
-        raise ConvError(v, "conv_plan")
+        raise ConvError(v, "conv_plan_variant")
     return v, bn[0], st[0], ct[0]
 
 

@@ -15,6 +15,7 @@
 #include "conv_halo.cuh"
 #include "conv_simt.cuh"
 #include "conv_tc.cuh"
+#include "conv_tct.cuh"
 
 namespace convfwd {
 namespace {
@@ -153,6 +154,8 @@ int set_kernel_attrs(int dev) {
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_t_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_t_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return CONV_ELAUNCH;
   g_dev[dev].attrs_set = true;
   return CONV_OK;
@@ -334,9 +337,65 @@ int plan_halo(const Problem& P, bool pair, int sms, TcPlan& plan) {
   return CONV_OK;
 }
 
+// Transposed orientation: M = 128 output channels, N = BP output pixels.
+// Needs what the im2col kernels need plus whole 128-channel tiles per group.
+// BP = 256 when that still gives every SM a tile, else 128.
+int plan_tc_t(const Problem& P, int sms, TcPlan& plan) {
+  bool rank5 = false;
+  if (!tma_fits(P, rank5) || P.Og % kTO != 0) return CONV_EUNSUPPORTED;
+  if (P.M > 0x7fffffffLL - 256) return CONV_EUNSUPPORTED;  // TMA store row coordinate
+  TcArgs& a = plan.args;
+  std::memset(&a, 0, sizeof(a));
+  a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.C = P.C; a.O = P.O;
+  a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
+  a.sd = P.s[0]; a.sh = P.s[1]; a.sw = P.s[2];
+  a.pd = P.p[0]; a.ph = P.p[1]; a.pw = P.p[2];
+  a.dd = P.d[0]; a.dh = P.d[1]; a.dw = P.d[2];
+  a.G = P.G; a.Cg = P.Cg; a.Og = P.Og;
+  a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
+  a.M = P.M;
+  a.K = static_cast<int>(P.K);
+  a.n_tiles = P.Og / kTO;
+  const long long wide_tiles = (P.M + 255) / 256 * a.n_tiles * P.G;
+  a.BN = wide_tiles >= sms ? 256 : 128;  // output pixels per tile (MMA N)
+  const long long mt = (P.M + a.BN - 1) / a.BN;
+  const long long tt = mt * a.n_tiles * P.G;
+  if (tt > 0x7fffffffLL) return CONV_EINVAL;
+  a.m_tiles = static_cast<int>(mt);
+  a.total_tiles = static_cast<int>(tt);
+  a.kc = (P.Cg % 64 == 0) ? 64 : (P.Cg % 32 == 0 ? 32 : 16);
+  a.cchunks = P.Cg / a.kc;
+  a.kblocks = P.kD * P.kH * P.kW * a.cchunks;
+  a.rank5 = rank5 ? 1 : 0;
+  a.layout_type = a.kc == 64 ? 2u : (a.kc == 32 ? 4u : 6u);
+  a.sbo = static_cast<uint32_t>(8 * a.kc * 2);
+  a.a_bytes = static_cast<uint32_t>(kTO * a.kc * 2);    // weight tile
+  a.b_bytes = static_cast<uint32_t>(a.BN * a.kc * 2);   // patch rows
+  a.sub_bytes = a.a_bytes + a.b_bytes;
+  const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
+                          64 - 2LL * kTEpiBytes;
+  int stages = 0;
+  a.kbs = choose_kbs(a.BN, a.kc, a.sub_bytes, avail, 8, stages);
+  if (stages < 2) return CONV_EUNSUPPORTED;
+  a.stages = stages;
+  a.stage_bytes = static_cast<uint32_t>(a.kbs) * a.sub_bytes;
+  const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
+  a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(a.BN >> 3) << 17) |
+            ((static_cast<uint32_t>(kTO) >> 4) << 24);
+  a.tmem_cols = next_pow2_cols(static_cast<uint32_t>(2 * a.BN));
+  a.timeout_ns = kWaitTimeoutNs;
+  plan.variant = CONV_VARIANT_TC_TMA_T;
+  plan.pair = false;
+  plan.ctas = std::min(a.total_tiles, sms);
+  plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + 2 * static_cast<size_t>(kTEpiBytes) + 1024 +
+              sizeof(TcSmemTail) + 64;
+  return CONV_OK;
+}
+
 int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
   if (variant == CONV_VARIANT_TC_HALO || variant == CONV_VARIANT_TC_HALO_PAIR)
     return plan_halo(P, variant == CONV_VARIANT_TC_HALO_PAIR, sms, plan);
+  if (variant == CONV_VARIANT_TC_TMA_T) return plan_tc_t(P, sms, plan);
   if (P.dtype == CONV_F32) return CONV_EUNSUPPORTED;
   TcArgs& a = plan.args;
   std::memset(&a, 0, sizeof(a));
@@ -380,7 +439,38 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
       a.gather_mode = GATHER_SCALAR;
     }
     a.Lp = round_up(P.kW * P.C, 8);
-    const long long kp = a.gather_mode == GATHER_SPAN ? static_cast<long long>(P.kD) * P.kH * a.Lp : P.K;
+    // Row staging: 2-D problems in span layout whose input rows are 16-byte
+    // strided and whose 128-pixel tiles touch at most two images get their
+    // input rows by TMA instead of per-thread loads.
+    if (a.gather_mode == GATHER_SPAN && P.D == 1 && P.kD == 1 && P.p[0] == 0 &&
+        (static_cast<long long>(P.W) * P.C) % 8 == 0 && static_cast<long long>(P.Ho) * P.Wo >= kBM) {
+      // a row of row_e = W*C elements is one box row of n_boxes x box_e, with
+      // box_e the largest multiple-of-8 divisor of row_e that is <= 256
+      const long long we = static_cast<long long>(P.W) * P.C;
+      int box_e = 0;
+      for (int b = 256; b >= 32; b -= 8)
+        if (we % b == 0) {
+          box_e = b;
+          break;
+        }
+      const long long n_boxes = box_e ? we / box_e : 0;
+      const int orows = std::min(P.Ho, (kBM - 1) / P.Wo + 2);
+      const long long stage_rows = static_cast<long long>(orows - 1) * P.s[1] + static_cast<long long>(P.kH - 1) * P.d[1] + 1;
+      const long long seg = (stage_rows * we * 2 + 127) / 128 * 128;
+      const long long rows_bytes = (2 * seg + 1023) / 1024 * 1024;
+      if (box_e && n_boxes <= 256 && stage_rows <= 256 && 3 * rows_bytes <= 108 * 1024 &&
+          P.N * static_cast<long long>(P.H) < (1LL << 31)) {
+        a.gather_mode = GATHER_ROWS;
+        a.box_e = box_e;
+        a.n_boxes = static_cast<int>(n_boxes);
+        a.stage_rows = static_cast<int>(stage_rows);
+        a.row_e = static_cast<int>(we);
+        a.seg_bytes = static_cast<uint32_t>(seg);
+        a.rows_bytes = static_cast<uint32_t>(rows_bytes);
+      }
+    }
+    const long long kp = (a.gather_mode == GATHER_SPAN || a.gather_mode == GATHER_ROWS)
+                             ? static_cast<long long>(P.kD) * P.kH * a.Lp : P.K;
     if (kp > 0x7fffffffLL - 64) return CONV_EINVAL;
     a.Kp = static_cast<int>(kp);
     a.kblocks = static_cast<int>((kp + 63) / 64);
@@ -400,8 +490,8 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
     }
   }
   a.sub_bytes = a.a_bytes + (a.b_resident ? 0u : a.b_bytes);
-  const long long avail =
-      static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64 - a.bres_bytes;
+  const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64 -
+                          a.bres_bytes - 3LL * a.rows_bytes;
   int stages = 0;
   a.kbs = choose_kbs(a.BN, a.kc, a.sub_bytes, avail, 8, stages);
   if (stages < 2) return CONV_EUNSUPPORTED;
@@ -415,18 +505,26 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
   a.timeout_ns = kWaitTimeoutNs;
   plan.variant = variant;
   plan.ctas = plan.pair ? 2 * std::min(a.total_tiles, sms / 2) : std::min(a.total_tiles, sms);
-  plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + a.bres_bytes + 1024 + sizeof(TcSmemTail) + 64;
+  plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + a.bres_bytes + 3 * static_cast<size_t>(a.rows_bytes) +
+              1024 + sizeof(TcSmemTail) + 64;
   return CONV_OK;
 }
 
-// f32 -> SIMT.  f16/bf16 -> TMA im2col when it can describe the problem
-// (CTA pairs once there are at least as many 256-row tiles as SM pairs),
-// else the in-kernel gather.  The halo kernels are explicit-only: on B200
-// they measure slower than im2col at every shape of the workload set.
+// f32 -> SIMT.  f16/bf16 -> TMA im2col when it can describe the problem,
+// else the in-kernel gather.  Among the im2col kernels: the transposed
+// orientation when the output channels per group come in 128-wide tiles that
+// a 256-wide one cannot cover (O/G = 128, 384, ...) and there are enough
+// 256-pixel tiles for every SM; otherwise CTA pairs once there are at least
+// as many 256-row tiles as SM pairs; otherwise single CTAs.  The halo kernels
+// are explicit-only: on B200 they measure slower than im2col at every shape
+// of the workload set.
 int choose_variant(const Problem& P, int sms) {
   if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
   bool r5;
   if (!tma_fits(P, r5)) return CONV_VARIANT_TC_GATHER;
+  if (P.Og % kTO == 0 && P.Og % 256 != 0 && P.M <= 0x7fffffffLL - 256 &&
+      (P.M + 255) / 256 * (P.Og / kTO) * P.G >= sms)
+    return CONV_VARIANT_TC_TMA_T;
   const long long og_tiles = (P.Og + 255) / 256;
   const long long pair_tiles = (P.M + 2 * kBM - 1) / (2 * kBM) * og_tiles * P.G;
   return pair_tiles >= sms / 2 ? CONV_VARIANT_TC_TMA_PAIR : CONV_VARIANT_TC_TMA;
@@ -434,11 +532,50 @@ int choose_variant(const Problem& P, int sms) {
 
 // ---------------------------------------------------------------- launches
 
+// y viewed as [M, O] (O innermost) for the transposed kernel's TMA stores:
+// boxes of 128 channels x 32 pixels, rows beyond M clipped.
+int encode_y_map(const Problem& P, void* y, CUtensorMap& my) {
+  std::memset(&my, 0, sizeof(my));
+  const DriverFns& drv = driver_fns();
+  if (!drv.tiled) return CONV_EDRIVER;
+  const CUtensorMapDataType dt =
+      P.dtype == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  cuuint64_t dim[2] = {static_cast<cuuint64_t>(P.O), static_cast<cuuint64_t>(P.M)};
+  cuuint64_t str[1] = {static_cast<cuuint64_t>(P.O) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTO), static_cast<cuuint32_t>(kTEpiRows)};
+  cuuint32_t est[2] = {1, 1};
+  const CUresult r = drv.tiled(&my, dt, 2, y, dim, str, box, est, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  small_tensor_fixup(my, static_cast<size_t>(P.M) * P.O * 2, drv.driver_version);
+  return CONV_OK;
+}
+
 int encode_maps(const Problem& P, const TcArgs& a, bool pair, bool halo, const void* x, const void* w,
-                CUtensorMap& mx, CUtensorMap& mw) {
+                CUtensorMap& mx, CUtensorMap& mw, int w_rows = 0) {
   std::memset(&mx, 0, sizeof(mx));
   std::memset(&mw, 0, sizeof(mw));
-  if (a.cchunks == 0) return CONV_OK;  // gather mode: maps unused
+  if (a.cchunks == 0 && a.gather_mode == GATHER_ROWS) {
+    // x viewed as [N*H][W*C / box_e][box_e]; one box of stage_rows whole rows, zero fill
+    const DriverFns& drv = driver_fns();
+    if (!drv.tiled) return CONV_EDRIVER;
+    const CUtensorMapDataType dt =
+        P.dtype == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    cuuint64_t rdim[3] = {static_cast<cuuint64_t>(a.box_e), static_cast<cuuint64_t>(a.n_boxes),
+                          static_cast<cuuint64_t>(P.N) * P.H};
+    cuuint64_t rstr[2] = {static_cast<cuuint64_t>(a.box_e) * 2, static_cast<cuuint64_t>(P.W) * P.C * 2};
+    cuuint32_t rbox[3] = {static_cast<cuuint32_t>(a.box_e), static_cast<cuuint32_t>(a.n_boxes),
+                          static_cast<cuuint32_t>(a.stage_rows)};
+    cuuint32_t rest[3] = {1, 1, 1};
+    const CUresult r = drv.tiled(&mx, dt, 3, const_cast<void*>(x), rdim, rstr, rbox, rest,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+    small_tensor_fixup(mx, P.x_bytes, drv.driver_version);
+    return CONV_OK;
+  }
+  if (a.cchunks == 0) return CONV_OK;  // other gather modes: maps unused
   const DriverFns& drv = driver_fns();
   if (!drv.tiled || !drv.im2col) return CONV_EDRIVER;
   const CUtensorMapDataType dt =
@@ -484,7 +621,8 @@ int encode_maps(const Problem& P, const TcArgs& a, bool pair, bool halo, const v
   // w viewed as [O, K] (K innermost)
   cuuint64_t wdim[2] = {static_cast<cuuint64_t>(P.K), static_cast<cuuint64_t>(P.O)};
   cuuint64_t wstr[1] = {static_cast<cuuint64_t>(P.K) * eb};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(a.kc), static_cast<cuuint32_t>(pair ? a.BN / 2 : a.BN)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(a.kc),
+                       static_cast<cuuint32_t>(w_rows > 0 ? w_rows : (pair ? a.BN / 2 : a.BN))};
   cuuint32_t west[2] = {1, 1};
   r = drv.tiled(&mw, dt, 2, const_cast<void*>(w), wdim, wstr, box, west, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -511,6 +649,15 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
   }
   CUtensorMap mx, mw;
   const bool halo = plan.variant == CONV_VARIANT_TC_HALO || plan.variant == CONV_VARIANT_TC_HALO_PAIR;
+  if (plan.variant == CONV_VARIANT_TC_TMA_T) {
+    CUtensorMap my;
+    rc = encode_maps(P, a, false, false, x, w, mx, mw, kTO);
+    if (rc == CONV_OK) rc = encode_y_map(P, y, my);
+    if (rc != CONV_OK) return rc;
+    if (P.dtype == CONV_BF16) conv_fwd_tc_t_kernel<true><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
+    else                      conv_fwd_tc_t_kernel<false><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
+    return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+  }
   rc = encode_maps(P, a, plan.pair, halo, x, w, mx, mw);
   if (rc != CONV_OK) return rc;
   const dim3 grid(plan.ctas), block(plan.variant == CONV_VARIANT_TC_TMA ? tc_threads<MODE_TMA>()
@@ -625,7 +772,7 @@ int conv_fwd_variant(const void* x, const void* w, void* y, int N, int D, int H,
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_PAIR) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_T) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -656,14 +803,16 @@ int conv_fwd_host(const void* x_host, const void* w_host, void* y_host, void* x_
   return CONV_OK;
 }
 
-int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
-              const int pad[3], const int dil[3], int groups, int dtype, int* bn, int* stages, int* ctas) {
+int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
+                      const int pad[3], const int dil[3], int groups, int dtype, int variant, int* bn,
+                      int* stages, int* ctas) {
   Problem P;
   int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
   if (rc != CONV_OK) return rc;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_T) return CONV_EINVAL;
   int dev, sms = 148;
   if (current_device(dev) == CONV_OK) device_sms(dev, sms);
-  const int variant = choose_variant(P, sms);
+  if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
   if (variant == CONV_VARIANT_SIMT) {
     if (bn) *bn = kSimtBN;
     if (stages) *stages = 1;
@@ -681,6 +830,12 @@ int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, 
   if (stages) *stages = plan.args.stages;
   if (ctas) *ctas = plan.ctas;
   return variant;
+}
+
+int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
+              const int pad[3], const int dil[3], int groups, int dtype, int* bn, int* stages, int* ctas) {
+  return conv_plan_variant(N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype, CONV_VARIANT_AUTO, bn,
+                           stages, ctas);
 }
 
 int conv_last_status(conv_stream_t stream) {

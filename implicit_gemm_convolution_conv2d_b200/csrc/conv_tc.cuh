@@ -83,7 +83,14 @@ struct TcArgs {
   uint32_t halo_slot_bytes;  // its shared-memory slot (1024-aligned)
   uint32_t halo_bytes;       // bytes one halo load delivers
   int a_slots;               // halo slots in the ring
-  int gather_mode;    // GATHER_SCALAR / GATHER_VEC8 / GATHER_SPAN
+  int gather_mode;    // GATHER_SCALAR / GATHER_VEC8 / GATHER_SPAN / GATHER_ROWS
+  // GATHER_ROWS: input rows of x (viewed as [N*H, W*C]) staged by TMA boxes of
+  // one TMA box of stage_rows whole input rows (row_e = W*C elements each,
+  // split as n_boxes x box_e so that every box dimension stays <= 256), which
+  // lands row after row, row_e elements apart; up to two image segments per tile
+  int box_e, n_boxes, stage_rows, row_e;
+  uint32_t seg_bytes;   // one segment: stage_rows * row_e * 2, rounded to 128
+  uint32_t rows_bytes;  // one buffer: 2 segments
   int Lp;             // span layout: filter-row length kW*C rounded up to 8
   int Kp;             // K as laid out in shared memory (>= K in span layout)
   long long x_elems;  // elements of x (bounds of the unaligned 16-byte loads)
@@ -106,6 +113,10 @@ struct __align__(8) TcSmemTail {
   uint64_t bres;      // resident weights loaded
   uint64_t afull[4];  // halo kernel: input halo slots
   uint64_t aempty[4];
+  uint64_t rfull[3];  // row staging (gather): rows of a tile landed
+  uint64_t rempty[3]; // row staging: every gather thread is done with the buffer
+  int seg_n[3][2];    // row staging, per buffer: image of segment 0 / 1
+  int seg_lo[3][2];   // first staged input row of segment 0 / 1
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -283,7 +294,7 @@ __device__ __forceinline__ uint4 load8_masked(const uint16_t* p, int e_lo, int e
 // multiple of 8), so a chunk never crosses a row; element j of row (kd, kh) is
 // x[n, id, ih, iw0, 0] + j and exists for j in [jlo, jhi).
 // GATHER_SCALAR: element-wise (kw, c) walk with its own bounds check.
-enum { GATHER_SCALAR = 0, GATHER_VEC8 = 1, GATHER_SPAN = 2 };
+enum { GATHER_SCALAR = 0, GATHER_VEC8 = 1, GATHER_SPAN = 2, GATHER_ROWS = 3 };
 
 __device__ __forceinline__ void gather_a_vec8(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
                                               int r, int chunk0) {
@@ -399,6 +410,54 @@ __device__ __forceinline__ void gather_a_span(const TcArgs& a, const GatherRow& 
   for (int q = 0; q < 4; ++q) store_chunk(a_tile, r, chunk0 + q, mask8(extract8(b0[q], b1[q], hsh[q]), msk[q]));
 }
 
+// GATHER_ROWS: the same span layout as gather_a_span, read from the input
+// rows staged in shared memory.  `rows` is the staging buffer of this tile,
+// seg_n / seg_lo its segments (image, first staged input row).
+__device__ __forceinline__ void gather_a_rows(const TcArgs& a, const GatherRow& st, int n, const uint8_t* rows,
+                                              const int* seg_n, const int* seg_lo, int k0, uint8_t* a_tile, int r,
+                                              int chunk0) {
+  const int span = k0 / a.Lp;
+  int j = k0 - span * a.Lp;
+  int kh = span % a.kH;
+  // the staged row holding filter row kh of this output pixel (or none)
+  const auto row_base = [&](int khh, bool& ok) -> const uint8_t* {
+    const int ih = st.ih0 + khh * a.dh;
+    const int seg = (n == seg_n[0]) ? 0 : 1;
+    const int lr = ih - seg_lo[seg];
+    ok = st.valid && khh < a.kH && static_cast<unsigned>(ih) < static_cast<unsigned>(a.H) &&
+         static_cast<unsigned>(lr) < static_cast<unsigned>(a.stage_rows);
+    return rows + seg * a.seg_bytes + static_cast<uint32_t>(lr) * static_cast<uint32_t>(a.row_e) * 2u;
+  };
+  bool rok;
+  const uint8_t* rb = row_base(kh, rok);
+  const int ebase = st.iw0 * a.C;  // element of x[n, ih, iw0, 0] within the row (may be negative)
+  uint4 v[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    v[q] = make_uint4(0, 0, 0, 0);
+    if (rok && j + 8 > st.jlo && j < st.jhi) {
+      const int lo = max(st.jlo - j, 0), hi = min(st.jhi - j, 8);
+      const int e0 = ebase + j;           // >= 0 whenever some element is valid
+      const int blk = e0 >> 3;            // aligned 8-element block holding e0 (floor, also for e0 < 0)
+      const unsigned h = static_cast<unsigned>(e0 - blk * 8);
+      // blocks blk and blk + 1; a block before the row start reads as zeros
+      uint4 b0 = make_uint4(0, 0, 0, 0), b1 = make_uint4(0, 0, 0, 0);
+      if (blk >= 0) b0 = *reinterpret_cast<const uint4*>(rb + blk * 16);
+      if (blk + 1 >= 0 && (blk + 1) * 8 < a.row_e) b1 = *reinterpret_cast<const uint4*>(rb + (blk + 1) * 16);
+      const unsigned m = ((1u << hi) - 1u) & ~((1u << lo) - 1u);
+      v[q] = mask8(extract8(b0, b1, h), m);
+    }
+    j += 8;
+    if (j == a.Lp) {
+      j = 0;
+      ++kh;
+      rb = row_base(kh, rok);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) store_chunk(a_tile, r, chunk0 + q, v[q]);
+}
+
 __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
                                                 int r, int chunk0) {
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
@@ -443,7 +502,8 @@ __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow
 __device__ __forceinline__ void gather_b_block(const TcArgs& a, int g, int n0, int kbase, uint8_t* b_tile,
                                                int tid, int nthreads) {
   const uint16_t* __restrict__ w = static_cast<const uint16_t*>(a.w);
-  const bool vec = (a.K & 7) == 0 && a.gather_mode != GATHER_SPAN;
+  const bool span_layout = a.gather_mode == GATHER_SPAN || a.gather_mode == GATHER_ROWS;
+  const bool vec = (a.K & 7) == 0 && !span_layout;
   const int L = a.kW * a.C;
 #pragma unroll 1
   for (int q = tid; q < a.BN * 8; q += nthreads) {
@@ -453,7 +513,7 @@ __device__ __forceinline__ void gather_b_block(const TcArgs& a, int g, int n0, i
     uint4 v = make_uint4(0, 0, 0, 0);
     if (oc < a.Og && kp0 < a.Kp) {
       const long long rowoff = static_cast<long long>(g * a.Og + oc) * a.K;
-      if (a.gather_mode == GATHER_SPAN) {
+      if (span_layout) {
         const int sp = kp0 / a.Lp;
         const int j0 = kp0 - sp * a.Lp;
         v = load8_masked(w + rowoff + static_cast<long long>(sp) * L + j0, 0, L - j0);
@@ -464,6 +524,48 @@ __device__ __forceinline__ void gather_b_block(const TcArgs& a, int g, int n0, i
       }
     }
     *reinterpret_cast<uint4*>(b_tile + sw128_offset(o, ch)) = v;
+  }
+}
+
+// GATHER_ROWS: stage the input rows one 128-row output tile reads.  The tile's
+// pixels lie in at most two images (host guarantees Ho*Wo >= 128); for each
+// image segment the contiguous range of input rows its filter rows touch is
+// loaded as one 3-D TMA box (box_e x n_boxes x stage_rows) from x viewed as
+// [N*H][row_e / box_e][box_e]
+// viewed as [N*H, W*C] (zero fill beyond the tensor).  Issued by one thread.
+__device__ __forceinline__ void issue_rows(const TcArgs& a, const CUtensorMap* tmap, TcSmemTail* tail, uint8_t* rowsbuf,
+                                           int tile, int b) {
+  const TileCoord tc = decode_tile(a, tile);
+  const long long m0 = static_cast<long long>(tc.mt) * kBM;
+  const long long m1 = min(m0 + kBM - 1, a.M - 1);
+  int n0, od, oh0, ow, n1, oh1;
+  decode_pixel(a, m0, n0, od, oh0, ow);
+  decode_pixel(a, m1, n1, od, oh1, ow);
+  const int segn[2] = {n0, n1 != n0 ? n1 : -1};
+  const int ohf[2] = {oh0, 0};
+  const int ohl[2] = {n1 != n0 ? a.Ho - 1 : oh1, oh1};
+  const uint32_t box_bytes = static_cast<uint32_t>(a.stage_rows) * static_cast<uint32_t>(a.row_e) * 2u;
+  int lo[2] = {0, 0};
+  bool load[2] = {false, false};
+  uint32_t bytes = 0;
+  for (int sg = 0; sg < 2; ++sg) {
+    if (segn[sg] < 0) continue;
+    const int ih_lo = max(0, ohf[sg] * a.sh - a.ph);
+    const int ih_hi = min(a.H - 1, ohl[sg] * a.sh - a.ph + (a.kH - 1) * a.dh);
+    lo[sg] = ih_lo;
+    load[sg] = ih_hi >= ih_lo;
+    if (load[sg]) bytes += box_bytes;
+  }
+  tail->seg_n[b][0] = segn[0];
+  tail->seg_n[b][1] = segn[1];
+  tail->seg_lo[b][0] = lo[0];
+  tail->seg_lo[b][1] = lo[1];
+  const uint32_t fb = ptx::smem_u32(&tail->rfull[b]);
+  ptx::mbar_arrive_expect_tx(fb, bytes);  // release: the segment table above is published with it
+  for (int sg = 0; sg < 2; ++sg) {
+    if (!load[sg]) continue;
+    ptx::tma_load_3d(ptx::smem_u32(rowsbuf + b * a.rows_bytes + sg * a.seg_bytes), tmap, fb, 0, 0,
+                     segn[sg] * a.H + lo[sg]);
   }
 }
 
@@ -481,7 +583,8 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* bres = smem + a.stages * a.stage_bytes;  // resident B (gather mode), 1024-aligned
-  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(bres + a.bres_bytes);
+  uint8_t* rowsbuf = bres + a.bres_bytes;            // staged input rows (GATHER_ROWS), 3 buffers
+  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(rowsbuf + 3 * a.rows_bytes);
   constexpr uint32_t kProdThreads = kProdWarps * 32;
 
   const int warp = threadIdx.x >> 5;
@@ -499,12 +602,16 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
     ptx::mbar_init(ptx::smem_u32(&tail->drain), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->bres), kProdThreads);
+    for (int b = 0; b < 3; ++b) {
+      ptx::mbar_init(ptx::smem_u32(&tail->rfull[b]), 1u);
+      ptx::mbar_init(ptx::smem_u32(&tail->rempty[b]), kProdThreads);
+    }
     tail->abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (MODE == MODE_TMA && threadIdx.x == 32) {
+  if (threadIdx.x == 32 && (MODE == MODE_TMA || a.gather_mode == GATHER_ROWS)) {
     ptx::prefetch_tmap(&tmap_x);
-    ptx::prefetch_tmap(&tmap_w);
+    if (MODE == MODE_TMA) ptx::prefetch_tmap(&tmap_w);
   }
   if (warp == kMmaWarp) {
     ptx::tmem_alloc(ptx::smem_u32(&tail->tmem_base), a.tmem_cols);
@@ -596,8 +703,17 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x) {
+      const bool rows_mode = a.gather_mode == GATHER_ROWS;
+      int lt = 0;  // local tile counter; row-staging buffer lt % 3, its use lt / 3
+      for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++lt) {
         const TileCoord tc = decode_tile(a, tile);
+        const int rb = lt % 3;
+        if (rows_mode &&
+            !wait_bounded(ptx::smem_u32(&tail->rfull[rb]), static_cast<uint32_t>((lt / 3) & 1), abort_flag,
+                          a.timeout_ns, kSiteProducerEmpty)) {
+          ok = false;
+          break;
+        }
         GatherRow st;
         const long long m = static_cast<long long>(tc.mt) * kBM + r;
         st.valid = m < a.M;
@@ -623,6 +739,9 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
             const int k0 = (kb + j) * 64 + half * 32;
             if (a.gather_mode == GATHER_VEC8)
               gather_a_vec8(a, st, k0, sa, r, half * 4);
+            else if (rows_mode)
+              gather_a_rows(a, st, n, rowsbuf + rb * a.rows_bytes, tail->seg_n[rb], tail->seg_lo[rb], k0, sa, r,
+                            half * 4);
             else if (a.gather_mode == GATHER_SPAN)
               gather_a_span(a, st, k0, sa, r, half * 4);
             else
@@ -636,10 +755,28 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
             phase ^= 1u;
           }
         }
+        // this thread is done reading the tile's staged rows
+        if (rows_mode && ok) ptx::mbar_arrive(ptx::smem_u32(&tail->rempty[rb]));
       }
       __syncwarp();
     }
   } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ row loader (GATHER_ROWS)
+    if (MODE == MODE_GATHER && a.gather_mode == GATHER_ROWS && lane == 1) {
+      int lt = 0;
+      for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++lt) {
+        const int rb = lt % 3, use = lt / 3;
+        if (use >= 1 && !wait_bounded(ptx::smem_u32(&tail->rempty[rb]), static_cast<uint32_t>((use - 1) & 1),
+                                      abort_flag, a.timeout_ns, kSiteProducerEmpty))
+          break;
+        issue_rows(a, &tmap_x, tail, rowsbuf, tile, rb);
+      }
+      // before the CTA can exit, every row load issued must have landed
+      for (int b = 0; b < 3 && b < lt; ++b) {
+        const int last_use = (lt - 1 - b) / 3;  // uses of buffer b: tiles b, b+3, ... < lt
+        wait_drain(ptx::smem_u32(&tail->rfull[b]), static_cast<uint32_t>(last_use & 1), a.timeout_ns);
+      }
+    }
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int stage = 0;

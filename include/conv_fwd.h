@@ -77,7 +77,10 @@ enum {
   CONV_VARIANT_TC_TMA_PAIR = 3, /* TC_TMA with CTA pairs: 256-row tiles, cta_group::2 */
   CONV_VARIANT_TC_HALO = 4,     /* tcgen05, one TMA box of input halo per 16x8 output block
                                    reused by every filter tap (stride 1, C/G % 64 == 0) */
-  CONV_VARIANT_TC_HALO_PAIR = 5 /* TC_HALO with CTA pairs (32x8 blocks, cta_group::2) */
+  CONV_VARIANT_TC_HALO_PAIR = 5, /* TC_HALO with CTA pairs (32x8 blocks, cta_group::2) */
+  CONV_VARIANT_TC_TMA_T = 6      /* TC_TMA in the transposed orientation: MMA M = 128
+                                   output channels, N = 256 output pixels, TMA-store
+                                   epilogue (C/G % 16 == 0, O/G % 128 == 0) */
 };
 
 /* Output extents.  stride/pad/dil: 3 ints (d, h, w).  out: 3 ints (Do, Ho, Wo).
@@ -90,10 +93,12 @@ int conv_out_dims(int D, int H, int W, int kD, int kH, int kW,
 /* Forward convolution on device buffers x, w, y (see the layouts above).
  * Queues the kernel on `stream`; returns CONV_OK or an error code (nothing is
  * queued on an error).  The variant is chosen from the type and shape:
- * f32 -> SIMT; f16/bf16 -> TC_TMA_PAIR (or TC_TMA when there are fewer
- * 256-row output tiles than SM pairs) when C/G % 16 == 0 and the geometry fits
- * a TMA im2col tensor map; otherwise TC_GATHER.  TC_HALO and TC_HALO_PAIR run
- * only when requested through conv_fwd_variant. */
+ * f32 -> SIMT; f16/bf16 with C/G % 16 == 0 and a geometry that fits a TMA
+ * im2col tensor map -> TC_TMA_T when O/G is an odd multiple of 128 and there
+ * are at least as many 256-pixel tiles as SMs, else TC_TMA_PAIR (or TC_TMA
+ * when there are fewer 256-row output tiles than SM pairs); otherwise
+ * TC_GATHER.  TC_HALO and TC_HALO_PAIR run only when requested through
+ * conv_fwd_variant. */
 int conv_fwd(const void* x, const void* w, void* y,
              int N, int D, int H, int W, int C, int O,
              int kD, int kH, int kW,
@@ -102,9 +107,10 @@ int conv_fwd(const void* x, const void* w, void* y,
 
 /* conv_fwd with an explicit kernel variant (CONV_VARIANT_*).  Returns
  * CONV_EUNSUPPORTED when that variant cannot run the shape or type
- * (the tensor-core variants need f16/bf16; TC_TMA and TC_TMA_PAIR need
- * C/G % 16 == 0 and a geometry inside the TMA im2col limits; TC_HALO and
- * TC_HALO_PAIR need stride 1 and C/G % 64 == 0). */
+ * (the tensor-core variants need f16/bf16; TC_TMA, TC_TMA_PAIR and TC_TMA_T
+ * need C/G % 16 == 0 and a geometry inside the TMA im2col limits, TC_TMA_T
+ * also O/G % 128 == 0; TC_HALO and TC_HALO_PAIR need stride 1 and
+ * C/G % 64 == 0). */
 int conv_fwd_variant(const void* x, const void* w, void* y,
                      int N, int D, int H, int W, int C, int O,
                      int kD, int kH, int kW,
@@ -131,6 +137,14 @@ int conv_fwd_host(const void* x_host, const void* w_host, void* y_host,
 int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
               const int stride[3], const int pad[3], const int dil[3],
               int groups, int dtype, int* bn, int* stages, int* ctas);
+
+/* conv_plan for an explicit variant (CONV_VARIANT_*; AUTO behaves as
+ * conv_plan).  Returns that variant, CONV_EUNSUPPORTED when it cannot run the
+ * shape or type (the same rule as conv_fwd_variant), or another negative
+ * error code.  Queues nothing. */
+int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
+                      const int stride[3], const int pad[3], const int dil[3],
+                      int groups, int dtype, int variant, int* bn, int* stages, int* ctas);
 
 /* Waits for `stream`, then reads and clears the current device's status word.
  * Returns CONV_OK, or CONV_ETIMEOUT if a kernel since the last call gave up on

@@ -58,6 +58,8 @@ def variants_for(wl):
         vs += [C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR]
     if (wl.C // wl.groups) % 64 == 0 and tuple(wl.stride) == (1, 1, 1) and wl.k[1] * wl.k[2] >= 4:
         vs += [C.VARIANT_TC_HALO, C.VARIANT_TC_HALO_PAIR]
+    if (wl.C // wl.groups) % 16 == 0 and (wl.O // wl.groups) % 128 == 0:
+        vs.append(C.VARIANT_TC_TMA_T)
     return vs
 
 
@@ -90,11 +92,22 @@ SMALL = [
     WL.case(2, 1, 8, 8, 6, 4, (1, 3, 3), pad=(0, 1, 1), groups=2, name="groups2_cg3_scalar"),
     WL.case(3, 1, 7, 9, 24, 40, (1, 3, 3), pad=(0, 1, 1), name="c24_vec8"),
     WL.case(1, 2, 9, 200, 3, 16, (1, 1, 7), (1, 1, 3), (0, 0, 3), name="wide_row_span"),
+    # row staging: 2-D, unaligned C, W*C % 8 == 0, tiles crossing image borders, rows over 256 elements
+    WL.case(3, 1, 37, 40, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), name="rows_stem_like"),
+    WL.case(2, 1, 21, 96, 5, 24, (1, 3, 5), (1, 1, 1), (0, 1, 2), name="rows_c5_wide"),
+    WL.case(4, 1, 17, 16, 3, 8, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 2, 1), name="rows_dil_h"),
     WL.case(2, 1, 20, 19, 128, 96, (1, 3, 3), pad=(0, 1, 1), name="halo_c128_o96"),
     WL.case(1, 3, 9, 13, 64, 64, (3, 3, 3), pad=(1, 1, 1), dil=(1, 2, 1), name="halo_3d_dil"),
     WL.case(2, 1, 17, 9, 128, 128, (1, 3, 3), pad=(0, 2, 2), dil=(1, 2, 2), groups=2, name="halo_groups2_dil2"),
     WL.case(1, 1, 12, 12, 64, 320, (1, 3, 3), pad=(0, 1, 1), name="halo_o320"),
     WL.case(3, 1, 33, 17, 64, 32, (1, 5, 5), pad=(0, 2, 2), name="halo_k5_ragged"),
+    # transposed orientation (128 output channels per tile): ragged pixel
+    # tail, groups with 32-channel chunks, 3-D with 16-channel chunks, two
+    # channel tiles at stride 2
+    WL.case(2, 1, 13, 11, 64, 128, (1, 3, 3), pad=(0, 1, 1), name="t_o128_ragged"),
+    WL.case(2, 1, 10, 10, 64, 256, (1, 3, 3), pad=(0, 1, 1), groups=2, name="t_groups2_cg32"),
+    WL.case(1, 6, 7, 9, 16, 128, (3, 3, 3), pad=(1, 1, 1), name="t_3d_c16"),
+    WL.case(1, 1, 17, 19, 64, 256, (1, 3, 3), (1, 2, 2), (0, 1, 1), name="t_s2_o256"),
 ]
 
 
@@ -107,6 +120,21 @@ def test_small_sweep(wl, dtype):
     for v in variants_for(wl):
         y = run_gpu(x, w, wl, v)
         assert_parity(y, y_ref, s_ref, dtype, f"{wl.name}/{dtype}/{C.VARIANT_NAMES[v]}")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_transposed_wide_pixel_tiles(dtype):
+    """Enough output pixels for 256-pixel tiles on every SM (the 128-pixel
+    tiles are covered by the small sweep): two images, ragged last tile,
+    every element against the oracle."""
+    wl = WL.case(4, 1, 100, 97, 16, 128, (1, 3, 3), pad=(0, 1, 1), dtype=dtype, seed=77)
+    v, bp, _, _ = C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil, wl.groups,
+                         dtype, C.VARIANT_TC_TMA_T)
+    assert v == C.VARIANT_TC_TMA_T and bp == 256
+    x, w = WL.make_inputs(wl)
+    y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups)
+    y = run_gpu(x, w, wl, C.VARIANT_TC_TMA_T)
+    assert_parity(y, y_ref, s_ref, dtype, "transposed/256-pixel tiles")
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
