@@ -16,6 +16,7 @@
 #include "conv_simt.cuh"
 #include "conv_tc.cuh"
 #include "conv_tct.cuh"
+#include "conv_halo_t.cuh"
 
 namespace convfwd {
 namespace {
@@ -156,6 +157,8 @@ int set_kernel_attrs(int dev) {
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_t_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_t_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return CONV_ELAUNCH;
   g_dev[dev].attrs_set = true;
   return CONV_OK;
@@ -392,7 +395,76 @@ int plan_tc_t(const Problem& P, int sms, TcPlan& plan) {
   return CONV_OK;
 }
 
+// Transposed orientation with halo reuse: M = 128 output channels, N = a
+// 32 x 8 block of output pixels read as views of one 8-pixel-wide input strip
+// per (64-channel chunk, kd, kw).  Stride 1, C/G % 64 == 0, O/G % 128 == 0.
+int plan_halo_t(const Problem& P, int sms, TcPlan& plan) {
+  if (P.dtype == CONV_F32 || P.Cg % 64 != 0 || P.Og % kTO != 0) return CONV_EUNSUPPORTED;
+  if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1) return CONV_EUNSUPPORTED;
+  if (P.N > 0x3fffffff) return CONV_EUNSUPPORTED;
+  const bool rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
+  const long long hw = kHTBlockW;  // one strip per width tap
+  const long long hh = kHTBlockH + static_cast<long long>(P.d[1]) * (P.kH - 1);
+  if (hh > 256) return CONV_EUNSUPPORTED;
+  TcArgs& a = plan.args;
+  std::memset(&a, 0, sizeof(a));
+  a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.C = P.C; a.O = P.O;
+  a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
+  a.sd = P.s[0]; a.sh = P.s[1]; a.sw = P.s[2];
+  a.pd = P.p[0]; a.ph = P.p[1]; a.pw = P.p[2];
+  a.dd = P.d[0]; a.dh = P.d[1]; a.dw = P.d[2];
+  a.G = P.G; a.Cg = P.Cg; a.Og = P.Og;
+  a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
+  a.M = P.M;
+  a.K = static_cast<int>(P.K);
+  a.BN = kHTBlockH * kHTBlockW;  // MMA N: output pixels per tile
+  a.n_tiles = P.Og / kTO;
+  a.tile_h = kHTBlockH;
+  a.tile_w = kHTBlockW;
+  a.tiles_h = (P.Ho + kHTBlockH - 1) / kHTBlockH;
+  a.tiles_w = (P.Wo + kHTBlockW - 1) / kHTBlockW;
+  const long long tt = static_cast<long long>(P.G) * P.N * P.Do * a.tiles_h * a.tiles_w * a.n_tiles;
+  if (tt > 0x7fffffffLL) return CONV_EINVAL;
+  a.total_tiles = static_cast<int>(tt);
+  a.m_tiles = 0;
+  a.halo_w = static_cast<int>(hw);
+  a.halo_h = static_cast<int>(hh);
+  a.halo_bytes = static_cast<uint32_t>(hw * hh * 128);
+  a.halo_slot_bytes = (a.halo_bytes + 1023u) & ~1023u;
+  a.a_slots = 2;
+  a.kc = 64;
+  a.cchunks = P.Cg / 64;
+  a.kblocks = P.kD * P.kH * P.kW * a.cchunks;
+  a.rank5 = rank5 ? 1 : 0;
+  a.layout_type = 2u;
+  a.sbo = 1024u;
+  a.a_bytes = 0;
+  a.b_bytes = static_cast<uint32_t>(kTO * 128);  // one weight tile: 128 channels x 64 K
+  a.sub_bytes = a.b_bytes;
+  const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
+                          64 - 2LL * kTEpiBytes - static_cast<long long>(a.a_slots) * a.halo_slot_bytes;
+  if (avail <= 0) return CONV_EUNSUPPORTED;
+  int stages = 0;
+  // a stage may span at most two (chunk, kd, kw) strip groups: kbs <= kH
+  a.kbs = choose_kbs(a.BN, 64, a.b_bytes, avail, std::min(8, P.kH), stages);
+  if (stages < 2) return CONV_EUNSUPPORTED;
+  a.stages = stages;
+  a.stage_bytes = static_cast<uint32_t>(a.kbs) * a.b_bytes;
+  const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
+  a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(a.BN >> 3) << 17) |
+            ((static_cast<uint32_t>(kTO) >> 4) << 24);
+  a.tmem_cols = next_pow2_cols(static_cast<uint32_t>(2 * a.BN));
+  a.timeout_ns = kWaitTimeoutNs;
+  plan.variant = CONV_VARIANT_TC_HALO_T;
+  plan.pair = false;
+  plan.ctas = std::min(a.total_tiles, sms);
+  plan.smem = static_cast<size_t>(a.a_slots) * a.halo_slot_bytes + static_cast<size_t>(a.stages) * a.stage_bytes +
+              2 * static_cast<size_t>(kTEpiBytes) + 1024 + sizeof(TcSmemTail) + 64;
+  return CONV_OK;
+}
+
 int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
+  if (variant == CONV_VARIANT_TC_HALO_T) return plan_halo_t(P, sms, plan);
   if (variant == CONV_VARIANT_TC_HALO || variant == CONV_VARIANT_TC_HALO_PAIR)
     return plan_halo(P, variant == CONV_VARIANT_TC_HALO_PAIR, sms, plan);
   if (variant == CONV_VARIANT_TC_TMA_T) return plan_tc_t(P, sms, plan);
@@ -552,6 +624,29 @@ int encode_y_map(const Problem& P, void* y, CUtensorMap& my) {
   return CONV_OK;
 }
 
+// y viewed as [N, (Do,) Ho, Wo, O] for the transposed halo kernel's TMA
+// stores: boxes of 128 channels x 8 columns x 4 rows, clipped at the edges.
+int encode_y_block_map(const Problem& P, bool rank5, void* y, CUtensorMap& my) {
+  std::memset(&my, 0, sizeof(my));
+  const DriverFns& drv = driver_fns();
+  if (!drv.tiled) return CONV_EDRIVER;
+  const CUtensorMapDataType dt =
+      P.dtype == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t eb = 2;
+  cuuint64_t dim[5] = {static_cast<cuuint64_t>(P.O), static_cast<cuuint64_t>(P.Wo), static_cast<cuuint64_t>(P.Ho),
+                       static_cast<cuuint64_t>(rank5 ? P.Do : P.N), static_cast<cuuint64_t>(P.N)};
+  cuuint64_t str[4] = {eb * P.O, eb * P.O * P.Wo, eb * P.O * P.Wo * P.Ho, eb * P.O * P.Wo * P.Ho * P.Do};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(kTO), static_cast<cuuint32_t>(kHTBlockW),
+                       static_cast<cuuint32_t>(kTEpiRows / kHTBlockW), 1u, 1u};
+  cuuint32_t est[5] = {1, 1, 1, 1, 1};
+  const CUresult r = drv.tiled(&my, dt, rank5 ? 5 : 4, y, dim, str, box, est, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  small_tensor_fixup(my, static_cast<size_t>(P.M) * P.O * 2, drv.driver_version);
+  return CONV_OK;
+}
+
 int encode_maps(const Problem& P, const TcArgs& a, bool pair, bool halo, const void* x, const void* w,
                 CUtensorMap& mx, CUtensorMap& mw, int w_rows = 0) {
   std::memset(&mx, 0, sizeof(mx));
@@ -649,6 +744,15 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
   }
   CUtensorMap mx, mw;
   const bool halo = plan.variant == CONV_VARIANT_TC_HALO || plan.variant == CONV_VARIANT_TC_HALO_PAIR;
+  if (plan.variant == CONV_VARIANT_TC_HALO_T) {
+    CUtensorMap my;
+    rc = encode_maps(P, a, false, true, x, w, mx, mw, kTO);
+    if (rc == CONV_OK) rc = encode_y_block_map(P, a.rank5 != 0, y, my);
+    if (rc != CONV_OK) return rc;
+    if (P.dtype == CONV_BF16) conv_fwd_tc_halo_t_kernel<true><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
+    else                      conv_fwd_tc_halo_t_kernel<false><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
+    return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+  }
   if (plan.variant == CONV_VARIANT_TC_TMA_T) {
     CUtensorMap my;
     rc = encode_maps(P, a, false, false, x, w, mx, mw, kTO);
@@ -772,7 +876,7 @@ int conv_fwd_variant(const void* x, const void* w, void* y, int N, int D, int H,
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_T) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_T) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -809,7 +913,7 @@ int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, 
   Problem P;
   int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_T) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_T) return CONV_EINVAL;
   int dev, sms = 148;
   if (current_device(dev) == CONV_OK) device_sms(dev, sms);
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);

@@ -78,9 +78,13 @@ enum {
   CONV_VARIANT_TC_HALO = 4,     /* tcgen05, one TMA box of input halo per 16x8 output block
                                    reused by every filter tap (stride 1, C/G % 64 == 0) */
   CONV_VARIANT_TC_HALO_PAIR = 5, /* TC_HALO with CTA pairs (32x8 blocks, cta_group::2) */
-  CONV_VARIANT_TC_TMA_T = 6      /* TC_TMA in the transposed orientation: MMA M = 128
+  CONV_VARIANT_TC_TMA_T = 6,     /* TC_TMA in the transposed orientation: MMA M = 128
                                    output channels, N = 256 output pixels, TMA-store
                                    epilogue (C/G % 16 == 0, O/G % 128 == 0) */
+  CONV_VARIANT_TC_HALO_T = 7     /* transposed orientation with halo reuse: N = a 32x8
+                                   output block read from one input halo box per
+                                   (64-channel chunk, kd) (stride 1, C/G % 64 == 0,
+                                   O/G % 128 == 0) */
 };
 
 /* Output extents.  stride/pad/dil: 3 ints (d, h, w).  out: 3 ints (Do, Ho, Wo).

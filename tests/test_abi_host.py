@@ -98,7 +98,7 @@ def test_invalid_arguments_rejected_on_host(C):
     big = 1 << 30
     assert call(X, Wt, Y, big, big, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
     # unknown variant
-    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 7, None) == -1
+    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 8, None) == -1
     assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, -2, None) == -1
 
 
@@ -154,5 +154,5 @@ def test_explicit_variant_plan(C):
         C.plan(*g3, "f32", C.VARIANT_TC_TMA)
     assert e.value.code == -7
     with pytest.raises(C.ConvError) as e:
-        C.plan(*g3, "bf16", 9)
+        C.plan(*g3, "bf16", 8)
     assert e.value.code == -1

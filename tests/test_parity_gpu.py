@@ -60,6 +60,8 @@ def variants_for(wl):
         vs += [C.VARIANT_TC_HALO, C.VARIANT_TC_HALO_PAIR]
     if (wl.C // wl.groups) % 16 == 0 and (wl.O // wl.groups) % 128 == 0:
         vs.append(C.VARIANT_TC_TMA_T)
+    if (wl.C // wl.groups) % 64 == 0 and (wl.O // wl.groups) % 128 == 0 and tuple(wl.stride) == (1, 1, 1):
+        vs.append(C.VARIANT_TC_HALO_T)
     return vs
 
 
@@ -108,6 +110,12 @@ SMALL = [
     WL.case(2, 1, 10, 10, 64, 256, (1, 3, 3), pad=(0, 1, 1), groups=2, name="t_groups2_cg32"),
     WL.case(1, 6, 7, 9, 16, 128, (3, 3, 3), pad=(1, 1, 1), name="t_3d_c16"),
     WL.case(1, 1, 17, 19, 64, 256, (1, 3, 3), (1, 2, 2), (0, 1, 1), name="t_s2_o256"),
+    # transposed halo: blocks cut by the image edge in h and w, dilation,
+    # 3-D with kd taps, two channel chunks and two channel tiles, groups
+    WL.case(2, 1, 37, 13, 64, 128, (1, 3, 3), pad=(0, 1, 1), name="ht_edges"),
+    WL.case(1, 3, 19, 11, 64, 128, (3, 3, 3), pad=(1, 2, 1), dil=(1, 2, 1), name="ht_3d_dil"),
+    WL.case(1, 1, 33, 17, 128, 256, (1, 5, 5), pad=(0, 2, 2), name="ht_c128_o256_k5"),
+    WL.case(2, 1, 9, 9, 128, 256, (1, 3, 3), pad=(0, 1, 1), groups=2, name="ht_groups2"),
 ]
 
 
