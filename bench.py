@@ -408,6 +408,7 @@ def bench_ours(args):
                    "variant": vname,
                    "tile": ([64, 64] if variant == C.VARIANT_SIMT else
                             [bn, 128] if variant in (C.VARIANT_TC_TMA_T, C.VARIANT_TC_HALO_T)
+                            else [bn, 256] if variant == C.VARIANT_TC_HALO_T_PAIR
                             else [256 if "pair" in vname else 128, bn]),
                    "stages": stages, "ctas": ctas,
                    "l2": f"inputs rotate over {nsets} buffer sets ({nsets * per_set / 2**20:.0f} MiB > 2x L2)"},
@@ -497,7 +498,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     ap.add_argument("--variant", default="AUTO",
-                    choices=["AUTO", "SIMT", "TC_TMA", "TC_GATHER", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T", "TC_HALO_T"],
+                    choices=["AUTO", "SIMT", "TC_TMA", "TC_GATHER", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T", "TC_HALO_T",
+                             "TC_HALO_T_PAIR"],
                     help="kernel variant (default: the library's own choice)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)

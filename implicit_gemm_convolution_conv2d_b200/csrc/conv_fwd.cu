@@ -157,8 +157,10 @@ int set_kernel_attrs(int dev) {
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_t_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_t_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return CONV_ELAUNCH;
   g_dev[dev].attrs_set = true;
   return CONV_OK;
@@ -396,15 +398,31 @@ int plan_tc_t(const Problem& P, int sms, TcPlan& plan) {
 }
 
 // Transposed orientation with halo reuse: M = 128 output channels, N = a
-// 32 x 8 block of output pixels read as views of one 8-pixel-wide input strip
-// per (64-channel chunk, kd, kw).  Stride 1, C/G % 64 == 0, O/G % 128 == 0.
-int plan_halo_t(const Problem& P, int sms, TcPlan& plan) {
-  if (P.dtype == CONV_F32 || P.Cg % 64 != 0 || P.Og % kTO != 0) return CONV_EUNSUPPORTED;
+// tile_h x 8 block of output pixels read as views of one 8-pixel-wide input
+// strip per (64-channel chunk, kd, kw).  Stride 1, C/G % 64 == 0,
+// O/G % 128 == 0.  With `pair`, two CTAs issue M = 256 (128 output channels
+// each) over the same block; each loads the strip of half the block's rows.
+int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
+  const int o_tile = pair ? 2 * kTO : kTO;
+  if (P.dtype == CONV_F32 || P.Cg % 64 != 0 || P.Og % o_tile != 0) return CONV_EUNSUPPORTED;
   if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1) return CONV_EUNSUPPORTED;
   if (P.N > 0x3fffffff) return CONV_EUNSUPPORTED;
   const bool rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
+  // block height: the multiple of 4 up to 32 that wastes the fewest rows of
+  // Ho (ties to the taller block, which reuses the strip over more rows)
+  int bh = kHTBlockHMax;
+  {
+    long long best = -1;
+    for (int h = kHTBlockHMax; h >= 16; h -= 4) {
+      const long long covered = static_cast<long long>((P.Ho + h - 1) / h) * h;
+      if (best < 0 || covered < best) {
+        best = covered;
+        bh = h;
+      }
+    }
+  }
   const long long hw = kHTBlockW;  // one strip per width tap
-  const long long hh = kHTBlockH + static_cast<long long>(P.d[1]) * (P.kH - 1);
+  const long long hh = (pair ? bh / 2 : bh) + static_cast<long long>(P.d[1]) * (P.kH - 1);  // rows per CTA
   if (hh > 256) return CONV_EUNSUPPORTED;
   TcArgs& a = plan.args;
   std::memset(&a, 0, sizeof(a));
@@ -417,11 +435,11 @@ int plan_halo_t(const Problem& P, int sms, TcPlan& plan) {
   a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
   a.M = P.M;
   a.K = static_cast<int>(P.K);
-  a.BN = kHTBlockH * kHTBlockW;  // MMA N: output pixels per tile
-  a.n_tiles = P.Og / kTO;
-  a.tile_h = kHTBlockH;
+  a.BN = bh * kHTBlockW;  // MMA N: output pixels per tile
+  a.n_tiles = P.Og / o_tile;
+  a.tile_h = bh;
   a.tile_w = kHTBlockW;
-  a.tiles_h = (P.Ho + kHTBlockH - 1) / kHTBlockH;
+  a.tiles_h = (P.Ho + bh - 1) / bh;
   a.tiles_w = (P.Wo + kHTBlockW - 1) / kHTBlockW;
   const long long tt = static_cast<long long>(P.G) * P.N * P.Do * a.tiles_h * a.tiles_w * a.n_tiles;
   if (tt > 0x7fffffffLL) return CONV_EINVAL;
@@ -441,30 +459,36 @@ int plan_halo_t(const Problem& P, int sms, TcPlan& plan) {
   a.a_bytes = 0;
   a.b_bytes = static_cast<uint32_t>(kTO * 128);  // one weight tile: 128 channels x 64 K
   a.sub_bytes = a.b_bytes;
-  const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
-                          64 - 2LL * kTEpiBytes - static_cast<long long>(a.a_slots) * a.halo_slot_bytes;
-  if (avail <= 0) return CONV_EUNSUPPORTED;
+  // strip slots: three when three weight stages still fit beside them (the
+  // strip producer then runs two groups ahead), else two
   int stages = 0;
-  // a stage may span at most two (chunk, kd, kw) strip groups: kbs <= kH
-  a.kbs = choose_kbs(a.BN, 64, a.b_bytes, avail, std::min(8, P.kH), stages);
+  for (int slots = 3; slots >= 2; --slots) {
+    const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
+                            64 - 2LL * kTEpiBytes - static_cast<long long>(slots) * a.halo_slot_bytes;
+    if (avail <= 0) continue;
+    a.a_slots = slots;
+    a.kbs = choose_kbs(a.BN, 64, a.b_bytes, avail, std::min(8, P.kH), stages);
+    if (stages >= 3 || slots == 2) break;
+  }
   if (stages < 2) return CONV_EUNSUPPORTED;
   a.stages = stages;
   a.stage_bytes = static_cast<uint32_t>(a.kbs) * a.b_bytes;
   const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
   a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(a.BN >> 3) << 17) |
-            ((static_cast<uint32_t>(kTO) >> 4) << 24);
-  a.tmem_cols = next_pow2_cols(static_cast<uint32_t>(2 * a.BN));
+            ((static_cast<uint32_t>(o_tile) >> 4) << 24);
+  a.tmem_cols = 2 * kHTAccStride;
   a.timeout_ns = kWaitTimeoutNs;
-  plan.variant = CONV_VARIANT_TC_HALO_T;
-  plan.pair = false;
-  plan.ctas = std::min(a.total_tiles, sms);
+  plan.variant = pair ? CONV_VARIANT_TC_HALO_T_PAIR : CONV_VARIANT_TC_HALO_T;
+  plan.pair = pair;
+  plan.ctas = pair ? 2 * std::min(a.total_tiles, sms / 2) : std::min(a.total_tiles, sms);
   plan.smem = static_cast<size_t>(a.a_slots) * a.halo_slot_bytes + static_cast<size_t>(a.stages) * a.stage_bytes +
               2 * static_cast<size_t>(kTEpiBytes) + 1024 + sizeof(TcSmemTail) + 64;
   return CONV_OK;
 }
 
 int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
-  if (variant == CONV_VARIANT_TC_HALO_T) return plan_halo_t(P, sms, plan);
+  if (variant == CONV_VARIANT_TC_HALO_T || variant == CONV_VARIANT_TC_HALO_T_PAIR)
+    return plan_halo_t(P, variant == CONV_VARIANT_TC_HALO_T_PAIR, sms, plan);
   if (variant == CONV_VARIANT_TC_HALO || variant == CONV_VARIANT_TC_HALO_PAIR)
     return plan_halo(P, variant == CONV_VARIANT_TC_HALO_PAIR, sms, plan);
   if (variant == CONV_VARIANT_TC_TMA_T) return plan_tc_t(P, sms, plan);
@@ -583,17 +607,23 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
 }
 
 // f32 -> SIMT.  f16/bf16 -> TMA im2col when it can describe the problem,
-// else the in-kernel gather.  Among the im2col kernels: the transposed
-// orientation when the output channels per group come in 128-wide tiles that
-// a 256-wide one cannot cover (O/G = 128, 384, ...) and there are enough
-// 256-pixel tiles for every SM; otherwise CTA pairs once there are at least
-// as many 256-row tiles as SM pairs; otherwise single CTAs.  The halo kernels
-// are explicit-only: on B200 they measure slower than im2col at every shape
-// of the workload set.
+// else the in-kernel gather.  When the output channels per group come in
+// 128-wide tiles that a 256-wide one cannot cover (O/G = 128, 384, ...): the
+// transposed halo kernel at stride 1 with 64-channel chunks and kH >= 2 (each
+// input strip then serves kH taps) and a tile for every SM, else the
+// transposed im2col kernel when there are enough 256-pixel tiles for every
+// SM.  Otherwise CTA pairs once there are at least as many 256-row tiles as
+// SM pairs, else single CTAs.  Every choice here is the fastest measured on
+// B200 for the shapes of the workload set; TC_HALO, TC_HALO_PAIR and
+// TC_HALO_T_PAIR stay explicit (slower there than the choice made here).
 int choose_variant(const Problem& P, int sms) {
   if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
   bool r5;
   if (!tma_fits(P, r5)) return CONV_VARIANT_TC_GATHER;
+  if (P.Og % kTO == 0 && P.Og % 256 != 0 && P.kH >= 2) {
+    TcPlan hp;
+    if (plan_halo_t(P, false, sms, hp) == CONV_OK && hp.args.total_tiles >= sms) return CONV_VARIANT_TC_HALO_T;
+  }
   if (P.Og % kTO == 0 && P.Og % 256 != 0 && P.M <= 0x7fffffffLL - 256 &&
       (P.M + 255) / 256 * (P.Og / kTO) * P.G >= sms)
     return CONV_VARIANT_TC_TMA_T;
@@ -744,14 +774,38 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
   }
   CUtensorMap mx, mw;
   const bool halo = plan.variant == CONV_VARIANT_TC_HALO || plan.variant == CONV_VARIANT_TC_HALO_PAIR;
-  if (plan.variant == CONV_VARIANT_TC_HALO_T) {
+  if (plan.variant == CONV_VARIANT_TC_HALO_T || plan.variant == CONV_VARIANT_TC_HALO_T_PAIR) {
     CUtensorMap my;
     rc = encode_maps(P, a, false, true, x, w, mx, mw, kTO);
     if (rc == CONV_OK) rc = encode_y_block_map(P, a.rank5 != 0, y, my);
     if (rc != CONV_OK) return rc;
-    if (P.dtype == CONV_BF16) conv_fwd_tc_halo_t_kernel<true><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
-    else                      conv_fwd_tc_halo_t_kernel<false><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
-    return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+    const bool bf = P.dtype == CONV_BF16;
+    if (!plan.pair) {
+      if (bf) conv_fwd_tc_halo_t_kernel<true, false><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
+      else    conv_fwd_tc_halo_t_kernel<false, false><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
+      return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(plan.ctas);
+    cfg.blockDim = dim3(kTThreads);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // never launch more pairs than can be resident together
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, conv_fwd_tc_halo_t_kernel<false, true>, &cfg) != cudaSuccess ||
+        clusters <= 0)
+      return CONV_ELAUNCH;
+    cfg.gridDim = dim3(2 * std::min(plan.ctas / 2, clusters));
+    const cudaError_t e = bf ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_halo_t_kernel<true, true>, mx, mw, my, a)
+                             : cudaLaunchKernelEx(&cfg, conv_fwd_tc_halo_t_kernel<false, true>, mx, mw, my, a);
+    return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
   }
   if (plan.variant == CONV_VARIANT_TC_TMA_T) {
     CUtensorMap my;
@@ -876,7 +930,7 @@ int conv_fwd_variant(const void* x, const void* w, void* y, int N, int D, int H,
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_T) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_T_PAIR) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -913,7 +967,7 @@ int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, 
   Problem P;
   int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_T) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_T_PAIR) return CONV_EINVAL;
   int dev, sms = 148;
   if (current_device(dev) == CONV_OK) device_sms(dev, sms);
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);

@@ -195,6 +195,11 @@ __global__ void __launch_bounds__(192, 1)
       if (a.inject_stall)
         ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
       const uint32_t sbo = static_cast<uint32_t>(a.halo_w) * 128u;
+      // descriptors built once; moved by constant offsets below
+      const uint64_t d_halo = ptx::smem_desc_sw128_view(ptx::smem_u32(halo), sbo, 0);
+      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, 2);
+      const uint64_t sub_off = desc_off(a.b_bytes), st_off = desc_off(a.stage_bytes);
+      const uint64_t slot_off = desc_off(a.halo_slot_bytes);
       for (int tile = unit; ok && tile < a.total_tiles; tile += nunits, ++t) {
         const int acc = t & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -206,7 +211,8 @@ __global__ void __launch_bounds__(192, 1)
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
         uint32_t accumulate = 0;
-        uint32_t hbase = 0;
+        uint64_t d_box = 0;
+        int kh = 0, kw = 0;  // tap of the next K block (taps run kw-fastest)
         for (int q0 = 0; ok && q0 < Q; q0 += a.kbs) {
           const int nsub = min(a.kbs, Q - q0);
           if (!wait_bounded(ptx::smem_u32(&tail->full[bst]), bph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
@@ -214,29 +220,27 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           ptx::tc_fence_after();
+          uint64_t db = d_ring + static_cast<uint64_t>(bst) * st_off;
           for (int j = 0; j < nsub; ++j) {
-            const int q = q0 + j;
-            const int tp = q % taps_hw;
-            if (tp == 0) {
+            if (kh == 0 && kw == 0) {
               if (!wait_bounded(ptx::smem_u32(&tail->afull[ast]), aph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
                 ok = false;
                 break;
               }
               ptx::tc_fence_after();
-              hbase = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
+              d_box = d_halo + static_cast<uint64_t>(ast) * slot_off;
             }
-            const int kh = tp / a.kW, kw = tp - (tp / a.kW) * a.kW;
-            const uint32_t view = hbase + static_cast<uint32_t>(kh * a.dh * a.halo_w + kw * a.dw) * 128u;
-            const uint32_t sb = ptx::smem_u32(bring + bst * a.stage_bytes + j * a.b_bytes);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t da = ptx::smem_desc_sw128_view(view + k * 32, sbo, 0);
-              const uint64_t db = ptx::smem_desc(sb + k * 32, 16, 1024, 2);
-              if constexpr (PAIR) ptx::mma_f16_pair(d_tmem, da, db, a.idesc, accumulate);
-              else ptx::mma_f16(d_tmem, da, db, a.idesc, accumulate);
-              accumulate = 1;
+            // the view of tap (kh, kw) starts (kh*dh*halo_w + kw*dw) halo pixels into the box
+            const uint64_t da = d_box + desc_off(static_cast<uint32_t>(kh * a.dh * a.halo_w + kw * a.dw) * 128u);
+            mma_ksteps<4, PAIR>(d_tmem, da, db, a.idesc, accumulate);
+            accumulate = 1;
+            db += sub_off;
+            const bool last_tap = kh == a.kH - 1 && kw == a.kW - 1;
+            if (++kw == a.kW) {
+              kw = 0;
+              if (++kh == a.kH) kh = 0;
             }
-            if (tp == taps_hw - 1) {
+            if (last_tap) {
               // last tap of this (cc, kd): its halo slot is free once these MMAs complete
               if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->aempty[ast]), both);
               else ptx::mma_commit(ptx::smem_u32(&tail->aempty[ast]));

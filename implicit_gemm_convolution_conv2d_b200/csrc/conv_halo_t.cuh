@@ -3,10 +3,11 @@
 //
 // The product is issued as y^T[o, m] = sum_k W[o, k] X[m, k] (see
 // conv_tct.cuh): MMA M = 128 output channels (A = a weight tile), N = 256
-// output pixels (B = patch rows).  The 256 pixels are a block of 32 x 8
-// output pixels (h x w) of one (n, od) plane, and B is not loaded per tap:
+// output pixels (B = patch rows).  The pixels are a block of tile_h x 8
+// output pixels (h x w, tile_h <= 32) of one (n, od) plane, and B is not
+// loaded per tap:
 // for each 64-channel chunk, depth tap kd and width tap kw, ONE tiled TMA box
-// brings the input column strip the block needs -- (32 + dh*(kH-1)) rows x 8
+// brings the input column strip the block needs -- (tile_h + dh*(kH-1)) rows x 8
 // columns (shifted by kw*dw) x 64 channels, zero-filled outside the image --
 // and every height tap kh reads a view of it that starts kh*dh rows down.
 // Pixel j = r*8 + c of the block reads strip pixel (r + kh*dh, c); the strip is
@@ -19,7 +20,7 @@
 // (chunk, kd, kw) instead of kH*kW times per (chunk, kd): per 64-deep K block
 // 16 KB of weights plus strip/kH instead of 16 KB plus 32 KB of patch rows.
 //
-// Epilogue: the accumulator holds [128 channels][256 pixels]; 32 columns are
+// Epilogue: the accumulator holds [128 channels][8 * tile_h pixels]; 32 columns are
 // 4 output rows x 8 output columns.  Four warps transpose each such chunk into
 // a [4][8][128] staging tile and one thread stores it with a 4-D / 5-D TMA
 // tensor store on y viewed as [N, (Do,) Ho, Wo, O], which clips the rows and
@@ -31,7 +32,11 @@
 
 namespace convfwd {
 
-constexpr int kHTBlockH = 32, kHTBlockW = 8;  // output block: MMA N = 256 pixels
+// Output block: tile_h (4 .. 32, a multiple of 4, chosen by the host to fit Ho)
+// x 8 pixels, so MMA N = 8 * tile_h <= 256.  The two accumulators sit 256
+// tensor-memory columns apart whatever N is.
+constexpr int kHTBlockHMax = 32, kHTBlockW = 8;
+constexpr uint32_t kHTAccStride = 256;
 
 struct HaloTTile {
   int g, n, od, h0, w0, ot;
@@ -57,7 +62,7 @@ __device__ __forceinline__ HaloTTile decode_halo_t_tile(const TcArgs& a, int til
   return t;
 }
 
-template <bool BF16>
+template <bool BF16, bool PAIR>
 __global__ void __launch_bounds__(kTThreads, 1)
     conv_fwd_tc_halo_t_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                               const __grid_constant__ CUtensorMap tmap_y, const TcArgs a) {
@@ -69,6 +74,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
   TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(stage_y + 2 * kTEpiBytes);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const uint32_t mult = PAIR ? 2u : 1u;  // CTAs whose loads complete on the leader's barriers
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
@@ -81,7 +89,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(ptx::smem_u32(&tail->acc_full[b]), 1u);
-      ptx::mbar_init(ptx::smem_u32(&tail->acc_empty[b]), 4u);
+      ptx::mbar_init(ptx::smem_u32(&tail->acc_empty[b]), PAIR ? 8u : 4u);
     }
     ptx::mbar_init(ptx::smem_u32(&tail->drain), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
@@ -94,32 +102,45 @@ __global__ void __launch_bounds__(kTThreads, 1)
     ptx::prefetch_tmap(&tmap_y);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_u32(&tail->tmem_base), a.tmem_cols);
-    ptx::tmem_relinquish();
+    if constexpr (PAIR) {
+      ptx::tmem_alloc_pair(ptx::smem_u32(&tail->tmem_base), a.tmem_cols);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(ptx::smem_u32(&tail->tmem_base), a.tmem_cols);
+      ptx::tmem_relinquish();
+    }
   }
   ptx::tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem_base = tail->tmem_base;
   volatile int* abort_flag = &tail->abort_flag;
   const int taps_hw = a.kH * a.kW;
-  const int BP = a.BN;  // 256 output pixels per tile
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nunits = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int o_tile = PAIR ? 2 * kTO : kTO;  // output channels per tile (a pair: 128 per CTA)
+  const int BP = a.BN;  // 8 * tile_h output pixels per tile
 
   // K blocks of a tile in issue order: q = ((cc * kD + kd) * kW + kw) * kH + kh.
   // A pipeline stage holds up to kbs consecutive K blocks (weight tiles); each
-  // (cc, kd, kw) group has one strip, loaded before its first K block.  With
-  // kbs <= kH a stage spans at most two groups, so two strip slots suffice.
+  // (cc, kd, kw) group has one strip in its own ring of a_slots slots.
   const int Q = a.cchunks * a.kD * taps_hw;
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producers
+    // Two threads, each running ahead on its own ring: lane 0 streams the
+    // weight tiles, lane 1 the input strips.  Each arms a barrier only right
+    // before issuing every load it covers, so a wait that gives up never
+    // leaves a barrier expecting bytes that were not requested.
     if (lane == 0) {
-      int bst = 0, ast = 0;
-      uint32_t bph = 0, aph = 0;
-      long long bfills = 0, afills = 0;
+      int bst = 0;
+      uint32_t bph = 0;
+      long long bfills = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x) {
+      for (int tile = unit; ok && tile < a.total_tiles; tile += nunits) {
         const HaloTTile ht = decode_halo_t_tile(a, tile);
-        const int orow = ht.g * a.Og + ht.ot * kTO;
+        const int orow = ht.g * a.Og + ht.ot * o_tile + static_cast<int>(rank) * kTO;
+        int kh = 0, kw = 0, kd = 0, cc = 0;  // tap of the next K block (kh fastest, then kw, kd, cc)
         for (int q0 = 0; ok && q0 < Q; q0 += a.kbs) {
           const int nsub = min(a.kbs, Q - q0);
           if (!wait_bounded(ptx::smem_u32(&tail->empty[bst]), bph ^ 1u, abort_flag, a.timeout_ns,
@@ -127,41 +148,24 @@ __global__ void __launch_bounds__(kTThreads, 1)
             ok = false;
             break;
           }
-          // halo boxes first: a wait that gives up here leaves no stage armed
-          for (int j = 0; j < nsub; ++j) {
-            const int q = q0 + j;
-            if (q % a.kH != 0) continue;
-            const int grp = q / a.kH;
-            const int kw = grp % a.kW, kd = (grp / a.kW) % a.kD, cc = grp / (a.kW * a.kD);
-            if (!wait_bounded(ptx::smem_u32(&tail->aempty[ast]), aph ^ 1u, abort_flag, a.timeout_ns,
-                              kSiteProducerEmpty)) {
-              ok = false;
-              break;
-            }
-            const uint32_t afb = ptx::smem_u32(&tail->afull[ast]);
-            ptx::mbar_arrive_expect_tx(afb, a.halo_bytes);
-            const uint32_t dst = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
-            const int c0 = ht.g * a.Cg + cc * 64;
-            const int wc = ht.w0 - a.pw + kw * a.dw, hc = ht.h0 - a.ph, dc = ht.od - a.pd + kd * a.dd;
-            if (a.rank5) ptx::tma_load_5d(dst, &tmap_x, afb, c0, wc, hc, dc, ht.n);
-            else ptx::tma_load_4d(dst, &tmap_x, afb, c0, wc, hc, ht.n);
-            ++afills;
-            if (++ast == a.a_slots) {
-              ast = 0;
-              aph ^= 1u;
-            }
-          }
-          if (!ok) break;
-          // then the stage's weight tiles, armed for exactly what is issued
           const uint32_t fb = ptx::smem_u32(&tail->full[bst]);
-          ptx::mbar_arrive_expect_tx(fb, static_cast<uint32_t>(nsub) * a.b_bytes);
+          if (leader) ptx::mbar_arrive_expect_tx(fb, mult * static_cast<uint32_t>(nsub) * a.b_bytes);
+          const uint32_t fb_l = PAIR ? ptx::mapa_shared(fb, 0) : fb;
           for (int j = 0; j < nsub; ++j) {
-            const int q = q0 + j;
-            const int kh = q % a.kH, grp = q / a.kH;
-            const int kw = grp % a.kW, kd = (grp / a.kW) % a.kD, cc = grp / (a.kW * a.kD);
             const uint32_t sb = ptx::smem_u32(bring + bst * a.stage_bytes + j * a.b_bytes);
             const int tap = (kd * a.kH + kh) * a.kW + kw;  // weight layout (kd, kh, kw)
-            ptx::tma_load_2d(sb, &tmap_w, fb, tap * a.Cg + cc * 64, orow);
+            if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, orow);
+            else ptx::tma_load_2d(sb, &tmap_w, fb, tap * a.Cg + cc * 64, orow);
+            if (++kh == a.kH) {
+              kh = 0;
+              if (++kw == a.kW) {
+                kw = 0;
+                if (++kd == a.kD) {
+                  kd = 0;
+                  ++cc;
+                }
+              }
+            }
           }
           ++bfills;
           if (++bst == a.stages) {
@@ -170,11 +174,52 @@ __global__ void __launch_bounds__(kTThreads, 1)
           }
         }
       }
-      if (!ok) {
+      // (a pair's loads all complete on the leader's barriers: the leader drains)
+      if (!ok && leader) {
         for (int s = 0; s < a.stages; ++s) {
           const long long arms = bfills / a.stages + (s < bfills % a.stages ? 1 : 0);
           if (arms > 0) wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
         }
+      }
+    } else if (lane == 1) {
+      int ast = 0;
+      uint32_t aph = 0;
+      long long afills = 0;
+      bool ok = true;
+      for (int tile = unit; ok && tile < a.total_tiles; tile += nunits) {
+        const HaloTTile ht = decode_halo_t_tile(a, tile);
+        for (int cc = 0; ok && cc < a.cchunks; ++cc)
+          for (int kd = 0; ok && kd < a.kD; ++kd)
+            for (int kw = 0; kw < a.kW; ++kw) {
+              if (!wait_bounded(ptx::smem_u32(&tail->aempty[ast]), aph ^ 1u, abort_flag, a.timeout_ns,
+                                kSiteProducerEmpty)) {
+                ok = false;
+                break;
+              }
+              const uint32_t afb = ptx::smem_u32(&tail->afull[ast]);
+              if (leader) ptx::mbar_arrive_expect_tx(afb, mult * a.halo_bytes);
+              const uint32_t afb_l = PAIR ? ptx::mapa_shared(afb, 0) : afb;
+              const uint32_t dst = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
+              const int c0 = ht.g * a.Cg + cc * 64;
+              // a pair splits the block's rows: each CTA loads the strip of its half
+              const int wc = ht.w0 - a.pw + kw * a.dw;
+              const int hc = ht.h0 + static_cast<int>(rank) * (a.tile_h / 2) - a.ph;
+              const int dc = ht.od - a.pd + kd * a.dd;
+              if constexpr (PAIR) {
+                if (a.rank5) ptx::tma_load_5d_pair(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
+                else ptx::tma_load_4d_pair(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
+              } else {
+                if (a.rank5) ptx::tma_load_5d(dst, &tmap_x, afb, c0, wc, hc, dc, ht.n);
+                else ptx::tma_load_4d(dst, &tmap_x, afb, c0, wc, hc, ht.n);
+              }
+              ++afills;
+              if (++ast == a.a_slots) {
+                ast = 0;
+                aph ^= 1u;
+              }
+            }
+      }
+      if (!ok && leader) {
         for (int s = 0; s < a.a_slots; ++s) {
           const long long arms = afills / a.a_slots + (s < afills % a.a_slots ? 1 : 0);
           if (arms > 0) wait_drain(ptx::smem_u32(&tail->afull[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
@@ -183,15 +228,21 @@ __global__ void __launch_bounds__(kTThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (a pair's leader)
+    if (leader && lane == 0) {
       int bst = 0, ast = 0;
       uint32_t bph = 0, aph = 0;
       bool ok = true;
       int t = 0;
       if (a.inject_stall)
         ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
-      for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++t) {
+      // descriptors built once; moved by constant offsets below
+      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, 2);
+      const uint64_t d_halo = ptx::smem_desc(ptx::smem_u32(halo), 16, 1024, 2);
+      const uint64_t sub_off = desc_off(a.b_bytes), st_off = desc_off(a.stage_bytes);
+      const uint64_t slot_off = desc_off(a.halo_slot_bytes);
+      const uint64_t row_off = desc_off(static_cast<uint32_t>(a.dh) * 1024u);
+      for (int tile = unit; ok && tile < a.total_tiles; tile += nunits, ++t) {
         const int acc = t & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
         if (!wait_bounded(ptx::smem_u32(&tail->acc_empty[acc]), acc_phase ^ 1u, abort_flag, a.timeout_ns,
@@ -200,9 +251,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BP);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kHTAccStride;
         uint32_t accumulate = 0;
-        uint32_t hbase = 0;
+        uint64_t d_strip = 0;
+        int kh = 0;  // height tap of the next K block (K blocks run kh-fastest)
         for (int q0 = 0; ok && q0 < Q; q0 += a.kbs) {
           const int nsub = min(a.kbs, Q - q0);
           if (!wait_bounded(ptx::smem_u32(&tail->full[bst]), bph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
@@ -210,47 +262,49 @@ __global__ void __launch_bounds__(kTThreads, 1)
             break;
           }
           ptx::tc_fence_after();
+          uint64_t dw = d_ring + static_cast<uint64_t>(bst) * st_off;
           for (int j = 0; j < nsub; ++j) {
-            const int q = q0 + j;
-            const int kh = q % a.kH;
             if (kh == 0) {
               if (!wait_bounded(ptx::smem_u32(&tail->afull[ast]), aph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
                 ok = false;
                 break;
               }
               ptx::tc_fence_after();
-              hbase = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
+              d_strip = d_halo + static_cast<uint64_t>(ast) * slot_off;
             }
             // strip rows are 8 pixels = 1024 bytes: the view for kh starts kh*dh atoms down
-            const uint32_t view = hbase + static_cast<uint32_t>(kh * a.dh) * 1024u;
-            const uint32_t sw = ptx::smem_u32(bring + bst * a.stage_bytes + j * a.b_bytes);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t da = ptx::smem_desc(sw + k * 32, 16, 1024, 2);
-              const uint64_t db = ptx::smem_desc(view + k * 32, 16, 1024, 2);
-              ptx::mma_f16(d_tmem, da, db, a.idesc, accumulate);
-              accumulate = 1;
-            }
+            mma_ksteps<4, PAIR>(d_tmem, dw, d_strip + static_cast<uint64_t>(kh) * row_off, a.idesc, accumulate);
+            accumulate = 1;
+            dw += sub_off;
             if (kh == a.kH - 1) {
               // last tap of this (cc, kd, kw): its strip slot is free once these MMAs complete
-              ptx::mma_commit(ptx::smem_u32(&tail->aempty[ast]));
+              if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->aempty[ast]), 3);
+              else ptx::mma_commit(ptx::smem_u32(&tail->aempty[ast]));
               if (++ast == a.a_slots) {
                 ast = 0;
                 aph ^= 1u;
               }
+              kh = 0;
+            } else {
+              ++kh;
             }
           }
           if (!ok) break;
-          ptx::mma_commit(ptx::smem_u32(&tail->empty[bst]));
+          if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[bst]), 3);
+          else ptx::mma_commit(ptx::smem_u32(&tail->empty[bst]));
           if (++bst == a.stages) {
             bst = 0;
             bph ^= 1u;
           }
         }
-        if (ok) ptx::mma_commit(ptx::smem_u32(&tail->acc_full[acc]));
+        if (ok) {
+          if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->acc_full[acc]), 3);
+          else ptx::mma_commit(ptx::smem_u32(&tail->acc_full[acc]));
+        }
       }
       // every MMA this thread issued has completed once `drain` fires
-      ptx::mma_commit(ptx::smem_u32(&tail->drain));
+      if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->drain), 1);
+      else ptx::mma_commit(ptx::smem_u32(&tail->drain));
       wait_drain(ptx::smem_u32(&tail->drain), 0, a.timeout_ns);
     }
     __syncwarp();
@@ -260,7 +314,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const bool store_thread = warp == 2 && lane == 0;
     constexpr int kRowsPerChunk = kTEpiRows / kHTBlockW;  // 4 output rows per 32 columns
     int t = 0, chunk_seq = 0;
-    for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++t) {
+    for (int tile = unit; tile < a.total_tiles; tile += nunits, ++t) {
       const int acc = t & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
       bool ok = wait_bounded_warp(ptx::smem_u32(&tail->acc_full[acc]), acc_phase, abort_flag, a.timeout_ns,
@@ -271,8 +325,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       const HaloTTile ht = decode_halo_t_tile(a, tile);
-      const int o0 = ht.g * a.Og + ht.ot * kTO;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BP);
+      const int o0 = ht.g * a.Og + ht.ot * o_tile + static_cast<int>(rank) * kTO;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc) * kHTAccStride;
       for (int c = 0; c < BP; c += kTEpiRows) {
         uint32_t r[32];
         ptx::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c), r);
@@ -297,7 +351,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&tail->acc_empty[acc]));
+      if (lane == 0) {
+        // a pair's accumulator buffer is reused once both CTAs' epilogues are done
+        const uint32_t ae = ptx::smem_u32(&tail->acc_empty[acc]);
+        if constexpr (PAIR) ptx::mbar_arrive_cluster(ptx::mapa_shared(ae, 0));
+        else ptx::mbar_arrive(ae);
+      }
     }
     // every store has finished (reading shared memory and writing y) before exit
     if (store_thread) ptx::bulk_wait_group<0>();
@@ -306,8 +365,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) ptx::cluster_sync();  // the leader's MMAs (which read this CTA's smem) are complete
   ptx::tc_fence_after();
-  if (warp == 1) ptx::tmem_dealloc(tmem_base, a.tmem_cols);
+  if (warp == 1) {
+    if constexpr (PAIR) ptx::tmem_dealloc_pair(tmem_base, a.tmem_cols);
+    else ptx::tmem_dealloc(tmem_base, a.tmem_cols);
+  }
 }
 
 }  // namespace convfwd

@@ -229,6 +229,43 @@ __device__ __forceinline__ uint16_t cvt1(float v) {
   }
 }
 
+// ----------------------------------------------------------------------------
+// MMA issue.  One thread issues every tcgen05.mma of a CTA, and on B200 the
+// instruction stream around the MMAs decides whether the tensor pipe stays
+// fed: a per-instruction rebuild of the operand descriptors in a loop with a
+// run-time trip count cost ~220 SM cycles per 128x256x16 MMA in a probe,
+// against 128 (the pipe's own rate) for fully unrolled issue of descriptors
+// that only advance by constants.  So descriptors are built once, moved by
+// 64-bit adds (the start address is bits 0..13 in 16-byte units, and shared
+// memory is below 256 KB, so an add never carries out of the field), and the
+// K steps of one sub-block are issued by an unrolled compile-time loop.
+// ----------------------------------------------------------------------------
+
+// Descriptor address units (16 bytes) for a byte offset.
+__device__ __forceinline__ uint64_t desc_off(uint32_t bytes) { return static_cast<uint64_t>(bytes >> 4); }
+
+// KS MMAs of K = 16 over one sub-block: both operands advance 32 bytes
+// (2 descriptor units) per step.  acc0 = 0 overwrites the accumulator with
+// the first product.
+template <int KS, bool PAIR>
+__device__ __forceinline__ void mma_ksteps(uint32_t d_tmem, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc0) {
+#pragma unroll
+  for (int k = 0; k < KS; ++k) {
+    if constexpr (PAIR) ptx::mma_f16_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, k == 0 ? acc0 : 1u);
+    else ptx::mma_f16(d_tmem, da + 2 * k, db + 2 * k, idesc, k == 0 ? acc0 : 1u);
+  }
+}
+
+// The same for a run-time step count of 4, 2 or 1 (channel chunks of 64, 32
+// or 16 elements).
+template <bool PAIR>
+__device__ __forceinline__ void mma_sub(int ksteps, uint32_t d_tmem, uint64_t da, uint64_t db, uint32_t idesc,
+                                        uint32_t acc0) {
+  if (ksteps == 4) mma_ksteps<4, PAIR>(d_tmem, da, db, idesc, acc0);
+  else if (ksteps == 2) mma_ksteps<2, PAIR>(d_tmem, da, db, idesc, acc0);
+  else mma_ksteps<1, PAIR>(d_tmem, da, db, idesc, acc0);
+}
+
 enum { MODE_TMA = 0, MODE_GATHER = 1 };
 
 template <int MODE>
@@ -787,7 +824,12 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
         ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
       if (ok && a.b_resident)
         ok = wait_bounded(ptx::smem_u32(&tail->bres), 0u, abort_flag, a.timeout_ns, kSiteMmaFull);
-      const uint32_t bres_addr = ptx::smem_u32(bres);
+      // descriptors built once; moved by constant offsets below
+      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(smem), 16, a.sbo, a.layout_type);
+      const uint64_t d_res = ptx::smem_desc(ptx::smem_u32(bres), 16, a.sbo, a.layout_type);
+      const uint64_t a_off = desc_off(a.a_bytes), sub_off = desc_off(a.sub_bytes), st_off = desc_off(a.stage_bytes);
+      const uint64_t res_step = desc_off(static_cast<uint32_t>(a.BN) * 128u);
+      const int ksteps = a.kc >> 4;
       for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++t) {
         const int acc = t & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -806,16 +848,11 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
             break;
           }
           ptx::tc_fence_after();
-          const int ksteps = a.kc >> 4;
+          uint64_t da = d_ring + static_cast<uint64_t>(stage) * st_off;
           for (int j = 0; j < nsub; ++j) {
-            const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes + j * a.sub_bytes);
-            const uint32_t sb = a.b_resident ? bres_addr + static_cast<uint32_t>(kb + j) * a.BN * 128u
-                                             : sa + a.a_bytes;
-            for (int k = 0; k < ksteps; ++k) {
-              const uint64_t da = ptx::smem_desc(sa + k * 32, 16, a.sbo, a.layout_type);
-              const uint64_t db = ptx::smem_desc(sb + k * 32, 16, a.sbo, a.layout_type);
-              ptx::mma_f16(d_tmem, da, db, a.idesc, ((kb + j) | k) != 0 ? 1u : 0u);
-            }
+            const uint64_t db = a.b_resident ? d_res + static_cast<uint64_t>(kb + j) * res_step : da + a_off;
+            mma_sub<false>(ksteps, d_tmem, da, db, a.idesc, (kb + j) != 0 ? 1u : 0u);
+            da += sub_off;
           }
           ptx::mma_commit(ptx::smem_u32(&tail->empty[stage]));
           if (++stage == a.stages) {
@@ -1016,6 +1053,10 @@ __global__ void __launch_bounds__(192, 1)
       int t = 0;
       if (a.inject_stall)
         ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
+      // descriptors built once; moved by constant offsets below
+      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(smem), 16, a.sbo, a.layout_type);
+      const uint64_t a_off = desc_off(a.a_bytes), sub_off = desc_off(a.sub_bytes), st_off = desc_off(a.stage_bytes);
+      const int ksteps = a.kc >> 4;
       for (int tile = pair; ok && tile < a.total_tiles; tile += npairs, ++t) {
         const int acc = t & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -1033,15 +1074,10 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           ptx::tc_fence_after();
-          const int ksteps = a.kc >> 4;
+          uint64_t da = d_ring + static_cast<uint64_t>(stage) * st_off;
           for (int j = 0; j < nsub; ++j) {
-            const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes + j * a.sub_bytes);
-            const uint32_t sb = sa + a.a_bytes;
-            for (int k = 0; k < ksteps; ++k) {
-              const uint64_t da = ptx::smem_desc(sa + k * 32, 16, a.sbo, a.layout_type);
-              const uint64_t db = ptx::smem_desc(sb + k * 32, 16, a.sbo, a.layout_type);
-              ptx::mma_f16_pair(d_tmem, da, db, a.idesc, ((kb + j) | k) != 0 ? 1u : 0u);
-            }
+            mma_sub<true>(ksteps, d_tmem, da, da + a_off, a.idesc, (kb + j) != 0 ? 1u : 0u);
+            da += sub_off;
           }
           ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[stage]), 3);
           if (++stage == a.stages) {

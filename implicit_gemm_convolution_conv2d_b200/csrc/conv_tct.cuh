@@ -178,6 +178,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
       int t = 0;
       if (a.inject_stall)
         ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
+      // descriptors built once; moved by constant offsets below
+      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(smem), 16, a.sbo, a.layout_type);
+      const uint64_t a_off = desc_off(a.a_bytes), sub_off = desc_off(a.sub_bytes), st_off = desc_off(a.stage_bytes);
+      const int ksteps = a.kc >> 4;
       for (int tile = blockIdx.x; ok && tile < a.total_tiles; tile += gridDim.x, ++t) {
         const int acc = t & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -195,15 +199,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
             break;
           }
           ptx::tc_fence_after();
-          const int ksteps = a.kc >> 4;
+          uint64_t da = d_ring + static_cast<uint64_t>(stage) * st_off;
           for (int j = 0; j < nsub; ++j) {
-            const uint32_t sa = ptx::smem_u32(smem + stage * a.stage_bytes + j * a.sub_bytes);
-            const uint32_t sb = sa + a.a_bytes;
-            for (int k = 0; k < ksteps; ++k) {
-              const uint64_t da = ptx::smem_desc(sa + k * 32, 16, a.sbo, a.layout_type);
-              const uint64_t db = ptx::smem_desc(sb + k * 32, 16, a.sbo, a.layout_type);
-              ptx::mma_f16(d_tmem, da, db, a.idesc, ((kb + j) | k) != 0 ? 1u : 0u);
-            }
+            mma_sub<false>(ksteps, d_tmem, da, da + a_off, a.idesc, (kb + j) != 0 ? 1u : 0u);
+            da += sub_off;
           }
           ptx::mma_commit(ptx::smem_u32(&tail->empty[stage]));
           if (++stage == a.stages) {

@@ -98,7 +98,7 @@ def test_invalid_arguments_rejected_on_host(C):
     big = 1 << 30
     assert call(X, Wt, Y, big, big, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
     # unknown variant
-    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 8, None) == -1
+    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 9, None) == -1
     assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, -2, None) == -1
 
 
@@ -116,9 +116,16 @@ def test_variant_plan(C):
     assert v == C.VARIANT_TC_TMA and bn == 64
     v, bn, _, _ = plan(4, 32, 32, 32, 64, 128, (3, 3, 3), (2, 2, 2), (1, 1, 1), (1, 1, 1), 1, "f16")
     assert v in (C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR) and bn == 128
-    # 128 output channels and enough pixels: the transposed orientation, 256-pixel tiles
+    # 128 output channels, stride 1, 64-channel chunks, kH >= 2: the transposed halo kernel
     v, bn, st, _ = plan(4, 32, 32, 32, 64, 128, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
-    assert v == C.VARIANT_TC_TMA_T and bn == 256 and st >= 2
+    assert v == C.VARIANT_TC_HALO_T and bn == 256 and st >= 2
+    # ... with kH = 1 (no strip reuse): the transposed im2col kernel
+    v, bn, _, _ = plan(4, 32, 32, 32, 64, 128, (3, 1, 1), (1, 1, 1), (1, 0, 0), (1, 1, 1), 1, "f16")
+    assert v == C.VARIANT_TC_TMA_T and bn == 256
+    # block height adapts to Ho: 56 rows -> blocks of 28 (MMA N = 224)
+    v, bn, _, _ = plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16",
+                       C.VARIANT_TC_HALO_T_PAIR)
+    assert v == C.VARIANT_TC_HALO_T_PAIR and bn == 224
     v, bn, _, _ = plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
     assert v == C.VARIANT_TC_GATHER and bn == 64
     v, bn, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
@@ -139,7 +146,8 @@ def test_explicit_variant_plan(C):
     """conv_plan_variant resolves an explicit variant or refuses it by the
     same rule conv_fwd_variant applies."""
     g3 = (64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1)
-    for name in ("TC_TMA", "TC_TMA_PAIR", "TC_GATHER", "TC_HALO", "TC_HALO_PAIR", "SIMT"):
+    for name in ("TC_TMA", "TC_TMA_PAIR", "TC_GATHER", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T", "TC_HALO_T",
+                 "TC_HALO_T_PAIR", "SIMT"):
         v = getattr(C, "VARIANT_" + name)
         assert C.plan(*g3, "bf16", v)[0] == v
     assert C.plan(*g3, "bf16", C.VARIANT_AUTO) == C.plan(*g3, "bf16")
@@ -154,5 +162,5 @@ def test_explicit_variant_plan(C):
         C.plan(*g3, "f32", C.VARIANT_TC_TMA)
     assert e.value.code == -7
     with pytest.raises(C.ConvError) as e:
-        C.plan(*g3, "bf16", 8)
+        C.plan(*g3, "bf16", 9)
     assert e.value.code == -1

@@ -35,10 +35,10 @@ def _geom(wl):
 
 
 @pytest.mark.parametrize("variant", ["TC_GATHER", "TC_TMA", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T",
-                                     "TC_HALO_T"])
+                                     "TC_HALO_T", "TC_HALO_T_PAIR"])
 def test_injected_stall_times_out_and_recovers(variant):
     v = getattr(C, "VARIANT_" + variant)
-    O = 128 if variant in ("TC_TMA_T", "TC_HALO_T") else 64
+    O = {"TC_TMA_T": 128, "TC_HALO_T": 128, "TC_HALO_T_PAIR": 256}.get(variant, 64)
     wl = WL.case(2, 1, 20, 20, 64, O, (1, 3, 3), pad=(0, 1, 1), dtype="f16", seed=21)
     x, w = WL.make_inputs(wl)
     xd, wd = x.cuda(), w.cuda()

@@ -62,6 +62,8 @@ def variants_for(wl):
         vs.append(C.VARIANT_TC_TMA_T)
     if (wl.C // wl.groups) % 64 == 0 and (wl.O // wl.groups) % 128 == 0 and tuple(wl.stride) == (1, 1, 1):
         vs.append(C.VARIANT_TC_HALO_T)
+    if (wl.C // wl.groups) % 64 == 0 and (wl.O // wl.groups) % 256 == 0 and tuple(wl.stride) == (1, 1, 1):
+        vs.append(C.VARIANT_TC_HALO_T_PAIR)
     return vs
 
 
@@ -116,6 +118,10 @@ SMALL = [
     WL.case(1, 3, 19, 11, 64, 128, (3, 3, 3), pad=(1, 2, 1), dil=(1, 2, 1), name="ht_3d_dil"),
     WL.case(1, 1, 33, 17, 128, 256, (1, 5, 5), pad=(0, 2, 2), name="ht_c128_o256_k5"),
     WL.case(2, 1, 9, 9, 128, 256, (1, 3, 3), pad=(0, 1, 1), groups=2, name="ht_groups2"),
+    # pairs of CTAs over 256 output channels: block heights 28 and 20, 3-D, groups
+    WL.case(2, 1, 28, 21, 64, 256, (1, 3, 3), pad=(0, 1, 1), name="htp_h28"),
+    WL.case(1, 3, 19, 11, 64, 256, (3, 3, 3), pad=(1, 2, 1), dil=(1, 2, 1), name="htp_3d_dil"),
+    WL.case(2, 1, 9, 10, 128, 512, (1, 3, 3), pad=(0, 1, 1), groups=2, name="htp_groups2"),
 ]
 
 
