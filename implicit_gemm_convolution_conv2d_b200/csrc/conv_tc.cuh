@@ -14,7 +14,7 @@
 //             K-elements, B: BN rows x the same), signalling `full[s]`;
 //             MODE_TMA: one thread issues a TMA im2col load (A) and a TMA tiled
 //             load (B) per stage -- the hardware walks the output pixels and
-//             zero-fills the halo;  MODE_GATHER: four warps compute every
+//             zero-fills the halo;  MODE_GATHER: 16 warps compute every
 //             element's address and zero-fill out-of-range taps and channels
 //             themselves (any C, any stride/dilation/groups);
 //   MMA       one thread issues tcgen05.mma (M=128, N=BN, K=16 per
@@ -191,8 +191,21 @@ __device__ __forceinline__ TileCoord decode_tile(const TcArgs& a, int tile) {
 }
 
 // Output pixel m -> (n, od, oh, ow).
+// 32-bit arithmetic whenever M fits (64-bit division is a long software
+// sequence, and every gather thread decodes its pixel once per tile).
 __device__ __forceinline__ void decode_pixel(const TcArgs& a, long long m, int& n, int& od, int& oh,
                                              int& ow) {
+  if (a.M <= 0x7fffffffLL) {
+    const unsigned mm = static_cast<unsigned>(m);
+    const unsigned q1 = mm / static_cast<unsigned>(a.Wo);
+    const unsigned q2 = q1 / static_cast<unsigned>(a.Ho);
+    const unsigned q3 = q2 / static_cast<unsigned>(a.Do);
+    ow = static_cast<int>(mm - q1 * static_cast<unsigned>(a.Wo));
+    oh = static_cast<int>(q1 - q2 * static_cast<unsigned>(a.Ho));
+    od = static_cast<int>(q2 - q3 * static_cast<unsigned>(a.Do));
+    n = static_cast<int>(q3);
+    return;
+  }
   ow = static_cast<int>(m % a.Wo);
   long long q = m / a.Wo;
   oh = static_cast<int>(q % a.Ho);
@@ -277,7 +290,7 @@ struct TcRoles<MODE_TMA> {
 };
 template <>
 struct TcRoles<MODE_GATHER> {
-  static constexpr int kProducerWarps = 8;
+  static constexpr int kProducerWarps = 16;
 };
 
 template <int MODE>
@@ -286,17 +299,46 @@ constexpr int tc_threads() {
 }
 
 // ----------------------------------------------------------------------------
-// Gather producer: 256 threads fill one stage from plain global loads with
-// zero fill.  Thread t owns A row t % 128 and half t / 128 of the 64 K
-// elements of each stage; element k of a row is (kd, kh, kw, c) in weight
-// order.  B is either resident (loaded once per CTA) or gathered per stage.
+// Gather producer: 512 threads (16 warps) fill one stage with zero fill.
+// Thread t owns A row t % 128 and the 16-element quarter t / 128 of every
+// 64-wide K block; element k of a row is (kd, kh, kw, c) in weight order (or
+// the span layout).  B is either resident (loaded once per CTA) or gathered
+// per stage.
 // ----------------------------------------------------------------------------
 struct GatherRow {
   bool valid;
   long long nbase;  // element offset of x[n, 0, 0, 0, g*Cg]
   int id0, ih0, iw0;
   int jlo, jhi;     // span mode: valid offsets within a filter row
+  uint32_t rseg;    // row staging: byte address of this pixel's image segment
+  int lr0;          // row staging: staged row of input row ih0 in that segment
 };
+
+// Position in the span layout of K: element j of filter row (kd, kh).  Each
+// gather thread walks it in steps of 8 instead of dividing k by Lp per call.
+struct SpanPos {
+  int j, kh, kd;
+};
+
+__device__ __forceinline__ void span_step8(const TcArgs& a, SpanPos& p) {
+  p.j += 8;
+  if (p.j == a.Lp) {
+    p.j = 0;
+    if (++p.kh == a.kH) {
+      p.kh = 0;
+      ++p.kd;
+    }
+  }
+}
+
+__device__ __forceinline__ SpanPos span_pos(const TcArgs& a, int k) {
+  const int span = k / a.Lp;
+  SpanPos p;
+  p.j = k - span * a.Lp;
+  p.kh = span % a.kH;
+  p.kd = span / a.kH;
+  return p;
+}
 
 // One filter row (kd, kh) of one output pixel: offset of x[n, id, ih, 0, g*Cg]
 // and whether that input row exists.
@@ -322,7 +364,7 @@ __device__ __forceinline__ uint4 load8_masked(const uint16_t* p, int e_lo, int e
   return make_uint4(v[0] | (v[1] << 16), v[2] | (v[3] << 16), v[4] | (v[5] << 16), v[6] | (v[7] << 16));
 }
 
-// Four 8-element chunks (K elements k0 .. k0+31) of one A row.
+// NCH 8-element chunks (K elements k0 .. k0+8*NCH-1) of one A row.
 //
 // GATHER_VEC8 (C/G % 8 == 0): a chunk is 8 channels of one input pixel, one
 // aligned 16-byte load, or zeros when the pixel is in the padding.
@@ -333,6 +375,7 @@ __device__ __forceinline__ uint4 load8_masked(const uint16_t* p, int e_lo, int e
 // GATHER_SCALAR: element-wise (kw, c) walk with its own bounds check.
 enum { GATHER_SCALAR = 0, GATHER_VEC8 = 1, GATHER_SPAN = 2, GATHER_ROWS = 3 };
 
+template <int NCH>
 __device__ __forceinline__ void gather_a_vec8(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
                                               int r, int chunk0) {
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
@@ -344,9 +387,9 @@ __device__ __forceinline__ void gather_a_vec8(const TcArgs& a, const GatherRow& 
   int kd = t2 / a.kH;
   long long rowptr;
   bool rok = gather_span(a, st, kd, kh, rowptr);
-  uint4 v[4];
+  uint4 v[NCH];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < NCH; ++q) {
     const int iw = st.iw0 + kw * a.dw;
     v[q] = make_uint4(0, 0, 0, 0);
     if (rok && static_cast<unsigned>(iw) < static_cast<unsigned>(a.W))
@@ -365,7 +408,7 @@ __device__ __forceinline__ void gather_a_vec8(const TcArgs& a, const GatherRow& 
     }
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) store_chunk(a_tile, r, chunk0 + q, v[q]);
+  for (int q = 0; q < NCH; ++q) store_chunk(a_tile, r, chunk0 + q, v[q]);
 }
 
 // Halfwords h .. h+7 of the 16 halfwords in (b0, b1), h in 0..7.
@@ -397,22 +440,20 @@ __device__ __forceinline__ uint4 mask8(uint4 v, unsigned m) {
   return v;
 }
 
-__device__ __forceinline__ void gather_a_span(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
+template <int NCH>
+__device__ __forceinline__ void gather_a_span(const TcArgs& a, const GatherRow& st, SpanPos& pos, uint8_t* a_tile,
                                               int r, int chunk0) {
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
-  const int span = k0 / a.Lp;
-  int j = k0 - span * a.Lp;
-  int kh = span % a.kH;
-  int kd = span / a.kH;
+  int j = pos.j, kh = pos.kh, kd = pos.kd;
   long long rowptr;
   bool rok = gather_span(a, st, kd, kh, rowptr);
   rowptr += static_cast<long long>(st.iw0) * a.C;
   // phase 1: issue every load of the four chunks (aligned 16-byte blocks that
   // cover the chunk; the halo and the row ends are masked afterwards)
-  uint4 b0[4], b1[4];
-  unsigned hsh[4], msk[4];
+  uint4 b0[NCH], b1[NCH];
+  unsigned hsh[NCH], msk[NCH];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < NCH; ++q) {
     b0[q] = make_uint4(0, 0, 0, 0);
     b1[q] = make_uint4(0, 0, 0, 0);
     hsh[q] = 0;
@@ -442,47 +483,70 @@ __device__ __forceinline__ void gather_a_span(const TcArgs& a, const GatherRow& 
       rowptr += static_cast<long long>(st.iw0) * a.C;
     }
   }
+  pos.j = j;
+  pos.kh = kh;
+  pos.kd = kd;
   // phase 2: shift into place, mask, store
 #pragma unroll
-  for (int q = 0; q < 4; ++q) store_chunk(a_tile, r, chunk0 + q, mask8(extract8(b0[q], b1[q], hsh[q]), msk[q]));
+  for (int q = 0; q < NCH; ++q) store_chunk(a_tile, r, chunk0 + q, mask8(extract8(b0[q], b1[q], hsh[q]), msk[q]));
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
 }
 
 // GATHER_ROWS: the same span layout as gather_a_span, read from the input
 // rows staged in shared memory.  `rows` is the staging buffer of this tile,
-// seg_n / seg_lo its segments (image, first staged input row).
-__device__ __forceinline__ void gather_a_rows(const TcArgs& a, const GatherRow& st, int n, const uint8_t* rows,
-                                              const int* seg_n, const int* seg_lo, int k0, uint8_t* a_tile, int r,
-                                              int chunk0) {
-  const int span = k0 / a.Lp;
-  int j = k0 - span * a.Lp;
-  int kh = span % a.kH;
-  // the staged row holding filter row kh of this output pixel (or none)
-  const auto row_base = [&](int khh, bool& ok) -> const uint8_t* {
+// seg_n / seg_lo its segments (image, first staged input row).  A chunk that
+// lies wholly inside the row is five aligned 32-bit loads shifted into place
+// (its first element may be odd); chunks at the image edge take element loads.
+template <int NCH>
+__device__ __forceinline__ void gather_a_rows(const TcArgs& a, const GatherRow& st, SpanPos& pos, uint8_t* a_tile,
+                                              int r, int chunk0) {
+  int j = pos.j, kh = pos.kh;
+  const bool in_k = pos.kd < a.kD;  // false in the zero padding after the last filter row
+  // byte address of the staged row holding filter row kh of this output pixel (or none)
+  const auto row_base = [&](int khh, bool& ok) -> uint32_t {
     const int ih = st.ih0 + khh * a.dh;
-    const int seg = (n == seg_n[0]) ? 0 : 1;
-    const int lr = ih - seg_lo[seg];
-    ok = st.valid && khh < a.kH && static_cast<unsigned>(ih) < static_cast<unsigned>(a.H) &&
+    const int lr = st.lr0 + khh * a.dh;
+    ok = st.valid && in_k && khh < a.kH && static_cast<unsigned>(ih) < static_cast<unsigned>(a.H) &&
          static_cast<unsigned>(lr) < static_cast<unsigned>(a.stage_rows);
-    return rows + seg * a.seg_bytes + static_cast<uint32_t>(lr) * static_cast<uint32_t>(a.row_e) * 2u;
+    return st.rseg + static_cast<uint32_t>(lr) * static_cast<uint32_t>(a.row_e) * 2u;
   };
   bool rok;
-  const uint8_t* rb = row_base(kh, rok);
+  uint32_t rb = row_base(kh, rok);
   const int ebase = st.iw0 * a.C;  // element of x[n, ih, iw0, 0] within the row (may be negative)
-  uint4 v[4];
+  uint4 v[NCH];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < NCH; ++q) {
     v[q] = make_uint4(0, 0, 0, 0);
     if (rok && j + 8 > st.jlo && j < st.jhi) {
-      const int lo = max(st.jlo - j, 0), hi = min(st.jhi - j, 8);
-      const int e0 = ebase + j;           // >= 0 whenever some element is valid
-      const int blk = e0 >> 3;            // aligned 8-element block holding e0 (floor, also for e0 < 0)
-      const unsigned h = static_cast<unsigned>(e0 - blk * 8);
-      // blocks blk and blk + 1; a block before the row start reads as zeros
-      uint4 b0 = make_uint4(0, 0, 0, 0), b1 = make_uint4(0, 0, 0, 0);
-      if (blk >= 0) b0 = *reinterpret_cast<const uint4*>(rb + blk * 16);
-      if (blk + 1 >= 0 && (blk + 1) * 8 < a.row_e) b1 = *reinterpret_cast<const uint4*>(rb + (blk + 1) * 16);
-      const unsigned m = ((1u << hi) - 1u) & ~((1u << lo) - 1u);
-      v[q] = mask8(extract8(b0, b1, h), m);
+      if (j >= st.jlo && j + 8 <= st.jhi) {
+        // all eight elements exist: element e0 >= 0
+        const int e0 = ebase + j;
+        const uint32_t addr = rb + static_cast<uint32_t>(e0 & ~1) * 2u;
+        const uint32_t sh = static_cast<uint32_t>(e0 & 1) * 16u;
+        const uint32_t w0 = lds32(addr), w1 = lds32(addr + 4), w2 = lds32(addr + 8), w3 = lds32(addr + 12),
+                       w4 = lds32(addr + 16);
+        v[q] = make_uint4(__funnelshift_r(w0, w1, sh), __funnelshift_r(w1, w2, sh), __funnelshift_r(w2, w3, sh),
+                          __funnelshift_r(w3, w4, sh));
+      } else {
+        uint32_t h[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int jj = j + i;
+          h[i] = (jj >= st.jlo && jj < st.jhi) ? lds16(rb + static_cast<uint32_t>(ebase + jj) * 2u) : 0u;
+        }
+        v[q] = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+      }
     }
     j += 8;
     if (j == a.Lp) {
@@ -491,14 +555,17 @@ __device__ __forceinline__ void gather_a_rows(const TcArgs& a, const GatherRow& 
       rb = row_base(kh, rok);
     }
   }
+  pos.j = j;
+  pos.kh = kh;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) store_chunk(a_tile, r, chunk0 + q, v[q]);
+  for (int q = 0; q < NCH; ++q) store_chunk(a_tile, r, chunk0 + q, v[q]);
 }
 
+template <int NCH>
 __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
                                                 int r, int chunk0) {
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
-  uint32_t v[32];
+  uint32_t v[8 * NCH];
   const int tap = k0 / a.Cg;
   int c = k0 - tap * a.Cg;
   int kw = tap % a.kW;
@@ -508,7 +575,7 @@ __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow
   long long rowptr;
   bool ok = gather_span(a, st, kd, kh, rowptr);
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
+  for (int e = 0; e < 8 * NCH; ++e) {
     const int iw = st.iw0 + kw * a.dw;
     v[e] = (ok && static_cast<unsigned>(iw) < static_cast<unsigned>(a.W))
                ? __ldg(x + rowptr + static_cast<long long>(iw) * a.C + c)
@@ -526,7 +593,7 @@ __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow
     }
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
+  for (int q = 0; q < NCH; ++q)
     store_chunk(a_tile, r, chunk0 + q,
                 make_uint4(v[8 * q] | (v[8 * q + 1] << 16), v[8 * q + 2] | (v[8 * q + 3] << 16),
                            v[8 * q + 4] | (v[8 * q + 5] << 16), v[8 * q + 6] | (v[8 * q + 7] << 16)));
@@ -728,7 +795,12 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
     } else {
       const int tid = threadIdx.x;  // 0 .. kProdThreads-1
       const int r = tid & 127;      // A row
-      const int half = tid >> 7;    // which 32 of the 64 K elements of a stage
+      // which 16 of the 64 K elements of every K block this thread builds
+      // (16 producer warps: enough threads in flight to hide each chunk's
+      // dependent address, load and shift chain)
+      constexpr int kParts = kProdThreads / kBM;
+      constexpr int kNch = 8 / kParts;  // 8-element chunks per thread per K block
+      const int part = tid >> 7;
       if (a.b_resident) {
         // the whole B matrix, once per CTA: [kblock][BN rows][128 B]
         for (int kb = 0; kb < a.kblocks; ++kb)
@@ -763,6 +835,13 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
         st.jlo = max(0, -st.iw0) * a.C;
         st.jhi = min(a.kW, a.W - st.iw0) * a.C;
         if (st.jhi < st.jlo) st.jhi = st.jlo;
+        if (rows_mode) {
+          const int seg = (n == tail->seg_n[rb][0]) ? 0 : 1;
+          st.rseg = ptx::smem_u32(rowsbuf + rb * a.rows_bytes) + static_cast<uint32_t>(seg) * a.seg_bytes;
+          st.lr0 = st.ih0 - tail->seg_lo[rb][seg];
+        }
+        // this thread's first K element of every 64-wide K block
+        SpanPos pos = span_pos(a, part * kNch * 8);
         const int n0 = tc.nt * a.BN;
         for (int kb = 0; kb < a.kblocks; kb += a.kbs) {
           const int nsub = min(a.kbs, a.kblocks - kb);
@@ -773,16 +852,16 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
           }
           for (int j = 0; j < nsub; ++j) {
             uint8_t* sa = smem + stage * a.stage_bytes + j * a.sub_bytes;
-            const int k0 = (kb + j) * 64 + half * 32;
+            const int k0 = (kb + j) * 64 + part * kNch * 8;
             if (a.gather_mode == GATHER_VEC8)
-              gather_a_vec8(a, st, k0, sa, r, half * 4);
-            else if (rows_mode)
-              gather_a_rows(a, st, n, rowsbuf + rb * a.rows_bytes, tail->seg_n[rb], tail->seg_lo[rb], k0, sa, r,
-                            half * 4);
-            else if (a.gather_mode == GATHER_SPAN)
-              gather_a_span(a, st, k0, sa, r, half * 4);
-            else
-              gather_a_scalar(a, st, k0, sa, r, half * 4);
+              gather_a_vec8<kNch>(a, st, k0, sa, r, part * kNch);
+            else if (rows_mode || a.gather_mode == GATHER_SPAN) {
+              if (rows_mode) gather_a_rows<kNch>(a, st, pos, sa, r, part * kNch);
+              else gather_a_span<kNch>(a, st, pos, sa, r, part * kNch);
+              // skip the other threads' chunks of this K block
+              for (int i = 0; i < 8 - kNch; ++i) span_step8(a, pos);
+            } else
+              gather_a_scalar<kNch>(a, st, k0, sa, r, part * kNch);
             if (!a.b_resident) gather_b_block(a, tc.g, n0, (kb + j) * 64, sa + a.a_bytes, tid, kProdThreads);
           }
           ptx::fence_proxy_async_smem();
