@@ -92,6 +92,16 @@ def kernel_source_hash():
     return h.hexdigest()[:12]
 
 
+def simt_tile(wl, dims, bn, ctas):
+    """[pixels, channels] of the SIMT kernel's tile: BN from the plan, BM (64 or
+    128) from the number of CTAs it launches."""
+    M = wl.N * dims[0] * dims[1] * dims[2]
+    og = wl.O // wl.groups
+    n_tiles = -(-og // bn) * wl.groups
+    m_tiles = ctas // max(n_tiles, 1)
+    return [128 if m_tiles == -(-M // 128) else 64, bn]
+
+
 def profiled_traffic(workload, variant_name):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel source (else None)."""
@@ -406,7 +416,7 @@ def bench_ours(args):
                    "groups": wl.groups, "out_DHW": list(dims), "gflop_per_step": round(flops / 1e9, 4),
                    "global_batch": wl.N * nranks, "parallelism": f"independent batches x{nranks}",
                    "variant": vname,
-                   "tile": ([64, 64] if variant == C.VARIANT_SIMT else
+                   "tile": (simt_tile(wl, dims, bn, ctas) if variant == C.VARIANT_SIMT else
                             [bn, 128] if variant in (C.VARIANT_TC_TMA_T, C.VARIANT_TC_HALO_T)
                             else [bn, 256] if variant == C.VARIANT_TC_HALO_T_PAIR
                             else [256 if "pair" in vname else 128, bn]),

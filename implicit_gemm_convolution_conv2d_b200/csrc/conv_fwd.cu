@@ -874,7 +874,44 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
   return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
 
-int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st) {
+// SIMT tile shape: TN (channels per thread, BN = 16*TN) from {2, 4, 5, 6, 8}
+// wasting the fewest padded channels of O/G (ties to the wider tile); TM = 4
+// (64-pixel tiles: at most 128 registers, two CTAs per SM; 128-pixel tiles
+// measured slower on B200 at 170-255 registers).  f16/bf16 (a cross-check
+// path) use the 4 x 4 shape only.
+struct SimtShape {
+  int tm, tn;
+};
+
+SimtShape simt_shape(const Problem& P, int sms) {
+  SimtShape sh{4, 4};
+  if (P.dtype != CONV_F32) return sh;
+  static const int kTns[5] = {8, 6, 5, 4, 2};
+  long long best = -1;
+  for (int tn : kTns) {
+    const long long padded = static_cast<long long>((P.Og + 16 * tn - 1) / (16 * tn)) * 16 * tn;
+    if (best < 0 || padded < best) {
+      best = padded;
+      sh.tn = tn;
+    }
+  }
+  (void)sms;
+  return sh;
+}
+
+template <typename T, int TM>
+cudaError_t launch_simt_tn(int tn, dim3 grid, cudaStream_t st, const SimtArgs& a) {
+  switch (tn) {
+    case 2: conv_fwd_simt_kernel<T, TM, 2><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 5: conv_fwd_simt_kernel<T, TM, 5><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 6: conv_fwd_simt_kernel<T, TM, 6><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 8: conv_fwd_simt_kernel<T, TM, 8><<<grid, kSimtThreads, 0, st>>>(a); break;
+    default: conv_fwd_simt_kernel<T, TM, 4><<<grid, kSimtThreads, 0, st>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
+int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st, int sms) {
   SimtArgs a;
   a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.C = P.C; a.O = P.O;
   a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
@@ -885,14 +922,22 @@ int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStr
   a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
   a.M = P.M; a.K = static_cast<int>(P.K);
   a.x = x; a.w = w; a.y = y;
-  const long long mt = (P.M + kSimtBM - 1) / kSimtBM;
-  const int nt = (P.Og + kSimtBN - 1) / kSimtBN;
+  const SimtShape sh = simt_shape(P, sms);
+  const long long mt = (P.M + 16 * sh.tm - 1) / (16 * sh.tm);
+  const long long nt = (P.Og + 16 * sh.tn - 1) / (16 * sh.tn);
   if (mt > 0x7fffffffLL || nt > 65535 || P.G > 65535) return CONV_EUNSUPPORTED;
-  const dim3 grid(static_cast<unsigned>(mt), nt, P.G), block(kSimtThreads);
-  if (P.dtype == CONV_F32) conv_fwd_simt_kernel<float><<<grid, block, 0, st>>>(a);
-  else if (P.dtype == CONV_F16) conv_fwd_simt_kernel<__half><<<grid, block, 0, st>>>(a);
-  else conv_fwd_simt_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+  const dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>(nt), P.G);
+  cudaError_t e;
+  if (P.dtype == CONV_F32) {
+    e = launch_simt_tn<float, 4>(sh.tn, grid, st, a);
+  } else if (P.dtype == CONV_F16) {
+    conv_fwd_simt_kernel<__half, 4, 4><<<grid, kSimtThreads, 0, st>>>(a);
+    e = cudaGetLastError();
+  } else {
+    conv_fwd_simt_kernel<__nv_bfloat16, 4, 4><<<grid, kSimtThreads, 0, st>>>(a);
+    e = cudaGetLastError();
+  }
+  return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
 
 int run(const Problem& P, const void* x, const void* w, void* y, int variant, cudaStream_t st) {
@@ -903,7 +948,7 @@ int run(const Problem& P, const void* x, const void* w, void* y, int variant, cu
   rc = device_sms(dev, sms);
   if (rc != CONV_OK) return rc;
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
-  if (variant == CONV_VARIANT_SIMT) return launch_simt(P, x, w, y, st);
+  if (variant == CONV_VARIANT_SIMT) return launch_simt(P, x, w, y, st, sms);
   TcPlan plan;
   rc = plan_tc(P, variant, sms, plan);
   if (rc != CONV_OK) return rc;
@@ -972,11 +1017,12 @@ int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, 
   if (current_device(dev) == CONV_OK) device_sms(dev, sms);
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
   if (variant == CONV_VARIANT_SIMT) {
-    if (bn) *bn = kSimtBN;
-    if (stages) *stages = 1;
+    const SimtShape sh = simt_shape(P, sms);
+    if (bn) *bn = 16 * sh.tn;
+    if (stages) *stages = 2;
     if (ctas) {
-      const long long mt = (P.M + kSimtBM - 1) / kSimtBM;
-      const long long c = mt * ((P.Og + kSimtBN - 1) / kSimtBN) * P.G;
+      const long long mt = (P.M + 16 * sh.tm - 1) / (16 * sh.tm);
+      const long long c = mt * ((P.Og + 16 * sh.tn - 1) / (16 * sh.tn)) * P.G;
       *ctas = static_cast<int>(std::min<long long>(c, 0x7fffffffLL));
     }
     return variant;

@@ -6,10 +6,10 @@
 // path for fp32 tensors: TF32 tensor cores would round every input to 10
 // mantissa bits, far outside a 1e-5 relative bound.
 //
-// Tile 64 pixels x 64 channels x 16 K per step, 256 threads, 4x4 outputs per
-// thread.  Each 16-wide K step is summed into a fresh partial that is then
-// added to the running total (two-level summation), which bounds the rounding
-// error by about (16 + K/16) units in the last place of sum|x*w| instead of K.
+// Tiles of (16*TM) pixels x (16*TN) channels x 16 K per step, 256 threads.
+// Each 16-wide K step is summed into a fresh partial that is then added to the
+// running total (two-level summation), which bounds the rounding error by
+// about (16 + K/16) units in the last place of sum|x*w| instead of K.
 #pragma once
 
 #include <cstdint>
@@ -49,12 +49,19 @@ __device__ __forceinline__ __half from_f32<__half>(float v) { return __float2hal
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
 
-constexpr int kSimtBM = 64, kSimtBN = 64, kSimtBK = 16, kSimtThreads = 256;
+constexpr int kSimtBK = 16, kSimtThreads = 256;
 
-template <typename T>
+// Thread (ty, tx) of a 16 x 16 grid owns output rows (pixels) ty*TM .. ty*TM+TM-1
+// of the tile and output channels tx + 16*j, j < TN; the tile is BM = 16*TM
+// pixels x BN = 16*TN channels.  BN is chosen on the host to fit O/G (32, 64,
+// 80, 96 or 128), so layers like O = 65 or 21 do not compute mostly padding.
+// Loads of the next K step go to registers before the current step's FMAs and
+// to the other shared-memory buffer after them: one barrier per step.
+template <typename T, int TM, int TN>
 __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtArgs a) {
-  __shared__ __align__(16) float As[kSimtBK][kSimtBM + 4];
-  __shared__ __align__(16) float Bs[kSimtBK][kSimtBN + 4];
+  constexpr int BM = 16 * TM, BN = 16 * TN;
+  __shared__ __align__(16) float As[2][kSimtBK][BM + 4];
+  __shared__ __align__(16) float Bs[2][kSimtBK][BN + 4];
 
   const T* __restrict__ x = static_cast<const T*>(a.x);
   const T* __restrict__ w = static_cast<const T*>(a.w);
@@ -62,18 +69,18 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
 
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
-  const long long m0 = static_cast<long long>(blockIdx.x) * kSimtBM;
-  const int n0 = blockIdx.y * kSimtBN;
+  const long long m0 = static_cast<long long>(blockIdx.x) * BM;
+  const int n0 = blockIdx.y * BN;
   const int g = blockIdx.z;
 
-  // loader roles: element (kl, row) with kl = tid & 15, row = (tid >> 4) + 16 i
-  const int kl = tid & 15;
-  bool rvalid[4];
-  long long rbase[4];
-  int rd0[4], rh0[4], rw0[4];
+  // loader roles: K element kl = tid & 15 of rows (tid >> 4) + 16 i
+  const int kl = tid & 15, lr = tid >> 4;
+  bool rvalid[TM];
+  long long rbase[TM];
+  int rd0[TM], rh0[TM], rw0[TM];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const long long m = m0 + (tid >> 4) + 16 * i;
+  for (int i = 0; i < TM; ++i) {
+    const long long m = m0 + lr + 16 * i;
     rvalid[i] = m < a.M;
     const long long mm = rvalid[i] ? m : 0;
     const int ow = static_cast<int>(mm % a.Wo);
@@ -87,6 +94,14 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
     rh0[i] = oh * a.sh - a.ph;
     rw0[i] = ow * a.sw - a.pw;
   }
+  const T* wrow[TN];
+  bool ovalid[TN];
+#pragma unroll
+  for (int j = 0; j < TN; ++j) {
+    const int o = n0 + lr + 16 * j;
+    ovalid[j] = o < a.Og;
+    wrow[j] = w + static_cast<long long>(g * a.Og + (ovalid[j] ? o : 0)) * a.K;
+  }
   // carried decode of k = k0 + kl into (kd, kh, kw, c)
   int c = kl, kw = 0, kh = 0, kd = 0;
   while (c >= a.Cg) {
@@ -94,75 +109,92 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
     if (++kw == a.kW) { kw = 0; if (++kh == a.kH) { kh = 0; ++kd; } }
   }
 
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-
-  for (int k0 = 0; k0 < a.K; k0 += kSimtBK) {
+  float ra[TM], rb[TN];
+  const auto load_step = [&](int k0) {
     const int k = k0 + kl;
-    // A tile
+    const bool kv = k < a.K;
+    const int id = kd * a.dd, ih = kh * a.dh, iw = kw * a.dw;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < TM; ++i) {
       float v = 0.f;
-      if (rvalid[i] && k < a.K) {
-        const int id = rd0[i] + kd * a.dd, ih = rh0[i] + kh * a.dh, iw = rw0[i] + kw * a.dw;
-        if (static_cast<unsigned>(id) < static_cast<unsigned>(a.D) &&
-            static_cast<unsigned>(ih) < static_cast<unsigned>(a.H) &&
-            static_cast<unsigned>(iw) < static_cast<unsigned>(a.W))
-          v = to_f32<T>(x[rbase[i] + ((static_cast<long long>(id) * a.H + ih) * a.W + iw) * a.C + c]);
-      }
-      As[kl][(tid >> 4) + 16 * i] = v;
-    }
-    // B tile
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int o = n0 + (tid >> 4) + 16 * i;
-      float v = 0.f;
-      if (o < a.Og && k < a.K)
-        v = to_f32<T>(w[static_cast<long long>(g * a.Og + o) * a.K + k]);
-      Bs[kl][(tid >> 4) + 16 * i] = v;
-    }
-    __syncthreads();
-
-    float part[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) part[i][j] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < kSimtBK; ++kk) {
-      const float4 av = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-      const float ar[4] = {av.x, av.y, av.z, av.w};
-      const float br[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(ar[i], br[j], part[i][j]);
+      const int zd = rd0[i] + id, zh = rh0[i] + ih, zw = rw0[i] + iw;
+      if (rvalid[i] && kv && static_cast<unsigned>(zd) < static_cast<unsigned>(a.D) &&
+          static_cast<unsigned>(zh) < static_cast<unsigned>(a.H) &&
+          static_cast<unsigned>(zw) < static_cast<unsigned>(a.W))
+        v = to_f32<T>(x[rbase[i] + ((static_cast<long long>(zd) * a.H + zh) * a.W + zw) * a.C + c]);
+      ra[i] = v;
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
-    __syncthreads();
-
+    for (int j = 0; j < TN; ++j) rb[j] = (ovalid[j] && kv) ? to_f32<T>(wrow[j][k]) : 0.f;
     // advance the carried decode by one K step
     c += kSimtBK;
     while (c >= a.Cg) {
       c -= a.Cg;
       if (++kw == a.kW) { kw = 0; if (++kh == a.kH) { kh = 0; ++kd; } }
     }
+  };
+  const auto store_step = [&](int buf) {
+#pragma unroll
+    for (int i = 0; i < TM; ++i) As[buf][kl][lr + 16 * i] = ra[i];
+#pragma unroll
+    for (int j = 0; j < TN; ++j) Bs[buf][kl][lr + 16 * j] = rb[j];
+  };
+
+  float acc[TM][TN];
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+
+  load_step(0);
+  store_step(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < a.K; k0 += kSimtBK) {
+    const bool more = k0 + kSimtBK < a.K;
+    if (more) load_step(k0 + kSimtBK);  // global loads in flight during the FMAs below
+    float part[TM][TN];
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) part[i][j] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < kSimtBK; ++kk) {
+      float ar[TM], br[TN];
+#pragma unroll
+      for (int i = 0; i < TM; i += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(&As[buf][kk][ty * TM + i]);
+        ar[i] = v.x;
+        ar[i + 1] = v.y;
+        ar[i + 2] = v.z;
+        ar[i + 3] = v.w;
+      }
+#pragma unroll
+      for (int j = 0; j < TN; ++j) br[j] = Bs[buf][kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) part[i][j] = fmaf(ar[i], br[j], part[i][j]);
+    }
+    // two-level summation: each 16-wide K step is summed apart, then added
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) acc[i][j] += part[i][j];
+    if (more) {
+      store_step(buf ^ 1);
+      __syncthreads();
+      buf ^= 1;
+    }
   }
 
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const long long m = m0 + ty * 4 + i;
+  for (int i = 0; i < TM; ++i) {
+    const long long m = m0 + ty * TM + i;
     if (m >= a.M) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int o = n0 + tx * 4 + j;
+    for (int j = 0; j < TN; ++j) {
+      const int o = n0 + tx + 16 * j;
       if (o < a.Og) y[m * a.O + static_cast<long long>(g) * a.Og + o] = from_f32<T>(acc[i][j]);
     }
   }
