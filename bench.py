@@ -355,6 +355,26 @@ def bench_ours(args):
     ms_per_step = ms / args.steps
     value = nranks * flops * args.steps / (ms * 1e-3) / 1e12
 
+    # ---- per-launch distribution (each launch between its own events, after
+    # the timed region): cold L2 (rotating buffer sets) and warm L2 (one set)
+    n_dist = max(5, min(args.steps, 50))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_dist + 1)]
+    evs[0].record(stream)
+    for i in range(n_dist):
+        step(i)
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    cold = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(n_dist))
+    evs[0].record(stream)
+    for i in range(n_dist):
+        step(0)
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    warm = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(n_dist))
+    launch_dist = {"n": n_dist, "median_ms": round(cold[n_dist // 2], 5), "min_ms": round(cold[0], 5),
+                   "warm_l2_median_ms": round(warm[n_dist // 2], 5), "warm_l2_min_ms": round(warm[0], 5),
+                   "how": "eager launches, one event pair each, after the timed region"}
+
     # ---- end to end through the host-buffer C entry point (pinned host memory)
     e2e = None
     if not args.no_e2e:
@@ -403,6 +423,7 @@ def bench_ours(args):
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(gbs / peak, 4), "peak_source": f"{peak_src} copy bandwidth (hbm_gbs)"}
     roof["traffic"] = profiled_traffic(args.workload, vname)
+    roof["launch_distribution"] = launch_dist
     roof["kernel"] = vname
     roof["ms_per_launch"] = round(kern_ms, 5)
 
@@ -465,8 +486,32 @@ def cpu_baseline(wl, budget_s=15.0):
         total_t += time.perf_counter() - t0
         total_f += f1 * k
         n_img += k
-    return {"value": round(total_f / total_t / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
-            "kind": "oracle", "sample": f"first {n_img} of {wl.N} images of {wl.name} ({total_t:.1f} s)"}
+    out = {"value": round(total_f / total_t / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+           "kind": "oracle", "sample": f"first {n_img} of {wl.N} images of {wl.name} ({total_t:.1f} s)"}
+    out["single_thread"] = _oracle_single_thread(wl, x, w)
+    return out
+
+
+def _oracle_single_thread(wl, x, w, max_flops=3e9):
+    """The oracle on one host thread: the full direct loop over the first image,
+    its depth halved (3-D) until the work is about `max_flops` or the depth is
+    down to 4 (FLOPs count every tap, as everywhere in this file, so a thinner
+    slab would count mostly padding taps)."""
+    import oracle
+    sub = wl.with_(N=1)
+    while conv_flops(sub) > max_flops and sub.D > 4:
+        sub = sub.with_(D=(sub.D + 1) // 2)
+    xs = x[:1, :sub.D].contiguous()
+    full = oracle.max_threads()
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.conv_fwd(xs, w, sub.stride, sub.pad, sub.dil, sub.groups)
+        dt = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(full)
+    return {"value": round(conv_flops(sub) / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+            "sample": f"image 0 of {wl.name}, depth {sub.D} of {wl.D} ({dt:.1f} s)"}
 
 
 def bench_reference(args):
