@@ -438,7 +438,8 @@ def bench_ours(args):
                    "global_batch": wl.N * nranks, "parallelism": f"independent batches x{nranks}",
                    "variant": vname,
                    "tile": (simt_tile(wl, dims, bn, ctas) if variant == C.VARIANT_SIMT else
-                            [bn, 128] if variant in (C.VARIANT_TC_TMA_T, C.VARIANT_TC_HALO_T)
+                            [bn, 128] if variant == C.VARIANT_TC_TMA_T
+                            else [bn, 128 if (wl.O // wl.groups) % 128 == 0 else 64] if variant == C.VARIANT_TC_HALO_T
                             else [bn, 256] if variant == C.VARIANT_TC_HALO_T_PAIR
                             else [256 if "pair" in vname else 128, bn]),
                    "stages": stages, "ctas": ctas,

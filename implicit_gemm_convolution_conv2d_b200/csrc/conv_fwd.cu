@@ -266,19 +266,17 @@ bool tma_fits(const Problem& P, bool& rank5) {
   return true;
 }
 
-// Can the halo kernel run this problem?  Stride 1, 64-channel chunks, the
-// halo box inside the TMA box limits (256 per dimension), rank 4 or 5.
+// Can the plain-orientation halo kernel run this problem?  Stride 1, channel
+// chunks of 64 or 32, the strip box inside the TMA box limits (256 per
+// dimension), rank 4 or 5.
 constexpr int kHaloTileH = 16, kHaloTileW = 8;
 
 bool halo_fits(const Problem& P, bool& rank5) {
-  if (P.dtype == CONV_F32 || P.Cg % 64 != 0) return false;
+  if (P.dtype == CONV_F32 || P.Cg % 32 != 0) return false;
   if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1) return false;
-  if (P.kH * P.kW < 4) return false;  // too few taps share a halo box to pay for it
   rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
-  const long long hw = kHaloTileW + static_cast<long long>(P.d[2]) * (P.kW - 1);
   const long long hh = kHaloTileH + static_cast<long long>(P.d[1]) * (P.kH - 1);
-  if (hw > 256 || hh > 256) return false;
-  if (hw * hh * 128 > 64 * 1024) return false;  // two slots must leave room for the weight ring
+  if (hh > 256) return false;
   if (P.N > 0x3fffffff) return false;
   return true;
 }
@@ -307,26 +305,32 @@ int plan_halo(const Problem& P, bool pair, int sms, TcPlan& plan) {
   if (tt > 0x7fffffffLL) return CONV_EINVAL;
   a.total_tiles = static_cast<int>(tt);
   a.m_tiles = 0;
-  a.halo_w = kHaloTileW + P.d[2] * (P.kW - 1);
-  a.halo_h = kHaloTileH + P.d[1] * (P.kH - 1);
-  a.halo_bytes = static_cast<uint32_t>(a.halo_w * a.halo_h * 128);
-  a.halo_slot_bytes = (a.halo_bytes + 1023u) & ~1023u;
-  a.a_slots = 2;
-  a.kc = 64;
-  a.cchunks = P.Cg / 64;
+  a.kc = (P.Cg % 64 == 0) ? 64 : 32;
+  a.cchunks = P.Cg / a.kc;
   a.kblocks = P.kD * P.kH * P.kW * a.cchunks;
   a.rank5 = rank5 ? 1 : 0;
-  a.layout_type = 2u;
-  a.sbo = 1024u;
+  a.layout_type = a.kc == 64 ? 2u : 4u;    // 128-byte or 64-byte swizzle
+  a.sbo = static_cast<uint32_t>(8 * a.kc * 2);  // one 8-row atom = one strip row of 8 pixels
+  // one strip per (chunk, kd, kw): (16 + dh*(kH-1)) rows x 8 pixels x kc channels
+  a.halo_w = kHaloTileW;
+  a.halo_h = kHaloTileH + P.d[1] * (P.kH - 1);
+  a.halo_bytes = static_cast<uint32_t>(a.halo_w * a.halo_h * a.kc * 2);
+  a.halo_slot_bytes = (a.halo_bytes + 1023u) & ~1023u;
   a.a_bytes = 0;
-  a.b_bytes = static_cast<uint32_t>((pair ? a.BN / 2 : a.BN) * 128);
+  a.b_bytes = static_cast<uint32_t>((pair ? a.BN / 2 : a.BN) * a.kc * 2);
   a.sub_bytes = a.b_bytes;
-  const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64 -
-                          static_cast<long long>(a.a_slots) * a.halo_slot_bytes;
+  // the weight and strip rings are independent (a stage may span any number of
+  // strip groups): first up to three weight stages beside two strip slots,
+  // then as many more strip slots (up to 8) as the rest of shared memory holds
+  // -- one strip serves only kH K blocks, so its load latency needs a deep ring
+  const long long budget = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64;
   int stages = 0;
-  // a stage may span at most two (chunk, kd) halo groups: kbs <= kH*kW
-  a.kbs = choose_kbs(a.BN, 64, a.b_bytes, avail, std::min(8, P.kH * P.kW), stages);
+  a.kbs = choose_kbs(a.BN, a.kc, a.b_bytes, budget - 2LL * a.halo_slot_bytes, 16, stages);
   if (stages < 2) return CONV_EUNSUPPORTED;
+  stages = std::min(stages, 3);
+  const long long left = budget - static_cast<long long>(stages) * a.kbs * a.b_bytes;
+  a.a_slots = static_cast<int>(std::min<long long>(8, left / a.halo_slot_bytes));
+  if (a.a_slots < 2) return CONV_EUNSUPPORTED;
   a.stages = stages;
   a.stage_bytes = static_cast<uint32_t>(a.kbs) * a.b_bytes;
   const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
@@ -403,8 +407,12 @@ int plan_tc_t(const Problem& P, int sms, TcPlan& plan) {
 // O/G % 128 == 0.  With `pair`, two CTAs issue M = 256 (128 output channels
 // each) over the same block; each loads the strip of half the block's rows.
 int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
-  const int o_tile = pair ? 2 * kTO : kTO;
-  if (P.dtype == CONV_F32 || P.Cg % 64 != 0 || P.Og % o_tile != 0) return CONV_EUNSUPPORTED;
+  // output channels per CTA: 128, or 64 when O/G is an odd multiple of 64
+  // (an M = 64 instruction takes as long as M = 128 on B200, so 64 only when
+  // 128 does not divide O/G); channel chunks of 64, or 32
+  const int mo = (P.Og % kTO == 0 || pair) ? kTO : 64;
+  const int o_tile = pair ? 2 * mo : mo;
+  if (P.dtype == CONV_F32 || P.Cg % 32 != 0 || P.Og % o_tile != 0) return CONV_EUNSUPPORTED;
   if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1) return CONV_EUNSUPPORTED;
   if (P.N > 0x3fffffff) return CONV_EUNSUPPORTED;
   const bool rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
@@ -447,30 +455,31 @@ int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
   a.m_tiles = 0;
   a.halo_w = static_cast<int>(hw);
   a.halo_h = static_cast<int>(hh);
-  a.halo_bytes = static_cast<uint32_t>(hw * hh * 128);
+  a.kc = (P.Cg % 64 == 0) ? 64 : 32;
+  a.halo_bytes = static_cast<uint32_t>(hw * hh * a.kc * 2);
   a.halo_slot_bytes = (a.halo_bytes + 1023u) & ~1023u;
   a.a_slots = 2;
-  a.kc = 64;
-  a.cchunks = P.Cg / 64;
+  a.mo = mo;
+  a.cchunks = P.Cg / a.kc;
   a.kblocks = P.kD * P.kH * P.kW * a.cchunks;
   a.rank5 = rank5 ? 1 : 0;
-  a.layout_type = 2u;
-  a.sbo = 1024u;
+  a.layout_type = a.kc == 64 ? 2u : 4u;          // 128-byte or 64-byte swizzle
+  a.sbo = static_cast<uint32_t>(8 * a.kc * 2);  // one atom = one strip row of 8 pixels
   a.a_bytes = 0;
-  a.b_bytes = static_cast<uint32_t>(kTO * 128);  // one weight tile: 128 channels x 64 K
+  a.b_bytes = static_cast<uint32_t>(mo * a.kc * 2);  // one weight tile: mo channels x kc
   a.sub_bytes = a.b_bytes;
-  // strip slots: three when three weight stages still fit beside them (the
-  // strip producer then runs two groups ahead), else two
+  // the weight and strip rings are independent: first up to three weight
+  // stages beside two strip slots, then as many more strip slots (up to 8) as
+  // the rest of shared memory holds
+  const long long budget = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
+                           64 - 2LL * kTEpiBytes;
   int stages = 0;
-  for (int slots = 3; slots >= 2; --slots) {
-    const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
-                            64 - 2LL * kTEpiBytes - static_cast<long long>(slots) * a.halo_slot_bytes;
-    if (avail <= 0) continue;
-    a.a_slots = slots;
-    a.kbs = choose_kbs(a.BN, 64, a.b_bytes, avail, std::min(8, P.kH), stages);
-    if (stages >= 3 || slots == 2) break;
-  }
+  a.kbs = choose_kbs(a.BN, a.kc, a.b_bytes, budget - 2LL * a.halo_slot_bytes, 16, stages);
   if (stages < 2) return CONV_EUNSUPPORTED;
+  stages = std::min(stages, 3);
+  const long long left = budget - static_cast<long long>(stages) * a.kbs * a.b_bytes;
+  a.a_slots = static_cast<int>(std::min<long long>(8, left / a.halo_slot_bytes));
+  if (a.a_slots < 2) return CONV_EUNSUPPORTED;
   a.stages = stages;
   a.stage_bytes = static_cast<uint32_t>(a.kbs) * a.b_bytes;
   const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
@@ -608,11 +617,11 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
 
 // f32 -> SIMT.  f16/bf16 -> TMA im2col when it can describe the problem,
 // else the in-kernel gather.  When the output channels per group come in
-// 128-wide tiles that a 256-wide one cannot cover (O/G = 128, 384, ...): the
-// transposed halo kernel at stride 1 with 64-channel chunks and kH >= 2 (each
-// input strip then serves kH taps) and a tile for every SM, else the
-// transposed im2col kernel when there are enough 256-pixel tiles for every
-// SM.  Otherwise CTA pairs once there are at least as many 256-row tiles as
+// 64- or 128-wide tiles that a 256-wide one cannot cover (O/G = 64, 128, 192,
+// 384, ...): the transposed halo kernel at stride 1 with 32- or 64-channel
+// chunks and kH >= 2 (each input strip then serves kH taps) and a tile for
+// every SM, else (O/G a multiple of 128) the transposed im2col kernel when
+// there are enough 256-pixel tiles for every SM.  Otherwise CTA pairs once there are at least as many 256-row tiles as
 // SM pairs, else single CTAs.  Every choice here is the fastest measured on
 // B200 for the shapes of the workload set; TC_HALO, TC_HALO_PAIR and
 // TC_HALO_T_PAIR stay explicit (slower there than the choice made here).
@@ -620,7 +629,7 @@ int choose_variant(const Problem& P, int sms) {
   if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
   bool r5;
   if (!tma_fits(P, r5)) return CONV_VARIANT_TC_GATHER;
-  if (P.Og % kTO == 0 && P.Og % 256 != 0 && P.kH >= 2) {
+  if (P.Og % 64 == 0 && P.Og % 256 != 0 && P.kH >= 2) {
     TcPlan hp;
     if (plan_halo_t(P, false, sms, hp) == CONV_OK && hp.args.total_tiles >= sms) return CONV_VARIANT_TC_HALO_T;
   }
@@ -655,8 +664,9 @@ int encode_y_map(const Problem& P, void* y, CUtensorMap& my) {
 }
 
 // y viewed as [N, (Do,) Ho, Wo, O] for the transposed halo kernel's TMA
-// stores: boxes of 128 channels x 8 columns x 4 rows, clipped at the edges.
-int encode_y_block_map(const Problem& P, bool rank5, void* y, CUtensorMap& my) {
+// stores: boxes of mo (64 or 128) channels x 8 columns x 4 rows, clipped at
+// the edges.
+int encode_y_block_map(const Problem& P, bool rank5, int mo, void* y, CUtensorMap& my) {
   std::memset(&my, 0, sizeof(my));
   const DriverFns& drv = driver_fns();
   if (!drv.tiled) return CONV_EDRIVER;
@@ -666,7 +676,7 @@ int encode_y_block_map(const Problem& P, bool rank5, void* y, CUtensorMap& my) {
   cuuint64_t dim[5] = {static_cast<cuuint64_t>(P.O), static_cast<cuuint64_t>(P.Wo), static_cast<cuuint64_t>(P.Ho),
                        static_cast<cuuint64_t>(rank5 ? P.Do : P.N), static_cast<cuuint64_t>(P.N)};
   cuuint64_t str[4] = {eb * P.O, eb * P.O * P.Wo, eb * P.O * P.Wo * P.Ho, eb * P.O * P.Wo * P.Ho * P.Do};
-  cuuint32_t box[5] = {static_cast<cuuint32_t>(kTO), static_cast<cuuint32_t>(kHTBlockW),
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(mo), static_cast<cuuint32_t>(kHTBlockW),
                        static_cast<cuuint32_t>(kTEpiRows / kHTBlockW), 1u, 1u};
   cuuint32_t est[5] = {1, 1, 1, 1, 1};
   const CUresult r = drv.tiled(&my, dt, rank5 ? 5 : 4, y, dim, str, box, est, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -731,11 +741,12 @@ int encode_maps(const Problem& P, const TcArgs& a, bool pair, bool halo, const v
   }
   CUresult r;
   if (halo) {
-    // a tiled box of 64 channels x halo_w x halo_h pixels (x 1 depth) x 1 image
-    cuuint32_t hbox[5] = {64u, static_cast<cuuint32_t>(a.halo_w), static_cast<cuuint32_t>(a.halo_h), 1u, 1u};
+    // a tiled box of kc channels x halo_w x halo_h pixels (x 1 depth) x 1 image
+    cuuint32_t hbox[5] = {static_cast<cuuint32_t>(a.kc), static_cast<cuuint32_t>(a.halo_w),
+                          static_cast<cuuint32_t>(a.halo_h), 1u, 1u};
     cuuint32_t hest[5] = {1u, 1u, 1u, 1u, 1u};
     r = drv.tiled(&mx, dt, rank, const_cast<void*>(x), gdim, gstr, hbox, hest, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   } else {
     r = drv.im2col(&mx, dt, rank, const_cast<void*>(x), gdim, gstr, lower, upper, static_cast<cuuint32_t>(a.kc),
                    static_cast<cuuint32_t>(kBM), estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
@@ -776,8 +787,8 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
   const bool halo = plan.variant == CONV_VARIANT_TC_HALO || plan.variant == CONV_VARIANT_TC_HALO_PAIR;
   if (plan.variant == CONV_VARIANT_TC_HALO_T || plan.variant == CONV_VARIANT_TC_HALO_T_PAIR) {
     CUtensorMap my;
-    rc = encode_maps(P, a, false, true, x, w, mx, mw, kTO);
-    if (rc == CONV_OK) rc = encode_y_block_map(P, a.rank5 != 0, y, my);
+    rc = encode_maps(P, a, false, true, x, w, mx, mw, a.mo);
+    if (rc == CONV_OK) rc = encode_y_block_map(P, a.rank5 != 0, a.mo, y, my);
     if (rc != CONV_OK) return rc;
     const bool bf = P.dtype == CONV_BF16;
     if (!plan.pair) {

@@ -1,25 +1,25 @@
-// conv_halo.cuh -- tcgen05 implicit-GEMM convolution forward with input-halo
-// reuse (stride 1, C/G a multiple of 64, f16/bf16).
+// conv_halo.cuh -- tcgen05 implicit-GEMM convolution forward with input reuse
+// in the plain orientation (rows = output pixels, columns = output channels):
+// stride 1, C/G a multiple of 32, f16/bf16.
 //
 // A CTA owns a block of 16 x 8 output pixels (h x w) of one (n, od) output
-// plane: GEMM rows m = r*8 + c for r < 16, c < 8.  For each 64-channel chunk
-// and each depth tap kd, ONE tiled TMA box brings the input halo of that block
-// -- (16 + dh*(kH-1)) x (8 + dw*(kW-1)) pixels x 64 channels -- into shared
-// memory (zero-filled outside the image).  Every (kh, kw) tap is then a view
-// of that box: output row r reads halo row r + kh*dh, output column c reads
-// halo column c + kw*dw.  Because the block is 8 pixels wide, each group of 8
-// GEMM rows is 8 consecutive halo pixels, and successive groups are one halo
-// row apart, so the view is a standard K-major 128B-swizzled UMMA operand with
-// stride (SBO) = halo width x 128 bytes, starting at tap offset
-// (kh*dh*halo_w + kw*dw) x 128 bytes.  Each input pixel of the block is
-// fetched once per (chunk, kd) instead of once per tap.
+// plane: GEMM rows m = r*8 + c for r < 16, c < 8 (a CTA pair stacks two such
+// blocks, 32 x 8, and issues M = 256).  For each channel chunk (kc = 64 or 32
+// channels), depth tap kd and width tap kw, ONE tiled TMA box brings the input
+// column strip the block needs -- (16 + dh*(kH-1)) rows x 8 columns (shifted by
+// kw*dw) x kc channels, zero-filled outside the image.  Every height tap kh
+// then reads a view of it that starts kh*dh strip rows down: a strip row is 8
+// pixels x kc*2 bytes, exactly one swizzle atom (1024 bytes with the 128-byte
+// swizzle at kc = 64, 512 bytes with the 64-byte swizzle at kc = 32), so every
+// view is a standard K-major operand on an atom boundary.  Each input pixel is
+// fetched once per (chunk, kd, kw) instead of once per tap.
 //
-// The weights stream through their own ring: one [BN x 64] tile per
-// (chunk, tap), kbs of them per pipeline stage so that one stage carries
-// enough tensor work (>= ~1000 cycles) to hide the wait/commit round trip.  Roles and the accumulator double-buffer are those of the
-// other tensor-core kernels.  With PAIR, two CTAs of a cluster stack their
-// blocks (32 x 8 output pixels), issue tcgen05.mma.cta_group::2 (M = 256) from
-// the leader, and each loads half of every weight tile.
+// The weights ([BN x kc] tiles, one per (chunk, tap)) stream through their
+// own ring and the strips through theirs, from two producer threads, so that
+// neither ring waits on the other.  Roles, bounded waits and the accumulator
+// double-buffer are those of the other tensor-core kernels.  With PAIR, the
+// leader issues tcgen05.mma.cta_group::2 and each CTA loads half of every
+// weight tile and the strip of its own 16 rows.
 #pragma once
 
 #include "conv_tc.cuh"
@@ -61,7 +61,6 @@ __global__ void __launch_bounds__(192, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
   const bool leader = rank == 0;
-  const uint16_t both = 3;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
@@ -105,21 +104,25 @@ __global__ void __launch_bounds__(192, 1)
   const int taps_hw = a.kH * a.kW;
   const uint32_t mult = PAIR ? 2u : 1u;
 
-  // K-blocks of a tile in issue order: q = (cc * kD + kd) * taps_hw + tap.  A
-  // pipeline stage holds up to kbs consecutive K-blocks (weight tiles); each
-  // (cc, kd) group has one halo box, loaded before its first K-block.  With
-  // taps_hw >= kbs a stage spans at most two groups, so two halo slots suffice.
+  // K blocks of a tile in issue order: q = ((cc * kD + kd) * kW + kw) * kH + kh.
+  // A pipeline stage holds kbs consecutive K blocks (weight tiles); each
+  // (cc, kd, kw) group has one strip in its own ring of a_slots slots.
   const int Q = a.cchunks * a.kD * taps_hw;
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producers
+    // lane 0 streams the weight tiles, lane 1 the input strips, each on its
+    // own ring; each arms a barrier only right before issuing every load it
+    // covers, so a wait that gives up never leaves bytes expected that were
+    // not requested.  (A pair's loads complete on the leader's barriers.)
     if (lane == 0) {
-      int bst = 0, ast = 0;
-      uint32_t bph = 0, aph = 0;
-      long long bfills = 0, afills = 0;
+      int bst = 0;
+      uint32_t bph = 0;
+      long long bfills = 0;
       bool ok = true;
       for (int tile = unit; ok && tile < a.total_tiles; tile += nunits) {
         const HaloTile ht = decode_halo_tile(a, tile, static_cast<int>(rank), PAIR);
         const int brow = ht.g * a.Og + ht.nt * a.BN + (PAIR ? static_cast<int>(rank) * (a.BN >> 1) : 0);
+        int kh = 0, kw = 0, kd = 0, cc = 0;  // tap of the next K block
         for (int q0 = 0; ok && q0 < Q; q0 += a.kbs) {
           const int nsub = min(a.kbs, Q - q0);
           if (!wait_bounded(ptx::smem_u32(&tail->empty[bst]), bph ^ 1u, abort_flag, a.timeout_ns,
@@ -131,40 +134,20 @@ __global__ void __launch_bounds__(192, 1)
           if (leader) ptx::mbar_arrive_expect_tx(fb, mult * static_cast<uint32_t>(nsub) * a.b_bytes);
           const uint32_t fb_l = PAIR ? ptx::mapa_shared(fb, 0) : fb;
           for (int j = 0; j < nsub; ++j) {
-            const int q = q0 + j;
-            const int t = q % taps_hw;
-            const int grp = q / taps_hw;
-            const int kd = grp % a.kD, cc = grp / a.kD;
-            if (t == 0) {
-              // the halo box of group (cc, kd)
-              if (!wait_bounded(ptx::smem_u32(&tail->aempty[ast]), aph ^ 1u, abort_flag, a.timeout_ns,
-                                kSiteProducerEmpty)) {
-                ok = false;
-                break;
-              }
-              const uint32_t afb = ptx::smem_u32(&tail->afull[ast]);
-              if (leader) ptx::mbar_arrive_expect_tx(afb, mult * a.halo_bytes);
-              const uint32_t afb_l = PAIR ? ptx::mapa_shared(afb, 0) : afb;
-              const uint32_t dst = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
-              const int c0 = ht.g * a.Cg + cc * 64;
-              const int wc = ht.w0 - a.pw, hc = ht.h0 - a.ph, dc = ht.od - a.pd + kd * a.dd;
-              if (a.rank5) {
-                if constexpr (PAIR) ptx::tma_load_5d_pair(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
-                else ptx::tma_load_5d(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
-              } else {
-                if constexpr (PAIR) ptx::tma_load_4d_pair(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
-                else ptx::tma_load_4d(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
-              }
-              ++afills;
-              if (++ast == a.a_slots) {
-                ast = 0;
-                aph ^= 1u;
+            const uint32_t sb = ptx::smem_u32(bring + bst * a.stage_bytes + j * a.b_bytes);
+            const int tap = (kd * a.kH + kh) * a.kW + kw;  // weight layout (kd, kh, kw)
+            if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, tap * a.Cg + cc * a.kc, brow);
+            else ptx::tma_load_2d(sb, &tmap_w, fb, tap * a.Cg + cc * a.kc, brow);
+            if (++kh == a.kH) {
+              kh = 0;
+              if (++kw == a.kW) {
+                kw = 0;
+                if (++kd == a.kD) {
+                  kd = 0;
+                  ++cc;
+                }
               }
             }
-            const uint32_t sb = ptx::smem_u32(bring + bst * a.stage_bytes + j * a.b_bytes);
-            const int tap = kd * taps_hw + t;
-            if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, brow);
-            else ptx::tma_load_2d(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, brow);
           }
           ++bfills;
           if (++bst == a.stages) {
@@ -178,6 +161,43 @@ __global__ void __launch_bounds__(192, 1)
           const long long arms = bfills / a.stages + (s < bfills % a.stages ? 1 : 0);
           if (arms > 0) wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
         }
+      }
+    } else if (lane == 1) {
+      int ast = 0;
+      uint32_t aph = 0;
+      long long afills = 0;
+      bool ok = true;
+      for (int tile = unit; ok && tile < a.total_tiles; tile += nunits) {
+        const HaloTile ht = decode_halo_tile(a, tile, static_cast<int>(rank), PAIR);
+        for (int cc = 0; ok && cc < a.cchunks; ++cc)
+          for (int kd = 0; ok && kd < a.kD; ++kd)
+            for (int kw = 0; kw < a.kW; ++kw) {
+              if (!wait_bounded(ptx::smem_u32(&tail->aempty[ast]), aph ^ 1u, abort_flag, a.timeout_ns,
+                                kSiteProducerEmpty)) {
+                ok = false;
+                break;
+              }
+              const uint32_t afb = ptx::smem_u32(&tail->afull[ast]);
+              if (leader) ptx::mbar_arrive_expect_tx(afb, mult * a.halo_bytes);
+              const uint32_t afb_l = PAIR ? ptx::mapa_shared(afb, 0) : afb;
+              const uint32_t dst = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
+              const int c0 = ht.g * a.Cg + cc * a.kc;
+              const int wc = ht.w0 - a.pw + kw * a.dw, hc = ht.h0 - a.ph, dc = ht.od - a.pd + kd * a.dd;
+              if constexpr (PAIR) {
+                if (a.rank5) ptx::tma_load_5d_pair(dst, &tmap_x, afb_l, c0, wc, hc, dc, ht.n);
+                else ptx::tma_load_4d_pair(dst, &tmap_x, afb_l, c0, wc, hc, ht.n);
+              } else {
+                if (a.rank5) ptx::tma_load_5d(dst, &tmap_x, afb, c0, wc, hc, dc, ht.n);
+                else ptx::tma_load_4d(dst, &tmap_x, afb, c0, wc, hc, ht.n);
+              }
+              ++afills;
+              if (++ast == a.a_slots) {
+                ast = 0;
+                aph ^= 1u;
+              }
+            }
+      }
+      if (!ok && leader) {
         for (int s = 0; s < a.a_slots; ++s) {
           const long long arms = afills / a.a_slots + (s < afills % a.a_slots ? 1 : 0);
           if (arms > 0) wait_drain(ptx::smem_u32(&tail->afull[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
@@ -186,7 +206,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer (a pair's leader)
     if (leader && lane == 0) {
       int bst = 0, ast = 0;
       uint32_t bph = 0, aph = 0;
@@ -194,12 +214,14 @@ __global__ void __launch_bounds__(192, 1)
       int t = 0;
       if (a.inject_stall)
         ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
-      const uint32_t sbo = static_cast<uint32_t>(a.halo_w) * 128u;
       // descriptors built once; moved by constant offsets below
-      const uint64_t d_halo = ptx::smem_desc_sw128_view(ptx::smem_u32(halo), sbo, 0);
-      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, 2);
+      const uint64_t d_halo = ptx::smem_desc(ptx::smem_u32(halo), 16, a.sbo, a.layout_type);
+      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(bring), 16, a.sbo, a.layout_type);
       const uint64_t sub_off = desc_off(a.b_bytes), st_off = desc_off(a.stage_bytes);
       const uint64_t slot_off = desc_off(a.halo_slot_bytes);
+      // a strip row (8 pixels x kc channels) is one swizzle atom: sbo bytes
+      const uint64_t row_off = desc_off(static_cast<uint32_t>(a.dh) * a.sbo);
+      const int ksteps = a.kc >> 4;
       for (int tile = unit; ok && tile < a.total_tiles; tile += nunits, ++t) {
         const int acc = t & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -211,8 +233,8 @@ __global__ void __launch_bounds__(192, 1)
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
         uint32_t accumulate = 0;
-        uint64_t d_box = 0;
-        int kh = 0, kw = 0;  // tap of the next K block (taps run kw-fastest)
+        uint64_t d_strip = 0;
+        int kh = 0;  // height tap of the next K block (K blocks run kh-fastest)
         for (int q0 = 0; ok && q0 < Q; q0 += a.kbs) {
           const int nsub = min(a.kbs, Q - q0);
           if (!wait_bounded(ptx::smem_u32(&tail->full[bst]), bph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
@@ -220,38 +242,34 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           ptx::tc_fence_after();
-          uint64_t db = d_ring + static_cast<uint64_t>(bst) * st_off;
+          uint64_t dw = d_ring + static_cast<uint64_t>(bst) * st_off;
           for (int j = 0; j < nsub; ++j) {
-            if (kh == 0 && kw == 0) {
+            if (kh == 0) {
               if (!wait_bounded(ptx::smem_u32(&tail->afull[ast]), aph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
                 ok = false;
                 break;
               }
               ptx::tc_fence_after();
-              d_box = d_halo + static_cast<uint64_t>(ast) * slot_off;
+              d_strip = d_halo + static_cast<uint64_t>(ast) * slot_off;
             }
-            // the view of tap (kh, kw) starts (kh*dh*halo_w + kw*dw) halo pixels into the box
-            const uint64_t da = d_box + desc_off(static_cast<uint32_t>(kh * a.dh * a.halo_w + kw * a.dw) * 128u);
-            mma_ksteps<4, PAIR>(d_tmem, da, db, a.idesc, accumulate);
+            mma_sub<PAIR>(ksteps, d_tmem, d_strip + static_cast<uint64_t>(kh) * row_off, dw, a.idesc, accumulate);
             accumulate = 1;
-            db += sub_off;
-            const bool last_tap = kh == a.kH - 1 && kw == a.kW - 1;
-            if (++kw == a.kW) {
-              kw = 0;
-              if (++kh == a.kH) kh = 0;
-            }
-            if (last_tap) {
-              // last tap of this (cc, kd): its halo slot is free once these MMAs complete
-              if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->aempty[ast]), both);
+            dw += sub_off;
+            if (kh == a.kH - 1) {
+              // last tap of this (cc, kd, kw): its strip slot is free once these MMAs complete
+              if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->aempty[ast]), 3);
               else ptx::mma_commit(ptx::smem_u32(&tail->aempty[ast]));
               if (++ast == a.a_slots) {
                 ast = 0;
                 aph ^= 1u;
               }
+              kh = 0;
+            } else {
+              ++kh;
             }
           }
           if (!ok) break;
-          if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[bst]), both);
+          if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[bst]), 3);
           else ptx::mma_commit(ptx::smem_u32(&tail->empty[bst]));
           if (++bst == a.stages) {
             bst = 0;
@@ -259,7 +277,7 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         if (ok) {
-          if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->acc_full[acc]), both);
+          if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->acc_full[acc]), 3);
           else ptx::mma_commit(ptx::smem_u32(&tail->acc_full[acc]));
         }
       }

@@ -119,7 +119,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
   const int taps_hw = a.kH * a.kW;
   const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int nunits = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
-  const int o_tile = PAIR ? 2 * kTO : kTO;  // output channels per tile (a pair: 128 per CTA)
+  const int mo = a.mo;                      // output channels per CTA (MMA M per CTA: 64 or 128)
+  const int o_tile = PAIR ? 2 * mo : mo;    // output channels per tile
   const int BP = a.BN;  // 8 * tile_h output pixels per tile
 
   // K blocks of a tile in issue order: q = ((cc * kD + kd) * kW + kw) * kH + kh.
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
       bool ok = true;
       for (int tile = unit; ok && tile < a.total_tiles; tile += nunits) {
         const HaloTTile ht = decode_halo_t_tile(a, tile);
-        const int orow = ht.g * a.Og + ht.ot * o_tile + static_cast<int>(rank) * kTO;
+        const int orow = ht.g * a.Og + ht.ot * o_tile + static_cast<int>(rank) * mo;
         int kh = 0, kw = 0, kd = 0, cc = 0;  // tap of the next K block (kh fastest, then kw, kd, cc)
         for (int q0 = 0; ok && q0 < Q; q0 += a.kbs) {
           const int nsub = min(a.kbs, Q - q0);
@@ -154,8 +155,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
           for (int j = 0; j < nsub; ++j) {
             const uint32_t sb = ptx::smem_u32(bring + bst * a.stage_bytes + j * a.b_bytes);
             const int tap = (kd * a.kH + kh) * a.kW + kw;  // weight layout (kd, kh, kw)
-            if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, tap * a.Cg + cc * 64, orow);
-            else ptx::tma_load_2d(sb, &tmap_w, fb, tap * a.Cg + cc * 64, orow);
+            if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, tap * a.Cg + cc * a.kc, orow);
+            else ptx::tma_load_2d(sb, &tmap_w, fb, tap * a.Cg + cc * a.kc, orow);
             if (++kh == a.kH) {
               kh = 0;
               if (++kw == a.kW) {
@@ -200,7 +201,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
               if (leader) ptx::mbar_arrive_expect_tx(afb, mult * a.halo_bytes);
               const uint32_t afb_l = PAIR ? ptx::mapa_shared(afb, 0) : afb;
               const uint32_t dst = ptx::smem_u32(halo + ast * a.halo_slot_bytes);
-              const int c0 = ht.g * a.Cg + cc * 64;
+              const int c0 = ht.g * a.Cg + cc * a.kc;
               // a pair splits the block's rows: each CTA loads the strip of its half
               const int wc = ht.w0 - a.pw + kw * a.dw;
               const int hc = ht.h0 + static_cast<int>(rank) * (a.tile_h / 2) - a.ph;
@@ -237,11 +238,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
       if (a.inject_stall)
         ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
       // descriptors built once; moved by constant offsets below
-      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(bring), 16, 1024, 2);
-      const uint64_t d_halo = ptx::smem_desc(ptx::smem_u32(halo), 16, 1024, 2);
+      const uint64_t d_ring = ptx::smem_desc(ptx::smem_u32(bring), 16, a.sbo, a.layout_type);
+      const uint64_t d_halo = ptx::smem_desc(ptx::smem_u32(halo), 16, a.sbo, a.layout_type);
       const uint64_t sub_off = desc_off(a.b_bytes), st_off = desc_off(a.stage_bytes);
       const uint64_t slot_off = desc_off(a.halo_slot_bytes);
-      const uint64_t row_off = desc_off(static_cast<uint32_t>(a.dh) * 1024u);
+      // a strip row (8 pixels x kc channels) is one swizzle atom: sbo bytes
+      const uint64_t row_off = desc_off(static_cast<uint32_t>(a.dh) * a.sbo);
+      const int ksteps = a.kc >> 4;
       for (int tile = unit; ok && tile < a.total_tiles; tile += nunits, ++t) {
         const int acc = t & 1;
         const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -272,8 +275,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
               ptx::tc_fence_after();
               d_strip = d_halo + static_cast<uint64_t>(ast) * slot_off;
             }
-            // strip rows are 8 pixels = 1024 bytes: the view for kh starts kh*dh atoms down
-            mma_ksteps<4, PAIR>(d_tmem, dw, d_strip + static_cast<uint64_t>(kh) * row_off, a.idesc, accumulate);
+            // the view for kh starts kh*dh strip rows (swizzle atoms) down
+            mma_sub<PAIR>(ksteps, d_tmem, dw, d_strip + static_cast<uint64_t>(kh) * row_off, a.idesc, accumulate);
             accumulate = 1;
             dw += sub_off;
             if (kh == a.kH - 1) {
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       const HaloTTile ht = decode_halo_t_tile(a, tile);
-      const int o0 = ht.g * a.Og + ht.ot * o_tile + static_cast<int>(rank) * kTO;
+      const int o0 = ht.g * a.Og + ht.ot * o_tile + static_cast<int>(rank) * mo;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc) * kHTAccStride;
       for (int c = 0; c < BP; c += kTEpiRows) {
         uint32_t r[32];
@@ -337,9 +340,17 @@ __global__ void __launch_bounds__(kTThreads, 1)
         // the store issued two chunks ago read this buffer; it must be done
         if (store_thread) ptx::bulk_wait_group_read<1>();
         named_bar_sync(1, 128);
-        uint16_t* dst = reinterpret_cast<uint16_t*>(buf) + q * 32 + lane;
+        // M = 128: lane l of quarter q holds channel 32q + l; M = 64: lanes 0..15 of
+        // quarter q hold channels 16q .. 16q+15 (the other 16 lanes are empty)
+        if (mo == kTO) {
+          uint16_t* dst = reinterpret_cast<uint16_t*>(buf) + q * 32 + lane;
 #pragma unroll
-        for (int p = 0; p < kTEpiRows; ++p) dst[p * kTO] = cvt1<BF16>(__uint_as_float(r[p]));
+          for (int p = 0; p < kTEpiRows; ++p) dst[p * kTO] = cvt1<BF16>(__uint_as_float(r[p]));
+        } else if (lane < 16) {
+          uint16_t* dst = reinterpret_cast<uint16_t*>(buf) + q * 16 + lane;
+#pragma unroll
+          for (int p = 0; p < kTEpiRows; ++p) dst[p * 64] = cvt1<BF16>(__uint_as_float(r[p]));
+        }
         ptx::fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (store_thread) {

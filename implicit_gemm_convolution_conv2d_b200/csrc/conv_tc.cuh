@@ -94,6 +94,7 @@ struct TcArgs {
   int Lp;             // span layout: filter-row length kW*C rounded up to 8
   int Kp;             // K as laid out in shared memory (>= K in span layout)
   long long x_elems;  // elements of x (bounds of the unaligned 16-byte loads)
+  int mo;             // transposed halo kernel: output channels per tile (MMA M: 64 or 128)
   int b_resident;     // gather: the whole B matrix stays in shared memory
   uint32_t bres_bytes;  // its size (kblocks * BN * 128), 0 when not resident
   const void* x;
@@ -111,8 +112,8 @@ struct __align__(8) TcSmemTail {
   uint64_t drain;
   uint64_t stall;     // never arrived on (the injected-timeout test waits here)
   uint64_t bres;      // resident weights loaded
-  uint64_t afull[4];  // halo kernel: input halo slots
-  uint64_t aempty[4];
+  uint64_t afull[8];  // halo kernels: input strip slots
+  uint64_t aempty[8];
   uint64_t rfull[3];  // row staging (gather): rows of a tile landed
   uint64_t rempty[3]; // row staging: every gather thread is done with the buffer
   int seg_n[3][2];    // row staging, per buffer: image of segment 0 / 1

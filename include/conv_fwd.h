@@ -81,10 +81,11 @@ enum {
   CONV_VARIANT_TC_TMA_T = 6,     /* TC_TMA in the transposed orientation: MMA M = 128
                                    output channels, N = 256 output pixels, TMA-store
                                    epilogue (C/G % 16 == 0, O/G % 128 == 0) */
-  CONV_VARIANT_TC_HALO_T = 7,    /* transposed orientation with halo reuse: N = an
-                                   (up to 32) x 8 output block read from one 8-wide
-                                   input strip per (64-channel chunk, kd, kw)
-                                   (stride 1, C/G % 64 == 0, O/G % 128 == 0) */
+  CONV_VARIANT_TC_HALO_T = 7,    /* transposed orientation with halo reuse: M = 128
+                                   (or 64) output channels, N = an (up to 32) x 8
+                                   output block read from one 8-wide input strip
+                                   per (channel chunk, kd, kw) (stride 1,
+                                   C/G % 32 == 0, O/G % 64 == 0) */
   CONV_VARIANT_TC_HALO_T_PAIR = 8 /* TC_HALO_T with CTA pairs: M = 256 output channels,
                                    cta_group::2 (O/G % 256 == 0) */
 };
@@ -100,9 +101,10 @@ int conv_out_dims(int D, int H, int W, int kD, int kH, int kW,
  * Queues the kernel on `stream`; returns CONV_OK or an error code (nothing is
  * queued on an error).  The variant is chosen from the type and shape:
  * f32 -> SIMT; f16/bf16 with C/G % 16 == 0 and a geometry that fits a TMA
- * im2col tensor map -> when O/G is an odd multiple of 128: TC_HALO_T at
- * stride 1 with C/G % 64 == 0, kH >= 2 and at least as many output blocks as
- * SMs, else TC_TMA_T when there are at least as many 256-pixel tiles as SMs;
+ * im2col tensor map -> when O/G is a multiple of 64 but not of 256: TC_HALO_T
+ * at stride 1 with C/G % 32 == 0, kH >= 2 and at least as many output blocks
+ * as SMs, else (O/G % 128 == 0) TC_TMA_T when there are at least as many
+ * 256-pixel tiles as SMs;
  * otherwise TC_TMA_PAIR (or TC_TMA when there are fewer 256-row output tiles
  * than SM pairs); otherwise TC_GATHER.  TC_HALO, TC_HALO_PAIR and
  * TC_HALO_T_PAIR run only when requested through conv_fwd_variant. */
@@ -117,7 +119,8 @@ int conv_fwd(const void* x, const void* w, void* y,
  * (the tensor-core variants need f16/bf16; TC_TMA, TC_TMA_PAIR and TC_TMA_T
  * need C/G % 16 == 0 and a geometry inside the TMA im2col limits, TC_TMA_T
  * also O/G % 128 == 0; TC_HALO and TC_HALO_PAIR need stride 1 and
- * C/G % 64 == 0). */
+ * C/G % 32 == 0; TC_HALO_T also O/G % 64 == 0, TC_HALO_T_PAIR
+ * O/G % 256 == 0). */
 int conv_fwd_variant(const void* x, const void* w, void* y,
                      int N, int D, int H, int W, int C, int O,
                      int kD, int kH, int kW,

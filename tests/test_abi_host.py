@@ -119,6 +119,9 @@ def test_variant_plan(C):
     # 128 output channels, stride 1, 64-channel chunks, kH >= 2: the transposed halo kernel
     v, bn, st, _ = plan(4, 32, 32, 32, 64, 128, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_HALO_T and bn == 256 and st >= 2
+    # 64 output channels, 32-channel chunks: the transposed halo kernel with M = 64
+    v, bn, _, _ = plan(2, 64, 64, 64, 32, 64, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
+    assert v == C.VARIANT_TC_HALO_T and bn == 256
     # ... with kH = 1 (no strip reuse): the transposed im2col kernel
     v, bn, _, _ = plan(4, 32, 32, 32, 64, 128, (3, 1, 1), (1, 1, 1), (1, 0, 0), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_TMA_T and bn == 256
@@ -136,7 +139,7 @@ def test_variant_plan(C):
     v, _, _, _ = plan(1, 40, 8, 8, 64, 64, (3, 3, 3), (1, 1, 1), (17, 1, 1), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_GATHER
     # channel chunks of 32 and 16
-    assert plan(2, 64, 64, 64, 32, 64, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA_PAIR
+    assert plan(2, 64, 64, 64, 32, 256, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA_PAIR
     assert plan(2, 64, 64, 64, 32, 384, (1, 1, 1), (1, 1, 1), (0, 0, 0), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA_T
     assert plan(1, 1, 9, 9, 48, 96, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 3, "f16")[0] == C.VARIANT_TC_TMA
     assert plan(1, 1, 9, 9, 128, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 2, "f16")[0] == C.VARIANT_TC_TMA

@@ -56,11 +56,11 @@ def variants_for(wl):
     vs.append(C.VARIANT_TC_GATHER)
     if (wl.C // wl.groups) % 16 == 0:
         vs += [C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR]
-    if (wl.C // wl.groups) % 64 == 0 and tuple(wl.stride) == (1, 1, 1) and wl.k[1] * wl.k[2] >= 4:
+    if (wl.C // wl.groups) % 32 == 0 and tuple(wl.stride) == (1, 1, 1):
         vs += [C.VARIANT_TC_HALO, C.VARIANT_TC_HALO_PAIR]
     if (wl.C // wl.groups) % 16 == 0 and (wl.O // wl.groups) % 128 == 0:
         vs.append(C.VARIANT_TC_TMA_T)
-    if (wl.C // wl.groups) % 64 == 0 and (wl.O // wl.groups) % 128 == 0 and tuple(wl.stride) == (1, 1, 1):
+    if (wl.C // wl.groups) % 32 == 0 and (wl.O // wl.groups) % 64 == 0 and tuple(wl.stride) == (1, 1, 1):
         vs.append(C.VARIANT_TC_HALO_T)
     if (wl.C // wl.groups) % 64 == 0 and (wl.O // wl.groups) % 256 == 0 and tuple(wl.stride) == (1, 1, 1):
         vs.append(C.VARIANT_TC_HALO_T_PAIR)
@@ -105,6 +105,9 @@ SMALL = [
     WL.case(2, 1, 17, 9, 128, 128, (1, 3, 3), pad=(0, 2, 2), dil=(1, 2, 2), groups=2, name="halo_groups2_dil2"),
     WL.case(1, 1, 12, 12, 64, 320, (1, 3, 3), pad=(0, 1, 1), name="halo_o320"),
     WL.case(3, 1, 33, 17, 64, 32, (1, 5, 5), pad=(0, 2, 2), name="halo_k5_ragged"),
+    # plain-orientation strips with 32-channel chunks (64-byte swizzle), 2-D and 3-D, dilation
+    WL.case(2, 1, 23, 13, 32, 64, (1, 3, 3), pad=(0, 1, 1), name="halo_c32_o64"),
+    WL.case(1, 5, 19, 10, 96, 64, (3, 3, 3), pad=(1, 2, 1), dil=(1, 2, 1), name="halo_c96_3d_dil"),
     # transposed orientation (128 output channels per tile): ragged pixel
     # tail, groups with 32-channel chunks, 3-D with 16-channel chunks, two
     # channel tiles at stride 2
@@ -122,6 +125,10 @@ SMALL = [
     WL.case(2, 1, 28, 21, 64, 256, (1, 3, 3), pad=(0, 1, 1), name="htp_h28"),
     WL.case(1, 3, 19, 11, 64, 256, (3, 3, 3), pad=(1, 2, 1), dil=(1, 2, 1), name="htp_3d_dil"),
     WL.case(2, 1, 9, 10, 128, 512, (1, 3, 3), pad=(0, 1, 1), groups=2, name="htp_groups2"),
+    # transposed halo with 64 output channels per tile (M = 64) and 32-channel chunks
+    WL.case(1, 1, 14, 12, 64, 192, (1, 3, 3), pad=(0, 1, 1), name="ht_o192_m64"),
+    WL.case(1, 1, 10, 9, 64, 128, (1, 3, 3), pad=(0, 1, 1), groups=2, name="ht_g2_og64_c32"),
+    WL.case(1, 4, 9, 18, 32, 64, (3, 3, 3), pad=(1, 1, 1), name="ht_3d_c32_o64"),
 ]
 
 
