@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libconvfwd.so")
 SOURCES = [os.path.join(CSRC, "conv_fwd.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("conv_tc.cuh", "conv_simt.cuh", "ptx.cuh")] + [
+DEPS = SOURCES + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(os.path.dirname(HERE), "include", "conv_fwd.h")]
 
 NVCC_FLAGS = [

@@ -458,6 +458,24 @@ int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
   a.kc = (P.Cg % 64 == 0) ? 64 : 32;
   a.halo_bytes = static_cast<uint32_t>(hw * hh * a.kc * 2);
   a.halo_slot_bytes = (a.halo_bytes + 1023u) & ~1023u;
+  // Resident weights: with one group and one output-channel tile every tile
+  // multiplies by the same weights, so when they fit beside two strip slots
+  // (with two epilogue staging tiles, else one) they are loaded once per CTA
+  // instead of once per tile.
+  const long long base_budget =
+      static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64;
+  const long long w_total = static_cast<long long>(P.kD) * P.kH * P.kW * P.Cg * mo * 2;
+  a.w_resident = 0;
+  a.epi_bufs = 2;
+  if (P.G == 1 && a.n_tiles == 1) {
+    for (int bufs = 2; bufs >= 1; --bufs) {
+      if (base_budget - bufs * static_cast<long long>(kTEpiBytes) - w_total >= 2LL * a.halo_slot_bytes) {
+        a.w_resident = 1;
+        a.epi_bufs = bufs;
+        break;
+      }
+    }
+  }
   a.a_slots = 2;
   a.mo = mo;
   a.cchunks = P.Cg / a.kc;
@@ -469,14 +487,18 @@ int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
   a.b_bytes = static_cast<uint32_t>(mo * a.kc * 2);  // one weight tile: mo channels x kc
   a.sub_bytes = a.b_bytes;
   // the weight and strip rings are independent: first up to three weight
-  // stages beside two strip slots, then as many more strip slots (up to 8) as
-  // the rest of shared memory holds
-  const long long budget = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
-                           64 - 2LL * kTEpiBytes;
+  // stages beside two strip slots (or the one resident stage), then as many
+  // more strip slots (up to 8) as the rest of shared memory holds
+  const long long budget = base_budget - a.epi_bufs * static_cast<long long>(kTEpiBytes);
   int stages = 0;
-  a.kbs = choose_kbs(a.BN, a.kc, a.b_bytes, budget - 2LL * a.halo_slot_bytes, 16, stages);
-  if (stages < 2) return CONV_EUNSUPPORTED;
-  stages = std::min(stages, 3);
+  if (a.w_resident) {
+    a.kbs = a.kblocks;
+    stages = 1;
+  } else {
+    a.kbs = choose_kbs(a.BN, a.kc, a.b_bytes, budget - 2LL * a.halo_slot_bytes, 16, stages);
+    if (stages < 2) return CONV_EUNSUPPORTED;
+    stages = std::min(stages, 3);
+  }
   const long long left = budget - static_cast<long long>(stages) * a.kbs * a.b_bytes;
   a.a_slots = static_cast<int>(std::min<long long>(8, left / a.halo_slot_bytes));
   if (a.a_slots < 2) return CONV_EUNSUPPORTED;
@@ -491,7 +513,7 @@ int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
   plan.pair = pair;
   plan.ctas = pair ? 2 * std::min(a.total_tiles, sms / 2) : std::min(a.total_tiles, sms);
   plan.smem = static_cast<size_t>(a.a_slots) * a.halo_slot_bytes + static_cast<size_t>(a.stages) * a.stage_bytes +
-              2 * static_cast<size_t>(kTEpiBytes) + 1024 + sizeof(TcSmemTail) + 64;
+              static_cast<size_t>(a.epi_bufs) * kTEpiBytes + 1024 + sizeof(TcSmemTail) + 64;
   return CONV_OK;
 }
 

@@ -70,8 +70,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* halo = smem;                                              // a_slots x halo_slot_bytes
   uint8_t* bring = smem + a.a_slots * a.halo_slot_bytes;             // stages x (kbs weight tiles)
-  uint8_t* stage_y = bring + static_cast<size_t>(a.stages) * a.stage_bytes;  // 2 staging tiles
-  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(stage_y + 2 * kTEpiBytes);
+  uint8_t* stage_y = bring + static_cast<size_t>(a.stages) * a.stage_bytes;  // epi_bufs staging tiles
+  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(stage_y + a.epi_bufs * kTEpiBytes);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
@@ -138,7 +138,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
       uint32_t bph = 0;
       long long bfills = 0;
       bool ok = true;
-      for (int tile = unit; ok && tile < a.total_tiles; tile += nunits) {
+      // resident weights (one output-channel tile, one group): the first
+      // tile's single fill of stage 0 serves every tile
+      const int tile_end = a.w_resident ? min(a.total_tiles, unit + 1) : a.total_tiles;
+      for (int tile = unit; ok && tile < tile_end; tile += nunits) {
         const HaloTTile ht = decode_halo_t_tile(a, tile);
         const int orow = ht.g * a.Og + ht.ot * o_tile + static_cast<int>(rank) * mo;
         int kh = 0, kw = 0, kd = 0, cc = 0;  // tap of the next K block (kh fastest, then kw, kd, cc)
@@ -176,7 +179,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
       }
       // (a pair's loads all complete on the leader's barriers: the leader drains)
-      if (!ok && leader) {
+      if (a.w_resident && ok && leader && bfills > 0) {
+        // the MMA thread may give up before it waits on the resident fill:
+        // the loads must have landed before this CTA can exit
+        wait_drain(ptx::smem_u32(&tail->full[0]), 0u, a.timeout_ns);
+      } else if (!ok && leader) {
         for (int s = 0; s < a.stages; ++s) {
           const long long arms = bfills / a.stages + (s < bfills % a.stages ? 1 : 0);
           if (arms > 0) wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
@@ -260,7 +267,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
         int kh = 0;  // height tap of the next K block (K blocks run kh-fastest)
         for (int q0 = 0; ok && q0 < Q; q0 += a.kbs) {
           const int nsub = min(a.kbs, Q - q0);
-          if (!wait_bounded(ptx::smem_u32(&tail->full[bst]), bph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
+          if ((!a.w_resident || t == 0) &&
+              !wait_bounded(ptx::smem_u32(&tail->full[bst]), bph, abort_flag, a.timeout_ns, kSiteMmaFull)) {
             ok = false;
             break;
           }
@@ -293,6 +301,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
             }
           }
           if (!ok) break;
+          if (a.w_resident) continue;  // resident weights are never released
           if constexpr (PAIR) ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[bst]), 3);
           else ptx::mma_commit(ptx::smem_u32(&tail->empty[bst]));
           if (++bst == a.stages) {
@@ -336,9 +345,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
         ptx::tmem_ld_wait();
         const int h = ht.h0 + (c / kTEpiRows) * kRowsPerChunk;
         if (h >= a.Ho) continue;  // the same for every epilogue thread
-        uint8_t* buf = stage_y + (chunk_seq & 1) * kTEpiBytes;
-        // the store issued two chunks ago read this buffer; it must be done
-        if (store_thread) ptx::bulk_wait_group_read<1>();
+        uint8_t* buf = stage_y + (a.epi_bufs == 2 ? (chunk_seq & 1) : 0) * kTEpiBytes;
+        // the store that last read this buffer (two chunks ago, or the
+        // previous one with a single buffer) must be done with it
+        if (store_thread) {
+          if (a.epi_bufs == 2) ptx::bulk_wait_group_read<1>();
+          else ptx::bulk_wait_group_read<0>();
+        }
         named_bar_sync(1, 128);
         // M = 128: lane l of quarter q holds channel 32q + l; M = 64: lanes 0..15 of
         // quarter q hold channels 16q .. 16q+15 (the other 16 lanes are empty)

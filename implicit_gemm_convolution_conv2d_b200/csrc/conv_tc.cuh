@@ -97,6 +97,8 @@ struct TcArgs {
   int mo;             // transposed halo kernel: output channels per tile (MMA M: 64 or 128)
   int b_resident;     // gather: the whole B matrix stays in shared memory
   uint32_t bres_bytes;  // its size (kblocks * BN * 128), 0 when not resident
+  int w_resident;     // transposed halo kernel: all weight tiles loaded once into stage 0
+  int epi_bufs;       // transposed halo kernel: epilogue staging tiles (1 or 2)
   const void* x;
   const void* w;
   void* y;

@@ -119,9 +119,14 @@ def test_variant_plan(C):
     # 128 output channels, stride 1, 64-channel chunks, kH >= 2: the transposed halo kernel
     v, bn, st, _ = plan(4, 32, 32, 32, 64, 128, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_HALO_T and bn == 256 and st >= 2
-    # 64 output channels, 32-channel chunks: the transposed halo kernel with M = 64
-    v, bn, _, _ = plan(2, 64, 64, 64, 32, 64, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
-    assert v == C.VARIANT_TC_HALO_T and bn == 256
+    # 64 output channels, 32-channel chunks: the transposed halo kernel with M = 64,
+    # all weights resident in shared memory (a single pipeline stage)
+    v, bn, st, _ = plan(2, 64, 64, 64, 32, 64, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
+    assert v == C.VARIANT_TC_HALO_T and bn == 256 and st == 1
+    # 1x3x3 64 -> 128: resident weights too; two groups: streamed weights
+    assert plan(4, 32, 32, 32, 64, 128, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "f16")[2] == 1
+    assert plan(2, 1, 9, 9, 128, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 2, "f16",
+                C.VARIANT_TC_HALO_T)[2] >= 2
     # ... with kH = 1 (no strip reuse): the transposed im2col kernel
     v, bn, _, _ = plan(4, 32, 32, 32, 64, 128, (3, 1, 1), (1, 1, 1), (1, 0, 0), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_TMA_T and bn == 256

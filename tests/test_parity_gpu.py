@@ -129,6 +129,9 @@ SMALL = [
     WL.case(1, 1, 14, 12, 64, 192, (1, 3, 3), pad=(0, 1, 1), name="ht_o192_m64"),
     WL.case(1, 1, 10, 9, 64, 128, (1, 3, 3), pad=(0, 1, 1), groups=2, name="ht_g2_og64_c32"),
     WL.case(1, 4, 9, 18, 32, 64, (3, 3, 3), pad=(1, 1, 1), name="ht_3d_c32_o64"),
+    # all weights resident in shared memory beside two 34-row strip slots and
+    # one epilogue staging tile
+    WL.case(1, 1, 32, 16, 64, 128, (1, 3, 3), pad=(0, 1, 1), name="ht_resident_one_staging_tile"),
 ]
 
 
