@@ -17,6 +17,7 @@
 #include "conv_tc.cuh"
 #include "conv_tct.cuh"
 #include "conv_halo_t.cuh"
+#include "conv_phase.cuh"
 
 namespace convfwd {
 namespace {
@@ -161,6 +162,8 @@ int set_kernel_attrs(int dev) {
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_phase_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_phase_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return CONV_ELAUNCH;
   g_dev[dev].attrs_set = true;
   return CONV_OK;
@@ -517,7 +520,96 @@ int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
   return CONV_OK;
 }
 
+// Phase-packed kernel (conv_phase.cuh) for 2-D layers with few input
+// channels: one GEMM row = P output pixels of a row, P the smallest count
+// whose windows start a multiple of 8 elements apart in the flattened input
+// row; N = P*O <= 256; CTA pairs, each CTA ph_rows output rows of a tile.
+int plan_phase(const Problem& P, int sms, TcPlan& plan) {
+  if (P.dtype == CONV_F32 || P.G != 1) return CONV_EUNSUPPORTED;
+  if (P.D != 1 || P.kD != 1 || P.p[0] != 0) return CONV_EUNSUPPORTED;  // 2-D
+  if (P.d[2] != 1) return CONV_EUNSUPPORTED;  // a filter row's taps are contiguous
+  const int sh = P.s[1], sw = P.s[2];
+  if (P.H % sh != 0) return CONV_EUNSUPPORTED;  // input rows as (ih / sh, ih % sh)
+  const long long WC = static_cast<long long>(P.W) * P.C;
+  if ((WC * 2) % 16 != 0 || static_cast<long long>(P.N) * P.H * WC > 0x7fffffffLL) return CONV_EUNSUPPORTED;
+  int Pg = 1;
+  while ((Pg * sw * P.C) % 8 != 0) ++Pg;
+  const int BN = Pg * P.O;
+  // (the epilogue reads the accumulator 32 columns at a time)
+  if (BN > 256 || BN % 32 != 0 || P.Wo % Pg != 0) return CONV_EUNSUPPORTED;
+  const int qtot = P.Wo / Pg;
+  const int al = round_up(P.p[2] * P.C, 8);
+  const long long pitch = static_cast<long long>(Pg) * sw * P.C;
+  const int span = al - P.p[2] * P.C + (Pg - 1) * sw * P.C + P.kW * P.C;
+  const int Kw = round_up(span, 16);
+  if (Kw > kPhWin) return CONV_EUNSUPPORTED;
+  // windows are loaded kPhWin elements wide (128-byte rows); the MMAs read Kw
+  int nleft = 0;
+  while (nleft < qtot && pitch * nleft - al < 0) ++nleft;
+  int nright = 0;
+  while (nright < qtot - nleft && pitch * (qtot - 1 - nright) - al + kPhWin > WC) ++nright;
+  const int qint = qtot - nleft - nright;
+  const int nedge = nleft + nright;
+  if (qint < 1 || qint > 256) return CONV_EUNSUPPORTED;
+  int R = 0;
+  for (int r = 8; r >= 1; r /= 2) {
+    if (round_up(r * qint, 8) + 8 * nedge <= kBM) {
+      R = r;
+      break;
+    }
+  }
+  if (R == 0) return CONV_EUNSUPPORTED;
+  TcArgs& a = plan.args;
+  std::memset(&a, 0, sizeof(a));
+  a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.C = P.C; a.O = P.O;
+  a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
+  a.sd = P.s[0]; a.sh = P.s[1]; a.sw = P.s[2];
+  a.pd = P.p[0]; a.ph = P.p[1]; a.pw = P.p[2];
+  a.dd = P.d[0]; a.dh = P.d[1]; a.dw = P.d[2];
+  a.G = P.G; a.Cg = P.Cg; a.Og = P.Og;
+  a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
+  a.M = P.M;
+  a.K = static_cast<int>(P.K);
+  a.BN = BN;
+  a.ph_P = Pg;
+  a.ph_ks = Kw / 16;
+  a.ph_qtot = qtot;
+  a.ph_qint = qint;
+  a.ph_nleft = nleft;
+  a.ph_nright = nright;
+  a.ph_rows = R;
+  a.ph_erow0 = round_up(R * qint, 8);
+  a.ph_align = al;
+  a.ph_wbytes = static_cast<uint32_t>(P.w_bytes);
+  a.ph_bblk = static_cast<uint32_t>(BN / 2 * 128);  // per CTA: BN/2 rows of 128 bytes
+  a.ph_epi_bytes = static_cast<uint32_t>(round_up(R * qtot * 64, 1024));
+  a.tiles_h = (P.Ho + 2 * R - 1) / (2 * R);  // a pair tile: 2 * ph_rows output rows
+  const long long tt = static_cast<long long>(P.N) * a.tiles_h;
+  if (tt > 0x7fffffffLL) return CONV_EINVAL;
+  a.total_tiles = static_cast<int>(tt);
+  a.stage_bytes = kPhAStage;
+  const long long b_bytes = static_cast<long long>(P.kH) * a.ph_bblk;
+  const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
+                          64 - b_bytes - 2LL * a.ph_epi_bytes;
+  if (avail < 2LL * a.stage_bytes) return CONV_EUNSUPPORTED;
+  a.stages = static_cast<int>(std::min<long long>(4, avail / a.stage_bytes));
+  // w is first copied into the A ring, from which B is built
+  if (static_cast<long long>(P.w_bytes) > static_cast<long long>(a.stages) * a.stage_bytes) return CONV_EUNSUPPORTED;
+  const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
+  a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+            ((static_cast<uint32_t>(2 * kBM) >> 4) << 24);
+  a.tmem_cols = next_pow2_cols(static_cast<uint32_t>(2 * BN));
+  a.timeout_ns = kWaitTimeoutNs;
+  plan.variant = CONV_VARIANT_TC_PHASE;
+  plan.pair = true;
+  plan.ctas = 2 * std::min(a.total_tiles, sms / 2);
+  plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + static_cast<size_t>(b_bytes) +
+              2 * static_cast<size_t>(a.ph_epi_bytes) + 1024 + sizeof(TcSmemTail) + 64;
+  return CONV_OK;
+}
+
 int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
+  if (variant == CONV_VARIANT_TC_PHASE) return plan_phase(P, sms, plan);
   if (variant == CONV_VARIANT_TC_HALO_T || variant == CONV_VARIANT_TC_HALO_T_PAIR)
     return plan_halo_t(P, variant == CONV_VARIANT_TC_HALO_T_PAIR, sms, plan);
   if (variant == CONV_VARIANT_TC_HALO || variant == CONV_VARIANT_TC_HALO_PAIR)
@@ -650,7 +742,10 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
 int choose_variant(const Problem& P, int sms) {
   if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
   bool r5;
-  if (!tma_fits(P, r5)) return CONV_VARIANT_TC_GATHER;
+  if (!tma_fits(P, r5)) {
+    TcPlan pp;
+    return plan_phase(P, sms, pp) == CONV_OK ? CONV_VARIANT_TC_PHASE : CONV_VARIANT_TC_GATHER;
+  }
   if (P.Og % 64 == 0 && P.Og % 256 != 0 && P.kH >= 2) {
     TcPlan hp;
     if (plan_halo_t(P, false, sms, hp) == CONV_OK && hp.args.total_tiles >= sms) return CONV_VARIANT_TC_HALO_T;
@@ -794,6 +889,60 @@ int encode_maps(const Problem& P, const TcArgs& a, bool pair, bool halo, const v
 // this limit in nanoseconds, so the kernel's timeout path runs.  One-shot.
 std::atomic<unsigned long long> g_inject_stall_ns{0};
 
+// Tensor maps of the phase-packed kernel: overlapping input windows (rows
+// pitch elements apart, inside the input row), plain input rows for the edge
+// windows, and y as [N, Ho, Wo/P, P*O].
+int encode_phase_maps(const Problem& P, const TcArgs& a, const void* x, void* y, CUtensorMap& min_,
+                      CUtensorMap& medge, CUtensorMap& my) {
+  std::memset(&min_, 0, sizeof(min_));
+  std::memset(&medge, 0, sizeof(medge));
+  std::memset(&my, 0, sizeof(my));
+  const DriverFns& drv = driver_fns();
+  if (!drv.tiled) return CONV_EDRIVER;
+  const CUtensorMapDataType dt =
+      P.dtype == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t eb = 2, WC = static_cast<cuuint64_t>(P.W) * P.C;
+  const cuuint64_t sh = static_cast<cuuint64_t>(P.s[1]);
+  const cuuint64_t pitch = static_cast<cuuint64_t>(a.ph_P) * P.s[2] * P.C;
+  cuuint32_t est[5] = {1, 1, 1, 1, 1};
+  {
+    const char* base = static_cast<const char*>(x) + eb * (pitch * a.ph_nleft - a.ph_align);
+    cuuint64_t dim[5] = {static_cast<cuuint64_t>(kPhWin), static_cast<cuuint64_t>(a.ph_qint), sh,
+                         static_cast<cuuint64_t>(P.H) / sh, static_cast<cuuint64_t>(P.N)};
+    cuuint64_t str[4] = {eb * pitch, eb * WC, eb * WC * sh, eb * WC * P.H};
+    cuuint32_t box[5] = {static_cast<cuuint32_t>(kPhWin), static_cast<cuuint32_t>(a.ph_qint), 1u,
+                         static_cast<cuuint32_t>(a.ph_rows), 1u};
+    const CUresult r = drv.tiled(&min_, dt, 5, const_cast<char*>(base), dim, str, box, est,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+    small_tensor_fixup(min_, P.x_bytes, drv.driver_version);
+  }
+  {
+    cuuint64_t dim[4] = {WC, sh, static_cast<cuuint64_t>(P.H) / sh, static_cast<cuuint64_t>(P.N)};
+    cuuint64_t str[3] = {eb * WC, eb * WC * sh, eb * WC * P.H};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(kPhWin), 1u, static_cast<cuuint32_t>(a.ph_rows), 1u};
+    const CUresult r = drv.tiled(&medge, dt, 4, const_cast<void*>(x), dim, str, box, est,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+    small_tensor_fixup(medge, P.x_bytes, drv.driver_version);
+  }
+  {
+    const cuuint64_t row = static_cast<cuuint64_t>(a.BN);  // P*O elements per GEMM row
+    cuuint64_t dim[4] = {row, static_cast<cuuint64_t>(a.ph_qtot), static_cast<cuuint64_t>(P.Ho),
+                         static_cast<cuuint64_t>(P.N)};
+    cuuint64_t str[3] = {eb * row, eb * row * a.ph_qtot, eb * row * a.ph_qtot * P.Ho};
+    cuuint32_t box[4] = {32u, static_cast<cuuint32_t>(a.ph_qtot), static_cast<cuuint32_t>(a.ph_rows), 1u};
+    const CUresult r = drv.tiled(&my, dt, 4, y, dim, str, box, est, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+    small_tensor_fixup(my, P.y_bytes, drv.driver_version);
+  }
+  return CONV_OK;
+}
+
 int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w, void* y, cudaStream_t st,
               int dev) {
   int rc = set_kernel_attrs(dev);
@@ -807,6 +956,32 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
   }
   CUtensorMap mx, mw;
   const bool halo = plan.variant == CONV_VARIANT_TC_HALO || plan.variant == CONV_VARIANT_TC_HALO_PAIR;
+  if (plan.variant == CONV_VARIANT_TC_PHASE) {
+    CUtensorMap me, my;
+    rc = encode_phase_maps(P, a, x, y, mx, me, my);
+    if (rc != CONV_OK) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(plan.ctas);
+    cfg.blockDim = dim3(kPhThreads);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // never launch more pairs than can be resident together
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, conv_fwd_tc_phase_kernel<false>, &cfg) != cudaSuccess ||
+        clusters <= 0)
+      return CONV_ELAUNCH;
+    cfg.gridDim = dim3(2 * std::min(plan.ctas / 2, clusters));
+    const cudaError_t e = P.dtype == CONV_BF16 ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_phase_kernel<true>, mx, me, my, a)
+                                               : cudaLaunchKernelEx(&cfg, conv_fwd_tc_phase_kernel<false>, mx, me, my, a);
+    return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+  }
   if (plan.variant == CONV_VARIANT_TC_HALO_T || plan.variant == CONV_VARIANT_TC_HALO_T_PAIR) {
     CUtensorMap my;
     rc = encode_maps(P, a, false, true, x, w, mx, mw, a.mo);
@@ -1008,7 +1183,7 @@ int conv_fwd_variant(const void* x, const void* w, void* y, int N, int D, int H,
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_T_PAIR) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_PHASE) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1045,7 +1220,7 @@ int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, 
   Problem P;
   int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_HALO_T_PAIR) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_PHASE) return CONV_EINVAL;
   int dev, sms = 148;
   if (current_device(dev) == CONV_OK) device_sms(dev, sms);
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);

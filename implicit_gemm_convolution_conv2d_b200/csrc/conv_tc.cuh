@@ -99,6 +99,18 @@ struct TcArgs {
   uint32_t bres_bytes;  // its size (kblocks * BN * 128), 0 when not resident
   int w_resident;     // transposed halo kernel: all weight tiles loaded once into stage 0
   int epi_bufs;       // transposed halo kernel: epilogue staging tiles (1 or 2)
+  // phase-packed kernel (few input channels): one GEMM row = P output pixels of a row
+  int ph_P;            // pixels per GEMM row (P * sw * C is a multiple of 8)
+  int ph_ks;           // 16-element K steps per filter row (window of 16 * ph_ks elements)
+  int ph_qtot;         // GEMM rows per output row (Wo / P)
+  int ph_qint;         // of them, rows whose window lies inside the input row
+  int ph_nleft, ph_nright;  // edge rows at the left / right end of an output row
+  int ph_rows;         // output rows per tile
+  int ph_erow0;        // A-tile row of the first edge row (edge rows use 8-row slots)
+  int ph_align;        // GEMM row q's window starts at element P*sw*C*q - ph_align
+  uint32_t ph_wbytes;  // bytes of w
+  uint32_t ph_bblk;    // one resident B block: N rows x 32 bytes
+  uint32_t ph_epi_bytes;  // one epilogue staging tile
   const void* x;
   const void* w;
   void* y;
@@ -272,12 +284,13 @@ __device__ __forceinline__ void mma_ksteps(uint32_t d_tmem, uint64_t da, uint64_
   }
 }
 
-// The same for a run-time step count of 4, 2 or 1 (channel chunks of 64, 32
-// or 16 elements).
+// The same for a run-time step count of 1 to 4 (channel chunks of 64, 32 or
+// 16 elements; 3 for a 48-element phase-packed window).
 template <bool PAIR>
 __device__ __forceinline__ void mma_sub(int ksteps, uint32_t d_tmem, uint64_t da, uint64_t db, uint32_t idesc,
                                         uint32_t acc0) {
   if (ksteps == 4) mma_ksteps<4, PAIR>(d_tmem, da, db, idesc, acc0);
+  else if (ksteps == 3) mma_ksteps<3, PAIR>(d_tmem, da, db, idesc, acc0);
   else if (ksteps == 2) mma_ksteps<2, PAIR>(d_tmem, da, db, idesc, acc0);
   else mma_ksteps<1, PAIR>(d_tmem, da, db, idesc, acc0);
 }

@@ -86,8 +86,13 @@ enum {
                                    output block read from one 8-wide input strip
                                    per (channel chunk, kd, kw) (stride 1,
                                    C/G % 32 == 0, O/G % 64 == 0) */
-  CONV_VARIANT_TC_HALO_T_PAIR = 8 /* TC_HALO_T with CTA pairs: M = 256 output channels,
+  CONV_VARIANT_TC_HALO_T_PAIR = 8, /* TC_HALO_T with CTA pairs: M = 256 output channels,
                                    cta_group::2 (O/G % 256 == 0) */
+  CONV_VARIANT_TC_PHASE = 9       /* 2-D layers with few input channels: one GEMM row =
+                                   P output pixels of a row (P*sw*C a multiple of 8),
+                                   its window of the flattened (w, c) input row loaded
+                                   by TMA; N = P*O <= 256, a multiple of 32 (groups 1, width dilation 1,
+                                   H % sh == 0, W*C*2 % 16 == 0, Wo % P == 0) */
 };
 
 /* Output extents.  stride/pad/dil: 3 ints (d, h, w).  out: 3 ints (Do, Ho, Wo).
@@ -106,7 +111,8 @@ int conv_out_dims(int D, int H, int W, int kD, int kH, int kW,
  * as SMs, else (O/G % 128 == 0) TC_TMA_T when there are at least as many
  * 256-pixel tiles as SMs;
  * otherwise TC_TMA_PAIR (or TC_TMA when there are fewer 256-row output tiles
- * than SM pairs); otherwise TC_GATHER.  TC_HALO, TC_HALO_PAIR and
+ * than SM pairs); otherwise TC_PHASE where its conditions hold, else
+ * TC_GATHER.  TC_HALO, TC_HALO_PAIR and
  * TC_HALO_T_PAIR run only when requested through conv_fwd_variant. */
 int conv_fwd(const void* x, const void* w, void* y,
              int N, int D, int H, int W, int C, int O,

@@ -98,7 +98,7 @@ def test_invalid_arguments_rejected_on_host(C):
     big = 1 << 30
     assert call(X, Wt, Y, big, big, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
     # unknown variant
-    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 9, None) == -1
+    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 10, None) == -1
     assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, -2, None) == -1
 
 
@@ -134,8 +134,12 @@ def test_variant_plan(C):
     v, bn, _, _ = plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16",
                        C.VARIANT_TC_HALO_T_PAIR)
     assert v == C.VARIANT_TC_HALO_T_PAIR and bn == 224
-    v, bn, _, _ = plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
-    assert v == C.VARIANT_TC_GATHER and bn == 64
+    # the stem: 3 input channels -> phase packing, 4 pixels x 64 channels per GEMM row
+    v, bn, st, _ = plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
+    assert v == C.VARIANT_TC_PHASE and bn == 256 and st >= 2
+    # ... unless a condition fails (odd H at stride 2; W*C*2 not a multiple of 16)
+    assert plan(2, 1, 15, 16, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
+    assert plan(2, 1, 16, 15, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
     v, bn, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_GATHER and bn == 96
     v, _, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f32")
@@ -165,10 +169,15 @@ def test_explicit_variant_plan(C):
         with pytest.raises(C.ConvError) as e:
             C.plan(*stem, "bf16", getattr(C, "VARIANT_" + name))
         assert e.value.code == -7
+    assert C.plan(*stem, "bf16", C.VARIANT_TC_PHASE)[0] == C.VARIANT_TC_PHASE
+    # phase packing needs C small enough that P*O <= 256
+    with pytest.raises(C.ConvError) as e:
+        C.plan(*g3, "bf16", C.VARIANT_TC_PHASE)
+    assert e.value.code == -7
     # tensor-core variants need f16/bf16
     with pytest.raises(C.ConvError) as e:
         C.plan(*g3, "f32", C.VARIANT_TC_TMA)
     assert e.value.code == -7
     with pytest.raises(C.ConvError) as e:
-        C.plan(*g3, "bf16", 9)
+        C.plan(*g3, "bf16", 10)
     assert e.value.code == -1

@@ -35,14 +35,18 @@ def _geom(wl):
 
 
 @pytest.mark.parametrize("variant", ["TC_GATHER", "TC_TMA", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T",
-                                     "TC_HALO_T", "TC_HALO_T_PAIR"])
+                                     "TC_HALO_T", "TC_HALO_T_PAIR", "TC_PHASE"])
 def test_injected_stall_times_out_and_recovers(variant):
     v = getattr(C, "VARIANT_" + variant)
     O = {"TC_TMA_T": 128, "TC_HALO_T": 128, "TC_HALO_T_PAIR": 256}.get(variant, 64)
-    wl = WL.case(2, 1, 20, 20, 64, O, (1, 3, 3), pad=(0, 1, 1), dtype="f16", seed=21)
+    if variant == "TC_PHASE":   # a stem-like layer: 3 input channels, 7x7 at stride 2
+        wl = WL.case(2, 1, 20, 24, 3, O, (1, 7, 7), (1, 2, 2), (0, 3, 3), dtype="f16", seed=21)
+    else:
+        wl = WL.case(2, 1, 20, 20, 64, O, (1, 3, 3), pad=(0, 1, 1), dtype="f16", seed=21)
     x, w = WL.make_inputs(wl)
     xd, wd = x.cuda(), w.cuda()
-    y = torch.zeros((2, 1, 20, 20, O), dtype=torch.float16, device="cuda")
+    dims = C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil)
+    y = torch.zeros((wl.N, *dims, O), dtype=torch.float16, device="cuda")
     assert C.last_status() == 0
     C.inject_stall(50_000_000)  # 50 ms
     t0 = time.perf_counter()

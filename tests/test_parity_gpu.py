@@ -64,7 +64,19 @@ def variants_for(wl):
         vs.append(C.VARIANT_TC_HALO_T)
     if (wl.C // wl.groups) % 64 == 0 and (wl.O // wl.groups) % 256 == 0 and tuple(wl.stride) == (1, 1, 1):
         vs.append(C.VARIANT_TC_HALO_T_PAIR)
+    if phase_applies(wl):
+        vs.append(C.VARIANT_TC_PHASE)
     return vs
+
+
+def phase_applies(wl):
+    """The phase-packed kernel's conditions, as the library's planner states them."""
+    try:
+        C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil, wl.groups, wl.dtype,
+               C.VARIANT_TC_PHASE)
+        return True
+    except C.ConvError:
+        return False
 
 
 # Small geometries: several 128-row tiles with a ragged tail, every stride /
@@ -132,6 +144,16 @@ SMALL = [
     # all weights resident in shared memory beside two 34-row strip slots and
     # one epilogue staging tile
     WL.case(1, 1, 32, 16, 64, 128, (1, 3, 3), pad=(0, 1, 1), name="ht_resident_one_staging_tile"),
+    # phase packing (few input channels, 2-D): P pixels per GEMM row; left and
+    # right edge windows, ragged last row block, P = 2 / 4 / 8, N = 32 .. 256,
+    # height dilation, no padding
+    WL.case(2, 1, 32, 32, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), name="phase_stem_like"),
+    WL.case(1, 1, 36, 40, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), name="phase_stem_ragged_rows"),
+    WL.case(2, 1, 11, 48, 3, 32, (1, 3, 3), pad=(0, 1, 1), name="phase_c3_s1_p8"),
+    WL.case(2, 1, 14, 30, 4, 64, (1, 5, 5), pad=(0, 2, 2), name="phase_c4_k5_p2"),
+    WL.case(2, 1, 18, 16, 6, 16, (1, 3, 3), (1, 2, 2), (0, 1, 1), name="phase_c6_s2_n32"),
+    WL.case(2, 1, 20, 128, 1, 32, (1, 5, 3), pad=(0, 2, 1), dil=(1, 2, 1), name="phase_c1_dil_h"),
+    WL.case(1, 1, 16, 32, 3, 64, (1, 2, 2), (1, 2, 2), (0, 0, 0), name="phase_patchify_k2s2"),
 ]
 
 
@@ -179,7 +201,7 @@ def test_auto_variant_choice():
     assert C.plan(1, 1, 56, 56, 64, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA
     assert C.plan(4, 32, 32, 32, 64, 128, (3, 3, 3), (2, 2, 2), (1, 1, 1), (1, 1, 1), 1, "f16")[0] in (
         C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR)
-    assert C.plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
+    assert C.plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_PHASE
     assert C.plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f32")[0] == C.VARIANT_SIMT
 
 
