@@ -582,7 +582,10 @@ int plan_phase(const Problem& P, int sms, TcPlan& plan) {
   a.ph_align = al;
   a.ph_wbytes = static_cast<uint32_t>(P.w_bytes);
   a.ph_bblk = static_cast<uint32_t>(BN / 2 * 128);  // per CTA: BN/2 rows of 128 bytes
-  a.ph_epi_bytes = static_cast<uint32_t>(round_up(R * qtot * 64, 1024));
+  a.ph_gcols = BN % 64 == 0 ? 64 : 32;  // store rows of 128 (or 64) bytes
+  // the two staging tiles also hold the copy of w that B is built from
+  a.ph_epi_bytes = static_cast<uint32_t>(
+      std::max<long long>(round_up(R * qtot * 2 * a.ph_gcols, 1024), (static_cast<long long>(P.w_bytes) / 2 + 1023) / 1024 * 1024));
   a.tiles_h = (P.Ho + 2 * R - 1) / (2 * R);  // a pair tile: 2 * ph_rows output rows
   const long long tt = static_cast<long long>(P.N) * a.tiles_h;
   if (tt > 0x7fffffffLL) return CONV_EINVAL;
@@ -593,8 +596,7 @@ int plan_phase(const Problem& P, int sms, TcPlan& plan) {
                           64 - b_bytes - 2LL * a.ph_epi_bytes;
   if (avail < 2LL * a.stage_bytes) return CONV_EUNSUPPORTED;
   a.stages = static_cast<int>(std::min<long long>(4, avail / a.stage_bytes));
-  // w is first copied into the A ring, from which B is built
-  if (static_cast<long long>(P.w_bytes) > static_cast<long long>(a.stages) * a.stage_bytes) return CONV_EUNSUPPORTED;
+  if (static_cast<long long>(P.w_bytes) > 2LL * a.ph_epi_bytes) return CONV_EUNSUPPORTED;
   const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
   a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
             ((static_cast<uint32_t>(2 * kBM) >> 4) << 24);
@@ -933,10 +935,11 @@ int encode_phase_maps(const Problem& P, const TcArgs& a, const void* x, void* y,
     cuuint64_t dim[4] = {row, static_cast<cuuint64_t>(a.ph_qtot), static_cast<cuuint64_t>(P.Ho),
                          static_cast<cuuint64_t>(P.N)};
     cuuint64_t str[3] = {eb * row, eb * row * a.ph_qtot, eb * row * a.ph_qtot * P.Ho};
-    cuuint32_t box[4] = {32u, static_cast<cuuint32_t>(a.ph_qtot), static_cast<cuuint32_t>(a.ph_rows), 1u};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(a.ph_gcols), static_cast<cuuint32_t>(a.ph_qtot),
+                         static_cast<cuuint32_t>(a.ph_rows), 1u};
     const CUresult r = drv.tiled(&my, dt, 4, y, dim, str, box, est, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                                 a.ph_gcols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return CONV_EDRIVER;
     small_tensor_fixup(my, P.y_bytes, drv.driver_version);
   }

@@ -32,16 +32,18 @@
 //
 // CTA pairs (cta_group::2): the pair's MMA is M = 256 (each CTA's 128 GEMM
 // rows: ph_rows output rows each) x N; each CTA holds half of B's N rows,
-// built once in shared memory from a bulk copy of w and kept resident for
-// all tiles.  The epilogue reorders each CTA's accumulator rows (interior
-// windows first, then the edge windows) into output order in a staging tile
-// and stores it with a 4-D TMA store on y viewed as [N, Ho, Wo/P, P*O], which
-// clips rows past Ho.
+// built once in shared memory (by warps 1..5, from a bulk copy of w, while
+// the producer already loads the first windows) and kept resident for all
+// tiles.  The epilogue reorders each CTA's accumulator rows (interior windows
+// first, then the edge windows) into output order, ph_gcols columns at a
+// time, in a swizzled staging tile of 128- (or 64-) byte rows, and stores it
+// with a 4-D TMA store on y viewed as [N, Ho, Wo/P, P*O], which clips rows
+// past Ho.  (Narrower store rows cost the TMA unit as much per row.)
 //
 // Warp roles (192 threads per CTA, one CTA per SM, static tile list): warp 0
 // TMA producer (both CTAs; loads complete on the leader's barriers), warp 1
-// TMEM allocator and, in the leader, MMA issuer, warps 2..5 epilogue; all six
-// build B first.  Waits are bounded as in the other tcgen05 kernels.
+// TMEM allocator and, in the leader, MMA issuer, warps 2..5 epilogue.  Waits
+// are bounded as in the other tcgen05 kernels.
 #pragma once
 
 #include "conv_tct.cuh"
@@ -60,7 +62,7 @@ __global__ void __launch_bounds__(kPhThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* aring = smem;                                                   // stages x one filter row
   uint8_t* bres = aring + static_cast<size_t>(a.stages) * kPhAStage;       // kH blocks of BN/2 rows x 128 B
-  uint8_t* stage_y = bres + static_cast<size_t>(a.kH) * a.ph_bblk;         // 2 staging tiles
+  uint8_t* stage_y = bres + static_cast<size_t>(a.kH) * a.ph_bblk;         // 2 staging tiles (first: w)
   TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(stage_y + 2 * a.ph_epi_bytes);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -81,6 +83,7 @@ __global__ void __launch_bounds__(kPhThreads, 1)
     ptx::mbar_init(ptx::smem_u32(&tail->drain), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->bres), 1u);
+    ptx::mbar_init(ptx::smem_u32(&tail->bready), 2u);  // one arrival per CTA of the pair
     tail->abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -101,58 +104,66 @@ __global__ void __launch_bounds__(kPhThreads, 1)
   volatile int* abort_flag = &tail->abort_flag;
 
   // ---------------------------------------------------------------- resident B
-  // w arrives by one bulk copy into the (not yet used) A ring; its last
-  // w_bytes % 16 bytes by plain loads.
-  const uint16_t* w_s = reinterpret_cast<const uint16_t*>(aring);
-  const uint32_t wb16 = a.ph_wbytes & ~15u;
-  bool ok = true;
-  if (threadIdx.x == 0 && wb16 > 0) {
-    ptx::mbar_arrive_expect_tx(ptx::smem_u32(&tail->bres), wb16);
-    ptx::bulk_load(ptx::smem_u32(aring), a.w, wb16, ptx::smem_u32(&tail->bres));
-  }
-  if (threadIdx.x == 0) {
-    const uint16_t* wg = static_cast<const uint16_t*>(a.w);
-    uint16_t* wt = reinterpret_cast<uint16_t*>(aring);
-    for (uint32_t e = wb16 / 2; e < a.ph_wbytes / 2; ++e) wt[e] = wg[e];
-  }
-  if (wb16 > 0) {
-    ok = wait_bounded(ptx::smem_u32(&tail->bres), 0u, abort_flag, a.timeout_ns, kSiteMmaFull);
-    // the copy must have landed before this CTA can exit, whatever happened
-    if (!ok && threadIdx.x == 0) wait_drain(ptx::smem_u32(&tail->bres), 0u, a.timeout_ns);
-  }
-  __syncthreads();
-  if (ok && !*abort_flag) {
-    // one (filter row, B row) per step: the row's 64 elements as eight
-    // 16-byte chunks, 128-byte swizzle (chunk index XOR row % 8)
-    const int KWC = a.kW * a.C;
-    const int taps_row = a.kH * KWC;  // elements of one output channel's weights
-    for (int pr = threadIdx.x; pr < a.kH * hb; pr += kPhThreads) {
-      const int kh = pr / hb, lr = pr - kh * hb;
-      const int row = static_cast<int>(rank) * hb + lr;
-      const int i = row / a.O, o = row - i * a.O;
-      const int off = a.ph_align - a.pw * a.C + i * a.sw * a.C;
-      const uint16_t* src = w_s + static_cast<long long>(o) * taps_row + kh * KWC;
-      uint8_t* dst = bres + static_cast<size_t>(kh) * a.ph_bblk + lr * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int j0 = 8 * c - off;  // w element of the chunk's first element
-        uint32_t v[4] = {0u, 0u, 0u, 0u};
-        if (j0 + 8 > 0 && j0 < KWC) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int ja = j0 + 2 * e, jb = ja + 1;
-            const uint32_t lo = (ja >= 0 && ja < KWC) ? src[ja] : 0u;
-            const uint32_t hi = (jb >= 0 && jb < KWC) ? src[jb] : 0u;
-            v[e] = lo | (hi << 16);
-          }
-        }
-        *reinterpret_cast<uint4*>(dst + ((c ^ (lr & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+  // w arrives by one bulk copy into the staging tiles (unused until the first
+  // accumulator is ready, which needs B); its last w_bytes % 16 bytes by plain
+  // loads.  Warps 1..5 build this CTA's half of B from it; warp 0 starts
+  // loading windows meanwhile.  The leader's MMA thread waits on `bready`.
+  if (warp != 0) {
+    const uint16_t* w_s = reinterpret_cast<const uint16_t*>(stage_y);
+    const uint32_t wb16 = a.ph_wbytes & ~15u;
+    const int btid = threadIdx.x - 32;
+    constexpr int kBuilders = kPhThreads - 32;
+    bool ok = true;
+    if (btid == 0) {
+      if (wb16 > 0) {
+        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&tail->bres), wb16);
+        ptx::bulk_load(ptx::smem_u32(stage_y), a.w, wb16, ptx::smem_u32(&tail->bres));
       }
+      const uint16_t* wg = static_cast<const uint16_t*>(a.w);
+      uint16_t* wt = reinterpret_cast<uint16_t*>(stage_y);
+      for (uint32_t e = wb16 / 2; e < a.ph_wbytes / 2; ++e) wt[e] = wg[e];
     }
+    if (wb16 > 0) {
+      ok = wait_bounded(ptx::smem_u32(&tail->bres), 0u, abort_flag, a.timeout_ns, kSiteMmaFull);
+      // the copy must have landed before this CTA can exit, whatever happened
+      if (!ok && btid == 0) wait_drain(ptx::smem_u32(&tail->bres), 0u, a.timeout_ns);
+    }
+    named_bar_sync(2, kBuilders);  // the plain-loaded tail of w is visible
+    if (ok) {
+      // one (filter row, B row) per step: the row's 64 elements as eight
+      // 16-byte chunks, 128-byte swizzle (chunk index XOR row % 8)
+      const int KWC = a.kW * a.C;
+      const int taps_row = a.kH * KWC;  // elements of one output channel's weights
+      for (int pr = btid; pr < a.kH * hb; pr += kBuilders) {
+        const int kh = pr / hb, lr = pr - kh * hb;
+        const int row = static_cast<int>(rank) * hb + lr;
+        const int i = row / a.O, o = row - i * a.O;
+        const int off = a.ph_align - a.pw * a.C + i * a.sw * a.C;
+        const uint16_t* src = w_s + static_cast<long long>(o) * taps_row + kh * KWC;
+        uint8_t* dst = bres + static_cast<size_t>(kh) * a.ph_bblk + lr * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int j0 = 8 * c - off;  // w element of the chunk's first element
+          uint32_t v[4] = {0u, 0u, 0u, 0u};
+          if (j0 + 8 > 0 && j0 < KWC) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int ja = j0 + 2 * e, jb = ja + 1;
+              const uint32_t lo = (ja >= 0 && ja < KWC) ? src[ja] : 0u;
+              const uint32_t hi = (jb >= 0 && jb < KWC) ? src[jb] : 0u;
+              v[e] = lo | (hi << 16);
+            }
+          }
+          *reinterpret_cast<uint4*>(dst + ((c ^ (lr & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+        }
+      }
+      ptx::fence_proxy_async_smem();  // B (generic-proxy stores) before the tensor core reads it
+    }
+    named_bar_sync(2, kBuilders);
+    // the leader's MMAs read both CTAs' halves: each CTA reports to the leader
+    // (nothing arrives after a failed copy; the MMA thread's wait then runs out)
+    if (btid == 0 && ok) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(&tail->bready), 0));
   }
-  ptx::fence_proxy_async_smem();  // B (generic-proxy stores) before the tensor core reads it
-  __syncthreads();
-  ptx::cluster_sync();            // the leader's MMAs read both CTAs' halves of B
 
   const int R = a.ph_rows;
   if (warp == 0) {
@@ -215,6 +226,8 @@ __global__ void __launch_bounds__(kPhThreads, 1)
       int t = 0;
       if (mok && a.inject_stall)
         mok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
+      if (mok) mok = wait_bounded(ptx::smem_u32(&tail->bready), 0u, abort_flag, a.timeout_ns, kSiteMmaFull);
+      ptx::tc_fence_after();
       const uint64_t d_a = ptx::smem_desc(ptx::smem_u32(aring), 16, 1024, 2u);  // 128-byte swizzle
       const uint64_t d_b = ptx::smem_desc(ptx::smem_u32(bres), 16, 1024, 2u);
       const uint64_t st_off = desc_off(kPhAStage), bblk = desc_off(a.ph_bblk);
@@ -270,7 +283,11 @@ __global__ void __launch_bounds__(kPhThreads, 1)
         pos = r * a.ph_qtot + (j < a.ph_nleft ? j : a.ph_qtot - a.ph_nright + (j - a.ph_nleft));
     }
     const bool store_thread = warp == 2 && lane == 0;
-    int t = 0, chunk_seq = 0;
+    const int G = a.ph_gcols;               // columns per store: 64 (128-byte rows) or 32 (64-byte)
+    const int row_bytes = 2 * G;
+    const int sw_mask = G == 64 ? 7 : 3;    // 16-byte chunk XOR pattern of the row's swizzle
+    const int sw_shift = G == 64 ? 0 : 1;
+    int t = 0, seq = 0;
     for (int tile = static_cast<int>(blockIdx.x >> 1); tile < a.total_tiles;
          tile += static_cast<int>(gridDim.x >> 1), ++t) {
       const int acc = t & 1;
@@ -284,34 +301,41 @@ __global__ void __launch_bounds__(kPhThreads, 1)
       const int n = tile / a.tiles_h;
       const int oh0 = (tile - n * a.tiles_h) * 2 * R + static_cast<int>(rank) * R;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c), r);
-        ptx::tmem_ld_wait();
-        if (oh0 >= a.Ho) continue;  // this CTA's rows of the last pair tile lie past the output
-        uint8_t* buf = stage_y + (chunk_seq & 1) * a.ph_epi_bytes;
-        // the store issued two steps ago read this buffer; it must be done
-        if (store_thread) ptx::bulk_wait_group_read<1>();
-        named_bar_sync(1, 128);
-        if (pos >= 0) {
-          uint4* dst = reinterpret_cast<uint4*>(buf + pos * 64);
+      const bool live = oh0 < a.Ho;  // this CTA's rows of the last pair tile may lie past the output
+      for (int g = 0; g < BN; g += G) {
+        uint8_t* buf = stage_y + (seq & 1) * a.ph_epi_bytes;
+        if (live) {
+          // the store issued two groups ago read this buffer; it must be done
+          if (store_thread) ptx::bulk_wait_group_read<1>();
+          named_bar_sync(1, 128);
+        }
+        for (int c = 0; c < G; c += 32) {
+          uint32_t r[32];
+          ptx::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(g + c), r);
+          ptx::tmem_ld_wait();
+          if (live && pos >= 0) {
+            uint8_t* rowp = buf + pos * row_bytes;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 v;
-            v.x = pack2<BF16>(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
-            v.y = pack2<BF16>(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
-            v.z = pack2<BF16>(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
-            v.w = pack2<BF16>(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
-            dst[j] = v;
+            for (int j = 0; j < 4; ++j) {
+              uint4 v;
+              v.x = pack2<BF16>(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+              v.y = pack2<BF16>(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+              v.z = pack2<BF16>(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+              v.w = pack2<BF16>(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+              const int chunk = (c >> 3) + j;  // 16-byte chunk of the staging row
+              *reinterpret_cast<uint4*>(rowp + ((chunk ^ ((pos >> sw_shift) & sw_mask)) << 4)) = v;
+            }
           }
         }
-        ptx::fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (store_thread) {
-          ptx::tma_store_4d(&tmap_y, ptx::smem_u32(buf), c, 0, oh0, n);
-          ptx::bulk_commit_group();
+        if (live) {
+          ptx::fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (store_thread) {
+            ptx::tma_store_4d(&tmap_y, ptx::smem_u32(buf), g, 0, oh0, n);
+            ptx::bulk_commit_group();
+          }
+          ++seq;
         }
-        ++chunk_seq;
       }
       ptx::tc_fence_before();
       __syncwarp();

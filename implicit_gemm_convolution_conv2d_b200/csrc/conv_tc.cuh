@@ -111,6 +111,7 @@ struct TcArgs {
   uint32_t ph_wbytes;  // bytes of w
   uint32_t ph_bblk;    // one resident B block: N rows x 32 bytes
   uint32_t ph_epi_bytes;  // one epilogue staging tile
+  int ph_gcols;        // output columns per epilogue store (64: 128-byte swizzle, 32: 64-byte)
   const void* x;
   const void* w;
   void* y;
@@ -126,6 +127,7 @@ struct __align__(8) TcSmemTail {
   uint64_t drain;
   uint64_t stall;     // never arrived on (the injected-timeout test waits here)
   uint64_t bres;      // resident weights loaded
+  uint64_t bready;    // phase-packed kernel: both CTAs' halves of B built (leader's)
   uint64_t afull[8];  // halo kernels: input strip slots
   uint64_t aempty[8];
   uint64_t rfull[3];  // row staging (gather): rows of a tile landed
