@@ -595,7 +595,7 @@ int plan_phase(const Problem& P, int sms, TcPlan& plan) {
   const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
                           64 - b_bytes - 2LL * a.ph_epi_bytes;
   if (avail < 2LL * a.stage_bytes) return CONV_EUNSUPPORTED;
-  a.stages = static_cast<int>(std::min<long long>(4, avail / a.stage_bytes));
+  a.stages = static_cast<int>(std::min<long long>(6, avail / a.stage_bytes));
   if (static_cast<long long>(P.w_bytes) > 2LL * a.ph_epi_bytes) return CONV_EUNSUPPORTED;
   const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
   a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |

@@ -130,31 +130,51 @@ __global__ void __launch_bounds__(kPhThreads, 1)
     }
     named_bar_sync(2, kBuilders);  // the plain-loaded tail of w is visible
     if (ok) {
-      // one (filter row, B row) per step: the row's 64 elements as eight
-      // 16-byte chunks, 128-byte swizzle (chunk index XOR row % 8)
+      // B rows eight per warp step, phase-major: for each filter row kh and
+      // phase i (window offset off_i) this CTA holds, lane l forms word l
+      // (elements 2l, 2l+1) of the 64-element rows of output channels o0..o0+7
+      // -- loads from clamped indices, all 16 issued before the step's stores,
+      // then masked outside the filter row -- and the warp stores each
+      // 128-byte row in the 128-byte swizzle (16-byte chunk XOR row % 8).
       const int KWC = a.kW * a.C;
       const int taps_row = a.kH * KWC;  // elements of one output channel's weights
-      for (int pr = btid; pr < a.kH * hb; pr += kBuilders) {
-        const int kh = pr / hb, lr = pr - kh * hb;
-        const int row = static_cast<int>(rank) * hb + lr;
-        const int i = row / a.O, o = row - i * a.O;
-        const int off = a.ph_align - a.pw * a.C + i * a.sw * a.C;
-        const uint16_t* src = w_s + static_cast<long long>(o) * taps_row + kh * KWC;
-        uint8_t* dst = bres + static_cast<size_t>(kh) * a.ph_bblk + lr * 128;
+      const int bwarp = btid >> 5;
+      constexpr int kBuilderWarps = kBuilders / 32;
+      const uint32_t ws_addr = ptx::smem_u32(w_s);
+      const uint32_t b_addr = ptx::smem_u32(bres);
+      const int r0 = static_cast<int>(rank) * hb;  // first B row of this CTA
+      const int i_begin = r0 / a.O, i_end = (r0 + hb + a.O - 1) / a.O;
+      for (int kh = 0; kh < a.kH; ++kh) {
+        for (int i = i_begin; i < i_end; ++i) {
+          const int off = a.ph_align - a.pw * a.C + i * a.sw * a.C;
+          const int ja = 2 * lane - off, jb = ja + 1;
+          const uint32_t ma = static_cast<unsigned>(ja) < static_cast<unsigned>(KWC) ? 0xffffu : 0u;
+          const uint32_t mb = static_cast<unsigned>(jb) < static_cast<unsigned>(KWC) ? 0xffffu : 0u;
+          const uint32_t ca = 2u * static_cast<uint32_t>(min(max(ja, 0), KWC - 1));
+          const uint32_t cb = 2u * static_cast<uint32_t>(min(max(jb, 0), KWC - 1));
+          const int o_begin = max(0, r0 - i * a.O), o_end = min(a.O, r0 + hb - i * a.O);
+          const int lrb = i * a.O - r0;  // this CTA's B row of (i, o = 0)
+          const uint32_t blk = b_addr + static_cast<uint32_t>(kh) * a.ph_bblk + ((lane & 3) << 2);
+          for (int o0 = o_begin + 8 * bwarp; o0 < o_end; o0 += 8 * kBuilderWarps) {
+            uint32_t ha[8], hv[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int j0 = 8 * c - off;  // w element of the chunk's first element
-          uint32_t v[4] = {0u, 0u, 0u, 0u};
-          if (j0 + 8 > 0 && j0 < KWC) {
+            for (int u = 0; u < 8; ++u) {
+              const int o = min(o0 + u, o_end - 1);
+              const uint32_t base = ws_addr + 2u * static_cast<uint32_t>(o * taps_row + kh * KWC);
+              ha[u] = lds16(base + ca);
+              hv[u] = lds16(base + cb);
+            }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int ja = j0 + 2 * e, jb = ja + 1;
-              const uint32_t lo = (ja >= 0 && ja < KWC) ? src[ja] : 0u;
-              const uint32_t hi = (jb >= 0 && jb < KWC) ? src[jb] : 0u;
-              v[e] = lo | (hi << 16);
+            for (int u = 0; u < 8; ++u) {
+              if (o0 + u < o_end) {
+                const int lr = lrb + o0 + u;
+                const uint32_t v = (ha[u] & ma) | ((hv[u] & mb) << 16);
+                asm volatile("st.shared.b32 [%0], %1;"
+                             ::"r"(blk + static_cast<uint32_t>(lr) * 128u + (((lane >> 2) ^ (lr & 7)) << 4)), "r"(v)
+                             : "memory");
+              }
             }
           }
-          *reinterpret_cast<uint4*>(dst + ((c ^ (lr & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
         }
       }
       ptx::fence_proxy_async_smem();  // B (generic-proxy stores) before the tensor core reads it
@@ -309,20 +329,24 @@ __global__ void __launch_bounds__(kPhThreads, 1)
           if (store_thread) ptx::bulk_wait_group_read<1>();
           named_bar_sync(1, 128);
         }
-        for (int c = 0; c < G; c += 32) {
-          uint32_t r[32];
-          ptx::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(g + c), r);
-          ptx::tmem_ld_wait();
-          if (live && pos >= 0) {
-            uint8_t* rowp = buf + pos * row_bytes;
+        // both 32-column halves of a 64-column group in flight before one wait
+        uint32_t r[2][32];
+        ptx::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(g), r[0]);
+        if (G == 64) ptx::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(g + 32), r[1]);
+        ptx::tmem_ld_wait();
+        if (live && pos >= 0) {
+          uint8_t* rowp = buf + pos * row_bytes;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (h * 32 >= G) break;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               uint4 v;
-              v.x = pack2<BF16>(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
-              v.y = pack2<BF16>(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
-              v.z = pack2<BF16>(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
-              v.w = pack2<BF16>(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
-              const int chunk = (c >> 3) + j;  // 16-byte chunk of the staging row
+              v.x = pack2<BF16>(__uint_as_float(r[h][8 * j + 0]), __uint_as_float(r[h][8 * j + 1]));
+              v.y = pack2<BF16>(__uint_as_float(r[h][8 * j + 2]), __uint_as_float(r[h][8 * j + 3]));
+              v.z = pack2<BF16>(__uint_as_float(r[h][8 * j + 4]), __uint_as_float(r[h][8 * j + 5]));
+              v.w = pack2<BF16>(__uint_as_float(r[h][8 * j + 6]), __uint_as_float(r[h][8 * j + 7]));
+              const int chunk = 4 * h + j;  // 16-byte chunk of the staging row
               *reinterpret_cast<uint4*>(rowp + ((chunk ^ ((pos >> sw_shift) & sw_mask)) << 4)) = v;
             }
           }
