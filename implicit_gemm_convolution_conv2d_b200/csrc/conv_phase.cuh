@@ -112,7 +112,8 @@ __global__ void __launch_bounds__(kPhThreads, 1)
     const uint16_t* w_s = reinterpret_cast<const uint16_t*>(stage_y);
     const uint32_t wb16 = a.ph_wbytes & ~15u;
     const int btid = threadIdx.x - 32;
-    constexpr int kBuilders = kPhThreads - 32;
+    constexpr int kBuilders = kPhThreads - 32;  // warps 1..5: all of them arrive on named barrier 2
+    static_assert(kBuilders == 160, "the B builders are exactly warps 1..5");
     bool ok = true;
     if (btid == 0) {
       if (wb16 > 0) {

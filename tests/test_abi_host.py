@@ -137,9 +137,9 @@ def test_variant_plan(C):
     # the stem: 3 input channels -> phase packing, 4 pixels x 64 channels per GEMM row
     v, bn, st, _ = plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
     assert v == C.VARIANT_TC_PHASE and bn == 256 and st >= 2
-    # ... unless a condition fails (odd H at stride 2; W*C*2 not a multiple of 16)
-    assert plan(2, 1, 15, 16, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
+    # ... unless a condition fails (W*C*2 not a multiple of 16; Wo not a multiple of P)
     assert plan(2, 1, 16, 15, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
+    assert plan(2, 1, 16, 24, 3, 64, (1, 7, 7), (1, 3, 3), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
     v, bn, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_GATHER and bn == 96
     v, _, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f32")

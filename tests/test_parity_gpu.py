@@ -154,6 +154,8 @@ SMALL = [
     WL.case(2, 1, 18, 16, 6, 16, (1, 3, 3), (1, 2, 2), (0, 1, 1), name="phase_c6_s2_n32"),
     WL.case(2, 1, 20, 128, 1, 32, (1, 5, 3), pad=(0, 2, 1), dil=(1, 2, 1), name="phase_c1_dil_h"),
     WL.case(1, 1, 16, 32, 3, 64, (1, 2, 2), (1, 2, 2), (0, 0, 0), name="phase_patchify_k2s2"),
+    WL.case(1, 1, 17, 32, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), name="phase_odd_h"),
+    WL.case(1, 1, 20, 200, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), name="phase_wide_rows_3_boxes"),
 ]
 
 
