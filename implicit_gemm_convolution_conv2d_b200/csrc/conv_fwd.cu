@@ -385,7 +385,7 @@ int plan_tc_t(const Problem& P, int sms, TcPlan& plan) {
   a.b_bytes = static_cast<uint32_t>(a.BN * a.kc * 2);   // patch rows
   a.sub_bytes = a.a_bytes + a.b_bytes;
   const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) -
-                          64 - 2LL * kTEpiBytes;
+                          64 - 2LL * kTEpiGroups * kTEpiBytes;
   int stages = 0;
   a.kbs = choose_kbs(a.BN, a.kc, a.sub_bytes, avail, 8, stages);
   if (stages < 2) return CONV_EUNSUPPORTED;
@@ -399,8 +399,8 @@ int plan_tc_t(const Problem& P, int sms, TcPlan& plan) {
   plan.variant = CONV_VARIANT_TC_TMA_T;
   plan.pair = false;
   plan.ctas = std::min(a.total_tiles, sms);
-  plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + 2 * static_cast<size_t>(kTEpiBytes) + 1024 +
-              sizeof(TcSmemTail) + 64;
+  plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + 2 * kTEpiGroups * static_cast<size_t>(kTEpiBytes) +
+              1024 + sizeof(TcSmemTail) + 64;
   return CONV_OK;
 }
 
@@ -1023,8 +1023,8 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
     rc = encode_maps(P, a, false, false, x, w, mx, mw, kTO);
     if (rc == CONV_OK) rc = encode_y_map(P, y, my);
     if (rc != CONV_OK) return rc;
-    if (P.dtype == CONV_BF16) conv_fwd_tc_t_kernel<true><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
-    else                      conv_fwd_tc_t_kernel<false><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
+    if (P.dtype == CONV_BF16) conv_fwd_tc_t_kernel<true><<<plan.ctas, kTTileThreads, plan.smem, st>>>(mx, mw, my, a);
+    else                      conv_fwd_tc_t_kernel<false><<<plan.ctas, kTTileThreads, plan.smem, st>>>(mx, mw, my, a);
     return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
   }
   rc = encode_maps(P, a, plan.pair, halo, x, w, mx, mw);

@@ -14,19 +14,23 @@
 // their roles change.
 //
 // The accumulator holds y^T: tensor-memory lane = output channel, column =
-// output pixel.  The epilogue therefore transposes through shared memory: each
-// of the four epilogue warps reads its 32 channels x 32 pixels, writes them as
-// 32 pixel rows of a [32 pixels][128 channels] staging tile, and one thread
+// output pixel.  The epilogue therefore transposes through shared memory: a
+// group of four warps reads 32 channels x 32 pixels each, writes them as 32
+// pixel rows of a [32 pixels][128 channels] staging tile, and one thread
 // stores the tile to y with a TMA tensor store (y viewed as [M][O]; rows
-// beyond M are clipped by the tensor map).  Two staging tiles alternate so the
-// next transpose overlaps the previous store.
+// beyond M are clipped by the tensor map).  Two staging tiles per group
+// alternate so the next transpose overlaps the previous store, and two groups
+// take alternate 32-pixel chunks (the epilogue, not the MMA, limits layers
+// with a short reduction such as 3x1x1 over 64 channels).
 //
-// Warp roles (192 threads, one CTA per SM, static tile list):
+// Warp roles (320 threads, one CTA per SM, static tile list):
 //   warp 0      TMA producer (one thread): per K sub-block one weight tile
 //               (128 x kc) and BP/128 im2col loads of 128 pixels x kc;
 //   warp 1      TMEM allocator and MMA issuer (one thread);
-//   warps 2..5  epilogue; warp w reads tensor-memory lanes 32*(w%4)..+31.
-// Waits are bounded exactly as in the other tcgen05 kernels.
+//   warps 2..9  epilogue, groups 2..5 and 6..9; warp w reads tensor-memory
+//               lanes 32*(w%4)..+31.
+// Waits are bounded exactly as in the other tcgen05 kernels; each group's
+// named barrier (1 or 2) is reached by exactly its four warps.
 #pragma once
 
 #include "conv_tc.cuh"
@@ -37,6 +41,10 @@ constexpr int kTO = 128;                 // output channels per tile (MMA M)
 constexpr int kTEpiRows = 32;            // pixels per staging tile
 constexpr uint32_t kTEpiBytes = kTEpiRows * kTO * 2;  // 8 KB
 constexpr int kTThreads = 192;
+// The transposed im2col kernel runs two epilogue groups of four warps (even
+// and odd 32-column chunks), each with its own staging tiles and store thread.
+constexpr int kTEpiGroups = 2;
+constexpr int kTTileThreads = 32 * (2 + 4 * kTEpiGroups);
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -57,13 +65,13 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bo
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kTThreads, 1)
+__global__ void __launch_bounds__(kTTileThreads, 1)
     conv_fwd_tc_t_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                          const __grid_constant__ CUtensorMap tmap_y, const TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* stage_y = smem + static_cast<size_t>(a.stages) * a.stage_bytes;
-  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(stage_y + 2 * kTEpiBytes);
+  uint8_t* stage_y = smem + static_cast<size_t>(a.stages) * a.stage_bytes;  // 2 per epilogue group
+  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(stage_y + 2 * kTEpiGroups * kTEpiBytes);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int BP = a.BN;                   // output pixels per tile (MMA N)
@@ -77,7 +85,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(ptx::smem_u32(&tail->acc_full[b]), 1u);
-      ptx::mbar_init(ptx::smem_u32(&tail->acc_empty[b]), 4u);
+      ptx::mbar_init(ptx::smem_u32(&tail->acc_empty[b]), 4u * kTEpiGroups);
     }
     ptx::mbar_init(ptx::smem_u32(&tail->drain), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
@@ -219,38 +227,44 @@ __global__ void __launch_bounds__(kTThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    // group g = (warp - 2) / 4 takes 32-column chunks g, g + 2, ...; its four
+    // warps cover the four tensor-memory lane quarters and synchronise on
+    // named barrier 1 + g
     const int q = warp & 3;                  // tensor-memory lane quarter: channels 32q .. 32q+31
-    const bool store_thread = warp == 2 && lane == 0;
+    const int grp = (warp - 2) >> 2;
+    const uint32_t bar_id = 1u + static_cast<uint32_t>(grp);
+    const bool store_thread = warp == 2 + 4 * grp && lane == 0;
+    uint8_t* const stage_g = stage_y + 2 * grp * kTEpiBytes;
     int t = 0, chunk_seq = 0;
     for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++t) {
       const int acc = t & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
       bool ok = wait_bounded_warp(ptx::smem_u32(&tail->acc_full[acc]), acc_phase, abort_flag, a.timeout_ns,
                                   kSiteEpiAccFull);
-      // the four warps agree before any of them enters the named barriers
-      // below: a warp whose wait gave up must not leave the others waiting
-      ok = named_bar_and(1, 128, ok);
+      // the group's four warps agree before any of them enters the named
+      // barriers below: a warp whose wait gave up must not leave the others waiting
+      ok = named_bar_and(bar_id, 128, ok);
       if (!ok) break;
       ptx::tc_fence_after();
       const TileCoord tc = decode_tile(a, tile);
       const long long m0 = static_cast<long long>(tc.mt) * BP;
       const int o0 = tc.g * a.Og + tc.nt * kTO;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BP);
-      for (int c = 0; c < BP; c += kTEpiRows) {
+      for (int c = grp * kTEpiRows; c < BP; c += kTEpiGroups * kTEpiRows) {
         uint32_t r[32];
         ptx::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c), r);
         ptx::tmem_ld_wait();
         const long long mrow = m0 + c;
-        if (mrow >= a.M) continue;           // the same for every epilogue thread
-        uint8_t* buf = stage_y + (chunk_seq & 1) * kTEpiBytes;
+        if (mrow >= a.M) continue;           // the same for every thread of the group
+        uint8_t* buf = stage_g + (chunk_seq & 1) * kTEpiBytes;
         // the store issued two chunks ago read this buffer; it must be done
         if (store_thread) ptx::bulk_wait_group_read<1>();
-        named_bar_sync(1, 128);
+        named_bar_sync(bar_id, 128);
         uint16_t* dst = reinterpret_cast<uint16_t*>(buf) + q * 32 + lane;
 #pragma unroll
         for (int p = 0; p < kTEpiRows; ++p) dst[p * kTO] = cvt1<BF16>(__uint_as_float(r[p]));
         ptx::fence_proxy_async_smem();
-        named_bar_sync(1, 128);
+        named_bar_sync(bar_id, 128);
         if (store_thread) {
           ptx::tma_store_2d(&tmap_y, ptx::smem_u32(buf), o0, static_cast<int32_t>(mrow));
           ptx::bulk_commit_group();
