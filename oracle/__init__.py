@@ -69,6 +69,15 @@ class Oracle:
         lib.oracle_conv_fwd_points.restype = ctypes.c_int
         lib.oracle_out_dims.argtypes = [ctypes.c_int] * 6 + [i3, i3, i3, i3]
         lib.oracle_out_dims.restype = ctypes.c_int
+        # padding below / above and the flip flag (the forms with "_ex")
+        common_ex = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int] + [ctypes.c_int] * 9 + \
+            [i3, i3, i3, i3, ctypes.c_int, ctypes.c_int]
+        lib.oracle_conv_fwd_ex.argtypes = common_ex + [dp, dp]
+        lib.oracle_conv_fwd_ex.restype = ctypes.c_int
+        lib.oracle_conv_fwd_points_ex.argtypes = common_ex + [ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, dp, dp]
+        lib.oracle_conv_fwd_points_ex.restype = ctypes.c_int
+        lib.oracle_out_dims_ex.argtypes = [ctypes.c_int] * 6 + [i3, i3, i3, i3, i3]
+        lib.oracle_out_dims_ex.restype = ctypes.c_int
         lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
         lib.oracle_f16_to_f64.restype = ctypes.c_double
         lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
@@ -82,52 +91,62 @@ class Oracle:
         self.lib = lib
         self.path = path
 
-    def out_dims(self, D, H, W, kD, kH, kW, stride, pad, dil):
-        """Output extents (Do, Ho, Wo): floor((I + 2p - dil*(k-1) - 1)/s) + 1 per dimension."""
+    def out_dims(self, D, H, W, kD, kH, kW, stride, pad, dil, pad_hi=None):
+        """Output extents (Do, Ho, Wo): floor((I + p_lo + p_hi - dil*(k-1) - 1)/s) + 1 per
+        dimension; `pad` is the padding below (and above, unless `pad_hi` is given)."""
         out = (ctypes.c_int * 3)()
-        rc = self.lib.oracle_out_dims(D, H, W, kD, kH, kW, _i3(stride), _i3(pad), _i3(dil), out)
+        rc = self.lib.oracle_out_dims_ex(D, H, W, kD, kH, kW, _i3(stride), _i3(pad),
+                                         _i3(pad if pad_hi is None else pad_hi), _i3(dil), out)
         if rc:
             raise ValueError("oracle.out_dims: invalid geometry")
         return tuple(out)
 
-    def conv_fwd(self, x, w, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1):
+    def conv_fwd(self, x, w, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1, pad_hi=None,
+                 flip=False):
         """Full output of the direct sum.
 
         x: [N, D, H, W, C] and w: [O, kD, kH, kW, C/groups] CPU tensors (float32,
-        float16 or bfloat16, both the same).  Returns (y, S), float64 NumPy arrays
-        of shape [N, Do, Ho, Wo, O]: y the sum, S = sum |x*w| over the same terms.
+        float16 or bfloat16, both the same).  `pad` pads below each dimension
+        (and above, unless `pad_hi` is given); `flip` reads the filter reversed
+        in every spatial dimension (a true convolution).  Returns (y, S), float64
+        NumPy arrays of shape [N, Do, Ho, Wo, O]: y the sum, S = sum |x*w| over
+        the same terms.
         """
         px, nx, kx = _raw(x)
         pw, nw, kw_ = _raw(w)
         if nx != nw:
             raise TypeError("oracle: x and w must share a dtype")
         N, D, H, W, C, O, kD, kH, kW = _shape_args(kx, kw_, groups)
-        Do, Ho, Wo = self.out_dims(D, H, W, kD, kH, kW, stride, pad, dil)
+        hi = pad if pad_hi is None else pad_hi
+        Do, Ho, Wo = self.out_dims(D, H, W, kD, kH, kW, stride, pad, dil, hi)
         y = np.empty((N, Do, Ho, Wo, O), dtype=np.float64)
         s = np.empty_like(y)
         dp = ctypes.POINTER(ctypes.c_double)
-        rc = self.lib.oracle_conv_fwd(px, pw, DTYPE_CODE[nx], N, D, H, W, C, O, kD, kH, kW,
-                                      _i3(stride), _i3(pad), _i3(dil), int(groups),
-                                      y.ctypes.data_as(dp), s.ctypes.data_as(dp))
+        rc = self.lib.oracle_conv_fwd_ex(px, pw, DTYPE_CODE[nx], N, D, H, W, C, O, kD, kH, kW,
+                                         _i3(stride), _i3(pad), _i3(hi), _i3(dil), int(groups), int(bool(flip)),
+                                         y.ctypes.data_as(dp), s.ctypes.data_as(dp))
         if rc:
             raise ValueError(f"oracle.conv_fwd failed ({rc})")
         return y, s
 
-    def conv_fwd_points(self, x, w, idx, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1):
+    def conv_fwd_points(self, x, w, idx, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1,
+                        pad_hi=None, flip=False):
         """Selected outputs: idx are flat indices into [N, Do, Ho, Wo, O]. Returns (y, S) float64."""
         px, nx, kx = _raw(x)
         pw, nw, kw_ = _raw(w)
         if nx != nw:
             raise TypeError("oracle: x and w must share a dtype")
         N, D, H, W, C, O, kD, kH, kW = _shape_args(kx, kw_, groups)
+        hi = pad if pad_hi is None else pad_hi
         idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int64).ravel())
         y = np.empty(idx.shape[0], dtype=np.float64)
         s = np.empty_like(y)
         dp = ctypes.POINTER(ctypes.c_double)
-        rc = self.lib.oracle_conv_fwd_points(px, pw, DTYPE_CODE[nx], N, D, H, W, C, O, kD, kH, kW,
-                                             _i3(stride), _i3(pad), _i3(dil), int(groups),
-                                             idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
-                                             idx.shape[0], y.ctypes.data_as(dp), s.ctypes.data_as(dp))
+        rc = self.lib.oracle_conv_fwd_points_ex(px, pw, DTYPE_CODE[nx], N, D, H, W, C, O, kD, kH, kW,
+                                                _i3(stride), _i3(pad), _i3(hi), _i3(dil), int(groups),
+                                                int(bool(flip)),
+                                                idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                                idx.shape[0], y.ctypes.data_as(dp), s.ctypes.data_as(dp))
         if rc:
             raise ValueError(f"oracle.conv_fwd_points failed ({rc})")
         return y, s
@@ -173,16 +192,17 @@ def _shape_args(x, w, groups):
     return N, D, H, W, C, O, kD, kH, kW
 
 
-def out_dims(D, H, W, kD, kH, kW, stride, pad, dil):
-    return default().out_dims(D, H, W, kD, kH, kW, stride, pad, dil)
+def out_dims(D, H, W, kD, kH, kW, stride, pad, dil, pad_hi=None):
+    return default().out_dims(D, H, W, kD, kH, kW, stride, pad, dil, pad_hi)
 
 
-def conv_fwd(x, w, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1):
-    return default().conv_fwd(x, w, stride, pad, dil, groups)
+def conv_fwd(x, w, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1, pad_hi=None, flip=False):
+    return default().conv_fwd(x, w, stride, pad, dil, groups, pad_hi, flip)
 
 
-def conv_fwd_points(x, w, idx, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1):
-    return default().conv_fwd_points(x, w, idx, stride, pad, dil, groups)
+def conv_fwd_points(x, w, idx, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1, pad_hi=None,
+                    flip=False):
+    return default().conv_fwd_points(x, w, idx, stride, pad, dil, groups, pad_hi, flip)
 
 
 conv_fwd.__doc__ = Oracle.conv_fwd.__doc__

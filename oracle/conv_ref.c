@@ -30,6 +30,15 @@
  *   The tutorial's ResNet-50 example (224x224 input, 7x7, stride 2, giving a
  *   112x112 output in its FLOP count) is consistent with this at pad 3.
  *
+ *   Two options are also provided, each in its plainest reading.  Flip (the
+ *   MLX pull request's "What changed" list: its input loader handles a
+ *   "correct flip" of the filter) reads the filter reversed in every spatial
+ *   dimension, w[o, kD-1-kd, kH-1-kh, kW-1-kw, c] -- a true convolution
+ *   instead of the cross-correlation.  Per-side padding is the general form
+ *   of the padding above: p_lo below and p_hi above a dimension (the index
+ *   origin is -p_lo; the extent uses p_lo + p_hi in place of 2p).  With
+ *   p_lo = p_hi = p and no flip they reduce to the definition above.
+ *
  * Alongside y the oracle returns S = sum |x*w| over the same receptive field;
  * the parity tolerance is expressed relative to S.
  *
@@ -134,25 +143,33 @@ uint16_t oracle_f64_to_bf16_rn(double v) {
 
 /* ---- output extent ---------------------------------------------------- */
 
-static int64_t extent(int64_t in, int k, int s, int p, int d) {
-  int64_t num = in + 2 * (int64_t)p - (int64_t)d * (k - 1) - 1;
+static int64_t extent(int64_t in, int k, int s, int p_lo, int p_hi, int d) {
+  int64_t num = in + (int64_t)p_lo + (int64_t)p_hi - (int64_t)d * (k - 1) - 1;
   if (num < 0) return 0;
   return num / s + 1;
+}
+
+/* Output extents with padding p_lo below and p_hi above each dimension. */
+int oracle_out_dims_ex(int D, int H, int W, int kD, int kH, int kW,
+                       const int stride[3], const int pad_lo[3],
+                       const int pad_hi[3], const int dil[3], int out[3]) {
+  const int in[3] = {D, H, W};
+  const int k[3] = {kD, kH, kW};
+  for (int i = 0; i < 3; ++i) {
+    if (in[i] <= 0 || k[i] <= 0 || stride[i] <= 0 || dil[i] <= 0 ||
+        pad_lo[i] < 0 || pad_hi[i] < 0)
+      return -1;
+    int64_t e = extent(in[i], k[i], stride[i], pad_lo[i], pad_hi[i], dil[i]);
+    if (e <= 0 || e > 0x7fffffff) return -1;
+    out[i] = (int)e;
+  }
+  return 0;
 }
 
 int oracle_out_dims(int D, int H, int W, int kD, int kH, int kW,
                     const int stride[3], const int pad[3], const int dil[3],
                     int out[3]) {
-  const int in[3] = {D, H, W};
-  const int k[3] = {kD, kH, kW};
-  for (int i = 0; i < 3; ++i) {
-    if (in[i] <= 0 || k[i] <= 0 || stride[i] <= 0 || dil[i] <= 0 || pad[i] < 0)
-      return -1;
-    int64_t e = extent(in[i], k[i], stride[i], pad[i], dil[i]);
-    if (e <= 0 || e > 0x7fffffff) return -1;
-    out[i] = (int)e;
-  }
-  return 0;
+  return oracle_out_dims_ex(D, H, W, kD, kH, kW, stride, pad, pad, dil, out);
 }
 
 /* ---- the direct sum ---------------------------------------------------- */
@@ -160,22 +177,27 @@ int oracle_out_dims(int D, int H, int W, int kD, int kH, int kW,
 typedef struct {
   int N, D, H, W, C, O, kD, kH, kW, G;
   int Do, Ho, Wo;
-  int s[3], p[3], d[3];
+  int s[3], p[3], d[3];  /* p: the padding below (the index origin is -p) */
+  int flip;              /* read the filter reversed in every spatial dimension */
 } shape_t;
 
 static int make_shape(shape_t* sh, int N, int D, int H, int W, int C, int O,
                       int kD, int kH, int kW, const int stride[3],
-                      const int pad[3], const int dil[3], int groups) {
+                      const int pad_lo[3], const int pad_hi[3],
+                      const int dil[3], int groups, int flip) {
   int out[3];
   if (N <= 0 || C <= 0 || O <= 0 || groups <= 0) return -1;
   if (C % groups || O % groups) return -1;
-  if (oracle_out_dims(D, H, W, kD, kH, kW, stride, pad, dil, out)) return -1;
+  if (flip != 0 && flip != 1) return -1;
+  if (oracle_out_dims_ex(D, H, W, kD, kH, kW, stride, pad_lo, pad_hi, dil, out))
+    return -1;
   sh->N = N; sh->D = D; sh->H = H; sh->W = W; sh->C = C; sh->O = O;
   sh->kD = kD; sh->kH = kH; sh->kW = kW; sh->G = groups;
   sh->Do = out[0]; sh->Ho = out[1]; sh->Wo = out[2];
   for (int i = 0; i < 3; ++i) {
-    sh->s[i] = stride[i]; sh->p[i] = pad[i]; sh->d[i] = dil[i];
+    sh->s[i] = stride[i]; sh->p[i] = pad_lo[i]; sh->d[i] = dil[i];
   }
+  sh->flip = flip;
   return 0;
 }
 
@@ -197,7 +219,10 @@ static int make_shape(shape_t* sh, int N, int D, int H, int W, int C, int O,
           if (iw < 0 || iw >= sh->W) continue;                               \
           int64_t xb = ((((int64_t)n * sh->D + id) * sh->H + ih) * sh->W + iw) \
                        * sh->C + (int64_t)g * Cg;                            \
-          int64_t wb = ((((int64_t)o * sh->kD + kd) * sh->kH + kh) * sh->kW + kw) \
+          const int fd = sh->flip ? sh->kD - 1 - kd : kd;                    \
+          const int fh = sh->flip ? sh->kH - 1 - kh : kh;                    \
+          const int fw = sh->flip ? sh->kW - 1 - kw : kw;                    \
+          int64_t wb = ((((int64_t)o * sh->kD + fd) * sh->kH + fh) * sh->kW + fw) \
                        * Cg;                                                 \
           for (int c = 0; c < Cg; ++c) {                                     \
             double t = XAT(xb + c) * WAT(wb + c);                            \
@@ -243,13 +268,15 @@ static double* decode_all(const void* p, int64_t n, int dtype) {
  * [N,Do,Ho,Wo,O] doubles.  dtype: 0 = binary32, 1 = binary16, 2 = bfloat16.
  * Returns 0, or -1 on an invalid shape, -2 on an unknown dtype, -3 when out
  * of host memory. */
-int oracle_conv_fwd(const void* x, const void* w, int dtype, int N, int D,
-                    int H, int W, int C, int O, int kD, int kH, int kW,
-                    const int stride[3], const int pad[3], const int dil[3],
-                    int groups, double* y, double* s) {
+int oracle_conv_fwd_ex(const void* x, const void* w, int dtype, int N, int D,
+                       int H, int W, int C, int O, int kD, int kH, int kW,
+                       const int stride[3], const int pad_lo[3],
+                       const int pad_hi[3], const int dil[3], int groups,
+                       int flip, double* y, double* s) {
   shape_t sh;
   if (dtype < 0 || dtype > 2) return -2;
-  if (make_shape(&sh, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups))
+  if (make_shape(&sh, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil,
+                 groups, flip))
     return -1;
   int64_t nx = (int64_t)N * D * H * W * C;
   int64_t nw = (int64_t)O * kD * kH * kW * (C / groups);
@@ -275,14 +302,16 @@ int oracle_conv_fwd(const void* x, const void* w, int dtype, int N, int D,
 /* Selected outputs only: idx[i] is a flat index into [N,Do,Ho,Wo,O].
  * Reads x and w in their storage type, so it needs no copy of the input.
  * Returns 0, -1 (shape), -2 (dtype) or -4 (an index out of range). */
-int oracle_conv_fwd_points(const void* x, const void* w, int dtype, int N,
-                           int D, int H, int W, int C, int O, int kD, int kH,
-                           int kW, const int stride[3], const int pad[3],
-                           const int dil[3], int groups, const int64_t* idx,
-                           int64_t npts, double* y, double* s) {
+int oracle_conv_fwd_points_ex(const void* x, const void* w, int dtype, int N,
+                              int D, int H, int W, int C, int O, int kD, int kH,
+                              int kW, const int stride[3], const int pad_lo[3],
+                              const int pad_hi[3], const int dil[3], int groups,
+                              int flip, const int64_t* idx, int64_t npts,
+                              double* y, double* s) {
   shape_t sh;
   if (dtype < 0 || dtype > 2) return -2;
-  if (make_shape(&sh, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups))
+  if (make_shape(&sh, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil,
+                 groups, flip))
     return -1;
   int64_t total = (int64_t)sh.N * sh.Do * sh.Ho * sh.Wo * sh.O;
   for (int64_t i = 0; i < npts; ++i)
@@ -299,6 +328,25 @@ int oracle_conv_fwd_points(const void* x, const void* w, int dtype, int N,
     point_raw(shp, x, w, dtype, n, od, oh, ow, o, &y[i], &s[i]);
   }
   return 0;
+}
+
+/* The symmetric-padding, unflipped forms (the definition above). */
+int oracle_conv_fwd(const void* x, const void* w, int dtype, int N, int D,
+                    int H, int W, int C, int O, int kD, int kH, int kW,
+                    const int stride[3], const int pad[3], const int dil[3],
+                    int groups, double* y, double* s) {
+  return oracle_conv_fwd_ex(x, w, dtype, N, D, H, W, C, O, kD, kH, kW, stride,
+                            pad, pad, dil, groups, 0, y, s);
+}
+
+int oracle_conv_fwd_points(const void* x, const void* w, int dtype, int N,
+                           int D, int H, int W, int C, int O, int kD, int kH,
+                           int kW, const int stride[3], const int pad[3],
+                           const int dil[3], int groups, const int64_t* idx,
+                           int64_t npts, double* y, double* s) {
+  return oracle_conv_fwd_points_ex(x, w, dtype, N, D, H, W, C, O, kD, kH, kW,
+                                   stride, pad, pad, dil, groups, 0, idx, npts,
+                                   y, s);
 }
 
 int oracle_max_threads(void) {

@@ -299,6 +299,67 @@ def pin_points_match_full(orc):
         assert np.array_equal(yp, y.ravel()[idx]) and np.array_equal(Sp, S.ravel()[idx])
 
 
+# ---------------------------------------------------------------------------
+# The two options of the MLX pull request's discussion: flip and per-side padding
+# ---------------------------------------------------------------------------
+
+def pin_flip_tutorial_example(orc):
+    """The tutorial's worked example with the filter flipped: the kernel acts as
+    [[-1,0],[0,1]], each output is x[i+1][j+1] - x[i][j] = 4 for the input 1..9,
+    exactly; flipping a filter that is its own reversal changes nothing."""
+    g = json.load(open(os.path.join(GOLDEN, "tutorial_tiny_example.json")))
+    x = _t(g["x_hw"]).reshape(1, 1, 3, 3, 1)
+    w = _t(g["k_hw"]).reshape(1, 1, 2, 2, 1)
+    y, _ = orc.conv_fwd(x, w, flip=True)
+    assert np.array_equal(y.reshape(2, 2), np.full((2, 2), 4.0)), y.reshape(2, 2)
+    sym = _t([[1.0, 2.0], [2.0, 1.0]]).reshape(1, 1, 2, 2, 1)
+    assert np.array_equal(orc.conv_fwd(x, sym, flip=True)[0], orc.conv_fwd(x, sym)[0])
+
+
+_GEOMS_EX = [
+    # (N, D, H, W, C, O, k, stride, pad_lo, pad_hi, dil, groups)
+    (1, 1, 7, 9, 3, 4, (1, 3, 3), (1, 1, 1), (0, 1, 2), (0, 2, 0), (1, 1, 1), 1),
+    (2, 5, 6, 7, 4, 6, (3, 2, 3), (2, 1, 2), (1, 0, 2), (0, 1, 1), (1, 2, 1), 2),
+    (1, 1, 9, 8, 2, 3, (1, 4, 3), (1, 2, 1), (0, 3, 0), (0, 0, 2), (1, 1, 2), 1),
+]
+
+
+def pin_flip_and_side_padding_torch_witness(orc):
+    """torch float64 convolution of the explicitly zero-padded input (F.pad with
+    the two sides' amounts, then no padding), with the filter reversed by torch
+    in its spatial dimensions for flip, agrees on y and on S."""
+    rng = np.random.default_rng(21)
+    for (N, D, H, W, C, O, k, s, pl, ph, dl, G) in _GEOMS_EX:
+        x = _t(rng.uniform(-1, 1, (N, D, H, W, C))).to(torch.float16)
+        w = _t(rng.standard_normal((O, *k, C // G))).to(torch.float16)
+        xp = torch.nn.functional.pad(x.double(), (0, 0, pl[2], ph[2], pl[1], ph[1], pl[0], ph[0]))
+        for flip in (False, True):
+            wr = w.double().flip(dims=(1, 2, 3)) if flip else w.double()
+            y, S = orc.conv_fwd(x, w, s, pl, dl, G, pad_hi=ph, flip=flip)
+            ref = _torch_conv_f64(xp, wr, s, (0, 0, 0), dl, G)
+            refS = _torch_conv_f64(xp.abs(), wr.abs(), s, (0, 0, 0), dl, G)
+            assert y.shape == ref.shape, (y.shape, ref.shape)
+            assert np.allclose(y, ref, rtol=1e-12, atol=1e-12), np.abs(y - ref).max()
+            assert np.allclose(S, refS, rtol=1e-12, atol=1e-12), np.abs(S - refS).max()
+
+
+def pin_side_padding_is_a_crop(orc):
+    """At stride 1, padding (p, q) below/above equals padding (p, p) with the last
+    p - q outputs of that dimension dropped (q <= p), or the first q - p of the
+    (q, q) result dropped (q >= p): the index origin moves only with the low side."""
+    rng = np.random.default_rng(22)
+    x = _t(_grid_values(rng, (1, 1, 8, 9, 3)))
+    w = _t(_grid_values(rng, (5, 1, 3, 3, 3)))
+    y_lo, _ = orc.conv_fwd(x, w, (1, 1, 1), (0, 2, 1), (1, 1, 1), 1, pad_hi=(0, 0, 1))
+    y_sym, _ = orc.conv_fwd(x, w, (1, 1, 1), (0, 2, 1), (1, 1, 1), 1)
+    assert np.array_equal(y_lo, y_sym[:, :, :-2, :, :])
+    y_hi, _ = orc.conv_fwd(x, w, (1, 1, 1), (0, 0, 1), (1, 1, 1), 1, pad_hi=(0, 2, 1))
+    y_sym2, _ = orc.conv_fwd(x, w, (1, 1, 1), (0, 2, 1), (1, 1, 1), 1)
+    assert np.array_equal(y_hi, y_sym2[:, :, 2:, :, :])
+    assert orc.out_dims(1, 8, 9, 1, 3, 3, (1, 1, 1), (0, 2, 1), (1, 1, 1), pad_hi=(0, 0, 1)) == (1, 8, 9)
+
+
 ALL_PINS = [pin_tutorial_example, pin_output_extent, pin_constant_input, pin_delta_kernel,
             pin_pointwise_is_matmul, pin_im2col_equivalence, pin_torch_witness, pin_linearity,
-            pin_translation, pin_groups_split, pin_points_match_full]
+            pin_translation, pin_groups_split, pin_points_match_full, pin_flip_tutorial_example,
+            pin_flip_and_side_padding_torch_witness, pin_side_padding_is_a_crop]

@@ -96,8 +96,10 @@ MUTATIONS = {
     "dilation_dropped": [(r"\(int64_t\)kw \* sh->d\[2\]", "(int64_t)kw")],
     "stride_wrong_dim": [(r"\(int64_t\)od \* sh->s\[0\]", "(int64_t)od * sh->s[1]")],
     "group_offset_dropped": [(r"\* sh->C \+ \(int64_t\)g \* Cg;", "* sh->C;")],
-    "weight_taps_transposed": [(r"\(\(\(\(int64_t\)o \* sh->kD \+ kd\) \* sh->kH \+ kh\) \* sh->kW \+ kw\)",
-                                "((((int64_t)o * sh->kD + kd) * sh->kW + kw) * sh->kH + kh)")],
+    "weight_taps_transposed": [(r"\(\(\(\(int64_t\)o \* sh->kD \+ fd\) \* sh->kH \+ fh\) \* sh->kW \+ fw\)",
+                                "((((int64_t)o * sh->kD + fd) * sh->kW + fw) * sh->kH + fh)")],
+    "flip_ignored_in_width": [(r"const int fw = sh->flip \? sh->kW - 1 - kw : kw;", "const int fw = kw;")],
+    "high_side_padding_ignored": [(r"in \+ \(int64_t\)p_lo \+ \(int64_t\)p_hi", "in + 2 * (int64_t)p_lo")],
     "magnitude_signed": [(r"mag \+= fabs\(t\);", "mag += t;")],
     "extent_off_by_one": [(r"\(int64_t\)d \* \(k - 1\) - 1;", "(int64_t)d * (k - 1);")],
     "f16_exponent_bias": [(r"e - 25\);", "e - 24);")],
