@@ -58,12 +58,18 @@ def lib() -> ctypes.CDLL:
         L.conv_fwd_host.argtypes = [vp] * 6 + geo + [vp]
         L.conv_plan.argtypes = geo + [i3, i3, i3]
         L.conv_plan_variant.argtypes = geo + [ci, i3, i3, i3]
+        # the general forms: per-side padding and flip (geo_ex: ..., stride, pad_lo, pad_hi, dil, groups, flip, dtype)
+        geo_ex = [ci] * 9 + [i3, i3, i3, i3, ci, ci, ci]
+        L.conv_out_dims_ex.argtypes = [ci] * 6 + [i3, i3, i3, i3, i3]
+        L.conv_fwd_ex.argtypes = [vp, vp, vp] + geo_ex + [ci, vp]
+        L.conv_plan_ex.argtypes = geo_ex + [ci, i3, i3, i3]
         L.conv_last_status.argtypes = [vp]
         L.conv_debug_inject_stall.argtypes = [ctypes.c_ulonglong]
         L.conv_strerror.argtypes = [ci]
         L.conv_strerror.restype = ctypes.c_char_p
         for f in ("conv_out_dims", "conv_fwd", "conv_fwd_variant", "conv_fwd_host", "conv_plan",
-                  "conv_plan_variant", "conv_last_status", "conv_version", "conv_debug_inject_stall"):
+                  "conv_plan_variant", "conv_last_status", "conv_version", "conv_debug_inject_stall",
+                  "conv_out_dims_ex", "conv_fwd_ex", "conv_plan_ex"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
@@ -96,10 +102,12 @@ def _dtype_code(t):
     return code
 
 
-def out_dims(D, H, W, kD, kH, kW, stride, pad, dil):
-    """(Do, Ho, Wo) as computed by the library (host only)."""
+def out_dims(D, H, W, kD, kH, kW, stride, pad, dil, pad_hi=None):
+    """(Do, Ho, Wo) as computed by the library (host only); `pad` pads below each
+    dimension, and above unless `pad_hi` is given."""
     out = (ctypes.c_int * 3)()
-    rc = lib().conv_out_dims(D, H, W, kD, kH, kW, _i3(stride), _i3(pad), _i3(dil), out)
+    rc = lib().conv_out_dims_ex(D, H, W, kD, kH, kW, _i3(stride), _i3(pad),
+                                _i3(pad if pad_hi is None else pad_hi), _i3(dil), out)
     if rc:
         raise ConvError(rc, "conv_out_dims")
     return tuple(out)
@@ -132,12 +140,15 @@ def _geometry(x, w, stride, padding, dilation):
     return two_d, (int(N), int(D), int(H), int(W), int(C), int(O), int(kD), int(kH), int(kW), int(Cg)), s, p, d
 
 
-def conv_fwd(x, w, stride=1, padding=0, dilation=1, groups=1, *, out=None, variant=VARIANT_AUTO, stream=None):
+def conv_fwd(x, w, stride=1, padding=0, dilation=1, groups=1, *, out=None, variant=VARIANT_AUTO, stream=None,
+             padding_hi=None, flip=False):
     """y = conv(x, w) on the current CUDA stream (or `stream`).  Returns y.
 
     x, w: contiguous CUDA tensors of one dtype (float16, bfloat16 or float32).
     `out` may supply a preallocated contiguous y.  `variant` forces a kernel
-    (VARIANT_*); the default lets the library choose.
+    (VARIANT_*); the default lets the library choose.  `padding` pads below
+    each spatial dimension and, unless `padding_hi` is given, above it too;
+    `flip` reads the filter reversed in every spatial dimension.
     """
     import torch
     if not (x.is_cuda and w.is_cuda):
@@ -147,7 +158,8 @@ def conv_fwd(x, w, stride=1, padding=0, dilation=1, groups=1, *, out=None, varia
     two_d, (N, D, H, W, C, O, kD, kH, kW, Cg), s, p, d = _geometry(x, w, stride, padding, dilation)
     if Cg * groups != C:
         raise ValueError(f"weight has {Cg} channels per group but C={C}, groups={groups}")
-    Do, Ho, Wo = out_dims(D, H, W, kD, kH, kW, s, p, d)
+    ph = p if padding_hi is None else _geometry(x, w, stride, padding_hi, dilation)[3]
+    Do, Ho, Wo = out_dims(D, H, W, kD, kH, kW, s, p, d, ph)
     shape = (N, Ho, Wo, O) if two_d else (N, Do, Ho, Wo, O)
     if out is None:
         out = torch.empty(shape, dtype=x.dtype, device=x.device)
@@ -157,19 +169,24 @@ def conv_fwd(x, w, stride=1, padding=0, dilation=1, groups=1, *, out=None, varia
     w = w.contiguous()
     st = stream if stream is not None else torch.cuda.current_stream(x.device)
     with torch.cuda.device(x.device):
-        rc = lib().conv_fwd_variant(x.data_ptr(), w.data_ptr(), out.data_ptr(), N, D, H, W, C, O, kD, kH, kW,
-                                    _i3(s), _i3(p), _i3(d), int(groups), _dtype_code(x), int(variant),
-                                    st.cuda_stream)
+        rc = lib().conv_fwd_ex(x.data_ptr(), w.data_ptr(), out.data_ptr(), N, D, H, W, C, O, kD, kH, kW,
+                               _i3(s), _i3(p), _i3(ph), _i3(d), int(groups), int(bool(flip)), _dtype_code(x),
+                               int(variant), st.cuda_stream)
     if rc:
         raise ConvError(rc, "conv_fwd")
     return out
 
 
-def conv_fwd_raw(x_ptr, w_ptr, y_ptr, geom, dtype, variant=VARIANT_AUTO, stream_handle=0):
-    """The C entry point on raw device pointers: geom = (N,D,H,W,C,O,kD,kH,kW,stride,pad,dil,groups)."""
+def conv_fwd_raw(x_ptr, w_ptr, y_ptr, geom, dtype, variant=VARIANT_AUTO, stream_handle=0, pad_hi=None, flip=0):
+    """The C entry point on raw device pointers: geom = (N,D,H,W,C,O,kD,kH,kW,stride,pad,dil,groups)
+    (conv_fwd_variant; conv_fwd_ex when `pad_hi` or `flip` is given)."""
     N, D, H, W, C, O, kD, kH, kW, s, p, d, g = geom
-    return lib().conv_fwd_variant(x_ptr, w_ptr, y_ptr, N, D, H, W, C, O, kD, kH, kW, _i3(s), _i3(p), _i3(d),
-                                  int(g), int(dtype), int(variant), stream_handle)
+    if pad_hi is None and not flip:
+        return lib().conv_fwd_variant(x_ptr, w_ptr, y_ptr, N, D, H, W, C, O, kD, kH, kW, _i3(s), _i3(p), _i3(d),
+                                      int(g), int(dtype), int(variant), stream_handle)
+    return lib().conv_fwd_ex(x_ptr, w_ptr, y_ptr, N, D, H, W, C, O, kD, kH, kW, _i3(s), _i3(p),
+                             _i3(p if pad_hi is None else pad_hi), _i3(d), int(g), int(flip), int(dtype),
+                             int(variant), stream_handle)
 
 
 def conv_fwd_host(x_host, w_host, y_host, x_dev, w_dev, y_dev, stride=1, padding=0, dilation=1, groups=1,
@@ -191,13 +208,13 @@ def conv_fwd_host(x_host, w_host, y_host, x_dev, w_dev, y_dev, stride=1, padding
     return y_host
 
 
-def plan(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype, variant=VARIANT_AUTO):
+def plan(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype, variant=VARIANT_AUTO, pad_hi=None, flip=0):
     """(variant, BN, stages, ctas) the library would use; dtype is 'f32' | 'f16' | 'bf16'.
     With an explicit `variant`, the plan of that variant (ConvError if it cannot run)."""
     code = {"f32": CONV_F32, "f16": CONV_F16, "bf16": CONV_BF16}[dtype]
     bn, st, ct = (ctypes.c_int * 1)(), (ctypes.c_int * 1)(), (ctypes.c_int * 1)()
-    v = lib().conv_plan_variant(N, D, H, W, C, O, *k, _i3(stride), _i3(pad), _i3(dil), int(groups), code,
-                                int(variant), bn, st, ct)
+    v = lib().conv_plan_ex(N, D, H, W, C, O, *k, _i3(stride), _i3(pad), _i3(pad if pad_hi is None else pad_hi),
+                           _i3(dil), int(groups), int(flip), code, int(variant), bn, st, ct)
     if v < 0:
         raise ConvError(v, "conv_plan_variant")
     return v, bn[0], st[0], ct[0]

@@ -30,7 +30,9 @@ constexpr long long kMaxResidentB = 96 * 1024;              // weights kept in s
 
 struct Problem {
   int N, D, H, W, C, O, kD, kH, kW;
-  int s[3], p[3], d[3];
+  int s[3], p[3], d[3];  // p: padding below each dimension (the index origin is -p)
+  int p_hi[3];           // padding above each dimension (sets the output extent with p)
+  int flip;              // 1: the filter is read reversed in every spatial dimension
   int G, Cg, Og;
   int Do, Ho, Wo;
   long long M;
@@ -40,20 +42,21 @@ struct Problem {
   size_t x_bytes, w_bytes, y_bytes;
 };
 
-long long extent(long long in, int k, int s, int p, int d) {
-  const long long num = in + 2LL * p - static_cast<long long>(d) * (k - 1) - 1;
+long long extent(long long in, int k, int s, int p_lo, int p_hi, int d) {
+  const long long num = in + static_cast<long long>(p_lo) + p_hi - static_cast<long long>(d) * (k - 1) - 1;
   if (num < 0) return 0;
   return num / s + 1;
 }
 
-int out_dims_impl(int D, int H, int W, int kD, int kH, int kW, const int stride[3], const int pad[3],
-                  const int dil[3], int out[3]) {
-  if (!stride || !pad || !dil || !out) return CONV_EINVAL;
+int out_dims_impl(int D, int H, int W, int kD, int kH, int kW, const int stride[3], const int pad_lo[3],
+                  const int pad_hi[3], const int dil[3], int out[3]) {
+  if (!stride || !pad_lo || !pad_hi || !dil || !out) return CONV_EINVAL;
   const int in[3] = {D, H, W};
   const int k[3] = {kD, kH, kW};
   for (int i = 0; i < 3; ++i) {
-    if (in[i] <= 0 || k[i] <= 0 || stride[i] <= 0 || dil[i] <= 0 || pad[i] < 0) return CONV_EINVAL;
-    const long long e = extent(in[i], k[i], stride[i], pad[i], dil[i]);
+    if (in[i] <= 0 || k[i] <= 0 || stride[i] <= 0 || dil[i] <= 0 || pad_lo[i] < 0 || pad_hi[i] < 0)
+      return CONV_EINVAL;
+    const long long e = extent(in[i], k[i], stride[i], pad_lo[i], pad_hi[i], dil[i]);
     if (e <= 0 || e > 0x7fffffffLL) return CONV_EINVAL;
     out[i] = static_cast<int>(e);
   }
@@ -68,15 +71,20 @@ bool mul_ok(long long a, long long b, long long& r) {
 }
 
 int make_problem(Problem& P, int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
-                 const int stride[3], const int pad[3], const int dil[3], int groups, int dtype) {
+                 const int stride[3], const int pad_lo[3], const int pad_hi[3], const int dil[3], int groups,
+                 int flip, int dtype) {
   if (dtype != CONV_F32 && dtype != CONV_F16 && dtype != CONV_BF16) return CONV_EDTYPE;
   if (N <= 0 || C <= 0 || O <= 0 || groups <= 0) return CONV_EINVAL;
   if (C % groups != 0 || O % groups != 0) return CONV_EINVAL;
+  if (flip != 0 && flip != 1) return CONV_EINVAL;
   int out[3];
-  const int rc = out_dims_impl(D, H, W, kD, kH, kW, stride, pad, dil, out);
+  const int rc = out_dims_impl(D, H, W, kD, kH, kW, stride, pad_lo, pad_hi, dil, out);
   if (rc != CONV_OK) return rc;
   P.N = N; P.D = D; P.H = H; P.W = W; P.C = C; P.O = O; P.kD = kD; P.kH = kH; P.kW = kW;
-  for (int i = 0; i < 3; ++i) { P.s[i] = stride[i]; P.p[i] = pad[i]; P.d[i] = dil[i]; }
+  for (int i = 0; i < 3; ++i) {
+    P.s[i] = stride[i]; P.p[i] = pad_lo[i]; P.p_hi[i] = pad_hi[i]; P.d[i] = dil[i];
+  }
+  P.flip = flip;
   P.G = groups; P.Cg = C / groups; P.Og = O / groups;
   P.Do = out[0]; P.Ho = out[1]; P.Wo = out[2];
   P.dtype = dtype;
@@ -252,16 +260,20 @@ uint32_t next_pow2_cols(uint32_t v) {
 // tensor rank (rank 4: [-128, 127]; rank 5: [-16, 15]); traversal strides
 // are at most 8; the pixel rows must be 16-byte strided (C % 8 == 0) and the
 // channel chunk a multiple of 16 elements for the MMA K step.
+// A 2-D problem: one input plane, one filter plane, and no depth padding on
+// either side (the depth extent is then 1).
+bool is_2d(const Problem& P) { return P.D == 1 && P.kD == 1 && P.p[0] == 0 && P.p_hi[0] == 0; }
+
 bool tma_fits(const Problem& P, bool& rank5) {
   if (P.dtype == CONV_F32) return false;
   if (P.Cg % 16 != 0) return false;
-  rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
+  rank5 = !is_2d(P);
   const int lo = rank5 ? -16 : -128, hi = rank5 ? 15 : 127;
   const int ks[3] = {P.kD, P.kH, P.kW};
   for (int i = rank5 ? 0 : 1; i < 3; ++i) {
     if (P.s[i] > 8) return false;
     const int lower = -P.p[i];
-    const long long upper = static_cast<long long>(P.p[i]) - static_cast<long long>(P.d[i]) * (ks[i] - 1);
+    const long long upper = static_cast<long long>(P.p_hi[i]) - static_cast<long long>(P.d[i]) * (ks[i] - 1);
     const long long off = static_cast<long long>(P.d[i]) * (ks[i] - 1);
     if (lower < lo || lower > hi || upper < lo || upper > hi || off > hi) return false;
   }
@@ -277,7 +289,7 @@ constexpr int kHaloTileH = 16, kHaloTileW = 8;
 bool halo_fits(const Problem& P, bool& rank5) {
   if (P.dtype == CONV_F32 || P.Cg % 32 != 0) return false;
   if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1) return false;
-  rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
+  rank5 = !is_2d(P);
   const long long hh = kHaloTileH + static_cast<long long>(P.d[1]) * (P.kH - 1);
   if (hh > 256) return false;
   if (P.N > 0x3fffffff) return false;
@@ -418,7 +430,7 @@ int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
   if (P.dtype == CONV_F32 || P.Cg % 32 != 0 || P.Og % o_tile != 0) return CONV_EUNSUPPORTED;
   if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1) return CONV_EUNSUPPORTED;
   if (P.N > 0x3fffffff) return CONV_EUNSUPPORTED;
-  const bool rank5 = !(P.D == 1 && P.kD == 1 && P.p[0] == 0);
+  const bool rank5 = !is_2d(P);
   // block height: the multiple of 4 up to 32 that wastes the fewest rows of
   // Ho (ties to the taller block, which reuses the strip over more rows)
   int bh = kHTBlockHMax;
@@ -526,7 +538,8 @@ int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
 // row; N = P*O <= 256; CTA pairs, each CTA ph_rows output rows of a tile.
 int plan_phase(const Problem& P, int sms, TcPlan& plan) {
   if (P.dtype == CONV_F32 || P.G != 1) return CONV_EUNSUPPORTED;
-  if (P.D != 1 || P.kD != 1 || P.p[0] != 0) return CONV_EUNSUPPORTED;  // 2-D
+  if (!is_2d(P)) return CONV_EUNSUPPORTED;
+  if (P.flip) return CONV_EUNSUPPORTED;  // B's phase rows assume the filter's own tap order
   if (P.d[2] != 1) return CONV_EUNSUPPORTED;  // a filter row's taps are contiguous
   const int sh = P.s[1], sw = P.s[2];
   if (P.H % sh != 0) return CONV_EUNSUPPORTED;  // input rows as (ih / sh, ih % sh)
@@ -654,7 +667,7 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
     // layout where each filter row (kd, kh) is padded to Lp = roundup(kW*C, 8)
     if (P.Cg % 8 == 0) {
       a.gather_mode = GATHER_VEC8;
-    } else if (P.G == 1 && P.d[2] == 1) {
+    } else if (P.G == 1 && P.d[2] == 1 && !P.flip) {  // (span layout: the filter's own tap order)
       a.gather_mode = GATHER_SPAN;
     } else {
       a.gather_mode = GATHER_SCALAR;
@@ -663,7 +676,7 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
     // Row staging: 2-D problems in span layout whose input rows are 16-byte
     // strided and whose 128-pixel tiles touch at most two images get their
     // input rows by TMA instead of per-thread loads.
-    if (a.gather_mode == GATHER_SPAN && P.D == 1 && P.kD == 1 && P.p[0] == 0 &&
+    if (a.gather_mode == GATHER_SPAN && is_2d(P) &&
         (static_cast<long long>(P.W) * P.C) % 8 == 0 && static_cast<long long>(P.Ho) * P.Wo >= kBM) {
       // a row of row_e = W*C elements is one box row of n_boxes x box_e, with
       // box_e the largest multiple-of-8 divisor of row_e that is <= 256
@@ -847,13 +860,13 @@ int encode_maps(const Problem& P, const TcArgs& a, bool pair, bool halo, const v
   gstr[1] = gstr[0] * P.W;
   gstr[2] = gstr[1] * P.H;
   estr[0] = 1; estr[1] = P.s[2]; estr[2] = P.s[1];
-  lower[0] = -P.p[2]; upper[0] = P.p[2] - P.d[2] * (P.kW - 1);
-  lower[1] = -P.p[1]; upper[1] = P.p[1] - P.d[1] * (P.kH - 1);
+  lower[0] = -P.p[2]; upper[0] = P.p_hi[2] - P.d[2] * (P.kW - 1);
+  lower[1] = -P.p[1]; upper[1] = P.p_hi[1] - P.d[1] * (P.kH - 1);
   if (rank == 5) {
     gdim[3] = P.D; gdim[4] = P.N;
     gstr[3] = gstr[2] * P.D;
     estr[3] = P.s[0]; estr[4] = 1;
-    lower[2] = -P.p[0]; upper[2] = P.p[0] - P.d[0] * (P.kD - 1);
+    lower[2] = -P.p[0]; upper[2] = P.p_hi[0] - P.d[0] * (P.kD - 1);
   } else {
     gdim[3] = P.N;
     estr[3] = 1;
@@ -952,6 +965,8 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
   if (rc != CONV_OK) return rc;
   TcArgs a = plan.args;
   a.x = x; a.w = w; a.y = y;
+  a.flip = P.flip;
+  a.taps = P.kD * P.kH * P.kW;
   const unsigned long long stall_ns = g_inject_stall_ns.exchange(0);
   if (stall_ns != 0) {
     a.inject_stall = 1;
@@ -1132,6 +1147,8 @@ int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStr
   a.G = P.G; a.Cg = P.Cg; a.Og = P.Og;
   a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
   a.M = P.M; a.K = static_cast<int>(P.K);
+  a.flip = P.flip;
+  a.taps = P.kD * P.kH * P.kW;
   a.x = x; a.w = w; a.y = y;
   const SimtShape sh = simt_shape(P, sms);
   const long long mt = (P.M + 16 * sh.tm - 1) / (16 * sh.tm);
@@ -1173,21 +1190,33 @@ using namespace convfwd;
 
 extern "C" {
 
-int conv_out_dims(int D, int H, int W, int kD, int kH, int kW, const int stride[3], const int pad[3],
-                  const int dil[3], int out[3]) {
-  return out_dims_impl(D, H, W, kD, kH, kW, stride, pad, dil, out);
+int conv_out_dims_ex(int D, int H, int W, int kD, int kH, int kW, const int stride[3], const int pad_lo[3],
+                     const int pad_hi[3], const int dil[3], int out[3]) {
+  return out_dims_impl(D, H, W, kD, kH, kW, stride, pad_lo, pad_hi, dil, out);
 }
 
-int conv_fwd_variant(const void* x, const void* w, void* y, int N, int D, int H, int W, int C, int O, int kD,
-                     int kH, int kW, const int stride[3], const int pad[3], const int dil[3], int groups,
-                     int dtype, int variant, conv_stream_t stream) {
+int conv_out_dims(int D, int H, int W, int kD, int kH, int kW, const int stride[3], const int pad[3],
+                  const int dil[3], int out[3]) {
+  return out_dims_impl(D, H, W, kD, kH, kW, stride, pad, pad, dil, out);
+}
+
+int conv_fwd_ex(const void* x, const void* w, void* y, int N, int D, int H, int W, int C, int O, int kD, int kH,
+                int kW, const int stride[3], const int pad_lo[3], const int pad_hi[3], const int dil[3], int groups,
+                int flip, int dtype, int variant, conv_stream_t stream) {
   Problem P;
-  int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
+  int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, flip, dtype);
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
   if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_PHASE) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int conv_fwd_variant(const void* x, const void* w, void* y, int N, int D, int H, int W, int C, int O, int kD,
+                     int kH, int kW, const int stride[3], const int pad[3], const int dil[3], int groups,
+                     int dtype, int variant, conv_stream_t stream) {
+  return conv_fwd_ex(x, w, y, N, D, H, W, C, O, kD, kH, kW, stride, pad, pad, dil, groups, 0, dtype, variant,
+                     stream);
 }
 
 int conv_fwd(const void* x, const void* w, void* y, int N, int D, int H, int W, int C, int O, int kD, int kH,
@@ -1201,7 +1230,7 @@ int conv_fwd_host(const void* x_host, const void* w_host, void* y_host, void* x_
                   int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
                   const int pad[3], const int dil[3], int groups, int dtype, conv_stream_t stream) {
   Problem P;
-  int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
+  int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, pad, dil, groups, 0, dtype);
   if (rc != CONV_OK) return rc;
   if (!x_host || !w_host || !y_host) return CONV_EINVAL;
   rc = check_pointers(P, x_dev, w_dev, y_dev);
@@ -1217,11 +1246,11 @@ int conv_fwd_host(const void* x_host, const void* w_host, void* y_host, void* x_
   return CONV_OK;
 }
 
-int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
-                      const int pad[3], const int dil[3], int groups, int dtype, int variant, int* bn,
-                      int* stages, int* ctas) {
+int conv_plan_ex(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
+                 const int pad_lo[3], const int pad_hi[3], const int dil[3], int groups, int flip, int dtype,
+                 int variant, int* bn, int* stages, int* ctas) {
   Problem P;
-  int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad, dil, groups, dtype);
+  int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, flip, dtype);
   if (rc != CONV_OK) return rc;
   if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_PHASE) return CONV_EINVAL;
   int dev, sms = 148;
@@ -1245,6 +1274,13 @@ int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, 
   if (stages) *stages = plan.args.stages;
   if (ctas) *ctas = plan.ctas;
   return variant;
+}
+
+int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
+                      const int pad[3], const int dil[3], int groups, int dtype, int variant, int* bn,
+                      int* stages, int* ctas) {
+  return conv_plan_ex(N, D, H, W, C, O, kD, kH, kW, stride, pad, pad, dil, groups, 0, dtype, variant, bn, stages,
+                      ctas);
 }
 
 int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],

@@ -136,8 +136,8 @@ __global__ void __launch_bounds__(192, 1)
           for (int j = 0; j < nsub; ++j) {
             const uint32_t sb = ptx::smem_u32(bring + bst * a.stage_bytes + j * a.b_bytes);
             const int tap = (kd * a.kH + kh) * a.kW + kw;  // weight layout (kd, kh, kw)
-            if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, tap * a.Cg + cc * a.kc, brow);
-            else ptx::tma_load_2d(sb, &tmap_w, fb, tap * a.Cg + cc * a.kc, brow);
+            if constexpr (PAIR) ptx::tma_load_2d_pair(sb, &tmap_w, fb_l, wtap(a, tap) * a.Cg + cc * a.kc, brow);
+            else ptx::tma_load_2d(sb, &tmap_w, fb, wtap(a, tap) * a.Cg + cc * a.kc, brow);
             if (++kh == a.kH) {
               kh = 0;
               if (++kw == a.kW) {

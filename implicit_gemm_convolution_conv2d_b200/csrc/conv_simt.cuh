@@ -26,6 +26,8 @@ struct SimtArgs {
   int Do, Ho, Wo;
   long long M;
   int K;
+  int flip;   // 1: the filter is read reversed in every spatial dimension
+  int taps;   // kD*kH*kW
   const void* x;
   const void* w;
   void* y;
@@ -124,8 +126,10 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
         v = to_f32<T>(x[rbase[i] + ((static_cast<long long>(zd) * a.H + zh) * a.W + zw) * a.C + c]);
       ra[i] = v;
     }
+    // the weight element: k itself, or with flip the mirrored tap's channel c
+    const int wk = a.flip ? (a.taps - 1 - ((kd * a.kH + kh) * a.kW + kw)) * a.Cg + c : k;
 #pragma unroll
-    for (int j = 0; j < TN; ++j) rb[j] = (ovalid[j] && kv) ? to_f32<T>(wrow[j][k]) : 0.f;
+    for (int j = 0; j < TN; ++j) rb[j] = (ovalid[j] && kv) ? to_f32<T>(wrow[j][wk]) : 0.f;
     // advance the carried decode by one K step
     c += kSimtBK;
     while (c >= a.Cg) {

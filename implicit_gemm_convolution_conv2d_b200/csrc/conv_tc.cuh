@@ -97,6 +97,8 @@ struct TcArgs {
   int mo;             // transposed halo kernel: output channels per tile (MMA M: 64 or 128)
   int b_resident;     // gather: the whole B matrix stays in shared memory
   uint32_t bres_bytes;  // its size (kblocks * BN * 128), 0 when not resident
+  int flip;           // 1: the filter is read reversed in every spatial dimension
+  int taps;           // kD*kH*kW
   int w_resident;     // transposed halo kernel: all weight tiles loaded once into stage 0
   int epi_bufs;       // transposed halo kernel: epilogue staging tiles (1 or 2)
   // phase-packed kernel (few input channels): one GEMM row = P output pixels of a row
@@ -285,6 +287,11 @@ __device__ __forceinline__ void mma_ksteps(uint32_t d_tmem, uint64_t da, uint64_
     else ptx::mma_f16(d_tmem, da + 2 * k, db + 2 * k, idesc, k == 0 ? acc0 : 1u);
   }
 }
+
+// Filter tap (kd*kH + kh)*kW + kw of the weights that input tap `tap` multiplies:
+// itself, or with flip the tap mirrored in every spatial dimension, which in
+// this numbering is taps - 1 - tap.
+__device__ __forceinline__ int wtap(const TcArgs& a, int tap) { return a.flip ? a.taps - 1 - tap : tap; }
 
 // The same for a run-time step count of 1 to 4 (channel chunks of 64, 32 or
 // 16 elements; 3 for a 48-element phase-packed window).
@@ -635,10 +642,20 @@ __device__ __forceinline__ void gather_b_block(const TcArgs& a, int g, int n0, i
     uint4 v = make_uint4(0, 0, 0, 0);
     if (oc < a.Og && kp0 < a.Kp) {
       const long long rowoff = static_cast<long long>(g * a.Og + oc) * a.K;
-      if (span_layout) {
+      if (span_layout) {  // (never with flip: the planner uses the other layouts)
         const int sp = kp0 / a.Lp;
         const int j0 = kp0 - sp * a.Lp;
         v = load8_masked(w + rowoff + static_cast<long long>(sp) * L + j0, 0, L - j0);
+      } else if (a.flip) {
+        // K element k = tap*Cg + c multiplies w[o, taps-1-tap, c]
+        uint16_t e8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int k = kp0 + e;
+          const int tap = k / a.Cg;
+          e8[e] = k < a.K ? w[rowoff + static_cast<long long>(wtap(a, tap)) * a.Cg + (k - tap * a.Cg)] : uint16_t(0);
+        }
+        v = *reinterpret_cast<const uint4*>(e8);
       } else if (vec) {
         v = __ldg(reinterpret_cast<const uint4*>(w + rowoff + kp0));
       } else {
@@ -786,7 +803,7 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
                                         static_cast<uint16_t>(kw * a.dw),
                                         static_cast<uint16_t>(kh * a.dh));
               }
-              ptx::tma_load_2d(sb, &tmap_w, fb, tap * a.Cg + cchunk * a.kc, orow);
+              ptx::tma_load_2d(sb, &tmap_w, fb, wtap(a, tap) * a.Cg + cchunk * a.kc, orow);
               if (++cchunk == a.cchunks) {
                 cchunk = 0;
                 ++tap;
@@ -1119,7 +1136,7 @@ __global__ void __launch_bounds__(192, 1)
             else
               ptx::tma_load_im2col_4d_pair(sa, &tmap_x, fb, c0, cw, chh, n, static_cast<uint16_t>(kw * a.dw),
                                            static_cast<uint16_t>(kh * a.dh));
-            ptx::tma_load_2d_pair(sb, &tmap_w, fb, tap * a.Cg + cchunk * a.kc, brow);
+            ptx::tma_load_2d_pair(sb, &tmap_w, fb, wtap(a, tap) * a.Cg + cchunk * a.kc, brow);
             if (++cchunk == a.cchunks) {
               cchunk = 0;
               ++tap;

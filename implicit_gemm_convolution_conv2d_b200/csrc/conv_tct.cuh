@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kTTileThreads, 1)
             const int kh = (tap / a.kW) % a.kH;
             const int kd = tap / (a.kW * a.kH);
             const int c0 = tc.g * a.Cg + cchunk * a.kc;
-            ptx::tma_load_2d(sa, &tmap_w, fb, tap * a.Cg + cchunk * a.kc, orow);
+            ptx::tma_load_2d(sa, &tmap_w, fb, wtap(a, tap) * a.Cg + cchunk * a.kc, orow);
             for (int h = 0; h < halves; ++h) {
               const uint32_t dst = sb + static_cast<uint32_t>(h) * half_bytes;
               if (a.rank5)

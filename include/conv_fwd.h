@@ -120,6 +120,24 @@ int conv_fwd(const void* x, const void* w, void* y,
              const int stride[3], const int pad[3], const int dil[3],
              int groups, int dtype, conv_stream_t stream);
 
+/* The general form: padding pad_lo[i] below and pad_hi[i] above spatial
+ * dimension i (the index origin is -pad_lo; the extent is
+ * floor((I + pad_lo + pad_hi - dil*(k-1) - 1) / s) + 1), and flip = 1 to read
+ * the filter reversed in every spatial dimension, w[o, kD-1-kd, kH-1-kh,
+ * kW-1-kw, c] (a true convolution; 0 is the cross-correlation above).  The
+ * flip is the MLX pull request's "correct flip" of its input loader ("What
+ * changed"); per-side padding generalises the symmetric padding.  variant is
+ * CONV_VARIANT_AUTO or an explicit CONV_VARIANT_*; with flip the phase-packed
+ * kernel and the gather kernel's filter-row layouts are not used (AUTO picks
+ * another).  Returns as conv_fwd / conv_fwd_variant; CONV_EINVAL also for a
+ * negative pad or a flip other than 0 or 1. */
+int conv_fwd_ex(const void* x, const void* w, void* y,
+                int N, int D, int H, int W, int C, int O,
+                int kD, int kH, int kW,
+                const int stride[3], const int pad_lo[3], const int pad_hi[3],
+                const int dil[3], int groups, int flip, int dtype, int variant,
+                conv_stream_t stream);
+
 /* conv_fwd with an explicit kernel variant (CONV_VARIANT_*).  Returns
  * CONV_EUNSUPPORTED when that variant cannot run the shape or type
  * (the tensor-core variants need f16/bf16; TC_TMA, TC_TMA_PAIR and TC_TMA_T
@@ -145,6 +163,18 @@ int conv_fwd_host(const void* x_host, const void* w_host, void* y_host,
                   int kD, int kH, int kW,
                   const int stride[3], const int pad[3], const int dil[3],
                   int groups, int dtype, conv_stream_t stream);
+
+/* Output extents with per-side padding (see conv_fwd_ex). */
+int conv_out_dims_ex(int D, int H, int W, int kD, int kH, int kW,
+                     const int stride[3], const int pad_lo[3], const int pad_hi[3],
+                     const int dil[3], int out[3]);
+
+/* conv_plan_variant for the general form of conv_fwd_ex (per-side padding,
+ * flip).  Queues nothing. */
+int conv_plan_ex(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
+                 const int stride[3], const int pad_lo[3], const int pad_hi[3],
+                 const int dil[3], int groups, int flip, int dtype, int variant,
+                 int* bn, int* stages, int* ctas);
 
 /* The variant conv_fwd would run for this shape and type (CONV_VARIANT_*), or
  * a negative error code.  Also reports the output-tile width BN, the number of

@@ -33,7 +33,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("conv_fwd", "conv_fwd_variant", "conv_fwd_host", "conv_out_dims", "conv_plan",
-              "conv_last_status", "conv_strerror", "conv_version"):
+              "conv_last_status", "conv_strerror", "conv_version", "conv_fwd_ex", "conv_out_dims_ex",
+              "conv_plan_ex"):
         assert n in names, n
 
 
@@ -62,6 +63,48 @@ def test_out_dims_match_oracle(C):
             continue
         assert C.out_dims(*dims, *k, s, p, d) == ref
         n += 1
+
+
+def test_side_padding_out_dims_match_oracle(C):
+    rng = np.random.default_rng(1)
+    n = 0
+    while n < 300:
+        dims = rng.integers(1, 30, 3)
+        k = rng.integers(1, 6, 3)
+        s = rng.integers(1, 4, 3)
+        pl = rng.integers(0, 4, 3)
+        ph = rng.integers(0, 4, 3)
+        d = rng.integers(1, 3, 3)
+        try:
+            ref = oracle.out_dims(*dims, *k, s, pl, d, pad_hi=ph)
+        except ValueError:
+            with pytest.raises(C.ConvError):
+                C.out_dims(*dims, *k, s, pl, d, ph)
+            continue
+        assert C.out_dims(*dims, *k, s, pl, d, ph) == ref
+        n += 1
+
+
+def test_flip_and_side_padding_arguments(C):
+    L = C.lib()
+    i3 = lambda *v: (ctypes.c_int * 3)(*v)
+    s, p, d = i3(1, 1, 1), i3(0, 1, 1), i3(1, 1, 1)
+    X, Wt, Y = 0x10000, 0x20000, 0x40000       # never dereferenced: checks come first
+    ex = lambda ph, flip, dt=1, v=-1: L.conv_fwd_ex(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, ph, d, 1, flip,
+                                                    dt, v, None)
+    assert ex(i3(0, -1, 0), 0) == -1           # negative high-side pad
+    assert ex(i3(0, 1, 1), 2) == -1            # flip is 0 or 1
+    assert ex(i3(0, 1, 1), 0, 9) == -2         # dtype
+    assert ex(i3(0, 1, 1), 0, 1, 10) == -1     # unknown variant
+    # the phase-packed kernel does not take flip; the automatic choice then avoids it
+    stem = (2, 1, 32, 32, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
+    assert C.plan(*stem)[0] == C.VARIANT_TC_PHASE
+    assert C.plan(*stem, flip=1)[0] == C.VARIANT_TC_GATHER
+    with pytest.raises(C.ConvError) as e:
+        C.plan(*stem, C.VARIANT_TC_PHASE, flip=1)
+    assert e.value.code == -7
+    # depth padding on one side makes a 2-D-looking problem 3-D (Do = 2)
+    assert C.out_dims(1, 8, 8, 1, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1), (1, 1, 1)) == (2, 8, 8)
 
 
 def test_out_dims_pinned_values(C):

@@ -170,6 +170,68 @@ def test_small_sweep(wl, dtype):
         assert_parity(y, y_ref, s_ref, dtype, f"{wl.name}/{dtype}/{C.VARIANT_NAMES[v]}")
 
 
+# Per-side padding and flip (conv_fwd_ex): every kernel that can run the shape,
+# against the oracle with the same options.
+FLIP_PAD = [
+    # (case, pad_hi)
+    (WL.case(2, 1, 13, 11, 64, 128, (1, 3, 3), pad=(0, 1, 0), name="fp_2d_c64_o128"), (0, 0, 2)),
+    (WL.case(1, 5, 7, 9, 32, 64, (3, 3, 3), pad=(1, 0, 1), name="fp_3d_c32_o64"), (0, 1, 2)),
+    (WL.case(1, 1, 9, 10, 64, 256, (1, 3, 3), pad=(0, 2, 1), dil=(1, 2, 1), name="fp_2d_o256_dil"), (0, 0, 1)),
+    (WL.case(2, 1, 32, 32, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 2), name="fp_stem_like"), (0, 1, 3)),
+    (WL.case(2, 4, 6, 7, 21, 21, (3, 3, 3), pad=(1, 1, 0), name="fp_3d_c21"), (2, 0, 1)),
+    (WL.case(2, 1, 9, 11, 5, 8, (1, 3, 3), (1, 2, 1), (0, 1, 2), dil=(1, 1, 2), name="fp_c5_s2_dil"), (0, 2, 0)),
+    (WL.case(1, 6, 7, 8, 64, 128, (3, 1, 1), pad=(2, 0, 0), name="fp_k311"), (0, 0, 0)),
+]
+
+ALL_VARIANTS = ["SIMT", "TC_TMA", "TC_GATHER", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T", "TC_HALO_T",
+                "TC_HALO_T_PAIR", "TC_PHASE"]
+
+
+def run_gpu_ex(x, w, wl, pad_hi, flip, variant, guard=64):
+    xd, wd = x.cuda(), w.cuda()
+    Do, Ho, Wo = C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil, pad_hi)
+    n = wl.N * Do * Ho * Wo * wl.O
+    es = x.element_size()
+    buf = torch.full((n + 2 * guard,), 0x5A5A if es == 2 else 0x5A5A5A5A,
+                     dtype=torch.int16 if es == 2 else torch.int32, device="cuda")
+    y = buf[guard:guard + n].view(x.dtype).view(wl.N, Do, Ho, Wo, wl.O)
+    rc = C.conv_fwd_raw(xd.data_ptr(), wd.data_ptr(), y.data_ptr(),
+                        (wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, *wl.k, wl.stride, wl.pad, wl.dil, wl.groups),
+                        {"f32": 0, "f16": 1, "bf16": 2}[wl.dtype], variant,
+                        torch.cuda.current_stream().cuda_stream, pad_hi=pad_hi, flip=int(flip))
+    assert rc == 0, C.strerror(rc)
+    torch.cuda.synchronize()
+    assert C.last_status() == 0, "device status word set (pipeline timeout)"
+    g = buf.cpu()
+    pat = 0x5A5A if es == 2 else 0x5A5A5A5A
+    assert torch.all(g[:guard] == pat) and torch.all(g[guard + n:] == pat), "write outside y"
+    return y.cpu()
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("case", FLIP_PAD, ids=lambda c: c[0].name)
+def test_flip_and_side_padding(case, dtype):
+    wl, pad_hi = case
+    wl = wl.with_(dtype=dtype, seed=zlib.crc32(wl.name.encode()) % 1000)
+    x, w = WL.make_inputs(wl)
+    for flip in (0, 1):
+        y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups, pad_hi=pad_hi, flip=bool(flip))
+        ran = 0
+        for name in (["SIMT"] if dtype == "f32" else ALL_VARIANTS):
+            v = getattr(C, "VARIANT_" + name)
+            try:
+                C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil, wl.groups, dtype, v,
+                       pad_hi=pad_hi, flip=flip)
+            except C.ConvError:
+                continue
+            y = run_gpu_ex(x, w, wl, pad_hi, flip, v)
+            assert_parity(y, y_ref, s_ref, dtype, f"{wl.name}/{dtype}/flip={flip}/{C.VARIANT_NAMES[v]}")
+            ran += 1
+        y = run_gpu_ex(x, w, wl, pad_hi, flip, C.VARIANT_AUTO)
+        assert_parity(y, y_ref, s_ref, dtype, f"{wl.name}/{dtype}/flip={flip}/auto")
+        assert ran >= 1
+
+
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_transposed_wide_pixel_tiles(dtype):
     """Enough output pixels for 256-pixel tiles on every SM (the 128-pixel
