@@ -49,9 +49,9 @@ PROFILE_DIR = os.path.join(ROOT, "profiles")
 
 # ---------------------------------------------------------------- counting
 
-def out_dims(wl):
+def out_dims(wl, pad_hi=None):
     import implicit_gemm_convolution_conv2d_b200 as C
-    return C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil)
+    return C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil, pad_hi)
 
 
 def conv_flops(wl, dims=None):
@@ -265,11 +265,15 @@ def bench_ours(args):
     dist = init_dist(ws, "nccl")
 
     wl = WL.WORKLOADS[args.workload]
-    dims = out_dims(wl)
+    # --pad-hi / --flip: the general form of the operation (per-side padding, true convolution)
+    pad_hi = tuple(int(v) for v in args.pad_hi.split(",")) if args.pad_hi else None
+    flip = 1 if args.flip else 0
+    dims = out_dims(wl, pad_hi)
     flops = conv_flops(wl, dims)
     xb, wb, yb = conv_bytes(wl, dims)
     variant, bn, stages, ctas = C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil,
-                                       wl.groups, wl.dtype, getattr(C, "VARIANT_" + args.variant))
+                                       wl.groups, wl.dtype, getattr(C, "VARIANT_" + args.variant), pad_hi=pad_hi,
+                                       flip=flip)
     vname = C.VARIANT_NAMES[variant]
 
     # inputs: seeded on the host (rank-dependent seed), copied once
@@ -291,7 +295,7 @@ def bench_ours(args):
         s = i % nsets
         # the launch goes to the current stream (the capture stream while a graph is recorded)
         rc = C.conv_fwd_raw(xs[s].data_ptr(), wts[s].data_ptr(), ys[s].data_ptr(), geo(s), dcode,
-                            variant, torch.cuda.current_stream(dev).cuda_stream)
+                            variant, torch.cuda.current_stream(dev).cuda_stream, pad_hi=pad_hi, flip=flip)
         if rc:
             raise C.ConvError(rc, "conv_fwd")
         launches += 1
@@ -377,7 +381,9 @@ def bench_ours(args):
 
     # ---- end to end through the host-buffer C entry point (pinned host memory)
     e2e = None
-    if not args.no_e2e:
+    if pad_hi is not None or flip:
+        e2e = {"skipped": "the host-buffer entry point takes symmetric padding and no flip"}
+    elif not args.no_e2e:
         xp = x_h.pin_memory()
         wp = w_h.pin_memory()
         yp = torch.empty(ys[0].shape, dtype=x_h.dtype).pin_memory()
@@ -451,7 +457,12 @@ def bench_ours(args):
         "gpu_launches": timed_launches,
         "clocks": clk,
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if pad_hi is not None or flip:
+        out["config"]["pad_hi"] = list(pad_hi) if pad_hi is not None else list(wl.pad)
+        out["config"]["flip"] = flip
+        if rank == 0 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = {"skipped": "the CPU baseline is timed on the workload's own padding, no flip"}
+    elif rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
     if dist is not None:
         dist.destroy_process_group()
@@ -555,9 +566,12 @@ def main(argv=None):
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     ap.add_argument("--variant", default="AUTO",
                     choices=["AUTO", "SIMT", "TC_TMA", "TC_GATHER", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T", "TC_HALO_T",
-                             "TC_HALO_T_PAIR"],
+                             "TC_HALO_T_PAIR", "TC_PHASE"],
                     help="kernel variant (default: the library's own choice)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--pad-hi", default=None,
+                    help="padding above each dimension, 'd,h,w' (the workload's pad stays the padding below)")
+    ap.add_argument("--flip", action="store_true", help="read the filter reversed (a true convolution)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least three untimed warm-up steps
     if args.impl == "reference":

@@ -539,7 +539,6 @@ int plan_halo_t(const Problem& P, bool pair, int sms, TcPlan& plan) {
 int plan_phase(const Problem& P, int sms, TcPlan& plan) {
   if (P.dtype == CONV_F32 || P.G != 1) return CONV_EUNSUPPORTED;
   if (!is_2d(P)) return CONV_EUNSUPPORTED;
-  if (P.flip) return CONV_EUNSUPPORTED;  // B's phase rows assume the filter's own tap order
   if (P.d[2] != 1) return CONV_EUNSUPPORTED;  // a filter row's taps are contiguous
   const int sh = P.s[1], sw = P.s[2];
   if (P.H % sh != 0) return CONV_EUNSUPPORTED;  // input rows as (ih / sh, ih % sh)

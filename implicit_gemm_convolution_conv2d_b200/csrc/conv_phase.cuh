@@ -151,8 +151,15 @@ __global__ void __launch_bounds__(kPhThreads, 1)
           const int ja = 2 * lane - off, jb = ja + 1;
           const uint32_t ma = static_cast<unsigned>(ja) < static_cast<unsigned>(KWC) ? 0xffffu : 0u;
           const uint32_t mb = static_cast<unsigned>(jb) < static_cast<unsigned>(KWC) ? 0xffffu : 0u;
-          const uint32_t ca = 2u * static_cast<uint32_t>(min(max(ja, 0), KWC - 1));
-          const uint32_t cb = 2u * static_cast<uint32_t>(min(max(jb, 0), KWC - 1));
+          // element j = kw*C + c of the filter row; with flip it reads filter row
+          // kH-1-kh (below) and, within it, kw mirrored: (kW-1-kw)*C + c
+          const auto src_elem = [&](int j) {
+            const int jc = min(max(j, 0), KWC - 1);
+            return a.flip ? (a.kW - 1 - jc / a.C) * a.C + jc % a.C : jc;
+          };
+          const uint32_t ca = 2u * static_cast<uint32_t>(src_elem(ja));
+          const uint32_t cb = 2u * static_cast<uint32_t>(src_elem(jb));
+          const int kh_src = a.flip ? a.kH - 1 - kh : kh;
           const int o_begin = max(0, r0 - i * a.O), o_end = min(a.O, r0 + hb - i * a.O);
           const int lrb = i * a.O - r0;  // this CTA's B row of (i, o = 0)
           const uint32_t blk = b_addr + static_cast<uint32_t>(kh) * a.ph_bblk + ((lane & 3) << 2);
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(kPhThreads, 1)
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               const int o = min(o0 + u, o_end - 1);
-              const uint32_t base = ws_addr + 2u * static_cast<uint32_t>(o * taps_row + kh * KWC);
+              const uint32_t base = ws_addr + 2u * static_cast<uint32_t>(o * taps_row + kh_src * KWC);
               ha[u] = lds16(base + ca);
               hv[u] = lds16(base + cb);
             }

@@ -127,9 +127,8 @@ int conv_fwd(const void* x, const void* w, void* y,
  * kW-1-kw, c] (a true convolution; 0 is the cross-correlation above).  The
  * flip is the MLX pull request's "correct flip" of its input loader ("What
  * changed"); per-side padding generalises the symmetric padding.  variant is
- * CONV_VARIANT_AUTO or an explicit CONV_VARIANT_*; with flip the phase-packed
- * kernel and the gather kernel's filter-row layouts are not used (AUTO picks
- * another).  Returns as conv_fwd / conv_fwd_variant; CONV_EINVAL also for a
+ * CONV_VARIANT_AUTO or an explicit CONV_VARIANT_*; with flip the gather
+ * kernel does not use its filter-row layouts.  Returns as conv_fwd / conv_fwd_variant; CONV_EINVAL also for a
  * negative pad or a flip other than 0 or 1. */
 int conv_fwd_ex(const void* x, const void* w, void* y,
                 int N, int D, int H, int W, int C, int O,

@@ -96,13 +96,10 @@ def test_flip_and_side_padding_arguments(C):
     assert ex(i3(0, 1, 1), 2) == -1            # flip is 0 or 1
     assert ex(i3(0, 1, 1), 0, 9) == -2         # dtype
     assert ex(i3(0, 1, 1), 0, 1, 10) == -1     # unknown variant
-    # the phase-packed kernel does not take flip; the automatic choice then avoids it
+    # flip keeps the phase-packed kernel (its B rows are built from the mirrored filter)
     stem = (2, 1, 32, 32, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
     assert C.plan(*stem)[0] == C.VARIANT_TC_PHASE
-    assert C.plan(*stem, flip=1)[0] == C.VARIANT_TC_GATHER
-    with pytest.raises(C.ConvError) as e:
-        C.plan(*stem, C.VARIANT_TC_PHASE, flip=1)
-    assert e.value.code == -7
+    assert C.plan(*stem, flip=1)[0] == C.VARIANT_TC_PHASE
     # depth padding on one side makes a 2-D-looking problem 3-D (Do = 2)
     assert C.out_dims(1, 8, 8, 1, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1), (1, 1, 1)) == (2, 8, 8)
 
