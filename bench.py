@@ -410,11 +410,17 @@ def bench_ours(args):
     peaks, peak_src = measured_peaks()
     kern_ms = local_ms / timed_launches
     achieved_tflops = flops / (kern_ms * 1e-3) / 1e12
-    tensor_bound = wl.dtype in ("f16", "bf16") and flops / (xb + wb + yb) > 300
-    if wl.dtype == "f32":
-        sm_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
-        props = torch.cuda.get_device_properties(dev)
-        peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
+    # The bound is the roof whose time is longer: FLOPs at the kernel's own
+    # arithmetic peak (FP32 FMA lanes for the SIMT and depthwise kernels, the
+    # tensor cores for the rest) against the algorithmic bytes at HBM speed.
+    sm_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
+    alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
+    fma_kernel = variant in (C.VARIANT_SIMT, C.VARIANT_DEPTHWISE, C.VARIANT_DEPTHWISE_DIRECT)
+    compute_peak = alu_peak if fma_kernel else float(peaks["bf16_tflops"])
+    hbm_bound = (xb + wb + yb) / (float(peaks["hbm_gbs"]) * 1e9) > flops / (compute_peak * 1e12)
+    tensor_bound = not fma_kernel and not hbm_bound
+    if fma_kernel and not hbm_bound:
+        peak = alu_peak
         roof = {"bound": "alu", "achieved": round(achieved_tflops, 3), "peak": round(peak, 2),
                 "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
                 "peak_source": "148 SMs x 128 FP32 lanes x 2 FLOP x max SM clock"}
@@ -444,7 +450,8 @@ def bench_ours(args):
                    "global_batch": wl.N * nranks, "parallelism": f"independent batches x{nranks}",
                    "variant": vname,
                    "tile": (simt_tile(wl, dims, bn, ctas) if variant == C.VARIANT_SIMT else
-                            [bn, 128] if variant == C.VARIANT_TC_TMA_T
+                            [4, bn] if variant in (C.VARIANT_DEPTHWISE, C.VARIANT_DEPTHWISE_DIRECT)  # pixels x channels per thread
+                            else [bn, 128] if variant == C.VARIANT_TC_TMA_T
                             else [bn, 128 if (wl.O // wl.groups) % 128 == 0 else 64] if variant == C.VARIANT_TC_HALO_T
                             else [bn, 256] if variant == C.VARIANT_TC_HALO_T_PAIR
                             else [256 if "pair" in vname else 128, bn]),
@@ -566,7 +573,7 @@ def main(argv=None):
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     ap.add_argument("--variant", default="AUTO",
                     choices=["AUTO", "SIMT", "TC_TMA", "TC_GATHER", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T", "TC_HALO_T",
-                             "TC_HALO_T_PAIR", "TC_PHASE"],
+                             "TC_HALO_T_PAIR", "TC_PHASE", "DEPTHWISE", "DEPTHWISE_DIRECT"],
                     help="kernel variant (default: the library's own choice)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--pad-hi", default=None,

@@ -18,6 +18,7 @@
 #include "conv_tct.cuh"
 #include "conv_halo_t.cuh"
 #include "conv_phase.cuh"
+#include "conv_dw.cuh"
 
 namespace convfwd {
 namespace {
@@ -753,7 +754,223 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
 // SM pairs, else single CTAs.  Every choice here is the fastest measured on
 // B200 for the shapes of the workload set; TC_HALO, TC_HALO_PAIR and
 // TC_HALO_T_PAIR stay explicit (slower there than the choice made here).
+// Depthwise kernels (conv_dw.cuh): one filter per channel (groups = C = O)
+// with 16-byte channel vectors, P = 4 output pixels per thread.  The
+// TMA-staged form (persistent CTAs, input slabs through an mbarrier ring) is
+// the DEPTHWISE variant wherever its slabs fit; the direct form (loads from
+// global memory, one block per CB x PB pixel groups) is DEPTHWISE_DIRECT and
+// the fallback.
+constexpr int kDwP = 4;
+constexpr size_t kDwTmaSmem = 220 * 1024;
+
+int dw_vec(const Problem& P) { return P.dtype == CONV_F32 ? 4 : 8; }
+
+bool dw_fits(const Problem& P) {
+  const long long taps = static_cast<long long>(P.kD) * P.kH * P.kW;
+  return P.Cg == 1 && P.Og == 1 && (static_cast<long long>(P.C) * static_cast<long long>(P.esize)) % 16 == 0 &&
+         taps * dw_vec(P) * 4 <= kDwSmemLimit;
+}
+
+void dw_geometry(const Problem& P, DwArgs& a) {
+  a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.C = P.C;
+  a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
+  a.sd = P.s[0]; a.sh = P.s[1]; a.sw = P.s[2];
+  a.pd = P.p[0]; a.ph = P.p[1]; a.pw = P.p[2];
+  a.dd = P.d[0]; a.dh = P.d[1]; a.dw = P.d[2];
+  a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
+  a.wg = (P.Wo + kDwP - 1) / kDwP;
+  a.flip = P.flip;
+}
+
+int plan_dw(const Problem& P, DwArgs& a, dim3& grid, dim3& block, size_t& smem) {
+  if (!dw_fits(P)) return CONV_EUNSUPPORTED;
+  dw_geometry(P, a);
+  const int V = dw_vec(P);
+  const int cvs = P.C / V;
+  const long long taps = static_cast<long long>(P.kD) * P.kH * P.kW;
+  int cb = std::min(cvs, kDwMaxCB);
+  while (cb > 1 && taps * cb * V * 4 > kDwSmemLimit) cb = (cb + 1) / 2;
+  a.cb = cb;
+  a.pb = std::max(1, kDwThreads / cb);
+  long long groups;
+  if (!mul_ok(static_cast<long long>(P.N) * P.Do, static_cast<long long>(P.Ho) * a.wg, groups))
+    return CONV_EINVAL;
+  if (groups > 0x7fffffffLL - kDwThreads) return CONV_EUNSUPPORTED;
+  a.groups = static_cast<int>(groups);
+  const long long bx = (groups + a.pb - 1) / a.pb;
+  const long long by = (cvs + cb - 1) / cb;
+  if (bx > 0x7fffffffLL || by > 65535) return CONV_EUNSUPPORTED;
+  grid = dim3(static_cast<unsigned>(bx), static_cast<unsigned>(by), 1);
+  block = dim3(static_cast<unsigned>(cb * a.pb), 1, 1);
+  smem = static_cast<size_t>(taps * cb * V) * sizeof(float);
+  return CONV_OK;
+}
+
+// Tile of the TMA-staged form: CB = up to 16 channel vectors (the channel
+// tiles balanced), GW = 4 pixel groups (16 columns) per tile row, TH rows to
+// fill the 256 consumer threads; rows, then columns, halved until the slab
+// box fits TMA's 256-element box limit and two slabs fit beside the filters.
+// Two CTAs share an SM (half the shared memory each) when that leaves them
+// two slabs or more; otherwise one CTA takes it all.
+int dw_tma_tile(const Problem& P, DwTmaArgs& t, long long budget) {
+  DwArgs& a = t.d;
+  const int V = dw_vec(P);
+  const long long taps = static_cast<long long>(P.kD) * P.kH * P.kW;
+  const long long wbytes = (taps * a.cb * V * 4 + 15) / 16 * 16;
+  const long long tail = static_cast<long long>(sizeof(DwTmaTail));
+  t.GW = std::min(4, a.wg);
+  t.TH = std::max(1, std::min(kDwTmaConsumers / (a.cb * t.GW), P.Ho));
+  while (true) {
+    t.TW = t.GW * kDwP;
+    t.span_h = (t.TH - 1) * P.s[1] + (P.kH - 1) * P.d[1] + 1;
+    t.span_w = (t.TW - 1) * P.s[2] + (P.kW - 1) * P.d[2] + 1;
+    const long long slab = static_cast<long long>(t.span_h) * t.span_w * a.cb * 16;
+    const long long pitch = (slab + 127) / 128 * 128;
+    const long long room = budget - wbytes - tail;
+    t.stages = room > 0 ? static_cast<int>(std::min<long long>(kDwTmaMaxStages, room / pitch)) : 0;
+    if (t.span_h <= 256 && t.span_w <= 256 && t.stages >= 2) {
+      t.slab_bytes = static_cast<uint32_t>(slab);
+      t.slab_pitch = static_cast<uint32_t>(pitch);
+      t.w_off = static_cast<uint32_t>(pitch * t.stages);
+      t.tail_off = static_cast<uint32_t>(t.w_off + wbytes);
+      return CONV_OK;
+    }
+    if (t.TH > 1) t.TH = (t.TH + 1) / 2;
+    else if (t.GW > 1) t.GW = (t.GW + 1) / 2;
+    else return CONV_EUNSUPPORTED;
+  }
+}
+
+int plan_dw_tma(const Problem& P, int sms, DwTmaArgs& t, int& grid, size_t& smem) {
+  if (!dw_fits(P)) return CONV_EUNSUPPORTED;
+  std::memset(&t, 0, sizeof(t));
+  DwArgs& a = t.d;
+  dw_geometry(P, a);
+  const int V = dw_vec(P);
+  const int cvs = P.C / V;
+  t.nct = (cvs + 15) / 16;
+  a.cb = (cvs + t.nct - 1) / t.nct;
+  int per_sm = 2;
+  if (dw_tma_tile(P, t, static_cast<long long>(kDwTmaSmem) / 2) != CONV_OK) {
+    per_sm = 1;
+    if (dw_tma_tile(P, t, static_cast<long long>(kDwTmaSmem)) != CONV_OK) return CONV_EUNSUPPORTED;
+  }
+  t.tiles_h = (P.Ho + t.TH - 1) / t.TH;
+  t.tiles_w = (P.Wo + t.TW - 1) / t.TW;
+  long long tiles;
+  if (!mul_ok(static_cast<long long>(P.N) * P.Do, static_cast<long long>(t.tiles_h) * t.tiles_w, tiles))
+    return CONV_EINVAL;
+  if (tiles > 0x7fffffffLL) return CONV_EUNSUPPORTED;
+  t.tiles = static_cast<int>(tiles);
+  const long long per_ct = std::max<long long>(1, std::min<long long>(static_cast<long long>(sms) * per_sm / t.nct, tiles));
+  const long long g = per_ct * t.nct;
+  if (g > 0x7fffffffLL) return CONV_EUNSUPPORTED;
+  grid = static_cast<int>(g);
+  smem = t.tail_off + sizeof(DwTmaTail);
+  t.timeout_ns = kWaitTimeoutNs;
+  return CONV_OK;
+}
+
+// x as a 5-D tensor (C, W, H, D, N); box = one slab of a channel tile.
+int encode_dw_map(const Problem& P, const DwTmaArgs& t, const void* x, CUtensorMap& m) {
+  std::memset(&m, 0, sizeof(m));
+  const DriverFns& drv = driver_fns();
+  if (!drv.tiled) return CONV_EDRIVER;
+  const CUtensorMapDataType dt = P.dtype == CONV_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : P.dtype == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t e = static_cast<cuuint64_t>(P.esize);
+  const cuuint64_t C = P.C, W = P.W, H = P.H, D = P.D;
+  cuuint64_t dim[5] = {C, W, H, D, static_cast<cuuint64_t>(P.N)};
+  cuuint64_t str[4] = {e * C, e * C * W, e * C * W * H, e * C * W * H * D};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(t.d.cb * dw_vec(P)), static_cast<cuuint32_t>(t.span_w),
+                       static_cast<cuuint32_t>(t.span_h), 1u, 1u};
+  cuuint32_t est[5] = {1, 1, 1, 1, 1};
+  const CUresult r = drv.tiled(&m, dt, 5, const_cast<void*>(x), dim, str, box, est, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  small_tensor_fixup(m, P.x_bytes, drv.driver_version);
+  return CONV_OK;
+}
+
+template <typename T, int V, int KW, int SW, int DW>
+cudaError_t launch_dw_t(const DwArgs& a, dim3 grid, dim3 block, size_t smem, cudaStream_t st) {
+  auto* k = conv_fwd_dw_direct_kernel<T, V, kDwP, KW, SW, DW>;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  k<<<grid, block, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T, int V, int KW, int SW, int DW>
+cudaError_t launch_dw_tma_t(const CUtensorMap& m, const DwTmaArgs& t, int grid, size_t smem, cudaStream_t st) {
+  auto* k = conv_fwd_dw_tma_kernel<T, V, kDwP, KW, SW, DW>;
+  const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  k<<<grid, kDwTmaThreads, smem, st>>>(m, t);
+  return cudaGetLastError();
+}
+
+// The filter-row forms compiled with their width, stride and dilation fixed
+// (the register window); any other width runs the generic form.
+template <typename T, int V>
+cudaError_t launch_dw_shape(const DwArgs& a, dim3 grid, dim3 block, size_t smem, cudaStream_t st) {
+  if (a.dw == 1 && a.sw == 1) {
+    if (a.kW == 3) return launch_dw_t<T, V, 3, 1, 1>(a, grid, block, smem, st);
+    if (a.kW == 5) return launch_dw_t<T, V, 5, 1, 1>(a, grid, block, smem, st);
+    if (a.kW == 7) return launch_dw_t<T, V, 7, 1, 1>(a, grid, block, smem, st);
+  }
+  if (a.dw == 1 && a.sw == 2 && a.kW == 3) return launch_dw_t<T, V, 3, 2, 1>(a, grid, block, smem, st);
+  return launch_dw_t<T, V, 0, 0, 0>(a, grid, block, smem, st);
+}
+
+template <typename T, int V>
+cudaError_t launch_dw_tma_shape(const CUtensorMap& m, const DwTmaArgs& t, int grid, size_t smem, cudaStream_t st) {
+  const DwArgs& a = t.d;
+  if (a.dw == 1 && a.sw == 1) {
+    if (a.kW == 3) return launch_dw_tma_t<T, V, 3, 1, 1>(m, t, grid, smem, st);
+    if (a.kW == 5) return launch_dw_tma_t<T, V, 5, 1, 1>(m, t, grid, smem, st);
+    if (a.kW == 7) return launch_dw_tma_t<T, V, 7, 1, 1>(m, t, grid, smem, st);
+  }
+  if (a.dw == 1 && a.sw == 2 && a.kW == 3) return launch_dw_tma_t<T, V, 3, 2, 1>(m, t, grid, smem, st);
+  return launch_dw_tma_t<T, V, 0, 0, 0>(m, t, grid, smem, st);
+}
+
+int launch_dw_direct(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st) {
+  DwArgs a;
+  dim3 grid, block;
+  size_t smem;
+  const int rc = plan_dw(P, a, grid, block, smem);
+  if (rc != CONV_OK) return rc;
+  a.x = x; a.w = w; a.y = y;
+  cudaError_t e;
+  if (P.dtype == CONV_F32) e = launch_dw_shape<float, 4>(a, grid, block, smem, st);
+  else if (P.dtype == CONV_F16) e = launch_dw_shape<__half, 8>(a, grid, block, smem, st);
+  else e = launch_dw_shape<__nv_bfloat16, 8>(a, grid, block, smem, st);
+  return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+}
+
+int launch_dw(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st, int sms) {
+  DwTmaArgs t;
+  int grid;
+  size_t smem;
+  if (plan_dw_tma(P, sms, t, grid, smem) != CONV_OK) return launch_dw_direct(P, x, w, y, st);
+  t.d.x = x; t.d.w = w; t.d.y = y;
+  CUtensorMap m;
+  const int rc = encode_dw_map(P, t, x, m);
+  if (rc != CONV_OK) return rc;
+  cudaError_t e;
+  if (P.dtype == CONV_F32) e = launch_dw_tma_shape<float, 4>(m, t, grid, smem, st);
+  else if (P.dtype == CONV_F16) e = launch_dw_tma_shape<__half, 8>(m, t, grid, smem, st);
+  else e = launch_dw_tma_shape<__nv_bfloat16, 8>(m, t, grid, smem, st);
+  return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+}
+
 int choose_variant(const Problem& P, int sms) {
+  if (dw_fits(P)) return CONV_VARIANT_DEPTHWISE;
   if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
   bool r5;
   if (!tma_fits(P, r5)) {
@@ -1176,6 +1393,8 @@ int run(const Problem& P, const void* x, const void* w, void* y, int variant, cu
   if (rc != CONV_OK) return rc;
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
   if (variant == CONV_VARIANT_SIMT) return launch_simt(P, x, w, y, st, sms);
+  if (variant == CONV_VARIANT_DEPTHWISE) return launch_dw(P, x, w, y, st, sms);
+  if (variant == CONV_VARIANT_DEPTHWISE_DIRECT) return launch_dw_direct(P, x, w, y, st);
   TcPlan plan;
   rc = plan_tc(P, variant, sms, plan);
   if (rc != CONV_OK) return rc;
@@ -1207,7 +1426,7 @@ int conv_fwd_ex(const void* x, const void* w, void* y, int N, int D, int H, int 
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_PHASE) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_DEPTHWISE_DIRECT) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1251,10 +1470,29 @@ int conv_plan_ex(int N, int D, int H, int W, int C, int O, int kD, int kH, int k
   Problem P;
   int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, flip, dtype);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_PHASE) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_DEPTHWISE_DIRECT) return CONV_EINVAL;
   int dev, sms = 148;
   if (current_device(dev) == CONV_OK) device_sms(dev, sms);
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
+  if (variant == CONV_VARIANT_DEPTHWISE || variant == CONV_VARIANT_DEPTHWISE_DIRECT) {
+    DwTmaArgs ta;
+    int tgrid;
+    size_t smem;
+    if (variant == CONV_VARIANT_DEPTHWISE && plan_dw_tma(P, sms, ta, tgrid, smem) == CONV_OK) {
+      if (bn) *bn = dw_vec(P);  // channels per thread
+      if (stages) *stages = ta.stages;
+      if (ctas) *ctas = tgrid;
+      return variant;
+    }
+    DwArgs da;
+    dim3 grid, block;
+    rc = plan_dw(P, da, grid, block, smem);
+    if (rc != CONV_OK) return rc;
+    if (bn) *bn = dw_vec(P);
+    if (stages) *stages = 1;
+    if (ctas) *ctas = static_cast<int>(std::min<long long>(static_cast<long long>(grid.x) * grid.y, 0x7fffffffLL));
+    return variant;
+  }
   if (variant == CONV_VARIANT_SIMT) {
     const SimtShape sh = simt_shape(P, sms);
     if (bn) *bn = 16 * sh.tn;

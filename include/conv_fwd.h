@@ -88,11 +88,16 @@ enum {
                                    C/G % 32 == 0, O/G % 64 == 0) */
   CONV_VARIANT_TC_HALO_T_PAIR = 8, /* TC_HALO_T with CTA pairs: M = 256 output channels,
                                    cta_group::2 (O/G % 256 == 0) */
-  CONV_VARIANT_TC_PHASE = 9       /* 2-D layers with few input channels: one GEMM row =
+  CONV_VARIANT_TC_PHASE = 9,      /* 2-D layers with few input channels: one GEMM row =
                                    P output pixels of a row (P*sw*C a multiple of 8),
                                    its window of the flattened (w, c) input row loaded
                                    by TMA; N = P*O <= 256, a multiple of 32 (groups 1, width dilation 1,
                                    H % sh == 0, W*C*2 % 16 == 0, Wo % P == 0) */
+  CONV_VARIANT_DEPTHWISE = 10,    /* depthwise (groups = C = O, C*elem % 16 == 0), any element
+                                   type, FP32 FMAs: persistent CTAs, input slabs staged by TMA
+                                   through an mbarrier ring (DEPTHWISE_DIRECT where the slabs do
+                                   not fit); the automatic choice for these shapes */
+  CONV_VARIANT_DEPTHWISE_DIRECT = 11 /* depthwise, loads straight from global memory */
 };
 
 /* Output extents.  stride/pad/dil: 3 ints (d, h, w).  out: 3 ints (Do, Ho, Wo).
@@ -112,7 +117,8 @@ int conv_out_dims(int D, int H, int W, int kD, int kH, int kW,
  * 256-pixel tiles as SMs;
  * otherwise TC_TMA_PAIR (or TC_TMA when there are fewer 256-row output tiles
  * than SM pairs); otherwise TC_PHASE where its conditions hold, else
- * TC_GATHER.  TC_HALO, TC_HALO_PAIR and
+ * TC_GATHER.  Depthwise problems (groups = C = O, C*elem % 16 == 0), of any
+ * type, run DEPTHWISE.  TC_HALO, TC_HALO_PAIR and
  * TC_HALO_T_PAIR run only when requested through conv_fwd_variant. */
 int conv_fwd(const void* x, const void* w, void* y,
              int N, int D, int H, int W, int C, int O,
@@ -177,7 +183,9 @@ int conv_plan_ex(int N, int D, int H, int W, int C, int O, int kD, int kH, int k
 
 /* The variant conv_fwd would run for this shape and type (CONV_VARIANT_*), or
  * a negative error code.  Also reports the output-tile width BN, the number of
- * pipeline stages and the number of CTAs it would launch (any may be NULL).
+ * pipeline stages and the number of CTAs it would launch (any may be NULL);
+ * for DEPTHWISE / DEPTHWISE_DIRECT, BN is the number of channels a thread
+ * computes and stages is the slab ring depth (1 for the direct form).
  * Queries the current device's SM count; queues nothing. */
 int conv_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
               const int stride[3], const int pad[3], const int dil[3],

@@ -95,7 +95,7 @@ def test_flip_and_side_padding_arguments(C):
     assert ex(i3(0, -1, 0), 0) == -1           # negative high-side pad
     assert ex(i3(0, 1, 1), 2) == -1            # flip is 0 or 1
     assert ex(i3(0, 1, 1), 0, 9) == -2         # dtype
-    assert ex(i3(0, 1, 1), 0, 1, 10) == -1     # unknown variant
+    assert ex(i3(0, 1, 1), 0, 1, 12) == -1     # unknown variant
     # flip keeps the phase-packed kernel (its B rows are built from the mirrored filter)
     stem = (2, 1, 32, 32, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
     assert C.plan(*stem)[0] == C.VARIANT_TC_PHASE
@@ -138,7 +138,7 @@ def test_invalid_arguments_rejected_on_host(C):
     big = 1 << 30
     assert call(X, Wt, Y, big, big, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
     # unknown variant
-    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 10, None) == -1
+    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 12, None) == -1
     assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, -2, None) == -1
 
 
@@ -218,6 +218,30 @@ def test_explicit_variant_plan(C):
     with pytest.raises(C.ConvError) as e:
         C.plan(*g3, "f32", C.VARIANT_TC_TMA)
     assert e.value.code == -7
+    # depthwise (groups = C = O) with 16-byte channel vectors, any type; 8
+    # channels per thread for 16-bit types, 4 for f32.  The TMA-staged form
+    # runs persistent CTAs (at most two per SM for each channel tile, the
+    # planner assumes 148 SMs without a device) over a ring of 2-4 slabs; the
+    # direct form launches one block per 256 (channel vector, pixel group) tasks
+    dw = (32, 1, 112, 112, 128, 128, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 128)
+    for dt, vec in (("f16", 8), ("bf16", 8), ("f32", 4)):
+        v, bn, stages, ctas = C.plan(*dw, dt)
+        assert (v, bn) == (C.VARIANT_DEPTHWISE, vec) and 2 <= stages <= 4 and ctas <= 2 * 148
+        v, bn, stages, ctas = C.plan(*dw, dt, C.VARIANT_DEPTHWISE_DIRECT)
+        assert (v, bn, stages) == (C.VARIANT_DEPTHWISE_DIRECT, vec, 1)
+        assert ctas == -(-32 * 112 * 28 * (128 // vec) // 256)
+    dw4 = (2, 1, 7, 9, 4, 4, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 4)
+    assert C.plan(*dw4, "f32")[0] == C.VARIANT_DEPTHWISE
+    assert C.plan(*dw4, "f16")[0] != C.VARIANT_DEPTHWISE
+    for args in ((*dw4, "f16"), (*g3, "bf16")):
+        for v in (C.VARIANT_DEPTHWISE, C.VARIANT_DEPTHWISE_DIRECT):
+            with pytest.raises(C.ConvError) as e:
+                C.plan(*args, v)
+            assert e.value.code == -7
+    # a slab taller than one TMA box allows (5 rows at height dilation 70 span
+    # 281 > 256 input rows): DEPTHWISE runs the direct form, one stage
+    tall = (1, 1, 200, 32, 16, 16, (1, 5, 3), (1, 1, 1), (0, 140, 1), (1, 70, 1), 16)
+    assert C.plan(*tall, "f16")[:3] == (C.VARIANT_DEPTHWISE, 8, 1)
     with pytest.raises(C.ConvError) as e:
-        C.plan(*g3, "bf16", 10)
+        C.plan(*g3, "bf16", 12)
     assert e.value.code == -1

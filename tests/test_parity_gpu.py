@@ -50,9 +50,9 @@ def run_gpu(x, w, wl, variant, guard=64):
 
 
 def variants_for(wl):
-    vs = []
+    vs = [C.VARIANT_DEPTHWISE, C.VARIANT_DEPTHWISE_DIRECT] if depthwise_applies(wl) else []
     if wl.dtype == "f32":
-        return [C.VARIANT_SIMT]
+        return vs + [C.VARIANT_SIMT]
     vs.append(C.VARIANT_TC_GATHER)
     if (wl.C // wl.groups) % 16 == 0:
         vs += [C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR]
@@ -67,6 +67,12 @@ def variants_for(wl):
     if phase_applies(wl):
         vs.append(C.VARIANT_TC_PHASE)
     return vs
+
+
+def depthwise_applies(wl):
+    """The direct depthwise kernel's conditions: one filter per channel and
+    16-byte channel vectors."""
+    return wl.groups == wl.C == wl.O and wl.C * WL.ELEM_BYTES[wl.dtype] % 16 == 0
 
 
 def phase_applies(wl):
@@ -156,6 +162,23 @@ SMALL = [
     WL.case(1, 1, 16, 32, 3, 64, (1, 2, 2), (1, 2, 2), (0, 0, 0), name="phase_patchify_k2s2"),
     WL.case(1, 1, 17, 32, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), name="phase_odd_h"),
     WL.case(1, 1, 20, 200, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), name="phase_wide_rows_3_boxes"),
+    # direct depthwise kernel (groups = C = O): 2-D and 3-D, ragged last pixel
+    # group (Wo % 4 != 0), stride 2, dilation, 5x5 and 7x7 filters, 8 and 24
+    # channels; C = 4 runs it in f32 only (8-byte f16 vectors fall back)
+    WL.case(2, 1, 13, 11, 64, 64, (1, 3, 3), pad=(0, 1, 1), groups=64, name="dw_c64_k3"),
+    WL.case(3, 1, 17, 19, 8, 8, (1, 3, 3), (1, 2, 2), (0, 1, 1), groups=8, name="dw_c8_s2_ragged"),
+    WL.case(1, 5, 6, 7, 16, 16, (3, 3, 3), pad=(1, 1, 1), groups=16, name="dw_3d_c16"),
+    WL.case(1, 1, 17, 18, 32, 32, (1, 5, 5), pad=(0, 4, 4), dil=(1, 2, 2), groups=32, name="dw_k5_dil2"),
+    WL.case(2, 1, 9, 30, 24, 24, (1, 7, 7), (1, 1, 2), (0, 3, 3), groups=24, name="dw_k7_c24_sw2"),
+    WL.case(2, 1, 7, 9, 4, 4, (1, 3, 3), pad=(0, 1, 1), groups=4, name="dw_c4"),
+    WL.case(1, 1, 3, 2, 8, 8, (1, 5, 5), pad=(0, 2, 2), groups=8, name="dw_kernel_larger_than_input"),
+    # several channel tiles (384 channels: three of 128; 200: two of 104, the
+    # last one partly past C), output planes whose filter taps all fall in the
+    # depth padding, and a slab taller than a TMA box (direct form)
+    WL.case(1, 1, 9, 21, 384, 384, (1, 3, 3), pad=(0, 1, 1), groups=384, name="dw_c384_three_ctiles"),
+    WL.case(2, 1, 9, 21, 200, 200, (1, 3, 3), pad=(0, 1, 1), groups=200, name="dw_c200_partial_ctile"),
+    WL.case(1, 3, 5, 6, 8, 8, (3, 3, 3), (2, 1, 1), (3, 1, 1), groups=8, name="dw_3d_empty_planes"),
+    WL.case(1, 1, 200, 32, 16, 16, (1, 5, 3), pad=(0, 140, 1), dil=(1, 70, 1), groups=16, name="dw_tall_slab"),
 ]
 
 
@@ -181,10 +204,12 @@ FLIP_PAD = [
     (WL.case(2, 4, 6, 7, 21, 21, (3, 3, 3), pad=(1, 1, 0), name="fp_3d_c21"), (2, 0, 1)),
     (WL.case(2, 1, 9, 11, 5, 8, (1, 3, 3), (1, 2, 1), (0, 1, 2), dil=(1, 1, 2), name="fp_c5_s2_dil"), (0, 2, 0)),
     (WL.case(1, 6, 7, 8, 64, 128, (3, 1, 1), pad=(2, 0, 0), name="fp_k311"), (0, 0, 0)),
+    (WL.case(2, 1, 11, 13, 32, 32, (1, 3, 5), (1, 1, 2), (0, 2, 1), groups=32, name="fp_depthwise"), (0, 0, 3)),
+    (WL.case(1, 4, 6, 7, 16, 16, (3, 3, 3), pad=(0, 1, 2), groups=16, name="fp_depthwise_3d"), (2, 1, 0)),
 ]
 
 ALL_VARIANTS = ["SIMT", "TC_TMA", "TC_GATHER", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T", "TC_HALO_T",
-                "TC_HALO_T_PAIR", "TC_PHASE"]
+                "TC_HALO_T_PAIR", "TC_PHASE", "DEPTHWISE", "DEPTHWISE_DIRECT"]
 
 
 def run_gpu_ex(x, w, wl, pad_hi, flip, variant, guard=64):
@@ -217,7 +242,7 @@ def test_flip_and_side_padding(case, dtype):
     for flip in (0, 1):
         y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups, pad_hi=pad_hi, flip=bool(flip))
         ran = 0
-        for name in (["SIMT"] if dtype == "f32" else ALL_VARIANTS):
+        for name in (["SIMT", "DEPTHWISE", "DEPTHWISE_DIRECT"] if dtype == "f32" else ALL_VARIANTS):
             v = getattr(C, "VARIANT_" + name)
             try:
                 C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil, wl.groups, dtype, v,
@@ -267,6 +292,10 @@ def test_auto_variant_choice():
         C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR)
     assert C.plan(32, 1, 224, 224, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_PHASE
     assert C.plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f32")[0] == C.VARIANT_SIMT
+    assert C.plan(32, 1, 112, 112, 128, 128, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 128, "f16")[0] == \
+        C.VARIANT_DEPTHWISE
+    assert C.plan(2, 1, 7, 9, 4, 4, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 4, "f32")[0] == C.VARIANT_DEPTHWISE
+    assert C.plan(2, 1, 7, 9, 4, 4, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 4, "f16")[0] != C.VARIANT_DEPTHWISE
 
 
 def test_python_api_2d_and_3d():

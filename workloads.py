@@ -91,6 +91,13 @@ for _dt in ("f16", "f32"):
         _n = f"conv3d_{_dt}_n{_N}_{_S}c_c{_C}_o{_O}_k333"
         WORKLOADS[_n] = _c3(_n, _N, _S, _S, _S, _C, _O, (3, 3, 3), (1, 1, 1), (1, 1, 1), _dt, 4)
 
+# Depthwise 3x3/1/1 (groups = C = O = 128) at 112x112, N=32, fp16, seed 5: the
+# tutorial's variants table lists depthwise layers as memory-bound work for
+# direct kernels; MobileNet-style block shape.
+WORKLOADS["dwconv_f16_n32_112x112_c128_k3"] = Workload(
+    "dwconv_f16_n32_112x112_c128_k3", 32, 1, 112, 112, 128, 128, (1, 3, 3), (1, 1, 1), (0, 1, 1),
+    groups=128, dtype="f16", seed=5)
+
 # Name of the workload the benchmark times by default: the tutorial's
 # arithmetic-intensity example (3x3, 256->256, 56x56) at batch 64.
 HEADLINE = "conv2d_bf16_n64_56x56_c256_o256_k3"
