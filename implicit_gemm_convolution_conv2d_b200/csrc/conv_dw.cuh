@@ -29,6 +29,8 @@
 #pragma once
 
 #include <cstdint>
+#include <cstring>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -236,26 +238,39 @@ __global__ void __launch_bounds__(kDwThreads, 2) conv_fwd_dw_direct_kernel(const
 
 // ---------------------------------------------------------------- TMA-staged form
 //
-// Persistent CTAs, each bound to one channel tile of CB = cb*V channels (its
+// Persistent CTAs, each bound to one channel tile of CB = cb*4 channels (its
 // filters stay in shared memory for the whole launch), walk a static list of
-// output tiles of TH rows x TW = GW*P columns of one (n, od).  A tile's input
-// is, per valid kd, one slab of span_h x span_w pixels x CB channels, which one
-// TMA tiled load brings into shared memory (the hardware zero-fills what lies
-// in the padding).  A producer warp keeps a ring of `stages` slabs ahead of the
-// eight consumer warps (full / empty mbarriers); a consumer thread owns V
-// channels of P output pixels of one tile row, reads the slab with 16-byte
-// shared loads and accumulates every tap in fp32.  CTA b serves channel tile
-// b % nct and tiles b / nct, b / nct + gridDim.x / nct, ...
+// output tiles of TH x TW pixels of one (n, od).  A tile's input is, per valid
+// kd, one slab of span_h x span_w pixels x CB channels, which one TMA tiled
+// load brings into shared memory (the hardware zero-fills what lies in the
+// padding).  A producer warp keeps a ring of `stages` slabs ahead of the eight
+// consumer warps (full / empty mbarriers).  CTA b serves channel tile b % nct
+// and tiles b / nct, b / nct + gridDim.x / nct, ...
+//
+// A consumer thread owns 4 channels (one 8-byte vector for 16-bit types, 16
+// bytes for f32) of a block of R output rows x P output columns; consecutive
+// threads take consecutive channel vectors of a block, so each slab read of
+// a warp is one contiguous run.  The tile is BR x BC blocks (TH = BR*R,
+// TW = BC*P).  Products accumulate in fp32 through packed two-lane FMAs.
+//
+// For square K x K filters with equal strides S and no dilation (K = 3,
+// S = 1 or 2), the K*K weight vectors of the current kd sit in registers and
+// the thread walks the (R-1)*S + K input rows and (P-1)*S + K input columns of
+// its block once each, converting every input vector to fp32 once and
+// applying it to every (output row, output column, tap) that reads it: the
+// pairing is resolved at compile time.  Any other filter runs the generic
+// consumer (R = 1, runtime taps, one slab read per (column, tap)).
 
 struct DwTmaArgs {
-  DwArgs d;              // geometry; d.cb = channel vectors per tile
-  int GW, TH, TW;        // pixel groups per tile row, tile rows, tile columns
+  DwArgs d;              // geometry; d.cb = channel vectors (of 4) per tile
+  int BR, BC;            // blocks per tile: rows, columns
+  int TH, TW;            // tile rows / columns (BR*R, BC*P)
   int span_h, span_w;    // input slab rows / columns
   int tiles_h, tiles_w;  // tiles per output plane
   int nct;               // channel tiles
   int stages;
   int tiles;             // N * Do * tiles_h * tiles_w (below 2^31)
-  uint32_t slab_bytes;   // span_h * span_w * cb * 16
+  uint32_t slab_bytes;   // span_h * span_w * cb * vector bytes
   uint32_t slab_pitch;   // slab_bytes rounded up to 128
   uint32_t w_off;        // byte offset of the filters (after the slabs)
   uint32_t tail_off;     // byte offset of the barriers
@@ -265,6 +280,7 @@ struct DwTmaArgs {
 constexpr int kDwTmaConsumers = 256;                 // eight warps
 constexpr int kDwTmaThreads = kDwTmaConsumers + 32;  // and one producer warp
 constexpr int kDwTmaMaxStages = 4;
+constexpr int kDwTmaP = 4;                           // output columns per block
 
 struct DwTmaTail {
   uint64_t full[kDwTmaMaxStages];
@@ -287,8 +303,8 @@ __device__ __forceinline__ DwUnit dw_unit(const DwTmaArgs& a, int t) {
   return r;
 }
 
-// Filters of channel tile `ct` into s_w (layout of dw_widx), by threads
-// [first, first + count) of the block.
+// Filters of channel tile `ct` into s_w (layout of dw_widx<V>), by threads
+// [tid, tid + count) of the block.
 template <typename T, int V>
 __device__ __forceinline__ void dw_fill_filters(float* s_w, const DwArgs& g, int ct, int taps, int tid,
                                                 int count) {
@@ -303,10 +319,90 @@ __device__ __forceinline__ void dw_fill_filters(float* s_w, const DwArgs& g, int
   }
 }
 
-template <typename T, int V, int P, int KW, int SW, int DW>
-__global__ void __launch_bounds__(kDwTmaThreads, 2)
+// Four channels of T as one vector (8 bytes for 16-bit types, 16 for f32).
+template <typename T>
+struct DwVec4;
+template <>
+struct DwVec4<float> {
+  using type = float4;
+};
+template <>
+struct DwVec4<__half> {
+  using type = uint2;
+};
+template <>
+struct DwVec4<__nv_bfloat16> {
+  using type = uint2;
+};
+
+__device__ __forceinline__ void dw_unpack4(const float4 r, float2 (&f)[2]) {
+  f[0] = make_float2(r.x, r.y);
+  f[1] = make_float2(r.z, r.w);
+}
+template <typename H2, typename U>
+__device__ __forceinline__ H2 dw_bits_as(U u) {
+  H2 h;
+  static_assert(sizeof(H2) == sizeof(U), "size");
+  memcpy(&h, &u, sizeof(h));
+  return h;
+}
+__device__ __forceinline__ void dw_unpack4(const uint2 r, float2 (&f)[2], __half) {
+  f[0] = __half22float2(dw_bits_as<__half2>(r.x));
+  f[1] = __half22float2(dw_bits_as<__half2>(r.y));
+}
+__device__ __forceinline__ void dw_unpack4(const uint2 r, float2 (&f)[2], __nv_bfloat16) {
+  f[0] = __bfloat1622float2(dw_bits_as<__nv_bfloat162>(r.x));
+  f[1] = __bfloat1622float2(dw_bits_as<__nv_bfloat162>(r.y));
+}
+template <typename T>
+__device__ __forceinline__ void dw_load4(const uint8_t* p, float2 (&f)[2]) {
+  if constexpr (sizeof(T) == 4) {
+    dw_unpack4(*reinterpret_cast<const float4*>(p), f);
+  } else {
+    const uint2 r = *reinterpret_cast<const uint2*>(p);
+    dw_unpack4(r, f, T());
+  }
+}
+template <typename T>
+__device__ __forceinline__ void dw_store4(T* dst, const float2 (&f)[2]) {
+  if constexpr (sizeof(T) == 4) {
+    *reinterpret_cast<float4*>(dst) = make_float4(f[0].x, f[0].y, f[1].x, f[1].y);
+  } else if constexpr (std::is_same<T, __half>::value) {
+    const __half2 a = __float22half2_rn(f[0]), b = __float22half2_rn(f[1]);
+    uint2 u;
+    memcpy(&u.x, &a, 4);
+    memcpy(&u.y, &b, 4);
+    *reinterpret_cast<uint2*>(dst) = u;
+  } else {
+    const __nv_bfloat162 a = __float22bfloat162_rn(f[0]), b = __float22bfloat162_rn(f[1]);
+    uint2 u;
+    memcpy(&u.x, &a, 4);
+    memcpy(&u.y, &b, 4);
+    *reinterpret_cast<uint2*>(dst) = u;
+  }
+}
+// The 4 fp32 weights of one tap for one channel vector (layout of dw_widx<4>).
+__device__ __forceinline__ void dw_wload4(const float* p, float2 (&w)[2]) {
+  const float4 t4 = *reinterpret_cast<const float4*>(p);
+  w[0] = make_float2(t4.x, t4.y);
+  w[1] = make_float2(t4.z, t4.w);
+}
+__device__ __forceinline__ void dw_fma4(float2 (&acc)[2], const float2 (&x)[2], const float2 (&w)[2]) {
+  acc[0] = __ffma2_rn(x[0], w[0], acc[0]);
+  acc[1] = __ffma2_rn(x[1], w[1], acc[1]);
+}
+
+// CTAs per SM a form is compiled for: the register forms need more than half
+// an SM's registers per thread (32-64 accumulators and 36 weights).
+constexpr int dw_tma_ctas_per_sm(int K, int R) { return K > 0 && R >= 1 ? 1 : 2; }
+
+// K > 0: the register-resident K x K / stride S consumer with R output rows
+// per block; K = 0: the generic consumer (R = 1).
+template <typename T, int K, int S, int R>
+__global__ void __launch_bounds__(kDwTmaThreads, dw_tma_ctas_per_sm(K, R))
     conv_fwd_dw_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, const DwTmaArgs a) {
-  using Vec = typename DwVec<T, V>::type;
+  constexpr int P = kDwTmaP;
+  constexpr int VB = 4 * static_cast<int>(sizeof(T));  // bytes per channel vector
   extern __shared__ __align__(128) uint8_t smem[];
   const DwArgs& g = a.d;
   const int taps = g.kD * g.kH * g.kW;
@@ -326,9 +422,9 @@ __global__ void __launch_bounds__(kDwTmaThreads, 2)
     ptx::fence_mbar_init();
   }
   if (warp == kDwTmaConsumers / 32 && lane == 0) ptx::prefetch_tmap(&tmap_x);
-  const int ct = static_cast<int>(blockIdx.x % a.nct);
+  const int ct = static_cast<int>(blockIdx.x) % a.nct;
   const int t_first = static_cast<int>(blockIdx.x) / a.nct, t_step = static_cast<int>(gridDim.x) / a.nct;
-  dw_fill_filters<T, V>(s_w, g, ct, taps, static_cast<int>(threadIdx.x), kDwTmaThreads);
+  dw_fill_filters<T, 4>(s_w, g, ct, taps, static_cast<int>(threadIdx.x), kDwTmaThreads);
   __syncthreads();
 
   if (warp == kDwTmaConsumers / 32) {
@@ -351,7 +447,7 @@ __global__ void __launch_bounds__(kDwTmaThreads, 2)
           const uint32_t fb = ptx::smem_u32(&tail->full[stage]);
           ptx::mbar_arrive_expect_tx(fb, a.slab_bytes);
           ptx::tma_load_5d(ptx::smem_u32(slabs + static_cast<size_t>(stage) * a.slab_pitch), &tmap_x, fb,
-                           ct * cb * V, uc.ow0 * g.sw - g.pw, uc.oh0 * g.sh - g.ph, id, uc.n);
+                           ct * cb * 4, uc.ow0 * g.sw - g.pw, uc.oh0 * g.sh - g.ph, id, uc.n);
           ++fills;
           if (++stage == a.stages) {
             stage = 0;
@@ -373,23 +469,29 @@ __global__ void __launch_bounds__(kDwTmaThreads, 2)
   // -------------------------------------------------------------- consumers
   const int tid = static_cast<int>(threadIdx.x);
   const int cv = tid % cb;
-  const int pg = tid / cb;
-  const bool px_active = pg < a.GW * a.TH;
-  const int r = pg / a.GW, gc = pg - (pg / a.GW) * a.GW;
-  const uint32_t rowpitch = static_cast<uint32_t>(a.span_w) * cb * 16;  // bytes per slab row
+  const int blk = tid / cb;
+  const bool blk_active = blk < a.BR * a.BC;
+  const int br = blk / a.BC, bc = blk - (blk / a.BC) * a.BC;
+  const int c0 = (ct * cb + cv) * 4;
+  const bool active = blk_active && c0 < g.C;
+  const uint32_t colb = static_cast<uint32_t>(cb) * VB;   // bytes per slab pixel
+  const uint32_t rowb = static_cast<uint32_t>(a.span_w) * colb;
   T* __restrict__ y = static_cast<T*>(g.y);
+  const float* wbase = s_w + cv * 4;
+
+  // register-resident weights of the current kd (square filters)
+  float2 wreg[K > 0 ? K : 1][K > 0 ? K : 1][2];
+  int wkd = -1;
+
   int stage = 0;
   uint32_t phase = 0;
-  const int c0 = (ct * cb + cv) * V;
-  const bool ch_active = c0 < g.C;
   for (int t = t_first; t < a.tiles; t += t_step) {
     const DwUnit uc = dw_unit(a, t);
-    const bool active = px_active && ch_active;
-    float acc[P][V];
+    float2 acc[R][P][2];
 #pragma unroll
-    for (int p = 0; p < P; ++p)
+    for (int rr = 0; rr < R; ++rr)
 #pragma unroll
-      for (int v = 0; v < V; ++v) acc[p][v] = 0.f;
+      for (int p = 0; p < P; ++p) acc[rr][p][0] = acc[rr][p][1] = make_float2(0.f, 0.f);
 
     for (int kd = 0; kd < g.kD; ++kd) {
       const int id = uc.od * g.sd - g.pd + kd * g.dd;
@@ -397,41 +499,50 @@ __global__ void __launch_bounds__(kDwTmaThreads, 2)
       if (!wait_bounded_warp(ptx::smem_u32(&tail->full[stage]), phase, abort_flag, a.timeout_ns, kSiteMmaFull))
         return;
       if (active) {
-        const uint8_t* slab = slabs + static_cast<size_t>(stage) * a.slab_pitch + static_cast<uint32_t>(cv) * 16;
-        for (int kh = 0; kh < g.kH; ++kh) {
-          const int rin = r * g.sh + kh * g.dh;
-          const float* wtap = s_w + (kd * g.kH + kh) * g.kW * cb * V + cv * 4;
-          if constexpr (KW > 0) {
-            constexpr int SPAN = (P - 1) * SW + (KW - 1) * DW + 1;
-            const uint8_t* rowp = slab + rin * rowpitch + static_cast<uint32_t>(gc * P * SW) * cb * 16;
-            float wv[KW][V];
+        const uint8_t* slab = slabs + static_cast<size_t>(stage) * a.slab_pitch + static_cast<uint32_t>(cv) * VB;
+        if constexpr (K > 0) {
+          if (kd != wkd) {
 #pragma unroll
-            for (int kw = 0; kw < KW; ++kw) dw_weights<V>(wtap + kw * cb * V, cb, wv[kw]);
+            for (int kh = 0; kh < K; ++kh)
+#pragma unroll
+              for (int kw = 0; kw < K; ++kw) dw_wload4(wbase + ((kd * K + kh) * K + kw) * cb * 4, wreg[kh][kw]);
+            wkd = kd;
+          }
+          constexpr int RIN = (R - 1) * S + K;
+          constexpr int SPAN = (P - 1) * S + K;
+          const uint8_t* bp = slab + static_cast<uint32_t>(br * R * S) * rowb + static_cast<uint32_t>(bc * P * S) * colb;
+#pragma unroll
+          for (int i = 0; i < RIN; ++i) {
 #pragma unroll
             for (int j = 0; j < SPAN; ++j) {
-              float xf[V];
-              const Vec raw = *reinterpret_cast<const Vec*>(rowp + static_cast<uint32_t>(j) * cb * 16);
-              dw_unpack<T, V>(raw, xf);
+              float2 xf[2];
+              dw_load4<T>(bp + static_cast<uint32_t>(i) * rowb + static_cast<uint32_t>(j) * colb, xf);
 #pragma unroll
-              for (int p = 0; p < P; ++p)
+              for (int rr = 0; rr < R; ++rr)
 #pragma unroll
-                for (int kw = 0; kw < KW; ++kw)
-                  if (p * SW + kw * DW == j) {
-                    dw_fma<V>(acc[p], xf, wv[kw]);
+                for (int kh = 0; kh < K; ++kh)
+                  if (rr * S + kh == i) {
+#pragma unroll
+                    for (int p = 0; p < P; ++p)
+#pragma unroll
+                      for (int kw = 0; kw < K; ++kw)
+                        if (p * S + kw == j) dw_fma4(acc[rr][p], xf, wreg[kh][kw]);
                   }
             }
-          } else {
-            const uint8_t* rowp = slab + rin * rowpitch;
+          }
+        } else {
+          const uint8_t* bp = slab + static_cast<uint32_t>(br * g.sh) * rowb;
+          for (int kh = 0; kh < g.kH; ++kh) {
+            const uint8_t* rowp = bp + static_cast<uint32_t>(kh * g.dh) * rowb;
             for (int kw = 0; kw < g.kW; ++kw) {
-              float wv[V];
-              dw_weights<V>(wtap + kw * cb * V, cb, wv);
+              float2 wv[2];
+              dw_wload4(wbase + ((kd * g.kH + kh) * g.kW + kw) * cb * 4, wv);
 #pragma unroll
               for (int p = 0; p < P; ++p) {
-                const int col = (gc * P + p) * g.sw + kw * g.dw;
-                float xf[V];
-                const Vec raw = *reinterpret_cast<const Vec*>(rowp + static_cast<uint32_t>(col) * cb * 16);
-                dw_unpack<T, V>(raw, xf);
-                dw_fma<V>(acc[p], xf, wv);
+                const int col = (bc * P + p) * g.sw + kw * g.dw;
+                float2 xf[2];
+                dw_load4<T>(rowp + static_cast<uint32_t>(col) * colb, xf);
+                dw_fma4(acc[0][p], xf, wv);
               }
             }
           }
@@ -445,18 +556,18 @@ __global__ void __launch_bounds__(kDwTmaThreads, 2)
       }
     }
 
-    const int oh = uc.oh0 + r;
-    if (active && oh < g.Ho) {
-      T* yrow = y + ((static_cast<long long>(uc.n) * g.Do + uc.od) * g.Ho + oh) * static_cast<long long>(g.Wo) * g.C + c0;
+    if (active) {
 #pragma unroll
-      for (int p = 0; p < P; ++p) {
-        const int ow = uc.ow0 + gc * P + p;
-        if (ow >= g.Wo) break;
-        Vec out;
-        T* e = reinterpret_cast<T*>(&out);
+      for (int rr = 0; rr < R; ++rr) {
+        const int oh = uc.oh0 + br * R + rr;
+        if (oh >= g.Ho) break;
+        T* yrow = y + ((static_cast<long long>(uc.n) * g.Do + uc.od) * g.Ho + oh) * static_cast<long long>(g.Wo) * g.C + c0;
 #pragma unroll
-        for (int v = 0; v < V; ++v) e[v] = from_f32<T>(acc[p][v]);
-        *reinterpret_cast<Vec*>(yrow + static_cast<long long>(ow) * g.C) = out;
+        for (int p = 0; p < P; ++p) {
+          const int ow = uc.ow0 + bc * P + p;
+          if (ow >= g.Wo) break;
+          dw_store4<T>(yrow + static_cast<long long>(ow) * g.C, acc[rr][p]);
+        }
       }
     }
   }

@@ -806,25 +806,42 @@ int plan_dw(const Problem& P, DwArgs& a, dim3& grid, dim3& block, size_t& smem) 
   return CONV_OK;
 }
 
-// Tile of the TMA-staged form: CB = up to 16 channel vectors (the channel
-// tiles balanced), GW = 4 pixel groups (16 columns) per tile row, TH rows to
-// fill the 256 consumer threads; rows, then columns, halved until the slab
-// box fits TMA's 256-element box limit and two slabs fit beside the filters.
-// Two CTAs share an SM (half the shared memory each) when that leaves them
-// two slabs or more; otherwise one CTA takes it all.
-int dw_tma_tile(const Problem& P, DwTmaArgs& t, long long budget) {
+// Consumer form of the TMA-staged kernel: 3x3 filters at equal strides 1 or
+// 2 without dilation keep their weights in registers and compute blocks of R
+// output rows (R = 4 at stride 1, 2 at stride 2); anything else runs the
+// generic consumer (K = 0, R = 1).
+int dw_tma_form(const Problem& P, int& K, int& S) {
+  if (P.kH == 3 && P.kW == 3 && P.s[1] == P.s[2] && (P.s[1] == 1 || P.s[1] == 2) && P.d[1] == 1 &&
+      P.d[2] == 1) {
+    K = 3;
+    S = P.s[1];
+    return S == 1 ? 4 : 2;
+  }
+  K = 0;
+  S = 0;
+  return 1;
+}
+
+// Tile of the TMA-staged form: the consumer threads are cb channel vectors x
+// BR x BC blocks of R x 4 output pixels (BC = 4 blocks across, BR to fill 256
+// threads, no more rows than the output has); block rows, then columns,
+// halved until the slab box fits TMA's 256-element box limit and two slabs
+// fit beside the filters in `budget` bytes.
+int dw_tma_tile(const Problem& P, DwTmaArgs& t, int R, long long budget) {
   DwArgs& a = t.d;
-  const int V = dw_vec(P);
+  const long long VB = 4LL * P.esize;
   const long long taps = static_cast<long long>(P.kD) * P.kH * P.kW;
-  const long long wbytes = (taps * a.cb * V * 4 + 15) / 16 * 16;
+  const long long wbytes = (taps * a.cb * 16 + 15) / 16 * 16;
   const long long tail = static_cast<long long>(sizeof(DwTmaTail));
-  t.GW = std::min(4, a.wg);
-  t.TH = std::max(1, std::min(kDwTmaConsumers / (a.cb * t.GW), P.Ho));
+  const int nb = kDwTmaConsumers / a.cb;
+  t.BC = std::max(1, std::min({4, nb, (P.Wo + kDwTmaP - 1) / kDwTmaP}));
+  t.BR = std::max(1, std::min(nb / t.BC, (P.Ho + R - 1) / R));
   while (true) {
-    t.TW = t.GW * kDwP;
+    t.TH = t.BR * R;
+    t.TW = t.BC * kDwTmaP;
     t.span_h = (t.TH - 1) * P.s[1] + (P.kH - 1) * P.d[1] + 1;
     t.span_w = (t.TW - 1) * P.s[2] + (P.kW - 1) * P.d[2] + 1;
-    const long long slab = static_cast<long long>(t.span_h) * t.span_w * a.cb * 16;
+    const long long slab = static_cast<long long>(t.span_h) * t.span_w * a.cb * VB;
     const long long pitch = (slab + 127) / 128 * 128;
     const long long room = budget - wbytes - tail;
     t.stages = room > 0 ? static_cast<int>(std::min<long long>(kDwTmaMaxStages, room / pitch)) : 0;
@@ -835,26 +852,43 @@ int dw_tma_tile(const Problem& P, DwTmaArgs& t, long long budget) {
       t.tail_off = static_cast<uint32_t>(t.w_off + wbytes);
       return CONV_OK;
     }
-    if (t.TH > 1) t.TH = (t.TH + 1) / 2;
-    else if (t.GW > 1) t.GW = (t.GW + 1) / 2;
+    if (t.BR > 1) t.BR = (t.BR + 1) / 2;
+    else if (t.BC > 1) t.BC = (t.BC + 1) / 2;
     else return CONV_EUNSUPPORTED;
   }
 }
 
-int plan_dw_tma(const Problem& P, int sms, DwTmaArgs& t, int& grid, size_t& smem) {
+// Two CTAs share an SM (half the shared memory each) when the form's
+// registers allow it and that leaves them two slabs or more; otherwise one CTA
+// takes it all.  The register form falls back to the generic consumer if its
+// tile does not fit.
+int plan_dw_tma(const Problem& P, int sms, DwTmaArgs& t, int& K, int& S, int& R, int& grid, size_t& smem) {
   if (!dw_fits(P)) return CONV_EUNSUPPORTED;
   std::memset(&t, 0, sizeof(t));
   DwArgs& a = t.d;
   dw_geometry(P, a);
-  const int V = dw_vec(P);
-  const int cvs = P.C / V;
-  t.nct = (cvs + 15) / 16;
+  const int cvs = P.C / 4;  // channel vectors of 4
+  t.nct = (cvs + 31) / 32;
   a.cb = (cvs + t.nct - 1) / t.nct;
+  if (P.esize == 2) a.cb = (a.cb + 1) / 2 * 2;  // 16-byte aligned channel tiles (TMA x coordinate)
+  if ((a.cb * 4 * P.esize) % 16 != 0 || a.cb > 32) return CONV_EUNSUPPORTED;
+  R = dw_tma_form(P, K, S);
   int per_sm = 2;
-  if (dw_tma_tile(P, t, static_cast<long long>(kDwTmaSmem) / 2) != CONV_OK) {
-    per_sm = 1;
-    if (dw_tma_tile(P, t, static_cast<long long>(kDwTmaSmem)) != CONV_OK) return CONV_EUNSUPPORTED;
+  bool fit = false;
+  for (int attempt = 0; attempt < 2 && !fit; ++attempt) {
+    if (attempt == 1) {
+      if (K == 0) break;
+      K = 0; S = 0; R = 1;  // generic consumer
+    }
+    per_sm = dw_tma_ctas_per_sm(K, R);
+    if (per_sm == 2 && dw_tma_tile(P, t, R, static_cast<long long>(kDwTmaSmem) / 2) == CONV_OK) {
+      fit = true;
+    } else if (dw_tma_tile(P, t, R, static_cast<long long>(kDwTmaSmem)) == CONV_OK) {
+      per_sm = 1;
+      fit = true;
+    }
   }
+  if (!fit) return CONV_EUNSUPPORTED;
   t.tiles_h = (P.Ho + t.TH - 1) / t.TH;
   t.tiles_w = (P.Wo + t.TW - 1) / t.TW;
   long long tiles;
@@ -862,7 +896,8 @@ int plan_dw_tma(const Problem& P, int sms, DwTmaArgs& t, int& grid, size_t& smem
     return CONV_EINVAL;
   if (tiles > 0x7fffffffLL) return CONV_EUNSUPPORTED;
   t.tiles = static_cast<int>(tiles);
-  const long long per_ct = std::max<long long>(1, std::min<long long>(static_cast<long long>(sms) * per_sm / t.nct, tiles));
+  const long long per_ct =
+      std::max<long long>(1, std::min<long long>(static_cast<long long>(sms) * per_sm / t.nct, tiles));
   const long long g = per_ct * t.nct;
   if (g > 0x7fffffffLL) return CONV_EUNSUPPORTED;
   grid = static_cast<int>(g);
@@ -883,7 +918,7 @@ int encode_dw_map(const Problem& P, const DwTmaArgs& t, const void* x, CUtensorM
   const cuuint64_t C = P.C, W = P.W, H = P.H, D = P.D;
   cuuint64_t dim[5] = {C, W, H, D, static_cast<cuuint64_t>(P.N)};
   cuuint64_t str[4] = {e * C, e * C * W, e * C * W * H, e * C * W * H * D};
-  cuuint32_t box[5] = {static_cast<cuuint32_t>(t.d.cb * dw_vec(P)), static_cast<cuuint32_t>(t.span_w),
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(t.d.cb * 4), static_cast<cuuint32_t>(t.span_w),
                        static_cast<cuuint32_t>(t.span_h), 1u, 1u};
   cuuint32_t est[5] = {1, 1, 1, 1, 1};
   const CUresult r = drv.tiled(&m, dt, 5, const_cast<void*>(x), dim, str, box, est, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -905,9 +940,9 @@ cudaError_t launch_dw_t(const DwArgs& a, dim3 grid, dim3 block, size_t smem, cud
   return cudaGetLastError();
 }
 
-template <typename T, int V, int KW, int SW, int DW>
+template <typename T, int K, int S, int R>
 cudaError_t launch_dw_tma_t(const CUtensorMap& m, const DwTmaArgs& t, int grid, size_t smem, cudaStream_t st) {
-  auto* k = conv_fwd_dw_tma_kernel<T, V, kDwP, KW, SW, DW>;
+  auto* k = conv_fwd_dw_tma_kernel<T, K, S, R>;
   const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   k<<<grid, kDwTmaThreads, smem, st>>>(m, t);
@@ -927,16 +962,12 @@ cudaError_t launch_dw_shape(const DwArgs& a, dim3 grid, dim3 block, size_t smem,
   return launch_dw_t<T, V, 0, 0, 0>(a, grid, block, smem, st);
 }
 
-template <typename T, int V>
-cudaError_t launch_dw_tma_shape(const CUtensorMap& m, const DwTmaArgs& t, int grid, size_t smem, cudaStream_t st) {
-  const DwArgs& a = t.d;
-  if (a.dw == 1 && a.sw == 1) {
-    if (a.kW == 3) return launch_dw_tma_t<T, V, 3, 1, 1>(m, t, grid, smem, st);
-    if (a.kW == 5) return launch_dw_tma_t<T, V, 5, 1, 1>(m, t, grid, smem, st);
-    if (a.kW == 7) return launch_dw_tma_t<T, V, 7, 1, 1>(m, t, grid, smem, st);
-  }
-  if (a.dw == 1 && a.sw == 2 && a.kW == 3) return launch_dw_tma_t<T, V, 3, 2, 1>(m, t, grid, smem, st);
-  return launch_dw_tma_t<T, V, 0, 0, 0>(m, t, grid, smem, st);
+template <typename T>
+cudaError_t launch_dw_tma_form(const CUtensorMap& m, const DwTmaArgs& t, int K, int S, int grid, size_t smem,
+                               cudaStream_t st) {
+  if (K == 3 && S == 1) return launch_dw_tma_t<T, 3, 1, 4>(m, t, grid, smem, st);
+  if (K == 3 && S == 2) return launch_dw_tma_t<T, 3, 2, 2>(m, t, grid, smem, st);
+  return launch_dw_tma_t<T, 0, 0, 1>(m, t, grid, smem, st);
 }
 
 int launch_dw_direct(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st) {
@@ -955,17 +986,17 @@ int launch_dw_direct(const Problem& P, const void* x, const void* w, void* y, cu
 
 int launch_dw(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st, int sms) {
   DwTmaArgs t;
-  int grid;
+  int grid, K, S, R;
   size_t smem;
-  if (plan_dw_tma(P, sms, t, grid, smem) != CONV_OK) return launch_dw_direct(P, x, w, y, st);
+  if (plan_dw_tma(P, sms, t, K, S, R, grid, smem) != CONV_OK) return launch_dw_direct(P, x, w, y, st);
   t.d.x = x; t.d.w = w; t.d.y = y;
   CUtensorMap m;
   const int rc = encode_dw_map(P, t, x, m);
   if (rc != CONV_OK) return rc;
   cudaError_t e;
-  if (P.dtype == CONV_F32) e = launch_dw_tma_shape<float, 4>(m, t, grid, smem, st);
-  else if (P.dtype == CONV_F16) e = launch_dw_tma_shape<__half, 8>(m, t, grid, smem, st);
-  else e = launch_dw_tma_shape<__nv_bfloat16, 8>(m, t, grid, smem, st);
+  if (P.dtype == CONV_F32) e = launch_dw_tma_form<float>(m, t, K, S, grid, smem, st);
+  else if (P.dtype == CONV_F16) e = launch_dw_tma_form<__half>(m, t, K, S, grid, smem, st);
+  else e = launch_dw_tma_form<__nv_bfloat16>(m, t, K, S, grid, smem, st);
   return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
 
@@ -1476,10 +1507,10 @@ int conv_plan_ex(int N, int D, int H, int W, int C, int O, int kD, int kH, int k
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
   if (variant == CONV_VARIANT_DEPTHWISE || variant == CONV_VARIANT_DEPTHWISE_DIRECT) {
     DwTmaArgs ta;
-    int tgrid;
+    int tgrid, K, S, R;
     size_t smem;
-    if (variant == CONV_VARIANT_DEPTHWISE && plan_dw_tma(P, sms, ta, tgrid, smem) == CONV_OK) {
-      if (bn) *bn = dw_vec(P);  // channels per thread
+    if (variant == CONV_VARIANT_DEPTHWISE && plan_dw_tma(P, sms, ta, K, S, R, tgrid, smem) == CONV_OK) {
+      if (bn) *bn = 4;  // channels per thread
       if (stages) *stages = ta.stages;
       if (ctas) *ctas = tgrid;
       return variant;

@@ -218,15 +218,16 @@ def test_explicit_variant_plan(C):
     with pytest.raises(C.ConvError) as e:
         C.plan(*g3, "f32", C.VARIANT_TC_TMA)
     assert e.value.code == -7
-    # depthwise (groups = C = O) with 16-byte channel vectors, any type; 8
-    # channels per thread for 16-bit types, 4 for f32.  The TMA-staged form
+    # depthwise (groups = C = O) with 16-byte channel vectors, any type.  The
+    # direct form computes 8 channels per thread for 16-bit types, 4 for
+    # f32; the TMA-staged form 4 channels of several pixels.  The TMA-staged form
     # runs persistent CTAs (at most two per SM for each channel tile, the
     # planner assumes 148 SMs without a device) over a ring of 2-4 slabs; the
     # direct form launches one block per 256 (channel vector, pixel group) tasks
     dw = (32, 1, 112, 112, 128, 128, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 128)
     for dt, vec in (("f16", 8), ("bf16", 8), ("f32", 4)):
         v, bn, stages, ctas = C.plan(*dw, dt)
-        assert (v, bn) == (C.VARIANT_DEPTHWISE, vec) and 2 <= stages <= 4 and ctas <= 2 * 148
+        assert (v, bn) == (C.VARIANT_DEPTHWISE, 4) and 2 <= stages <= 4 and ctas <= 2 * 148
         v, bn, stages, ctas = C.plan(*dw, dt, C.VARIANT_DEPTHWISE_DIRECT)
         assert (v, bn, stages) == (C.VARIANT_DEPTHWISE_DIRECT, vec, 1)
         assert ctas == -(-32 * 112 * 28 * (128 // vec) // 256)
@@ -241,7 +242,7 @@ def test_explicit_variant_plan(C):
     # a slab taller than one TMA box allows (5 rows at height dilation 70 span
     # 281 > 256 input rows): DEPTHWISE runs the direct form, one stage
     tall = (1, 1, 200, 32, 16, 16, (1, 5, 3), (1, 1, 1), (0, 140, 1), (1, 70, 1), 16)
-    assert C.plan(*tall, "f16")[:3] == (C.VARIANT_DEPTHWISE, 8, 1)
+    assert C.plan(*tall, "f16")[:3] == (C.VARIANT_DEPTHWISE, 8, 1)  # the direct form's 8 channels
     with pytest.raises(C.ConvError) as e:
         C.plan(*g3, "bf16", 12)
     assert e.value.code == -1
