@@ -243,8 +243,8 @@ __global__ void __launch_bounds__(kDwThreads, 2) conv_fwd_dw_direct_kernel(const
 // output tiles of TH x TW pixels of one (n, od).  A tile's input is, per valid
 // kd, one slab of span_h x span_w pixels x CB channels, which one TMA tiled
 // load brings into shared memory (the hardware zero-fills what lies in the
-// padding).  A producer warp keeps a ring of `stages` slabs ahead of the eight
-// consumer warps (full / empty mbarriers).  CTA b serves channel tile b % nct
+// padding).  A producer warp keeps a ring of `stages` slabs ahead of eight or
+// twelve consumer warps (full / empty mbarriers).  CTA b serves channel tile b % nct
 // and tiles b / nct, b / nct + gridDim.x / nct, ...
 //
 // A consumer thread owns 4 channels (one 8-byte vector for 16-bit types, 16
@@ -253,13 +253,10 @@ __global__ void __launch_bounds__(kDwThreads, 2) conv_fwd_dw_direct_kernel(const
 // a warp is one contiguous run.  The tile is BR x BC blocks (TH = BR*R,
 // TW = BC*P).  Products accumulate in fp32 through packed two-lane FMAs.
 //
-// For square K x K filters with equal strides S and no dilation (K = 3,
-// S = 1 or 2), the K*K weight vectors of the current kd sit in registers and
-// the thread walks the (R-1)*S + K input rows and (P-1)*S + K input columns of
-// its block once each, converting every input vector to fp32 once and
-// applying it to every (output row, output column, tap) that reads it: the
-// pairing is resolved at compile time.  Any other filter runs the generic
-// consumer (R = 1, runtime taps, one slab read per (column, tap)).
+// The consumer forms (kDwSquare, kDwRows, kDwGeneric below) differ in how
+// much of the filter sits in registers; in the first two, each input vector a
+// thread reads is converted to fp32 once and applied to every (output row,
+// output column, tap) that uses it, the pairing resolved at compile time.
 
 struct DwTmaArgs {
   DwArgs d;              // geometry; d.cb = channel vectors (of 4) per tile
@@ -277,8 +274,6 @@ struct DwTmaArgs {
   unsigned long long timeout_ns;
 };
 
-constexpr int kDwTmaConsumers = 256;                 // eight warps
-constexpr int kDwTmaThreads = kDwTmaConsumers + 32;  // and one producer warp
 constexpr int kDwTmaMaxStages = 4;
 constexpr int kDwTmaP = 4;                           // output columns per block
 
@@ -392,14 +387,27 @@ __device__ __forceinline__ void dw_fma4(float2 (&acc)[2], const float2 (&x)[2], 
   acc[1] = __ffma2_rn(x[1], w[1], acc[1]);
 }
 
-// CTAs per SM a form is compiled for: the register forms need more than half
-// an SM's registers per thread (32-64 accumulators and 36 weights).
-constexpr int dw_tma_ctas_per_sm(int K, int R) { return K > 0 && R >= 1 ? 1 : 2; }
+// Consumer forms.
+//   kDwSquare: K x K filters (K = 3) at width and height stride S, no
+//     dilation; all K*K weight vectors of the current kd in registers, blocks
+//     of R output rows, every input vector of a block read and converted once.
+//   kDwRows: filter width K (5 or 7) at width stride S, no width dilation,
+//     any height; one filter row's K weight vectors in registers at a time,
+//     R = 1, every input vector of a block row read once per filter row.
+//   kDwGeneric: any filter; one slab read per (column, tap).
+constexpr int kDwGeneric = 0, kDwSquare = 1, kDwRows = 2;
 
-// K > 0: the register-resident K x K / stride S consumer with R output rows
-// per block; K = 0: the generic consumer (R = 1).
-template <typename T, int K, int S, int R>
-__global__ void __launch_bounds__(kDwTmaThreads, dw_tma_ctas_per_sm(K, R))
+// CTAs per SM a form is compiled for: the square form (36 weights and 16-64
+// accumulators a thread) needs more than half an SM's registers; with twelve
+// consumer warps (13 with the producer: at most 4 on each of the SM's four
+// schedulers) the limit is 128 registers a thread.  The other forms run two
+// CTAs of eight consumer warps.
+constexpr int dw_tma_ctas_per_sm(int MODE, int R, int NCW) { return MODE == kDwSquare ? 1 : 2; }
+
+// MODE: consumer form; K, S: its filter width and stride (0 for the generic
+// form); R: output rows per block; NCW: consumer warps (warp NCW produces).
+template <typename T, int MODE, int K, int S, int R, int NCW>
+__global__ void __launch_bounds__(32 * (NCW + 1), dw_tma_ctas_per_sm(MODE, R, NCW))
     conv_fwd_dw_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, const DwTmaArgs a) {
   constexpr int P = kDwTmaP;
   constexpr int VB = 4 * static_cast<int>(sizeof(T));  // bytes per channel vector
@@ -416,18 +424,18 @@ __global__ void __launch_bounds__(kDwTmaThreads, dw_tma_ctas_per_sm(K, R))
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
       ptx::mbar_init(ptx::smem_u32(&tail->full[s]), 1u);
-      ptx::mbar_init(ptx::smem_u32(&tail->empty[s]), kDwTmaConsumers / 32);
+      ptx::mbar_init(ptx::smem_u32(&tail->empty[s]), NCW);
     }
     tail->abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == kDwTmaConsumers / 32 && lane == 0) ptx::prefetch_tmap(&tmap_x);
+  if (warp == NCW && lane == 0) ptx::prefetch_tmap(&tmap_x);
   const int ct = static_cast<int>(blockIdx.x) % a.nct;
   const int t_first = static_cast<int>(blockIdx.x) / a.nct, t_step = static_cast<int>(gridDim.x) / a.nct;
-  dw_fill_filters<T, 4>(s_w, g, ct, taps, static_cast<int>(threadIdx.x), kDwTmaThreads);
+  dw_fill_filters<T, 4>(s_w, g, ct, taps, static_cast<int>(threadIdx.x), 32 * (NCW + 1));
   __syncthreads();
 
-  if (warp == kDwTmaConsumers / 32) {
+  if (warp == NCW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
@@ -480,7 +488,7 @@ __global__ void __launch_bounds__(kDwTmaThreads, dw_tma_ctas_per_sm(K, R))
   const float* wbase = s_w + cv * 4;
 
   // register-resident weights of the current kd (square filters)
-  float2 wreg[K > 0 ? K : 1][K > 0 ? K : 1][2];
+  float2 wreg[MODE == kDwSquare ? K : 1][MODE == kDwSquare ? K : 1][2];
   int wkd = -1;
 
   int stage = 0;
@@ -500,7 +508,7 @@ __global__ void __launch_bounds__(kDwTmaThreads, dw_tma_ctas_per_sm(K, R))
         return;
       if (active) {
         const uint8_t* slab = slabs + static_cast<size_t>(stage) * a.slab_pitch + static_cast<uint32_t>(cv) * VB;
-        if constexpr (K > 0) {
+        if constexpr (MODE == kDwSquare) {
           if (kd != wkd) {
 #pragma unroll
             for (int kh = 0; kh < K; ++kh)
@@ -528,6 +536,25 @@ __global__ void __launch_bounds__(kDwTmaThreads, dw_tma_ctas_per_sm(K, R))
                       for (int kw = 0; kw < K; ++kw)
                         if (p * S + kw == j) dw_fma4(acc[rr][p], xf, wreg[kh][kw]);
                   }
+            }
+          }
+        } else if constexpr (MODE == kDwRows) {
+          constexpr int SPAN = (P - 1) * S + K;
+          const uint8_t* bp = slab + static_cast<uint32_t>(br * g.sh) * rowb + static_cast<uint32_t>(bc * P * S) * colb;
+          for (int kh = 0; kh < g.kH; ++kh) {
+            const uint8_t* rowp = bp + static_cast<uint32_t>(kh * g.dh) * rowb;
+            float2 wv[K][2];
+#pragma unroll
+            for (int kw = 0; kw < K; ++kw) dw_wload4(wbase + ((kd * g.kH + kh) * K + kw) * cb * 4, wv[kw]);
+#pragma unroll
+            for (int j = 0; j < SPAN; ++j) {
+              float2 xf[2];
+              dw_load4<T>(rowp + static_cast<uint32_t>(j) * colb, xf);
+#pragma unroll
+              for (int p = 0; p < P; ++p)
+#pragma unroll
+                for (int kw = 0; kw < K; ++kw)
+                  if (p * S + kw == j) dw_fma4(acc[0][p], xf, wv[kw]);
             }
           }
         } else {

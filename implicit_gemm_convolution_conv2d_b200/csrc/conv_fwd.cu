@@ -806,34 +806,39 @@ int plan_dw(const Problem& P, DwArgs& a, dim3& grid, dim3& block, size_t& smem) 
   return CONV_OK;
 }
 
-// Consumer form of the TMA-staged kernel: 3x3 filters at equal strides 1 or
-// 2 without dilation keep their weights in registers and compute blocks of R
-// output rows (R = 4 at stride 1, 2 at stride 2); anything else runs the
-// generic consumer (K = 0, R = 1).
-int dw_tma_form(const Problem& P, int& K, int& S) {
-  if (P.kH == 3 && P.kW == 3 && P.s[1] == P.s[2] && (P.s[1] == 1 || P.s[1] == 2) && P.d[1] == 1 &&
-      P.d[2] == 1) {
-    K = 3;
-    S = P.s[1];
-    return S == 1 ? 4 : 2;
+// Consumer form of the TMA-staged kernel (the shapes measured fastest on
+// B200 with each): 3x3 filters at equal strides 1 or 2 without dilation keep
+// all nine weights in registers (16-bit types: four-row blocks at stride 1,
+// two at stride 2, eight consumer warps; f32: two / one rows, twelve warps);
+// 5- or 7-wide filters at width stride 1 or 2 without width dilation stream
+// filter rows; anything else runs the generic consumer.
+struct DwForm {
+  int mode, K, S, R, ncw;
+};
+
+DwForm dw_tma_form(const Problem& P) {
+  const bool w_plain = P.d[2] == 1 && (P.s[2] == 1 || P.s[2] == 2);
+  if (P.kH == 3 && P.kW == 3 && P.s[1] == P.s[2] && P.d[1] == 1 && w_plain) {
+    const bool s1 = P.s[1] == 1;
+    if (P.esize == 2) return {kDwSquare, 3, P.s[1], s1 ? 4 : 2, 8};
+    return {kDwSquare, 3, P.s[1], s1 ? 2 : 1, 12};
   }
-  K = 0;
-  S = 0;
-  return 1;
+  if ((P.kW == 5 || P.kW == 7) && w_plain) return {kDwRows, P.kW, P.s[2], 1, 8};
+  return {kDwGeneric, 0, 0, 1, 8};
 }
 
 // Tile of the TMA-staged form: the consumer threads are cb channel vectors x
-// BR x BC blocks of R x 4 output pixels (BC = 4 blocks across, BR to fill 256
-// threads, no more rows than the output has); block rows, then columns,
+// BR x BC blocks of R x 4 output pixels (BC = 4 blocks across, BR to fill the
+// consumer threads, no more rows than the output has); block rows, then columns,
 // halved until the slab box fits TMA's 256-element box limit and two slabs
 // fit beside the filters in `budget` bytes.
-int dw_tma_tile(const Problem& P, DwTmaArgs& t, int R, long long budget) {
+int dw_tma_tile(const Problem& P, DwTmaArgs& t, int R, int consumers, long long budget) {
   DwArgs& a = t.d;
   const long long VB = 4LL * P.esize;
   const long long taps = static_cast<long long>(P.kD) * P.kH * P.kW;
   const long long wbytes = (taps * a.cb * 16 + 15) / 16 * 16;
   const long long tail = static_cast<long long>(sizeof(DwTmaTail));
-  const int nb = kDwTmaConsumers / a.cb;
+  const int nb = consumers / a.cb;
   t.BC = std::max(1, std::min({4, nb, (P.Wo + kDwTmaP - 1) / kDwTmaP}));
   t.BR = std::max(1, std::min(nb / t.BC, (P.Ho + R - 1) / R));
   while (true) {
@@ -860,9 +865,9 @@ int dw_tma_tile(const Problem& P, DwTmaArgs& t, int R, long long budget) {
 
 // Two CTAs share an SM (half the shared memory each) when the form's
 // registers allow it and that leaves them two slabs or more; otherwise one CTA
-// takes it all.  The register form falls back to the generic consumer if its
+// takes it all.  A specialised form falls back to the generic consumer if its
 // tile does not fit.
-int plan_dw_tma(const Problem& P, int sms, DwTmaArgs& t, int& K, int& S, int& R, int& grid, size_t& smem) {
+int plan_dw_tma(const Problem& P, int sms, DwTmaArgs& t, DwForm& f, int& grid, size_t& smem) {
   if (!dw_fits(P)) return CONV_EUNSUPPORTED;
   std::memset(&t, 0, sizeof(t));
   DwArgs& a = t.d;
@@ -872,18 +877,19 @@ int plan_dw_tma(const Problem& P, int sms, DwTmaArgs& t, int& K, int& S, int& R,
   a.cb = (cvs + t.nct - 1) / t.nct;
   if (P.esize == 2) a.cb = (a.cb + 1) / 2 * 2;  // 16-byte aligned channel tiles (TMA x coordinate)
   if ((a.cb * 4 * P.esize) % 16 != 0 || a.cb > 32) return CONV_EUNSUPPORTED;
-  R = dw_tma_form(P, K, S);
+  f = dw_tma_form(P);
   int per_sm = 2;
   bool fit = false;
   for (int attempt = 0; attempt < 2 && !fit; ++attempt) {
     if (attempt == 1) {
-      if (K == 0) break;
-      K = 0; S = 0; R = 1;  // generic consumer
+      if (f.mode == kDwGeneric) break;
+      f = {kDwGeneric, 0, 0, 1, 8};
     }
-    per_sm = dw_tma_ctas_per_sm(K, R);
-    if (per_sm == 2 && dw_tma_tile(P, t, R, static_cast<long long>(kDwTmaSmem) / 2) == CONV_OK) {
+    per_sm = dw_tma_ctas_per_sm(f.mode, f.R, f.ncw);
+    const int consumers = 32 * f.ncw;
+    if (per_sm == 2 && dw_tma_tile(P, t, f.R, consumers, static_cast<long long>(kDwTmaSmem) / 2) == CONV_OK) {
       fit = true;
-    } else if (dw_tma_tile(P, t, R, static_cast<long long>(kDwTmaSmem)) == CONV_OK) {
+    } else if (dw_tma_tile(P, t, f.R, consumers, static_cast<long long>(kDwTmaSmem)) == CONV_OK) {
       per_sm = 1;
       fit = true;
     }
@@ -929,23 +935,38 @@ int encode_dw_map(const Problem& P, const DwTmaArgs& t, const void* x, CUtensorM
   return CONV_OK;
 }
 
+// Raises a kernel's dynamic shared-memory limit to the 227 KB maximum once
+// per device (bit `dev` of `done`; devices beyond 63 set it every launch).
+template <typename Kern>
+cudaError_t dw_smem_attr(Kern* k, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 63;
+  const uint64_t bit = dev < 63 ? (1ull << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
+
 template <typename T, int V, int KW, int SW, int DW>
 cudaError_t launch_dw_t(const DwArgs& a, dim3 grid, dim3 block, size_t smem, cudaStream_t st) {
+  static std::atomic<uint64_t> attr_done{0};
   auto* k = conv_fwd_dw_direct_kernel<T, V, kDwP, KW, SW, DW>;
   if (smem > 48 * 1024) {
-    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    const cudaError_t e = dw_smem_attr(k, attr_done);
     if (e != cudaSuccess) return e;
   }
   k<<<grid, block, smem, st>>>(a);
   return cudaGetLastError();
 }
 
-template <typename T, int K, int S, int R>
+template <typename T, int MODE, int K, int S, int R, int NCW>
 cudaError_t launch_dw_tma_t(const CUtensorMap& m, const DwTmaArgs& t, int grid, size_t smem, cudaStream_t st) {
-  auto* k = conv_fwd_dw_tma_kernel<T, K, S, R>;
-  const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  static std::atomic<uint64_t> attr_done{0};
+  auto* k = conv_fwd_dw_tma_kernel<T, MODE, K, S, R, NCW>;
+  const cudaError_t e = dw_smem_attr(k, attr_done);
   if (e != cudaSuccess) return e;
-  k<<<grid, kDwTmaThreads, smem, st>>>(m, t);
+  k<<<grid, 32 * (NCW + 1), smem, st>>>(m, t);
   return cudaGetLastError();
 }
 
@@ -962,12 +983,23 @@ cudaError_t launch_dw_shape(const DwArgs& a, dim3 grid, dim3 block, size_t smem,
   return launch_dw_t<T, V, 0, 0, 0>(a, grid, block, smem, st);
 }
 
+// One instantiation per form dw_tma_form returns (16-bit and f32 square
+// forms differ in rows and warps).
 template <typename T>
-cudaError_t launch_dw_tma_form(const CUtensorMap& m, const DwTmaArgs& t, int K, int S, int grid, size_t smem,
+cudaError_t launch_dw_tma_form(const CUtensorMap& m, const DwTmaArgs& t, const DwForm& f, int grid, size_t smem,
                                cudaStream_t st) {
-  if (K == 3 && S == 1) return launch_dw_tma_t<T, 3, 1, 4>(m, t, grid, smem, st);
-  if (K == 3 && S == 2) return launch_dw_tma_t<T, 3, 2, 2>(m, t, grid, smem, st);
-  return launch_dw_tma_t<T, 0, 0, 1>(m, t, grid, smem, st);
+  constexpr bool h = sizeof(T) == 2;
+  if (f.mode == kDwSquare && f.S == 1)
+    return launch_dw_tma_t<T, kDwSquare, 3, 1, h ? 4 : 2, h ? 8 : 12>(m, t, grid, smem, st);
+  if (f.mode == kDwSquare && f.S == 2)
+    return launch_dw_tma_t<T, kDwSquare, 3, 2, h ? 2 : 1, h ? 8 : 12>(m, t, grid, smem, st);
+  if (f.mode == kDwRows) {
+    if (f.K == 5 && f.S == 1) return launch_dw_tma_t<T, kDwRows, 5, 1, 1, 8>(m, t, grid, smem, st);
+    if (f.K == 5 && f.S == 2) return launch_dw_tma_t<T, kDwRows, 5, 2, 1, 8>(m, t, grid, smem, st);
+    if (f.K == 7 && f.S == 1) return launch_dw_tma_t<T, kDwRows, 7, 1, 1, 8>(m, t, grid, smem, st);
+    if (f.K == 7 && f.S == 2) return launch_dw_tma_t<T, kDwRows, 7, 2, 1, 8>(m, t, grid, smem, st);
+  }
+  return launch_dw_tma_t<T, kDwGeneric, 0, 0, 1, 8>(m, t, grid, smem, st);
 }
 
 int launch_dw_direct(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st) {
@@ -986,17 +1018,18 @@ int launch_dw_direct(const Problem& P, const void* x, const void* w, void* y, cu
 
 int launch_dw(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st, int sms) {
   DwTmaArgs t;
-  int grid, K, S, R;
+  DwForm f;
+  int grid;
   size_t smem;
-  if (plan_dw_tma(P, sms, t, K, S, R, grid, smem) != CONV_OK) return launch_dw_direct(P, x, w, y, st);
+  if (plan_dw_tma(P, sms, t, f, grid, smem) != CONV_OK) return launch_dw_direct(P, x, w, y, st);
   t.d.x = x; t.d.w = w; t.d.y = y;
   CUtensorMap m;
   const int rc = encode_dw_map(P, t, x, m);
   if (rc != CONV_OK) return rc;
   cudaError_t e;
-  if (P.dtype == CONV_F32) e = launch_dw_tma_form<float>(m, t, K, S, grid, smem, st);
-  else if (P.dtype == CONV_F16) e = launch_dw_tma_form<__half>(m, t, K, S, grid, smem, st);
-  else e = launch_dw_tma_form<__nv_bfloat16>(m, t, K, S, grid, smem, st);
+  if (P.dtype == CONV_F32) e = launch_dw_tma_form<float>(m, t, f, grid, smem, st);
+  else if (P.dtype == CONV_F16) e = launch_dw_tma_form<__half>(m, t, f, grid, smem, st);
+  else e = launch_dw_tma_form<__nv_bfloat16>(m, t, f, grid, smem, st);
   return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
 
@@ -1507,9 +1540,10 @@ int conv_plan_ex(int N, int D, int H, int W, int C, int O, int kD, int kH, int k
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
   if (variant == CONV_VARIANT_DEPTHWISE || variant == CONV_VARIANT_DEPTHWISE_DIRECT) {
     DwTmaArgs ta;
-    int tgrid, K, S, R;
+    DwForm f;
+    int tgrid;
     size_t smem;
-    if (variant == CONV_VARIANT_DEPTHWISE && plan_dw_tma(P, sms, ta, K, S, R, tgrid, smem) == CONV_OK) {
+    if (variant == CONV_VARIANT_DEPTHWISE && plan_dw_tma(P, sms, ta, f, tgrid, smem) == CONV_OK) {
       if (bn) *bn = 4;  // channels per thread
       if (stages) *stages = ta.stages;
       if (ctas) *ctas = tgrid;

@@ -179,6 +179,12 @@ SMALL = [
     WL.case(2, 1, 9, 21, 200, 200, (1, 3, 3), pad=(0, 1, 1), groups=200, name="dw_c200_partial_ctile"),
     WL.case(1, 3, 5, 6, 8, 8, (3, 3, 3), (2, 1, 1), (3, 1, 1), groups=8, name="dw_3d_empty_planes"),
     WL.case(1, 1, 200, 32, 16, 16, (1, 5, 3), pad=(0, 140, 1), dil=(1, 70, 1), groups=16, name="dw_tall_slab"),
+    # filter-row streaming form (5- and 7-wide filters): stride 1, height
+    # dilation, a 3-D filter one row high
+    WL.case(2, 1, 13, 21, 32, 32, (1, 5, 5), pad=(0, 2, 2), groups=32, name="dw_k5_rows"),
+    WL.case(1, 1, 17, 19, 16, 16, (1, 5, 5), pad=(0, 4, 2), dil=(1, 2, 1), groups=16, name="dw_k5_dil_h"),
+    WL.case(1, 4, 6, 11, 16, 16, (3, 1, 5), pad=(1, 0, 2), groups=16, name="dw_3d_k315"),
+    WL.case(1, 1, 15, 30, 24, 24, (1, 7, 7), (1, 2, 2), (0, 3, 3), groups=24, name="dw_k7_s2"),
 ]
 
 
