@@ -13,6 +13,9 @@ kernel", section 5's variants table) and groups (same table), in the
 channels-last layouts of section 7 and of the MLX conv3d pull request's
 benchmark table: x (N, D, H, W, C), w (O, kD, kH, kW, C/groups).
 
+The same file holds the transposed ("upsampling") convolution of the same
+page's variants table, read as the adjoint of the forward pass.
+
 Every function here is pinned by ``tests/test_oracle_pins.py`` against things
 other than itself: the tutorial's worked example, its printed FLOP and byte
 counts, closed forms (delta kernels, constant inputs), invariants (linearity,
@@ -78,6 +81,16 @@ class Oracle:
         lib.oracle_conv_fwd_points_ex.restype = ctypes.c_int
         lib.oracle_out_dims_ex.argtypes = [ctypes.c_int] * 6 + [i3, i3, i3, i3, i3]
         lib.oracle_out_dims_ex.restype = ctypes.c_int
+        # transposed convolution: ..., stride, pad, out_pad, dil, groups
+        common_t = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int] + [ctypes.c_int] * 9 + \
+            [i3, i3, i3, i3, ctypes.c_int]
+        lib.oracle_conv_transpose.argtypes = common_t + [dp, dp]
+        lib.oracle_conv_transpose.restype = ctypes.c_int
+        lib.oracle_conv_transpose_points.argtypes = common_t + [ctypes.POINTER(ctypes.c_int64), ctypes.c_int64,
+                                                                dp, dp]
+        lib.oracle_conv_transpose_points.restype = ctypes.c_int
+        lib.oracle_convT_out_dims.argtypes = [ctypes.c_int] * 6 + [i3, i3, i3, i3, i3]
+        lib.oracle_convT_out_dims.restype = ctypes.c_int
         lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
         lib.oracle_f16_to_f64.restype = ctypes.c_double
         lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
@@ -152,6 +165,64 @@ class Oracle:
         return y, s
 
 
+    def convT_out_dims(self, D, H, W, kD, kH, kW, stride, pad, out_pad, dil):
+        """Transposed-convolution extents: (I-1)*s - 2p + d*(k-1) + 1 + op per dimension."""
+        out = (ctypes.c_int * 3)()
+        rc = self.lib.oracle_convT_out_dims(D, H, W, kD, kH, kW, _i3(stride), _i3(pad), _i3(out_pad), _i3(dil),
+                                            out)
+        if rc:
+            raise ValueError("oracle.convT_out_dims: invalid geometry")
+        return tuple(out)
+
+    def conv_transpose(self, x, w, stride=(1, 1, 1), pad=(0, 0, 0), out_pad=(0, 0, 0), dil=(1, 1, 1), groups=1):
+        """Full output of the transposed convolution (the adjoint of conv_fwd with
+        the same weights).
+
+        x: [N, D, H, W, Cin] and w: [Cin, kD, kH, kW, Cout/groups] CPU tensors of
+        one dtype.  Returns (y, S) float64 arrays of shape [N, Qd, Qh, Qw, Cout].
+        """
+        px, nx, kx = _raw(x)
+        pw, nw, kw_ = _raw(w)
+        if nx != nw:
+            raise TypeError("oracle: x and w must share a dtype")
+        N, D, H, W, Cin = (int(v) for v in kx.shape)
+        Ci, kD, kH, kW, Cog = (int(v) for v in kw_.shape)
+        if Ci != Cin:
+            raise ValueError("oracle: w's first dimension must be x's channel count")
+        Cout = Cog * groups
+        Q = self.convT_out_dims(D, H, W, kD, kH, kW, stride, pad, out_pad, dil)
+        y = np.empty((N, *Q, Cout), dtype=np.float64)
+        s = np.empty_like(y)
+        dp = ctypes.POINTER(ctypes.c_double)
+        rc = self.lib.oracle_conv_transpose(px, pw, DTYPE_CODE[nx], N, D, H, W, Cin, Cout, kD, kH, kW,
+                                            _i3(stride), _i3(pad), _i3(out_pad), _i3(dil), int(groups),
+                                            y.ctypes.data_as(dp), s.ctypes.data_as(dp))
+        if rc:
+            raise ValueError(f"oracle.conv_transpose failed ({rc})")
+        return y, s
+
+    def conv_transpose_points(self, x, w, idx, stride=(1, 1, 1), pad=(0, 0, 0), out_pad=(0, 0, 0),
+                              dil=(1, 1, 1), groups=1):
+        """Selected outputs of the transposed convolution (flat indices into [N, Qd, Qh, Qw, Cout])."""
+        px, nx, kx = _raw(x)
+        pw, nw, kw_ = _raw(w)
+        if nx != nw:
+            raise TypeError("oracle: x and w must share a dtype")
+        N, D, H, W, Cin = (int(v) for v in kx.shape)
+        _, kD, kH, kW, Cog = (int(v) for v in kw_.shape)
+        idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int64).ravel())
+        y = np.empty(idx.shape[0], dtype=np.float64)
+        s = np.empty_like(y)
+        dp = ctypes.POINTER(ctypes.c_double)
+        rc = self.lib.oracle_conv_transpose_points(px, pw, DTYPE_CODE[nx], N, D, H, W, Cin, Cog * groups, kD, kH,
+                                                   kW, _i3(stride), _i3(pad), _i3(out_pad), _i3(dil), int(groups),
+                                                   idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                                   idx.shape[0], y.ctypes.data_as(dp), s.ctypes.data_as(dp))
+        if rc:
+            raise ValueError(f"oracle.conv_transpose_points failed ({rc})")
+        return y, s
+
+
 _default = None
 
 
@@ -205,6 +276,20 @@ def conv_fwd_points(x, w, idx, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), g
     return default().conv_fwd_points(x, w, idx, stride, pad, dil, groups, pad_hi, flip)
 
 
+def convT_out_dims(D, H, W, kD, kH, kW, stride, pad, out_pad, dil):
+    return default().convT_out_dims(D, H, W, kD, kH, kW, stride, pad, out_pad, dil)
+
+
+def conv_transpose(x, w, stride=(1, 1, 1), pad=(0, 0, 0), out_pad=(0, 0, 0), dil=(1, 1, 1), groups=1):
+    return default().conv_transpose(x, w, stride, pad, out_pad, dil, groups)
+
+
+def conv_transpose_points(x, w, idx, stride=(1, 1, 1), pad=(0, 0, 0), out_pad=(0, 0, 0), dil=(1, 1, 1),
+                          groups=1):
+    return default().conv_transpose_points(x, w, idx, stride, pad, out_pad, dil, groups)
+
+
+conv_transpose.__doc__ = Oracle.conv_transpose.__doc__
 conv_fwd.__doc__ = Oracle.conv_fwd.__doc__
 conv_fwd_points.__doc__ = Oracle.conv_fwd_points.__doc__
 out_dims.__doc__ = Oracle.out_dims.__doc__

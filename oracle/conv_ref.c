@@ -349,6 +349,196 @@ int oracle_conv_fwd_points(const void* x, const void* w, int dtype, int N,
                                    y, s);
 }
 
+/* ---- transposed convolution ----------------------------------------------
+ *
+ * "Convolutions" tutorial, "Convolution variants worth knowing": the
+ * transposed ("upsampling") convolution of decoders and diffusion models.  The
+ * page gives no formula; its plainest reading, and the one every framework
+ * uses, is the adjoint of the forward pass above: with the same weight tensor
+ * w[Cin, kD, kH, kW, Cout/G] (the forward pass's [O, k, C/G] with O = Cin
+ * input and C = Cout output channels), every input element x[n, i, ci]
+ * scatters x * w[ci, k, c] onto the output position q = i*s - p + k*d:
+ *
+ *   y[n, q, g*Cog + c] = sum over taps k and input channels ci of group g
+ *                        with q = i*s - p + k*d, 0 <= i < I, of
+ *                        x[n, i, ci] * w[ci, k, c]          (per dimension)
+ *
+ * where Cog = Cout/G and group g holds input channels [g*Cin/G, (g+1)*Cin/G).
+ * Output extent per dimension: (I-1)*s - 2p + d*(k-1) + 1 + op, op (the
+ * output padding) in [0, max(s, d)) extending the high end.  Written here as
+ * a sum per output element: the i that reach q through tap k are those with
+ * q + p - k*d divisible by s.
+ */
+
+static int64_t extent_t(int64_t in, int k, int s, int p, int op, int d) {
+  return (in - 1) * s - 2 * (int64_t)p + (int64_t)d * (k - 1) + 1 + op;
+}
+
+int oracle_convT_out_dims(int D, int H, int W, int kD, int kH, int kW,
+                          const int stride[3], const int pad[3],
+                          const int out_pad[3], const int dil[3], int out[3]) {
+  const int in[3] = {D, H, W};
+  const int k[3] = {kD, kH, kW};
+  for (int i = 0; i < 3; ++i) {
+    if (in[i] <= 0 || k[i] <= 0 || stride[i] <= 0 || dil[i] <= 0 ||
+        pad[i] < 0 || out_pad[i] < 0)
+      return -1;
+    if (out_pad[i] >= stride[i] && out_pad[i] >= dil[i]) return -1;
+    int64_t e = extent_t(in[i], k[i], stride[i], pad[i], out_pad[i], dil[i]);
+    if (e <= 0 || e > 0x7fffffff) return -1;
+    out[i] = (int)e;
+  }
+  return 0;
+}
+
+typedef struct {
+  int N, D, H, W, Ci, Co, kD, kH, kW, G;
+  int Qd, Qh, Qw;
+  int s[3], p[3], d[3];
+} tshape_t;
+
+static int make_tshape(tshape_t* t, int N, int D, int H, int W, int Cin,
+                       int Cout, int kD, int kH, int kW, const int stride[3],
+                       const int pad[3], const int out_pad[3],
+                       const int dil[3], int groups) {
+  int out[3];
+  if (N <= 0 || Cin <= 0 || Cout <= 0 || groups <= 0) return -1;
+  if (Cin % groups || Cout % groups) return -1;
+  if (oracle_convT_out_dims(D, H, W, kD, kH, kW, stride, pad, out_pad, dil,
+                            out))
+    return -1;
+  t->N = N; t->D = D; t->H = H; t->W = W; t->Ci = Cin; t->Co = Cout;
+  t->kD = kD; t->kH = kH; t->kW = kW; t->G = groups;
+  t->Qd = out[0]; t->Qh = out[1]; t->Qw = out[2];
+  for (int i = 0; i < 3; ++i) {
+    t->s[i] = stride[i]; t->p[i] = pad[i]; t->d[i] = dil[i];
+  }
+  return 0;
+}
+
+/* The input index i that reaches output q through tap k, or -1. */
+static int64_t src_index(int64_t q, int k, int s, int p, int d, int64_t in) {
+  int64_t num = q + p - (int64_t)k * d;
+  if (num < 0 || num % s) return -1;
+  num /= s;
+  return num < in ? num : -1;
+}
+
+#define ORACLE_TPOINT_BODY(XAT, WAT)                                         \
+  do {                                                                       \
+    const int Cig = t->Ci / t->G, Cog = t->Co / t->G;                        \
+    const int g = c / Cog, cl = c - g * Cog;                                 \
+    double acc = 0.0, mag = 0.0;                                             \
+    for (int kd = 0; kd < t->kD; ++kd) {                                     \
+      int64_t id = src_index(qd, kd, t->s[0], t->p[0], t->d[0], t->D);       \
+      if (id < 0) continue;                                                  \
+      for (int kh = 0; kh < t->kH; ++kh) {                                   \
+        int64_t ih = src_index(qh, kh, t->s[1], t->p[1], t->d[1], t->H);     \
+        if (ih < 0) continue;                                                \
+        for (int kw = 0; kw < t->kW; ++kw) {                                 \
+          int64_t iw = src_index(qw, kw, t->s[2], t->p[2], t->d[2], t->W);   \
+          if (iw < 0) continue;                                              \
+          int64_t xb = ((((int64_t)n * t->D + id) * t->H + ih) * t->W + iw)  \
+                       * t->Ci + (int64_t)g * Cig;                           \
+          for (int ci = 0; ci < Cig; ++ci) {                                 \
+            int64_t wi = (((((int64_t)g * Cig + ci) * t->kD + kd) * t->kH + kh) \
+                          * t->kW + kw) * Cog + cl;                          \
+            double v = XAT(xb + ci) * WAT(wi);                               \
+            acc += v;                                                        \
+            mag += fabs(v);                                                  \
+          }                                                                  \
+        }                                                                    \
+      }                                                                      \
+    }                                                                        \
+    *py = acc;                                                               \
+    *ps = mag;                                                               \
+  } while (0)
+
+static void tpoint_f64(const tshape_t* t, const double* x, const double* w,
+                       int n, int qd, int qh, int qw, int c, double* py,
+                       double* ps) {
+#define XD(i) x[i]
+#define WD(i) w[i]
+  ORACLE_TPOINT_BODY(XD, WD);
+#undef XD
+#undef WD
+}
+
+static void tpoint_raw(const tshape_t* t, const void* x, const void* w,
+                       int dtype, int n, int qd, int qh, int qw, int c,
+                       double* py, double* ps) {
+#define XR(i) load_elem(x, i, dtype)
+#define WR(i) load_elem(w, i, dtype)
+  ORACLE_TPOINT_BODY(XR, WR);
+#undef XR
+#undef WR
+}
+
+/* Full output of the transposed convolution.  x: [N,D,H,W,Cin]; w:
+ * [Cin,kD,kH,kW,Cout/G]; y and s: [N,Qd,Qh,Qw,Cout] doubles.  Returns 0, -1
+ * (shape), -2 (dtype) or -3 (out of host memory). */
+int oracle_conv_transpose(const void* x, const void* w, int dtype, int N,
+                          int D, int H, int W, int Cin, int Cout, int kD,
+                          int kH, int kW, const int stride[3],
+                          const int pad[3], const int out_pad[3],
+                          const int dil[3], int groups, double* y, double* s) {
+  tshape_t ts;
+  if (dtype < 0 || dtype > 2) return -2;
+  if (make_tshape(&ts, N, D, H, W, Cin, Cout, kD, kH, kW, stride, pad, out_pad,
+                  dil, groups))
+    return -1;
+  int64_t nx = (int64_t)N * D * H * W * Cin;
+  int64_t nw = (int64_t)Cin * kD * kH * kW * (Cout / groups);
+  double* xd = decode_all(x, nx, dtype);
+  double* wd = decode_all(w, nw, dtype);
+  if (!xd || !wd) { free(xd); free(wd); return -3; }
+  const tshape_t* t = &ts;
+#pragma omp parallel for collapse(3) schedule(dynamic, 1)
+  for (int n = 0; n < ts.N; ++n)
+    for (int qd = 0; qd < ts.Qd; ++qd)
+      for (int qh = 0; qh < ts.Qh; ++qh)
+        for (int qw = 0; qw < t->Qw; ++qw)
+          for (int c = 0; c < t->Co; ++c) {
+            int64_t q = ((((int64_t)n * t->Qd + qd) * t->Qh + qh) * t->Qw + qw)
+                        * t->Co + c;
+            tpoint_f64(t, xd, wd, n, qd, qh, qw, c, &y[q], &s[q]);
+          }
+  free(xd);
+  free(wd);
+  return 0;
+}
+
+/* Selected outputs (flat indices into [N,Qd,Qh,Qw,Cout]), read in the storage
+ * type.  Returns 0, -1, -2 or -4 (an index out of range). */
+int oracle_conv_transpose_points(const void* x, const void* w, int dtype,
+                                 int N, int D, int H, int W, int Cin, int Cout,
+                                 int kD, int kH, int kW, const int stride[3],
+                                 const int pad[3], const int out_pad[3],
+                                 const int dil[3], int groups,
+                                 const int64_t* idx, int64_t npts, double* y,
+                                 double* s) {
+  tshape_t ts;
+  if (dtype < 0 || dtype > 2) return -2;
+  if (make_tshape(&ts, N, D, H, W, Cin, Cout, kD, kH, kW, stride, pad, out_pad,
+                  dil, groups))
+    return -1;
+  int64_t total = (int64_t)ts.N * ts.Qd * ts.Qh * ts.Qw * ts.Co;
+  for (int64_t i = 0; i < npts; ++i)
+    if (idx[i] < 0 || idx[i] >= total) return -4;
+  const tshape_t* t = &ts;
+#pragma omp parallel for schedule(dynamic, 64)
+  for (int64_t i = 0; i < npts; ++i) {
+    int64_t q = idx[i];
+    int c = (int)(q % t->Co); q /= t->Co;
+    int qw = (int)(q % t->Qw); q /= t->Qw;
+    int qh = (int)(q % t->Qh); q /= t->Qh;
+    int qd = (int)(q % t->Qd); q /= t->Qd;
+    int n = (int)q;
+    tpoint_raw(t, x, w, dtype, n, qd, qh, qw, c, &y[i], &s[i]);
+  }
+  return 0;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -359,7 +359,84 @@ def pin_side_padding_is_a_crop(orc):
     assert orc.out_dims(1, 8, 9, 1, 3, 3, (1, 1, 1), (0, 2, 1), (1, 1, 1), pad_hi=(0, 0, 1)) == (1, 8, 9)
 
 
+# ---------------------------------------------------------------------------
+# Transposed ("upsampling") convolution (tutorial variants table)
+# ---------------------------------------------------------------------------
+
+_T_GEOMS = [
+    # (N, D, H, W, C, O, k, stride, pad, dil, groups) of the forward pass
+    (2, 1, 7, 6, 3, 4, (1, 3, 3), (1, 2, 2), (0, 1, 1), (1, 1, 1), 1),
+    (1, 5, 6, 7, 4, 6, (3, 3, 3), (2, 1, 2), (1, 1, 0), (1, 2, 1), 2),
+    (1, 1, 9, 8, 6, 3, (1, 4, 4), (1, 2, 3), (0, 1, 2), (1, 1, 1), 3),
+    (2, 1, 5, 5, 2, 2, (1, 2, 2), (1, 2, 2), (0, 0, 0), (1, 1, 1), 1),
+]
+
+
+def _t_out_pad(I, k, s, p, d):
+    """Output padding that makes the transposed pass return the forward input's extent."""
+    return tuple((I[i] + 2 * p[i] - d[i] * (k[i] - 1) - 1) % s[i] for i in range(3))
+
+
+def pin_transpose_adjoint(orc):
+    """The transposed convolution is the adjoint of the forward pass with the
+    same weights: sum(conv(a, w) * b) == sum(a * convT(b, w)) exactly, for
+    integer-valued a, w, b (every product and sum exact in binary64).  This
+    ties the transposed pass to the forward oracle, which the other pins fix."""
+    rng = np.random.default_rng(21)
+    for N, D, H, W, C, O, k, s, p, d, G in _T_GEOMS:
+        a = _t(rng.integers(-4, 5, (N, D, H, W, C)))
+        w = _t(rng.integers(-4, 5, (O, *k, C // G)))
+        f, _ = orc.conv_fwd(a, w, s, p, d, G)
+        b = _t(rng.integers(-4, 5, f.shape))
+        op = _t_out_pad((D, H, W), k, s, p, d)
+        t, _ = orc.conv_transpose(b, w, s, p, op, d, G)
+        assert t.shape == tuple(a.shape)
+        assert float(np.sum(f * b.double().numpy())) == float(np.sum(a.double().numpy() * t))
+
+
+def pin_transpose_torch_witness(orc):
+    """torch's CPU float64 conv_transpose3d (NCDHW; weight [Cin, Cout/G, k...])
+    agrees with the oracle's transposed pass, y and the magnitude sum S."""
+    rng = np.random.default_rng(22)
+    for N, D, H, W, C, O, k, s, p, d, G in _T_GEOMS:
+        Do, Ho, Wo = orc.out_dims(D, H, W, *k, s, p, d)
+        x = _t(rng.uniform(-1, 1, (N, Do, Ho, Wo, O)))
+        w = _t(rng.standard_normal((O, *k, C // G)))
+        op = _t_out_pad((D, H, W), k, s, p, d)
+        y, S = orc.conv_transpose(x, w, s, p, op, d, G)
+        xt = x.double().permute(0, 4, 1, 2, 3)
+        wt = w.double().permute(0, 4, 1, 2, 3)
+        yt = torch.nn.functional.conv_transpose3d(xt, wt, stride=s, padding=p, output_padding=op, groups=G,
+                                                  dilation=d).permute(0, 2, 3, 4, 1).numpy()
+        st = torch.nn.functional.conv_transpose3d(xt.abs(), wt.abs(), stride=s, padding=p, output_padding=op,
+                                                  groups=G, dilation=d).permute(0, 2, 3, 4, 1).numpy()
+        assert y.shape == yt.shape
+        assert np.allclose(y, yt, rtol=1e-12, atol=1e-12) and np.allclose(S, st, rtol=1e-12, atol=1e-12)
+
+
+def pin_transpose_delta_upsamples(orc):
+    """Closed form: a one-tap filter (1 at kh = kw = 0) with stride 2 and no
+    padding inserts zeros: y[2i, 2j] = x[i, j], every other output 0; a centre
+    tap with padding 1 does the same shifted into place."""
+    x = _t(np.arange(1, 13, dtype=np.float32).reshape(1, 1, 3, 4, 1))
+    w = torch.zeros(1, 1, 3, 3, 1)
+    w[0, 0, 0, 0, 0] = 1.0
+    y, _ = orc.conv_transpose(x, w, (1, 2, 2), (0, 0, 0), (0, 0, 0))
+    assert y.shape == (1, 1, 7, 9, 1)
+    ref = np.zeros((7, 9))
+    ref[0:6:2, 0:8:2] = x.numpy().reshape(3, 4)
+    assert np.array_equal(y.reshape(7, 9), ref)
+    wc = torch.zeros(1, 1, 3, 3, 1)
+    wc[0, 0, 1, 1, 0] = 1.0
+    y2, _ = orc.conv_transpose(x, wc, (1, 2, 2), (0, 1, 1), (0, 1, 1))
+    assert y2.shape == (1, 1, 6, 8, 1)
+    ref2 = np.zeros((6, 8))
+    ref2[0:6:2, 0:8:2] = x.numpy().reshape(3, 4)
+    assert np.array_equal(y2.reshape(6, 8), ref2)
+
+
 ALL_PINS = [pin_tutorial_example, pin_output_extent, pin_constant_input, pin_delta_kernel,
             pin_pointwise_is_matmul, pin_im2col_equivalence, pin_torch_witness, pin_linearity,
             pin_translation, pin_groups_split, pin_points_match_full, pin_flip_tutorial_example,
-            pin_flip_and_side_padding_torch_witness, pin_side_padding_is_a_crop]
+            pin_flip_and_side_padding_torch_witness, pin_side_padding_is_a_crop, pin_transpose_adjoint,
+            pin_transpose_torch_witness, pin_transpose_delta_upsamples]

@@ -104,6 +104,9 @@ MUTATIONS = {
     "extent_off_by_one": [(r"\(int64_t\)d \* \(k - 1\) - 1;", "(int64_t)d * (k - 1);")],
     "f16_exponent_bias": [(r"e - 25\);", "e - 24);")],
     "bf16_mantissa_width": [(r"\(double\)\(128 \+ m\), e - 134\)", "(double)(128 + m), e - 133)")],
+    "transpose_stride_divisibility_dropped": [(r"if \(num < 0 \|\| num % s\) return -1;", "if (num < 0) return -1;")],
+    "transpose_pad_sign": [(r"int64_t num = q \+ p - \(int64_t\)k \* d;", "int64_t num = q - p - (int64_t)k * d;")],
+    "transpose_out_channel_index": [(r"\* t->kW \+ kw\) \* Cog \+ cl;", "* t->kW + kw) * Cog + (Cog - 1 - cl);")],
     "padding_not_zero": [(r"if \(ih < 0 \|\| ih >= sh->H\) continue;", "if (ih < 0 || ih >= sh->H) ih = ih < 0 ? 0 : sh->H - 1;")],
 }
 
