@@ -15,7 +15,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["conv_fwd", "conv_fwd_host", "out_dims", "plan", "last_status", "strerror", "lib",
+__all__ = ["conv_fwd", "conv_fwd_host", "out_dims", "plan", "conv_transpose", "transpose_out_dims",
+           "transpose_plan", "last_status", "strerror", "lib",
            "CONV_F32", "CONV_F16", "CONV_BF16", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC_TMA",
            "VARIANT_TC_GATHER", "VARIANT_TC_TMA_PAIR", "VARIANT_TC_HALO", "VARIANT_TC_HALO_PAIR",
            "VARIANT_TC_TMA_T", "VARIANT_TC_HALO_T", "VARIANT_TC_HALO_T_PAIR", "VARIANT_TC_PHASE", "VARIANT_DEPTHWISE", "VARIANT_DEPTHWISE_DIRECT", "ConvError"]
@@ -66,6 +67,11 @@ def lib() -> ctypes.CDLL:
         L.conv_out_dims_ex.argtypes = [ci] * 6 + [i3, i3, i3, i3, i3]
         L.conv_fwd_ex.argtypes = [vp, vp, vp] + geo_ex + [ci, vp]
         L.conv_plan_ex.argtypes = geo_ex + [ci, i3, i3, i3]
+        # transposed convolution: ..., stride, pad, out_pad, dil, groups, dtype
+        geo_t = [ci] * 9 + [i3, i3, i3, i3, ci, ci]
+        L.conv_transpose_out_dims.argtypes = [ci] * 6 + [i3, i3, i3, i3, i3]
+        L.conv_transpose.argtypes = [vp, vp, vp] + geo_t + [ci, vp]
+        L.conv_transpose_plan.argtypes = geo_t + [ci, i3, i3, i3]
         L.conv_last_status.argtypes = [vp]
         L.conv_debug_inject_stall.argtypes = [ctypes.c_ulonglong]
         L.conv_strerror.argtypes = [ci]
@@ -178,6 +184,71 @@ def conv_fwd(x, w, stride=1, padding=0, dilation=1, groups=1, *, out=None, varia
     if rc:
         raise ConvError(rc, "conv_fwd")
     return out
+
+
+def transpose_out_dims(D, H, W, kD, kH, kW, stride, pad, out_pad, dil):
+    """(Qd, Qh, Qw) of the transposed convolution, as computed by the library (host only)."""
+    out = (ctypes.c_int * 3)()
+    rc = lib().conv_transpose_out_dims(D, H, W, kD, kH, kW, _i3(stride), _i3(pad), _i3(out_pad), _i3(dil), out)
+    if rc:
+        raise ConvError(rc, "conv_transpose_out_dims")
+    return tuple(out)
+
+
+def conv_transpose(x, w, stride=1, padding=0, output_padding=0, dilation=1, groups=1, *, out=None,
+                   variant=VARIANT_AUTO, stream=None):
+    """Transposed ("upsampling") convolution on the current CUDA stream (or
+    `stream`): the adjoint of conv_fwd with the same weights.  Returns y.
+
+    x: [N, (D,) H, W, Cin]; w: [Cin, (kD,) kH, kW, Cout/groups] (conv_fwd's
+    weight layout with O = Cin); y: [N, (Qd,) Qh, Qw, Cout] with
+    Q = (I-1)*s - 2p + d*(k-1) + 1 + output_padding per dimension.
+    """
+    import torch
+    if not (x.is_cuda and w.is_cuda):
+        raise ValueError("conv_transpose runs on CUDA tensors only")
+    if x.dtype != w.dtype:
+        raise TypeError("x and w must share a dtype")
+    two_d, (N, D, H, W, Cin, Ci, kD, kH, kW, Cog), s, p, d = _geometry(x, w, stride, padding, dilation)
+    op = _geometry(x, w, stride, output_padding, dilation)[3]
+    if Ci != Cin:
+        raise ValueError(f"weight's first dimension {Ci} must equal the input channels {Cin}")
+    Cout = Cog * groups
+    Qd, Qh, Qw = transpose_out_dims(D, H, W, kD, kH, kW, s, p, op, d)
+    shape = (N, Qh, Qw, Cout) if two_d else (N, Qd, Qh, Qw, Cout)
+    if out is None:
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+    elif tuple(out.shape) != shape or out.dtype != x.dtype or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {x.dtype} tensor of shape {shape}")
+    x = x.contiguous()
+    w = w.contiguous()
+    st = stream if stream is not None else torch.cuda.current_stream(x.device)
+    with torch.cuda.device(x.device):
+        rc = lib().conv_transpose(x.data_ptr(), w.data_ptr(), out.data_ptr(), N, D, H, W, Cin, Cout, kD, kH, kW,
+                                  _i3(s), _i3(p), _i3(op), _i3(d), int(groups), _dtype_code(x), int(variant),
+                                  st.cuda_stream)
+    if rc:
+        raise ConvError(rc, "conv_transpose")
+    return out
+
+
+def conv_transpose_raw(x_ptr, w_ptr, y_ptr, geom, dtype, variant=VARIANT_AUTO, stream_handle=0):
+    """The C entry point on raw device pointers: geom = (N,D,H,W,Cin,Cout,kD,kH,kW,stride,pad,out_pad,dil,groups)."""
+    N, D, H, W, Ci, Co, kD, kH, kW, s, p, op, d, g = geom
+    return lib().conv_transpose(x_ptr, w_ptr, y_ptr, N, D, H, W, Ci, Co, kD, kH, kW, _i3(s), _i3(p), _i3(op),
+                                _i3(d), int(g), int(dtype), int(variant), stream_handle)
+
+
+def transpose_plan(N, D, H, W, Cin, Cout, k, stride, pad, out_pad, dil, groups, dtype, variant=VARIANT_AUTO):
+    """(variant, BN, stages, CTAs) the library would use for a transposed convolution."""
+    bn, st, ct = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    code = {"f32": CONV_F32, "f16": CONV_F16, "bf16": CONV_BF16}[dtype]
+    rc = lib().conv_transpose_plan(N, D, H, W, Cin, Cout, *k, _i3(stride), _i3(pad), _i3(out_pad), _i3(dil),
+                                   int(groups), code, int(variant), ctypes.byref(bn), ctypes.byref(st),
+                                   ctypes.byref(ct))
+    if rc < 0:
+        raise ConvError(rc, "conv_transpose_plan")
+    return rc, bn.value, st.value, ct.value
 
 
 def conv_fwd_raw(x_ptr, w_ptr, y_ptr, geom, dtype, variant=VARIANT_AUTO, stream_handle=0, pad_hi=None, flip=0):

@@ -34,6 +34,8 @@ struct Problem {
   int s[3], p[3], d[3];  // p: padding below each dimension (the index origin is -p)
   int p_hi[3];           // padding above each dimension (sets the output extent with p)
   int flip;              // 1: the filter is read reversed in every spatial dimension
+  int idil[3];           // input dilation (a transposed convolution's stride); 1 = none
+  int wtrans;            // 1: w is stored [G*Cg][taps][Og] (a transposed convolution's weights)
   int G, Cg, Og;
   int Do, Ho, Wo;
   long long M;
@@ -86,6 +88,8 @@ int make_problem(Problem& P, int N, int D, int H, int W, int C, int O, int kD, i
     P.s[i] = stride[i]; P.p[i] = pad_lo[i]; P.p_hi[i] = pad_hi[i]; P.d[i] = dil[i];
   }
   P.flip = flip;
+  P.idil[0] = P.idil[1] = P.idil[2] = 1;
+  P.wtrans = 0;
   P.G = groups; P.Cg = C / groups; P.Og = O / groups;
   P.Do = out[0]; P.Ho = out[1]; P.Wo = out[2];
   P.dtype = dtype;
@@ -105,6 +109,69 @@ int make_problem(Problem& P, int N, int D, int H, int W, int C, int O, int kD, i
   P.w_bytes = static_cast<size_t>(nw) * P.esize;
   P.y_bytes = static_cast<size_t>(ny) * P.esize;
   return CONV_OK;
+}
+
+// Output extents of the transposed convolution: (I-1)*s - 2p + d*(k-1) + 1 + op
+// per dimension, op (output padding) in [0, max(s, d)).
+int convT_dims_impl(int D, int H, int W, int kD, int kH, int kW, const int stride[3], const int pad[3],
+                    const int out_pad[3], const int dil[3], int out[3]) {
+  if (!stride || !pad || !out_pad || !dil || !out) return CONV_EINVAL;
+  const int in[3] = {D, H, W};
+  const int k[3] = {kD, kH, kW};
+  for (int i = 0; i < 3; ++i) {
+    if (in[i] <= 0 || k[i] <= 0 || stride[i] <= 0 || dil[i] <= 0 || pad[i] < 0 || out_pad[i] < 0)
+      return CONV_EINVAL;
+    if (out_pad[i] >= stride[i] && out_pad[i] >= dil[i]) return CONV_EINVAL;
+    const long long e = (static_cast<long long>(in[i]) - 1) * stride[i] - 2LL * pad[i] +
+                        static_cast<long long>(dil[i]) * (k[i] - 1) + 1 + out_pad[i];
+    if (e <= 0 || e > 0x7fffffffLL) return CONV_EINVAL;
+    out[i] = static_cast<int>(e);
+  }
+  return CONV_OK;
+}
+
+// The transposed convolution of x [N,D,H,W,Cin] by w [Cin,kD,kH,kW,Cout/G] as
+// a forward convolution: the input zero-dilated by the stride, stride 1, the
+// filter mirrored (flip) with its channel axes exchanged (wtrans), and padding
+// d*(k-1) - p below and d*(k-1) - p + op above.  Padding beyond d*(k-1) (a
+// crop of the dilated sum) is not supported.
+int make_transpose_problem(Problem& P, int N, int D, int H, int W, int Cin, int Cout, int kD, int kH, int kW,
+                           const int stride[3], const int pad[3], const int out_pad[3], const int dil[3],
+                           int groups, int dtype) {
+  int out[3];
+  int rc = convT_dims_impl(D, H, W, kD, kH, kW, stride, pad, out_pad, dil, out);
+  if (rc != CONV_OK) return rc;
+  const int k[3] = {kD, kH, kW};
+  int lo[3], hi[3], one[3] = {1, 1, 1};
+  for (int i = 0; i < 3; ++i) {
+    const long long span = static_cast<long long>(dil[i]) * (k[i] - 1);
+    if (pad[i] > span) return CONV_EUNSUPPORTED;
+    lo[i] = static_cast<int>(span - pad[i]);
+    hi[i] = static_cast<int>(span - pad[i] + out_pad[i]);
+  }
+  // extents of the zero-dilated input
+  long long dd[3];
+  const int in[3] = {D, H, W};
+  for (int i = 0; i < 3; ++i) {
+    dd[i] = (static_cast<long long>(in[i]) - 1) * stride[i] + 1;
+    if (dd[i] > 0x7fffffffLL) return CONV_EINVAL;
+  }
+  rc = make_problem(P, N, static_cast<int>(dd[0]), static_cast<int>(dd[1]), static_cast<int>(dd[2]), Cin, Cout, kD,
+                    kH, kW, one, lo, hi, dil, groups, 1, dtype);
+  if (rc != CONV_OK) return rc;
+  if (P.Do != out[0] || P.Ho != out[1] || P.Wo != out[2]) return CONV_EINVAL;  // (the two extents agree)
+  P.D = D; P.H = H; P.W = W;
+  for (int i = 0; i < 3; ++i) P.idil[i] = stride[i];
+  P.wtrans = 1;
+  long long nx, t;
+  if (!mul_ok(N, D, t) || !mul_ok(t, H, t) || !mul_ok(t, W, t) || !mul_ok(t, Cin, nx)) return CONV_EINVAL;
+  P.x_bytes = static_cast<size_t>(nx) * P.esize;
+  return CONV_OK;
+}
+
+// Problems every kernel can take: no input dilation, weights in the forward layout.
+bool plain_input(const Problem& P) {
+  return P.idil[0] == 1 && P.idil[1] == 1 && P.idil[2] == 1 && !P.wtrans;
 }
 
 bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
@@ -624,6 +691,8 @@ int plan_phase(const Problem& P, int sms, TcPlan& plan) {
 }
 
 int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
+  // input dilation and transposed weights: the gather kernel only
+  if (!plain_input(P) && variant != CONV_VARIANT_TC_GATHER) return CONV_EUNSUPPORTED;
   if (variant == CONV_VARIANT_TC_PHASE) return plan_phase(P, sms, plan);
   if (variant == CONV_VARIANT_TC_HALO_T || variant == CONV_VARIANT_TC_HALO_T_PAIR)
     return plan_halo_t(P, variant == CONV_VARIANT_TC_HALO_T_PAIR, sms, plan);
@@ -667,7 +736,7 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
     // layout where each filter row (kd, kh) is padded to Lp = roundup(kW*C, 8)
     if (P.Cg % 8 == 0) {
       a.gather_mode = GATHER_VEC8;
-    } else if (P.G == 1 && P.d[2] == 1 && !P.flip) {  // (span layout: the filter's own tap order)
+    } else if (P.G == 1 && P.d[2] == 1 && !P.flip && plain_input(P)) {  // (span layout: the filter's own tap order)
       a.gather_mode = GATHER_SPAN;
     } else {
       a.gather_mode = GATHER_SCALAR;
@@ -710,6 +779,9 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
     a.kblocks = static_cast<int>((kp + 63) / 64);
   }
   a.x_elems = static_cast<long long>(P.x_bytes / P.esize);
+  a.idil_on = plain_input(P) ? 0 : 1;
+  a.idd = P.idil[0]; a.idh = P.idil[1]; a.idw = P.idil[2];
+  a.wtrans = P.wtrans;
   a.layout_type = a.kc == 64 ? 2u : (a.kc == 32 ? 4u : 6u);
   a.sbo = static_cast<uint32_t>(8 * a.kc * 2);
   a.a_bytes = static_cast<uint32_t>(kBM * a.kc * 2);
@@ -768,7 +840,7 @@ int dw_vec(const Problem& P) { return P.dtype == CONV_F32 ? 4 : 8; }
 bool dw_fits(const Problem& P) {
   const long long taps = static_cast<long long>(P.kD) * P.kH * P.kW;
   return P.Cg == 1 && P.Og == 1 && (static_cast<long long>(P.C) * static_cast<long long>(P.esize)) % 16 == 0 &&
-         taps * dw_vec(P) * 4 <= kDwSmemLimit;
+         taps * dw_vec(P) * 4 <= kDwSmemLimit && plain_input(P);
 }
 
 void dw_geometry(const Problem& P, DwArgs& a) {
@@ -1034,6 +1106,7 @@ int launch_dw(const Problem& P, const void* x, const void* w, void* y, cudaStrea
 }
 
 int choose_variant(const Problem& P, int sms) {
+  if (!plain_input(P)) return P.dtype == CONV_F32 ? CONV_VARIANT_SIMT : CONV_VARIANT_TC_GATHER;
   if (dw_fits(P)) return CONV_VARIANT_DEPTHWISE;
   if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
   bool r5;
@@ -1429,6 +1502,8 @@ int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStr
   a.M = P.M; a.K = static_cast<int>(P.K);
   a.flip = P.flip;
   a.taps = P.kD * P.kH * P.kW;
+  a.idd = P.idil[0]; a.idh = P.idil[1]; a.idw = P.idil[2];
+  a.wtrans = P.wtrans;
   a.x = x; a.w = w; a.y = y;
   const SimtShape sh = simt_shape(P, sms);
   const long long mt = (P.M + 16 * sh.tm - 1) / (16 * sh.tm);
@@ -1465,6 +1540,12 @@ int run(const Problem& P, const void* x, const void* w, void* y, int variant, cu
   return launch_tc(P, plan, x, w, y, st, dev);
 }
 
+}  // namespace
+}  // namespace convfwd
+
+namespace convfwd {
+namespace {
+int plan_problem(const Problem& P, int variant, int* bn, int* stages, int* ctas);
 }  // namespace
 }  // namespace convfwd
 
@@ -1534,6 +1615,42 @@ int conv_plan_ex(int N, int D, int H, int W, int C, int O, int kD, int kH, int k
   Problem P;
   int rc = make_problem(P, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, flip, dtype);
   if (rc != CONV_OK) return rc;
+  return plan_problem(P, variant, bn, stages, ctas);
+}
+
+int conv_transpose_out_dims(int D, int H, int W, int kD, int kH, int kW, const int stride[3], const int pad[3],
+                            const int out_pad[3], const int dil[3], int out[3]) {
+  return convT_dims_impl(D, H, W, kD, kH, kW, stride, pad, out_pad, dil, out);
+}
+
+int conv_transpose(const void* x, const void* w, void* y, int N, int D, int H, int W, int Cin, int Cout, int kD,
+                   int kH, int kW, const int stride[3], const int pad[3], const int out_pad[3], const int dil[3],
+                   int groups, int dtype, int variant, conv_stream_t stream) {
+  Problem P;
+  int rc = make_transpose_problem(P, N, D, H, W, Cin, Cout, kD, kH, kW, stride, pad, out_pad, dil, groups, dtype);
+  if (rc != CONV_OK) return rc;
+  rc = check_pointers(P, x, w, y);
+  if (rc != CONV_OK) return rc;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_DEPTHWISE_DIRECT) return CONV_EINVAL;
+  return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int conv_transpose_plan(int N, int D, int H, int W, int Cin, int Cout, int kD, int kH, int kW, const int stride[3],
+                        const int pad[3], const int out_pad[3], const int dil[3], int groups, int dtype, int variant,
+                        int* bn, int* stages, int* ctas) {
+  Problem P;
+  int rc = make_transpose_problem(P, N, D, H, W, Cin, Cout, kD, kH, kW, stride, pad, out_pad, dil, groups, dtype);
+  if (rc != CONV_OK) return rc;
+  return plan_problem(P, variant, bn, stages, ctas);
+}
+
+}  // extern "C"
+
+namespace convfwd {
+namespace {
+
+int plan_problem(const Problem& P, int variant, int* bn, int* stages, int* ctas) {
+  int rc;
   if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_DEPTHWISE_DIRECT) return CONV_EINVAL;
   int dev, sms = 148;
   if (current_device(dev) == CONV_OK) device_sms(dev, sms);
@@ -1577,6 +1694,11 @@ int conv_plan_ex(int N, int D, int H, int W, int C, int O, int kD, int kH, int k
   if (ctas) *ctas = plan.ctas;
   return variant;
 }
+
+}  // namespace
+}  // namespace convfwd
+
+extern "C" {
 
 int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
                       const int pad[3], const int dil[3], int groups, int dtype, int variant, int* bn,

@@ -28,6 +28,8 @@ struct SimtArgs {
   int K;
   int flip;   // 1: the filter is read reversed in every spatial dimension
   int taps;   // kD*kH*kW
+  int idd, idh, idw;  // input dilation: position z holds x[z / id*] when id* divides z, else 0
+  int wtrans;         // 1: w is stored [G*Cg][taps][Og] (a transposed convolution's weights)
   const void* x;
   const void* w;
   void* y;
@@ -59,6 +61,15 @@ constexpr int kSimtBK = 16, kSimtThreads = 256;
 // 80, 96 or 128), so layers like O = 65 or 21 do not compute mostly padding.
 // Loads of the next K step go to registers before the current step's FMAs and
 // to the other shared-memory buffer after them: one barrier per step.
+// Input position z of a dimension dilated by s: true, with z replaced by the
+// element index, when the position holds an input element (s = 1: plain bounds).
+__device__ __forceinline__ bool simt_undilate(int& z, int s, int n) {
+  if (s == 1) return static_cast<unsigned>(z) < static_cast<unsigned>(n);
+  if (z < 0 || z % s != 0) return false;
+  z /= s;
+  return z < n;
+}
+
 template <typename T, int TM, int TN>
 __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtArgs a) {
   constexpr int BM = 16 * TM, BN = 16 * TN;
@@ -119,17 +130,25 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
 #pragma unroll
     for (int i = 0; i < TM; ++i) {
       float v = 0.f;
-      const int zd = rd0[i] + id, zh = rh0[i] + ih, zw = rw0[i] + iw;
-      if (rvalid[i] && kv && static_cast<unsigned>(zd) < static_cast<unsigned>(a.D) &&
-          static_cast<unsigned>(zh) < static_cast<unsigned>(a.H) &&
-          static_cast<unsigned>(zw) < static_cast<unsigned>(a.W))
+      int zd = rd0[i] + id, zh = rh0[i] + ih, zw = rw0[i] + iw;
+      if (rvalid[i] && kv && simt_undilate(zd, a.idd, a.D) && simt_undilate(zh, a.idh, a.H) &&
+          simt_undilate(zw, a.idw, a.W))
         v = to_f32<T>(x[rbase[i] + ((static_cast<long long>(zd) * a.H + zh) * a.W + zw) * a.C + c]);
       ra[i] = v;
     }
-    // the weight element: k itself, or with flip the mirrored tap's channel c
-    const int wk = a.flip ? (a.taps - 1 - ((kd * a.kH + kh) * a.kW + kw)) * a.Cg + c : k;
+    // the weight element: k itself, or with flip the mirrored tap's channel c;
+    // transposed storage [G*Cg][taps][Og] puts it at ((g*Cg + c)*taps + tap)*Og + o
+    const int tapk = (kd * a.kH + kh) * a.kW + kw;
+    const int wt = a.flip ? a.taps - 1 - tapk : tapk;
+    if (a.wtrans) {
+      const long long wb = (static_cast<long long>(g * a.Cg + c) * a.taps + wt) * a.Og;
 #pragma unroll
-    for (int j = 0; j < TN; ++j) rb[j] = (ovalid[j] && kv) ? to_f32<T>(wrow[j][wk]) : 0.f;
+      for (int j = 0; j < TN; ++j) rb[j] = (ovalid[j] && kv) ? to_f32<T>(w[wb + n0 + lr + 16 * j]) : 0.f;
+    } else {
+      const int wk = wt * a.Cg + c;
+#pragma unroll
+      for (int j = 0; j < TN; ++j) rb[j] = (ovalid[j] && kv) ? to_f32<T>(wrow[j][wk]) : 0.f;
+    }
     // advance the carried decode by one K step
     c += kSimtBK;
     while (c >= a.Cg) {

@@ -59,6 +59,10 @@ struct TcArgs {
   int N, D, H, W, C, O;
   int kD, kH, kW;
   int sd, sh, sw, pd, ph, pw, dd, dh, dw;
+  // input dilation (gather modes only): input position z of the zero-inserted
+  // input holds x[z / id*] when z is a multiple of id*, else 0
+  int idil_on, idd, idh, idw;
+  int wtrans;         // 1: w is stored [G*Cg][taps][Og] (a transposed convolution's weights)
   int G, Cg, Og;
   int Do, Ho, Wo;
   long long M;
@@ -365,16 +369,36 @@ __device__ __forceinline__ SpanPos span_pos(const TcArgs& a, int k) {
   return p;
 }
 
+// Position z of an input dimension dilated by s (zeros inserted between
+// elements): true, with z replaced by the element index, when z is a multiple
+// of s inside the input of n elements.
+__device__ __forceinline__ bool undilate(int& z, int s, int n) {
+  if (z < 0 || z % s != 0) return false;
+  z /= s;
+  return z < n;
+}
+
 // One filter row (kd, kh) of one output pixel: offset of x[n, id, ih, 0, g*Cg]
 // and whether that input row exists.
 __device__ __forceinline__ bool gather_span(const TcArgs& a, const GatherRow& st, int kd, int kh,
                                             long long& rowptr) {
-  const int id = st.id0 + kd * a.dd;
-  const int ih = st.ih0 + kh * a.dh;
-  const bool ok = st.valid && kd < a.kD && static_cast<unsigned>(id) < static_cast<unsigned>(a.D) &&
-                  static_cast<unsigned>(ih) < static_cast<unsigned>(a.H);
-  rowptr = st.nbase + (static_cast<long long>(id) * a.H + ih) * static_cast<long long>(a.W) * a.C;
+  int id = st.id0 + kd * a.dd;
+  int ih = st.ih0 + kh * a.dh;
+  bool ok;
+  if (a.idil_on) {
+    ok = st.valid && kd < a.kD && undilate(id, a.idd, a.D) && undilate(ih, a.idh, a.H);
+  } else {
+    ok = st.valid && kd < a.kD && static_cast<unsigned>(id) < static_cast<unsigned>(a.D) &&
+         static_cast<unsigned>(ih) < static_cast<unsigned>(a.H);
+  }
+  rowptr = st.nbase + (static_cast<long long>(ok ? id : 0) * a.H + (ok ? ih : 0)) * static_cast<long long>(a.W) * a.C;
   return ok;
+}
+
+// Input column of one tap: the element index (in place) and whether it exists.
+__device__ __forceinline__ bool gather_col(const TcArgs& a, int& iw) {
+  if (a.idil_on) return undilate(iw, a.idw, a.W);
+  return static_cast<unsigned>(iw) < static_cast<unsigned>(a.W);
 }
 
 __device__ __forceinline__ void store_chunk(uint8_t* a_tile, int r, int ch, uint4 v) {
@@ -415,9 +439,9 @@ __device__ __forceinline__ void gather_a_vec8(const TcArgs& a, const GatherRow& 
   uint4 v[NCH];
 #pragma unroll
   for (int q = 0; q < NCH; ++q) {
-    const int iw = st.iw0 + kw * a.dw;
+    int iw = st.iw0 + kw * a.dw;
     v[q] = make_uint4(0, 0, 0, 0);
-    if (rok && static_cast<unsigned>(iw) < static_cast<unsigned>(a.W))
+    if (rok && gather_col(a, iw))
       v[q] = __ldg(reinterpret_cast<const uint4*>(x + rowptr + static_cast<long long>(iw) * a.C + c));
     c += 8;
     if (c == a.Cg) {
@@ -601,10 +625,8 @@ __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow
   bool ok = gather_span(a, st, kd, kh, rowptr);
 #pragma unroll
   for (int e = 0; e < 8 * NCH; ++e) {
-    const int iw = st.iw0 + kw * a.dw;
-    v[e] = (ok && static_cast<unsigned>(iw) < static_cast<unsigned>(a.W))
-               ? __ldg(x + rowptr + static_cast<long long>(iw) * a.C + c)
-               : 0u;
+    int iw = st.iw0 + kw * a.dw;
+    v[e] = (ok && gather_col(a, iw)) ? __ldg(x + rowptr + static_cast<long long>(iw) * a.C + c) : 0u;
     if (++c == a.Cg) {
       c = 0;
       if (++kw == a.kW) {
@@ -642,7 +664,20 @@ __device__ __forceinline__ void gather_b_block(const TcArgs& a, int g, int n0, i
     uint4 v = make_uint4(0, 0, 0, 0);
     if (oc < a.Og && kp0 < a.Kp) {
       const long long rowoff = static_cast<long long>(g * a.Og + oc) * a.K;
-      if (span_layout) {  // (never with flip: the planner uses the other layouts)
+      if (a.wtrans) {
+        // w stored [G*Cg][taps][Og]: K element k = tap*Cg + c of output
+        // channel oc multiplies w[g*Cg + c][tap (mirrored under flip)][oc]
+        uint16_t e8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int k = kp0 + e;
+          const int tap = k / a.Cg;
+          const long long wi =
+              (static_cast<long long>(g * a.Cg + (k - tap * a.Cg)) * a.taps + wtap(a, tap)) * a.Og + oc;
+          e8[e] = k < a.K ? w[wi] : uint16_t(0);
+        }
+        v = *reinterpret_cast<const uint4*>(e8);
+      } else if (span_layout) {  // (never with flip: the planner uses the other layouts)
         const int sp = kp0 / a.Lp;
         const int j0 = kp0 - sp * a.Lp;
         v = load8_masked(w + rowoff + static_cast<long long>(sp) * L + j0, 0, L - j0);

@@ -199,6 +199,41 @@ int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, 
                       const int stride[3], const int pad[3], const int dil[3],
                       int groups, int dtype, int variant, int* bn, int* stages, int* ctas);
 
+/* ---- transposed ("upsampling") convolution ----------------------------
+ *
+ * "Convolutions" tutorial, "Convolution variants worth knowing": the
+ * transposed convolution of decoders and diffusion models, read as the
+ * adjoint (data gradient) of conv_fwd with the same weights:
+ *
+ *   y[n, q, g*Cout/G + c] = sum over taps k and input channels ci of group g
+ *                           with q = i*s - p + k*d (per dimension) of
+ *                           x[n, i, ci] * w[ci, k, c]
+ *
+ * x: [N, D, H, W, Cin]; w: [Cin, kD, kH, kW, Cout/groups] (conv_fwd's weight
+ * layout with O = Cin, C = Cout); y: [N, Qd, Qh, Qw, Cout] with
+ * Q = (I-1)*s - 2p + d*(k-1) + 1 + op per dimension, the output padding op in
+ * [0, max(s, d)).  Requires p <= d*(k-1) per dimension (CONV_EUNSUPPORTED
+ * otherwise).  It runs as a forward convolution over the input zero-dilated
+ * by the stride (the inserted zeros are never stored: the gather producers and
+ * the FP32 kernel skip them when computing addresses) with the mirrored,
+ * channel-exchanged filter: variants AUTO (TC_GATHER for f16/bf16, SIMT for
+ * f32), TC_GATHER and SIMT; any other variant returns CONV_EUNSUPPORTED.
+ * Buffers, alignment, streams and errors as for conv_fwd. */
+
+/* Extents (Qd, Qh, Qw) of the transposed convolution. */
+int conv_transpose_out_dims(int D, int H, int W, int kD, int kH, int kW, const int stride[3],
+                            const int pad[3], const int out_pad[3], const int dil[3], int out[3]);
+
+/* Queues the transposed convolution on `stream`; allocates nothing. */
+int conv_transpose(const void* x, const void* w, void* y, int N, int D, int H, int W, int Cin, int Cout,
+                   int kD, int kH, int kW, const int stride[3], const int pad[3], const int out_pad[3],
+                   const int dil[3], int groups, int dtype, int variant, conv_stream_t stream);
+
+/* conv_plan_variant for the transposed convolution.  Queues nothing. */
+int conv_transpose_plan(int N, int D, int H, int W, int Cin, int Cout, int kD, int kH, int kW,
+                        const int stride[3], const int pad[3], const int out_pad[3], const int dil[3],
+                        int groups, int dtype, int variant, int* bn, int* stages, int* ctas);
+
 /* Waits for `stream`, then reads and clears the current device's status word.
  * Returns CONV_OK, or CONV_ETIMEOUT if a kernel since the last call gave up on
  * a pipeline wait (the kernel then wrote no further output and returned), or

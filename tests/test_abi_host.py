@@ -246,3 +246,27 @@ def test_explicit_variant_plan(C):
     with pytest.raises(C.ConvError) as e:
         C.plan(*g3, "bf16", 12)
     assert e.value.code == -1
+
+
+def test_transpose_extents_and_plans(C):
+    """Transposed-convolution extents agree with the oracle's; the planner runs
+    it on the gather kernel (16-bit) or the FP32 kernel and refuses the rest."""
+    import oracle
+    for D, H, W, k, s, p, op, d in ((3, 4, 5, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1)),
+                                    (5, 6, 7, (3, 3, 3), (2, 1, 2), (1, 1, 0), (1, 0, 1), (1, 2, 1)),
+                                    (1, 28, 28, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1))):
+        assert C.transpose_out_dims(D, H, W, *k, s, p, op, d) == oracle.convT_out_dims(D, H, W, *k, s, p, op, d)
+    g = (2, 1, 28, 28, 256, 128, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1)
+    assert C.transpose_plan(*g, "f16")[0] == C.VARIANT_TC_GATHER
+    assert C.transpose_plan(*g, "f32")[0] == C.VARIANT_SIMT
+    for v in (C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR, C.VARIANT_TC_HALO_T, C.VARIANT_TC_PHASE, C.VARIANT_DEPTHWISE):
+        with pytest.raises(C.ConvError) as e:
+            C.transpose_plan(*g, "f16", v)
+        assert e.value.code == -7
+    # padding beyond d*(k-1) (a crop of the dilated sum) is not supported
+    with pytest.raises(C.ConvError) as e:
+        C.transpose_plan(1, 1, 8, 8, 16, 16, (1, 3, 3), (1, 2, 2), (0, 3, 3), (0, 0, 0), (1, 1, 1), 1, "f16")
+    assert e.value.code == -7
+    # output padding must stay below max(stride, dilation)
+    with pytest.raises(C.ConvError):
+        C.transpose_out_dims(1, 8, 8, 1, 3, 3, (1, 2, 2), (0, 1, 1), (0, 2, 2), (1, 1, 1))

@@ -263,6 +263,72 @@ def test_flip_and_side_padding(case, dtype):
         assert ran >= 1
 
 
+# Transposed ("upsampling") convolution: (name, N, D, H, W, Cin, Cout, k, stride, pad, out_pad, dil, groups).
+# 8-channel vectors and scalar gathers, strides 1-3, output padding, dilation,
+# groups, 2-D and 3-D, several ragged 128-row tiles.
+TRANSPOSE = [
+    ("t_k3s2p1_op1", 2, 1, 7, 6, 16, 24, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+    ("t_k4s2p1_decoder", 2, 1, 9, 8, 32, 16, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1),
+    ("t_3d_mixed_groups2", 1, 4, 5, 6, 8, 12, (3, 3, 3), (2, 1, 2), (1, 1, 0), (1, 0, 1), (1, 2, 1), 2),
+    ("t_c5_scalar", 2, 1, 6, 7, 5, 7, (1, 2, 2), (1, 2, 2), (0, 0, 0), (0, 0, 0), (1, 1, 1), 1),
+    ("t_stride1", 1, 1, 12, 11, 64, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1),
+    ("t_s3_d2", 1, 1, 6, 5, 16, 8, (1, 3, 3), (1, 3, 3), (0, 2, 1), (0, 2, 1), (1, 2, 2), 1),
+    ("t_groups4", 2, 1, 8, 9, 32, 32, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1), 4),
+    ("t_ragged_tiles", 2, 1, 20, 17, 24, 40, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+]
+
+
+def run_gpu_transpose(x, w, geom, dtype, variant, guard=64):
+    N, D, H, W, Cin, Cout, k, s, p, op, d, G = geom
+    Q = C.transpose_out_dims(D, H, W, *k, s, p, op, d)
+    n = N * Q[0] * Q[1] * Q[2] * Cout
+    es = x.element_size()
+    buf = torch.full((n + 2 * guard,), 0x5A5A if es == 2 else 0x5A5A5A5A,
+                     dtype=torch.int16 if es == 2 else torch.int32, device="cuda")
+    y = buf[guard:guard + n].view(x.dtype).view(N, *Q, Cout)
+    xd, wd = x.cuda(), w.cuda()
+    rc = C.conv_transpose_raw(xd.data_ptr(), wd.data_ptr(), y.data_ptr(), (N, D, H, W, Cin, Cout, *k, s, p, op, d, G),
+                              {"f32": 0, "f16": 1, "bf16": 2}[dtype], variant,
+                              torch.cuda.current_stream().cuda_stream)
+    assert rc == 0, C.strerror(rc)
+    torch.cuda.synchronize()
+    assert C.last_status() == 0
+    g = buf.cpu()
+    pat = 0x5A5A if es == 2 else 0x5A5A5A5A
+    assert torch.all(g[:guard] == pat) and torch.all(g[guard + n:] == pat), "write outside y"
+    return y.cpu()
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("case", TRANSPOSE, ids=lambda c: c[0])
+def test_transpose_parity(case, dtype):
+    name, *geom = case
+    N, D, H, W, Cin, Cout, k, s, p, op, d, G = geom
+    gen = torch.Generator().manual_seed(zlib.crc32(name.encode()) % 1000)
+    dt = WL.TORCH_DTYPE[dtype]
+    x = (torch.rand((N, D, H, W, Cin), generator=gen) * 2 - 1).to(dt)
+    w = (torch.randn((Cin, *k, Cout // G), generator=gen) / (Cin // G * k[0] * k[1] * k[2]) ** 0.5).to(dt)
+    y_ref, s_ref = oracle.conv_transpose(x, w, s, p, op, d, G)
+    for v in ([C.VARIANT_SIMT] if dtype == "f32" else [C.VARIANT_TC_GATHER, C.VARIANT_SIMT]) + [C.VARIANT_AUTO]:
+        y = run_gpu_transpose(x, w, geom, dtype, v)
+        assert_parity(y, y_ref, s_ref, dtype, f"{name}/{dtype}/{C.VARIANT_NAMES.get(v, 'auto')}")
+
+
+def test_transpose_python_api():
+    """conv_transpose on 2-D tensors against the oracle; a forced TMA variant is refused."""
+    gen = torch.Generator().manual_seed(3)
+    x = (torch.rand((2, 9, 8, 32), generator=gen) * 2 - 1).to(torch.bfloat16)
+    w = (torch.randn((32, 4, 4, 16), generator=gen) / 16).to(torch.bfloat16)
+    y = C.conv_transpose(x.cuda(), w.cuda(), stride=2, padding=1)
+    torch.cuda.synchronize()
+    assert tuple(y.shape) == (2, 18, 16, 16)
+    y_ref, s_ref = oracle.conv_transpose(x.unsqueeze(1), w.unsqueeze(1), (1, 2, 2), (0, 1, 1))
+    assert_parity(y.cpu().unsqueeze(1), y_ref, s_ref, "bf16", "python api")
+    with pytest.raises(C.ConvError) as e:
+        C.conv_transpose(x.cuda(), w.cuda(), stride=2, padding=1, variant=C.VARIANT_TC_TMA)
+    assert e.value.code == -7
+
+
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_transposed_wide_pixel_tiles(dtype):
     """Enough output pixels for 256-pixel tiles on every SM (the 128-pixel
