@@ -51,11 +51,17 @@ PROFILE_DIR = os.path.join(ROOT, "profiles")
 
 def out_dims(wl, pad_hi=None):
     import implicit_gemm_convolution_conv2d_b200 as C
+    if wl.transpose:
+        return C.transpose_out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.out_pad, wl.dil)
     return C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil, pad_hi)
 
 
 def conv_flops(wl, dims=None):
-    """Algorithmic FLOPs: 2 * N * Do*Ho*Wo * O * kD*kH*kW * C/groups (padding taps counted)."""
+    """Algorithmic FLOPs: 2 * N * Do*Ho*Wo * O * kD*kH*kW * C/groups (padding taps counted).
+    A transposed convolution counts those of the forward pass it is the adjoint
+    of: 2 * N * D*H*W (its input pixels) * C * kD*kH*kW * O/groups."""
+    if wl.transpose:
+        return 2 * wl.N * wl.D * wl.H * wl.W * wl.C * wl.k[0] * wl.k[1] * wl.k[2] * (wl.O // wl.groups)
     Do, Ho, Wo = dims if dims is not None else out_dims(wl)
     return 2 * wl.N * Do * Ho * Wo * wl.O * wl.k[0] * wl.k[1] * wl.k[2] * (wl.C // wl.groups)
 
@@ -271,9 +277,14 @@ def bench_ours(args):
     dims = out_dims(wl, pad_hi)
     flops = conv_flops(wl, dims)
     xb, wb, yb = conv_bytes(wl, dims)
-    variant, bn, stages, ctas = C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil,
-                                       wl.groups, wl.dtype, getattr(C, "VARIANT_" + args.variant), pad_hi=pad_hi,
-                                       flip=flip)
+    if wl.transpose:
+        variant, bn, stages, ctas = C.transpose_plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad,
+                                                     wl.out_pad, wl.dil, wl.groups, wl.dtype,
+                                                     getattr(C, "VARIANT_" + args.variant))
+    else:
+        variant, bn, stages, ctas = C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil,
+                                           wl.groups, wl.dtype, getattr(C, "VARIANT_" + args.variant),
+                                           pad_hi=pad_hi, flip=flip)
     vname = C.VARIANT_NAMES[variant]
 
     # inputs: seeded on the host (rank-dependent seed), copied once
@@ -294,8 +305,13 @@ def bench_ours(args):
         nonlocal launches
         s = i % nsets
         # the launch goes to the current stream (the capture stream while a graph is recorded)
-        rc = C.conv_fwd_raw(xs[s].data_ptr(), wts[s].data_ptr(), ys[s].data_ptr(), geo(s), dcode,
-                            variant, torch.cuda.current_stream(dev).cuda_stream, pad_hi=pad_hi, flip=flip)
+        if wl.transpose:
+            rc = C.conv_transpose_raw(xs[s].data_ptr(), wts[s].data_ptr(), ys[s].data_ptr(),
+                                      (wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, *wl.k, wl.stride, wl.pad, wl.out_pad,
+                                       wl.dil, wl.groups), dcode, variant, torch.cuda.current_stream(dev).cuda_stream)
+        else:
+            rc = C.conv_fwd_raw(xs[s].data_ptr(), wts[s].data_ptr(), ys[s].data_ptr(), geo(s), dcode,
+                                variant, torch.cuda.current_stream(dev).cuda_stream, pad_hi=pad_hi, flip=flip)
         if rc:
             raise C.ConvError(rc, "conv_fwd")
         launches += 1
@@ -383,6 +399,8 @@ def bench_ours(args):
     e2e = None
     if pad_hi is not None or flip:
         e2e = {"skipped": "the host-buffer entry point takes symmetric padding and no flip"}
+    elif wl.transpose:
+        e2e = {"skipped": "the host-buffer entry point is the forward convolution's"}
     elif not args.no_e2e:
         xp = x_h.pin_memory()
         wp = w_h.pin_memory()
@@ -446,7 +464,8 @@ def bench_ours(args):
         "frac_of_dense_peak": round(value / nranks / SPEC_DENSE_TFLOPS, 4),
         "config": {"workload": wl.name, "N": wl.N, "DHW": [wl.D, wl.H, wl.W], "C": wl.C, "O": wl.O,
                    "kernel": list(wl.k), "stride": list(wl.stride), "pad": list(wl.pad), "dil": list(wl.dil),
-                   "groups": wl.groups, "out_DHW": list(dims), "gflop_per_step": round(flops / 1e9, 4),
+                   "groups": wl.groups, "out_DHW": list(dims),
+                   **({"transpose": True, "out_pad": list(wl.out_pad)} if wl.transpose else {}), "gflop_per_step": round(flops / 1e9, 4),
                    "global_batch": wl.N * nranks, "parallelism": f"independent batches x{nranks}",
                    "variant": vname,
                    "tile": (simt_tile(wl, dims, bn, ctas) if variant == C.VARIANT_SIMT else
@@ -482,7 +501,10 @@ def bench_ours(args):
 def _oracle_sample_step(wl, x, w, n_img):
     import oracle
     xs = x[:n_img].contiguous()
-    y, _ = oracle.conv_fwd(xs, w, wl.stride, wl.pad, wl.dil, wl.groups)
+    if wl.transpose:
+        y, _ = oracle.conv_transpose(xs, w, wl.stride, wl.pad, wl.out_pad, wl.dil, wl.groups)
+    else:
+        y, _ = oracle.conv_fwd(xs, w, wl.stride, wl.pad, wl.dil, wl.groups)
     return y
 
 
@@ -525,7 +547,7 @@ def _oracle_single_thread(wl, x, w, max_flops=3e9):
     oracle.set_threads(1)
     try:
         t0 = time.perf_counter()
-        oracle.conv_fwd(xs, w, sub.stride, sub.pad, sub.dil, sub.groups)
+        _oracle_sample_step(sub, xs, w, 1)
         dt = time.perf_counter() - t0
     finally:
         oracle.set_threads(full)

@@ -435,8 +435,13 @@ def _reduced(wl, max_macs=3e9):
 def test_workload_reduced_batch(name):
     wl = _reduced(WL.WORKLOADS[name])
     x, w = WL.make_inputs(wl)
-    y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups)
-    y = run_gpu(x, w, wl, C.VARIANT_AUTO)
+    if wl.transpose:
+        y_ref, s_ref = oracle.conv_transpose(x, w, wl.stride, wl.pad, wl.out_pad, wl.dil, wl.groups)
+        y = run_gpu_transpose(x, w, (wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.out_pad,
+                                     wl.dil, wl.groups), wl.dtype, C.VARIANT_AUTO)
+    else:
+        y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups)
+        y = run_gpu(x, w, wl, C.VARIANT_AUTO)
     assert_parity(y, y_ref, s_ref, wl.dtype, name)
 
 
@@ -459,12 +464,19 @@ def _sample_indices(shape, rng, n_random=6000):
 def test_workload_full_size_sampled(name):
     wl = WL.WORKLOADS[name]
     x, w = WL.make_inputs(wl)
-    y = C.conv_fwd(x.cuda(), w.cuda(), stride=wl.stride, padding=wl.pad, dilation=wl.dil, groups=wl.groups)
+    if wl.transpose:
+        y = C.conv_transpose(x.cuda(), w.cuda(), stride=wl.stride, padding=wl.pad, output_padding=wl.out_pad,
+                             dilation=wl.dil, groups=wl.groups)
+    else:
+        y = C.conv_fwd(x.cuda(), w.cuda(), stride=wl.stride, padding=wl.pad, dilation=wl.dil, groups=wl.groups)
     torch.cuda.synchronize()
     assert C.last_status() == 0
     rng = np.random.default_rng(0)
     idx = _sample_indices(tuple(y.shape), rng)
-    y_ref, s_ref = oracle.conv_fwd_points(x, w, idx, wl.stride, wl.pad, wl.dil, wl.groups)
+    if wl.transpose:
+        y_ref, s_ref = oracle.conv_transpose_points(x, w, idx, wl.stride, wl.pad, wl.out_pad, wl.dil, wl.groups)
+    else:
+        y_ref, s_ref = oracle.conv_fwd_points(x, w, idx, wl.stride, wl.pad, wl.dil, wl.groups)
     yv = y.reshape(-1)[torch.as_tensor(idx, device="cuda")].cpu()
     assert_parity(yv, y_ref, s_ref, wl.dtype, name)
     assert torch.isfinite(y.float()).all()

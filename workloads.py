@@ -43,6 +43,8 @@ class Workload:
     groups: int = 1
     dtype: str = "f16"
     seed: int = 0
+    transpose: bool = False      # transposed ("upsampling") convolution: x has C channels, y has O
+    out_pad: tuple = (0, 0, 0)   # its output padding
 
     @property
     def x_shape(self):
@@ -50,6 +52,9 @@ class Workload:
 
     @property
     def w_shape(self):
+        # forward: [O, k, C/groups]; transposed: [C, k, O/groups] (the forward layout with O = C)
+        if self.transpose:
+            return (self.C, *self.k, self.O // self.groups)
         return (self.O, *self.k, self.C // self.groups)
 
     def with_(self, **kw):
@@ -98,12 +103,27 @@ WORKLOADS["dwconv_f16_n32_112x112_c128_k3"] = Workload(
     "dwconv_f16_n32_112x112_c128_k3", 32, 1, 112, 112, 128, 128, (1, 3, 3), (1, 1, 1), (0, 1, 1),
     groups=128, dtype="f16", seed=5)
 
+# Transposed convolution 4x4/2/1 (a decoder's 2x upsampling layer), 256 -> 128
+# channels, 56x56 -> 112x112, N=16, bf16, seed 6: the tutorial's variants
+# table names transposed convolutions for decoders and diffusion models.
+WORKLOADS["convT_bf16_n16_56x56_c256_o128_k4s2"] = Workload(
+    "convT_bf16_n16_56x56_c256_o128_k4s2", 16, 1, 56, 56, 256, 128, (1, 4, 4), (1, 2, 2), (0, 1, 1),
+    dtype="bf16", seed=6, transpose=True)
+
 # Name of the workload the benchmark times by default: the tutorial's
 # arithmetic-intensity example (3x3, 256->256, 56x56) at batch 64.
 HEADLINE = "conv2d_bf16_n64_56x56_c256_o256_k3"
 
 
 def fan_in(wl: Workload) -> int:
+    """Inputs summed into one output: C/groups x taps (forward), or the
+    transposed pass's input channels per group x the taps that reach an
+    output (taps / stride per dimension, rounded up)."""
+    if wl.transpose:
+        reach = 1
+        for k, s in zip(wl.k, wl.stride):
+            reach *= -(-k // s)
+        return (wl.C // wl.groups) * reach
     return (wl.C // wl.groups) * wl.k[0] * wl.k[1] * wl.k[2]
 
 
