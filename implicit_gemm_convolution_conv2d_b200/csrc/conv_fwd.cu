@@ -226,6 +226,10 @@ int set_kernel_attrs(int dev) {
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_TMA, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, false, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_kernel<MODE_GATHER, true, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -690,6 +694,68 @@ int plan_phase(const Problem& P, int sms, TcPlan& plan) {
   return CONV_OK;
 }
 
+// Sub-pixel phases of a transposed convolution on the gather kernel: output
+// pixel q (per dimension) is reached only by taps k with
+// (q - p_lo + k*d) divisible by the input dilation s, and that set depends on
+// q mod s alone.  Each phase gets its own m tiles and reads only its taps, so
+// no MMA multiplies an inserted zero.  Needs 64-channel K blocks (Cg % 64 ==
+// 0, one tap per K block) and at most kMaxTp non-empty phases.
+bool plan_tp(const Problem& P, TcArgs& a) {
+  if (!P.wtrans || a.gather_mode != GATHER_VEC8 || P.Cg % 64 != 0) return false;
+  if (P.idil[0] == 1 && P.idil[1] == 1 && P.idil[2] == 1) return false;
+  const int k[3] = {P.kD, P.kH, P.kW};
+  const int Q[3] = {P.Do, P.Ho, P.Wo};
+  int A[3][64], k0[3][64], nk[3][64];
+  for (int i = 0; i < 3; ++i) {
+    const int sd = P.idil[i];
+    if (sd > 64) return false;
+    int g = sd, b = P.d[i];
+    while (b) { const int t = g % b; g = b; b = t; }  // gcd(s, d)
+    a.tp_step[i] = sd / g;
+    for (int r = 0; r < sd; ++r) {
+      A[i][r] = r < Q[i] ? (Q[i] - r + sd - 1) / sd : 0;
+      k0[i][r] = 0;
+      nk[i][r] = 0;
+      for (int kk = 0; kk < k[i]; ++kk) {
+        const long long v = static_cast<long long>(r) - P.p[i] + static_cast<long long>(kk) * P.d[i];
+        if (((v % sd) + sd) % sd == 0) {
+          if (nk[i][r] == 0) k0[i][r] = kk;
+          ++nk[i][r];
+        }
+      }
+    }
+  }
+  int count = 0;
+  long long tiles = 0;
+  for (int rd = 0; rd < P.idil[0]; ++rd)
+    for (int rh = 0; rh < P.idil[1]; ++rh)
+      for (int rw = 0; rw < P.idil[2]; ++rw) {
+        const long long Mph = static_cast<long long>(P.N) * A[0][rd] * A[1][rh] * A[2][rw];
+        if (Mph == 0) continue;
+        if (count == kMaxTp || Mph > 0x7fffffffLL - kBM) return false;
+        const int rr[3] = {rd, rh, rw};
+        for (int i = 0; i < 3; ++i) {
+          a.tp_r[count][i] = rr[i];
+          a.tp_A[count][i] = A[i][rr[i]];
+          a.tp_k0[count][i] = k0[i][rr[i]];
+          a.tp_nk[count][i] = nk[i][rr[i]];
+        }
+        a.tp_tbase[count] = static_cast<int>(tiles);
+        tiles += (Mph + kBM - 1) / kBM;
+        if (tiles > 0x7fffffffLL) return false;
+        ++count;
+      }
+  a.tp_tbase[count] = static_cast<int>(tiles);
+  a.tp_count = count;
+  a.tp_cpt = P.Cg / 64;
+  a.m_tiles = static_cast<int>(tiles);
+  const long long tt = tiles * a.n_tiles * P.G;
+  if (tt > 0x7fffffffLL) return false;
+  a.total_tiles = static_cast<int>(tt);
+  a.tp_on = 1;
+  return true;
+}
+
 int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
   // input dilation and transposed weights: the gather kernel only
   if (!plain_input(P) && variant != CONV_VARIANT_TC_GATHER) return CONV_EUNSUPPORTED;
@@ -778,6 +844,7 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
     a.Kp = static_cast<int>(kp);
     a.kblocks = static_cast<int>((kp + 63) / 64);
   }
+  if (variant == CONV_VARIANT_TC_GATHER) plan_tp(P, a);
   a.x_elems = static_cast<long long>(P.x_bytes / P.esize);
   a.idil_on = plain_input(P) ? 0 : 1;
   a.idd = P.idil[0]; a.idh = P.idil[1]; a.idw = P.idil[2];
@@ -1447,8 +1514,16 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
     if (bf) conv_fwd_tc_kernel<MODE_TMA, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
     else    conv_fwd_tc_kernel<MODE_TMA, false><<<grid, block, plan.smem, st>>>(mx, mw, a);
   } else {
-    if (bf) conv_fwd_tc_kernel<MODE_GATHER, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
-    else    conv_fwd_tc_kernel<MODE_GATHER, false><<<grid, block, plan.smem, st>>>(mx, mw, a);
+    if (a.tp_on) {
+      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true, true, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
+      else    conv_fwd_tc_kernel<MODE_GATHER, false, true, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
+    } else if (a.idil_on || a.wtrans) {
+      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
+      else    conv_fwd_tc_kernel<MODE_GATHER, false, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
+    } else {
+      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
+      else    conv_fwd_tc_kernel<MODE_GATHER, false><<<grid, block, plan.smem, st>>>(mx, mw, a);
+    }
   }
   return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }

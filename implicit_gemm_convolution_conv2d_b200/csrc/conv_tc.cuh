@@ -40,6 +40,7 @@
 namespace convfwd {
 
 constexpr int kMaxStages = 16;
+constexpr int kMaxTp = 16;  // transposed-convolution phases the gather kernel tracks
 constexpr int kBM = 128;
 
 // Device status word, one per device; bit 0 = a pipeline wait timed out.
@@ -118,6 +119,19 @@ struct TcArgs {
   uint32_t ph_bblk;    // one resident B block: N rows x 32 bytes
   uint32_t ph_epi_bytes;  // one epilogue staging tile
   int ph_gcols;        // output columns per epilogue store (64: 128-byte swizzle, 32: 64-byte)
+  // transposed convolution by sub-pixel phases (gather kernel, VEC8, Cg % 64
+  // == 0): output pixels are grouped by their position modulo the input
+  // dilation (the transposed stride); a tile holds pixels of one phase and
+  // reads only the taps that reach that phase (the others would multiply the
+  // inserted zeros)
+  int tp_on;
+  int tp_count;                          // phases with at least one output pixel
+  int tp_cpt;                            // 64-wide K blocks per tap (Cg / 64)
+  int tp_step[3];                        // tap step per dimension: s / gcd(s, d)
+  int tp_r[kMaxTp][3];                   // phase residues (output position mod s)
+  int tp_A[kMaxTp][3];                   // output extent of the phase per dimension
+  int tp_k0[kMaxTp][3], tp_nk[kMaxTp][3];  // first valid tap and valid taps per dimension
+  int tp_tbase[kMaxTp + 1];              // first m tile of each phase
   const void* x;
   const void* w;
   void* y;
@@ -202,6 +216,41 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, unsign
 struct TileCoord {
   int g, mt, nt;
 };
+
+// Transposed-convolution phases: the phase of m tile `mt`, its K-block count,
+// its j-th K block, and the output pixel of its local row (false past the
+// phase's pixels).
+__device__ __forceinline__ int tp_phase(const TcArgs& a, int mt) {
+  int ph = 0;
+  while (ph + 1 < a.tp_count && mt >= a.tp_tbase[ph + 1]) ++ph;
+  return ph;
+}
+__device__ __forceinline__ int tp_nkb(const TcArgs& a, int ph) {
+  return a.tp_nk[ph][0] * a.tp_nk[ph][1] * a.tp_nk[ph][2] * a.tp_cpt;
+}
+__device__ __forceinline__ int tp_kb(const TcArgs& a, int ph, int j) {
+  const int ti = j / a.tp_cpt, chunk = j - (j / a.tp_cpt) * a.tp_cpt;
+  const int tw = ti % a.tp_nk[ph][2];
+  const int t2 = ti / a.tp_nk[ph][2];
+  const int th = t2 % a.tp_nk[ph][1];
+  const int td = t2 / a.tp_nk[ph][1];
+  const int kd = a.tp_k0[ph][0] + td * a.tp_step[0];
+  const int kh = a.tp_k0[ph][1] + th * a.tp_step[1];
+  const int kw = a.tp_k0[ph][2] + tw * a.tp_step[2];
+  return ((kd * a.kH + kh) * a.kW + kw) * a.tp_cpt + chunk;
+}
+__device__ __forceinline__ bool tp_pixel(const TcArgs& a, int ph, int lrow, int& n, int& qd, int& qh, int& qw) {
+  const int Ad = a.tp_A[ph][0], Ah = a.tp_A[ph][1], Aw = a.tp_A[ph][2];
+  const unsigned u = static_cast<unsigned>(lrow);
+  const unsigned t1 = u / static_cast<unsigned>(Aw);
+  const unsigned t2 = t1 / static_cast<unsigned>(Ah);
+  const unsigned t3 = t2 / static_cast<unsigned>(Ad);
+  n = static_cast<int>(t3);
+  qw = a.tp_r[ph][2] + a.idw * static_cast<int>(u - t1 * static_cast<unsigned>(Aw));
+  qh = a.tp_r[ph][1] + a.idh * static_cast<int>(t1 - t2 * static_cast<unsigned>(Ah));
+  qd = a.tp_r[ph][0] + a.idd * static_cast<int>(t2 - t3 * static_cast<unsigned>(Ad));
+  return n < a.N;
+}
 
 __device__ __forceinline__ TileCoord decode_tile(const TcArgs& a, int tile) {
   TileCoord t;
@@ -380,12 +429,13 @@ __device__ __forceinline__ bool undilate(int& z, int s, int n) {
 
 // One filter row (kd, kh) of one output pixel: offset of x[n, id, ih, 0, g*Cg]
 // and whether that input row exists.
+template <bool TR = false>
 __device__ __forceinline__ bool gather_span(const TcArgs& a, const GatherRow& st, int kd, int kh,
                                             long long& rowptr) {
   int id = st.id0 + kd * a.dd;
   int ih = st.ih0 + kh * a.dh;
   bool ok;
-  if (a.idil_on) {
+  if (TR && a.idil_on) {
     ok = st.valid && kd < a.kD && undilate(id, a.idd, a.D) && undilate(ih, a.idh, a.H);
   } else {
     ok = st.valid && kd < a.kD && static_cast<unsigned>(id) < static_cast<unsigned>(a.D) &&
@@ -396,8 +446,9 @@ __device__ __forceinline__ bool gather_span(const TcArgs& a, const GatherRow& st
 }
 
 // Input column of one tap: the element index (in place) and whether it exists.
+template <bool TR = false>
 __device__ __forceinline__ bool gather_col(const TcArgs& a, int& iw) {
-  if (a.idil_on) return undilate(iw, a.idw, a.W);
+  if (TR && a.idil_on) return undilate(iw, a.idw, a.W);
   return static_cast<unsigned>(iw) < static_cast<unsigned>(a.W);
 }
 
@@ -424,7 +475,7 @@ __device__ __forceinline__ uint4 load8_masked(const uint16_t* p, int e_lo, int e
 // GATHER_SCALAR: element-wise (kw, c) walk with its own bounds check.
 enum { GATHER_SCALAR = 0, GATHER_VEC8 = 1, GATHER_SPAN = 2, GATHER_ROWS = 3 };
 
-template <int NCH>
+template <int NCH, bool TR = false>
 __device__ __forceinline__ void gather_a_vec8(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
                                               int r, int chunk0) {
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
@@ -435,13 +486,13 @@ __device__ __forceinline__ void gather_a_vec8(const TcArgs& a, const GatherRow& 
   int kh = t2 % a.kH;
   int kd = t2 / a.kH;
   long long rowptr;
-  bool rok = gather_span(a, st, kd, kh, rowptr);
+  bool rok = gather_span<TR>(a, st, kd, kh, rowptr);
   uint4 v[NCH];
 #pragma unroll
   for (int q = 0; q < NCH; ++q) {
     int iw = st.iw0 + kw * a.dw;
     v[q] = make_uint4(0, 0, 0, 0);
-    if (rok && gather_col(a, iw))
+    if (rok && gather_col<TR>(a, iw))
       v[q] = __ldg(reinterpret_cast<const uint4*>(x + rowptr + static_cast<long long>(iw) * a.C + c));
     c += 8;
     if (c == a.Cg) {
@@ -452,7 +503,7 @@ __device__ __forceinline__ void gather_a_vec8(const TcArgs& a, const GatherRow& 
           kh = 0;
           ++kd;
         }
-        rok = gather_span(a, st, kd, kh, rowptr);
+        rok = gather_span<TR>(a, st, kd, kh, rowptr);
       }
     }
   }
@@ -610,7 +661,7 @@ __device__ __forceinline__ void gather_a_rows(const TcArgs& a, const GatherRow& 
   for (int q = 0; q < NCH; ++q) store_chunk(a_tile, r, chunk0 + q, v[q]);
 }
 
-template <int NCH>
+template <int NCH, bool TR = false>
 __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow& st, int k0, uint8_t* a_tile,
                                                 int r, int chunk0) {
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
@@ -622,11 +673,11 @@ __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow
   int kh = t2 % a.kH;
   int kd = t2 / a.kH;
   long long rowptr;
-  bool ok = gather_span(a, st, kd, kh, rowptr);
+  bool ok = gather_span<TR>(a, st, kd, kh, rowptr);
 #pragma unroll
   for (int e = 0; e < 8 * NCH; ++e) {
     int iw = st.iw0 + kw * a.dw;
-    v[e] = (ok && gather_col(a, iw)) ? __ldg(x + rowptr + static_cast<long long>(iw) * a.C + c) : 0u;
+    v[e] = (ok && gather_col<TR>(a, iw)) ? __ldg(x + rowptr + static_cast<long long>(iw) * a.C + c) : 0u;
     if (++c == a.Cg) {
       c = 0;
       if (++kw == a.kW) {
@@ -635,7 +686,7 @@ __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow
           kh = 0;
           ++kd;
         }
-        ok = gather_span(a, st, kd, kh, rowptr);
+        ok = gather_span<TR>(a, st, kd, kh, rowptr);
       }
     }
   }
@@ -650,9 +701,49 @@ __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow
 // starting at n0, into a swizzled BN x 128-byte tile.  `nthreads` threads
 // share the 8*BN chunks.  In span layout, padded K element kp of filter row
 // s = kp / Lp, offset j = kp % Lp, is w[o, s*kW*C + j] for j < kW*C, else 0.
+template <bool TR = false>
 __device__ __forceinline__ void gather_b_block(const TcArgs& a, int g, int n0, int kbase, uint8_t* b_tile,
                                                int tid, int nthreads) {
   const uint16_t* __restrict__ w = static_cast<const uint16_t*>(a.w);
+  if (TR && a.wtrans && (a.Cg & 7) == 0 && (a.Og & 7) == 0) {
+    // Transposed weights [G*Cg][taps][Og], 8-aligned channel counts: a thread
+    // takes 8 B rows (output channels) x one 8-element K chunk (8 channels c of
+    // one tap); the 8 channels' rows of 8 output channels are 16-byte loads,
+    // transposed in registers into the 8 rows' chunks.
+#pragma unroll 1
+    for (int q = tid; q < a.BN; q += nthreads) {
+      const int rg = q >> 3, ch = q & 7;
+      const int oc0 = n0 + rg * 8;
+      const int kp0 = kbase + ch * 8;
+      uint32_t in[8][4];
+      if (oc0 < a.Og && kp0 < a.K) {
+        const int tap = kp0 / a.Cg;
+        const int c0 = kp0 - tap * a.Cg;
+        const long long base = (static_cast<long long>(g * a.Cg + c0) * a.taps + wtap(a, tap)) * a.Og + oc0;
+        const long long pitch = static_cast<long long>(a.taps) * a.Og;  // between consecutive channels c
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(w + base + e * pitch));
+          in[e][0] = v.x; in[e][1] = v.y; in[e][2] = v.z; in[e][3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) in[e][0] = in[e][1] = in[e][2] = in[e][3] = 0u;
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        // row r (output channel oc0 + r): halfword r of each channel's vector
+        const uint32_t sel = (r & 1) ? 0x7632u : 0x5410u;
+        uint4 o;
+        o.x = __byte_perm(in[0][r >> 1], in[1][r >> 1], sel);
+        o.y = __byte_perm(in[2][r >> 1], in[3][r >> 1], sel);
+        o.z = __byte_perm(in[4][r >> 1], in[5][r >> 1], sel);
+        o.w = __byte_perm(in[6][r >> 1], in[7][r >> 1], sel);
+        *reinterpret_cast<uint4*>(b_tile + sw128_offset(rg * 8 + r, ch)) = o;
+      }
+    }
+    return;
+  }
   const bool span_layout = a.gather_mode == GATHER_SPAN || a.gather_mode == GATHER_ROWS;
   const bool vec = (a.K & 7) == 0 && !span_layout;
   const int L = a.kW * a.C;
@@ -664,7 +755,7 @@ __device__ __forceinline__ void gather_b_block(const TcArgs& a, int g, int n0, i
     uint4 v = make_uint4(0, 0, 0, 0);
     if (oc < a.Og && kp0 < a.Kp) {
       const long long rowoff = static_cast<long long>(g * a.Og + oc) * a.K;
-      if (a.wtrans) {
+      if (TR && a.wtrans) {
         // w stored [G*Cg][taps][Og]: K element k = tap*Cg + c of output
         // channel oc multiplies w[g*Cg + c][tap (mirrored under flip)][oc]
         uint16_t e8[8];
@@ -746,7 +837,10 @@ __device__ __forceinline__ void issue_rows(const TcArgs& a, const CUtensorMap* t
 // ----------------------------------------------------------------------------
 // The kernel.
 // ----------------------------------------------------------------------------
-template <int MODE, bool BF16>
+// TR: the transposed-convolution gather (input dilation, transposed weights);
+// TP: with sub-pixel phases.  Separate instantiations, so that the forward
+// gather kernel keeps its registers.
+template <int MODE, bool BF16, bool TR = false, bool TP = false>
 __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
     conv_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
                        const __grid_constant__ CUtensorMap tmap_w, const TcArgs a) {
@@ -874,7 +968,7 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
       if (a.b_resident) {
         // the whole B matrix, once per CTA: [kblock][BN rows][128 B]
         for (int kb = 0; kb < a.kblocks; ++kb)
-          gather_b_block(a, 0, 0, kb * 64, bres + static_cast<uint32_t>(kb) * a.BN * 128u, tid,
+          gather_b_block<TR>(a, 0, 0, kb * 64, bres + static_cast<uint32_t>(kb) * a.BN * 128u, tid,
                          kProdThreads);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(ptx::smem_u32(&tail->bres));
@@ -894,10 +988,18 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
           break;
         }
         GatherRow st;
-        const long long m = static_cast<long long>(tc.mt) * kBM + r;
-        st.valid = m < a.M;
         int n = 0, od = 0, oh = 0, ow = 0;
-        if (st.valid) decode_pixel(a, m, n, od, oh, ow);
+        int tph = 0, nkb = a.kblocks;
+        if constexpr (TP) {
+          tph = tp_phase(a, tc.mt);
+          nkb = tp_nkb(a, tph);
+          st.valid = tp_pixel(a, tph, (tc.mt - a.tp_tbase[tph]) * kBM + r, n, od, oh, ow);
+          if (!st.valid) n = od = oh = ow = 0;
+        } else {
+          const long long m = static_cast<long long>(tc.mt) * kBM + r;
+          st.valid = m < a.M;
+          if (st.valid) decode_pixel(a, m, n, od, oh, ow);
+        }
         st.nbase = static_cast<long long>(n) * a.D * a.H * a.W * a.C + static_cast<long long>(tc.g) * a.Cg;
         st.id0 = od * a.sd - a.pd;
         st.ih0 = oh * a.sh - a.ph;
@@ -913,8 +1015,8 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
         // this thread's first K element of every 64-wide K block
         SpanPos pos = span_pos(a, part * kNch * 8);
         const int n0 = tc.nt * a.BN;
-        for (int kb = 0; kb < a.kblocks; kb += a.kbs) {
-          const int nsub = min(a.kbs, a.kblocks - kb);
+        for (int kb = 0; kb < nkb; kb += a.kbs) {
+          const int nsub = min(a.kbs, nkb - kb);
           if (!wait_bounded(ptx::smem_u32(&tail->empty[stage]), phase ^ 1u, abort_flag, a.timeout_ns,
                             kSiteProducerEmpty)) {
             ok = false;
@@ -922,17 +1024,18 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
           }
           for (int j = 0; j < nsub; ++j) {
             uint8_t* sa = smem + stage * a.stage_bytes + j * a.sub_bytes;
-            const int k0 = (kb + j) * 64 + part * kNch * 8;
+            const int kbm = TP ? tp_kb(a, tph, kb + j) : kb + j;  // the K block loaded
+            const int k0 = kbm * 64 + part * kNch * 8;
             if (a.gather_mode == GATHER_VEC8)
-              gather_a_vec8<kNch>(a, st, k0, sa, r, part * kNch);
+              gather_a_vec8<kNch, TR>(a, st, k0, sa, r, part * kNch);
             else if (rows_mode || a.gather_mode == GATHER_SPAN) {
               if (rows_mode) gather_a_rows<kNch>(a, st, pos, sa, r, part * kNch);
               else gather_a_span<kNch>(a, st, pos, sa, r, part * kNch);
               // skip the other threads' chunks of this K block
               for (int i = 0; i < 8 - kNch; ++i) span_step8(a, pos);
             } else
-              gather_a_scalar<kNch>(a, st, k0, sa, r, part * kNch);
-            if (!a.b_resident) gather_b_block(a, tc.g, n0, (kb + j) * 64, sa + a.a_bytes, tid, kProdThreads);
+              gather_a_scalar<kNch, TR>(a, st, k0, sa, r, part * kNch);
+            if (!a.b_resident) gather_b_block<TR>(a, tc.g, n0, kbm * 64, sa + a.a_bytes, tid, kProdThreads);
           }
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(ptx::smem_u32(&tail->full[stage]));
@@ -989,8 +1092,13 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * a.BN);
-        for (int kb = 0; kb < a.kblocks; kb += a.kbs) {
-          const int nsub = min(a.kbs, a.kblocks - kb);
+        int tph = 0, nkb = a.kblocks;
+        if constexpr (TP) {
+          tph = tp_phase(a, decode_tile(a, tile).mt);
+          nkb = tp_nkb(a, tph);  // 0: no tap reaches the phase, the epilogue writes zeros
+        }
+        for (int kb = 0; kb < nkb; kb += a.kbs) {
+          const int nsub = min(a.kbs, nkb - kb);
           if (!wait_bounded(ptx::smem_u32(&tail->full[stage]), phase, abort_flag, a.timeout_ns,
                             kSiteMmaFull)) {
             ok = false;
@@ -999,7 +1107,8 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
           ptx::tc_fence_after();
           uint64_t da = d_ring + static_cast<uint64_t>(stage) * st_off;
           for (int j = 0; j < nsub; ++j) {
-            const uint64_t db = a.b_resident ? d_res + static_cast<uint64_t>(kb + j) * res_step : da + a_off;
+            const int kbm = TP ? tp_kb(a, tph, kb + j) : kb + j;
+            const uint64_t db = a.b_resident ? d_res + static_cast<uint64_t>(kbm) * res_step : da + a_off;
             mma_sub<false>(ksteps, d_tmem, da, db, a.idesc, (kb + j) != 0 ? 1u : 0u);
             da += sub_off;
           }
@@ -1030,18 +1139,32 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
         break;
       ptx::tc_fence_after();
       const TileCoord tc = decode_tile(a, tile);
-      const long long m = static_cast<long long>(tc.mt) * kBM + row;
+      long long m = static_cast<long long>(tc.mt) * kBM + row;
+      bool mvalid = m < a.M;
+      bool zero = false;  // a phase no tap reaches: its outputs are 0
+      if constexpr (TP) {
+        const int tph = tp_phase(a, tc.mt);
+        int n, qd, qh, qw;
+        mvalid = tp_pixel(a, tph, (tc.mt - a.tp_tbase[tph]) * kBM + row, n, qd, qh, qw);
+        m = mvalid ? ((static_cast<long long>(n) * a.Do + qd) * a.Ho + qh) * a.Wo + qw : 0;
+        zero = tp_nkb(a, tph) == 0;
+      }
       const int n0 = tc.nt * a.BN;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * a.BN);
       const long long ybase = m * a.O + static_cast<long long>(tc.g) * a.Og;
       for (int c = 0; c < a.BN; c += 32) {
         uint32_t r[32];
-        ptx::tmem_ld_32x32b_x32(taddr + c, r);
-        ptx::tmem_ld_wait();
+        if (zero) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = 0u;  // +0.0f
+        } else {
+          ptx::tmem_ld_32x32b_x32(taddr + c, r);
+          ptx::tmem_ld_wait();
+        }
         const int col0 = n0 + c;
         const int nvalid = min(32, a.Og - col0);
-        if (m < a.M && nvalid > 0) {
+        if (mvalid && nvalid > 0) {
           uint16_t* dst = y + ybase + col0;
           if (nvalid == 32 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
             uint4* d4 = reinterpret_cast<uint4*>(dst);

@@ -275,6 +275,15 @@ TRANSPOSE = [
     ("t_s3_d2", 1, 1, 6, 5, 16, 8, (1, 3, 3), (1, 3, 3), (0, 2, 1), (0, 2, 1), (1, 2, 2), 1),
     ("t_groups4", 2, 1, 8, 9, 32, 32, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1), 4),
     ("t_ragged_tiles", 2, 1, 20, 17, 24, 40, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+    # sub-pixel phases (64-channel K blocks): phases with 1 and 2 taps per
+    # dimension, phases no tap reaches (written as zeros), 3-D, groups, dilation
+    ("tp_k4s2_c64", 2, 1, 9, 11, 64, 32, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1),
+    ("tp_k3s2_op1_c128", 1, 1, 10, 7, 128, 64, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+    ("tp_k1s2_zero_phases", 2, 1, 6, 5, 64, 16, (1, 1, 1), (1, 2, 2), (0, 0, 0), (0, 1, 1), (1, 1, 1), 1),
+    ("tp_3d", 1, 3, 5, 6, 64, 16, (2, 3, 3), (2, 2, 1), (0, 1, 1), (1, 1, 0), (1, 1, 1), 1),
+    ("tp_groups2", 1, 1, 7, 6, 128, 64, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 2),
+    ("tp_dil2_s2", 1, 1, 6, 6, 64, 32, (1, 3, 3), (1, 2, 2), (0, 2, 2), (0, 1, 1), (1, 2, 2), 1),
+    ("tp_s3_k5", 1, 1, 5, 6, 64, 24, (1, 5, 5), (1, 3, 3), (0, 2, 2), (0, 2, 1), (1, 1, 1), 1),
 ]
 
 
