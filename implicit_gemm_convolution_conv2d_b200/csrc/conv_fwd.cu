@@ -705,21 +705,26 @@ bool plan_tp(const Problem& P, TcArgs& a) {
   if (P.idil[0] == 1 && P.idil[1] == 1 && P.idil[2] == 1) return false;
   const int k[3] = {P.kD, P.kH, P.kW};
   const int Q[3] = {P.Do, P.Ho, P.Wo};
-  int A[3][64], k0[3][64], nk[3][64];
+  int A[3][64], k0[3][64], nk[3][64], c0[3][64];
   for (int i = 0; i < 3; ++i) {
     const int sd = P.idil[i];
     if (sd > 64) return false;
     int g = sd, b = P.d[i];
     while (b) { const int t = g % b; g = b; b = t; }  // gcd(s, d)
     a.tp_step[i] = sd / g;
+    a.tp_dstep[i] = P.d[i] / g;
     for (int r = 0; r < sd; ++r) {
       A[i][r] = r < Q[i] ? (Q[i] - r + sd - 1) / sd : 0;
       k0[i][r] = 0;
       nk[i][r] = 0;
+      c0[i][r] = 0;
       for (int kk = 0; kk < k[i]; ++kk) {
         const long long v = static_cast<long long>(r) - P.p[i] + static_cast<long long>(kk) * P.d[i];
         if (((v % sd) + sd) % sd == 0) {
-          if (nk[i][r] == 0) k0[i][r] = kk;
+          if (nk[i][r] == 0) {
+            k0[i][r] = kk;
+            c0[i][r] = static_cast<int>(v / sd);  // exact
+          }
           ++nk[i][r];
         }
       }
@@ -739,6 +744,7 @@ bool plan_tp(const Problem& P, TcArgs& a) {
           a.tp_A[count][i] = A[i][rr[i]];
           a.tp_k0[count][i] = k0[i][rr[i]];
           a.tp_nk[count][i] = nk[i][rr[i]];
+          a.tp_c0[count][i] = c0[i][rr[i]];
         }
         a.tp_tbase[count] = static_cast<int>(tiles);
         tiles += (Mph + kBM - 1) / kBM;

@@ -131,6 +131,8 @@ struct TcArgs {
   int tp_r[kMaxTp][3];                   // phase residues (output position mod s)
   int tp_A[kMaxTp][3];                   // output extent of the phase per dimension
   int tp_k0[kMaxTp][3], tp_nk[kMaxTp][3];  // first valid tap and valid taps per dimension
+  int tp_c0[kMaxTp][3];                  // input offset of the first valid tap: (r - p_lo + k0*d) / s
+  int tp_dstep[3];                       // input offset between consecutive valid taps: d / gcd(s, d)
   int tp_tbase[kMaxTp + 1];              // first m tile of each phase
   const void* x;
   const void* w;
@@ -239,6 +241,20 @@ __device__ __forceinline__ int tp_kb(const TcArgs& a, int ph, int j) {
   const int kw = a.tp_k0[ph][2] + tw * a.tp_step[2];
   return ((kd * a.kH + kh) * a.kW + kw) * a.tp_cpt + chunk;
 }
+// Local row of a phase -> image n and the phase-local output position (ad, ah, aw).
+__device__ __forceinline__ bool tp_local(const TcArgs& a, int ph, int lrow, int& n, int& ad, int& ah, int& aw) {
+  const int Ad = a.tp_A[ph][0], Ah = a.tp_A[ph][1], Aw = a.tp_A[ph][2];
+  const unsigned u = static_cast<unsigned>(lrow);
+  const unsigned t1 = u / static_cast<unsigned>(Aw);
+  const unsigned t2 = t1 / static_cast<unsigned>(Ah);
+  const unsigned t3 = t2 / static_cast<unsigned>(Ad);
+  n = static_cast<int>(t3);
+  aw = static_cast<int>(u - t1 * static_cast<unsigned>(Aw));
+  ah = static_cast<int>(t1 - t2 * static_cast<unsigned>(Ah));
+  ad = static_cast<int>(t2 - t3 * static_cast<unsigned>(Ad));
+  return n < a.N;
+}
+
 __device__ __forceinline__ bool tp_pixel(const TcArgs& a, int ph, int lrow, int& n, int& qd, int& qh, int& qw) {
   const int Ad = a.tp_A[ph][0], Ah = a.tp_A[ph][1], Aw = a.tp_A[ph][2];
   const unsigned u = static_cast<unsigned>(lrow);
@@ -697,6 +713,36 @@ __device__ __forceinline__ void gather_a_scalar(const TcArgs& a, const GatherRow
                            v[8 * q + 4] | (v[8 * q + 5] << 16), v[8 * q + 6] | (v[8 * q + 7] << 16)));
 }
 
+// Sub-pixel phase tiles of a transposed convolution: the j-th K block of
+// phase ph is 64 channels of one valid tap, whose input pixel is the row's
+// phase-local position (held in st.id0/ih0/iw0) plus the tap's offset, with
+// no division; NCH 16-byte chunks of that pixel.
+template <int NCH>
+__device__ __forceinline__ void gather_a_tp(const TcArgs& a, const GatherRow& st, int ph, int j, uint8_t* a_tile,
+                                            int r, int chunk0) {
+  const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
+  const int ti = j / a.tp_cpt;
+  const int cblk = j - ti * a.tp_cpt;
+  const int tw = ti % a.tp_nk[ph][2];
+  const int t2 = ti / a.tp_nk[ph][2];
+  const int th = t2 % a.tp_nk[ph][1];
+  const int td = t2 / a.tp_nk[ph][1];
+  const int id = st.id0 + a.tp_c0[ph][0] + td * a.tp_dstep[0];
+  const int ih = st.ih0 + a.tp_c0[ph][1] + th * a.tp_dstep[1];
+  const int iw = st.iw0 + a.tp_c0[ph][2] + tw * a.tp_dstep[2];
+  const bool ok = st.valid && static_cast<unsigned>(id) < static_cast<unsigned>(a.D) &&
+                  static_cast<unsigned>(ih) < static_cast<unsigned>(a.H) &&
+                  static_cast<unsigned>(iw) < static_cast<unsigned>(a.W);
+  const long long p = st.nbase + ((static_cast<long long>(ok ? id : 0) * a.H + (ok ? ih : 0)) * a.W + (ok ? iw : 0)) *
+                                     static_cast<long long>(a.C) +
+                      cblk * 64 + chunk0 * 8;
+#pragma unroll
+  for (int q = 0; q < NCH; ++q) {
+    const uint4 v = ok ? __ldg(reinterpret_cast<const uint4*>(x + p + q * 8)) : make_uint4(0, 0, 0, 0);
+    store_chunk(a_tile, r, chunk0 + q, v);
+  }
+}
+
 // B rows [0, BN) x K elements [kbase, kbase+64) of group g, output channels
 // starting at n0, into a swizzled BN x 128-byte tile.  `nthreads` threads
 // share the 8*BN chunks.  In span layout, padded K element kp of filter row
@@ -991,9 +1037,10 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
         int n = 0, od = 0, oh = 0, ow = 0;
         int tph = 0, nkb = a.kblocks;
         if constexpr (TP) {
+          // od, oh, ow: the phase-local output position (input offsets are added per tap)
           tph = tp_phase(a, tc.mt);
           nkb = tp_nkb(a, tph);
-          st.valid = tp_pixel(a, tph, (tc.mt - a.tp_tbase[tph]) * kBM + r, n, od, oh, ow);
+          st.valid = tp_local(a, tph, (tc.mt - a.tp_tbase[tph]) * kBM + r, n, od, oh, ow);
           if (!st.valid) n = od = oh = ow = 0;
         } else {
           const long long m = static_cast<long long>(tc.mt) * kBM + r;
@@ -1001,9 +1048,15 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
           if (st.valid) decode_pixel(a, m, n, od, oh, ow);
         }
         st.nbase = static_cast<long long>(n) * a.D * a.H * a.W * a.C + static_cast<long long>(tc.g) * a.Cg;
-        st.id0 = od * a.sd - a.pd;
-        st.ih0 = oh * a.sh - a.ph;
-        st.iw0 = ow * a.sw - a.pw;
+        if constexpr (TP) {
+          st.id0 = od;
+          st.ih0 = oh;
+          st.iw0 = ow;
+        } else {
+          st.id0 = od * a.sd - a.pd;
+          st.ih0 = oh * a.sh - a.ph;
+          st.iw0 = ow * a.sw - a.pw;
+        }
         st.jlo = max(0, -st.iw0) * a.C;
         st.jhi = min(a.kW, a.W - st.iw0) * a.C;
         if (st.jhi < st.jlo) st.jhi = st.jlo;
@@ -1026,7 +1079,9 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
             uint8_t* sa = smem + stage * a.stage_bytes + j * a.sub_bytes;
             const int kbm = TP ? tp_kb(a, tph, kb + j) : kb + j;  // the K block loaded
             const int k0 = kbm * 64 + part * kNch * 8;
-            if (a.gather_mode == GATHER_VEC8)
+            if (TP)
+              gather_a_tp<kNch>(a, st, tph, kb + j, sa, r, part * kNch);
+            else if (a.gather_mode == GATHER_VEC8)
               gather_a_vec8<kNch, TR>(a, st, k0, sa, r, part * kNch);
             else if (rows_mode || a.gather_mode == GATHER_SPAN) {
               if (rows_mode) gather_a_rows<kNch>(a, st, pos, sa, r, part * kNch);
