@@ -1559,14 +1559,14 @@ SimtShape simt_shape(const Problem& P, int sms) {
   return sh;
 }
 
-template <typename T, int TM>
+template <typename T, int TM, bool TR>
 cudaError_t launch_simt_tn(int tn, dim3 grid, cudaStream_t st, const SimtArgs& a) {
   switch (tn) {
-    case 2: conv_fwd_simt_kernel<T, TM, 2><<<grid, kSimtThreads, 0, st>>>(a); break;
-    case 5: conv_fwd_simt_kernel<T, TM, 5><<<grid, kSimtThreads, 0, st>>>(a); break;
-    case 6: conv_fwd_simt_kernel<T, TM, 6><<<grid, kSimtThreads, 0, st>>>(a); break;
-    case 8: conv_fwd_simt_kernel<T, TM, 8><<<grid, kSimtThreads, 0, st>>>(a); break;
-    default: conv_fwd_simt_kernel<T, TM, 4><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 2: conv_fwd_simt_kernel<T, TM, 2, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 5: conv_fwd_simt_kernel<T, TM, 5, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 6: conv_fwd_simt_kernel<T, TM, 6, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 8: conv_fwd_simt_kernel<T, TM, 8, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
+    default: conv_fwd_simt_kernel<T, TM, 4, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
   }
   return cudaGetLastError();
 }
@@ -1592,13 +1592,16 @@ int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStr
   if (mt > 0x7fffffffLL || nt > 65535 || P.G > 65535) return CONV_EUNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>(nt), P.G);
   cudaError_t e;
+  const bool tr = !plain_input(P);
   if (P.dtype == CONV_F32) {
-    e = launch_simt_tn<float, 4>(sh.tn, grid, st, a);
+    e = tr ? launch_simt_tn<float, 4, true>(sh.tn, grid, st, a) : launch_simt_tn<float, 4, false>(sh.tn, grid, st, a);
   } else if (P.dtype == CONV_F16) {
-    conv_fwd_simt_kernel<__half, 4, 4><<<grid, kSimtThreads, 0, st>>>(a);
+    if (tr) conv_fwd_simt_kernel<__half, 4, 4, true><<<grid, kSimtThreads, 0, st>>>(a);
+    else conv_fwd_simt_kernel<__half, 4, 4><<<grid, kSimtThreads, 0, st>>>(a);
     e = cudaGetLastError();
   } else {
-    conv_fwd_simt_kernel<__nv_bfloat16, 4, 4><<<grid, kSimtThreads, 0, st>>>(a);
+    if (tr) conv_fwd_simt_kernel<__nv_bfloat16, 4, 4, true><<<grid, kSimtThreads, 0, st>>>(a);
+    else conv_fwd_simt_kernel<__nv_bfloat16, 4, 4><<<grid, kSimtThreads, 0, st>>>(a);
     e = cudaGetLastError();
   }
   return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;

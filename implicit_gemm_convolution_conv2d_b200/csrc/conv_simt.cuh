@@ -70,7 +70,9 @@ __device__ __forceinline__ bool simt_undilate(int& z, int s, int n) {
   return z < n;
 }
 
-template <typename T, int TM, int TN>
+// TR: the transposed-convolution form (input dilation, transposed weight
+// layout), a separate instantiation so the forward kernel is unchanged.
+template <typename T, int TM, int TN, bool TR = false>
 __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtArgs a) {
   constexpr int BM = 16 * TM, BN = 16 * TN;
   __shared__ __align__(16) float As[2][kSimtBK][BM + 4];
@@ -131,8 +133,15 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
     for (int i = 0; i < TM; ++i) {
       float v = 0.f;
       int zd = rd0[i] + id, zh = rh0[i] + ih, zw = rw0[i] + iw;
-      if (rvalid[i] && kv && simt_undilate(zd, a.idd, a.D) && simt_undilate(zh, a.idh, a.H) &&
-          simt_undilate(zw, a.idw, a.W))
+      bool in;
+      if constexpr (TR) {
+        in = simt_undilate(zd, a.idd, a.D) && simt_undilate(zh, a.idh, a.H) && simt_undilate(zw, a.idw, a.W);
+      } else {
+        in = static_cast<unsigned>(zd) < static_cast<unsigned>(a.D) &&
+             static_cast<unsigned>(zh) < static_cast<unsigned>(a.H) &&
+             static_cast<unsigned>(zw) < static_cast<unsigned>(a.W);
+      }
+      if (rvalid[i] && kv && in)
         v = to_f32<T>(x[rbase[i] + ((static_cast<long long>(zd) * a.H + zh) * a.W + zw) * a.C + c]);
       ra[i] = v;
     }
@@ -140,7 +149,7 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
     // transposed storage [G*Cg][taps][Og] puts it at ((g*Cg + c)*taps + tap)*Og + o
     const int tapk = (kd * a.kH + kh) * a.kW + kw;
     const int wt = a.flip ? a.taps - 1 - tapk : tapk;
-    if (a.wtrans) {
+    if (TR && a.wtrans) {
       const long long wb = (static_cast<long long>(g * a.Cg + c) * a.taps + wt) * a.Og;
 #pragma unroll
       for (int j = 0; j < TN; ++j) rb[j] = (ovalid[j] && kv) ? to_f32<T>(w[wb + n0 + lr + 16 * j]) : 0.f;

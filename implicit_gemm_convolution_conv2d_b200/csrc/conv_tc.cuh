@@ -457,7 +457,11 @@ __device__ __forceinline__ bool gather_span(const TcArgs& a, const GatherRow& st
     ok = st.valid && kd < a.kD && static_cast<unsigned>(id) < static_cast<unsigned>(a.D) &&
          static_cast<unsigned>(ih) < static_cast<unsigned>(a.H);
   }
-  rowptr = st.nbase + (static_cast<long long>(ok ? id : 0) * a.H + (ok ? ih : 0)) * static_cast<long long>(a.W) * a.C;
+  if (TR) {
+    rowptr = st.nbase + (static_cast<long long>(ok ? id : 0) * a.H + (ok ? ih : 0)) * static_cast<long long>(a.W) * a.C;
+  } else {
+    rowptr = st.nbase + (static_cast<long long>(id) * a.H + ih) * static_cast<long long>(a.W) * a.C;
+  }
   return ok;
 }
 
