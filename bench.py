@@ -87,14 +87,37 @@ def measured_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+# Device and host source files each kernel variant's behaviour depends on: a
+# traffic record taken with ncu stays valid while these files are unchanged.
+_COMMON_SRC = ["conv_fwd.cu", "ptx.cuh", "conv_tc.cuh"]
+KERNEL_SOURCES = {
+    "tcgen05_tma_im2col": _COMMON_SRC,
+    "tcgen05_tma_im2col_pair": _COMMON_SRC,
+    "tcgen05_gather": _COMMON_SRC,
+    "tcgen05_tma_im2col_t": _COMMON_SRC + ["conv_tct.cuh"],
+    "tcgen05_tma_halo": _COMMON_SRC + ["conv_halo.cuh"],
+    "tcgen05_tma_halo_pair": _COMMON_SRC + ["conv_halo.cuh"],
+    "tcgen05_tma_halo_t": _COMMON_SRC + ["conv_halo.cuh", "conv_tct.cuh", "conv_halo_t.cuh"],
+    "tcgen05_tma_halo_t_pair": _COMMON_SRC + ["conv_halo.cuh", "conv_tct.cuh", "conv_halo_t.cuh"],
+    "tcgen05_tma_phase": _COMMON_SRC + ["conv_phase.cuh"],
+    "simt_ffma": ["conv_fwd.cu", "conv_simt.cuh"],
+    "depthwise_tma": _COMMON_SRC + ["conv_simt.cuh", "conv_dw.cuh"],
+    "depthwise_direct": ["conv_fwd.cu", "conv_simt.cuh", "conv_dw.cuh"],
+}
+
+
+def kernel_source_hash(kernel=None):
+    """Short hash of the sources a kernel variant depends on (all CUDA sources
+    when `kernel` is None or unknown)."""
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "implicit_gemm_convolution_conv2d_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    names = KERNEL_SOURCES.get(kernel) if kernel else None
+    if names is None:
+        names = [n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh"))]
+    for name in sorted(names):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:12]
 
 
@@ -113,7 +136,7 @@ def profiled_traffic(workload, variant_name):
     the current kernel source (else None)."""
     if not os.path.isdir(PROFILE_DIR):
         return None
-    src = kernel_source_hash()
+    src = kernel_source_hash(variant_name)
     for name in sorted(os.listdir(PROFILE_DIR)):
         if not name.endswith((".txt", ".md")):
             continue
