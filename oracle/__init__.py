@@ -14,7 +14,8 @@ channels-last layouts of section 7 and of the MLX conv3d pull request's
 benchmark table: x (N, D, H, W, C), w (O, kD, kH, kW, C/groups).
 
 The same file holds the transposed ("upsampling") convolution of the same
-page's variants table, read as the adjoint of the forward pass.
+page's variants table, read as the adjoint of the forward pass, and the
+weight gradient of the forward pass.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against things
 other than itself: the tutorial's worked example, its printed FLOP and byte
@@ -91,6 +92,10 @@ class Oracle:
         lib.oracle_conv_transpose_points.restype = ctypes.c_int
         lib.oracle_convT_out_dims.argtypes = [ctypes.c_int] * 6 + [i3, i3, i3, i3, i3]
         lib.oracle_convT_out_dims.restype = ctypes.c_int
+        # weight gradient: x, dy, dtype, N..kW, stride, pad_lo, pad_hi, dil, groups, dw, s
+        lib.oracle_conv_wgrad.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int] + [ctypes.c_int] * 9 + \
+            [i3, i3, i3, i3, ctypes.c_int, dp, dp]
+        lib.oracle_conv_wgrad.restype = ctypes.c_int
         lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
         lib.oracle_f16_to_f64.restype = ctypes.c_double
         lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
@@ -223,6 +228,31 @@ class Oracle:
         return y, s
 
 
+    def conv_wgrad(self, x, dy, k, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1, pad_hi=None):
+        """Weight gradient of conv_fwd: dw[o, k, c] = sum over pixels of dy * x.
+
+        x: [N, D, H, W, C]; dy: [N, Do, Ho, Wo, O] (one dtype); k = (kD, kH, kW).
+        Returns (dw, S) float64 arrays of shape [O, kD, kH, kW, C/groups].
+        """
+        px, nx, kx = _raw(x)
+        py, ny, ky = _raw(dy)
+        if nx != ny:
+            raise TypeError("oracle: x and dy must share a dtype")
+        N, D, H, W, C = (int(v) for v in kx.shape)
+        O = int(ky.shape[-1])
+        hi = pad if pad_hi is None else pad_hi
+        if tuple(ky.shape[1:4]) != self.out_dims(D, H, W, *k, stride, pad, dil, hi):
+            raise ValueError("oracle: dy's extents do not match the forward pass")
+        dw = np.empty((O, *k, C // groups), dtype=np.float64)
+        s = np.empty_like(dw)
+        dp = ctypes.POINTER(ctypes.c_double)
+        rc = self.lib.oracle_conv_wgrad(px, py, DTYPE_CODE[nx], N, D, H, W, C, O, *k, _i3(stride), _i3(pad),
+                                        _i3(hi), _i3(dil), int(groups), dw.ctypes.data_as(dp), s.ctypes.data_as(dp))
+        if rc:
+            raise ValueError(f"oracle.conv_wgrad failed ({rc})")
+        return dw, s
+
+
 _default = None
 
 
@@ -289,6 +319,11 @@ def conv_transpose_points(x, w, idx, stride=(1, 1, 1), pad=(0, 0, 0), out_pad=(0
     return default().conv_transpose_points(x, w, idx, stride, pad, out_pad, dil, groups)
 
 
+def conv_wgrad(x, dy, k, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1, pad_hi=None):
+    return default().conv_wgrad(x, dy, k, stride, pad, dil, groups, pad_hi)
+
+
+conv_wgrad.__doc__ = Oracle.conv_wgrad.__doc__
 conv_transpose.__doc__ = Oracle.conv_transpose.__doc__
 conv_fwd.__doc__ = Oracle.conv_fwd.__doc__
 conv_fwd_points.__doc__ = Oracle.conv_fwd_points.__doc__

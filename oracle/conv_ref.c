@@ -539,6 +539,72 @@ int oracle_conv_transpose_points(const void* x, const void* w, int dtype,
   return 0;
 }
 
+/* ---- weight gradient ------------------------------------------------------
+ *
+ * The gradient of the forward pass above with respect to its weights, given
+ * the gradient dy of its output (the third of the convolution's three passes;
+ * the data gradient is the transposed convolution above):
+ *
+ *   dw[o, kd, kh, kw, c] = sum over n, od, oh, ow of
+ *       dy[n, od, oh, ow, o] * x[n, od*sd - pd + kd*dd, oh*sh - ph + kh*dh,
+ *                                ow*sw - pw + kw*dw, g*Cg + c]
+ *
+ * with g = o / Og, x = 0 outside the input, padding p_lo below (the index
+ * origin) and the output extent fixed by p_lo + p_hi as in the forward pass.
+ * Written as the plain sum per weight element; S = sum |dy * x| alongside.
+ */
+int oracle_conv_wgrad(const void* x, const void* dy, int dtype, int N, int D,
+                      int H, int W, int C, int O, int kD, int kH, int kW,
+                      const int stride[3], const int pad_lo[3],
+                      const int pad_hi[3], const int dil[3], int groups,
+                      double* dw, double* s) {
+  shape_t sh;
+  if (dtype < 0 || dtype > 2) return -2;
+  if (make_shape(&sh, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil,
+                 groups, 0))
+    return -1;
+  int64_t nx = (int64_t)N * D * H * W * C;
+  int64_t ny = (int64_t)N * sh.Do * sh.Ho * sh.Wo * O;
+  double* xd = decode_all(x, nx, dtype);
+  double* yd = decode_all(dy, ny, dtype);
+  if (!xd || !yd) { free(xd); free(yd); return -3; }
+  const shape_t* t = &sh;
+  const int Cg = C / groups, Og = O / groups;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int o = 0; o < O; ++o)
+    for (int kd = 0; kd < kD; ++kd)
+      for (int kh = 0; kh < t->kH; ++kh)
+        for (int kw = 0; kw < t->kW; ++kw)
+          for (int c = 0; c < Cg; ++c) {
+            const int g = o / Og;
+            double acc = 0.0, mag = 0.0;
+            for (int n = 0; n < t->N; ++n)
+              for (int od = 0; od < t->Do; ++od) {
+                int64_t id = (int64_t)od * t->s[0] - t->p[0] + (int64_t)kd * t->d[0];
+                if (id < 0 || id >= t->D) continue;
+                for (int oh = 0; oh < t->Ho; ++oh) {
+                  int64_t ih = (int64_t)oh * t->s[1] - t->p[1] + (int64_t)kh * t->d[1];
+                  if (ih < 0 || ih >= t->H) continue;
+                  for (int ow = 0; ow < t->Wo; ++ow) {
+                    int64_t iw = (int64_t)ow * t->s[2] - t->p[2] + (int64_t)kw * t->d[2];
+                    if (iw < 0 || iw >= t->W) continue;
+                    double gy = yd[((((int64_t)n * t->Do + od) * t->Ho + oh) * t->Wo + ow) * t->O + o];
+                    double xv = xd[((((int64_t)n * t->D + id) * t->H + ih) * t->W + iw) * t->C +
+                                   (int64_t)g * Cg + c];
+                    acc += gy * xv;
+                    mag += fabs(gy * xv);
+                  }
+                }
+              }
+            int64_t q = ((((int64_t)o * kD + kd) * t->kH + kh) * t->kW + kw) * Cg + c;
+            dw[q] = acc;
+            s[q] = mag;
+          }
+  free(xd);
+  free(yd);
+  return 0;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

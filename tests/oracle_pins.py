@@ -435,8 +435,71 @@ def pin_transpose_delta_upsamples(orc):
     assert np.array_equal(y2.reshape(6, 8), ref2)
 
 
+# ---------------------------------------------------------------------------
+# Weight gradient of the forward pass
+# ---------------------------------------------------------------------------
+
+_W_GEOMS = [
+    # (N, D, H, W, C, O, k, stride, pad_lo, pad_hi, dil, groups)
+    (2, 1, 7, 6, 3, 4, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+    (1, 4, 5, 6, 4, 6, (3, 3, 2), (2, 1, 1), (1, 0, 1), (0, 2, 0), (1, 2, 1), 2),
+    (2, 1, 8, 7, 6, 3, (1, 2, 3), (1, 1, 2), (0, 1, 0), (0, 0, 2), (1, 2, 1), 3),
+]
+
+
+def pin_wgrad_adjoint(orc):
+    """The weight gradient is the adjoint of the forward pass in w:
+    sum(conv(x, w) * dy) == sum(w * wgrad(x, dy)) exactly for integer data."""
+    rng = np.random.default_rng(31)
+    for N, D, H, W, C, O, k, s, p, ph, d, G in _W_GEOMS:
+        x = _t(rng.integers(-4, 5, (N, D, H, W, C)))
+        w = _t(rng.integers(-4, 5, (O, *k, C // G)))
+        y, _ = orc.conv_fwd(x, w, s, p, d, G, pad_hi=ph)
+        dy = _t(rng.integers(-4, 5, y.shape))
+        g, _ = orc.conv_wgrad(x, dy, k, s, p, d, G, pad_hi=ph)
+        assert g.shape == tuple(w.shape)
+        assert float(np.sum(y * dy.double().numpy())) == float(np.sum(w.double().numpy() * g))
+
+
+def pin_wgrad_torch_witness(orc):
+    """torch's float64 autograd of conv3d with respect to the weight agrees
+    (symmetric padding), and so does its magnitude sum with |x|, |dy|."""
+    rng = np.random.default_rng(32)
+    for N, D, H, W, C, O, k, s, p, _, d, G in _W_GEOMS:
+        x = _t(rng.uniform(-1, 1, (N, D, H, W, C)))
+        Do, Ho, Wo = orc.out_dims(D, H, W, *k, s, p, d)
+        dy = _t(rng.uniform(-1, 1, (N, Do, Ho, Wo, O)))
+        g, S = orc.conv_wgrad(x, dy, k, s, p, d, G)
+
+        def torch_grad(xa, dya):
+            xt = torch.as_tensor(xa, dtype=torch.float64).permute(0, 4, 1, 2, 3)
+            wt = torch.zeros((O, C // G, *k), dtype=torch.float64, requires_grad=True)
+            yt = torch.nn.functional.conv3d(xt, wt, stride=s, padding=p, dilation=d, groups=G)
+            yt.backward(torch.as_tensor(dya, dtype=torch.float64).permute(0, 4, 1, 2, 3))
+            return wt.grad.permute(0, 2, 3, 4, 1).numpy()
+
+        try:
+            ref, ref_s = torch_grad(x, dy), torch_grad(x.abs(), dy.abs())
+        except RuntimeError as e:  # dy shaped by the oracle's extents does not fit torch's output
+            raise AssertionError(f"torch rejects the oracle's output extents: {e}") from None
+        assert np.allclose(g, ref, rtol=1e-12, atol=1e-12)
+        assert np.allclose(S, ref_s, rtol=1e-12, atol=1e-12)
+
+
+def pin_wgrad_pointwise_is_matmul(orc):
+    """Closed form: for a 1x1 filter at stride 1 the weight gradient is the
+    matrix product dy^T x over all pixels (exact on integer data)."""
+    rng = np.random.default_rng(33)
+    x = rng.integers(-4, 5, (2, 3, 4, 5, 6))
+    dy = rng.integers(-4, 5, (2, 3, 4, 5, 7))
+    g, _ = orc.conv_wgrad(_t(x), _t(dy), (1, 1, 1))
+    ref = dy.reshape(-1, 7).T.astype(np.float64) @ x.reshape(-1, 6).astype(np.float64)
+    assert np.array_equal(g.reshape(7, 6), ref)
+
+
 ALL_PINS = [pin_tutorial_example, pin_output_extent, pin_constant_input, pin_delta_kernel,
             pin_pointwise_is_matmul, pin_im2col_equivalence, pin_torch_witness, pin_linearity,
             pin_translation, pin_groups_split, pin_points_match_full, pin_flip_tutorial_example,
             pin_flip_and_side_padding_torch_witness, pin_side_padding_is_a_crop, pin_transpose_adjoint,
-            pin_transpose_torch_witness, pin_transpose_delta_upsamples]
+            pin_transpose_torch_witness, pin_transpose_delta_upsamples, pin_wgrad_adjoint, pin_wgrad_torch_witness,
+            pin_wgrad_pointwise_is_matmul]

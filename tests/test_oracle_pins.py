@@ -107,6 +107,9 @@ MUTATIONS = {
     "transpose_stride_divisibility_dropped": [(r"if \(num < 0 \|\| num % s\) return -1;", "if (num < 0) return -1;")],
     "transpose_pad_sign": [(r"int64_t num = q \+ p - \(int64_t\)k \* d;", "int64_t num = q - p - (int64_t)k * d;")],
     "transpose_out_channel_index": [(r"\* t->kW \+ kw\) \* Cog \+ cl;", "* t->kW + kw) * Cog + (Cog - 1 - cl);")],
+    "wgrad_dy_channel_reversed": [(r"\* t->Wo \+ ow\) \* t->O \+ o\];", "* t->Wo + ow) * t->O + (t->O - 1 - o)];")],
+    "wgrad_tap_sign": [(r"int64_t iw = \(int64_t\)ow \* t->s\[2\] - t->p\[2\] \+ \(int64_t\)kw \* t->d\[2\];",
+                        "int64_t iw = (int64_t)ow * t->s[2] - t->p[2] - (int64_t)kw * t->d[2];")],
     "padding_not_zero": [(r"if \(ih < 0 \|\| ih >= sh->H\) continue;", "if (ih < 0 || ih >= sh->H) ih = ih < 0 ? 0 : sh->H - 1;")],
 }
 
