@@ -16,7 +16,7 @@ import ctypes
 import os
 
 __all__ = ["conv_fwd", "conv_fwd_host", "out_dims", "plan", "conv_transpose", "transpose_out_dims",
-           "transpose_plan", "last_status", "strerror", "lib",
+           "transpose_plan", "conv_wgrad", "wgrad_workspace_size", "last_status", "strerror", "lib",
            "CONV_F32", "CONV_F16", "CONV_BF16", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC_TMA",
            "VARIANT_TC_GATHER", "VARIANT_TC_TMA_PAIR", "VARIANT_TC_HALO", "VARIANT_TC_HALO_PAIR",
            "VARIANT_TC_TMA_T", "VARIANT_TC_HALO_T", "VARIANT_TC_HALO_T_PAIR", "VARIANT_TC_PHASE", "VARIANT_DEPTHWISE", "VARIANT_DEPTHWISE_DIRECT", "ConvError"]
@@ -72,6 +72,9 @@ def lib() -> ctypes.CDLL:
         L.conv_transpose_out_dims.argtypes = [ci] * 6 + [i3, i3, i3, i3, i3]
         L.conv_transpose.argtypes = [vp, vp, vp] + geo_t + [ci, vp]
         L.conv_transpose_plan.argtypes = geo_t + [ci, i3, i3, i3]
+        # weight gradient: ..., stride, pad_lo, pad_hi, dil, groups, dtype
+        L.conv_wgrad_workspace_size.argtypes = geo_ex[:-2] + [ci, ctypes.POINTER(ctypes.c_ulonglong)]
+        L.conv_wgrad.argtypes = [vp, vp, vp] + geo_ex[:-2] + [ci, vp, ctypes.c_ulonglong, vp]
         L.conv_last_status.argtypes = [vp]
         L.conv_debug_inject_stall.argtypes = [ctypes.c_ulonglong]
         L.conv_strerror.argtypes = [ci]
@@ -183,6 +186,71 @@ def conv_fwd(x, w, stride=1, padding=0, dilation=1, groups=1, *, out=None, varia
                                int(variant), st.cuda_stream)
     if rc:
         raise ConvError(rc, "conv_fwd")
+    return out
+
+
+def wgrad_workspace_size(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype, pad_hi=None):
+    """Bytes of fp32 workspace conv_wgrad needs for these shapes (0 for f32)."""
+    code = {"f32": CONV_F32, "f16": CONV_F16, "bf16": CONV_BF16}[dtype]
+    out = ctypes.c_ulonglong()
+    rc = lib().conv_wgrad_workspace_size(N, D, H, W, C, O, *k, _i3(stride), _i3(pad),
+                                         _i3(pad if pad_hi is None else pad_hi), _i3(dil), int(groups), code,
+                                         ctypes.byref(out))
+    if rc:
+        raise ConvError(rc, "conv_wgrad_workspace_size")
+    return out.value
+
+
+def conv_wgrad(x, dy, kernel_size, stride=1, padding=0, dilation=1, groups=1, *, padding_hi=None, out=None,
+               workspace=None, stream=None):
+    """Weight gradient of conv_fwd: dw[o, k, c] = sum over output pixels of dy * x.
+
+    x: [N, (D,) H, W, C]; dy: [N, (Do,) Ho, Wo, O]; kernel_size: (kD,) kH, kW.
+    Returns dw [O, (kD,) kH, kW, C/groups] in x's dtype.  A 16-bit dtype needs
+    an fp32 workspace; one is allocated with torch when `workspace` is None.
+    """
+    import torch
+    if not (x.is_cuda and dy.is_cuda):
+        raise ValueError("conv_wgrad runs on CUDA tensors only")
+    if x.dtype != dy.dtype:
+        raise TypeError("x and dy must share a dtype")
+    two_d = x.dim() == 4
+    k = tuple(kernel_size) if not isinstance(kernel_size, int) else (kernel_size,) * (2 if two_d else 3)
+    if two_d:
+        k = (1, *k)
+        N, H, W, C = x.shape
+        D = 1
+        s = (1, stride, stride) if isinstance(stride, int) else (1, *stride)
+        p = (0, padding, padding) if isinstance(padding, int) else (0, *padding)
+        d = (1, dilation, dilation) if isinstance(dilation, int) else (1, *dilation)
+        ph = p if padding_hi is None else ((0, padding_hi, padding_hi) if isinstance(padding_hi, int)
+                                           else (0, *padding_hi))
+    else:
+        N, D, H, W, C = x.shape
+        s, p, d = _triple(stride, "stride"), _triple(padding, "padding"), _triple(dilation, "dilation")
+        ph = p if padding_hi is None else _triple(padding_hi, "padding_hi")
+    O = int(dy.shape[-1])
+    N, D, H, W, C = int(N), int(D), int(H), int(W), int(C)
+    Do, Ho, Wo = out_dims(D, H, W, *k, s, p, d, ph)
+    if (dy.shape[1:-1] if not two_d else (1, *dy.shape[1:-1])) != ((Do, Ho, Wo) if not two_d else (1, Ho, Wo)):
+        raise ValueError("dy's extents do not match the forward pass")
+    shape = (O, *k[1:], C // groups) if two_d else (O, *k, C // groups)
+    if out is None:
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+    code = _dtype_code(x)
+    need = wgrad_workspace_size(N, D, H, W, C, O, k, s, p, d, groups,
+                                {CONV_F32: "f32", CONV_F16: "f16", CONV_BF16: "bf16"}[code], ph)
+    if need and workspace is None:
+        workspace = torch.empty(need // 4, dtype=torch.float32, device=x.device)
+    x = x.contiguous()
+    dy = dy.contiguous()
+    st = stream if stream is not None else torch.cuda.current_stream(x.device)
+    with torch.cuda.device(x.device):
+        rc = lib().conv_wgrad(x.data_ptr(), dy.data_ptr(), out.data_ptr(), N, D, H, W, C, O, *k, _i3(s), _i3(p),
+                              _i3(ph), _i3(d), int(groups), code, workspace.data_ptr() if need else None,
+                              int(workspace.numel() * workspace.element_size()) if need else 0, st.cuda_stream)
+    if rc:
+        raise ConvError(rc, "conv_wgrad")
     return out
 
 

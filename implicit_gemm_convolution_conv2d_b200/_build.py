@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libconvfwd.so")
-SOURCES = [os.path.join(CSRC, "conv_fwd.cu")]
+SOURCES = [os.path.join(CSRC, "conv_fwd.cu"), os.path.join(CSRC, "conv_wgrad.cu")]
 DEPS = SOURCES + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(os.path.dirname(HERE), "include", "conv_fwd.h")]
 

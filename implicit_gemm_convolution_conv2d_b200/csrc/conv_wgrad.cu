@@ -1,0 +1,169 @@
+// conv_wgrad.cu -- C ABI of the weight gradient (see conv_wgrad.cuh).
+//
+// A separate translation unit of libconvfwd.so: validation, the split of the
+// pixel reduction across blocks, and the launches (zero the fp32 accumulator,
+// the split-K kernel, the rounding kernel for 16-bit outputs).  Allocates
+// nothing: 16-bit outputs accumulate in a caller-provided fp32 workspace.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "../../include/conv_fwd.h"
+#include "conv_wgrad.cuh"
+
+namespace convfwd {
+namespace {
+
+bool wg_mul_ok(long long a, long long b, long long& r) {
+  if (a < 0 || b < 0) return false;
+  if (a != 0 && b > 0x3fffffffffffffffLL / a) return false;
+  r = a * b;
+  return true;
+}
+
+long long wg_extent(long long in, int k, int s, int p_lo, int p_hi, int d) {
+  const long long num = in + static_cast<long long>(p_lo) + p_hi - static_cast<long long>(d) * (k - 1) - 1;
+  if (num < 0) return 0;
+  return num / s + 1;
+}
+
+struct WgProblem {
+  WgArgs a;
+  int dtype;
+  size_t esize;
+  size_t x_bytes, dy_bytes, dw_bytes;
+  long long dw_elems;
+};
+
+int wg_make(WgProblem& q, int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
+            const int pad_lo[3], const int pad_hi[3], const int dil[3], int groups, int dtype) {
+  if (dtype != CONV_F32 && dtype != CONV_F16 && dtype != CONV_BF16) return CONV_EDTYPE;
+  if (!stride || !pad_lo || !pad_hi || !dil) return CONV_EINVAL;
+  if (N <= 0 || C <= 0 || O <= 0 || groups <= 0 || C % groups != 0 || O % groups != 0) return CONV_EINVAL;
+  const int in[3] = {D, H, W}, k[3] = {kD, kH, kW};
+  int out[3];
+  for (int i = 0; i < 3; ++i) {
+    if (in[i] <= 0 || k[i] <= 0 || stride[i] <= 0 || dil[i] <= 0 || pad_lo[i] < 0 || pad_hi[i] < 0)
+      return CONV_EINVAL;
+    const long long e = wg_extent(in[i], k[i], stride[i], pad_lo[i], pad_hi[i], dil[i]);
+    if (e <= 0 || e > 0x7fffffffLL) return CONV_EINVAL;
+    out[i] = static_cast<int>(e);
+  }
+  WgArgs& a = q.a;
+  a.N = N; a.D = D; a.H = H; a.W = W; a.C = C; a.O = O;
+  a.kD = kD; a.kH = kH; a.kW = kW;
+  a.sd = stride[0]; a.sh = stride[1]; a.sw = stride[2];
+  a.pd = pad_lo[0]; a.ph = pad_lo[1]; a.pw = pad_lo[2];
+  a.dd = dil[0]; a.dh = dil[1]; a.dw = dil[2];
+  a.G = groups; a.Cg = C / groups; a.Og = O / groups;
+  a.Do = out[0]; a.Ho = out[1]; a.Wo = out[2];
+  long long t, nx, ny, nw;
+  if (!wg_mul_ok(kD, kH, t) || !wg_mul_ok(t, kW, t) || t > 0x7fffffffLL) return CONV_EINVAL;
+  a.taps = static_cast<int>(t);
+  if (!wg_mul_ok(t, a.Cg, t) || t > 0x7fffffffLL) return CONV_EINVAL;
+  a.ncols = static_cast<int>(t);
+  if (!wg_mul_ok(N, out[0], t) || !wg_mul_ok(t, out[1], t) || !wg_mul_ok(t, out[2], a.P)) return CONV_EINVAL;
+  if (!wg_mul_ok(N, D, t) || !wg_mul_ok(t, H, t) || !wg_mul_ok(t, W, t) || !wg_mul_ok(t, C, nx)) return CONV_EINVAL;
+  if (!wg_mul_ok(a.P, O, ny) || !wg_mul_ok(O, a.ncols, nw)) return CONV_EINVAL;
+  q.dtype = dtype;
+  q.esize = dtype == CONV_F32 ? 4 : 2;
+  if (nx > (1LL << 50) || ny > (1LL << 50) || nw > (1LL << 40)) return CONV_EINVAL;
+  q.x_bytes = static_cast<size_t>(nx) * q.esize;
+  q.dy_bytes = static_cast<size_t>(ny) * q.esize;
+  q.dw_bytes = static_cast<size_t>(nw) * q.esize;
+  q.dw_elems = nw;
+  return CONV_OK;
+}
+
+size_t wg_workspace(const WgProblem& q) {
+  return q.dtype == CONV_F32 ? 0 : static_cast<size_t>(q.dw_elems) * sizeof(float);
+}
+
+bool wg_overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bn && b0 < a0 + an;
+}
+
+// Splits of the pixel reduction: enough blocks for two per SM, each split at
+// least 64 K steps (1024 pixels) long.
+void wg_split(WgArgs& a, int sms) {
+  const long long tiles = static_cast<long long>((a.ncols + kWgBN - 1) / kWgBN) * ((a.Og + kWgBM - 1) / kWgBM) * a.G;
+  const long long steps = (a.P + kWgBK - 1) / kWgBK;
+  long long ns = std::max<long long>(1, (2LL * sms + tiles - 1) / tiles);
+  ns = std::min<long long>(ns, std::max<long long>(1, steps / 64));
+  ns = std::min<long long>(ns, 65535 / a.G);
+  a.nsplit = static_cast<int>(std::max<long long>(1, ns));
+  a.chunk = (steps + a.nsplit - 1) / a.nsplit * kWgBK;
+}
+
+}  // namespace
+}  // namespace convfwd
+
+using namespace convfwd;
+
+extern "C" {
+
+int conv_wgrad_workspace_size(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
+                              const int stride[3], const int pad_lo[3], const int pad_hi[3], const int dil[3],
+                              int groups, int dtype, unsigned long long* bytes) {
+  WgProblem q;
+  const int rc = wg_make(q, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, dtype);
+  if (rc != CONV_OK) return rc;
+  if (!bytes) return CONV_EINVAL;
+  *bytes = wg_workspace(q);
+  return CONV_OK;
+}
+
+int conv_wgrad(const void* x, const void* dy, void* dw, int N, int D, int H, int W, int C, int O, int kD, int kH,
+               int kW, const int stride[3], const int pad_lo[3], const int pad_hi[3], const int dil[3], int groups,
+               int dtype, void* workspace, unsigned long long workspace_bytes, conv_stream_t stream) {
+  WgProblem q;
+  int rc = wg_make(q, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, dtype);
+  if (rc != CONV_OK) return rc;
+  if (!x || !dy || !dw) return CONV_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(dw)) & 15)
+    return CONV_EALIGN;
+  if (wg_overlaps(dw, q.dw_bytes, x, q.x_bytes) || wg_overlaps(dw, q.dw_bytes, dy, q.dy_bytes)) return CONV_EALIAS;
+  const size_t ws = wg_workspace(q);
+  if (ws > 0) {
+    if (!workspace || workspace_bytes < ws) return CONV_EINVAL;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15) return CONV_EALIGN;
+    if (wg_overlaps(workspace, ws, x, q.x_bytes) || wg_overlaps(workspace, ws, dy, q.dy_bytes) ||
+        wg_overlaps(workspace, ws, dw, q.dw_bytes))
+      return CONV_EALIAS;
+  }
+  if ((q.dw_elems + 255) / 256 > 0x7fffffffLL) return CONV_EUNSUPPORTED;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ELAUNCH;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return CONV_ELAUNCH;
+  WgArgs a = q.a;
+  wg_split(a, sms);
+  a.x = x;
+  a.dy = dy;
+  a.acc = ws > 0 ? static_cast<float*>(workspace) : static_cast<float*>(dw);
+  const dim3 grid(static_cast<unsigned>((a.ncols + kWgBN - 1) / kWgBN), static_cast<unsigned>((a.Og + kWgBM - 1) / kWgBM),
+                  static_cast<unsigned>(a.G * a.nsplit));
+  if (grid.y > 65535 || grid.z > 65535) return CONV_EUNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(a.acc, 0, static_cast<size_t>(q.dw_elems) * sizeof(float), st) != cudaSuccess)
+    return CONV_ELAUNCH;
+
+  if (dtype == CONV_F32) conv_wgrad_kernel<float><<<grid, kWgThreads, 0, st>>>(a);
+  else if (dtype == CONV_F16) conv_wgrad_kernel<__half><<<grid, kWgThreads, 0, st>>>(a);
+  else conv_wgrad_kernel<__nv_bfloat16><<<grid, kWgThreads, 0, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
+  if (ws > 0) {
+    const long long n = q.dw_elems;
+    const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
+    if (dtype == CONV_F16)
+      conv_wgrad_round_kernel<__half><<<blocks, 256, 0, st>>>(a.acc, static_cast<__half*>(dw), n);
+    else
+      conv_wgrad_round_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(a.acc, static_cast<__nv_bfloat16*>(dw), n);
+    if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
+  }
+  return CONV_OK;
+}
+
+}  // extern "C"

@@ -234,6 +234,34 @@ int conv_transpose_plan(int N, int D, int H, int W, int Cin, int Cout, int kD, i
                         const int stride[3], const int pad[3], const int out_pad[3], const int dil[3],
                         int groups, int dtype, int variant, int* bn, int* stages, int* ctas);
 
+/* ---- weight gradient ----------------------------------------------------
+ *
+ * The gradient of conv_fwd's weights given the gradient dy of its output
+ * (the forward pass with padding pad_lo below and pad_hi above, no flip):
+ *
+ *   dw[o, kd, kh, kw, c] = sum over n, od, oh, ow of dy[n, od, oh, ow, o] *
+ *       x[n, od*sd - pd + kd*dd, oh*sh - ph + kh*dh, ow*sw - pw + kw*dw, g*C/G + c]
+ *
+ * x: [N, D, H, W, C]; dy: [N, Do, Ho, Wo, O] (the forward output's extents);
+ * dw: [O, kD, kH, kW, C/groups], written (not accumulated into).  FP32 FMAs
+ * with fp32 accumulation, the pixel reduction split across blocks and summed
+ * with fp32 atomics (summation order not deterministic).  f32 outputs are
+ * accumulated in dw itself; f16/bf16 outputs need a caller-provided fp32
+ * workspace of conv_wgrad_workspace_size bytes (16-byte aligned, disjoint
+ * from x, dy, dw), rounded to nearest into dw at the end.  Queues three
+ * operations on `stream` (a memset and two kernels); allocates nothing.
+ * Errors as for conv_fwd; CONV_EINVAL also for a missing or short workspace. */
+
+/* Bytes of fp32 workspace conv_wgrad needs (0 for f32). */
+int conv_wgrad_workspace_size(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
+                              const int stride[3], const int pad_lo[3], const int pad_hi[3],
+                              const int dil[3], int groups, int dtype, unsigned long long* bytes);
+
+int conv_wgrad(const void* x, const void* dy, void* dw, int N, int D, int H, int W, int C, int O,
+               int kD, int kH, int kW, const int stride[3], const int pad_lo[3], const int pad_hi[3],
+               const int dil[3], int groups, int dtype, void* workspace,
+               unsigned long long workspace_bytes, conv_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the current device's status word.
  * Returns CONV_OK, or CONV_ETIMEOUT if a kernel since the last call gave up on
  * a pipeline wait (the kernel then wrote no further output and returned), or

@@ -338,6 +338,57 @@ def test_transpose_python_api():
     assert e.value.code == -7
 
 
+# Weight gradient: (name, N, D, H, W, C, O, k, stride, pad_lo, pad_hi, dil, groups).
+WGRAD = [
+    ("wg_2d_c16_o32", 2, 1, 13, 11, 16, 32, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+    ("wg_s2_groups2", 2, 1, 17, 15, 32, 64, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1), 2),
+    ("wg_3d_dil", 1, 5, 6, 7, 8, 12, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 2, 1), 1),
+    ("wg_side_padding", 2, 1, 9, 10, 24, 40, (1, 3, 4), (1, 1, 2), (0, 1, 0), (0, 2, 1), (1, 1, 1), 1),
+    ("wg_depthwise", 2, 1, 12, 12, 32, 32, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1), 32),
+    ("wg_split_reduction", 4, 1, 32, 32, 64, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+    ("wg_stem_like", 2, 1, 30, 30, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (0, 3, 3), (1, 1, 1), 1),
+]
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("case", WGRAD, ids=lambda c: c[0])
+def test_wgrad_parity(case, dtype):
+    """Weight gradient against the oracle on every element.  The pixel sum is
+    an fp32 reduction of P terms split into chunks, so besides the forward
+    tolerance the bound allows (P + 64) * 2^-24 * S (recursive summation)."""
+    name, N, D, H, W, Cc, O, k, s, p, ph, d, G = case
+    gen = torch.Generator().manual_seed(zlib.crc32(name.encode()) % 1000)
+    dt = WL.TORCH_DTYPE[dtype]
+    Do, Ho, Wo = C.out_dims(D, H, W, *k, s, p, d, ph)
+    x = (torch.rand((N, D, H, W, Cc), generator=gen) * 2 - 1).to(dt)
+    dy = (torch.rand((N, Do, Ho, Wo, O), generator=gen) * 2 - 1).to(dt)
+    g_ref, s_ref = oracle.conv_wgrad(x, dy, k, s, p, d, G, pad_hi=ph)
+    g = C.conv_wgrad(x.cuda(), dy.cuda(), k, stride=s, padding=p, dilation=d, groups=G, padding_hi=ph)
+    torch.cuda.synchronize()
+    assert tuple(g.shape) == g_ref.shape
+    P = N * Do * Ho * Wo
+    assert_parity(g.cpu(), g_ref, s_ref, dtype, f"{name}/{dtype}", rel_floor=(P + 64) * 2.0 ** -24)
+
+
+def test_wgrad_2d_api_and_errors():
+    """2-D tensors through the Python API; a short workspace and a misaligned
+    buffer are refused with nothing queued."""
+    gen = torch.Generator().manual_seed(5)
+    x = (torch.rand((2, 9, 8, 16), generator=gen) * 2 - 1).to(torch.bfloat16).cuda()
+    dy = (torch.rand((2, 9, 8, 24), generator=gen) * 2 - 1).to(torch.bfloat16).cuda()
+    g = C.conv_wgrad(x, dy, 3, stride=1, padding=1)
+    torch.cuda.synchronize()
+    assert tuple(g.shape) == (24, 3, 3, 16)
+    g_ref, s_ref = oracle.conv_wgrad(x.cpu().unsqueeze(1), dy.cpu().unsqueeze(1), (1, 3, 3), (1, 1, 1), (0, 1, 1))
+    assert_parity(g.cpu().unsqueeze(1), g_ref, s_ref, "bf16", "wgrad 2-D", rel_floor=(2 * 72 + 64) * 2.0 ** -24)
+    need = C.wgrad_workspace_size(2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")
+    assert need == 24 * 9 * 16 * 4
+    with pytest.raises(C.ConvError) as e:
+        C.conv_wgrad(x, dy, 3, padding=1, workspace=torch.empty(10, dtype=torch.float32, device="cuda"))
+    assert e.value.code == -1
+    assert C.last_status() == 0
+
+
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_transposed_wide_pixel_tiles(dtype):
     """Enough output pixels for 256-pixel tiles on every SM (the 128-pixel
