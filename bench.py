@@ -300,7 +300,14 @@ def bench_ours(args):
     dims = out_dims(wl, pad_hi)
     flops = conv_flops(wl, dims)
     xb, wb, yb = conv_bytes(wl, dims)
-    if wl.transpose:
+    if wl.wgrad:
+        # the weight gradient: inputs x and dy, output dw; the FP32 split-K kernel
+        e = WL.ELEM_BYTES[wl.dtype]
+        wb = e * wl.N * dims[0] * dims[1] * dims[2] * wl.O        # dy
+        yb = e * wl.O * wl.k[0] * wl.k[1] * wl.k[2] * (wl.C // wl.groups)  # dw
+        variant, bn, stages, ctas = None, 64, 1, 0
+        vname = "simt_wgrad"
+    elif wl.transpose:
         variant, bn, stages, ctas = C.transpose_plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad,
                                                      wl.out_pad, wl.dil, wl.groups, wl.dtype,
                                                      getattr(C, "VARIANT_" + args.variant))
@@ -308,17 +315,27 @@ def bench_ours(args):
         variant, bn, stages, ctas = C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil,
                                            wl.groups, wl.dtype, getattr(C, "VARIANT_" + args.variant),
                                            pad_hi=pad_hi, flip=flip)
-    vname = C.VARIANT_NAMES[variant]
+    if not wl.wgrad:
+        vname = C.VARIANT_NAMES[variant]
 
     # inputs: seeded on the host (rank-dependent seed), copied once
-    x_h, w_h = WL.make_inputs(wl, seed=wl.seed + 1000 * rank)
+    if wl.wgrad:
+        x_h, w_h = WL.make_wgrad_inputs(wl, (wl.N, *dims, wl.O), seed=wl.seed + 1000 * rank)  # w_h: dy
+    else:
+        x_h, w_h = WL.make_inputs(wl, seed=wl.seed + 1000 * rank)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     per_set = xb + wb + yb
     nsets = max(2, min(64, math.ceil(2 * l2 / per_set) + 1))
     xs = [x_h.to(dev) for _ in range(nsets)]
     wts = [w_h.to(dev) for _ in range(nsets)]
     Do, Ho, Wo = dims
-    ys = [torch.empty((wl.N, Do, Ho, Wo, wl.O), dtype=x_h.dtype, device=dev) for _ in range(nsets)]
+    if wl.wgrad:
+        ys = [torch.empty(wl.w_shape, dtype=x_h.dtype, device=dev) for _ in range(nsets)]  # dw
+        ws_bytes = C.wgrad_workspace_size(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil,
+                                          wl.groups, wl.dtype)
+        wsbuf = torch.empty(max(1, ws_bytes // 4), dtype=torch.float32, device=dev)
+    else:
+        ys = [torch.empty((wl.N, Do, Ho, Wo, wl.O), dtype=x_h.dtype, device=dev) for _ in range(nsets)]
     stream = torch.cuda.current_stream(dev)
     geo = lambda i: (wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, *wl.k, wl.stride, wl.pad, wl.dil, wl.groups)
     dcode = {"f32": 0, "f16": 1, "bf16": 2}[wl.dtype]
@@ -328,7 +345,12 @@ def bench_ours(args):
         nonlocal launches
         s = i % nsets
         # the launch goes to the current stream (the capture stream while a graph is recorded)
-        if wl.transpose:
+        if wl.wgrad:
+            rc = C.conv_wgrad_raw(xs[s].data_ptr(), wts[s].data_ptr(), ys[s].data_ptr(),
+                                  (wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, *wl.k, wl.stride, wl.pad, wl.pad, wl.dil,
+                                   wl.groups), dcode, wsbuf.data_ptr() if ws_bytes else None, ws_bytes,
+                                  torch.cuda.current_stream(dev).cuda_stream)
+        elif wl.transpose:
             rc = C.conv_transpose_raw(xs[s].data_ptr(), wts[s].data_ptr(), ys[s].data_ptr(),
                                       (wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, *wl.k, wl.stride, wl.pad, wl.out_pad,
                                        wl.dil, wl.groups), dcode, variant, torch.cuda.current_stream(dev).cuda_stream)
@@ -422,7 +444,7 @@ def bench_ours(args):
     e2e = None
     if pad_hi is not None or flip:
         e2e = {"skipped": "the host-buffer entry point takes symmetric padding and no flip"}
-    elif wl.transpose:
+    elif wl.transpose or wl.wgrad:
         e2e = {"skipped": "the host-buffer entry point is the forward convolution's"}
     elif not args.no_e2e:
         xp = x_h.pin_memory()
@@ -456,7 +478,7 @@ def bench_ours(args):
     # tensor cores for the rest) against the algorithmic bytes at HBM speed.
     sm_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
     alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
-    fma_kernel = variant in (C.VARIANT_SIMT, C.VARIANT_DEPTHWISE, C.VARIANT_DEPTHWISE_DIRECT)
+    fma_kernel = wl.wgrad or variant in (C.VARIANT_SIMT, C.VARIANT_DEPTHWISE, C.VARIANT_DEPTHWISE_DIRECT)
     compute_peak = alu_peak if fma_kernel else float(peaks["bf16_tflops"])
     hbm_bound = (xb + wb + yb) / (float(peaks["hbm_gbs"]) * 1e9) > flops / (compute_peak * 1e12)
     tensor_bound = not fma_kernel and not hbm_bound
@@ -488,10 +510,12 @@ def bench_ours(args):
         "config": {"workload": wl.name, "N": wl.N, "DHW": [wl.D, wl.H, wl.W], "C": wl.C, "O": wl.O,
                    "kernel": list(wl.k), "stride": list(wl.stride), "pad": list(wl.pad), "dil": list(wl.dil),
                    "groups": wl.groups, "out_DHW": list(dims),
-                   **({"transpose": True, "out_pad": list(wl.out_pad)} if wl.transpose else {}), "gflop_per_step": round(flops / 1e9, 4),
+                   **({"transpose": True, "out_pad": list(wl.out_pad)} if wl.transpose else {}),
+                   **({"pass": "weight gradient (x, dy -> dw)"} if wl.wgrad else {}), "gflop_per_step": round(flops / 1e9, 4),
                    "global_batch": wl.N * nranks, "parallelism": f"independent batches x{nranks}",
                    "variant": vname,
-                   "tile": (simt_tile(wl, dims, bn, ctas) if variant == C.VARIANT_SIMT else
+                   "tile": ([64, 64] if wl.wgrad  # output channels x weight columns per block
+                            else simt_tile(wl, dims, bn, ctas) if variant == C.VARIANT_SIMT else
                             [4, bn] if variant in (C.VARIANT_DEPTHWISE, C.VARIANT_DEPTHWISE_DIRECT)  # pixels x channels per thread
                             else [bn, 128] if variant == C.VARIANT_TC_TMA_T
                             else [bn, 128 if (wl.O // wl.groups) % 128 == 0 else 64] if variant == C.VARIANT_TC_HALO_T
@@ -503,7 +527,8 @@ def bench_ours(args):
         "launch": "cuda_graph_of_steps" if graph is not None else "eager",
         "eager_ms_per_step": round(eager_ms, 5),
         "e2e": e2e,
-        "gpu_launches": timed_launches,
+        # the weight gradient queues two kernels per call for 16-bit types (the split-K sum, the rounding)
+        "gpu_launches": timed_launches * (2 if wl.wgrad and wl.dtype != "f32" else 1),
         "clocks": clk,
     }
     if pad_hi is not None or flip:
@@ -521,10 +546,19 @@ def bench_ours(args):
 
 # ---------------------------------------------------------------- CPU oracle
 
+def _sample_inputs(wl):
+    """The workload's host inputs: (x, w), or (x, dy) for a weight gradient."""
+    if wl.wgrad:
+        return WL.make_wgrad_inputs(wl, (wl.N, *out_dims(wl), wl.O))
+    return WL.make_inputs(wl)
+
+
 def _oracle_sample_step(wl, x, w, n_img):
     import oracle
     xs = x[:n_img].contiguous()
-    if wl.transpose:
+    if wl.wgrad:  # w is dy here
+        y, _ = oracle.conv_wgrad(xs, w[:n_img].contiguous(), wl.k, wl.stride, wl.pad, wl.dil, wl.groups)
+    elif wl.transpose:
         y, _ = oracle.conv_transpose(xs, w, wl.stride, wl.pad, wl.out_pad, wl.dil, wl.groups)
     else:
         y, _ = oracle.conv_fwd(xs, w, wl.stride, wl.pad, wl.dil, wl.groups)
@@ -535,7 +569,7 @@ def cpu_baseline(wl, budget_s=15.0):
     """The oracle as it stands, on the host cores, over the first images of the
     workload (as many as fit the time budget)."""
     import oracle
-    x, w = WL.make_inputs(wl)
+    x, w = _sample_inputs(wl)
     one = wl.with_(N=1)
     f1 = conv_flops(one)
     t0 = time.perf_counter()
@@ -585,7 +619,7 @@ def bench_reference(args):
         return
     import oracle
     wl = WL.WORKLOADS[args.workload]
-    x, w = WL.make_inputs(wl)
+    x, w = _sample_inputs(wl)
     one = wl.with_(N=1)
     f1 = conv_flops(one)
     # one step = the oracle on one image of the workload (a bounded sample)

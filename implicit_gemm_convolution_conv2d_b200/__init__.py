@@ -254,6 +254,13 @@ def conv_wgrad(x, dy, kernel_size, stride=1, padding=0, dilation=1, groups=1, *,
     return out
 
 
+def conv_wgrad_raw(x_ptr, dy_ptr, dw_ptr, geom, dtype, ws_ptr=None, ws_bytes=0, stream_handle=0):
+    """The C entry point on raw device pointers: geom = (N,D,H,W,C,O,kD,kH,kW,stride,pad_lo,pad_hi,dil,groups)."""
+    N, D, H, W, Cc, O, kD, kH, kW, s, p, ph, d, g = geom
+    return lib().conv_wgrad(x_ptr, dy_ptr, dw_ptr, N, D, H, W, Cc, O, kD, kH, kW, _i3(s), _i3(p), _i3(ph), _i3(d),
+                            int(g), int(dtype), ws_ptr, int(ws_bytes), stream_handle)
+
+
 def transpose_out_dims(D, H, W, kD, kH, kW, stride, pad, out_pad, dil):
     """(Qd, Qh, Qw) of the transposed convolution, as computed by the library (host only)."""
     out = (ctypes.c_int * 3)()

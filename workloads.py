@@ -45,6 +45,7 @@ class Workload:
     seed: int = 0
     transpose: bool = False      # transposed ("upsampling") convolution: x has C channels, y has O
     out_pad: tuple = (0, 0, 0)   # its output padding
+    wgrad: bool = False          # the weight gradient of the forward pass (inputs x and dy)
 
     @property
     def x_shape(self):
@@ -110,6 +111,12 @@ WORKLOADS["convT_bf16_n16_56x56_c256_o128_k4s2"] = Workload(
     "convT_bf16_n16_56x56_c256_o128_k4s2", 16, 1, 56, 56, 256, 128, (1, 4, 4), (1, 2, 2), (0, 1, 1),
     dtype="bf16", seed=6, transpose=True)
 
+# Weight gradient of the 3x3 256->256 layer at 56x56, N=64, bf16, seed 7 (the
+# headline forward layer's third pass).
+WORKLOADS["wgrad_bf16_n64_56x56_c256_o256_k3"] = Workload(
+    "wgrad_bf16_n64_56x56_c256_o256_k3", 64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1),
+    dtype="bf16", seed=7, wgrad=True)
+
 # Name of the workload the benchmark times by default: the tutorial's
 # arithmetic-intensity example (3x3, 256->256, 56x56) at batch 64.
 HEADLINE = "conv2d_bf16_n64_56x56_c256_o256_k3"
@@ -136,6 +143,18 @@ def make_inputs(wl: Workload, seed: int | None = None):
     w = torch.randn(wl.w_shape, generator=g, dtype=torch.float32) * sigma
     dt = TORCH_DTYPE[wl.dtype]
     return x.to(dt).contiguous(), w.to(dt).contiguous()
+
+
+def make_wgrad_inputs(wl: Workload, dy_shape, seed: int | None = None):
+    """Seeded host tensors (x, dy) for a weight-gradient workload: x as above,
+    then dy = U[-1, 1) in the forward output's shape `dy_shape` (computed by
+    the caller), both rounded to the workload's dtype."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(wl.seed if seed is None else seed)
+    x = torch.rand(wl.x_shape, generator=g, dtype=torch.float32) * 2.0 - 1.0
+    dy = torch.rand(tuple(dy_shape), generator=g, dtype=torch.float32) * 2.0 - 1.0
+    dt = TORCH_DTYPE[wl.dtype]
+    return x.to(dt).contiguous(), dy.to(dt).contiguous()
 
 
 def case(N, D, H, W, C, O, k, stride=(1, 1, 1), pad=(0, 0, 0), dil=(1, 1, 1), groups=1,
