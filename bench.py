@@ -103,6 +103,7 @@ KERNEL_SOURCES = {
     "simt_ffma": ["conv_fwd.cu", "conv_simt.cuh"],
     "depthwise_tma": _COMMON_SRC + ["conv_simt.cuh", "conv_dw.cuh"],
     "depthwise_direct": ["conv_fwd.cu", "conv_simt.cuh", "conv_dw.cuh"],
+    "simt_wgrad": ["conv_wgrad.cu", "conv_wgrad.cuh", "conv_simt.cuh"],
 }
 
 
