@@ -270,3 +270,20 @@ def test_transpose_extents_and_plans(C):
     # output padding must stay below max(stride, dilation)
     with pytest.raises(C.ConvError):
         C.transpose_out_dims(1, 8, 8, 1, 3, 3, (1, 2, 2), (0, 1, 1), (0, 2, 2), (1, 1, 1))
+
+
+def test_wgrad_workspace_and_arguments(C):
+    """The weight gradient's fp32 workspace: O x taps x C/G floats for 16-bit
+    outputs, none for f32; bad shapes are refused on the host."""
+    g = (2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1)
+    assert C.wgrad_workspace_size(*g, "bf16") == 24 * 9 * 16 * 4
+    assert C.wgrad_workspace_size(*g, "f16") == 24 * 9 * 16 * 4
+    assert C.wgrad_workspace_size(*g, "f32") == 0
+    assert C.wgrad_workspace_size(2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 4, "bf16") == \
+        24 * 9 * 4 * 4
+    with pytest.raises(C.ConvError) as e:   # C not divisible by groups
+        C.wgrad_workspace_size(2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 5, "bf16")
+    assert e.value.code == -1
+    with pytest.raises(C.ConvError) as e:   # a kernel larger than the padded input
+        C.wgrad_workspace_size(1, 1, 2, 2, 8, 8, (1, 5, 5), (1, 1, 1), (0, 0, 0), (1, 1, 1), 1, "f32")
+    assert e.value.code == -1
