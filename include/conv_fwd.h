@@ -26,7 +26,13 @@
  *
  * Element types: CONV_F16 and CONV_BF16 run on the tcgen05 tensor cores with
  * fp32 accumulation in tensor memory and round-to-nearest-even output;
- * CONV_F32 runs an fp32 FFMA kernel (no TF32).  x, w and y share one type.
+ * CONV_F32 runs an fp32 FFMA kernel (no TF32); depthwise problems of any type
+ * run FP32-FMA depthwise kernels.  x, w and y share one type.
+ *
+ * Besides the forward pass (conv_fwd, conv_fwd_variant, conv_fwd_ex,
+ * conv_fwd_host), the header declares its other two passes: the transposed
+ * convolution, which is the data gradient (conv_transpose), and the weight
+ * gradient (conv_wgrad), each documented at its declaration below.
  *
  * Ownership: the caller owns every buffer.  conv_fwd allocates nothing, does
  * not synchronise, and returns after queueing its work on `stream`.
