@@ -90,3 +90,33 @@ def test_flop_and_byte_counters_match_the_tutorial():
                      (xb + wb + yb, "bytes_printed")):
         assert abs(got / c3[key] - 1) < c3["bytes_rel_tol"], (key, got)
     assert abs(f / (xb + wb + yb) / c3["intensity_printed"] - 1) < c3["intensity_rel_tol"]
+
+
+def test_kernel_source_sets_cover_every_kernel():
+    """Every kernel name a bench line can report has the list of source files
+    its traffic record is keyed on, and those files exist."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import implicit_gemm_convolution_conv2d_b200 as C
+    names = set(C.VARIANT_NAMES.values()) | {"simt_wgrad"}
+    csrc = os.path.join(ROOT, "implicit_gemm_convolution_conv2d_b200", "csrc")
+    for name in names:
+        assert name in bench.KERNEL_SOURCES, name
+        for f in bench.KERNEL_SOURCES[name]:
+            assert os.path.exists(os.path.join(csrc, f)), (name, f)
+        assert len(bench.kernel_source_hash(name)) == 12
+
+
+def test_transposed_and_weight_gradient_counters():
+    """A transposed convolution counts the FLOPs of the forward pass it is the
+    adjoint of (2 x its input pixels x Cin x taps x Cout/G); the weight
+    gradient counts those of the forward pass."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as WL
+    t = WL.WORKLOADS["convT_bf16_n16_56x56_c256_o128_k4s2"]
+    assert bench.conv_flops(t) == 2 * 16 * 56 * 56 * 256 * 16 * 128
+    g = WL.WORKLOADS["wgrad_bf16_n64_56x56_c256_o256_k3"]
+    assert bench.conv_flops(g, (1, 56, 56)) == 2 * 64 * 56 * 56 * 256 * 9 * 256
