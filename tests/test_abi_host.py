@@ -287,3 +287,37 @@ def test_wgrad_workspace_and_arguments(C):
     with pytest.raises(C.ConvError) as e:   # a kernel larger than the padded input
         C.wgrad_workspace_size(1, 1, 2, 2, 8, 8, (1, 5, 5), (1, 1, 1), (0, 0, 0), (1, 1, 1), 1, "f32")
     assert e.value.code == -1
+
+
+def test_planner_on_random_geometries(C):
+    """The planners answer every geometry with a variant or a clean error code
+    (seeded random forward, depthwise and transposed shapes, all types)."""
+    import random
+    rng = random.Random(7)
+    valid_codes = {-1, -7}
+    for _ in range(300):
+        G = rng.choice([1, 1, 2, 4])
+        dw = rng.random() < 0.3
+        Cc = rng.choice([3, 4, 8, 16, 24, 32, 64, 128, 200, 256]) * (1 if dw else G)
+        O = Cc if dw else rng.choice([8, 16, 32, 64, 96, 128, 256]) * G
+        if dw:
+            G = Cc
+        two_d = rng.random() < 0.6
+        D = 1 if two_d else rng.randint(1, 12)
+        H, W = rng.randint(1, 40), rng.randint(1, 40)
+        k = (1 if two_d else rng.randint(1, 3), rng.randint(1, 7), rng.randint(1, 7))
+        s = (1 if two_d else rng.randint(1, 2), rng.randint(1, 3), rng.randint(1, 3))
+        d = (1, rng.randint(1, 2), rng.randint(1, 2))
+        p = tuple(rng.randint(0, (k[i] - 1) * d[i]) for i in range(3))
+        dt = rng.choice(["f16", "bf16", "f32"])
+        try:
+            v, bn, st, ct = C.plan(rng.randint(1, 4), D, H, W, Cc, O, k, s, p, d, G, dt)
+            assert v in C.VARIANT_NAMES and bn > 0 and st >= 1 and ct >= 1, (v, bn, st, ct)
+        except C.ConvError as e:
+            assert e.code in valid_codes, e.code
+        op = tuple(rng.randint(0, max(s[i], d[i]) - 1) for i in range(3))
+        try:
+            v, bn, st, ct = C.transpose_plan(rng.randint(1, 4), D, H, W, Cc, O, k, s, p, op, d, G, dt)
+            assert v in (C.VARIANT_TC_GATHER, C.VARIANT_SIMT) and ct >= 1, (v, ct)
+        except C.ConvError as e:
+            assert e.code in valid_codes, e.code
