@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         # weight gradient: ..., stride, pad_lo, pad_hi, dil, groups, dtype
         L.conv_wgrad_workspace_size.argtypes = geo_ex[:-2] + [ci, ctypes.POINTER(ctypes.c_ulonglong)]
         L.conv_wgrad.argtypes = [vp, vp, vp] + geo_ex[:-2] + [ci, vp, ctypes.c_ulonglong, vp]
+        L.conv_wgrad_noalloc.argtypes = [vp, vp, vp] + geo_ex[:-2] + [ci, vp]
         L.conv_last_status.argtypes = [vp]
         L.conv_debug_inject_stall.argtypes = [ctypes.c_ulonglong]
         L.conv_strerror.argtypes = [ci]
@@ -259,6 +260,14 @@ def conv_wgrad_raw(x_ptr, dy_ptr, dw_ptr, geom, dtype, ws_ptr=None, ws_bytes=0, 
     N, D, H, W, Cc, O, kD, kH, kW, s, p, ph, d, g = geom
     return lib().conv_wgrad(x_ptr, dy_ptr, dw_ptr, N, D, H, W, Cc, O, kD, kH, kW, _i3(s), _i3(p), _i3(ph), _i3(d),
                             int(g), int(dtype), ws_ptr, int(ws_bytes), stream_handle)
+
+
+def conv_wgrad_noalloc_raw(x_ptr, dy_ptr, dw_ptr, geom, dtype, stream_handle=0):
+    """conv_wgrad_noalloc on raw device pointers (no workspace: the library's
+    static scratch array); geom as for conv_wgrad_raw."""
+    N, D, H, W, Cc, O, kD, kH, kW, s, p, ph, d, g = geom
+    return lib().conv_wgrad_noalloc(x_ptr, dy_ptr, dw_ptr, N, D, H, W, Cc, O, kD, kH, kW, _i3(s), _i3(p), _i3(ph),
+                                    _i3(d), int(g), int(dtype), stream_handle)
 
 
 def transpose_out_dims(D, H, W, kD, kH, kW, stride, pad, out_pad, dil):

@@ -1820,6 +1820,7 @@ const char* conv_strerror(int code) {
     case CONV_ETIMEOUT: return "kernel pipeline wait timed out";
     case CONV_EUNSUPPORTED: return "variant cannot run this shape or type";
     case CONV_EDRIVER: return "TMA tensor map encoding failed";
+    case CONV_ESCRATCH: return "problem needs more scratch than the library's static buffer holds";
     default: return "unknown error";
   }
 }

@@ -9,9 +9,15 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/conv_fwd.h"
 #include "conv_wgrad.cuh"
+
+// Scratch of conv_wgrad_noalloc: a fixed array in the library's own device
+// image, so that entry point never allocates.  Every device that loads the
+// library holds it until the process exits.
+static __device__ __align__(256) float g_wgrad_static_scratch[CONV_WGRAD_STATIC_SCRATCH_BYTES / sizeof(float)];
 
 namespace convfwd {
 namespace {
@@ -98,6 +104,31 @@ void wg_split(WgArgs& a, int sms) {
   a.chunk = (steps + a.nsplit - 1) / a.nsplit * kWgBK;
 }
 
+constexpr size_t kWgStaticScratchBytes = CONV_WGRAD_STATIC_SCRATCH_BYTES;
+static_assert(kWgStaticScratchBytes % 256 == 0, "static scratch size");
+
+// The array's device address, looked up once per device.  In host code the
+// array's name is only a host-side stand-in; the address a kernel may be given
+// comes from cudaGetSymbolAddress with that device current.
+constexpr int kWgMaxDevices = 256;
+std::mutex g_static_mu;
+void* g_static_addr[kWgMaxDevices] = {};
+
+int wg_static_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= kWgMaxDevices) return CONV_ELAUNCH;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_wgrad_static_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return CONV_ELAUNCH;
+    }
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  return CONV_OK;
+}
+
 }  // namespace
 }  // namespace convfwd
 
@@ -164,6 +195,25 @@ int conv_wgrad(const void* x, const void* dy, void* dw, int N, int D, int H, int
     if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
   }
   return CONV_OK;
+}
+
+int conv_wgrad_noalloc(const void* x, const void* dy, void* dw, int N, int D, int H, int W, int C, int O, int kD,
+                       int kH, int kW, const int stride[3], const int pad_lo[3], const int pad_hi[3],
+                       const int dil[3], int groups, int dtype, conv_stream_t stream) {
+  WgProblem q;
+  const int rc = wg_make(q, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, dtype);
+  if (rc != CONV_OK) return rc;
+  const size_t ws = wg_workspace(q);
+  if (ws > kWgStaticScratchBytes) return CONV_ESCRATCH;
+  void* scratch = nullptr;
+  if (ws > 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ELAUNCH;
+    const int r = wg_static_scratch(dev, &scratch);
+    if (r != CONV_OK) return r;
+  }
+  return conv_wgrad(x, dy, dw, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, dtype, scratch,
+                    ws > 0 ? kWgStaticScratchBytes : 0, stream);
 }
 
 }  // extern "C"

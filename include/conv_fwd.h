@@ -71,7 +71,9 @@ enum {
   CONV_ELAUNCH = -5,     /* the CUDA runtime refused the launch or a copy */
   CONV_ETIMEOUT = -6,    /* a kernel's pipeline wait ran out (device status) */
   CONV_EUNSUPPORTED = -7,/* the requested kernel variant cannot run this shape */
-  CONV_EDRIVER = -8      /* the driver could not encode a TMA tensor map */
+  CONV_EDRIVER = -8,     /* the driver could not encode a TMA tensor map */
+  CONV_ESCRATCH = -9     /* conv_wgrad_noalloc: the problem needs more scratch
+                            than CONV_WGRAD_STATIC_SCRATCH_BYTES */
 };
 
 /* Kernel variants (for conv_fwd_variant and conv_plan). */
@@ -267,6 +269,39 @@ int conv_wgrad(const void* x, const void* dy, void* dw, int N, int D, int H, int
                int kD, int kH, int kW, const int stride[3], const int pad_lo[3], const int pad_hi[3],
                const int dil[3], int groups, int dtype, void* workspace,
                unsigned long long workspace_bytes, conv_stream_t stream);
+
+/* ---- weight gradient without allocation -------------------------------
+ *
+ * No counterpart in the pages: this entry point exists for callers that cannot
+ * allocate device memory.  Examples are a plugin inside a framework whose
+ * caching allocator owns all of the device's memory, a real-time loop that
+ * forbids cudaMalloc/cudaFree because they can block or synchronise the
+ * device, and a runtime that reserved its whole memory budget at start-up.
+ * Such callers cannot provide conv_wgrad's workspace.
+ *
+ * conv_wgrad_noalloc computes what conv_wgrad computes, with the same
+ * arguments minus the workspace.  Its fp32 scratch is a fixed array of
+ * CONV_WGRAD_STATIC_SCRATCH_BYTES inside the library's device image.  Every
+ * device that loads the library holds that array until the process exits.
+ * The call allocates nothing and calls no allocating routine.
+ *
+ *  - Limit: a 16-bit problem needs O * kD*kH*kW * C/groups * 4 bytes of
+ *    scratch (conv_wgrad_workspace_size).  Above the limit the call returns
+ *    CONV_ESCRATCH and queues nothing.  f32 problems use no scratch.
+ *  - Set-up: the first call on a device (with that device current) looks up
+ *    the array's device address once.  Make that first call before any stream
+ *    capture.
+ *  - Sharing: every call on a device uses the same array.  Each call clears
+ *    it on its stream before use.  Calls whose work overlaps on the GPU (two
+ *    streams, or two host threads on different streams) race on it and give
+ *    wrong results; order them on one stream or with events.
+ *
+ * Returns as conv_wgrad, plus CONV_ESCRATCH. */
+#define CONV_WGRAD_STATIC_SCRATCH_BYTES (16ull << 20)
+
+int conv_wgrad_noalloc(const void* x, const void* dy, void* dw, int N, int D, int H, int W, int C, int O,
+                       int kD, int kH, int kW, const int stride[3], const int pad_lo[3], const int pad_hi[3],
+                       const int dil[3], int groups, int dtype, conv_stream_t stream);
 
 /* Waits for `stream`, then reads and clears the current device's status word.
  * Returns CONV_OK, or CONV_ETIMEOUT if a kernel since the last call gave up on
