@@ -447,6 +447,28 @@ _W_GEOMS = [
 ]
 
 
+def pin_transpose_points_match_full(orc):
+    """The transposed sampled-output entry point returns the same values as the
+    full transposed pass (itself tied to the forward oracle by the adjoint pin),
+    on odd extents (Qh != Qw, so a swapped index decode shows), strides, output
+    padding and groups, in every storage type."""
+    rng = np.random.default_rng(23)
+    geoms = [
+        # (N, D, H, W, Cin, Cout, k, stride, pad, out_pad, dil, groups) of the transposed pass
+        (2, 1, 5, 7, 6, 9, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 0), (1, 1, 1), 3),
+        (1, 3, 4, 6, 4, 6, (2, 3, 3), (2, 1, 3), (0, 1, 1), (1, 0, 2), (1, 1, 1), 2),
+        (3, 1, 6, 5, 5, 7, (1, 4, 2), (1, 2, 1), (0, 1, 0), (0, 1, 0), (1, 1, 2), 1),
+    ]
+    for N, D, H, W, Ci, Co, k, s, p, op, d, G in geoms:
+        for dt in (torch.float32, torch.float16, torch.bfloat16):
+            x = _t(rng.uniform(-1, 1, (N, D, H, W, Ci))).to(dt)
+            w = _t(rng.standard_normal((Ci, *k, Co // G))).to(dt)
+            y, S = orc.conv_transpose(x, w, s, p, op, d, G)
+            idx = np.concatenate([rng.integers(0, y.size, 300), [0, y.size - 1]])
+            yp, Sp = orc.conv_transpose_points(x, w, idx, s, p, op, d, G)
+            assert np.array_equal(yp, y.ravel()[idx]) and np.array_equal(Sp, S.ravel()[idx])
+
+
 def pin_wgrad_adjoint(orc):
     """The weight gradient is the adjoint of the forward pass in w:
     sum(conv(x, w) * dy) == sum(w * wgrad(x, dy)) exactly for integer data."""
@@ -501,5 +523,6 @@ ALL_PINS = [pin_tutorial_example, pin_output_extent, pin_constant_input, pin_del
             pin_pointwise_is_matmul, pin_im2col_equivalence, pin_torch_witness, pin_linearity,
             pin_translation, pin_groups_split, pin_points_match_full, pin_flip_tutorial_example,
             pin_flip_and_side_padding_torch_witness, pin_side_padding_is_a_crop, pin_transpose_adjoint,
-            pin_transpose_torch_witness, pin_transpose_delta_upsamples, pin_wgrad_adjoint, pin_wgrad_torch_witness,
+            pin_transpose_torch_witness, pin_transpose_delta_upsamples, pin_transpose_points_match_full,
+            pin_wgrad_adjoint, pin_wgrad_torch_witness,
             pin_wgrad_pointwise_is_matmul]

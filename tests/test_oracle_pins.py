@@ -106,6 +106,8 @@ MUTATIONS = {
     "bf16_mantissa_width": [(r"\(double\)\(128 \+ m\), e - 134\)", "(double)(128 + m), e - 133)")],
     "transpose_stride_divisibility_dropped": [(r"if \(num < 0 \|\| num % s\) return -1;", "if (num < 0) return -1;")],
     "transpose_pad_sign": [(r"int64_t num = q \+ p - \(int64_t\)k \* d;", "int64_t num = q - p - (int64_t)k * d;")],
+    "transpose_points_qw_qh_swapped": [(r"int qw = \(int\)\(q % t->Qw\); q /= t->Qw;\n    int qh = \(int\)\(q % t->Qh\); q /= t->Qh;",
+                                        "int qh = (int)(q % t->Qh); q /= t->Qh;\n    int qw = (int)(q % t->Qw); q /= t->Qw;")],
     "transpose_out_channel_index": [(r"\* t->kW \+ kw\) \* Cog \+ cl;", "* t->kW + kw) * Cog + (Cog - 1 - cl);")],
     "wgrad_dy_channel_reversed": [(r"\* t->Wo \+ ow\) \* t->O \+ o\];", "* t->Wo + ow) * t->O + (t->O - 1 - o)];")],
     "wgrad_tap_sign": [(r"int64_t iw = \(int64_t\)ow \* t->s\[2\] - t->p\[2\] \+ \(int64_t\)kw \* t->d\[2\];",
