@@ -49,20 +49,27 @@ PROFILE_DIR = os.path.join(ROOT, "profiles")
 
 # ---------------------------------------------------------------- counting
 
-def out_dims(wl, pad_hi=None):
+def out_dims(wl, pad_hi=None, via_oracle=False):
+    """Output extents from the library, or from the oracle on the CPU arms
+    (which must not load the library)."""
+    if via_oracle:
+        import oracle as C
+        if wl.transpose:
+            return C.convT_out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.out_pad, wl.dil)
+        return C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil, pad_hi)
     import implicit_gemm_convolution_conv2d_b200 as C
     if wl.transpose:
         return C.transpose_out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.out_pad, wl.dil)
     return C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil, pad_hi)
 
 
-def conv_flops(wl, dims=None):
+def conv_flops(wl, dims=None, via_oracle=False):
     """Algorithmic FLOPs: 2 * N * Do*Ho*Wo * O * kD*kH*kW * C/groups (padding taps counted).
     A transposed convolution counts those of the forward pass it is the adjoint
     of: 2 * N * D*H*W (its input pixels) * C * kD*kH*kW * O/groups."""
     if wl.transpose:
         return 2 * wl.N * wl.D * wl.H * wl.W * wl.C * wl.k[0] * wl.k[1] * wl.k[2] * (wl.O // wl.groups)
-    Do, Ho, Wo = dims if dims is not None else out_dims(wl)
+    Do, Ho, Wo = dims if dims is not None else out_dims(wl, via_oracle=via_oracle)
     return 2 * wl.N * Do * Ho * Wo * wl.O * wl.k[0] * wl.k[1] * wl.k[2] * (wl.C // wl.groups)
 
 
@@ -550,8 +557,20 @@ def bench_ours(args):
 def _sample_inputs(wl):
     """The workload's host inputs: (x, w), or (x, dy) for a weight gradient."""
     if wl.wgrad:
-        return WL.make_wgrad_inputs(wl, (wl.N, *out_dims(wl), wl.O))
+        return WL.make_wgrad_inputs(wl, (wl.N, *out_dims(wl, via_oracle=True), wl.O))
     return WL.make_inputs(wl)
+
+
+def host_cpu_model():
+    """The host CPU's model name (Linux /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def _oracle_sample_step(wl, x, w, n_img):
@@ -572,7 +591,7 @@ def cpu_baseline(wl, budget_s=15.0):
     import oracle
     x, w = _sample_inputs(wl)
     one = wl.with_(N=1)
-    f1 = conv_flops(one)
+    f1 = conv_flops(one, via_oracle=True)
     t0 = time.perf_counter()
     _oracle_sample_step(wl, x, w, 1)
     t1 = time.perf_counter() - t0
@@ -586,6 +605,7 @@ def cpu_baseline(wl, budget_s=15.0):
         total_f += f1 * k
         n_img += k
     out = {"value": round(total_f / total_t / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+           "cpu_model": host_cpu_model(),
            "kind": "oracle", "sample": f"first {n_img} of {wl.N} images of {wl.name} ({total_t:.1f} s)"}
     out["single_thread"] = _oracle_single_thread(wl, x, w)
     return out
@@ -598,7 +618,7 @@ def _oracle_single_thread(wl, x, w, max_flops=3e9):
     slab would count mostly padding taps)."""
     import oracle
     sub = wl.with_(N=1)
-    while conv_flops(sub) > max_flops and sub.D > 4:
+    while conv_flops(sub, via_oracle=True) > max_flops and sub.D > 4:
         sub = sub.with_(D=(sub.D + 1) // 2)
     xs = x[:1, :sub.D].contiguous()
     full = oracle.max_threads()
@@ -609,7 +629,7 @@ def _oracle_single_thread(wl, x, w, max_flops=3e9):
         dt = time.perf_counter() - t0
     finally:
         oracle.set_threads(full)
-    return {"value": round(conv_flops(sub) / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+    return {"value": round(conv_flops(sub, via_oracle=True) / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
             "sample": f"image 0 of {wl.name}, depth {sub.D} of {wl.D} ({dt:.1f} s)"}
 
 
@@ -622,7 +642,7 @@ def bench_reference(args):
     wl = WL.WORKLOADS[args.workload]
     x, w = _sample_inputs(wl)
     one = wl.with_(N=1)
-    f1 = conv_flops(one)
+    f1 = conv_flops(one, via_oracle=True)
     # one step = the oracle on one image of the workload (a bounded sample)
     for i in range(args.warmup):
         _oracle_sample_step(wl, x[i % wl.N:], w, 1)
@@ -634,8 +654,11 @@ def bench_reference(args):
     out = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 0, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-           "config": {"workload": wl.name, "sample": "one image per step"},
+           "config": {"workload": wl.name, "global_batch": wl.N,
+                      "sample": f"one image of the {wl.N}-image batch per step (a bounded sample of the same "
+                                f"workload; the metric is per FLOP, so the value compares with the full batch)"},
            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+                            "cpu_model": host_cpu_model(),
                             "kind": "oracle", "sample": f"one image of {wl.name} per step, {args.steps} steps"},
            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)

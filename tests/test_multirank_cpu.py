@@ -120,3 +120,24 @@ def test_transposed_and_weight_gradient_counters():
     assert bench.conv_flops(t) == 2 * 16 * 56 * 56 * 256 * 16 * 128
     g = WL.WORKLOADS["wgrad_bf16_n64_56x56_c256_o256_k3"]
     assert bench.conv_flops(g, (1, 56, 56)) == 2 * 64 * 56 * 56 * 256 * 9 * 256
+
+
+@pytest.mark.timeout(300)
+def test_reference_arm_loads_only_the_oracle():
+    """`bench.py --impl reference` times the oracle and must not map the CUDA
+    library into its process: after a short run, /proc/self/maps holds
+    liboracle.so and no libconvfwd.so; its line carries the CPU model."""
+    import json
+    import subprocess
+    import sys
+    code = ("import sys, json; sys.argv = ['bench.py', '--impl', 'reference', '--steps', '1', '--warmup', '3', "
+            "'--workload', 'conv2d_f16_n1_56x56_c64_o64_k3']; sys.path.insert(0, %r); import bench; bench.main(); "
+            "m = open('/proc/self/maps').read(); "
+            "print(json.dumps({'oracle': 'liboracle.so' in m, 'product': 'libconvfwd.so' in m}))" % ROOT)
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=280)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+    line, maps = lines[0], lines[-1]
+    assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
+    assert "cpu_model" in line["cpu_baseline"]
+    assert maps == {"oracle": True, "product": False}
