@@ -203,6 +203,20 @@ class ClockSampler:
                 return
         self._t.start()
 
+    def sample_now(self):
+        """One NVML sample from the calling thread (used while the timed
+        launches run, so that a region of a few milliseconds has samples)."""
+        if self._nvml is None:
+            return
+        pynvml, h = self._nvml
+        try:
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.samples.append((float(sm), float(mx), int(rs), time.perf_counter()))
+        except Exception:
+            pass
+
     def _poll_nvml(self):
         pynvml, h = self._nvml
         mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
@@ -415,6 +429,9 @@ def bench_ours(args):
         for i in range(args.steps):
             step(args.warmup + i)
     ev1.record(stream)
+    while not ev1.query():      # the launches run: sample the clocks meanwhile
+        clocks.sample_now()
+        time.sleep(0.0002)
     torch.cuda.synchronize(dev)
     t_wall1 = time.perf_counter()
     barrier(dist, dev)
@@ -535,8 +552,8 @@ def bench_ours(args):
         "launch": "cuda_graph_of_steps" if graph is not None else "eager",
         "eager_ms_per_step": round(eager_ms, 5),
         "e2e": e2e,
-        # the weight gradient queues two kernels per call for 16-bit types (the split-K sum, the rounding)
-        "gpu_launches": timed_launches * (2 if wl.wgrad and wl.dtype != "f32" else 1),
+        # the weight gradient queues two kernels per call (the split-K partial sums, their ordered sum)
+        "gpu_launches": timed_launches * (2 if wl.wgrad else 1),
         "clocks": clk,
     }
     if pad_hi is not None or flip:

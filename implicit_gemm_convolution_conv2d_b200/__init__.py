@@ -162,6 +162,11 @@ def conv_fwd(x, w, stride=1, padding=0, dilation=1, groups=1, *, out=None, varia
     (VARIANT_*); the default lets the library choose.  `padding` pads below
     each spatial dimension and, unless `padding_hi` is given, above it too;
     `flip` reads the filter reversed in every spatial dimension.
+
+    The call only queues the kernel.  A kernel that gives up on a pipeline
+    wait (after 2 s) writes no further output and records it in the device
+    status word: check ``last_status()`` (it waits for the stream) before
+    trusting y.
     """
     import torch
     if not (x.is_cuda and w.is_cuda):
@@ -191,7 +196,8 @@ def conv_fwd(x, w, stride=1, padding=0, dilation=1, groups=1, *, out=None, varia
 
 
 def wgrad_workspace_size(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype, pad_hi=None):
-    """Bytes of fp32 workspace conv_wgrad needs for these shapes (0 for f32)."""
+    """Bytes of fp32 workspace conv_wgrad needs for these shapes (one slice of
+    partial sums per range of the split pixel reduction)."""
     code = {"f32": CONV_F32, "f16": CONV_F16, "bf16": CONV_BF16}[dtype]
     out = ctypes.c_ulonglong()
     rc = lib().conv_wgrad_workspace_size(N, D, H, W, C, O, *k, _i3(stride), _i3(pad),
@@ -207,8 +213,9 @@ def conv_wgrad(x, dy, kernel_size, stride=1, padding=0, dilation=1, groups=1, *,
     """Weight gradient of conv_fwd: dw[o, k, c] = sum over output pixels of dy * x.
 
     x: [N, (D,) H, W, C]; dy: [N, (Do,) Ho, Wo, O]; kernel_size: (kD,) kH, kW.
-    Returns dw [O, (kD,) kH, kW, C/groups] in x's dtype.  A 16-bit dtype needs
-    an fp32 workspace; one is allocated with torch when `workspace` is None.
+    Returns dw [O, (kD,) kH, kW, C/groups] in x's dtype.  The call needs an
+    fp32 workspace of wgrad_workspace_size bytes; one is allocated with torch
+    when `workspace` is None.
     """
     import torch
     if not (x.is_cuda and dy.is_cuda):
@@ -349,7 +356,9 @@ def conv_fwd_raw(x_ptr, w_ptr, y_ptr, geom, dtype, variant=VARIANT_AUTO, stream_
 
 def conv_fwd_host(x_host, w_host, y_host, x_dev, w_dev, y_dev, stride=1, padding=0, dilation=1, groups=1,
                   stream=None):
-    """Host-buffer entry point: copies x, w in, runs, copies y out, waits.
+    """Host-buffer entry point: copies x, w in, runs, copies y out, waits
+    (chunks of the batch overlap their copies with the kernels).  Raises
+    ConvError, code -6, when a kernel gave up on a pipeline wait.
 
     x_host/w_host/y_host: CPU tensors (pinned for asynchronous copies);
     x_dev/w_dev/y_dev: CUDA tensors of the same shapes (caller-owned scratch).

@@ -193,8 +193,10 @@ struct DeviceInfo {
   bool init = false;
   int sms = 0;
   bool attrs_set = false;
-  size_t pair_smem = 0;     // dynamic smem the cached cluster count was measured for
-  int pair_clusters = 0;    // CTA pairs that fit on the device at once
+  // CTA pairs that fit on the device at once, per launched pair kernel
+  // (index: halo * 2 + bf16), with the dynamic smem each count was measured for
+  size_t pair_smem[4] = {0, 0, 0, 0};
+  int pair_clusters[4] = {0, 0, 0, 0};
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
@@ -1495,16 +1497,22 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
     // partial wave of pairs would double the tail)
     int clusters = 0;
     {
+      const int slot = (halo ? 2 : 0) + (bf ? 1 : 0);
       std::lock_guard<std::mutex> lk(g_mu);
-      if (g_dev[dev].pair_smem != plan.smem) {
+      if (g_dev[dev].pair_smem[slot] != plan.smem) {
         int c = 0;
-        const cudaError_t oe = halo ? cudaOccupancyMaxActiveClusters(&c, conv_fwd_tc_halo_kernel<false, true>, &cfg)
-                                    : cudaOccupancyMaxActiveClusters(&c, conv_fwd_tc_pair_kernel<false>, &cfg);
+        cudaError_t oe;
+        if (halo)
+          oe = bf ? cudaOccupancyMaxActiveClusters(&c, conv_fwd_tc_halo_kernel<true, true>, &cfg)
+                  : cudaOccupancyMaxActiveClusters(&c, conv_fwd_tc_halo_kernel<false, true>, &cfg);
+        else
+          oe = bf ? cudaOccupancyMaxActiveClusters(&c, conv_fwd_tc_pair_kernel<true>, &cfg)
+                  : cudaOccupancyMaxActiveClusters(&c, conv_fwd_tc_pair_kernel<false>, &cfg);
         if (oe != cudaSuccess || c <= 0) return CONV_ELAUNCH;
-        g_dev[dev].pair_smem = plan.smem;
-        g_dev[dev].pair_clusters = c;
+        g_dev[dev].pair_smem[slot] = plan.smem;
+        g_dev[dev].pair_clusters[slot] = c;
       }
-      clusters = g_dev[dev].pair_clusters;
+      clusters = g_dev[dev].pair_clusters[slot];
     }
     cfg.gridDim = dim3(2 * std::min(plan.ctas / 2, clusters));
     cudaError_t e;
@@ -1607,6 +1615,63 @@ int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStr
   return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
 
+// ---------------------------------------------------------------- host-buffer pipeline
+
+// conv_fwd_host splits the batch into chunks so that the upload of chunk i+1,
+// the kernel on chunk i and the download of chunk i-1 overlap (PCIe carries
+// both directions at once).  Two copy streams and the events that order them
+// are created once per device and kept; a mutex makes calls on one device
+// take turns (the call waits for its result anyway).
+constexpr int kHostMaxChunks = 16;
+constexpr size_t kHostMinChunkBytes = size_t(4) << 20;
+
+struct HostPipe {
+  std::mutex mu;
+  bool init = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, finished = nullptr;
+  cudaEvent_t loaded[kHostMaxChunks] = {}, computed[kHostMaxChunks] = {};
+};
+HostPipe g_host_pipe[kMaxDevices];
+
+int host_pipe_init(HostPipe& hp) {
+  if (hp.init) return CONV_OK;
+  const unsigned f = cudaEventDisableTiming;
+  if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&hp.start, f) != cudaSuccess || cudaEventCreateWithFlags(&hp.finished, f) != cudaSuccess)
+    return CONV_ELAUNCH;
+  for (int i = 0; i < kHostMaxChunks; ++i)
+    if (cudaEventCreateWithFlags(&hp.loaded[i], f) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.computed[i], f) != cudaSuccess)
+      return CONV_ELAUNCH;
+  hp.init = true;
+  return CONV_OK;
+}
+
+// Chunks of whole images, at most kHostMaxChunks, each moving at least
+// kHostMinChunkBytes of x and y (small problems run as one chunk), and one
+// chunk when an image's bytes are not a multiple of 16.
+int host_chunks(const Problem& P) {
+  // chunk offsets must keep the 16-byte alignment the tensor maps need
+  if ((P.x_bytes / P.N) % 16 != 0 || (P.y_bytes / P.N) % 16 != 0) return 1;
+  const long long by_bytes = static_cast<long long>((P.x_bytes + P.y_bytes) / kHostMinChunkBytes);
+  const long long n = std::min<long long>({static_cast<long long>(P.N), static_cast<long long>(kHostMaxChunks),
+                                           std::max<long long>(1, by_bytes)});
+  return static_cast<int>(std::max<long long>(1, n));
+}
+
+// Reads the device status word after the caller's stream has finished; clears
+// it and returns CONV_ETIMEOUT if a kernel gave up on a pipeline wait.
+int read_and_clear_status() {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_conv_status, sizeof(v)) != cudaSuccess) return CONV_ELAUNCH;
+  if (v == 0) return CONV_OK;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(g_conv_status, &zero, sizeof(zero)) != cudaSuccess) return CONV_ELAUNCH;
+  return CONV_ETIMEOUT;
+}
+
 int run(const Problem& P, const void* x, const void* w, void* y, int variant, cudaStream_t st) {
   int dev;
   int rc = current_device(dev);
@@ -1683,14 +1748,55 @@ int conv_fwd_host(const void* x_host, const void* w_host, void* y_host, void* x_
   rc = check_pointers(P, x_dev, w_dev, y_dev);
   if (rc != CONV_OK) return rc;
   if (overlaps(x_dev, P.x_bytes, w_dev, P.w_bytes)) return CONV_EALIAS;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(x_dev, x_host, P.x_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return CONV_ELAUNCH;
-  if (cudaMemcpyAsync(w_dev, w_host, P.w_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return CONV_ELAUNCH;
-  rc = run(P, x_dev, w_dev, y_dev, CONV_VARIANT_AUTO, st);
+  int dev;
+  rc = current_device(dev);
   if (rc != CONV_OK) return rc;
-  if (cudaMemcpyAsync(y_host, y_dev, P.y_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return CONV_ELAUNCH;
+  int sms;
+  rc = device_sms(dev, sms);
+  if (rc != CONV_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Every chunk runs the variant chosen for the whole batch, so the result is
+  // the one conv_fwd gives on the same buffers.
+  const int variant = choose_variant(P, sms);
+  const int nch = host_chunks(P);
+  HostPipe& hp = g_host_pipe[dev];
+  std::lock_guard<std::mutex> lk(hp.mu);
+  rc = host_pipe_init(hp);
+  if (rc != CONV_OK) return rc;
+  const size_t x_img = P.x_bytes / P.N, y_img = P.y_bytes / P.N;
+  const char* xh = static_cast<const char*>(x_host);
+  char* yh = static_cast<char*>(y_host);
+  char* xd = static_cast<char*>(x_dev);
+  char* yd = static_cast<char*>(y_dev);
+  // the copy streams start after the work already queued on the caller's stream
+  if (cudaEventRecord(hp.start, st) != cudaSuccess || cudaStreamWaitEvent(hp.h2d, hp.start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp.d2h, hp.start, 0) != cudaSuccess)
+    return CONV_ELAUNCH;
+  if (cudaMemcpyAsync(w_dev, w_host, P.w_bytes, cudaMemcpyHostToDevice, hp.h2d) != cudaSuccess) return CONV_ELAUNCH;
+  int n0 = 0;
+  for (int i = 0; i < nch; ++i) {
+    const int nc = (P.N - n0) / (nch - i);
+    Problem Pc;
+    rc = make_problem(Pc, nc, D, H, W, C, O, kD, kH, kW, stride, pad, pad, dil, groups, 0, dtype);
+    if (rc != CONV_OK) return rc;
+    // input chunk i on the upload stream (after w), then the kernel on the
+    // caller's stream, then the result chunk on the download stream
+    if (cudaMemcpyAsync(xd + n0 * x_img, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, hp.h2d) != cudaSuccess ||
+        cudaEventRecord(hp.loaded[i], hp.h2d) != cudaSuccess || cudaStreamWaitEvent(st, hp.loaded[i], 0) != cudaSuccess)
+      return CONV_ELAUNCH;
+    rc = run(Pc, xd + n0 * x_img, w_dev, yd + n0 * y_img, variant, st);
+    if (rc == CONV_EUNSUPPORTED) rc = run(Pc, xd + n0 * x_img, w_dev, yd + n0 * y_img, CONV_VARIANT_AUTO, st);
+    if (rc != CONV_OK) return rc;
+    if (cudaEventRecord(hp.computed[i], st) != cudaSuccess || cudaStreamWaitEvent(hp.d2h, hp.computed[i], 0) != cudaSuccess ||
+        cudaMemcpyAsync(yh + n0 * y_img, yd + n0 * y_img, nc * y_img, cudaMemcpyDeviceToHost, hp.d2h) != cudaSuccess)
+      return CONV_ELAUNCH;
+    n0 += nc;
+  }
+  if (cudaEventRecord(hp.finished, hp.d2h) != cudaSuccess || cudaStreamWaitEvent(st, hp.finished, 0) != cudaSuccess)
+    return CONV_ELAUNCH;
   if (cudaStreamSynchronize(st) != cudaSuccess) return CONV_ELAUNCH;
-  return CONV_OK;
+  // a kernel that gave up on a pipeline wait left y partial: report it (and clear the word)
+  return read_and_clear_status();
 }
 
 int conv_plan_ex(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],

@@ -156,8 +156,10 @@ struct __align__(8) TcSmemTail {
   uint64_t rempty[3]; // row staging: every gather thread is done with the buffer
   int seg_n[3][2];    // row staging, per buffer: image of segment 0 / 1
   int seg_lo[3][2];   // first staged input row of segment 0 / 1
+  uint64_t peer_done; // CTA pairs: the peer's producer finished issuing (leader's)
   uint32_t tmem_base;
   volatile int abort_flag;
+  volatile int peer_fills;  // CTA pairs: ring fills the peer's producer issued (leader's)
 };
 
 __device__ __forceinline__ void raise_timeout(volatile int* abort_flag, unsigned site) {
@@ -213,6 +215,46 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, unsign
     }
   }
   return true;
+}
+
+// CTA-pair producers, after their fill loops: every load either CTA issued
+// must have landed before the pair may exit (the loads write the issuing CTA's
+// shared memory and signal the leader's barrier).  The leader can see that
+// only for ring fills it armed.  So the peer (rank 1) publishes how many fills
+// it issued; the leader arms the fills that only the peer issued (with the
+// peer's bytes), counts the peer's bytes of fills that only the leader issued
+// as done, and waits for the last armed phase of every stage.  A stage is at
+// most one phase behind its last armed fill, so one parity wait per stage is
+// exact.  peer_bytes(k) gives the peer's bytes of fill k.
+template <typename PeerBytes>
+__device__ void pair_settle_ring(TcSmemTail* tail, int stages, bool leader, long long fills,
+                                 unsigned long long timeout_ns, PeerBytes peer_bytes) {
+  if (!leader) {
+    ptx::st_shared_cluster_u32(ptx::mapa_shared(ptx::smem_u32(const_cast<int*>(&tail->peer_fills)), 0),
+                               static_cast<uint32_t>(fills));
+    ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(&tail->peer_done), 0));
+    return;
+  }
+  const uint32_t pd = ptx::smem_u32(&tail->peer_done);
+  const uint64_t t0 = ptx::globaltimer_ns();
+  bool heard = true;
+  while (!ptx::mbar_try_wait_cluster(pd, 0u)) {
+    if (ptx::globaltimer_ns() - t0 > timeout_ns) {
+      atomicOr(&g_conv_status, 1u | (kSiteDrain << 8));
+      heard = false;
+      break;
+    }
+  }
+  const long long peer = heard ? static_cast<long long>(static_cast<uint32_t>(tail->peer_fills)) : fills;
+  for (long long k = fills; k < peer; ++k)
+    ptx::mbar_arrive_expect_tx(ptx::smem_u32(&tail->full[k % stages]), peer_bytes(k));
+  for (long long k = peer; k < fills; ++k)
+    ptx::mbar_complete_tx(ptx::smem_u32(&tail->full[k % stages]), peer_bytes(k));
+  const long long total = fills > peer ? fills : peer;
+  for (int s = 0; s < stages; ++s) {
+    const long long arms = total / stages + (s < total % stages ? 1 : 0);
+    if (arms > 0) wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), timeout_ns);
+  }
 }
 
 struct TileCoord {
@@ -1295,7 +1337,9 @@ __global__ void __launch_bounds__(192, 1)
     }
     ptx::mbar_init(ptx::smem_u32(&tail->drain), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
+    ptx::mbar_init(ptx::smem_u32(&tail->peer_done), 1u);
     tail->abort_flag = 0;
+    tail->peer_fills = 0;
     ptx::fence_mbar_init();
   }
   if (threadIdx.x == 32) {
@@ -1366,13 +1410,12 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
-      if (!ok && leader) {
-        for (int s = 0; s < a.stages; ++s) {
-          const long long arms = fills / a.stages + (s < fills % a.stages ? 1 : 0);
-          if (arms > 0)
-            wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
-        }
-      }
+      // fill k of a tile's sequence carries nsub = min(kbs, kblocks - j*kbs) sub-blocks, j = k mod fills per tile
+      const int fpt = (a.kblocks + a.kbs - 1) / a.kbs;
+      pair_settle_ring(tail, a.stages, leader, fills, a.timeout_ns, [&](long long k) {
+        const int j = static_cast<int>(k % fpt);
+        return static_cast<uint32_t>(min(a.kbs, a.kblocks - j * a.kbs)) * (a.a_bytes + a.b_bytes);
+      });
     }
     __syncwarp();
   } else if (warp == 1) {

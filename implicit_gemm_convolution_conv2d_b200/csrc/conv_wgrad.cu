@@ -1,9 +1,11 @@
 // conv_wgrad.cu -- C ABI of the weight gradient (see conv_wgrad.cuh).
 //
 // A separate translation unit of libconvfwd.so: validation, the split of the
-// pixel reduction across blocks, and the launches (zero the fp32 accumulator,
-// the split-K kernel, the rounding kernel for 16-bit outputs).  Allocates
-// nothing: 16-bit outputs accumulate in a caller-provided fp32 workspace.
+// pixel reduction across blocks, and the launches (the split-K kernel, which
+// writes one fp32 partial slice per split into a caller-provided workspace,
+// then the kernel that adds the slices in split order and rounds).  The split
+// count depends on the problem's shape only, so a result is the same bits on
+// every run and every device.  Allocates nothing.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -83,8 +85,26 @@ int wg_make(WgProblem& q, int N, int D, int H, int W, int C, int O, int kD, int 
   return CONV_OK;
 }
 
-size_t wg_workspace(const WgProblem& q) {
-  return q.dtype == CONV_F32 ? 0 : static_cast<size_t>(q.dw_elems) * sizeof(float);
+// Splits of the pixel reduction: enough blocks for two per SM of a 148-SM
+// B200 (a fixed target, so the summation order never depends on the device),
+// each split at least 64 K steps (1024 pixels) long, at most `max_split`.
+constexpr long long kWgTargetBlocks = 2 * 148;
+
+void wg_split(WgArgs& a, long long max_split) {
+  const long long tiles = static_cast<long long>((a.ncols + kWgBN - 1) / kWgBN) * ((a.Og + kWgBM - 1) / kWgBM) * a.G;
+  const long long steps = (a.P + kWgBK - 1) / kWgBK;
+  long long ns = std::max<long long>(1, (kWgTargetBlocks + tiles - 1) / tiles);
+  ns = std::min<long long>(ns, std::max<long long>(1, steps / 64));
+  ns = std::min<long long>(ns, 65535 / a.G);
+  ns = std::min<long long>(ns, max_split);
+  a.nsplit = static_cast<int>(std::max<long long>(1, ns));
+  a.chunk = (steps + a.nsplit - 1) / a.nsplit * kWgBK;
+}
+
+size_t wg_workspace(const WgProblem& q, long long max_split = 1LL << 30) {
+  WgArgs a = q.a;
+  wg_split(a, max_split);
+  return static_cast<size_t>(a.nsplit) * static_cast<size_t>(q.dw_elems) * sizeof(float);
 }
 
 bool wg_overlaps(const void* a, size_t an, const void* b, size_t bn) {
@@ -92,16 +112,45 @@ bool wg_overlaps(const void* a, size_t an, const void* b, size_t bn) {
   return a0 < b0 + bn && b0 < a0 + an;
 }
 
-// Splits of the pixel reduction: enough blocks for two per SM, each split at
-// least 64 K steps (1024 pixels) long.
-void wg_split(WgArgs& a, int sms) {
-  const long long tiles = static_cast<long long>((a.ncols + kWgBN - 1) / kWgBN) * ((a.Og + kWgBM - 1) / kWgBM) * a.G;
-  const long long steps = (a.P + kWgBK - 1) / kWgBK;
-  long long ns = std::max<long long>(1, (2LL * sms + tiles - 1) / tiles);
-  ns = std::min<long long>(ns, std::max<long long>(1, steps / 64));
-  ns = std::min<long long>(ns, 65535 / a.G);
-  a.nsplit = static_cast<int>(std::max<long long>(1, ns));
-  a.chunk = (steps + a.nsplit - 1) / a.nsplit * kWgBK;
+// Validates the buffers and queues the split-K kernel and the reduction,
+// with at most `max_split` splits.
+int wg_launch(const WgProblem& q, const void* x, const void* dy, void* dw, void* workspace,
+              unsigned long long workspace_bytes, long long max_split, cudaStream_t st) {
+  if (!x || !dy || !dw) return CONV_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(dw)) & 15)
+    return CONV_EALIGN;
+  if (wg_overlaps(dw, q.dw_bytes, x, q.x_bytes) || wg_overlaps(dw, q.dw_bytes, dy, q.dy_bytes)) return CONV_EALIAS;
+  WgArgs a = q.a;
+  wg_split(a, max_split);
+  const size_t ws = static_cast<size_t>(a.nsplit) * static_cast<size_t>(q.dw_elems) * sizeof(float);
+  if (!workspace || workspace_bytes < ws) return CONV_EINVAL;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15) return CONV_EALIGN;
+  if (wg_overlaps(workspace, ws, x, q.x_bytes) || wg_overlaps(workspace, ws, dy, q.dy_bytes) ||
+      wg_overlaps(workspace, ws, dw, q.dw_bytes))
+    return CONV_EALIAS;
+  if ((q.dw_elems + 255) / 256 > 0x7fffffffLL) return CONV_EUNSUPPORTED;
+  a.x = x;
+  a.dy = dy;
+  a.part = static_cast<float*>(workspace);
+  const dim3 grid(static_cast<unsigned>((a.ncols + kWgBN - 1) / kWgBN), static_cast<unsigned>((a.Og + kWgBM - 1) / kWgBM),
+                  static_cast<unsigned>(a.G * a.nsplit));
+  if (grid.y > 65535 || grid.z > 65535) return CONV_EUNSUPPORTED;
+  const int dtype = q.dtype;
+  if (dtype == CONV_F32) conv_wgrad_kernel<float><<<grid, kWgThreads, 0, st>>>(a);
+  else if (dtype == CONV_F16) conv_wgrad_kernel<__half><<<grid, kWgThreads, 0, st>>>(a);
+  else conv_wgrad_kernel<__nv_bfloat16><<<grid, kWgThreads, 0, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
+  const long long n = q.dw_elems;
+  const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
+  if (dtype == CONV_F32)
+    conv_wgrad_reduce_kernel<float><<<blocks, 256, 0, st>>>(a.part, static_cast<float*>(dw), n, a.nsplit);
+  else if (dtype == CONV_F16)
+    conv_wgrad_reduce_kernel<__half><<<blocks, 256, 0, st>>>(a.part, static_cast<__half*>(dw), n, a.nsplit);
+  else
+    conv_wgrad_reduce_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(a.part, static_cast<__nv_bfloat16*>(dw), n,
+                                                                    a.nsplit);
+  if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
+  return CONV_OK;
 }
 
 constexpr size_t kWgStaticScratchBytes = CONV_WGRAD_STATIC_SCRATCH_BYTES;
@@ -151,50 +200,9 @@ int conv_wgrad(const void* x, const void* dy, void* dw, int N, int D, int H, int
                int kW, const int stride[3], const int pad_lo[3], const int pad_hi[3], const int dil[3], int groups,
                int dtype, void* workspace, unsigned long long workspace_bytes, conv_stream_t stream) {
   WgProblem q;
-  int rc = wg_make(q, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, dtype);
+  const int rc = wg_make(q, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, dtype);
   if (rc != CONV_OK) return rc;
-  if (!x || !dy || !dw) return CONV_EINVAL;
-  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(dw)) & 15)
-    return CONV_EALIGN;
-  if (wg_overlaps(dw, q.dw_bytes, x, q.x_bytes) || wg_overlaps(dw, q.dw_bytes, dy, q.dy_bytes)) return CONV_EALIAS;
-  const size_t ws = wg_workspace(q);
-  if (ws > 0) {
-    if (!workspace || workspace_bytes < ws) return CONV_EINVAL;
-    if (reinterpret_cast<uintptr_t>(workspace) & 15) return CONV_EALIGN;
-    if (wg_overlaps(workspace, ws, x, q.x_bytes) || wg_overlaps(workspace, ws, dy, q.dy_bytes) ||
-        wg_overlaps(workspace, ws, dw, q.dw_bytes))
-      return CONV_EALIAS;
-  }
-  if ((q.dw_elems + 255) / 256 > 0x7fffffffLL) return CONV_EUNSUPPORTED;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ELAUNCH;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return CONV_ELAUNCH;
-  WgArgs a = q.a;
-  wg_split(a, sms);
-  a.x = x;
-  a.dy = dy;
-  a.acc = ws > 0 ? static_cast<float*>(workspace) : static_cast<float*>(dw);
-  const dim3 grid(static_cast<unsigned>((a.ncols + kWgBN - 1) / kWgBN), static_cast<unsigned>((a.Og + kWgBM - 1) / kWgBM),
-                  static_cast<unsigned>(a.G * a.nsplit));
-  if (grid.y > 65535 || grid.z > 65535) return CONV_EUNSUPPORTED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(a.acc, 0, static_cast<size_t>(q.dw_elems) * sizeof(float), st) != cudaSuccess)
-    return CONV_ELAUNCH;
-
-  if (dtype == CONV_F32) conv_wgrad_kernel<float><<<grid, kWgThreads, 0, st>>>(a);
-  else if (dtype == CONV_F16) conv_wgrad_kernel<__half><<<grid, kWgThreads, 0, st>>>(a);
-  else conv_wgrad_kernel<__nv_bfloat16><<<grid, kWgThreads, 0, st>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
-  if (ws > 0) {
-    const long long n = q.dw_elems;
-    const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
-    if (dtype == CONV_F16)
-      conv_wgrad_round_kernel<__half><<<blocks, 256, 0, st>>>(a.acc, static_cast<__half*>(dw), n);
-    else
-      conv_wgrad_round_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(a.acc, static_cast<__nv_bfloat16*>(dw), n);
-    if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
-  }
-  return CONV_OK;
+  return wg_launch(q, x, dy, dw, workspace, workspace_bytes, 1LL << 30, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int conv_wgrad_noalloc(const void* x, const void* dy, void* dw, int N, int D, int H, int W, int C, int O, int kD,
@@ -203,17 +211,17 @@ int conv_wgrad_noalloc(const void* x, const void* dy, void* dw, int N, int D, in
   WgProblem q;
   const int rc = wg_make(q, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, dtype);
   if (rc != CONV_OK) return rc;
-  const size_t ws = wg_workspace(q);
-  if (ws > kWgStaticScratchBytes) return CONV_ESCRATCH;
+  // as many splits as the static array holds slices (fewer than conv_wgrad
+  // may use, so the two can differ in the last bits)
+  const size_t slice = static_cast<size_t>(q.dw_elems) * sizeof(float);
+  const long long max_split = static_cast<long long>(kWgStaticScratchBytes / slice);
+  if (max_split < 1) return CONV_ESCRATCH;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ELAUNCH;
   void* scratch = nullptr;
-  if (ws > 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ELAUNCH;
-    const int r = wg_static_scratch(dev, &scratch);
-    if (r != CONV_OK) return r;
-  }
-  return conv_wgrad(x, dy, dw, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, dtype, scratch,
-                    ws > 0 ? kWgStaticScratchBytes : 0, stream);
+  const int r = wg_static_scratch(dev, &scratch);
+  if (r != CONV_OK) return r;
+  return wg_launch(q, x, dy, dw, scratch, kWgStaticScratchBytes, max_split, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

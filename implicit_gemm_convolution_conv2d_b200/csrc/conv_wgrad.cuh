@@ -11,11 +11,16 @@
 // output pixels, its B operand being the im2col matrix of x read in place.
 //
 // FP32 FMA kernel: a block computes a 64 x 64 tile of one group's dw over one
-// contiguous range of pixels (split-K across blocks) and adds it into an fp32
-// accumulator with atomics; a second kernel rounds the accumulator to the
-// output type.  Each 16-pixel K step stages dy (16 x 64 output channels) and
-// the im2col rows (16 x 64 weight columns) in shared memory as fp32; a thread
-// owns 4 x 4 outputs.
+// contiguous range of pixels (split-K across blocks) and stores that partial
+// tile, in fp32, into its own slice of a workspace [split][O][taps*Cg]; a
+// second kernel adds the slices of every element in split order and rounds
+// the sum to the output type.  No atomics: the result does not depend on the
+// order in which blocks run.  Each 16-pixel K step stages dy (16 x 64 output
+// channels) and the im2col rows (16 x 64 weight columns) in shared memory as
+// fp32; a thread owns 4 x 4 outputs, which it sums in three levels (a K step
+// into a fresh partial, 16 steps into a segment, segments into the total) so
+// that rounding grows with the number of terms per level, not with the
+// length of the range.
 #pragma once
 
 #include <cstdint>
@@ -38,10 +43,11 @@ struct WgArgs {
   int nsplit;        // splits of the reduction (gridDim.z = G * nsplit)
   const void* x;
   const void* dy;
-  float* acc;        // [O, taps, Cg] fp32 accumulator (zeroed before the launch)
+  float* part;       // [nsplit][O][taps*Cg] fp32 partial sums (every element written)
 };
 
 constexpr int kWgBM = 64, kWgBN = 64, kWgBK = 16, kWgThreads = 256;
+constexpr int kWgSegSteps = 16;  // K steps per segment of the three-level sum
 
 template <typename T>
 __global__ void __launch_bounds__(kWgThreads) conv_wgrad_kernel(const WgArgs a) {
@@ -76,12 +82,13 @@ __global__ void __launch_bounds__(kWgThreads) conv_wgrad_kernel(const WgArgs a) 
     bkd[j] = tap / (a.kW * a.kH);
   }
 
-  float acc[4][4];
+  float acc[4][4], seg[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = seg[i][j] = 0.f;
 
+  int nstep = 0;
   for (long long p0 = p_begin; p0 < p_end; p0 += kWgBK) {
     const long long p = p0 + kk;
     const bool pv = p < p_end;
@@ -118,6 +125,11 @@ __global__ void __launch_bounds__(kWgThreads) conv_wgrad_kernel(const WgArgs a) 
       Bs[kk][tx * 4 + j] = v;
     }
     __syncthreads();
+    float st[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) st[i][j] = 0.f;
 #pragma unroll
     for (int k = 0; k < kWgBK; ++k) {
       const float4 av = *reinterpret_cast<const float4*>(&As[k][ty * 4]);
@@ -127,11 +139,26 @@ __global__ void __launch_bounds__(kWgThreads) conv_wgrad_kernel(const WgArgs a) 
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ar[i], br[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) st[i][j] = fmaf(ar[i], br[j], st[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) seg[i][j] += st[i][j];
+    if (++nstep == kWgSegSteps) {
+      nstep = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j] += seg[i][j];
+          seg[i][j] = 0.f;
+        }
     }
     __syncthreads();
   }
 
+  float* __restrict__ part = a.part + static_cast<long long>(split) * a.O * a.ncols;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int o = o0 + ty * 4 + i;
@@ -139,18 +166,21 @@ __global__ void __launch_bounds__(kWgThreads) conv_wgrad_kernel(const WgArgs a) 
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int col = col0 + tx * 4 + j;
-      if (col < a.ncols)
-        atomicAdd(a.acc + static_cast<long long>(g * a.Og + o) * a.ncols + col, acc[i][j]);
+      if (col < a.ncols) part[static_cast<long long>(g * a.Og + o) * a.ncols + col] = acc[i][j] + seg[i][j];
     }
   }
 }
 
-// dw = the fp32 accumulator rounded to nearest in the output type.
+// dw[i] = the sum of the nsplit partial slices of element i, added in split
+// order in fp32, rounded to nearest in the output type.
 template <typename T>
-__global__ void __launch_bounds__(256) conv_wgrad_round_kernel(const float* __restrict__ acc, T* __restrict__ dw,
-                                                               long long n) {
+__global__ void __launch_bounds__(256) conv_wgrad_reduce_kernel(const float* __restrict__ part, T* __restrict__ dw,
+                                                                long long n, int nsplit) {
   const long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
-  if (i < n) dw[i] = from_f32<T>(acc[i]);
+  if (i >= n) return;
+  float s = part[i];
+  for (int k = 1; k < nsplit; ++k) s += part[static_cast<long long>(k) * n + i];
+  dw[i] = from_f32<T>(s);
 }
 
 }  // namespace convfwd

@@ -166,10 +166,17 @@ int conv_fwd_variant(const void* x, const void* w, void* y,
 
 /* The same computation on HOST buffers x_host, w_host, y_host.  The caller
  * also provides device buffers x_dev, w_dev, y_dev of the matching sizes
- * (the library allocates nothing).  Queues, on `stream`: the two host->device
- * copies, the kernel, the device->host copy of y; then waits for the stream,
- * so y_host holds the result on return.  Host buffers should be page-locked
- * for the copies to be asynchronous. */
+ * (the library allocates no device memory).  The batch is split into chunks
+ * of whole images (up to 16, each moving at least 4 MiB): the upload of a
+ * chunk, the kernel on the previous chunk (on `stream`) and the download of
+ * the one before overlap, on two copy streams the library creates once per
+ * device and orders against `stream` with events.  Every chunk runs the kernel
+ * variant chosen for the whole batch, so y equals conv_fwd's result.  The
+ * call waits for the result, so y_host holds it on return, and then reads and
+ * clears the device status word: CONV_ETIMEOUT means a kernel gave up on a
+ * pipeline wait and y_host is incomplete.  Host buffers should be
+ * page-locked for the copies to be asynchronous.  Calls on one device take
+ * turns. */
 int conv_fwd_host(const void* x_host, const void* w_host, void* y_host,
                   void* x_dev, void* w_dev, void* y_dev,
                   int N, int D, int H, int W, int C, int O,
@@ -252,15 +259,16 @@ int conv_transpose_plan(int N, int D, int H, int W, int Cin, int Cout, int kD, i
  *
  * x: [N, D, H, W, C]; dy: [N, Do, Ho, Wo, O] (the forward output's extents);
  * dw: [O, kD, kH, kW, C/groups], written (not accumulated into).  FP32 FMAs
- * with fp32 accumulation, the pixel reduction split across blocks and summed
- * with fp32 atomics (summation order not deterministic).  f32 outputs are
- * accumulated in dw itself; f16/bf16 outputs need a caller-provided fp32
- * workspace of conv_wgrad_workspace_size bytes (16-byte aligned, disjoint
- * from x, dy, dw), rounded to nearest into dw at the end.  Queues three
- * operations on `stream` (a memset and two kernels); allocates nothing.
- * Errors as for conv_fwd; CONV_EINVAL also for a missing or short workspace. */
+ * with fp32 accumulation.  The pixel reduction is split into ranges; each
+ * range's fp32 partial sums go to their own slice of a caller-provided
+ * workspace of conv_wgrad_workspace_size bytes (16-byte aligned, disjoint from
+ * x, dy, dw), and a second kernel adds the slices in range order and rounds to
+ * nearest into dw.  No atomics, and the split depends on the shape alone, so
+ * a result is the same bits on every run and every device.  Queues two
+ * kernels on `stream`; allocates nothing.  Errors as for conv_fwd;
+ * CONV_EINVAL also for a missing or short workspace. */
 
-/* Bytes of fp32 workspace conv_wgrad needs (0 for f32). */
+/* Bytes of fp32 workspace conv_wgrad needs (any element type). */
 int conv_wgrad_workspace_size(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,
                               const int stride[3], const int pad_lo[3], const int pad_hi[3],
                               const int dil[3], int groups, int dtype, unsigned long long* bytes);
@@ -285,16 +293,21 @@ int conv_wgrad(const void* x, const void* dy, void* dw, int N, int D, int H, int
  * device that loads the library holds that array until the process exits.
  * The call allocates nothing and calls no allocating routine.
  *
- *  - Limit: a 16-bit problem needs O * kD*kH*kW * C/groups * 4 bytes of
- *    scratch (conv_wgrad_workspace_size).  Above the limit the call returns
- *    CONV_ESCRATCH and queues nothing.  f32 problems use no scratch.
+ *  - Limit: each range of the split pixel reduction needs a slice of
+ *    O * kD*kH*kW * C/groups * 4 bytes.  The call splits the reduction as
+ *    conv_wgrad does when those slices fit in the array, else into as many
+ *    ranges as fit (the two entry points may then differ in the last bits).
+ *    A problem whose one slice exceeds CONV_WGRAD_STATIC_SCRATCH_BYTES
+ *    returns CONV_ESCRATCH and queues nothing.
  *  - Set-up: the first call on a device (with that device current) looks up
  *    the array's device address once.  Make that first call before any stream
  *    capture.
- *  - Sharing: every call on a device uses the same array.  Each call clears
- *    it on its stream before use.  Calls whose work overlaps on the GPU (two
- *    streams, or two host threads on different streams) race on it and give
- *    wrong results; order them on one stream or with events.
+ *  - Sharing: every call on a device uses the same array, which keeps the
+ *    last call's contents.  Each call writes every element of the slices it
+ *    uses before reading them, so nothing of an earlier call reaches its
+ *    result.  Calls whose work overlaps on the GPU (two streams, or two host
+ *    threads on different streams) race on the array and give wrong results;
+ *    order them on one stream or with events.
  *
  * Returns as conv_wgrad, plus CONV_ESCRATCH. */
 #define CONV_WGRAD_STATIC_SCRATCH_BYTES (16ull << 20)

@@ -273,14 +273,18 @@ def test_transpose_extents_and_plans(C):
 
 
 def test_wgrad_workspace_and_arguments(C):
-    """The weight gradient's fp32 workspace: O x taps x C/G floats for 16-bit
-    outputs, none for f32; bad shapes are refused on the host."""
+    """The weight gradient's fp32 workspace: one slice of O x taps x C/G floats
+    per range of the split pixel reduction, for every type; the split depends
+    on the shape alone; bad shapes are refused on the host."""
     g = (2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1)
-    assert C.wgrad_workspace_size(*g, "bf16") == 24 * 9 * 16 * 4
-    assert C.wgrad_workspace_size(*g, "f16") == 24 * 9 * 16 * 4
-    assert C.wgrad_workspace_size(*g, "f32") == 0
+    # 144 pixels: too few for a second range
+    for dt in ("bf16", "f16", "f32"):
+        assert C.wgrad_workspace_size(*g, dt) == 24 * 9 * 16 * 4
     assert C.wgrad_workspace_size(2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 4, "bf16") == \
         24 * 9 * 4 * 4
+    # the 3x3 256->256 layer at batch 64: 144 tiles of 64 x 64, so 3 ranges for ~296 blocks
+    big = C.wgrad_workspace_size(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")
+    assert big % (256 * 9 * 256 * 4) == 0 and big // (256 * 9 * 256 * 4) == 3
     with pytest.raises(C.ConvError) as e:   # C not divisible by groups
         C.wgrad_workspace_size(2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 5, "bf16")
     assert e.value.code == -1

@@ -353,9 +353,9 @@ WGRAD = [
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
 @pytest.mark.parametrize("case", WGRAD, ids=lambda c: c[0])
 def test_wgrad_parity(case, dtype):
-    """Weight gradient against the oracle on every element.  The pixel sum is
-    an fp32 reduction of P terms split into chunks, so besides the forward
-    tolerance the bound allows (P + 64) * 2^-24 * S (recursive summation)."""
+    """Weight gradient against the oracle on every element, at the forward
+    pass's tolerance (the pixel sum is split into ranges whose fp32 partial
+    sums are added in a fixed order)."""
     name, N, D, H, W, Cc, O, k, s, p, ph, d, G = case
     gen = torch.Generator().manual_seed(zlib.crc32(name.encode()) % 1000)
     dt = WL.TORCH_DTYPE[dtype]
@@ -367,7 +367,7 @@ def test_wgrad_parity(case, dtype):
     torch.cuda.synchronize()
     assert tuple(g.shape) == g_ref.shape
     P = N * Do * Ho * Wo
-    assert_parity(g.cpu(), g_ref, s_ref, dtype, f"{name}/{dtype}", rel_floor=(P + 64) * 2.0 ** -24)
+    assert_parity(g.cpu(), g_ref, s_ref, dtype, f"{name}/{dtype}")
 
 
 def test_wgrad_2d_api_and_errors():
@@ -380,7 +380,7 @@ def test_wgrad_2d_api_and_errors():
     torch.cuda.synchronize()
     assert tuple(g.shape) == (24, 3, 3, 16)
     g_ref, s_ref = oracle.conv_wgrad(x.cpu().unsqueeze(1), dy.cpu().unsqueeze(1), (1, 3, 3), (1, 1, 1), (0, 1, 1))
-    assert_parity(g.cpu().unsqueeze(1), g_ref, s_ref, "bf16", "wgrad 2-D", rel_floor=(2 * 72 + 64) * 2.0 ** -24)
+    assert_parity(g.cpu().unsqueeze(1), g_ref, s_ref, "bf16", "wgrad 2-D")
     need = C.wgrad_workspace_size(2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")
     assert need == 24 * 9 * 16 * 4
     with pytest.raises(C.ConvError) as e:
@@ -454,6 +454,27 @@ def test_host_buffer_entry_point():
     assert torch.equal(yh, ydev.cpu())
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_host_buffer_entry_point_chunked(dtype):
+    """A batch large enough to be split into chunks whose copies and kernels
+    overlap: the host-buffer result equals the device entry point's, bit for
+    bit (every chunk runs the variant chosen for the whole batch)."""
+    wl = WL.case(16, 1, 56, 56, 64, 128, (1, 3, 3), pad=(0, 1, 1), dtype=dtype, seed=8)
+    x, w = WL.make_inputs(wl)
+    xh, wh = x[:, 0].contiguous().pin_memory(), w[:, 0].contiguous().pin_memory()
+    yh = torch.full((16, 56, 56, 128), float("nan"), dtype=x.dtype).pin_memory()
+    xd, wd = torch.empty_like(xh, device="cuda"), torch.empty_like(wh, device="cuda")
+    yd = torch.empty(yh.shape, dtype=x.dtype, device="cuda")
+    C.conv_fwd_host(xh, wh, yh, xd, wd, yd, stride=1, padding=1)
+    ydev = C.conv_fwd(x[:, 0].cuda(), w[:, 0].cuda(), stride=1, padding=1)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, ydev.cpu())
+    # the same buffers again (the library's copy streams are reused)
+    yh.fill_(float("nan"))
+    C.conv_fwd_host(xh, wh, yh, xd, wd, yd, stride=1, padding=1)
+    assert torch.equal(yh, ydev.cpu())
+
+
 def test_errors_queue_nothing():
     x = torch.zeros(1, 1, 4, 4, 16, dtype=torch.float16, device="cuda")
     w = torch.zeros(16, 1, 3, 3, 16, dtype=torch.float16, device="cuda")
@@ -501,7 +522,7 @@ def test_workload_reduced_batch(name):
         g = C.conv_wgrad(x.cuda(), dy.cuda(), wl.k, stride=wl.stride, padding=wl.pad, dilation=wl.dil,
                          groups=wl.groups)
         torch.cuda.synchronize()
-        assert_parity(g.cpu(), g_ref, s_ref, wl.dtype, name, rel_floor=(wl.N * Do * Ho * Wo + 64) * 2.0 ** -24)
+        assert_parity(g.cpu(), g_ref, s_ref, wl.dtype, name)
         return
     x, w = WL.make_inputs(wl)
     if wl.transpose:
@@ -551,3 +572,42 @@ def test_workload_full_size_sampled(name):
     yv = y.reshape(-1)[torch.as_tensor(idx, device="cuda")].cpu()
     assert_parity(yv, y_ref, s_ref, wl.dtype, name)
     assert torch.isfinite(y.float()).all()
+
+
+@pytest.mark.parametrize("name", list(WL.WORKLOADS))
+def test_workload_full_size_every_element(name):
+    """Every named workload at its full size, in the bench's launch
+    configuration (the library's automatic choice over the whole batch), with
+    every output element checked against the oracle, image by image (the
+    weight gradient in one pass: each weight sums every pixel of the batch)."""
+    wl = WL.WORKLOADS[name]
+    if wl.wgrad:
+        Do, Ho, Wo = C.out_dims(wl.D, wl.H, wl.W, *wl.k, wl.stride, wl.pad, wl.dil)
+        x, dy = WL.make_wgrad_inputs(wl, (wl.N, Do, Ho, Wo, wl.O))
+        g = C.conv_wgrad(x.cuda(), dy.cuda(), wl.k, stride=wl.stride, padding=wl.pad, dilation=wl.dil,
+                         groups=wl.groups)
+        torch.cuda.synchronize()
+        assert C.last_status() == 0
+        g_ref, s_ref = oracle.conv_wgrad(x, dy, wl.k, wl.stride, wl.pad, wl.dil, wl.groups)
+        assert_parity(g.cpu(), g_ref, s_ref, wl.dtype, name)
+        return
+    x, w = WL.make_inputs(wl)
+    if wl.transpose:
+        y = C.conv_transpose(x.cuda(), w.cuda(), stride=wl.stride, padding=wl.pad, output_padding=wl.out_pad,
+                             dilation=wl.dil, groups=wl.groups)
+    else:
+        y = C.conv_fwd(x.cuda(), w.cuda(), stride=wl.stride, padding=wl.pad, dilation=wl.dil, groups=wl.groups)
+    torch.cuda.synchronize()
+    assert C.last_status() == 0
+    y = y.cpu()
+    n2_total = 0
+    for n in range(wl.N):
+        xs = x[n:n + 1].contiguous()
+        if wl.transpose:
+            y_ref, s_ref = oracle.conv_transpose(xs, w, wl.stride, wl.pad, wl.out_pad, wl.dil, wl.groups)
+        else:
+            y_ref, s_ref = oracle.conv_fwd(xs, w, wl.stride, wl.pad, wl.dil, wl.groups)
+        n2, _ = assert_parity(y[n:n + 1], y_ref, s_ref, wl.dtype, f"{name}/image {n}")
+        n2_total += n2
+    # the correctly-rounded clause (reading of the bf16 bound) is needed by very few elements
+    assert n2_total <= max(16, y.numel() // 100000), n2_total

@@ -8,7 +8,8 @@ workspace, so conv_wgrad_noalloc takes its scratch from a fixed array inside
 the library.  These tests call it through the C ABI and check it against
 conv_wgrad, the entry point with a caller workspace, on two calls in a row: the
 array keeps the previous call's contents, so the second call (a smaller
-problem after a larger one) shows whether each call clears what it uses.
+problem after a larger one, split into fewer ranges) shows whether a call
+reads anything it did not write itself.
 This file is collected last on purpose.
 """
 from __future__ import annotations
@@ -34,7 +35,7 @@ ESCRATCH = -9
 # (name, N, D, H, W, C, O, k, stride, pad_lo, pad_hi, dil, groups): the first
 # problem needs more scratch than the second, so stale partial sums would show.
 CALLS = [
-    ("na_large_3d", 2, 4, 12, 10, 48, 64, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1),
+    ("na_large_3d", 4, 8, 16, 16, 48, 64, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1),
     ("na_small_2d_groups", 3, 1, 13, 11, 32, 24, (1, 3, 3), (1, 2, 1), (0, 1, 1), (0, 2, 1), (1, 1, 2), 2),
 ]
 
@@ -45,7 +46,7 @@ def _inputs(case, dtype):
     Do, Ho, Wo = C.out_dims(D, H, W, *k, s, p, d, ph)
     x = (torch.rand((N, D, H, W, Cc), generator=gen) * 2 - 1).to(DT[dtype])
     dy = (torch.rand((N, Do, Ho, Wo, O), generator=gen) * 2 - 1).to(DT[dtype])
-    return x, dy, (N, D, H, W, Cc, O, *k, s, p, ph, d, G), N * Do * Ho * Wo
+    return x, dy, (N, D, H, W, Cc, O, *k, s, p, ph, d, G)
 
 
 def _noalloc(xd, dyd, shape, geom, dtype):
@@ -61,7 +62,7 @@ def test_noalloc_matches_conv_wgrad_on_two_calls(dtype):
         pytest.skip("no CUDA device")
     for case in CALLS:
         name, N, D, H, W, Cc, O, k, s, p, ph, d, G = case
-        x, dy, geom, P = _inputs(case, dtype)
+        x, dy, geom = _inputs(case, dtype)
         xd, dyd = x.cuda(), dy.cuda()
         shape = (O, *k, Cc // G)
         need = C.wgrad_workspace_size(N, D, H, W, Cc, O, k, s, p, d, G, dtype, ph)
@@ -79,9 +80,8 @@ def test_noalloc_matches_conv_wgrad_on_two_calls(dtype):
         tol = rel * np.asarray(s_ref, np.float64).ravel() + ab
         assert np.all(np.abs(a - b) <= tol), f"{name}/{dtype}: no-alloc and workspace results differ"
         # ... and each meets the oracle
-        floor = (P + 64) * 2.0 ** -24
-        assert_parity(g_na.cpu(), g_ref, s_ref, dtype, f"{name}/{dtype}/noalloc", rel_floor=floor)
-        assert_parity(g_ws.cpu(), g_ref, s_ref, dtype, f"{name}/{dtype}/workspace", rel_floor=floor)
+        assert_parity(g_na.cpu(), g_ref, s_ref, dtype, f"{name}/{dtype}/noalloc")
+        assert_parity(g_ws.cpu(), g_ref, s_ref, dtype, f"{name}/{dtype}/workspace")
 
 
 def test_noalloc_rejects_problems_beyond_the_static_scratch():
