@@ -871,8 +871,14 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
     }
   }
   a.sub_bytes = a.a_bytes + (a.b_resident ? 0u : a.b_bytes);
+  // TMA-store epilogue: y rows 16-byte strided, every 32-channel box inside one
+  // group (or clipped by the tensor's own extent when there is one group), row
+  // coordinates within int32; the transposed-convolution phase tiles (rows not
+  // consecutive) keep register stores
+  a.y_tma = (P.O % 8 == 0 && (P.G == 1 || P.Og % 32 == 0) && P.M <= 0x7fffffffLL - 256 && !a.tp_on) ? 1 : 0;
+  a.epi_bytes = a.y_tma ? kEpiRowBytes + 1024u : 0u;  // the staging buffers start on a 1 KB boundary
   const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64 -
-                          a.bres_bytes - 3LL * a.rows_bytes;
+                          a.bres_bytes - 3LL * a.rows_bytes - a.epi_bytes;
   int stages = 0;
   a.kbs = choose_kbs(a.BN, a.kc, a.sub_bytes, avail, 8, stages);
   if (stages < 2) return CONV_EUNSUPPORTED;
@@ -887,7 +893,7 @@ int plan_tc(const Problem& P, int variant, int sms, TcPlan& plan) {
   plan.variant = variant;
   plan.ctas = plan.pair ? 2 * std::min(a.total_tiles, sms / 2) : std::min(a.total_tiles, sms);
   plan.smem = static_cast<size_t>(a.stages) * a.stage_bytes + a.bres_bytes + 3 * static_cast<size_t>(a.rows_bytes) +
-              1024 + sizeof(TcSmemTail) + 64;
+              a.epi_bytes + 1024 + sizeof(TcSmemTail) + 64;
   return CONV_OK;
 }
 
@@ -1223,6 +1229,27 @@ int encode_y_map(const Problem& P, void* y, CUtensorMap& my) {
   return CONV_OK;
 }
 
+// y viewed as [M, O] for the plain-orientation kernels' TMA stores: boxes of
+// 32 channels x 32 pixel rows in the 64-byte swizzle pattern, rows beyond M
+// and channels beyond O clipped.
+int encode_y_rows_map(const Problem& P, void* y, CUtensorMap& my) {
+  std::memset(&my, 0, sizeof(my));
+  const DriverFns& drv = driver_fns();
+  if (!drv.tiled) return CONV_EDRIVER;
+  const CUtensorMapDataType dt =
+      P.dtype == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  cuuint64_t dim[2] = {static_cast<cuuint64_t>(P.O), static_cast<cuuint64_t>(P.M)};
+  cuuint64_t str[1] = {static_cast<cuuint64_t>(P.O) * 2};
+  cuuint32_t box[2] = {32u, 32u};
+  cuuint32_t est[2] = {1, 1};
+  const CUresult r = drv.tiled(&my, dt, 2, y, dim, str, box, est, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  small_tensor_fixup(my, static_cast<size_t>(P.M) * P.O * 2, drv.driver_version);
+  return CONV_OK;
+}
+
 // y viewed as [N, (Do,) Ho, Wo, O] for the transposed halo kernel's TMA
 // stores: boxes of mo (64 or 128) channels x 8 columns x 4 rows, clipped at
 // the edges.
@@ -1472,6 +1499,12 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
   }
   rc = encode_maps(P, a, plan.pair, halo, x, w, mx, mw);
   if (rc != CONV_OK) return rc;
+  CUtensorMap my;
+  std::memset(&my, 0, sizeof(my));
+  if (a.y_tma) {
+    rc = encode_y_rows_map(P, y, my);
+    if (rc != CONV_OK) return rc;
+  }
   const dim3 grid(plan.ctas), block(plan.variant == CONV_VARIANT_TC_TMA ? tc_threads<MODE_TMA>()
                                                                          : tc_threads<MODE_GATHER>());
   const bool bf = P.dtype == CONV_BF16;
@@ -1520,23 +1553,23 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
       e = bf ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_halo_kernel<true, true>, mx, mw, a)
              : cudaLaunchKernelEx(&cfg, conv_fwd_tc_halo_kernel<false, true>, mx, mw, a);
     else
-      e = bf ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_pair_kernel<true>, mx, mw, a)
-             : cudaLaunchKernelEx(&cfg, conv_fwd_tc_pair_kernel<false>, mx, mw, a);
+      e = bf ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_pair_kernel<true>, mx, mw, my, a)
+             : cudaLaunchKernelEx(&cfg, conv_fwd_tc_pair_kernel<false>, mx, mw, my, a);
     return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
   }
   if (plan.variant == CONV_VARIANT_TC_TMA) {
-    if (bf) conv_fwd_tc_kernel<MODE_TMA, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
-    else    conv_fwd_tc_kernel<MODE_TMA, false><<<grid, block, plan.smem, st>>>(mx, mw, a);
+    if (bf) conv_fwd_tc_kernel<MODE_TMA, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
+    else    conv_fwd_tc_kernel<MODE_TMA, false><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
   } else {
     if (a.tp_on) {
-      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true, true, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
-      else    conv_fwd_tc_kernel<MODE_GATHER, false, true, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
+      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true, true, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
+      else    conv_fwd_tc_kernel<MODE_GATHER, false, true, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
     } else if (a.idil_on || a.wtrans) {
-      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
-      else    conv_fwd_tc_kernel<MODE_GATHER, false, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
+      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
+      else    conv_fwd_tc_kernel<MODE_GATHER, false, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
     } else {
-      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true><<<grid, block, plan.smem, st>>>(mx, mw, a);
-      else    conv_fwd_tc_kernel<MODE_GATHER, false><<<grid, block, plan.smem, st>>>(mx, mw, a);
+      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
+      else    conv_fwd_tc_kernel<MODE_GATHER, false><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
     }
   }
   return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;

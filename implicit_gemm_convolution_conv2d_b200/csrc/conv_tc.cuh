@@ -102,6 +102,8 @@ struct TcArgs {
   int mo;             // transposed halo kernel: output channels per tile (MMA M: 64 or 128)
   int b_resident;     // gather: the whole B matrix stays in shared memory
   uint32_t bres_bytes;  // its size (kblocks * BN * 128), 0 when not resident
+  int y_tma;          // plain-orientation kernels: the epilogue stores y by TMA tensor stores
+  uint32_t epi_bytes; // their staging area (kEpiRowBytes + 1 KB alignment slack), 0 when y_tma is off
   int flip;           // 1: the filter is read reversed in every spatial dimension
   int taps;           // kD*kH*kW
   int w_resident;     // transposed halo kernel: all weight tiles loaded once into stage 0
@@ -371,6 +373,44 @@ __device__ __forceinline__ uint16_t cvt1(float v) {
     return *reinterpret_cast<uint16_t*>(&h);
   }
 }
+
+// Plain-orientation epilogue (accumulator lanes = output pixels, columns =
+// output channels): each epilogue warp owns 32 consecutive rows of the tile.
+// Per 32-column chunk it writes its rows' 16-bit values into one of its two
+// 2 KB staging buffers, [32 rows][64 bytes] in the 64-byte swizzle pattern
+// (16-byte chunk j of row r at position j ^ ((r >> 1) & 3), so the 16-byte
+// stores of a warp fall in distinct banks), and lane 0 issues one TMA tensor
+// store of the [32 x 32] box at (column, first row); rows beyond M are clipped
+// by the tensor map.  A buffer is rewritten only after the store issued from
+// it two chunks earlier has read it.
+constexpr uint32_t kEpiWarpBytes = 4096;   // two 2 KB buffers per epilogue warp
+constexpr uint32_t kEpiRowBytes = 4 * kEpiWarpBytes;
+
+template <bool BF16>
+__device__ __forceinline__ void epi_store_chunk_tma(uint8_t* warp_bufs, int seq, const uint32_t (&r)[32],
+                                                    const CUtensorMap* tmap_y, int col, long long row0) {
+  const int lane = threadIdx.x & 31;
+  uint8_t* buf = warp_bufs + (seq & 1) * 2048;
+  if (lane == 0) ptx::bulk_wait_group_read<1>();
+  __syncwarp();
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 v;
+    v.x = pack2<BF16>(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+    v.y = pack2<BF16>(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+    v.z = pack2<BF16>(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+    v.w = pack2<BF16>(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+    *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ sw) << 4)) = v;
+  }
+  ptx::fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    ptx::tma_store_2d(tmap_y, ptx::smem_u32(buf), col, static_cast<int32_t>(row0));
+    ptx::bulk_commit_group();
+  }
+}
+
 
 // ----------------------------------------------------------------------------
 // MMA issue.  One thread issues every tcgen05.mma of a CTA, and on B200 the
@@ -935,7 +975,8 @@ __device__ __forceinline__ void issue_rows(const TcArgs& a, const CUtensorMap* t
 template <int MODE, bool BF16, bool TR = false, bool TP = false>
 __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
     conv_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                       const __grid_constant__ CUtensorMap tmap_w, const TcArgs a) {
+                       const __grid_constant__ CUtensorMap tmap_w,
+                       const __grid_constant__ CUtensorMap tmap_y, const TcArgs a) {
   constexpr int kProdWarps = TcRoles<MODE>::kProducerWarps;
   constexpr int kMmaWarp = kProdWarps;
 
@@ -944,7 +985,10 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* bres = smem + a.stages * a.stage_bytes;  // resident B (gather mode), 1024-aligned
   uint8_t* rowsbuf = bres + a.bres_bytes;            // staged input rows (GATHER_ROWS), 3 buffers
-  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(rowsbuf + 3 * a.rows_bytes);
+  uint8_t* epi_area = rowsbuf + 3 * a.rows_bytes;    // epilogue staging (y_tma), with 1 KB of slack
+  uint8_t* epibuf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(epi_area) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(epi_area + a.epi_bytes);
   constexpr uint32_t kProdThreads = kProdWarps * 32;
 
   const int warp = threadIdx.x >> 5;
@@ -1231,7 +1275,7 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
     const int q = warp & 3;  // tensor-memory lane quarter this warp may access
     const int row = q * 32 + lane;
     uint16_t* __restrict__ y = static_cast<uint16_t*>(a.y);
-    int t = 0;
+    int t = 0, epi_seq = 0;
     for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++t) {
       const int acc = t & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -1253,6 +1297,21 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
       const int n0 = tc.nt * a.BN;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * a.BN);
+      if (!TP && a.y_tma) {
+        // staged TMA stores of this warp's 32 rows (never the phase tiles, whose rows are not consecutive)
+        const long long row0 = static_cast<long long>(tc.mt) * kBM + q * 32;
+        const int ncols = row0 < a.M ? min(a.BN, a.Og - n0) : 0;  // no store starts past the last row
+        for (int c = 0; c < ncols; c += 32) {
+          uint32_t r[32];
+          ptx::tmem_ld_32x32b_x32(taddr + c, r);
+          ptx::tmem_ld_wait();
+          epi_store_chunk_tma<BF16>(epibuf + q * kEpiWarpBytes, epi_seq++, r, &tmap_y, tc.g * a.Og + n0 + c, row0);
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&tail->acc_empty[acc]));
+        continue;
+      }
       const long long ybase = m * a.O + static_cast<long long>(tc.g) * a.Og;
       for (int c = 0; c < a.BN; c += 32) {
         uint32_t r[32];
@@ -1289,6 +1348,8 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&tail->acc_empty[acc]));
     }
+    // every tensor store has read its buffer and written y before exit
+    if (lane == 0 && a.y_tma) ptx::bulk_wait_group<0>();
     __syncwarp();
   }
 
@@ -1315,11 +1376,15 @@ namespace convfwd {
 template <bool BF16>
 __global__ void __launch_bounds__(192, 1)
     conv_fwd_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                            const __grid_constant__ CUtensorMap tmap_w, const TcArgs a) {
+                            const __grid_constant__ CUtensorMap tmap_w,
+                            const __grid_constant__ CUtensorMap tmap_y, const TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(smem + a.stages * a.stage_bytes);
+  uint8_t* epi_area = smem + a.stages * a.stage_bytes;  // epilogue staging (y_tma), with 1 KB of slack
+  uint8_t* epibuf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(epi_area) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+  TcSmemTail* tail = reinterpret_cast<TcSmemTail*>(epi_area + a.epi_bytes);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
@@ -1470,7 +1535,7 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;
     const int row = q * 32 + lane;
     uint16_t* __restrict__ y = static_cast<uint16_t*>(a.y);
-    int t = 0;
+    int t = 0, epi_seq = 0;
     for (int tile = pair; tile < a.total_tiles; tile += npairs, ++t) {
       const int acc = t & 1;
       const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -1482,6 +1547,21 @@ __global__ void __launch_bounds__(192, 1)
       const long long m = static_cast<long long>(tc.mt) * (2 * kBM) + rank * kBM + row;
       const int n0 = tc.nt * a.BN;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * a.BN);
+      if (a.y_tma) {
+        // staged TMA stores of this warp's 32 rows
+        const long long row0 = static_cast<long long>(tc.mt) * (2 * kBM) + rank * kBM + q * 32;
+        const int ncols = row0 < a.M ? min(a.BN, a.Og - n0) : 0;  // no store starts past the last row
+        for (int c = 0; c < ncols; c += 32) {
+          uint32_t r[32];
+          ptx::tmem_ld_32x32b_x32(taddr + c, r);
+          ptx::tmem_ld_wait();
+          epi_store_chunk_tma<BF16>(epibuf + q * kEpiWarpBytes, epi_seq++, r, &tmap_y, tc.g * a.Og + n0 + c, row0);
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(&tail->acc_empty[acc]), 0));
+        continue;
+      }
       const long long ybase = m * a.O + static_cast<long long>(tc.g) * a.Og;
       for (int c = 0; c < a.BN; c += 32) {
         uint32_t r[32];
@@ -1513,6 +1593,8 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(&tail->acc_empty[acc]), 0));
     }
+    // every tensor store has read its buffer and written y before exit
+    if (lane == 0 && a.y_tma) ptx::bulk_wait_group<0>();
     __syncwarp();
   }
 
