@@ -111,6 +111,8 @@ KERNEL_SOURCES = {
     "depthwise_tma": _COMMON_SRC + ["conv_simt.cuh", "conv_dw.cuh"],
     "depthwise_direct": ["conv_fwd.cu", "conv_simt.cuh", "conv_dw.cuh"],
     "simt_wgrad": ["conv_wgrad.cu", "conv_wgrad.cuh", "conv_simt.cuh"],
+    "tcgen05_wgrad_pair": ["conv_fwd.cu", "conv_wgrad.cu", "conv_wgrad.cuh", "conv_wgrad_tc.cuh", "conv_tc.cuh",
+                           "ptx.cuh"],
 }
 
 
@@ -327,8 +329,10 @@ def bench_ours(args):
         e = WL.ELEM_BYTES[wl.dtype]
         wb = e * wl.N * dims[0] * dims[1] * dims[2] * wl.O        # dy
         yb = e * wl.O * wl.k[0] * wl.k[1] * wl.k[2] * (wl.C // wl.groups)  # dw
-        variant, bn, stages, ctas = None, 64, 1, 0
-        vname = "simt_wgrad"
+        wpath, wsplit = C.wgrad_plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil,
+                                     wl.groups, wl.dtype)
+        variant, bn, stages, ctas = None, (256 if wpath == C.WGRAD_TENSOR_CORES else 64), 1, 0
+        vname = C.WGRAD_PATH_NAMES[wpath]
     elif wl.transpose:
         variant, bn, stages, ctas = C.transpose_plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad,
                                                      wl.out_pad, wl.dil, wl.groups, wl.dtype,
@@ -503,7 +507,8 @@ def bench_ours(args):
     # tensor cores for the rest) against the algorithmic bytes at HBM speed.
     sm_mhz = (clk or {}).get("sm_max_mhz") or 1965.0
     alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
-    fma_kernel = wl.wgrad or variant in (C.VARIANT_SIMT, C.VARIANT_DEPTHWISE, C.VARIANT_DEPTHWISE_DIRECT)
+    fma_kernel = (wl.wgrad and vname == "simt_wgrad") or variant in (C.VARIANT_SIMT, C.VARIANT_DEPTHWISE,
+                                                                      C.VARIANT_DEPTHWISE_DIRECT)
     compute_peak = alu_peak if fma_kernel else float(peaks["bf16_tflops"])
     hbm_bound = (xb + wb + yb) / (float(peaks["hbm_gbs"]) * 1e9) > flops / (compute_peak * 1e12)
     tensor_bound = not fma_kernel and not hbm_bound
@@ -539,7 +544,7 @@ def bench_ours(args):
                    **({"pass": "weight gradient (x, dy -> dw)"} if wl.wgrad else {}), "gflop_per_step": round(flops / 1e9, 4),
                    "global_batch": wl.N * nranks, "parallelism": f"independent batches x{nranks}",
                    "variant": vname,
-                   "tile": ([64, 64] if wl.wgrad  # output channels x weight columns per block
+                   "tile": ([bn, bn] if wl.wgrad  # output channels x weight columns per block (or CTA pair)
                             else simt_tile(wl, dims, bn, ctas) if variant == C.VARIANT_SIMT else
                             [4, bn] if variant in (C.VARIANT_DEPTHWISE, C.VARIANT_DEPTHWISE_DIRECT)  # pixels x channels per thread
                             else [bn, 128] if variant == C.VARIANT_TC_TMA_T

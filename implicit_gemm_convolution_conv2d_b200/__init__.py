@@ -16,7 +16,7 @@ import ctypes
 import os
 
 __all__ = ["conv_fwd", "conv_fwd_host", "out_dims", "plan", "conv_transpose", "transpose_out_dims",
-           "transpose_plan", "conv_wgrad", "wgrad_workspace_size", "last_status", "strerror", "lib",
+           "transpose_plan", "conv_wgrad", "wgrad_workspace_size", "wgrad_plan", "last_status", "strerror", "lib",
            "CONV_F32", "CONV_F16", "CONV_BF16", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC_TMA",
            "VARIANT_TC_GATHER", "VARIANT_TC_TMA_PAIR", "VARIANT_TC_HALO", "VARIANT_TC_HALO_PAIR",
            "VARIANT_TC_TMA_T", "VARIANT_TC_HALO_T", "VARIANT_TC_HALO_T_PAIR", "VARIANT_TC_PHASE", "VARIANT_DEPTHWISE", "VARIANT_DEPTHWISE_DIRECT", "ConvError"]
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
         L.conv_wgrad_workspace_size.argtypes = geo_ex[:-2] + [ci, ctypes.POINTER(ctypes.c_ulonglong)]
         L.conv_wgrad.argtypes = [vp, vp, vp] + geo_ex[:-2] + [ci, vp, ctypes.c_ulonglong, vp]
         L.conv_wgrad_noalloc.argtypes = [vp, vp, vp] + geo_ex[:-2] + [ci, vp]
+        L.conv_wgrad_plan.argtypes = geo_ex[:-2] + [ci, i3, i3]
         L.conv_last_status.argtypes = [vp]
         L.conv_debug_inject_stall.argtypes = [ctypes.c_ulonglong]
         L.conv_strerror.argtypes = [ci]
@@ -206,6 +207,22 @@ def wgrad_workspace_size(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype, p
     if rc:
         raise ConvError(rc, "conv_wgrad_workspace_size")
     return out.value
+
+
+WGRAD_FP32, WGRAD_TENSOR_CORES = 0, 1
+WGRAD_PATH_NAMES = {WGRAD_FP32: "simt_wgrad", WGRAD_TENSOR_CORES: "tcgen05_wgrad_pair"}
+
+
+def wgrad_plan(N, D, H, W, C, O, k, stride, pad, dil, groups, dtype, pad_hi=None):
+    """(path, ranges) conv_wgrad takes for these shapes: WGRAD_FP32 or
+    WGRAD_TENSOR_CORES, and the number of ranges of its split pixel reduction."""
+    code = {"f32": CONV_F32, "f16": CONV_F16, "bf16": CONV_BF16}[dtype]
+    path, ns = (ctypes.c_int * 1)(), (ctypes.c_int * 1)()
+    rc = lib().conv_wgrad_plan(N, D, H, W, C, O, *k, _i3(stride), _i3(pad), _i3(pad if pad_hi is None else pad_hi),
+                               _i3(dil), int(groups), code, path, ns)
+    if rc:
+        raise ConvError(rc, "conv_wgrad_plan")
+    return path[0], ns[0]
 
 
 def conv_wgrad(x, dy, kernel_size, stride=1, padding=0, dilation=1, groups=1, *, padding_hi=None, out=None,

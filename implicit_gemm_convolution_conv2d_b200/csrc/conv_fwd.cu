@@ -19,6 +19,8 @@
 #include "conv_halo_t.cuh"
 #include "conv_phase.cuh"
 #include "conv_dw.cuh"
+#include "conv_wgrad.cuh"
+#include "conv_wgrad_tc.cuh"
 
 namespace convfwd {
 namespace {
@@ -246,6 +248,8 @@ int set_kernel_attrs(int dev) {
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_halo_t_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_phase_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_phase_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_wgrad_tc_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_wgrad_tc_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return CONV_ELAUNCH;
   g_dev[dev].attrs_set = true;
   return CONV_OK;
@@ -1723,6 +1727,164 @@ int run(const Problem& P, const void* x, const void* w, void* y, int variant, cu
 }
 
 }  // namespace
+}  // namespace convfwd
+
+// ---------------------------------------------------------------- weight gradient on the tensor cores
+// (called from conv_wgrad.cu; the kernel lives in this translation unit with
+// the device status word and the tensor-map helpers)
+
+namespace convfwd {
+
+constexpr int kWgtKbs = 2;        // 64-pixel sub-blocks per pipeline stage (8 pair MMAs, 1024 tensor cycles)
+constexpr int kWgtPairs = 74;     // CTA pairs of a 148-SM B200: the split target (fixed, so the
+                                  // summation order never depends on the device)
+
+// Can the tensor-core weight gradient run this problem?  16-bit types, whole
+// 256-channel output tiles and 64-channel column blocks per group, and an
+// input geometry the TMA im2col unit describes (as for the forward kernels).
+bool wgrad_tc_fits(const WgArgs& a, int dtype) {
+  if (dtype != CONV_F16 && dtype != CONV_BF16) return false;
+  if (a.Cg % 64 != 0 || a.Og % 256 != 0 || a.C % 8 != 0) return false;
+  const bool rank5 = !(a.D == 1 && a.kD == 1 && a.pd == 0 && a.pd_hi == 0);
+  const int lo = rank5 ? -16 : -128, hi = rank5 ? 15 : 127;
+  const int s[3] = {a.sd, a.sh, a.sw}, p[3] = {a.pd, a.ph, a.pw}, ph[3] = {a.pd_hi, a.ph_hi, a.pw_hi};
+  const int d[3] = {a.dd, a.dh, a.dw}, k[3] = {a.kD, a.kH, a.kW};
+  for (int i = rank5 ? 0 : 1; i < 3; ++i) {
+    if (s[i] > 8) return false;
+    const long long lower = -p[i];
+    const long long upper = static_cast<long long>(ph[i]) - static_cast<long long>(d[i]) * (k[i] - 1);
+    const long long off = static_cast<long long>(d[i]) * (k[i] - 1);
+    if (lower < lo || lower > hi || upper < lo || upper > hi || off > hi) return false;
+  }
+  return a.P + 2LL * kWgtBK * kWgtKbs * kWgtPairs < 0x7fffffffLL;
+}
+
+// Ranges of the pixel reduction for the tensor-core path (a function of the
+// shape and `max_split` only): enough units for every CTA pair of a 148-SM
+// B200, each range at least 8 sub-blocks (512 pixels) long and a whole number
+// of pipeline stages; no range is empty.
+void wgrad_tc_split(const WgArgs& a, long long max_split, int& nsplit, int& chunk_sub) {
+  const long long per_split = static_cast<long long>(a.G) * (a.Og / 256) * ((a.ncols + 255) / 256);
+  const long long total_sub = (a.P + kWgtBK - 1) / kWgtBK;
+  long long ns = std::max<long long>(1, kWgtPairs / per_split);
+  ns = std::min<long long>(ns, std::max<long long>(1, total_sub / 8));
+  ns = std::max<long long>(1, std::min<long long>(ns, max_split));
+  long long cs = (total_sub + ns - 1) / ns;
+  cs = (cs + kWgtKbs - 1) / kWgtKbs * kWgtKbs;
+  nsplit = static_cast<int>((total_sub + cs - 1) / cs);
+  chunk_sub = static_cast<int>(cs);
+}
+
+int wgrad_tc_launch(const WgArgs& w, int dtype, long long max_split, const void* x, const void* dy, float* part,
+                    cudaStream_t st) {
+  int dev;
+  int rc = current_device(dev);
+  if (rc != CONV_OK) return rc;
+  rc = set_kernel_attrs(dev);
+  if (rc != CONV_OK) return rc;
+  WgTcArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.N = w.N; a.D = w.D; a.H = w.H; a.W = w.W; a.C = w.C; a.O = w.O;
+  a.kD = w.kD; a.kH = w.kH; a.kW = w.kW;
+  a.sd = w.sd; a.sh = w.sh; a.sw = w.sw; a.pd = w.pd; a.ph = w.ph; a.pw = w.pw;
+  a.dd = w.dd; a.dh = w.dh; a.dw = w.dw;
+  a.G = w.G; a.Cg = w.Cg; a.Og = w.Og; a.Do = w.Do; a.Ho = w.Ho; a.Wo = w.Wo;
+  a.P = w.P;
+  a.ncols = w.ncols;
+  a.jtiles = (w.ncols + 255) / 256;
+  a.otiles = w.Og / 256;
+  wgrad_tc_split(w, max_split, a.nsplit, a.chunk_sub);
+  const long long units = static_cast<long long>(a.G) * a.otiles * a.jtiles * a.nsplit;
+  if (units > 0x7fffffffLL) return CONV_EUNSUPPORTED;
+  a.total_units = static_cast<int>(units);
+  a.kbs = kWgtKbs;
+  a.stage_bytes = static_cast<uint32_t>(a.kbs) * kWgtSub;
+  const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64;
+  a.stages = static_cast<int>(std::min<long long>(kMaxStages, avail / a.stage_bytes));
+  if (a.stages < 2) return CONV_EUNSUPPORTED;
+  const uint32_t ab = dtype == CONV_BF16 ? 1u : 0u;
+  // fp32 accumulator, both operands MN-major (transpose bits 15 and 16), N = 256, M = 256
+  a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (1u << 15) | (1u << 16) | ((256u >> 3) << 17) | ((256u >> 4) << 24);
+  a.rank5 = (w.D == 1 && w.kD == 1 && w.pd == 0 && w.pd_hi == 0) ? 0 : 1;
+  a.timeout_ns = kWaitTimeoutNs;
+  const unsigned long long stall_ns = g_inject_stall_ns.exchange(0);
+  if (stall_ns != 0) {
+    a.inject_stall = 1;
+    a.timeout_ns = stall_ns;
+  }
+  a.part = part;
+
+  const DriverFns& drv = driver_fns();
+  if (!drv.tiled || !drv.im2col) return CONV_EDRIVER;
+  const CUtensorMapDataType dt = dtype == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t eb = 2;
+  CUtensorMap mx, mdy;
+  std::memset(&mx, 0, sizeof(mx));
+  std::memset(&mdy, 0, sizeof(mdy));
+  // x: im2col over the forward pass's output pixels, boxes of 64 channels x 64 pixels
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t estr[5];
+  int lower[3], upper[3];
+  const int rank = a.rank5 ? 5 : 4;
+  gdim[0] = w.C; gdim[1] = w.W; gdim[2] = w.H;
+  gstr[0] = eb * w.C;
+  gstr[1] = gstr[0] * w.W;
+  gstr[2] = gstr[1] * w.H;
+  estr[0] = 1; estr[1] = w.sw; estr[2] = w.sh;
+  lower[0] = -w.pw; upper[0] = w.pw_hi - w.dw * (w.kW - 1);
+  lower[1] = -w.ph; upper[1] = w.ph_hi - w.dh * (w.kH - 1);
+  if (rank == 5) {
+    gdim[3] = w.D; gdim[4] = w.N;
+    gstr[3] = gstr[2] * w.D;
+    estr[3] = w.sd; estr[4] = 1;
+    lower[2] = -w.pd; upper[2] = w.pd_hi - w.dd * (w.kD - 1);
+  } else {
+    gdim[3] = w.N;
+    estr[3] = 1;
+  }
+  CUresult r = drv.im2col(&mx, dt, rank, const_cast<void*>(x), gdim, gstr, lower, upper, 64u,
+                          static_cast<cuuint32_t>(kWgtBK), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  const size_t x_bytes = static_cast<size_t>(w.N) * w.D * w.H * w.W * w.C * eb;
+  small_tensor_fixup(mx, x_bytes, drv.driver_version);
+  // dy viewed as [P, O] (O innermost), boxes of 64 channels x 64 pixels; rows past P read zeros
+  cuuint64_t ddim[2] = {static_cast<cuuint64_t>(w.O), static_cast<cuuint64_t>(w.P)};
+  cuuint64_t dstr[1] = {static_cast<cuuint64_t>(w.O) * eb};
+  cuuint32_t dbox[2] = {64u, static_cast<cuuint32_t>(kWgtBK)};
+  cuuint32_t dest[2] = {1, 1};
+  r = drv.tiled(&mdy, dt, 2, const_cast<void*>(dy), ddim, dstr, dbox, dest, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  small_tensor_fixup(mdy, static_cast<size_t>(w.P) * w.O * eb, drv.driver_version);
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  const size_t smem = static_cast<size_t>(a.stages) * a.stage_bytes + 1024 + sizeof(TcSmemTail) + 64;
+  int sms = 0;
+  rc = device_sms(dev, sms);
+  if (rc != CONV_OK) return rc;
+  cfg.gridDim = dim3(2 * std::min(a.total_units, sms / 2));
+  cfg.blockDim = dim3(kWgtThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, conv_wgrad_tc_pair_kernel<false>, &cfg) != cudaSuccess ||
+      clusters <= 0)
+    return CONV_ELAUNCH;
+  cfg.gridDim = dim3(2 * std::min(a.total_units, clusters));
+  const cudaError_t e = dtype == CONV_BF16 ? cudaLaunchKernelEx(&cfg, conv_wgrad_tc_pair_kernel<true>, mx, mdy, a)
+                                           : cudaLaunchKernelEx(&cfg, conv_wgrad_tc_pair_kernel<false>, mx, mdy, a);
+  return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+}
+
 }  // namespace convfwd
 
 namespace convfwd {

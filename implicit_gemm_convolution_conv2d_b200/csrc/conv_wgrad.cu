@@ -22,6 +22,14 @@
 static __device__ __align__(256) float g_wgrad_static_scratch[CONV_WGRAD_STATIC_SCRATCH_BYTES / sizeof(float)];
 
 namespace convfwd {
+
+// The tensor-core path (conv_wgrad_tc.cuh; defined in conv_fwd.cu, which holds
+// the device status word and the tensor-map helpers).
+bool wgrad_tc_fits(const WgArgs& a, int dtype);
+void wgrad_tc_split(const WgArgs& a, long long max_split, int& nsplit, int& chunk_sub);
+int wgrad_tc_launch(const WgArgs& w, int dtype, long long max_split, const void* x, const void* dy, float* part,
+                    cudaStream_t st);
+
 namespace {
 
 bool wg_mul_ok(long long a, long long b, long long& r) {
@@ -64,6 +72,7 @@ int wg_make(WgProblem& q, int N, int D, int H, int W, int C, int O, int kD, int 
   a.kD = kD; a.kH = kH; a.kW = kW;
   a.sd = stride[0]; a.sh = stride[1]; a.sw = stride[2];
   a.pd = pad_lo[0]; a.ph = pad_lo[1]; a.pw = pad_lo[2];
+  a.pd_hi = pad_hi[0]; a.ph_hi = pad_hi[1]; a.pw_hi = pad_hi[2];
   a.dd = dil[0]; a.dh = dil[1]; a.dw = dil[2];
   a.G = groups; a.Cg = C / groups; a.Og = O / groups;
   a.Do = out[0]; a.Ho = out[1]; a.Wo = out[2];
@@ -101,10 +110,21 @@ void wg_split(WgArgs& a, long long max_split) {
   a.chunk = (steps + a.nsplit - 1) / a.nsplit * kWgBK;
 }
 
-size_t wg_workspace(const WgProblem& q, long long max_split = 1LL << 30) {
+// Ranges of the pixel reduction for the path the problem runs on: the
+// tensor-core kernel for 16-bit types where it fits, else the FP32 kernel.
+int wg_nsplit(const WgProblem& q, long long max_split) {
+  if (wgrad_tc_fits(q.a, q.dtype)) {
+    int ns = 1, cs = 1;
+    wgrad_tc_split(q.a, max_split, ns, cs);
+    return ns;
+  }
   WgArgs a = q.a;
   wg_split(a, max_split);
-  return static_cast<size_t>(a.nsplit) * static_cast<size_t>(q.dw_elems) * sizeof(float);
+  return a.nsplit;
+}
+
+size_t wg_workspace(const WgProblem& q, long long max_split = 1LL << 30) {
+  return static_cast<size_t>(wg_nsplit(q, max_split)) * static_cast<size_t>(q.dw_elems) * sizeof(float);
 }
 
 bool wg_overlaps(const void* a, size_t an, const void* b, size_t bn) {
@@ -122,6 +142,11 @@ int wg_launch(const WgProblem& q, const void* x, const void* dy, void* dw, void*
   if (wg_overlaps(dw, q.dw_bytes, x, q.x_bytes) || wg_overlaps(dw, q.dw_bytes, dy, q.dy_bytes)) return CONV_EALIAS;
   WgArgs a = q.a;
   wg_split(a, max_split);
+  const bool tc = wgrad_tc_fits(q.a, q.dtype);
+  if (tc) {
+    int cs = 1;
+    wgrad_tc_split(q.a, max_split, a.nsplit, cs);
+  }
   const size_t ws = static_cast<size_t>(a.nsplit) * static_cast<size_t>(q.dw_elems) * sizeof(float);
   if (!workspace || workspace_bytes < ws) return CONV_EINVAL;
   if (reinterpret_cast<uintptr_t>(workspace) & 15) return CONV_EALIGN;
@@ -136,10 +161,15 @@ int wg_launch(const WgProblem& q, const void* x, const void* dy, void* dw, void*
                   static_cast<unsigned>(a.G * a.nsplit));
   if (grid.y > 65535 || grid.z > 65535) return CONV_EUNSUPPORTED;
   const int dtype = q.dtype;
-  if (dtype == CONV_F32) conv_wgrad_kernel<float><<<grid, kWgThreads, 0, st>>>(a);
-  else if (dtype == CONV_F16) conv_wgrad_kernel<__half><<<grid, kWgThreads, 0, st>>>(a);
-  else conv_wgrad_kernel<__nv_bfloat16><<<grid, kWgThreads, 0, st>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
+  if (tc) {
+    const int rc = wgrad_tc_launch(q.a, dtype, max_split, x, dy, a.part, st);
+    if (rc != CONV_OK) return rc;
+  } else {
+    if (dtype == CONV_F32) conv_wgrad_kernel<float><<<grid, kWgThreads, 0, st>>>(a);
+    else if (dtype == CONV_F16) conv_wgrad_kernel<__half><<<grid, kWgThreads, 0, st>>>(a);
+    else conv_wgrad_kernel<__nv_bfloat16><<<grid, kWgThreads, 0, st>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
+  }
   const long long n = q.dw_elems;
   const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
   if (dtype == CONV_F32)
@@ -193,6 +223,17 @@ int conv_wgrad_workspace_size(int N, int D, int H, int W, int C, int O, int kD, 
   if (rc != CONV_OK) return rc;
   if (!bytes) return CONV_EINVAL;
   *bytes = wg_workspace(q);
+  return CONV_OK;
+}
+
+int conv_wgrad_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
+                    const int pad_lo[3], const int pad_hi[3], const int dil[3], int groups, int dtype, int* path,
+                    int* nsplit) {
+  WgProblem q;
+  const int rc = wg_make(q, N, D, H, W, C, O, kD, kH, kW, stride, pad_lo, pad_hi, dil, groups, dtype);
+  if (rc != CONV_OK) return rc;
+  if (path) *path = wgrad_tc_fits(q.a, q.dtype) ? CONV_WGRAD_TENSOR_CORES : CONV_WGRAD_FP32;
+  if (nsplit) *nsplit = wg_nsplit(q, 1LL << 30);
   return CONV_OK;
 }
 

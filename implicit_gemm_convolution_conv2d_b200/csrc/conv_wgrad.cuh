@@ -35,6 +35,7 @@ struct WgArgs {
   int N, D, H, W, C, O;
   int kD, kH, kW;
   int sd, sh, sw, pd, ph, pw, dd, dh, dw;
+  int pd_hi, ph_hi, pw_hi;  // padding above each dimension
   int G, Cg, Og;
   int Do, Ho, Wo;
   int taps, ncols;   // kD*kH*kW, taps*Cg

@@ -258,15 +258,30 @@ int conv_transpose_plan(int N, int D, int H, int W, int Cin, int Cout, int kD, i
  *       x[n, od*sd - pd + kd*dd, oh*sh - ph + kh*dh, ow*sw - pw + kw*dw, g*C/G + c]
  *
  * x: [N, D, H, W, C]; dy: [N, Do, Ho, Wo, O] (the forward output's extents);
- * dw: [O, kD, kH, kW, C/groups], written (not accumulated into).  FP32 FMAs
- * with fp32 accumulation.  The pixel reduction is split into ranges; each
- * range's fp32 partial sums go to their own slice of a caller-provided
- * workspace of conv_wgrad_workspace_size bytes (16-byte aligned, disjoint from
- * x, dy, dw), and a second kernel adds the slices in range order and rounds to
- * nearest into dw.  No atomics, and the split depends on the shape alone, so
- * a result is the same bits on every run and every device.  Queues two
+ * dw: [O, kD, kH, kW, C/groups], written (not accumulated into).  As a GEMM
+ * per group: M = O/G output channels, N = taps * C/G weight columns, and a
+ * reduction over the output pixels, split into ranges.  Two kernels compute
+ * the ranges' fp32 partial sums:
+ *  - CONV_WGRAD_TENSOR_CORES (f16/bf16, C/G % 64 == 0, O/G % 256 == 0, an
+ *    input geometry the TMA im2col unit describes): tcgen05 CTA pairs, 256
+ *    output channels x 256 columns per unit, dy rows and im2col rows of x
+ *    staged by TMA as in the forward pass and read as MN-major operands;
+ *  - CONV_WGRAD_FP32 (everything else): FP32 FMAs.
+ * Each range's partial sums go to their own slice of a caller-provided
+ * workspace of conv_wgrad_workspace_size bytes (16-byte aligned, disjoint
+ * from x, dy, dw); a second kernel adds the slices in range order and rounds
+ * to nearest into dw.  No atomics, and the split depends on the shape alone,
+ * so a result is the same bits on every run and every device.  Queues two
  * kernels on `stream`; allocates nothing.  Errors as for conv_fwd;
  * CONV_EINVAL also for a missing or short workspace. */
+
+enum { CONV_WGRAD_FP32 = 0, CONV_WGRAD_TENSOR_CORES = 1 };
+
+/* The path conv_wgrad takes for these shapes (CONV_WGRAD_*) and the number of
+ * ranges of its pixel reduction (either may be NULL).  Host-only. */
+int conv_wgrad_plan(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW, const int stride[3],
+                    const int pad_lo[3], const int pad_hi[3], const int dil[3], int groups, int dtype, int* path,
+                    int* nsplit);
 
 /* Bytes of fp32 workspace conv_wgrad needs (any element type). */
 int conv_wgrad_workspace_size(int N, int D, int H, int W, int C, int O, int kD, int kH, int kW,

@@ -282,9 +282,13 @@ def test_wgrad_workspace_and_arguments(C):
         assert C.wgrad_workspace_size(*g, dt) == 24 * 9 * 16 * 4
     assert C.wgrad_workspace_size(2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 4, "bf16") == \
         24 * 9 * 4 * 4
-    # the 3x3 256->256 layer at batch 64: 144 tiles of 64 x 64, so 3 ranges for ~296 blocks
-    big = C.wgrad_workspace_size(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")
-    assert big % (256 * 9 * 256 * 4) == 0 and big // (256 * 9 * 256 * 4) == 3
+    # the 3x3 256->256 layer at batch 64.  16-bit: the tensor-core path, 9 tiles of 256 x 256
+    # columns, so 8 ranges for the 74 CTA pairs of a 148-SM B200; f32: the FP32 path, 144 tiles
+    # of 64 x 64, so 3 ranges for ~296 blocks
+    geo = (64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1)
+    slice_bytes = 256 * 9 * 256 * 4
+    assert C.wgrad_workspace_size(*geo, "bf16") == 8 * slice_bytes
+    assert C.wgrad_workspace_size(*geo, "f32") == 3 * slice_bytes
     with pytest.raises(C.ConvError) as e:   # C not divisible by groups
         C.wgrad_workspace_size(2, 1, 9, 8, 16, 24, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 5, "bf16")
     assert e.value.code == -1

@@ -73,3 +73,26 @@ def test_inject_rejects_bad_limits():
         C.inject_stall(0)
     with pytest.raises(C.ConvError):
         C.inject_stall(20_000_000_000)
+
+
+def test_injected_stall_in_the_tensor_core_weight_gradient():
+    """The same hook in the tensor-core weight-gradient kernel (CTA pairs):
+    the stalled launch gives up and the status word reads CONV_ETIMEOUT; the
+    next call matches the oracle."""
+    gen = torch.Generator().manual_seed(23)
+    x = (torch.rand((2, 1, 12, 12, 64), generator=gen) * 2 - 1).to(torch.bfloat16)
+    dy = (torch.rand((2, 1, 12, 12, 256), generator=gen) * 2 - 1).to(torch.bfloat16)
+    xd, dyd = x.cuda(), dy.cuda()
+    assert C.last_status() == 0
+    C.inject_stall(50_000_000)
+    t0 = time.perf_counter()
+    C.conv_wgrad(xd, dyd, (1, 3, 3), padding=(0, 1, 1))
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 10.0
+    assert C.last_status() == ETIMEOUT
+    assert C.last_status() == 0
+    g = C.conv_wgrad(xd, dyd, (1, 3, 3), padding=(0, 1, 1))
+    torch.cuda.synchronize()
+    assert C.last_status() == 0
+    g_ref, s_ref = oracle.conv_wgrad(x, dy, (1, 3, 3), (1, 1, 1), (0, 1, 1))
+    assert_parity(g.cpu(), g_ref, s_ref, "bf16", "wgrad after stall")

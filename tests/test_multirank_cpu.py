@@ -99,7 +99,7 @@ def test_kernel_source_sets_cover_every_kernel():
     sys.path.insert(0, ROOT)
     import bench
     import implicit_gemm_convolution_conv2d_b200 as C
-    names = set(C.VARIANT_NAMES.values()) | {"simt_wgrad"}
+    names = set(C.VARIANT_NAMES.values()) | set(C.WGRAD_PATH_NAMES.values())
     csrc = os.path.join(ROOT, "implicit_gemm_convolution_conv2d_b200", "csrc")
     for name in names:
         assert name in bench.KERNEL_SOURCES, name

@@ -347,6 +347,14 @@ WGRAD = [
     ("wg_depthwise", 2, 1, 12, 12, 32, 32, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1), 32),
     ("wg_split_reduction", 4, 1, 32, 32, 64, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
     ("wg_stem_like", 2, 1, 30, 30, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (0, 3, 3), (1, 1, 1), 1),
+    # tensor-core path (16-bit types; 256-channel output tiles, 64-channel column blocks): a
+    # partial last column tile (9 taps x 64 = 576 columns), groups, 3-D with stride and
+    # per-side padding, a ragged pixel tail, several ranges of the split reduction
+    ("wgt_k3_c64_partial_tile", 2, 1, 14, 13, 64, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+    ("wgt_groups2", 2, 1, 9, 11, 128, 512, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1), 2),
+    ("wgt_3d_s2_side_pad", 1, 6, 9, 10, 64, 256, (3, 3, 3), (2, 2, 1), (1, 1, 1), (0, 1, 2), (1, 1, 2), 1),
+    ("wgt_many_ranges", 4, 1, 33, 31, 128, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+    ("wgt_c256_1x1", 3, 1, 20, 21, 256, 256, (1, 1, 1), (1, 1, 1), (0, 0, 0), (0, 0, 0), (1, 1, 1), 1),
 ]
 
 

@@ -32,9 +32,13 @@ DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 STATIC_SCRATCH_BYTES = 16 << 20
 ESCRATCH = -9
 
-# (name, N, D, H, W, C, O, k, stride, pad_lo, pad_hi, dil, groups): the first
-# problem needs more scratch than the second, so stale partial sums would show.
+# (name, N, D, H, W, C, O, k, stride, pad_lo, pad_hi, dil, groups), in call
+# order, each needing less scratch than the one before, so stale partial sums
+# would show.  The first runs on the tensor-core path with more ranges than the
+# static array holds slices for (conv_wgrad: 4 ranges of 4.5 MiB; here 3);
+# the other two run the FP32 kernel.
 CALLS = [
+    ("na_tc_capped_ranges", 2, 1, 32, 32, 256, 512, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
     ("na_large_3d", 4, 8, 16, 16, 48, 64, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1),
     ("na_small_2d_groups", 3, 1, 13, 11, 32, 24, (1, 3, 3), (1, 2, 1), (0, 1, 1), (0, 2, 1), (1, 1, 2), 2),
 ]
@@ -65,8 +69,8 @@ def test_noalloc_matches_conv_wgrad_on_two_calls(dtype):
         x, dy, geom = _inputs(case, dtype)
         xd, dyd = x.cuda(), dy.cuda()
         shape = (O, *k, Cc // G)
-        need = C.wgrad_workspace_size(N, D, H, W, Cc, O, k, s, p, d, G, dtype, ph)
-        assert need <= STATIC_SCRATCH_BYTES
+        slice_bytes = O * k[0] * k[1] * k[2] * (Cc // G) * 4
+        assert slice_bytes <= STATIC_SCRATCH_BYTES
         g_ws = C.conv_wgrad(xd, dyd, k, stride=s, padding=p, dilation=d, groups=G, padding_hi=ph)
         rc, g_na = _noalloc(xd, dyd, shape, geom, dtype)
         assert rc == 0, C.strerror(rc)
