@@ -272,6 +272,7 @@ struct DwTmaArgs {
   uint32_t w_off;        // byte offset of the filters (after the slabs)
   uint32_t tail_off;     // byte offset of the barriers
   unsigned long long timeout_ns;
+  int inject_stall;      // test hook: consumer warp 0 first waits on a barrier nothing arrives at
 };
 
 constexpr int kDwTmaMaxStages = 4;
@@ -280,6 +281,7 @@ constexpr int kDwTmaP = 4;                           // output columns per block
 struct DwTmaTail {
   uint64_t full[kDwTmaMaxStages];
   uint64_t empty[kDwTmaMaxStages];
+  uint64_t stall;  // never arrived on (the injected-timeout test waits here)
   volatile int abort_flag;
 };
 
@@ -426,6 +428,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), dw_tma_ctas_per_sm(MODE, R, NC
       ptx::mbar_init(ptx::smem_u32(&tail->full[s]), 1u);
       ptx::mbar_init(ptx::smem_u32(&tail->empty[s]), NCW);
     }
+    ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
     tail->abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -486,6 +489,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), dw_tma_ctas_per_sm(MODE, R, NC
   const uint32_t rowb = static_cast<uint32_t>(a.span_w) * colb;
   T* __restrict__ y = static_cast<T*>(g.y);
   const float* wbase = s_w + cv * 4;
+
+  // failure-detection test hook: this warp waits, with the short injected
+  // limit, on a barrier nothing arrives at; it gives up and raises the abort
+  // flag, the other consumers stop at their next wait, the producer drains
+  if (a.inject_stall && warp == 0 &&
+      !wait_bounded_warp(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected))
+    return;
 
   // register-resident weights of the current kd (square filters)
   float2 wreg[MODE == kDwSquare ? K : 1][MODE == kDwSquare ? K : 1][2];

@@ -191,6 +191,12 @@ int check_pointers(const Problem& P, const void* x, const void* w, const void* y
 
 // ---------------------------------------------------------------- device info
 
+// Test hook (conv_debug_inject_stall): when non-zero, the next launch of a
+// kernel with pipeline waits (the tensor-core kernels, the TMA depthwise
+// kernel) makes one of its threads wait on a barrier that nothing arrives at,
+// with this limit in nanoseconds, so the kernel's timeout path runs.  One-shot.
+std::atomic<unsigned long long> g_inject_stall_ns{0};
+
 struct DeviceInfo {
   bool init = false;
   int sms = 0;
@@ -1180,6 +1186,12 @@ int launch_dw(const Problem& P, const void* x, const void* w, void* y, cudaStrea
   size_t smem;
   if (plan_dw_tma(P, sms, t, f, grid, smem) != CONV_OK) return launch_dw_direct(P, x, w, y, st);
   t.d.x = x; t.d.w = w; t.d.y = y;
+  t.inject_stall = 0;
+  const unsigned long long stall_ns = g_inject_stall_ns.exchange(0);
+  if (stall_ns != 0) {
+    t.inject_stall = 1;
+    t.timeout_ns = stall_ns;
+  }
   CUtensorMap m;
   const int rc = encode_dw_map(P, t, x, m);
   if (rc != CONV_OK) return rc;
@@ -1358,10 +1370,6 @@ int encode_maps(const Problem& P, const TcArgs& a, bool pair, bool halo, const v
   return CONV_OK;
 }
 
-// Test hook (conv_debug_inject_stall): when non-zero, the next tensor-core
-// launch makes its MMA thread wait on a barrier that nothing arrives at, with
-// this limit in nanoseconds, so the kernel's timeout path runs.  One-shot.
-std::atomic<unsigned long long> g_inject_stall_ns{0};
 
 // Tensor maps of the phase-packed kernel: overlapping input windows (rows
 // pitch elements apart, inside the input row), plain input rows for the edge
@@ -1604,14 +1612,14 @@ SimtShape simt_shape(const Problem& P, int sms) {
   return sh;
 }
 
-template <typename T, int TM, bool TR>
+template <typename T, int TM, bool TR, bool MASK = false>
 cudaError_t launch_simt_tn(int tn, dim3 grid, cudaStream_t st, const SimtArgs& a) {
   switch (tn) {
-    case 2: conv_fwd_simt_kernel<T, TM, 2, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
-    case 5: conv_fwd_simt_kernel<T, TM, 5, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
-    case 6: conv_fwd_simt_kernel<T, TM, 6, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
-    case 8: conv_fwd_simt_kernel<T, TM, 8, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
-    default: conv_fwd_simt_kernel<T, TM, 4, TR><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 2: conv_fwd_simt_kernel<T, TM, 2, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 5: conv_fwd_simt_kernel<T, TM, 5, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 6: conv_fwd_simt_kernel<T, TM, 6, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 8: conv_fwd_simt_kernel<T, TM, 8, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
+    default: conv_fwd_simt_kernel<T, TM, 4, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
   }
   return cudaGetLastError();
 }
@@ -1639,7 +1647,11 @@ int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStr
   cudaError_t e;
   const bool tr = !plain_input(P);
   if (P.dtype == CONV_F32) {
-    e = tr ? launch_simt_tn<float, 4, true>(sh.tn, grid, st, a) : launch_simt_tn<float, 4, false>(sh.tn, grid, st, a);
+    // forward problems with at most 32 filter taps: the masked loader
+    const bool mask = !tr && a.taps <= 32;
+    e = tr ? launch_simt_tn<float, 4, true>(sh.tn, grid, st, a)
+           : (mask ? launch_simt_tn<float, 4, false, true>(sh.tn, grid, st, a)
+                   : launch_simt_tn<float, 4, false>(sh.tn, grid, st, a));
   } else if (P.dtype == CONV_F16) {
     if (tr) conv_fwd_simt_kernel<__half, 4, 4, true><<<grid, kSimtThreads, 0, st>>>(a);
     else conv_fwd_simt_kernel<__half, 4, 4><<<grid, kSimtThreads, 0, st>>>(a);

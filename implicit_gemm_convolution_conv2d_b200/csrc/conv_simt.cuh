@@ -72,11 +72,22 @@ __device__ __forceinline__ bool simt_undilate(int& z, int s, int n) {
 
 // TR: the transposed-convolution form (input dilation, transposed weight
 // layout), a separate instantiation so the forward kernel is unchanged.
-template <typename T, int TM, int TN, bool TR = false>
+// MASK (forward form, at most 32 filter taps): each loader row keeps a bit
+// mask of the taps whose input position lies inside the input and the offset
+// of its window origin, so an element costs a mask test and one add instead
+// of three bounds checks and an index product.
+template <typename T, int TM, int TN, bool TR = false, bool MASK = false>
 __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtArgs a) {
   constexpr int BM = 16 * TM, BN = 16 * TN;
-  __shared__ __align__(16) float As[2][kSimtBK][BM + 4];
-  __shared__ __align__(16) float Bs[2][kSimtBK][BN + 4];
+  // Row strides of BM + 2 and BN + 2 floats (twice an odd number): the loader's
+  // stores (K row kl = lane & 15 of the warp, pixel / channel lr + 16 i with
+  // lr = lane >> 4) then fall in 32 distinct banks; with a stride that is a
+  // multiple of 4, rows kl and kl + 8 shared banks (2-way conflicts on every
+  // store).  The pixel reads are float2 pairs (8-byte aligned rows).
+  static_assert(((BM + 2) / 2) % 2 == 1 && ((BN + 2) / 2) % 2 == 1, "row strides must be 2 x odd");
+  static_assert(TM % 2 == 0, "pixel reads are float2 pairs");
+  __shared__ __align__(16) float As[2][kSimtBK][BM + 2];
+  __shared__ __align__(16) float Bs[2][kSimtBK][BN + 2];
 
   const T* __restrict__ x = static_cast<const T*>(a.x);
   const T* __restrict__ w = static_cast<const T*>(a.w);
@@ -109,6 +120,28 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
     rh0[i] = oh * a.sh - a.ph;
     rw0[i] = ow * a.sw - a.pw;
   }
+  // MASK: the window origin of each loader row (possibly outside the input) as
+  // an element offset, and the taps that land inside the input
+  long long rorg[MASK ? TM : 1];
+  uint32_t rmask[MASK ? TM : 1];
+  if constexpr (MASK) {
+#pragma unroll
+    for (int i = 0; i < TM; ++i) {
+      rorg[i] = rbase[i] + ((static_cast<long long>(rd0[i]) * a.H + rh0[i]) * a.W + rw0[i]) * a.C;
+      uint32_t msk = 0;
+      int t = 0;
+      for (int kd = 0; kd < a.kD; ++kd)
+        for (int kh = 0; kh < a.kH; ++kh)
+          for (int kw = 0; kw < a.kW; ++kw, ++t) {
+            const int zd = rd0[i] + kd * a.dd, zh = rh0[i] + kh * a.dh, zw = rw0[i] + kw * a.dw;
+            if (static_cast<unsigned>(zd) < static_cast<unsigned>(a.D) &&
+                static_cast<unsigned>(zh) < static_cast<unsigned>(a.H) &&
+                static_cast<unsigned>(zw) < static_cast<unsigned>(a.W))
+              msk |= 1u << t;
+          }
+      rmask[i] = rvalid[i] ? msk : 0u;
+    }
+  }
   const T* wrow[TN];
   bool ovalid[TN];
 #pragma unroll
@@ -129,8 +162,16 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
     const int k = k0 + kl;
     const bool kv = k < a.K;
     const int id = kd * a.dd, ih = kh * a.dh, iw = kw * a.dw;
+    if constexpr (MASK) {
+      const int tapk = (kd * a.kH + kh) * a.kW + kw;
+      const long long toff = (static_cast<long long>(id) * a.H + ih) * static_cast<long long>(a.W) * a.C +
+                             static_cast<long long>(iw) * a.C + c;
+      const uint32_t bit = kv ? (1u << tapk) : 0u;
 #pragma unroll
-    for (int i = 0; i < TM; ++i) {
+      for (int i = 0; i < TM; ++i) ra[i] = (rmask[i] & bit) ? to_f32<T>(x[rorg[i] + toff]) : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < (MASK ? 0 : TM); ++i) {
       float v = 0.f;
       int zd = rd0[i] + id, zh = rh0[i] + ih, zw = rw0[i] + iw;
       bool in;
@@ -194,12 +235,10 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
     for (int kk = 0; kk < kSimtBK; ++kk) {
       float ar[TM], br[TN];
 #pragma unroll
-      for (int i = 0; i < TM; i += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(&As[buf][kk][ty * TM + i]);
+      for (int i = 0; i < TM; i += 2) {
+        const float2 v = *reinterpret_cast<const float2*>(&As[buf][kk][ty * TM + i]);
         ar[i] = v.x;
         ar[i + 1] = v.y;
-        ar[i + 2] = v.z;
-        ar[i + 3] = v.w;
       }
 #pragma unroll
       for (int j = 0; j < TN; ++j) br[j] = Bs[buf][kk][tx + 16 * j];

@@ -343,8 +343,10 @@ const char* conv_strerror(int code);
 /* Library version as major*10000 + minor*100 + patch. */
 int conv_version(void);
 
-/* Failure-detection test hook.  The next tensor-core launch on this process
- * makes its MMA thread wait on a pipeline barrier that nothing arrives at,
+/* Failure-detection test hook.  The next launch on this process of a kernel
+ * with pipeline waits (the tensor-core kernels, including the weight
+ * gradient's, and the TMA depthwise kernel) makes its MMA thread (depthwise:
+ * its first consumer warp) wait on a pipeline barrier that nothing arrives at,
  * with a limit of `timeout_ns` (1 ns .. 10 s) instead of the usual 2 s: the
  * wait runs out, the kernel raises its abort flag, every role drains what it
  * has in flight, tensor memory is freed, the kernel returns without writing

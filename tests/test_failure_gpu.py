@@ -35,12 +35,16 @@ def _geom(wl):
 
 
 @pytest.mark.parametrize("variant", ["TC_GATHER", "TC_TMA", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T",
-                                     "TC_HALO_T", "TC_HALO_T_PAIR", "TC_PHASE"])
+                                     "TC_HALO_T", "TC_HALO_T_PAIR", "TC_PHASE", "DEPTHWISE"])
 def test_injected_stall_times_out_and_recovers(variant):
     v = getattr(C, "VARIANT_" + variant)
     O = {"TC_TMA_T": 128, "TC_HALO_T": 128, "TC_HALO_T_PAIR": 256}.get(variant, 64)
     if variant == "TC_PHASE":   # a stem-like layer: 3 input channels, 7x7 at stride 2
         wl = WL.case(2, 1, 20, 24, 3, O, (1, 7, 7), (1, 2, 2), (0, 3, 3), dtype="f16", seed=21)
+    elif variant == "DEPTHWISE":   # one filter per channel; the TMA-staged slabs
+        wl = WL.case(2, 1, 30, 28, 64, 64, (1, 3, 3), pad=(0, 1, 1), groups=64, dtype="f16", seed=21)
+        assert C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil, wl.groups, "f16",
+                      v)[0] == v
     else:
         wl = WL.case(2, 1, 20, 20, 64, O, (1, 3, 3), pad=(0, 1, 1), dtype="f16", seed=21)
     x, w = WL.make_inputs(wl)
