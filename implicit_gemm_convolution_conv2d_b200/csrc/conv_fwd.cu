@@ -21,6 +21,7 @@
 #include "conv_dw.cuh"
 #include "conv_wgrad.cuh"
 #include "conv_wgrad_tc.cuh"
+#include "conv_tconv.cuh"
 
 namespace convfwd {
 namespace {
@@ -256,6 +257,8 @@ int set_kernel_attrs(int dev) {
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_phase_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_wgrad_tc_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_wgrad_tc_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_tconv_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_tconv_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return CONV_ELAUNCH;
   g_dev[dev].attrs_set = true;
   return CONV_OK;
@@ -1202,8 +1205,171 @@ int launch_dw(const Problem& P, const void* x, const void* w, void* y, cudaStrea
   return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
 
+// ---------------------------------------------------------------- transposed convolution by phases
+
+// The phase decomposition of a transposed convolution (conv_tconv.cuh) and
+// whether the TMA-fed phase kernel can run it.  The Problem of a transposed
+// convolution holds the undilated input extents, the stride as input dilation
+// (idil), padding p_lo = d(k-1) - pad and p_hi = p_lo + out_pad.
+int plan_tconv(const Problem& P, int sms, TconvArgs& a, int& ctas, size_t& smem) {
+  if (!P.wtrans || (P.dtype != CONV_F16 && P.dtype != CONV_BF16)) return CONV_EUNSUPPORTED;
+  if (P.Cg % 64 != 0 || P.Og % 128 != 0 || P.O % 8 != 0) return CONV_EUNSUPPORTED;
+  std::memset(&a, 0, sizeof(a));
+  const int in[3] = {P.D, P.H, P.W}, k[3] = {P.kD, P.kH, P.kW}, out[3] = {P.Do, P.Ho, P.Wo};
+  int maxoff[3];
+  for (int i = 0; i < 3; ++i) {
+    const int s = P.idil[i];
+    if (P.d[i] != 1 || s > kTcvMaxStride) return CONV_EUNSUPPORTED;
+    const int pad = (k[i] - 1) - P.p[i];
+    a.s[i] = s;
+    int lower = 0, moff = 0, tm = 0;
+    bool any = false;
+    for (int r = 0; r < s; ++r) {
+      const int kr = (r + pad) % s;
+      const int J = kr < k[i] ? (k[i] - kr + s - 1) / s : 0;
+      const int c = (r + pad - kr) / s;
+      const int T = out[i] > r ? (out[i] - r + s - 1) / s : 0;
+      a.ph_k[i][r] = kr;
+      a.ph_J[i][r] = J;
+      a.ph_c[i][r] = c;
+      a.ph_T[i][r] = T;
+      tm = std::max(tm, T);
+      if (J > 0) {
+        lower = any ? std::min(lower, c - J + 1) : c - J + 1;
+        moff = any ? std::max(moff, c) : c;
+        any = true;
+      }
+    }
+    a.lower[i] = lower;
+    a.Tm[i] = tm;
+    maxoff[i] = moff - lower;
+  }
+  // 2-D problems (one input plane, one filter plane) use a rank-4 walk
+  const bool rank5 = !(P.D == 1 && P.kD == 1 && P.Do == 1 && a.s[0] == 1 && a.lower[0] == 0);
+  const int lo = rank5 ? -16 : -128, hi = rank5 ? 15 : 127;
+  for (int i = rank5 ? 0 : 1; i < 3; ++i) {
+    const long long upper = static_cast<long long>(a.Tm[i]) - in[i] + a.lower[i];
+    if (a.lower[i] < lo || a.lower[i] > hi || upper < lo || upper > hi || maxoff[i] > hi) return CONV_EUNSUPPORTED;
+  }
+  a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.Cin = P.C; a.Cout = P.O;
+  a.G = P.G; a.Cig = P.Cg; a.Cog = P.Og;
+  a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
+  a.Qd = P.Do; a.Qh = P.Ho; a.Qw = P.Wo;
+  a.rank5 = rank5 ? 1 : 0;
+  a.Mph = static_cast<long long>(P.N) * a.Tm[0] * a.Tm[1] * a.Tm[2];
+  if (a.Mph > 0x7fffffffLL - 512) return CONV_EUNSUPPORTED;
+  a.nphase = a.s[0] * a.s[1] * a.s[2];
+  a.BN = P.Og % 256 == 0 ? 256 : 128;
+  a.n_tiles = P.Og / a.BN;
+  a.m_tiles = static_cast<int>((a.Mph + 255) / 256);
+  const long long tt = static_cast<long long>(a.nphase) * P.G * a.n_tiles * a.m_tiles;
+  if (tt > 0x7fffffffLL) return CONV_EUNSUPPORTED;
+  a.total_tiles = static_cast<int>(tt);
+  a.cchunks = P.Cg / 64;
+  a.a_bytes = static_cast<uint32_t>(kBM * 64 * 2);                 // 128 pixels x 64 channels
+  a.b_bytes = static_cast<uint32_t>((a.BN / 2 / 64) * 8192);       // this CTA's 64-channel weight boxes
+  a.sub_bytes = a.a_bytes + a.b_bytes;
+  const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64;
+  int stages = 0;
+  a.kbs = choose_kbs(a.BN, 64, a.sub_bytes, avail, 8, stages);
+  if (stages < 2) return CONV_EUNSUPPORTED;
+  a.stages = stages;
+  a.stage_bytes = static_cast<uint32_t>(a.kbs) * a.sub_bytes;
+  const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
+  // fp32 accumulator, B MN-major (transpose bit 16), N = BN, M = 256
+  a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (1u << 16) | (static_cast<uint32_t>(a.BN >> 3) << 17) |
+            ((256u >> 4) << 24);
+  a.tmem_cols = next_pow2_cols(static_cast<uint32_t>(2 * a.BN));
+  a.timeout_ns = kWaitTimeoutNs;
+  ctas = 2 * std::min(a.total_tiles, sms / 2);
+  smem = static_cast<size_t>(a.stages) * a.stage_bytes + 1024 + sizeof(TcSmemTail) + 64;
+  return CONV_OK;
+}
+
+int launch_tconv(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st, int dev, int sms) {
+  TconvArgs a;
+  int ctas = 0;
+  size_t smem = 0;
+  int rc = plan_tconv(P, sms, a, ctas, smem);
+  if (rc != CONV_OK) return rc;
+  rc = set_kernel_attrs(dev);
+  if (rc != CONV_OK) return rc;
+  a.y = y;
+  const unsigned long long stall_ns = g_inject_stall_ns.exchange(0);
+  if (stall_ns != 0) {
+    a.inject_stall = 1;
+    a.timeout_ns = stall_ns;
+  }
+  const DriverFns& drv = driver_fns();
+  if (!drv.tiled || !drv.im2col) return CONV_EDRIVER;
+  const CUtensorMapDataType dt = P.dtype == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t eb = 2;
+  CUtensorMap mx, mw;
+  std::memset(&mx, 0, sizeof(mx));
+  std::memset(&mw, 0, sizeof(mw));
+  // x: the shared im2col walk of Tm pixels per dimension from the lower corner, stride 1
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  int lower[3], upper[3];
+  const int rank = a.rank5 ? 5 : 4;
+  gdim[0] = P.C; gdim[1] = P.W; gdim[2] = P.H;
+  gstr[0] = eb * P.C;
+  gstr[1] = gstr[0] * P.W;
+  gstr[2] = gstr[1] * P.H;
+  lower[0] = a.lower[2]; upper[0] = a.Tm[2] - P.W + a.lower[2];
+  lower[1] = a.lower[1]; upper[1] = a.Tm[1] - P.H + a.lower[1];
+  if (rank == 5) {
+    gdim[3] = P.D; gdim[4] = P.N;
+    gstr[3] = gstr[2] * P.D;
+    lower[2] = a.lower[0]; upper[2] = a.Tm[0] - P.D + a.lower[0];
+  } else {
+    gdim[3] = P.N;
+  }
+  CUresult r = drv.im2col(&mx, dt, rank, const_cast<void*>(x), gdim, gstr, lower, upper, 64u,
+                          static_cast<cuuint32_t>(kBM), estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  small_tensor_fixup(mx, P.x_bytes, drv.driver_version);
+  // w [Cin][taps][Cout/G] as (co, tap, ci): boxes of 64 co x 1 tap x 64 ci
+  const cuuint64_t taps = static_cast<cuuint64_t>(P.kD) * P.kH * P.kW;
+  cuuint64_t wdim[3] = {static_cast<cuuint64_t>(P.Og), taps, static_cast<cuuint64_t>(P.C)};
+  cuuint64_t wstr[2] = {eb * P.Og, eb * P.Og * taps};
+  cuuint32_t wbox[3] = {64u, 1u, 64u};
+  cuuint32_t west[3] = {1, 1, 1};
+  r = drv.tiled(&mw, dt, 3, const_cast<void*>(w), wdim, wstr, wbox, west, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return CONV_EDRIVER;
+  small_tensor_fixup(mw, P.w_bytes, drv.driver_version);
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(kTcvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, conv_tconv_pair_kernel<false>, &cfg) != cudaSuccess || clusters <= 0)
+    return CONV_ELAUNCH;
+  cfg.gridDim = dim3(2 * std::min(ctas / 2, clusters));
+  const cudaError_t e = P.dtype == CONV_BF16 ? cudaLaunchKernelEx(&cfg, conv_tconv_pair_kernel<true>, mx, mw, a)
+                                             : cudaLaunchKernelEx(&cfg, conv_tconv_pair_kernel<false>, mx, mw, a);
+  return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+}
+
 int choose_variant(const Problem& P, int sms) {
-  if (!plain_input(P)) return P.dtype == CONV_F32 ? CONV_VARIANT_SIMT : CONV_VARIANT_TC_GATHER;
+  if (!plain_input(P)) {
+    if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
+    TconvArgs ta;
+    int c;
+    size_t sm;
+    return plan_tconv(P, sms, ta, c, sm) == CONV_OK ? CONV_VARIANT_TC_TMA_PHASES : CONV_VARIANT_TC_GATHER;
+  }
   if (dw_fits(P)) return CONV_VARIANT_DEPTHWISE;
   if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
   bool r5;
@@ -1732,6 +1898,7 @@ int run(const Problem& P, const void* x, const void* w, void* y, int variant, cu
   if (variant == CONV_VARIANT_SIMT) return launch_simt(P, x, w, y, st, sms);
   if (variant == CONV_VARIANT_DEPTHWISE) return launch_dw(P, x, w, y, st, sms);
   if (variant == CONV_VARIANT_DEPTHWISE_DIRECT) return launch_dw_direct(P, x, w, y, st);
+  if (variant == CONV_VARIANT_TC_TMA_PHASES) return launch_tconv(P, x, w, y, st, dev, sms);
   TcPlan plan;
   rc = plan_tc(P, variant, sms, plan);
   if (rc != CONV_OK) return rc;
@@ -1927,7 +2094,7 @@ int conv_fwd_ex(const void* x, const void* w, void* y, int N, int D, int H, int 
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_DEPTHWISE_DIRECT) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_PHASES) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -2028,7 +2195,7 @@ int conv_transpose(const void* x, const void* w, void* y, int N, int D, int H, i
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_DEPTHWISE_DIRECT) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_PHASES) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -2048,7 +2215,7 @@ namespace {
 
 int plan_problem(const Problem& P, int variant, int* bn, int* stages, int* ctas) {
   int rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_DEPTHWISE_DIRECT) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_PHASES) return CONV_EINVAL;
   int dev, sms = 148;
   if (current_device(dev) == CONV_OK) device_sms(dev, sms);
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
@@ -2070,6 +2237,17 @@ int plan_problem(const Problem& P, int variant, int* bn, int* stages, int* ctas)
     if (bn) *bn = dw_vec(P);
     if (stages) *stages = 1;
     if (ctas) *ctas = static_cast<int>(std::min<long long>(static_cast<long long>(grid.x) * grid.y, 0x7fffffffLL));
+    return variant;
+  }
+  if (variant == CONV_VARIANT_TC_TMA_PHASES) {
+    TconvArgs ta;
+    int c;
+    size_t sm;
+    rc = plan_tconv(P, sms, ta, c, sm);
+    if (rc != CONV_OK) return rc;
+    if (bn) *bn = ta.BN;
+    if (stages) *stages = ta.stages;
+    if (ctas) *ctas = c;
     return variant;
   }
   if (variant == CONV_VARIANT_SIMT) {

@@ -105,7 +105,12 @@ enum {
                                    type, FP32 FMAs: persistent CTAs, input slabs staged by TMA
                                    through an mbarrier ring (DEPTHWISE_DIRECT where the slabs do
                                    not fit); the automatic choice for these shapes */
-  CONV_VARIANT_DEPTHWISE_DIRECT = 11 /* depthwise, loads straight from global memory */
+  CONV_VARIANT_DEPTHWISE_DIRECT = 11, /* depthwise, loads straight from global memory */
+  CONV_VARIANT_TC_TMA_PHASES = 12  /* conv_transpose only: one stride-1 implicit GEMM per
+                                   sub-pixel phase on tcgen05 CTA pairs, A by TMA im2col of
+                                   the undilated input, B straight from w as MN-major tiles
+                                   (f16/bf16, dilation 1, Cin/G % 64 == 0, Cout/G % 128 == 0,
+                                   strides <= 8, a geometry inside the TMA im2col limits) */
 };
 
 /* Output extents.  stride/pad/dil: 3 ints (d, h, w).  out: 3 ints (Do, Ho, Wo).
@@ -231,8 +236,12 @@ int conv_plan_variant(int N, int D, int H, int W, int C, int O, int kD, int kH, 
  * otherwise).  It runs as a forward convolution over the input zero-dilated
  * by the stride (the inserted zeros are never stored: the gather producers and
  * the FP32 kernel skip them when computing addresses) with the mirrored,
- * channel-exchanged filter: variants AUTO (TC_GATHER for f16/bf16, SIMT for
- * f32), TC_GATHER and SIMT; any other variant returns CONV_EUNSUPPORTED.
+ * channel-exchanged filter, or, where it fits, by sub-pixel phases
+ * (CONV_VARIANT_TC_TMA_PHASES): output q = s*t + r takes only the taps
+ * k = (r + p) mod s (mod s), a stride-1 convolution of the undilated input per
+ * phase, fed by TMA.  Variants: AUTO (TC_TMA_PHASES where it fits, else
+ * TC_GATHER for f16/bf16; SIMT for f32), TC_TMA_PHASES, TC_GATHER and SIMT;
+ * any other variant returns CONV_EUNSUPPORTED.
  * Buffers, alignment, streams and errors as for conv_fwd. */
 
 /* Extents (Qd, Qh, Qw) of the transposed convolution. */

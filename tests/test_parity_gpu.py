@@ -284,6 +284,17 @@ TRANSPOSE = [
     ("tp_groups2", 1, 1, 7, 6, 128, 64, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 2),
     ("tp_dil2_s2", 1, 1, 6, 6, 64, 32, (1, 3, 3), (1, 2, 2), (0, 2, 2), (0, 1, 1), (1, 2, 2), 1),
     ("tp_s3_k5", 1, 1, 5, 6, 64, 24, (1, 5, 5), (1, 3, 3), (0, 2, 2), (0, 2, 1), (1, 1, 1), 1),
+    # the TMA-fed phase kernel (Cin/G % 64 == 0, Cout/G % 128 == 0, dilation 1): phases with
+    # 1 and 2 taps and one row fewer than others, phases no tap reaches (zeros), 3-D, groups,
+    # 256-channel tiles at stride 3, stride 1 (a single phase), several 256-row tiles
+    ("tq_k4s2_decoder", 2, 1, 9, 11, 64, 128, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1),
+    ("tq_k3s2_op1", 1, 1, 10, 7, 128, 128, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1), 1),
+    ("tq_k1s2_zero_phases", 2, 1, 6, 5, 64, 128, (1, 1, 1), (1, 2, 2), (0, 0, 0), (0, 1, 1), (1, 1, 1), 1),
+    ("tq_3d", 1, 3, 5, 6, 64, 128, (2, 3, 3), (2, 2, 1), (0, 1, 1), (1, 1, 0), (1, 1, 1), 1),
+    ("tq_groups2", 1, 1, 7, 6, 128, 256, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 2),
+    ("tq_s3_k5_o256", 1, 1, 5, 6, 64, 256, (1, 5, 5), (1, 3, 3), (0, 2, 2), (0, 2, 1), (1, 1, 1), 1),
+    ("tq_stride1", 1, 1, 12, 11, 64, 128, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1),
+    ("tq_many_tiles", 3, 1, 21, 19, 128, 128, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1),
 ]
 
 
@@ -318,7 +329,14 @@ def test_transpose_parity(case, dtype):
     x = (torch.rand((N, D, H, W, Cin), generator=gen) * 2 - 1).to(dt)
     w = (torch.randn((Cin, *k, Cout // G), generator=gen) / (Cin // G * k[0] * k[1] * k[2]) ** 0.5).to(dt)
     y_ref, s_ref = oracle.conv_transpose(x, w, s, p, op, d, G)
-    for v in ([C.VARIANT_SIMT] if dtype == "f32" else [C.VARIANT_TC_GATHER, C.VARIANT_SIMT]) + [C.VARIANT_AUTO]:
+    vs = [C.VARIANT_SIMT] if dtype == "f32" else [C.VARIANT_TC_GATHER, C.VARIANT_SIMT]
+    try:
+        C.transpose_plan(N, D, H, W, Cin, Cout, k, s, p, op, d, G, dtype, C.VARIANT_TC_TMA_PHASES)
+        vs.append(C.VARIANT_TC_TMA_PHASES)
+        assert name.startswith("tq_") or dtype == "f32", "the phase kernel takes an unexpected case"
+    except C.ConvError:
+        assert not (name.startswith("tq_") and dtype != "f32"), f"{name}: the phase kernel refused the case"
+    for v in vs + [C.VARIANT_AUTO]:
         y = run_gpu_transpose(x, w, geom, dtype, v)
         assert_parity(y, y_ref, s_ref, dtype, f"{name}/{dtype}/{C.VARIANT_NAMES.get(v, 'auto')}")
 
