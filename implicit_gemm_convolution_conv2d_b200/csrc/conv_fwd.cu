@@ -1813,8 +1813,10 @@ int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStr
   cudaError_t e;
   const bool tr = !plain_input(P);
   if (P.dtype == CONV_F32) {
-    // forward problems with at most 32 filter taps: the masked loader
-    const bool mask = !tr && a.taps <= 32;
+    // forward problems with at most 32 filter taps and at least 16 channels a
+    // tap: the masked loader (its per-block mask set-up costs more than it
+    // saves when K is a few steps long)
+    const bool mask = !tr && a.taps <= 32 && a.Cg >= 16;
     e = tr ? launch_simt_tn<float, 4, true>(sh.tn, grid, st, a)
            : (mask ? launch_simt_tn<float, 4, false, true>(sh.tn, grid, st, a)
                    : launch_simt_tn<float, 4, false>(sh.tn, grid, st, a));

@@ -642,36 +642,42 @@ __device__ __forceinline__ uint4 mask8(uint4 v, unsigned m) {
   return v;
 }
 
+// The loads of gather_a_span, issued apart from their use so that other work
+// (the B chunks of the same K block) can run while they are in flight.
 template <int NCH>
-__device__ __forceinline__ void gather_a_span(const TcArgs& a, const GatherRow& st, SpanPos& pos, uint8_t* a_tile,
-                                              int r, int chunk0) {
+struct SpanLoads {
+  uint4 b0[NCH], b1[NCH];
+  unsigned hsh[NCH], msk[NCH];
+};
+
+template <int NCH>
+__device__ __forceinline__ void gather_a_span_issue(const TcArgs& a, const GatherRow& st, SpanPos& pos,
+                                                    SpanLoads<NCH>& L) {
   const uint16_t* __restrict__ x = static_cast<const uint16_t*>(a.x);
   int j = pos.j, kh = pos.kh, kd = pos.kd;
   long long rowptr;
   bool rok = gather_span(a, st, kd, kh, rowptr);
   rowptr += static_cast<long long>(st.iw0) * a.C;
-  // phase 1: issue every load of the four chunks (aligned 16-byte blocks that
-  // cover the chunk; the halo and the row ends are masked afterwards)
-  uint4 b0[NCH], b1[NCH];
-  unsigned hsh[NCH], msk[NCH];
+  // every load of the NCH chunks: aligned 16-byte blocks that cover the chunk
+  // (the halo and the row ends are masked when the chunks are stored)
 #pragma unroll
   for (int q = 0; q < NCH; ++q) {
-    b0[q] = make_uint4(0, 0, 0, 0);
-    b1[q] = make_uint4(0, 0, 0, 0);
-    hsh[q] = 0;
-    msk[q] = 0;
+    L.b0[q] = make_uint4(0, 0, 0, 0);
+    L.b1[q] = make_uint4(0, 0, 0, 0);
+    L.hsh[q] = 0;
+    L.msk[q] = 0;
     if (rok && j + 8 > st.jlo && j < st.jhi) {
       const int lo = max(st.jlo - j, 0), hi = min(st.jhi - j, 8);
       const long long e0 = rowptr + j;
       const long long a0 = e0 & ~7LL;
       if (a0 >= 0 && a0 + 16 <= a.x_elems) {
-        hsh[q] = static_cast<unsigned>(e0 - a0);
-        msk[q] = ((1u << hi) - 1u) & ~((1u << lo) - 1u);
-        b0[q] = __ldg(reinterpret_cast<const uint4*>(x + a0));
-        if (hsh[q] != 0) b1[q] = __ldg(reinterpret_cast<const uint4*>(x + a0 + 8));
+        L.hsh[q] = static_cast<unsigned>(e0 - a0);
+        L.msk[q] = ((1u << hi) - 1u) & ~((1u << lo) - 1u);
+        L.b0[q] = __ldg(reinterpret_cast<const uint4*>(x + a0));
+        if (L.hsh[q] != 0) L.b1[q] = __ldg(reinterpret_cast<const uint4*>(x + a0 + 8));
       } else {
-        b0[q] = load8_masked(x + e0, lo, hi);  // at the tensor's ends: element loads
-        msk[q] = 0xFFu;
+        L.b0[q] = load8_masked(x + e0, lo, hi);  // at the tensor's ends: element loads
+        L.msk[q] = 0xFFu;
       }
     }
     j += 8;
@@ -688,9 +694,13 @@ __device__ __forceinline__ void gather_a_span(const TcArgs& a, const GatherRow& 
   pos.j = j;
   pos.kh = kh;
   pos.kd = kd;
-  // phase 2: shift into place, mask, store
+}
+
+// Shift the loaded blocks into place, mask, store.
+template <int NCH>
+__device__ __forceinline__ void gather_a_span_store(const SpanLoads<NCH>& L, uint8_t* a_tile, int r, int chunk0) {
 #pragma unroll
-  for (int q = 0; q < NCH; ++q) store_chunk(a_tile, r, chunk0 + q, mask8(extract8(b0[q], b1[q], hsh[q]), msk[q]));
+  for (int q = 0; q < NCH; ++q) store_chunk(a_tile, r, chunk0 + q, mask8(extract8(L.b0[q], L.b1[q], L.hsh[q]), L.msk[q]));
 }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
@@ -901,9 +911,23 @@ __device__ __forceinline__ void gather_b_block(const TcArgs& a, int g, int n0, i
         }
         v = *reinterpret_cast<const uint4*>(e8);
       } else if (span_layout) {  // (never with flip: the planner uses the other layouts)
+        // the 8 elements at w[o, sp*kW*C + j0 ...] (those past the filter row's
+        // kW*C are zero): two aligned 16-byte loads shifted into place
         const int sp = kp0 / a.Lp;
         const int j0 = kp0 - sp * a.Lp;
-        v = load8_masked(w + rowoff + static_cast<long long>(sp) * L + j0, 0, L - j0);
+        const int cnt = min(8, L - j0);
+        if (cnt > 0) {
+          const long long e0 = rowoff + static_cast<long long>(sp) * L + j0;
+          const long long a0 = e0 & ~7LL;
+          if (a0 + 16 <= static_cast<long long>(a.O) * a.K) {
+            const unsigned h = static_cast<unsigned>(e0 - a0);
+            const uint4 b0 = __ldg(reinterpret_cast<const uint4*>(w + a0));
+            const uint4 b1 = h != 0 ? __ldg(reinterpret_cast<const uint4*>(w + a0 + 8)) : make_uint4(0, 0, 0, 0);
+            v = mask8(extract8(b0, b1, h), (1u << cnt) - 1u);
+          } else {
+            v = load8_masked(w + e0, 0, cnt);  // at the tensor's end: element loads
+          }
+        }
       } else if (a.flip) {
         // K element k = tap*Cg + c multiplies w[o, taps-1-tap, c]
         uint16_t e8[8];
@@ -1173,11 +1197,18 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
               gather_a_tp<kNch>(a, st, tph, kb + j, sa, r, part * kNch);
             else if (a.gather_mode == GATHER_VEC8)
               gather_a_vec8<kNch, TR>(a, st, k0, sa, r, part * kNch);
-            else if (rows_mode || a.gather_mode == GATHER_SPAN) {
-              if (rows_mode) gather_a_rows<kNch>(a, st, pos, sa, r, part * kNch);
-              else gather_a_span<kNch>(a, st, pos, sa, r, part * kNch);
+            else if (rows_mode) {
+              gather_a_rows<kNch>(a, st, pos, sa, r, part * kNch);
               // skip the other threads' chunks of this K block
               for (int i = 0; i < 8 - kNch; ++i) span_step8(a, pos);
+            } else if (a.gather_mode == GATHER_SPAN) {
+              // the A loads are in flight while this thread gathers its share of B
+              SpanLoads<kNch> sl;
+              gather_a_span_issue<kNch>(a, st, pos, sl);
+              for (int i = 0; i < 8 - kNch; ++i) span_step8(a, pos);
+              if (!a.b_resident) gather_b_block<TR>(a, tc.g, n0, kbm * 64, sa + a.a_bytes, tid, kProdThreads);
+              gather_a_span_store<kNch>(sl, sa, r, part * kNch);
+              continue;
             } else
               gather_a_scalar<kNch, TR>(a, st, k0, sa, r, part * kNch);
             if (!a.b_resident) gather_b_block<TR>(a, tc.g, n0, kbm * 64, sa + a.a_bytes, tid, kProdThreads);
