@@ -93,7 +93,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
     }
     ptx::mbar_init(ptx::smem_u32(&tail->drain), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
+    ptx::mbar_init(ptx::smem_u32(&tail->peer_done), 1u);
+    ptx::mbar_init(ptx::smem_u32(&tail->peer_done_a), 1u);
     tail->abort_flag = 0;
+    tail->peer_fills = 0;
+    tail->peer_fills_a = 0;
     ptx::fence_mbar_init();
   }
   if (threadIdx.x == 32) {
@@ -178,12 +182,18 @@ __global__ void __launch_bounds__(kTThreads, 1)
           }
         }
       }
-      // (a pair's loads all complete on the leader's barriers: the leader drains)
-      if (a.w_resident && ok && leader && bfills > 0) {
+      if constexpr (PAIR) {
+        // both CTAs' loads complete on the leader's barriers: the two producers
+        // settle every fill either issued (the resident fill included)
+        const int fpt = (Q + a.kbs - 1) / a.kbs;
+        pair_settle_ring(tail, a.stages, leader, bfills, a.timeout_ns, [&](long long k) {
+          return static_cast<uint32_t>(min(a.kbs, Q - static_cast<int>(k % fpt) * a.kbs)) * a.b_bytes;
+        });
+      } else if (a.w_resident && ok && bfills > 0) {
         // the MMA thread may give up before it waits on the resident fill:
         // the loads must have landed before this CTA can exit
         wait_drain(ptx::smem_u32(&tail->full[0]), 0u, a.timeout_ns);
-      } else if (!ok && leader) {
+      } else if (!ok) {
         for (int s = 0; s < a.stages; ++s) {
           const long long arms = bfills / a.stages + (s < bfills % a.stages ? 1 : 0);
           if (arms > 0) wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
@@ -227,7 +237,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
               }
             }
       }
-      if (!ok && leader) {
+      if constexpr (PAIR) {
+        pair_settle_ring(tail->afull, a.a_slots, &tail->peer_done_a, &tail->peer_fills_a, leader, afills,
+                         a.timeout_ns, [&](long long) { return a.halo_bytes; });
+      } else if (!ok) {
         for (int s = 0; s < a.a_slots; ++s) {
           const long long arms = afills / a.a_slots + (s < afills % a.a_slots ? 1 : 0);
           if (arms > 0) wait_drain(ptx::smem_u32(&tail->afull[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);

@@ -84,7 +84,9 @@ __global__ void __launch_bounds__(kPhThreads, 1)
     ptx::mbar_init(ptx::smem_u32(&tail->stall), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->bres), 1u);
     ptx::mbar_init(ptx::smem_u32(&tail->bready), 2u);  // one arrival per CTA of the pair
+    ptx::mbar_init(ptx::smem_u32(&tail->peer_done), 1u);
     tail->abort_flag = 0;
+    tail->peer_fills = 0;
     ptx::fence_mbar_init();
   }
   if (threadIdx.x == 32) {
@@ -196,11 +198,11 @@ __global__ void __launch_bounds__(kPhThreads, 1)
   const int R = a.ph_rows;
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && !*abort_flag) {
+    if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       long long fills = 0;
-      bool pok = true;
+      bool pok = !*abort_flag;  // (no loads at all after a failed copy of w)
       const int nedge = a.ph_nleft + a.ph_nright;
       const uint32_t bytes = static_cast<uint32_t>((R * a.ph_qint + nedge * R) * kPhWin * 2);
       const int pitch = a.ph_P * a.sw * a.C;  // elements between consecutive windows
@@ -235,14 +237,9 @@ __global__ void __launch_bounds__(kPhThreads, 1)
           }
         }
       }
-      if (!pok && leader) {
-        // a pair's loads all complete on the leader's barriers: the leader
-        // waits for every fill issued (each stage armed fills/stages (+1) times)
-        for (int s = 0; s < a.stages; ++s) {
-          const long long arms = fills / a.stages + (s < fills % a.stages ? 1 : 0);
-          if (arms > 0) wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), a.timeout_ns);
-        }
-      }
+      // a pair's loads all complete on the leader's barriers: the two producers
+      // settle every fill either issued (each carries `bytes` per CTA)
+      pair_settle_ring(tail, a.stages, leader, fills, a.timeout_ns, [&](long long) { return bytes; });
     }
     __syncwarp();
   } else if (warp == 1) {

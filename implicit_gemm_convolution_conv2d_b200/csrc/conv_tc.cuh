@@ -158,10 +158,12 @@ struct __align__(8) TcSmemTail {
   uint64_t rempty[3]; // row staging: every gather thread is done with the buffer
   int seg_n[3][2];    // row staging, per buffer: image of segment 0 / 1
   int seg_lo[3][2];   // first staged input row of segment 0 / 1
-  uint64_t peer_done; // CTA pairs: the peer's producer finished issuing (leader's)
+  uint64_t peer_done;   // CTA pairs: the peer's producer finished issuing (leader's)
+  uint64_t peer_done_a; // the same for the input-strip ring of the halo kernels
   uint32_t tmem_base;
   volatile int abort_flag;
-  volatile int peer_fills;  // CTA pairs: ring fills the peer's producer issued (leader's)
+  volatile int peer_fills;    // CTA pairs: ring fills the peer's producer issued (leader's)
+  volatile int peer_fills_a;  // the same for the input-strip ring
 };
 
 __device__ __forceinline__ void raise_timeout(volatile int* abort_flag, unsigned site) {
@@ -229,15 +231,15 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, unsign
 // most one phase behind its last armed fill, so one parity wait per stage is
 // exact.  peer_bytes(k) gives the peer's bytes of fill k.
 template <typename PeerBytes>
-__device__ void pair_settle_ring(TcSmemTail* tail, int stages, bool leader, long long fills,
-                                 unsigned long long timeout_ns, PeerBytes peer_bytes) {
+__device__ void pair_settle_ring(uint64_t* ring, int nslots, uint64_t* peer_done, volatile int* peer_fills,
+                                 bool leader, long long fills, unsigned long long timeout_ns, PeerBytes peer_bytes) {
   if (!leader) {
-    ptx::st_shared_cluster_u32(ptx::mapa_shared(ptx::smem_u32(const_cast<int*>(&tail->peer_fills)), 0),
+    ptx::st_shared_cluster_u32(ptx::mapa_shared(ptx::smem_u32(const_cast<int*>(peer_fills)), 0),
                                static_cast<uint32_t>(fills));
-    ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(&tail->peer_done), 0));
+    ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(peer_done), 0));
     return;
   }
-  const uint32_t pd = ptx::smem_u32(&tail->peer_done);
+  const uint32_t pd = ptx::smem_u32(peer_done);
   const uint64_t t0 = ptx::globaltimer_ns();
   bool heard = true;
   while (!ptx::mbar_try_wait_cluster(pd, 0u)) {
@@ -247,16 +249,21 @@ __device__ void pair_settle_ring(TcSmemTail* tail, int stages, bool leader, long
       break;
     }
   }
-  const long long peer = heard ? static_cast<long long>(static_cast<uint32_t>(tail->peer_fills)) : fills;
-  for (long long k = fills; k < peer; ++k)
-    ptx::mbar_arrive_expect_tx(ptx::smem_u32(&tail->full[k % stages]), peer_bytes(k));
-  for (long long k = peer; k < fills; ++k)
-    ptx::mbar_complete_tx(ptx::smem_u32(&tail->full[k % stages]), peer_bytes(k));
+  const long long peer = heard ? static_cast<long long>(static_cast<uint32_t>(*peer_fills)) : fills;
+  for (long long k = fills; k < peer; ++k) ptx::mbar_arrive_expect_tx(ptx::smem_u32(&ring[k % nslots]), peer_bytes(k));
+  for (long long k = peer; k < fills; ++k) ptx::mbar_complete_tx(ptx::smem_u32(&ring[k % nslots]), peer_bytes(k));
   const long long total = fills > peer ? fills : peer;
-  for (int s = 0; s < stages; ++s) {
-    const long long arms = total / stages + (s < total % stages ? 1 : 0);
-    if (arms > 0) wait_drain(ptx::smem_u32(&tail->full[s]), static_cast<uint32_t>((arms - 1) & 1), timeout_ns);
+  for (int s = 0; s < nslots; ++s) {
+    const long long arms = total / nslots + (s < total % nslots ? 1 : 0);
+    if (arms > 0) wait_drain(ptx::smem_u32(&ring[s]), static_cast<uint32_t>((arms - 1) & 1), timeout_ns);
   }
+}
+
+// The weight / patch ring of a pair kernel (`full`, `stages` slots).
+template <typename PeerBytes>
+__device__ void pair_settle_ring(TcSmemTail* tail, int stages, bool leader, long long fills,
+                                 unsigned long long timeout_ns, PeerBytes peer_bytes) {
+  pair_settle_ring(tail->full, stages, &tail->peer_done, &tail->peer_fills, leader, fills, timeout_ns, peer_bytes);
 }
 
 struct TileCoord {
