@@ -1916,7 +1916,7 @@ int run(const Problem& P, const void* x, const void* w, void* y, int variant, cu
 
 namespace convfwd {
 
-constexpr int kWgtKbs = 2;        // 64-pixel sub-blocks per pipeline stage (8 pair MMAs, 1024 tensor cycles)
+constexpr int kWgtKbs = 1;        // 128-pixel sub-blocks per pipeline stage (8 pair MMAs, 1024 tensor cycles)
 constexpr int kWgtPairs = 74;     // CTA pairs of a 148-SM B200: the split target (fixed, so the
                                   // summation order never depends on the device)
 
@@ -1942,7 +1942,7 @@ bool wgrad_tc_fits(const WgArgs& a, int dtype) {
 
 // Ranges of the pixel reduction for the tensor-core path (a function of the
 // shape and `max_split` only): enough units for every CTA pair of a 148-SM
-// B200, each range at least 8 sub-blocks (512 pixels) long and a whole number
+// B200, each range at least 8 sub-blocks (1024 pixels) long and a whole number
 // of pipeline stages; no range is empty.
 void wgrad_tc_split(const WgArgs& a, long long max_split, int& nsplit, int& chunk_sub) {
   const long long per_split = static_cast<long long>(a.G) * (a.Og / 256) * ((a.ncols + 255) / 256);

@@ -4,14 +4,14 @@
 // im2col matrix of x (the weight gradient of the forward pass; see
 // conv_wgrad.cuh).  As a GEMM: M = output channels, N = weight columns
 // (tap, channel), K = output pixels.  Both operands arrive exactly as the
-// forward kernels load their tiles: dy rows by a 2-D TMA box of [64 pixels]
-// [64 output channels], x by a TMA im2col box of [64 pixels][64 channels]
+// forward kernels load their tiles: dy rows by a 2-D TMA box of [128 pixels]
+// [64 output channels], x by a TMA im2col box of [128 pixels][64 channels]
 // per tap, both in the 128-byte swizzle.  In the forward pass such a tile is
 // a K-major operand (K = channels); here the same bytes are MN-major operands
 // (K = pixels, the 64 channels of a row contiguous), which the instruction
 // descriptor's transpose bits select: one K step of 16 pixels is two 8-row
 // groups (SBO = 1024 bytes apart), the second 64-channel block of a 128-wide
-// operand half sits LBO = one box (8 KB) further.
+// operand half sits LBO = one box (16 KB) further.
 //
 // CTA pair (cta_group::2): M = 256 output channels (128 per CTA, their dy
 // boxes), N = 256 weight columns (each CTA loads the im2col boxes of its 128).
@@ -38,7 +38,7 @@ struct WgTcArgs {
   int ncols;             // taps * Cg (columns of one group's dw)
   int jtiles, otiles;    // 256-column tiles of ncols, 256-channel tiles of Og
   int nsplit;            // ranges of the pixel reduction
-  int chunk_sub;         // 64-pixel sub-blocks per range (a multiple of kbs)
+  int chunk_sub;         // kWgtBK-pixel sub-blocks per range (a multiple of kbs)
   int total_units;       // G * otiles * jtiles * nsplit
   int kbs, stages;       // sub-blocks per pipeline stage, stages
   uint32_t stage_bytes;  // kbs * kWgtSub
@@ -49,8 +49,8 @@ struct WgTcArgs {
   float* part;           // [nsplit][O][ncols] fp32 partial sums
 };
 
-constexpr int kWgtBK = 64;                    // pixels per sub-block (K)
-constexpr uint32_t kWgtBox = 8192;            // one [64 px][64 ch] box
+constexpr int kWgtBK = 128;                   // pixels per sub-block (K)
+constexpr uint32_t kWgtBox = kWgtBK * 128;    // one [128 px][64 ch] box, 128-byte rows
 constexpr uint32_t kWgtSub = 4 * kWgtBox;     // per CTA: two dy boxes (A) + two im2col boxes (B)
 constexpr int kWgtThreads = 192;
 constexpr uint32_t kWgtTmemCols = 512;        // two 256-column fp32 accumulators
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kWgtThreads, 1)
           if (leader) ptx::mbar_arrive_expect_tx(fb_local, 2u * static_cast<uint32_t>(a.kbs) * kWgtSub);
           const uint32_t fb = ptx::mapa_shared(fb_local, 0);
           for (int j = 0; j < a.kbs; ++j) {
-            // pixels p0 .. p0+63 of the range; past the last pixel every box reads zeros
+            // pixels p0 .. p0+kWgtBK-1 of the range; past the last pixel every box reads zeros
             const long long p0 = (sb0 + f + j) * kWgtBK;
             const long long n = p0 / spp;
             long long r = p0 - n * spp;
