@@ -1265,13 +1265,16 @@ int plan_tconv(const Problem& P, int sms, TconvArgs& a, int& ctas, size_t& smem)
   const long long tt = static_cast<long long>(a.nphase) * P.G * a.n_tiles * a.m_tiles;
   if (tt > 0x7fffffffLL) return CONV_EUNSUPPORTED;
   a.total_tiles = static_cast<int>(tt);
-  a.cchunks = P.Cg / 64;
-  a.a_bytes = static_cast<uint32_t>(kBM * 64 * 2);                 // 128 pixels x 64 channels
-  a.b_bytes = static_cast<uint32_t>((a.BN / 2 / 64) * 8192);       // this CTA's 64-channel weight boxes
+  // 128 input channels per sub-block where possible: 16 KB TMA boxes (half the
+  // operations per byte of 64-channel ones)
+  a.kc = P.Cg % 128 == 0 ? 128 : 64;
+  a.cchunks = P.Cg / a.kc;
+  a.a_bytes = static_cast<uint32_t>(kBM * a.kc * 2);                   // 128 pixels x kc channels
+  a.b_bytes = static_cast<uint32_t>((a.BN / 2 / 64) * a.kc * 128);     // this CTA's [kc][64] weight boxes
   a.sub_bytes = a.a_bytes + a.b_bytes;
   const long long avail = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(TcSmemTail)) - 64;
   int stages = 0;
-  a.kbs = choose_kbs(a.BN, 64, a.sub_bytes, avail, 8, stages);
+  a.kbs = choose_kbs(a.BN, a.kc, a.sub_bytes, avail, 8, stages);
   if (stages < 2) return CONV_EUNSUPPORTED;
   a.stages = stages;
   a.stage_bytes = static_cast<uint32_t>(a.kbs) * a.sub_bytes;
@@ -1334,7 +1337,7 @@ int launch_tconv(const Problem& P, const void* x, const void* w, void* y, cudaSt
   const cuuint64_t taps = static_cast<cuuint64_t>(P.kD) * P.kH * P.kW;
   cuuint64_t wdim[3] = {static_cast<cuuint64_t>(P.Og), taps, static_cast<cuuint64_t>(P.C)};
   cuuint64_t wstr[2] = {eb * P.Og, eb * P.Og * taps};
-  cuuint32_t wbox[3] = {64u, 1u, 64u};
+  cuuint32_t wbox[3] = {64u, 1u, static_cast<cuuint32_t>(a.kc)};
   cuuint32_t west[3] = {1, 1, 1};
   r = drv.tiled(&mw, dt, 3, const_cast<void*>(w), wdim, wstr, wbox, west, CU_TENSOR_MAP_INTERLEAVE_NONE,
                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

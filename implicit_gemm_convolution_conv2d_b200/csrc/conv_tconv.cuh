@@ -16,6 +16,8 @@
 // w [Cin][taps][Cout/G] holds, for one tap, a [ci][co] matrix whose rows are
 // 64-channel TMA boxes in the 128-byte swizzle, read as an MN-major operand
 // (N = co contiguous; one K step = 16 ci rows = 2 KB; LBO = the next 64-co box).
+// A sub-block carries 128 input channels where Cin/G allows (two im2col boxes,
+// one 16 KB weight box per 64 output channels), else 64.
 //
 // CTA pair (cta_group::2): M = 256 phase pixels (128 per CTA, its own im2col
 // box), N = BN output channels (each CTA loads the boxes of its BN/2).  A tile
@@ -51,7 +53,8 @@ struct TconvArgs {
   long long Mph;               // rows per phase: N * Tm[0] * Tm[1] * Tm[2]
   int nphase;                  // s[0] * s[1] * s[2]
   int m_tiles, n_tiles, BN, total_tiles;
-  int cchunks;                 // Cig / 64
+  int kc;                      // input channels per sub-block: 128 (when Cig allows) or 64
+  int cchunks;                 // Cig / kc
   int kbs, stages;
   uint32_t a_bytes, b_bytes, sub_bytes, stage_bytes;
   uint32_t idesc, tmem_cols;
@@ -193,15 +196,20 @@ __global__ void __launch_bounds__(kTcvThreads, 1)
             const int kh = a.ph_k[1][u.r[1]] + a.s[1] * jh;
             const int kw = a.ph_k[2][u.r[2]] + a.s[2] * jw;
             const int tap = (kd * a.kH + kh) * a.kW + kw;
-            const int ci0 = u.g * a.Cig + cc * 64;
-            if (a.rank5)
-              ptx::tma_load_im2col_5d_pair(sa, &tmap_x, fb, ci0, cw, chh, cd, n, static_cast<uint16_t>(ow),
-                                           static_cast<uint16_t>(oh), static_cast<uint16_t>(od));
-            else
-              ptx::tma_load_im2col_4d_pair(sa, &tmap_x, fb, ci0, cw, chh, n, static_cast<uint16_t>(ow),
-                                           static_cast<uint16_t>(oh));
+            const int ci0 = u.g * a.Cig + cc * a.kc;
+            // A: one [128 px][64 ch] im2col box per 64 channels of the sub-block
+            for (int h = 0; h < a.kc / 64; ++h) {
+              if (a.rank5)
+                ptx::tma_load_im2col_5d_pair(sa + h * 16384u, &tmap_x, fb, ci0 + h * 64, cw, chh, cd, n,
+                                             static_cast<uint16_t>(ow), static_cast<uint16_t>(oh),
+                                             static_cast<uint16_t>(od));
+              else
+                ptx::tma_load_im2col_4d_pair(sa + h * 16384u, &tmap_x, fb, ci0 + h * 64, cw, chh, n,
+                                             static_cast<uint16_t>(ow), static_cast<uint16_t>(oh));
+            }
+            // B: one [kc ci][64 co] box per 64 output channels of this CTA's half
             for (int b = 0; b < half_bn / 64; ++b)
-              ptx::tma_load_3d_pair(sb + b * 8192u, &tmap_w, fb, co0 + b * 64, tap, ci0);
+              ptx::tma_load_3d_pair(sb + b * static_cast<uint32_t>(a.kc) * 128u, &tmap_w, fb, co0 + b * 64, tap, ci0);
             if (++cc == a.cchunks) {
               cc = 0;
               if (++jw == u.J[2]) {
@@ -233,10 +241,12 @@ __global__ void __launch_bounds__(kTcvThreads, 1)
       int t = 0;
       if (a.inject_stall)
         ok = wait_bounded(ptx::smem_u32(&tail->stall), 0u, abort_flag, a.timeout_ns, kSiteInjected);
-      // A: K-major im2col rows (K step = 32 bytes); B: MN-major weight boxes
-      // (LBO = the next 64-channel box, SBO = 8 ci rows, K step = 16 rows = 2 KB)
+      // A: K-major im2col rows (K step = 32 bytes within a 64-channel box, the
+      // next box 16 KB on); B: MN-major weight boxes (LBO = the next 64-channel
+      // box, SBO = 8 ci rows, K step = 16 rows = 2 KB)
       const uint64_t d_a = ptx::smem_desc(ptx::smem_u32(smem), 16, 1024, 2u);
-      const uint64_t d_b = ptx::smem_desc(ptx::smem_u32(smem + a.a_bytes), 8192, 1024, 2u);
+      const uint64_t d_b = ptx::smem_desc(ptx::smem_u32(smem + a.a_bytes), static_cast<uint32_t>(a.kc) * 128u, 1024, 2u);
+      const int ksteps = a.kc >> 4;
       const uint64_t sub_off = desc_off(a.sub_bytes), st_off = desc_off(a.stage_bytes);
       for (int tile = pair; ok && tile < a.total_tiles; tile += npairs, ++t) {
         const int acc = t & 1;
@@ -260,9 +270,17 @@ __global__ void __launch_bounds__(kTcvThreads, 1)
           for (int j = 0; j < nsub; ++j) {
             const uint64_t da = d_a + so + static_cast<uint64_t>(j) * sub_off;
             const uint64_t db = d_b + so + static_cast<uint64_t>(j) * sub_off;
+            // (unrolled: descriptor offsets are constants)
+            if (ksteps == 8) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              ptx::mma_f16_pair(d_tmem, da + 2 * k, db + 128 * k, a.idesc, (kb + j + k) != 0 ? 1u : 0u);
+              for (int k = 0; k < 8; ++k)
+                ptx::mma_f16_pair(d_tmem, da + (k >> 2) * 1024 + 2 * (k & 3), db + 128 * k, a.idesc,
+                                  (kb + j + k) != 0 ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                ptx::mma_f16_pair(d_tmem, da + 2 * k, db + 128 * k, a.idesc, (kb + j + k) != 0 ? 1u : 0u);
+            }
           }
           ptx::mma_commit_pair(ptx::smem_u32(&tail->empty[stage]), 3);
           if (++stage == a.stages) {
