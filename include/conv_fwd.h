@@ -126,8 +126,8 @@ int conv_out_dims(int D, int H, int W, int kD, int kH, int kW,
  * f32 -> SIMT; f16/bf16 with C/G % 16 == 0 and a geometry that fits a TMA
  * im2col tensor map -> when O/G is a multiple of 64 but not of 256: TC_HALO_T
  * at stride 1 with C/G % 32 == 0, kH >= 2 and at least as many output blocks
- * as SMs, else (O/G % 128 == 0) TC_TMA_T when there are at least as many
- * 256-pixel tiles as SMs;
+ * as SMs, else (O/G % 128 == 0) TC_TMA for reductions of K <= 256 elements,
+ * else TC_TMA_T when there are at least as many 256-pixel tiles as SMs;
  * otherwise TC_TMA_PAIR (or TC_TMA when there are fewer 256-row output tiles
  * than SM pairs); otherwise TC_PHASE where its conditions hold, else
  * TC_GATHER.  Depthwise problems (groups = C = O, C*elem % 16 == 0), of any
