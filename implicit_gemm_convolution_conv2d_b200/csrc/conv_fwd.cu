@@ -2104,6 +2104,7 @@ int conv_fwd_ex(const void* x, const void* w, void* y, int N, int D, int H, int 
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
   if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_PHASES) return CONV_EINVAL;
+  if (variant == CONV_VARIANT_TC_TMA_PHASES) return CONV_EUNSUPPORTED;  // transposed convolutions only
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 

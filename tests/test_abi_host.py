@@ -95,7 +95,8 @@ def test_flip_and_side_padding_arguments(C):
     assert ex(i3(0, -1, 0), 0) == -1           # negative high-side pad
     assert ex(i3(0, 1, 1), 2) == -1            # flip is 0 or 1
     assert ex(i3(0, 1, 1), 0, 9) == -2         # dtype
-    assert ex(i3(0, 1, 1), 0, 1, 12) == -1     # unknown variant
+    assert ex(i3(0, 1, 1), 0, 1, 13) == -1     # unknown variant
+    assert ex(i3(0, 1, 1), 0, 1, 12) == -7     # the transposed-convolution phase kernel: not a forward variant
     # flip keeps the phase-packed kernel (its B rows are built from the mirrored filter)
     stem = (2, 1, 32, 32, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
     assert C.plan(*stem)[0] == C.VARIANT_TC_PHASE
@@ -138,7 +139,7 @@ def test_invalid_arguments_rejected_on_host(C):
     big = 1 << 30
     assert call(X, Wt, Y, big, big, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
     # unknown variant
-    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 12, None) == -1
+    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 13, None) == -1
     assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, -2, None) == -1
 
 
@@ -167,8 +168,11 @@ def test_variant_plan(C):
     assert plan(4, 32, 32, 32, 64, 128, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "f16")[2] == 1
     assert plan(2, 1, 9, 9, 128, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 2, "f16",
                 C.VARIANT_TC_HALO_T)[2] >= 2
-    # ... with kH = 1 (no strip reuse): the transposed im2col kernel
+    # ... with kH = 1 (no strip reuse) and a short reduction (K = 192): the plain
+    # single-CTA im2col kernel; with a longer one (K = 5 x 128): the transposed im2col kernel
     v, bn, _, _ = plan(4, 32, 32, 32, 64, 128, (3, 1, 1), (1, 1, 1), (1, 0, 0), (1, 1, 1), 1, "f16")
+    assert v == C.VARIANT_TC_TMA and bn == 128
+    v, bn, _, _ = plan(4, 32, 32, 32, 128, 128, (5, 1, 1), (1, 1, 1), (2, 0, 0), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_TMA_T and bn == 256
     # block height adapts to Ho: 56 rows -> blocks of 28 (MMA N = 224)
     v, bn, _, _ = plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16",
@@ -189,7 +193,9 @@ def test_variant_plan(C):
     assert v == C.VARIANT_TC_GATHER
     # channel chunks of 32 and 16
     assert plan(2, 64, 64, 64, 32, 256, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA_PAIR
-    assert plan(2, 64, 64, 64, 32, 384, (1, 1, 1), (1, 1, 1), (0, 0, 0), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA_T
+    assert plan(2, 64, 64, 64, 32, 384, (1, 1, 1), (1, 1, 1), (0, 0, 0), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA
+    assert plan(2, 64, 64, 64, 128, 384, (3, 1, 1), (1, 1, 1), (1, 0, 0), (1, 1, 1), 1, "f16")[0] == \
+        C.VARIANT_TC_TMA_T
     assert plan(1, 1, 9, 9, 48, 96, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 3, "f16")[0] == C.VARIANT_TC_TMA
     assert plan(1, 1, 9, 9, 128, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 2, "f16")[0] == C.VARIANT_TC_TMA
 
@@ -244,21 +250,36 @@ def test_explicit_variant_plan(C):
     tall = (1, 1, 200, 32, 16, 16, (1, 5, 3), (1, 1, 1), (0, 140, 1), (1, 70, 1), 16)
     assert C.plan(*tall, "f16")[:3] == (C.VARIANT_DEPTHWISE, 8, 1)  # the direct form's 8 channels
     with pytest.raises(C.ConvError) as e:
-        C.plan(*g3, "bf16", 12)
+        C.plan(*g3, "bf16", 13)
     assert e.value.code == -1
+    with pytest.raises(C.ConvError) as e:   # the transposed-convolution phase kernel
+        C.plan(*g3, "bf16", C.VARIANT_TC_TMA_PHASES)
+    assert e.value.code == -7
 
 
 def test_transpose_extents_and_plans(C):
     """Transposed-convolution extents agree with the oracle's; the planner runs
-    it on the gather kernel (16-bit) or the FP32 kernel and refuses the rest."""
+    it on the TMA-fed phase kernel where that fits (16-bit, dilation 1,
+    64-/128-channel multiples), else the gather kernel (16-bit) or the FP32
+    kernel, and refuses the forward-only variants."""
     import oracle
     for D, H, W, k, s, p, op, d in ((3, 4, 5, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 1, 1)),
                                     (5, 6, 7, (3, 3, 3), (2, 1, 2), (1, 1, 0), (1, 0, 1), (1, 2, 1)),
                                     (1, 28, 28, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1))):
         assert C.transpose_out_dims(D, H, W, *k, s, p, op, d) == oracle.convT_out_dims(D, H, W, *k, s, p, op, d)
     g = (2, 1, 28, 28, 256, 128, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1)
-    assert C.transpose_plan(*g, "f16")[0] == C.VARIANT_TC_GATHER
+    assert C.transpose_plan(*g, "f16")[0] == C.VARIANT_TC_TMA_PHASES
+    assert C.transpose_plan(*g, "f16", C.VARIANT_TC_GATHER)[0] == C.VARIANT_TC_GATHER
     assert C.transpose_plan(*g, "f32")[0] == C.VARIANT_SIMT
+    # dilation 2, or 32 input channels, or 64 output channels: the gather kernel
+    g_dil = (2, 1, 28, 28, 256, 128, (1, 3, 3), (1, 2, 2), (0, 1, 1), (0, 1, 1), (1, 2, 2), 1)
+    g_c32 = (2, 1, 28, 28, 32, 128, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1)
+    g_o64 = (2, 1, 28, 28, 256, 64, (1, 4, 4), (1, 2, 2), (0, 1, 1), (0, 0, 0), (1, 1, 1), 1)
+    for gg in (g_dil, g_c32, g_o64):
+        assert C.transpose_plan(*gg, "f16")[0] == C.VARIANT_TC_GATHER
+        with pytest.raises(C.ConvError) as e:
+            C.transpose_plan(*gg, "f16", C.VARIANT_TC_TMA_PHASES)
+        assert e.value.code == -7
     for v in (C.VARIANT_TC_TMA, C.VARIANT_TC_TMA_PAIR, C.VARIANT_TC_HALO_T, C.VARIANT_TC_PHASE, C.VARIANT_DEPTHWISE):
         with pytest.raises(C.ConvError) as e:
             C.transpose_plan(*g, "f16", v)
@@ -326,6 +347,8 @@ def test_planner_on_random_geometries(C):
         op = tuple(rng.randint(0, max(s[i], d[i]) - 1) for i in range(3))
         try:
             v, bn, st, ct = C.transpose_plan(rng.randint(1, 4), D, H, W, Cc, O, k, s, p, op, d, G, dt)
-            assert v in (C.VARIANT_TC_GATHER, C.VARIANT_SIMT) and ct >= 1, (v, ct)
+            assert v in (C.VARIANT_TC_GATHER, C.VARIANT_SIMT, C.VARIANT_TC_TMA_PHASES) and ct >= 1, (v, ct)
+            if v == C.VARIANT_TC_TMA_PHASES:   # its conditions, as the header states them
+                assert dt != "f32" and d == (1, 1, 1) and (Cc // G) % 64 == 0 and (O // G) % 128 == 0
         except C.ConvError as e:
             assert e.code in valid_codes, e.code
