@@ -171,6 +171,18 @@ int wg_launch(const WgProblem& q, const void* x, const void* dy, void* dw, void*
     if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
   }
   const long long n = q.dw_elems;
+  if (n % 4 == 0) {
+    // four elements a thread (dw is 16-byte aligned, so every slice is when n % 4 == 0)
+    const unsigned blocks4 = static_cast<unsigned>((n / 4 + 255) / 256);
+    if (dtype == CONV_F32)
+      conv_wgrad_reduce4_kernel<float><<<blocks4, 256, 0, st>>>(a.part, static_cast<float*>(dw), n, a.nsplit);
+    else if (dtype == CONV_F16)
+      conv_wgrad_reduce4_kernel<__half><<<blocks4, 256, 0, st>>>(a.part, static_cast<__half*>(dw), n, a.nsplit);
+    else
+      conv_wgrad_reduce4_kernel<__nv_bfloat16><<<blocks4, 256, 0, st>>>(a.part, static_cast<__nv_bfloat16*>(dw), n,
+                                                                       a.nsplit);
+    return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+  }
   const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
   if (dtype == CONV_F32)
     conv_wgrad_reduce_kernel<float><<<blocks, 256, 0, st>>>(a.part, static_cast<float*>(dw), n, a.nsplit);

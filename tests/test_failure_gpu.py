@@ -100,3 +100,25 @@ def test_injected_stall_in_the_tensor_core_weight_gradient():
     assert C.last_status() == 0
     g_ref, s_ref = oracle.conv_wgrad(x, dy, (1, 3, 3), (1, 1, 1), (0, 1, 1))
     assert_parity(g.cpu(), g_ref, s_ref, "bf16", "wgrad after stall")
+
+
+def test_host_buffer_path_reports_a_timeout():
+    """conv_fwd_host waits for its result and then reads the status word: a
+    kernel that gave up on a pipeline wait (the injected stall) makes the call
+    fail with CONV_ETIMEOUT instead of returning a partial y; the word is then
+    clear and the next call is exact."""
+    wl = WL.case(2, 1, 20, 20, 64, 64, (1, 3, 3), pad=(0, 1, 1), dtype="f16", seed=24)
+    x, w = WL.make_inputs(wl)
+    xh, wh = x[:, 0].contiguous().pin_memory(), w[:, 0].contiguous().pin_memory()
+    yh = torch.zeros((2, 20, 20, 64), dtype=torch.float16).pin_memory()
+    xd, wd = torch.empty_like(xh, device="cuda"), torch.empty_like(wh, device="cuda")
+    yd = torch.empty(yh.shape, dtype=torch.float16, device="cuda")
+    assert C.last_status() == 0
+    C.inject_stall(50_000_000)
+    with pytest.raises(C.ConvError) as e:
+        C.conv_fwd_host(xh, wh, yh, xd, wd, yd, stride=1, padding=1)
+    assert e.value.code == ETIMEOUT
+    assert C.last_status() == 0
+    C.conv_fwd_host(xh, wh, yh, xd, wd, yd, stride=1, padding=1)
+    y_ref, s_ref = oracle.conv_fwd(x, w, wl.stride, wl.pad, wl.dil, wl.groups)
+    assert_parity(yh.unsqueeze(1), y_ref, s_ref, "f16", "host path after a timeout")
