@@ -326,7 +326,7 @@ def bench_ours(args):
     flops = conv_flops(wl, dims)
     xb, wb, yb = conv_bytes(wl, dims)
     if wl.wgrad:
-        # the weight gradient: inputs x and dy, output dw; the FP32 split-K kernel
+        # the weight gradient: inputs x and dy, output dw; the path (tensor cores or FP32) from its planner
         e = WL.ELEM_BYTES[wl.dtype]
         wb = e * wl.N * dims[0] * dims[1] * dims[2] * wl.O        # dy
         yb = e * wl.O * wl.k[0] * wl.k[1] * wl.k[2] * (wl.C // wl.groups)  # dw

@@ -1,7 +1,8 @@
 // conv_wgrad.cu -- C ABI of the weight gradient (see conv_wgrad.cuh).
 //
 // A separate translation unit of libconvfwd.so: validation, the split of the
-// pixel reduction across blocks, and the launches (the split-K kernel, which
+// pixel reduction across blocks, and the launches (the tensor-core kernel in
+// conv_wgrad_tc.cuh or the FP32 split-K kernel, either of which
 // writes one fp32 partial slice per split into a caller-provided workspace,
 // then the kernel that adds the slices in split order and rounds).  The split
 // count depends on the problem's shape only, so a result is the same bits on
@@ -132,7 +133,7 @@ bool wg_overlaps(const void* a, size_t an, const void* b, size_t bn) {
   return a0 < b0 + bn && b0 < a0 + an;
 }
 
-// Validates the buffers and queues the split-K kernel and the reduction,
+// Validates the buffers and queues the partial-sum kernel (tensor cores or FP32) and the ordered sum,
 // with at most `max_split` splits.
 int wg_launch(const WgProblem& q, const void* x, const void* dy, void* dw, void* workspace,
               unsigned long long workspace_bytes, long long max_split, cudaStream_t st) {
