@@ -1914,6 +1914,49 @@ int run(const Problem& P, const void* x, const void* w, void* y, int variant, cu
   return launch_tc(P, plan, x, w, y, st, dev);
 }
 
+// Queues conv_fwd_host's copies and kernels: the upload of chunk i on the
+// upload stream, its kernel on the caller's stream, its download on the
+// download stream, ordered by events; the caller's stream finally waits for
+// the last download.  Returns at the first failure (work already queued stays
+// queued; the caller drains the streams).
+int host_pipeline(const Problem& P, HostPipe& hp, int variant, int nch, const void* x_host, const void* w_host,
+                  void* y_host, void* x_dev, const void* w_dev, void* y_dev, cudaStream_t st) {
+  const size_t x_img = P.x_bytes / P.N, y_img = P.y_bytes / P.N;
+  const char* xh = static_cast<const char*>(x_host);
+  char* yh = static_cast<char*>(y_host);
+  char* xd = static_cast<char*>(x_dev);
+  char* yd = static_cast<char*>(y_dev);
+  const int stride[3] = {P.s[0], P.s[1], P.s[2]}, pad[3] = {P.p[0], P.p[1], P.p[2]}, dil[3] = {P.d[0], P.d[1], P.d[2]};
+  // the copy streams start after the work already queued on the caller's stream
+  if (cudaEventRecord(hp.start, st) != cudaSuccess || cudaStreamWaitEvent(hp.h2d, hp.start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp.d2h, hp.start, 0) != cudaSuccess)
+    return CONV_ELAUNCH;
+  if (cudaMemcpyAsync(const_cast<void*>(w_dev), w_host, P.w_bytes, cudaMemcpyHostToDevice, hp.h2d) != cudaSuccess)
+    return CONV_ELAUNCH;
+  int n0 = 0;
+  for (int i = 0; i < nch; ++i) {
+    const int nc = (P.N - n0) / (nch - i);
+    Problem Pc;
+    int rc = make_problem(Pc, nc, P.D, P.H, P.W, P.C, P.O, P.kD, P.kH, P.kW, stride, pad, pad, dil, P.G, 0, P.dtype);
+    if (rc != CONV_OK) return rc;
+    // input chunk i on the upload stream (after w), then the kernel on the
+    // caller's stream, then the result chunk on the download stream
+    if (cudaMemcpyAsync(xd + n0 * x_img, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, hp.h2d) != cudaSuccess ||
+        cudaEventRecord(hp.loaded[i], hp.h2d) != cudaSuccess || cudaStreamWaitEvent(st, hp.loaded[i], 0) != cudaSuccess)
+      return CONV_ELAUNCH;
+    rc = run(Pc, xd + n0 * x_img, w_dev, yd + n0 * y_img, variant, st);
+    if (rc == CONV_EUNSUPPORTED) rc = run(Pc, xd + n0 * x_img, w_dev, yd + n0 * y_img, CONV_VARIANT_AUTO, st);
+    if (rc != CONV_OK) return rc;
+    if (cudaEventRecord(hp.computed[i], st) != cudaSuccess || cudaStreamWaitEvent(hp.d2h, hp.computed[i], 0) != cudaSuccess ||
+        cudaMemcpyAsync(yh + n0 * y_img, yd + n0 * y_img, nc * y_img, cudaMemcpyDeviceToHost, hp.d2h) != cudaSuccess)
+      return CONV_ELAUNCH;
+    n0 += nc;
+  }
+  if (cudaEventRecord(hp.finished, hp.d2h) != cudaSuccess || cudaStreamWaitEvent(st, hp.finished, 0) != cudaSuccess)
+    return CONV_ELAUNCH;
+  return CONV_OK;
+}
+
 }  // namespace
 }  // namespace convfwd
 
@@ -2147,37 +2190,15 @@ int conv_fwd_host(const void* x_host, const void* w_host, void* y_host, void* x_
   std::lock_guard<std::mutex> lk(hp.mu);
   rc = host_pipe_init(hp);
   if (rc != CONV_OK) return rc;
-  const size_t x_img = P.x_bytes / P.N, y_img = P.y_bytes / P.N;
-  const char* xh = static_cast<const char*>(x_host);
-  char* yh = static_cast<char*>(y_host);
-  char* xd = static_cast<char*>(x_dev);
-  char* yd = static_cast<char*>(y_dev);
-  // the copy streams start after the work already queued on the caller's stream
-  if (cudaEventRecord(hp.start, st) != cudaSuccess || cudaStreamWaitEvent(hp.h2d, hp.start, 0) != cudaSuccess ||
-      cudaStreamWaitEvent(hp.d2h, hp.start, 0) != cudaSuccess)
-    return CONV_ELAUNCH;
-  if (cudaMemcpyAsync(w_dev, w_host, P.w_bytes, cudaMemcpyHostToDevice, hp.h2d) != cudaSuccess) return CONV_ELAUNCH;
-  int n0 = 0;
-  for (int i = 0; i < nch; ++i) {
-    const int nc = (P.N - n0) / (nch - i);
-    Problem Pc;
-    rc = make_problem(Pc, nc, D, H, W, C, O, kD, kH, kW, stride, pad, pad, dil, groups, 0, dtype);
-    if (rc != CONV_OK) return rc;
-    // input chunk i on the upload stream (after w), then the kernel on the
-    // caller's stream, then the result chunk on the download stream
-    if (cudaMemcpyAsync(xd + n0 * x_img, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, hp.h2d) != cudaSuccess ||
-        cudaEventRecord(hp.loaded[i], hp.h2d) != cudaSuccess || cudaStreamWaitEvent(st, hp.loaded[i], 0) != cudaSuccess)
-      return CONV_ELAUNCH;
-    rc = run(Pc, xd + n0 * x_img, w_dev, yd + n0 * y_img, variant, st);
-    if (rc == CONV_EUNSUPPORTED) rc = run(Pc, xd + n0 * x_img, w_dev, yd + n0 * y_img, CONV_VARIANT_AUTO, st);
-    if (rc != CONV_OK) return rc;
-    if (cudaEventRecord(hp.computed[i], st) != cudaSuccess || cudaStreamWaitEvent(hp.d2h, hp.computed[i], 0) != cudaSuccess ||
-        cudaMemcpyAsync(yh + n0 * y_img, yd + n0 * y_img, nc * y_img, cudaMemcpyDeviceToHost, hp.d2h) != cudaSuccess)
-      return CONV_ELAUNCH;
-    n0 += nc;
+  rc = host_pipeline(P, hp, variant, nch, x_host, w_host, y_host, x_dev, w_dev, y_dev, st);
+  if (rc != CONV_OK) {
+    // nothing queued by this call may still run once it returns: the caller
+    // may free its buffers
+    cudaStreamSynchronize(hp.h2d);
+    cudaStreamSynchronize(hp.d2h);
+    cudaStreamSynchronize(st);
+    return rc;
   }
-  if (cudaEventRecord(hp.finished, hp.d2h) != cudaSuccess || cudaStreamWaitEvent(st, hp.finished, 0) != cudaSuccess)
-    return CONV_ELAUNCH;
   if (cudaStreamSynchronize(st) != cudaSuccess) return CONV_ELAUNCH;
   // a kernel that gave up on a pipeline wait left y partial: report it (and clear the word)
   return read_and_clear_status();
