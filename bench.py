@@ -96,7 +96,7 @@ def measured_peaks():
 
 # Device and host source files each kernel variant's behaviour depends on: a
 # traffic record taken with ncu stays valid while these files are unchanged.
-_COMMON_SRC = ["conv_fwd.cu", "ptx.cuh", "conv_tc.cuh"]
+_COMMON_SRC = ["conv_fwd.cu", "ptx.cuh", "conv_tc.cuh", "launch.cuh"]
 KERNEL_SOURCES = {
     "tcgen05_tma_im2col": _COMMON_SRC,
     "tcgen05_tma_im2col_pair": _COMMON_SRC,
@@ -107,13 +107,13 @@ KERNEL_SOURCES = {
     "tcgen05_tma_halo_t": _COMMON_SRC + ["conv_halo.cuh", "conv_tct.cuh", "conv_halo_t.cuh"],
     "tcgen05_tma_halo_t_pair": _COMMON_SRC + ["conv_halo.cuh", "conv_tct.cuh", "conv_halo_t.cuh"],
     "tcgen05_tma_phase": _COMMON_SRC + ["conv_phase.cuh"],
-    "simt_ffma": ["conv_fwd.cu", "conv_simt.cuh"],
+    "simt_ffma": ["conv_fwd.cu", "conv_simt.cuh", "ptx.cuh", "launch.cuh"],
     "depthwise_tma": _COMMON_SRC + ["conv_simt.cuh", "conv_dw.cuh"],
-    "depthwise_direct": ["conv_fwd.cu", "conv_simt.cuh", "conv_dw.cuh"],
-    "simt_wgrad": ["conv_wgrad.cu", "conv_wgrad.cuh", "conv_simt.cuh"],
+    "depthwise_direct": ["conv_fwd.cu", "conv_simt.cuh", "conv_dw.cuh", "ptx.cuh", "launch.cuh"],
+    "simt_wgrad": ["conv_wgrad.cu", "conv_wgrad.cuh", "conv_simt.cuh", "ptx.cuh", "launch.cuh"],
     "tcgen05_tma_phases_pair": _COMMON_SRC + ["conv_tconv.cuh"],
     "tcgen05_wgrad_pair": ["conv_fwd.cu", "conv_wgrad.cu", "conv_wgrad.cuh", "conv_wgrad_tc.cuh", "conv_tc.cuh",
-                           "ptx.cuh"],
+                           "ptx.cuh", "launch.cuh"],
 }
 
 

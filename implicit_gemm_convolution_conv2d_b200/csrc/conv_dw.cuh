@@ -136,6 +136,9 @@ __global__ void __launch_bounds__(kDwThreads, 2) conv_fwd_dw_direct_kernel(const
   const int taps = a.kD * a.kH * a.kW;
   const int cbv = a.cb * V;
   const int cbase = blockIdx.y * cbv;  // first channel of the block
+  // (no early trigger: several blocks of this kernel share an SM; the next
+  // launch starts as they exit)
+  ptx::pdl_wait_prev();  // the previous launch's writes are visible from here on
 
   // Filters of the block's channels, tap-major, mirrored under flip.  Read in
   // w's own order (channel-major) so the global reads are contiguous.
@@ -433,6 +436,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), dw_tma_ctas_per_sm(MODE, R, NC
     ptx::fence_mbar_init();
   }
   if (warp == NCW && lane == 0) ptx::prefetch_tmap(&tmap_x);
+  ptx::pdl_allow_next();  // setup done: the next launch may start its own
+  ptx::pdl_wait_prev();   // the previous launch's writes are visible from here on
   const int ct = static_cast<int>(blockIdx.x) % a.nct;
   const int t_first = static_cast<int>(blockIdx.x) / a.nct, t_step = static_cast<int>(gridDim.x) / a.nct;
   dw_fill_filters<T, 4>(s_w, g, ct, taps, static_cast<int>(threadIdx.x), 32 * (NCW + 1));

@@ -20,6 +20,7 @@
 #include "conv_phase.cuh"
 #include "conv_dw.cuh"
 #include "conv_wgrad.cuh"
+#include "launch.cuh"
 #include "conv_wgrad_tc.cuh"
 #include "conv_tconv.cuh"
 
@@ -1122,8 +1123,7 @@ cudaError_t launch_dw_t(const DwArgs& a, dim3 grid, dim3 block, size_t smem, cud
     const cudaError_t e = dw_smem_attr(k, attr_done);
     if (e != cudaSuccess) return e;
   }
-  k<<<grid, block, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, block, smem, st, 1, a);
 }
 
 template <typename T, int MODE, int K, int S, int R, int NCW>
@@ -1132,8 +1132,7 @@ cudaError_t launch_dw_tma_t(const CUtensorMap& m, const DwTmaArgs& t, int grid, 
   auto* k = conv_fwd_dw_tma_kernel<T, MODE, K, S, R, NCW>;
   const cudaError_t e = dw_smem_attr(k, attr_done);
   if (e != cudaSuccess) return e;
-  k<<<grid, 32 * (NCW + 1), smem, st>>>(m, t);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(grid), dim3(32 * (NCW + 1)), smem, st, 1, m, t);
 }
 
 // The filter-row forms compiled with their width, stride and dilation fixed
@@ -1345,7 +1344,7 @@ int launch_tconv(const Problem& P, const void* x, const void* w, void* y, cudaSt
   small_tensor_fixup(mw, P.w_bytes, drv.driver_version);
 
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
@@ -1360,6 +1359,7 @@ int launch_tconv(const Problem& P, const void* x, const void* w, void* y, cudaSt
   if (cudaOccupancyMaxActiveClusters(&clusters, conv_tconv_pair_kernel<false>, &cfg) != cudaSuccess || clusters <= 0)
     return CONV_ELAUNCH;
   cfg.gridDim = dim3(2 * std::min(ctas / 2, clusters));
+  add_pdl(cfg, attr);
   const cudaError_t e = P.dtype == CONV_BF16 ? cudaLaunchKernelEx(&cfg, conv_tconv_pair_kernel<true>, mx, mw, a)
                                              : cudaLaunchKernelEx(&cfg, conv_tconv_pair_kernel<false>, mx, mw, a);
   return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
@@ -1440,8 +1440,8 @@ int encode_y_rows_map(const Problem& P, void* y, CUtensorMap& my) {
 }
 
 // y viewed as [N, (Do,) Ho, Wo, O] for the transposed halo kernel's TMA
-// stores: boxes of mo (64 or 128) channels x 8 columns x 4 rows, clipped at
-// the edges.
+// stores: boxes of mo/4 channels (one epilogue warp's quarter of the tile's
+// 64 or 128) x 8 columns x 4 rows, clipped at the edges.
 int encode_y_block_map(const Problem& P, bool rank5, int mo, void* y, CUtensorMap& my) {
   std::memset(&my, 0, sizeof(my));
   const DriverFns& drv = driver_fns();
@@ -1452,7 +1452,7 @@ int encode_y_block_map(const Problem& P, bool rank5, int mo, void* y, CUtensorMa
   cuuint64_t dim[5] = {static_cast<cuuint64_t>(P.O), static_cast<cuuint64_t>(P.Wo), static_cast<cuuint64_t>(P.Ho),
                        static_cast<cuuint64_t>(rank5 ? P.Do : P.N), static_cast<cuuint64_t>(P.N)};
   cuuint64_t str[4] = {eb * P.O, eb * P.O * P.Wo, eb * P.O * P.Wo * P.Ho, eb * P.O * P.Wo * P.Ho * P.Do};
-  cuuint32_t box[5] = {static_cast<cuuint32_t>(mo), static_cast<cuuint32_t>(kHTBlockW),
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(mo / 4), static_cast<cuuint32_t>(kHTBlockW),
                        static_cast<cuuint32_t>(kTEpiRows / kHTBlockW), 1u, 1u};
   cuuint32_t est[5] = {1, 1, 1, 1, 1};
   const CUresult r = drv.tiled(&my, dt, rank5 ? 5 : 4, y, dim, str, box, est, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1619,7 +1619,7 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
     rc = encode_phase_maps(P, a, x, y, mx, me, my);
     if (rc != CONV_OK) return rc;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
@@ -1636,6 +1636,7 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
         clusters <= 0)
       return CONV_ELAUNCH;
     cfg.gridDim = dim3(2 * std::min(plan.ctas / 2, clusters));
+    add_pdl(cfg, attr);
     const cudaError_t e = P.dtype == CONV_BF16 ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_phase_kernel<true>, mx, me, my, a)
                                                : cudaLaunchKernelEx(&cfg, conv_fwd_tc_phase_kernel<false>, mx, me, my, a);
     return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
@@ -1647,12 +1648,12 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
     if (rc != CONV_OK) return rc;
     const bool bf = P.dtype == CONV_BF16;
     if (!plan.pair) {
-      if (bf) conv_fwd_tc_halo_t_kernel<true, false><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
-      else    conv_fwd_tc_halo_t_kernel<false, false><<<plan.ctas, kTThreads, plan.smem, st>>>(mx, mw, my, a);
-      return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+      const cudaError_t e1 = launch_pdl(bf ? conv_fwd_tc_halo_t_kernel<true, false> : conv_fwd_tc_halo_t_kernel<false, false>,
+                                        dim3(plan.ctas), dim3(kTThreads), plan.smem, st, 1, mx, mw, my, a);
+      return e1 == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
     }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
@@ -1669,6 +1670,7 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
         clusters <= 0)
       return CONV_ELAUNCH;
     cfg.gridDim = dim3(2 * std::min(plan.ctas / 2, clusters));
+    add_pdl(cfg, attr);
     const cudaError_t e = bf ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_halo_t_kernel<true, true>, mx, mw, my, a)
                              : cudaLaunchKernelEx(&cfg, conv_fwd_tc_halo_t_kernel<false, true>, mx, mw, my, a);
     return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
@@ -1678,9 +1680,9 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
     rc = encode_maps(P, a, false, false, x, w, mx, mw, kTO);
     if (rc == CONV_OK) rc = encode_y_map(P, y, my);
     if (rc != CONV_OK) return rc;
-    if (P.dtype == CONV_BF16) conv_fwd_tc_t_kernel<true><<<plan.ctas, kTTileThreads, plan.smem, st>>>(mx, mw, my, a);
-    else                      conv_fwd_tc_t_kernel<false><<<plan.ctas, kTTileThreads, plan.smem, st>>>(mx, mw, my, a);
-    return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+    const cudaError_t e = launch_pdl(P.dtype == CONV_BF16 ? conv_fwd_tc_t_kernel<true> : conv_fwd_tc_t_kernel<false>,
+                                     dim3(plan.ctas), dim3(kTTileThreads), plan.smem, st, 1, mx, mw, my, a);
+    return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
   }
   rc = encode_maps(P, a, plan.pair, halo, x, w, mx, mw);
   if (rc != CONV_OK) return rc;
@@ -1694,13 +1696,13 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
                                                                          : tc_threads<MODE_GATHER>());
   const bool bf = P.dtype == CONV_BF16;
   if (halo && !plan.pair) {
-    if (bf) conv_fwd_tc_halo_kernel<true, false><<<grid, 192, plan.smem, st>>>(mx, mw, a);
-    else    conv_fwd_tc_halo_kernel<false, false><<<grid, 192, plan.smem, st>>>(mx, mw, a);
-    return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+    const cudaError_t e = launch_pdl(bf ? conv_fwd_tc_halo_kernel<true, false> : conv_fwd_tc_halo_kernel<false, false>,
+                                     grid, dim3(192), plan.smem, st, 1, mx, mw, a);
+    return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
   }
   if (plan.pair) {
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
@@ -1733,6 +1735,7 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
       clusters = g_dev[dev].pair_clusters[slot];
     }
     cfg.gridDim = dim3(2 * std::min(plan.ctas / 2, clusters));
+    add_pdl(cfg, attr);
     cudaError_t e;
     if (halo)
       e = bf ? cudaLaunchKernelEx(&cfg, conv_fwd_tc_halo_kernel<true, true>, mx, mw, a)
@@ -1742,22 +1745,18 @@ int launch_tc(const Problem& P, const TcPlan& plan, const void* x, const void* w
              : cudaLaunchKernelEx(&cfg, conv_fwd_tc_pair_kernel<false>, mx, mw, my, a);
     return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
   }
-  if (plan.variant == CONV_VARIANT_TC_TMA) {
-    if (bf) conv_fwd_tc_kernel<MODE_TMA, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
-    else    conv_fwd_tc_kernel<MODE_TMA, false><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
-  } else {
-    if (a.tp_on) {
-      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true, true, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
-      else    conv_fwd_tc_kernel<MODE_GATHER, false, true, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
-    } else if (a.idil_on || a.wtrans) {
-      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
-      else    conv_fwd_tc_kernel<MODE_GATHER, false, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
-    } else {
-      if (bf) conv_fwd_tc_kernel<MODE_GATHER, true><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
-      else    conv_fwd_tc_kernel<MODE_GATHER, false><<<grid, block, plan.smem, st>>>(mx, mw, my, a);
-    }
+  // every instantiation below has the same signature
+  auto* k = bf ? conv_fwd_tc_kernel<MODE_TMA, true> : conv_fwd_tc_kernel<MODE_TMA, false>;
+  if (plan.variant != CONV_VARIANT_TC_TMA) {
+    if (a.tp_on)
+      k = bf ? conv_fwd_tc_kernel<MODE_GATHER, true, true, true> : conv_fwd_tc_kernel<MODE_GATHER, false, true, true>;
+    else if (a.idil_on || a.wtrans)
+      k = bf ? conv_fwd_tc_kernel<MODE_GATHER, true, true> : conv_fwd_tc_kernel<MODE_GATHER, false, true>;
+    else
+      k = bf ? conv_fwd_tc_kernel<MODE_GATHER, true> : conv_fwd_tc_kernel<MODE_GATHER, false>;
   }
-  return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+  const cudaError_t e = launch_pdl(k, grid, block, plan.smem, st, 1, mx, mw, my, a);
+  return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
 
 // SIMT tile shape: TN (channels per thread, BN = 16*TN) from {2, 4, 5, 6, 8}
@@ -1787,14 +1786,15 @@ SimtShape simt_shape(const Problem& P, int sms) {
 
 template <typename T, int TM, bool TR, bool MASK = false>
 cudaError_t launch_simt_tn(int tn, dim3 grid, cudaStream_t st, const SimtArgs& a) {
+  auto* k = conv_fwd_simt_kernel<T, TM, 4, TR, MASK>;
   switch (tn) {
-    case 2: conv_fwd_simt_kernel<T, TM, 2, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
-    case 5: conv_fwd_simt_kernel<T, TM, 5, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
-    case 6: conv_fwd_simt_kernel<T, TM, 6, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
-    case 8: conv_fwd_simt_kernel<T, TM, 8, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
-    default: conv_fwd_simt_kernel<T, TM, 4, TR, MASK><<<grid, kSimtThreads, 0, st>>>(a); break;
+    case 2: k = conv_fwd_simt_kernel<T, TM, 2, TR, MASK>; break;
+    case 5: k = conv_fwd_simt_kernel<T, TM, 5, TR, MASK>; break;
+    case 6: k = conv_fwd_simt_kernel<T, TM, 6, TR, MASK>; break;
+    case 8: k = conv_fwd_simt_kernel<T, TM, 8, TR, MASK>; break;
+    default: break;
   }
-  return cudaGetLastError();
+  return launch_pdl(k, grid, dim3(kSimtThreads), 0, st, 1, a);
 }
 
 int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st, int sms) {
@@ -1828,13 +1828,11 @@ int launch_simt(const Problem& P, const void* x, const void* w, void* y, cudaStr
            : (mask ? launch_simt_tn<float, 4, false, true>(sh.tn, grid, st, a)
                    : launch_simt_tn<float, 4, false>(sh.tn, grid, st, a));
   } else if (P.dtype == CONV_F16) {
-    if (tr) conv_fwd_simt_kernel<__half, 4, 4, true><<<grid, kSimtThreads, 0, st>>>(a);
-    else conv_fwd_simt_kernel<__half, 4, 4><<<grid, kSimtThreads, 0, st>>>(a);
-    e = cudaGetLastError();
+    e = launch_pdl(tr ? conv_fwd_simt_kernel<__half, 4, 4, true> : conv_fwd_simt_kernel<__half, 4, 4>, grid,
+                   dim3(kSimtThreads), 0, st, 1, a);
   } else {
-    if (tr) conv_fwd_simt_kernel<__nv_bfloat16, 4, 4, true><<<grid, kSimtThreads, 0, st>>>(a);
-    else conv_fwd_simt_kernel<__nv_bfloat16, 4, 4><<<grid, kSimtThreads, 0, st>>>(a);
-    e = cudaGetLastError();
+    e = launch_pdl(tr ? conv_fwd_simt_kernel<__nv_bfloat16, 4, 4, true> : conv_fwd_simt_kernel<__nv_bfloat16, 4, 4>,
+                   grid, dim3(kSimtThreads), 0, st, 1, a);
   }
   return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
@@ -2091,7 +2089,7 @@ int wgrad_tc_launch(const WgArgs& w, int dtype, long long max_split, const void*
   small_tensor_fixup(mdy, static_cast<size_t>(w.P) * w.O * eb, drv.driver_version);
 
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
@@ -2111,6 +2109,7 @@ int wgrad_tc_launch(const WgArgs& w, int dtype, long long max_split, const void*
       clusters <= 0)
     return CONV_ELAUNCH;
   cfg.gridDim = dim3(2 * std::min(a.total_units, clusters));
+  add_pdl(cfg, attr);
   const cudaError_t e = dtype == CONV_BF16 ? cudaLaunchKernelEx(&cfg, conv_wgrad_tc_pair_kernel<true>, mx, mdy, a)
                                            : cudaLaunchKernelEx(&cfg, conv_wgrad_tc_pair_kernel<false>, mx, mdy, a);
   return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;

@@ -37,6 +37,7 @@ namespace convfwd {
 // tensor-memory columns apart whatever N is.
 constexpr int kHTBlockHMax = 32, kHTBlockW = 8;
 constexpr uint32_t kHTAccStride = 256;
+constexpr uint32_t kTEpiWarpBytes = kTEpiBytes / 4;
 
 struct HaloTTile {
   int g, n, od, h0, w0, ot;
@@ -118,6 +119,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
   __syncthreads();
   if constexpr (PAIR) ptx::cluster_sync();
   ptx::tc_fence_after();
+  ptx::pdl_allow_next();  // setup done: the next launch may start its own
+  ptx::pdl_wait_prev();   // the previous launch's writes are visible from here on
   const uint32_t tmem_base = tail->tmem_base;
   volatile int* abort_flag = &tail->abort_flag;
   const int taps_hw = a.kH * a.kW;
@@ -335,8 +338,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // tensor-memory lane quarter: channels 32q .. 32q+31
-    const bool store_thread = warp == 2 && lane == 0;
+    // Each warp works alone on its quarter of the channels: it converts a
+    // 32-column chunk (its channels x 32 pixels) into its own slice of the
+    // staging tile and stores that slice with one TMA store issued by its
+    // lane 0, so no warp waits for another between chunks.
+    const int q = warp & 3;          // tensor-memory lane quarter
+    const int qch = mo / 4;          // channels per warp: 32 (M = 128) or 16 (M = 64)
     constexpr int kRowsPerChunk = kTEpiRows / kHTBlockW;  // 4 output rows per 32 columns
     int t = 0, chunk_seq = 0;
     for (int tile = unit; tile < a.total_tiles; tile += nunits, ++t) {
@@ -344,13 +351,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
       const uint32_t acc_phase = static_cast<uint32_t>(t >> 1) & 1u;
       bool ok = wait_bounded_warp(ptx::smem_u32(&tail->acc_full[acc]), acc_phase, abort_flag, a.timeout_ns,
                                   kSiteEpiAccFull);
-      // the four warps agree before any of them enters the named barriers
-      // below: a warp whose wait gave up must not leave the others waiting
+      // the four warps leave together when one of them gave up
       ok = named_bar_and(1, 128, ok);
       if (!ok) break;
       ptx::tc_fence_after();
       const HaloTTile ht = decode_halo_t_tile(a, tile);
-      const int o0 = ht.g * a.Og + ht.ot * o_tile + static_cast<int>(rank) * mo;
+      const int o0 = ht.g * a.Og + ht.ot * o_tile + static_cast<int>(rank) * mo + q * qch;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc) * kHTAccStride;
       for (int c = 0; c < BP; c += kTEpiRows) {
         uint32_t r[32];
@@ -358,28 +364,25 @@ __global__ void __launch_bounds__(kTThreads, 1)
         ptx::tmem_ld_wait();
         const int h = ht.h0 + (c / kTEpiRows) * kRowsPerChunk;
         if (h >= a.Ho) continue;  // the same for every epilogue thread
-        uint8_t* buf = stage_y + (a.epi_bufs == 2 ? (chunk_seq & 1) : 0) * kTEpiBytes;
-        // the store that last read this buffer (two chunks ago, or the
+        uint8_t* buf = stage_y + (a.epi_bufs == 2 ? (chunk_seq & 1) : 0) * kTEpiBytes + q * kTEpiWarpBytes;
+        // this warp's store that last read the slice (two chunks ago, or the
         // previous one with a single buffer) must be done with it
-        if (store_thread) {
+        if (lane == 0) {
           if (a.epi_bufs == 2) ptx::bulk_wait_group_read<1>();
           else ptx::bulk_wait_group_read<0>();
         }
-        named_bar_sync(1, 128);
-        // M = 128: lane l of quarter q holds channel 32q + l; M = 64: lanes 0..15 of
-        // quarter q hold channels 16q .. 16q+15 (the other 16 lanes are empty)
-        if (mo == kTO) {
-          uint16_t* dst = reinterpret_cast<uint16_t*>(buf) + q * 32 + lane;
+        __syncwarp();
+        // slice [4 rows][8 columns][qch channels]: M = 128: lane l holds
+        // channel 32q + l; M = 64: lanes 0..15 hold channels 16q .. 16q+15
+        // (the other 16 lanes are empty)
+        if (lane < qch) {
+          uint16_t* dst = reinterpret_cast<uint16_t*>(buf) + lane;
 #pragma unroll
-          for (int p = 0; p < kTEpiRows; ++p) dst[p * kTO] = cvt1<BF16>(__uint_as_float(r[p]));
-        } else if (lane < 16) {
-          uint16_t* dst = reinterpret_cast<uint16_t*>(buf) + q * 16 + lane;
-#pragma unroll
-          for (int p = 0; p < kTEpiRows; ++p) dst[p * 64] = cvt1<BF16>(__uint_as_float(r[p]));
+          for (int p = 0; p < kTEpiRows; ++p) dst[p * qch] = cvt1<BF16>(__uint_as_float(r[p]));
         }
         ptx::fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (store_thread) {
+        __syncwarp();
+        if (lane == 0) {
           if (a.rank5) ptx::tma_store_5d(&tmap_y, ptx::smem_u32(buf), o0, ht.w0, h, ht.od, ht.n);
           else ptx::tma_store_4d(&tmap_y, ptx::smem_u32(buf), o0, ht.w0, h, ht.n);
           ptx::bulk_commit_group();
@@ -395,8 +398,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
         else ptx::mbar_arrive(ae);
       }
     }
-    // every store has finished (reading shared memory and writing y) before exit
-    if (store_thread) ptx::bulk_wait_group<0>();
+    // every store of this warp has finished (reading shared memory and writing y) before exit
+    if (lane == 0) ptx::bulk_wait_group<0>();
     __syncwarp();
   }
 

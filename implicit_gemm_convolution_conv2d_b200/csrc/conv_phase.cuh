@@ -102,6 +102,8 @@ __global__ void __launch_bounds__(kPhThreads, 1)
   __syncthreads();
   ptx::cluster_sync();
   ptx::tc_fence_after();
+  ptx::pdl_allow_next();  // setup done: the next launch may start its own
+  ptx::pdl_wait_prev();   // the previous launch's writes are visible from here on
   const uint32_t tmem_base = tail->tmem_base;
   volatile int* abort_flag = &tail->abort_flag;
 

@@ -16,6 +16,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "ptx.cuh"  // programmatic dependent launch
+
 namespace convfwd {
 
 struct SimtArgs {
@@ -92,6 +94,10 @@ __global__ void __launch_bounds__(kSimtThreads) conv_fwd_simt_kernel(const SimtA
   const T* __restrict__ x = static_cast<const T*>(a.x);
   const T* __restrict__ w = static_cast<const T*>(a.w);
   T* __restrict__ y = static_cast<T*>(a.y);
+  // (no early trigger: several blocks of this kernel share an SM, and blocks of
+  // the next launch waiting beside them slow them down; the next launch starts
+  // as these blocks exit)
+  ptx::pdl_wait_prev();  // the previous launch's writes are visible from here on
 
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;

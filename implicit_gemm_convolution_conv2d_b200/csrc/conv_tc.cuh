@@ -1055,6 +1055,8 @@ __global__ void __launch_bounds__(tc_threads<MODE>(), 1)
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  ptx::pdl_allow_next();  // setup done: the next launch may start its own
+  ptx::pdl_wait_prev();   // the previous launch's writes are visible from here on
   const uint32_t tmem_base = tail->tmem_base;
   volatile int* abort_flag = &tail->abort_flag;
 
@@ -1457,6 +1459,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   ptx::cluster_sync();  // barriers of both CTAs initialised before any remote use
   ptx::tc_fence_after();
+  ptx::pdl_allow_next();  // setup done: the next launch may start its own
+  ptx::pdl_wait_prev();   // the previous launch's writes are visible from here on
   const uint32_t tmem_base = tail->tmem_base;
   volatile int* abort_flag = &tail->abort_flag;
   const int pair = blockIdx.x >> 1;

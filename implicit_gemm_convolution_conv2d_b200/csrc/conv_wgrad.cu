@@ -16,6 +16,7 @@
 
 #include "../../include/conv_fwd.h"
 #include "conv_wgrad.cuh"
+#include "launch.cuh"
 
 // Scratch of conv_wgrad_noalloc: a fixed array in the library's own device
 // image, so that entry point never allocates.  Every device that loads the
@@ -166,34 +167,38 @@ int wg_launch(const WgProblem& q, const void* x, const void* dy, void* dw, void*
     const int rc = wgrad_tc_launch(q.a, dtype, max_split, x, dy, a.part, st);
     if (rc != CONV_OK) return rc;
   } else {
-    if (dtype == CONV_F32) conv_wgrad_kernel<float><<<grid, kWgThreads, 0, st>>>(a);
-    else if (dtype == CONV_F16) conv_wgrad_kernel<__half><<<grid, kWgThreads, 0, st>>>(a);
-    else conv_wgrad_kernel<__nv_bfloat16><<<grid, kWgThreads, 0, st>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
+    auto* k = dtype == CONV_F32 ? conv_wgrad_kernel<float>
+                                : (dtype == CONV_F16 ? conv_wgrad_kernel<__half> : conv_wgrad_kernel<__nv_bfloat16>);
+    if (launch_pdl(k, grid, dim3(kWgThreads), 0, st, 1, a) != cudaSuccess) return CONV_ELAUNCH;
   }
   const long long n = q.dw_elems;
   if (n % 4 == 0) {
     // four elements a thread (dw is 16-byte aligned, so every slice is when n % 4 == 0)
-    const unsigned blocks4 = static_cast<unsigned>((n / 4 + 255) / 256);
+    const dim3 blocks4(static_cast<unsigned>((n / 4 + 255) / 256));
+    cudaError_t e;
     if (dtype == CONV_F32)
-      conv_wgrad_reduce4_kernel<float><<<blocks4, 256, 0, st>>>(a.part, static_cast<float*>(dw), n, a.nsplit);
+      e = launch_pdl(conv_wgrad_reduce4_kernel<float>, blocks4, dim3(256), 0, st, 1, a.part, static_cast<float*>(dw),
+                     n, a.nsplit);
     else if (dtype == CONV_F16)
-      conv_wgrad_reduce4_kernel<__half><<<blocks4, 256, 0, st>>>(a.part, static_cast<__half*>(dw), n, a.nsplit);
+      e = launch_pdl(conv_wgrad_reduce4_kernel<__half>, blocks4, dim3(256), 0, st, 1, a.part, static_cast<__half*>(dw),
+                     n, a.nsplit);
     else
-      conv_wgrad_reduce4_kernel<__nv_bfloat16><<<blocks4, 256, 0, st>>>(a.part, static_cast<__nv_bfloat16*>(dw), n,
-                                                                       a.nsplit);
-    return cudaGetLastError() == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+      e = launch_pdl(conv_wgrad_reduce4_kernel<__nv_bfloat16>, blocks4, dim3(256), 0, st, 1, a.part,
+                     static_cast<__nv_bfloat16*>(dw), n, a.nsplit);
+    return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
   }
-  const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
+  const dim3 blocks(static_cast<unsigned>((n + 255) / 256));
+  cudaError_t e;
   if (dtype == CONV_F32)
-    conv_wgrad_reduce_kernel<float><<<blocks, 256, 0, st>>>(a.part, static_cast<float*>(dw), n, a.nsplit);
+    e = launch_pdl(conv_wgrad_reduce_kernel<float>, blocks, dim3(256), 0, st, 1, a.part, static_cast<float*>(dw), n,
+                   a.nsplit);
   else if (dtype == CONV_F16)
-    conv_wgrad_reduce_kernel<__half><<<blocks, 256, 0, st>>>(a.part, static_cast<__half*>(dw), n, a.nsplit);
+    e = launch_pdl(conv_wgrad_reduce_kernel<__half>, blocks, dim3(256), 0, st, 1, a.part, static_cast<__half*>(dw), n,
+                   a.nsplit);
   else
-    conv_wgrad_reduce_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(a.part, static_cast<__nv_bfloat16*>(dw), n,
-                                                                    a.nsplit);
-  if (cudaGetLastError() != cudaSuccess) return CONV_ELAUNCH;
-  return CONV_OK;
+    e = launch_pdl(conv_wgrad_reduce_kernel<__nv_bfloat16>, blocks, dim3(256), 0, st, 1, a.part,
+                   static_cast<__nv_bfloat16*>(dw), n, a.nsplit);
+  return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
 
 constexpr size_t kWgStaticScratchBytes = CONV_WGRAD_STATIC_SCRATCH_BYTES;

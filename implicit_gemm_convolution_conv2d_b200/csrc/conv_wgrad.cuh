@@ -57,6 +57,10 @@ __global__ void __launch_bounds__(kWgThreads) conv_wgrad_kernel(const WgArgs a) 
 
   const T* __restrict__ x = static_cast<const T*>(a.x);
   const T* __restrict__ dy = static_cast<const T*>(a.dy);
+  // (no early trigger: several blocks of this kernel share an SM, and blocks of
+  // the next launch waiting beside them slow them down; the next launch starts
+  // as these blocks exit)
+  ptx::pdl_wait_prev();  // the previous launch's writes are visible from here on
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const int col0 = blockIdx.x * kWgBN;
@@ -178,6 +182,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) conv_wgrad_reduce_kernel(const float* __restrict__ part, T* __restrict__ dw,
                                                                 long long n, int nsplit) {
   const long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  ptx::pdl_wait_prev();  // the ranges' partial sums are complete and visible
   if (i >= n) return;
   float s = part[i];
   for (int k = 1; k < nsplit; ++k) s += part[static_cast<long long>(k) * n + i];
@@ -190,6 +195,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) conv_wgrad_reduce4_kernel(const float* __restrict__ part, T* __restrict__ dw,
                                                                  long long n, int nsplit) {
   const long long i = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) * 4;
+  ptx::pdl_wait_prev();  // the ranges' partial sums are complete and visible
   if (i >= n) return;
   float4 s = *reinterpret_cast<const float4*>(part + i);
   for (int k = 1; k < nsplit; ++k) {

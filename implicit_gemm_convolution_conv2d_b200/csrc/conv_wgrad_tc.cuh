@@ -111,6 +111,9 @@ __global__ void __launch_bounds__(kWgtThreads, 1)
   __syncthreads();
   ptx::cluster_sync();  // barriers of both CTAs initialised before any remote use
   ptx::tc_fence_after();
+  // (no early trigger: the ordered sum that follows this kernel would wait
+  // beside it on every SM; it starts as these CTAs exit)
+  ptx::pdl_wait_prev();   // the previous launch's writes are visible from here on
   const uint32_t tmem_base = tail->tmem_base;
   volatile int* abort_flag = &tail->abort_flag;
   const int pair = blockIdx.x >> 1;

@@ -10,6 +10,15 @@
 namespace convfwd {
 namespace ptx {
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel on its stream is still
+// running: it lets the next launch start (launch_dependents) once its own
+// setup is done, then waits (griddepcontrol.wait) until the previous grid has
+// completed and its memory writes are visible, before its first access to
+// global memory.  Without that launch attribute the wait returns at once.
+__device__ __forceinline__ void pdl_allow_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_prev() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
