@@ -112,6 +112,7 @@ KERNEL_SOURCES = {
     "depthwise_direct": ["conv_fwd.cu", "conv_simt.cuh", "conv_dw.cuh", "ptx.cuh", "launch.cuh"],
     "simt_wgrad": ["conv_wgrad.cu", "conv_wgrad.cuh", "conv_simt.cuh", "ptx.cuh", "launch.cuh"],
     "tcgen05_tma_phases_pair": _COMMON_SRC + ["conv_tconv.cuh"],
+    "tcgen05_staged_t": _COMMON_SRC + ["conv_tct.cuh", "conv_staged.cuh"],
     "tcgen05_wgrad_pair": ["conv_fwd.cu", "conv_wgrad.cu", "conv_wgrad.cuh", "conv_wgrad_tc.cuh", "conv_tc.cuh",
                            "ptx.cuh", "launch.cuh"],
 }
@@ -699,7 +700,8 @@ def main(argv=None):
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     ap.add_argument("--variant", default="AUTO",
                     choices=["AUTO", "SIMT", "TC_TMA", "TC_GATHER", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T", "TC_HALO_T",
-                             "TC_HALO_T_PAIR", "TC_PHASE", "DEPTHWISE", "DEPTHWISE_DIRECT", "TC_TMA_PHASES"],
+                             "TC_HALO_T_PAIR", "TC_PHASE", "DEPTHWISE", "DEPTHWISE_DIRECT", "TC_TMA_PHASES",
+                             "TC_STAGED"],
                     help="kernel variant (default: the library's own choice)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--pad-hi", default=None,

@@ -20,7 +20,7 @@ __all__ = ["conv_fwd", "conv_fwd_host", "out_dims", "plan", "conv_transpose", "t
            "CONV_F32", "CONV_F16", "CONV_BF16", "VARIANT_AUTO", "VARIANT_SIMT", "VARIANT_TC_TMA",
            "VARIANT_TC_GATHER", "VARIANT_TC_TMA_PAIR", "VARIANT_TC_HALO", "VARIANT_TC_HALO_PAIR",
            "VARIANT_TC_TMA_T", "VARIANT_TC_HALO_T", "VARIANT_TC_HALO_T_PAIR", "VARIANT_TC_PHASE", "VARIANT_DEPTHWISE", "VARIANT_DEPTHWISE_DIRECT",
-           "VARIANT_TC_TMA_PHASES", "ConvError"]
+           "VARIANT_TC_TMA_PHASES", "VARIANT_TC_STAGED", "ConvError"]
 
 CONV_F32, CONV_F16, CONV_BF16 = 0, 1, 2
 VARIANT_AUTO, VARIANT_SIMT, VARIANT_TC_TMA, VARIANT_TC_GATHER, VARIANT_TC_TMA_PAIR = -1, 0, 1, 2, 3
@@ -29,13 +29,14 @@ VARIANT_TC_PHASE = 9
 VARIANT_DEPTHWISE = 10
 VARIANT_DEPTHWISE_DIRECT = 11
 VARIANT_TC_TMA_PHASES = 12       # conv_transpose only: sub-pixel phases fed by TMA, CTA pairs
+VARIANT_TC_STAGED = 13           # any channel count: realigned input regions read as per-tap views
 VARIANT_NAMES = {VARIANT_SIMT: "simt_ffma", VARIANT_TC_TMA: "tcgen05_tma_im2col",
                  VARIANT_TC_GATHER: "tcgen05_gather", VARIANT_TC_TMA_PAIR: "tcgen05_tma_im2col_pair",
                  VARIANT_TC_HALO: "tcgen05_tma_halo", VARIANT_TC_HALO_PAIR: "tcgen05_tma_halo_pair",
                  VARIANT_TC_TMA_T: "tcgen05_tma_im2col_t", VARIANT_TC_HALO_T: "tcgen05_tma_halo_t",
                  VARIANT_TC_HALO_T_PAIR: "tcgen05_tma_halo_t_pair", VARIANT_TC_PHASE: "tcgen05_tma_phase",
                  VARIANT_DEPTHWISE: "depthwise_tma", VARIANT_DEPTHWISE_DIRECT: "depthwise_direct",
-                 VARIANT_TC_TMA_PHASES: "tcgen05_tma_phases_pair"}
+                 VARIANT_TC_TMA_PHASES: "tcgen05_tma_phases_pair", VARIANT_TC_STAGED: "tcgen05_staged_t"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libconvfwd.so")

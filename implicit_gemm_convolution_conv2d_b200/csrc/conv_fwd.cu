@@ -19,6 +19,7 @@
 #include "conv_halo_t.cuh"
 #include "conv_phase.cuh"
 #include "conv_dw.cuh"
+#include "conv_staged.cuh"
 #include "conv_wgrad.cuh"
 #include "launch.cuh"
 #include "conv_wgrad_tc.cuh"
@@ -260,6 +261,14 @@ int set_kernel_attrs(int dev) {
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_wgrad_tc_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_tconv_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_tconv_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_staged_kernel<false, 3, 3, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_staged_kernel<false, 3, 3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_staged_kernel<false, 0, 0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_staged_kernel<false, 0, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_staged_kernel<true, 3, 3, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_staged_kernel<true, 3, 3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_staged_kernel<true, 0, 0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  e = e != cudaSuccess ? e : cudaFuncSetAttribute(conv_fwd_tc_staged_kernel<true, 0, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return CONV_ELAUNCH;
   g_dev[dev].attrs_set = true;
   return CONV_OK;
@@ -1365,6 +1374,112 @@ int launch_tconv(const Problem& P, const void* x, const void* w, void* y, cudaSt
   return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
 }
 
+// Staged kernel (conv_staged.cuh) for channel counts that TMA cannot address:
+// f16/bf16, one group, stride 1, O <= 128, no flip, a forward (undilated)
+// input.  The block height is the multiple of 4 up to 32 that wastes the
+// fewest rows of Ho (ties to the taller block); the pipeline takes as many
+// slots (weights of the kH*kW taps + two region planes) as shared memory holds.
+int plan_staged(const Problem& P, int sms, StArgs& a, int& ctas, size_t& smem) {
+  if (P.dtype == CONV_F32 || P.G != 1 || P.flip || !plain_input(P)) return CONV_EUNSUPPORTED;
+  if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1 || P.O > 128) return CONV_EUNSUPPORTED;
+  int bh = 32;
+  long long best = -1;
+  for (int h = 32; h >= 4; h -= 4) {
+    const long long covered = static_cast<long long>((P.Ho + h - 1) / h) * h;
+    if (best < 0 || covered < best) {
+      best = covered;
+      bh = h;
+    }
+  }
+  const long long Hr = bh + static_cast<long long>(P.d[1]) * (P.kH - 1);
+  const long long Wr = kStBlockW + static_cast<long long>(P.d[2]) * (P.kW - 1);
+  const long long plane = Hr * Wr * 16;
+  const long long groups = (P.O + 7) / 8;
+  const long long abytes = static_cast<long long>(P.kH) * P.kW * groups * kStAGroupBytes + (16 - groups) * kStAGroupBytes;
+  const long long stage = (abytes + 2 * plane + 127) / 128 * 128;
+  const long long budget = static_cast<long long>(kSmemBudget) - 1024 - static_cast<long long>(sizeof(StTail)) - 64;
+  long long nst = std::min<long long>(kMaxStages, budget / stage);
+  if (nst < 2) return CONV_EUNSUPPORTED;
+  // raw mode when the staged input rows and weight rows fit beside two slots:
+  // a row's 16-byte cover is at most its bytes + 30
+  const long long taps_hw = static_cast<long long>(P.kH) * P.kW;
+  // rows 16 bytes past a multiple of 128 apart, so that eight consecutive
+  // rows' 16-byte reads fall in different banks
+  const long long rx_row = (Wr * P.C * 2 + 30 + 127) / 128 * 128 + 16;
+  const long long rw_row = (taps_hw * P.C * 2 + 30 + 127) / 128 * 128 + 16;
+  const long long raw_bytes = Hr * rx_row + static_cast<long long>(P.O) * rw_row;
+  // (and each builder thread has at most kStBatch units a slot, decoded once per (block, kd))
+  const long long units = 2 * Hr * Wr + taps_hw * P.O * 2;
+  const bool raw = budget - raw_bytes >= 2 * stage && units <= static_cast<long long>(kStBatch) * kStBuilders;
+  if (raw) nst = std::min<long long>(kMaxStages, (budget - raw_bytes) / stage);
+  const long long tiles_h = (P.Ho + bh - 1) / bh, tiles_w = (P.Wo + kStBlockW - 1) / kStBlockW;
+  const long long total = static_cast<long long>(P.N) * P.Do * tiles_h * tiles_w;
+  if (total > 0x7fffffffLL) return CONV_EINVAL;
+  std::memset(&a, 0, sizeof(a));
+  a.N = P.N; a.D = P.D; a.H = P.H; a.W = P.W; a.C = P.C; a.O = P.O;
+  a.kD = P.kD; a.kH = P.kH; a.kW = P.kW;
+  a.pd = P.p[0]; a.ph = P.p[1]; a.pw = P.p[2];
+  a.dd = P.d[0]; a.dh = P.d[1]; a.dw = P.d[2];
+  a.Do = P.Do; a.Ho = P.Ho; a.Wo = P.Wo;
+  a.K = P.K;
+  a.x_blocks = static_cast<long long>((P.x_bytes + 15) / 16);
+  a.w_blocks = static_cast<long long>((P.w_bytes + 15) / 16);
+  a.tile_h = bh;
+  a.tiles_h = static_cast<int>(tiles_h);
+  a.tiles_w = static_cast<int>(tiles_w);
+  a.total_tiles = static_cast<int>(total);
+  a.nc16 = (P.C + 15) / 16;
+  a.Hr = static_cast<int>(Hr);
+  a.Wr = static_cast<int>(Wr);
+  a.plane_bytes = static_cast<uint32_t>(plane);
+  a.tap_bytes = static_cast<uint32_t>(groups * kStAGroupBytes);
+  a.a_bytes = static_cast<uint32_t>(abytes);
+  a.stage_bytes = static_cast<uint32_t>(stage);
+  a.stages = static_cast<int>(nst);
+  a.raw = raw ? 1 : 0;
+  a.rx_row = static_cast<uint32_t>(rx_row);
+  a.rw_row = static_cast<uint32_t>(rw_row);
+  a.raw_x_off = static_cast<uint32_t>(nst * stage);
+  a.raw_w_off = a.raw_x_off + static_cast<uint32_t>(Hr * rx_row);
+  a.tail_off = static_cast<uint32_t>(nst * stage + (raw ? raw_bytes : 0));
+  const uint32_t ab = P.dtype == CONV_BF16 ? 1u : 0u;
+  a.idesc = (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(kStBlockW * bh >> 3) << 17) |
+            ((128u >> 4) << 24);
+  a.tmem_cols = 2 * kStAccStride;
+  a.timeout_ns = kWaitTimeoutNs;
+  ctas = static_cast<int>(std::min<long long>(total, sms));
+  smem = static_cast<size_t>(a.tail_off) + 1024 + sizeof(StTail) + 64;
+  return CONV_OK;
+}
+
+int launch_staged(const Problem& P, const void* x, const void* w, void* y, cudaStream_t st, int dev, int sms) {
+  StArgs a;
+  int ctas = 0;
+  size_t smem = 0;
+  int rc = plan_staged(P, sms, a, ctas, smem);
+  if (rc != CONV_OK) return rc;
+  rc = set_kernel_attrs(dev);
+  if (rc != CONV_OK) return rc;
+  a.x = x;
+  a.w = w;
+  a.y = y;
+  const unsigned long long stall_ns = g_inject_stall_ns.exchange(0);
+  if (stall_ns != 0) {
+    a.inject_stall = 1;
+    a.timeout_ns = stall_ns;
+  }
+  const bool bf = P.dtype == CONV_BF16, k33 = P.kH == 3 && P.kW == 3;
+  auto* k = conv_fwd_tc_staged_kernel<false, 0, 0, false>;  // every instantiation has this signature
+  if (a.raw)
+    k = bf ? (k33 ? conv_fwd_tc_staged_kernel<true, 3, 3, true> : conv_fwd_tc_staged_kernel<true, 0, 0, true>)
+           : (k33 ? conv_fwd_tc_staged_kernel<false, 3, 3, true> : conv_fwd_tc_staged_kernel<false, 0, 0, true>);
+  else
+    k = bf ? (k33 ? conv_fwd_tc_staged_kernel<true, 3, 3, false> : conv_fwd_tc_staged_kernel<true, 0, 0, false>)
+           : (k33 ? conv_fwd_tc_staged_kernel<false, 3, 3, false> : conv_fwd_tc_staged_kernel<false, 0, 0, false>);
+  const cudaError_t e = launch_pdl(k, dim3(ctas), dim3(kStThreads), smem, st, 1, a);
+  return e == cudaSuccess ? CONV_OK : CONV_ELAUNCH;
+}
+
 int choose_variant(const Problem& P, int sms) {
   if (!plain_input(P)) {
     if (P.dtype == CONV_F32) return CONV_VARIANT_SIMT;
@@ -1378,7 +1493,15 @@ int choose_variant(const Problem& P, int sms) {
   bool r5;
   if (!tma_fits(P, r5)) {
     TcPlan pp;
-    return plan_phase(P, sms, pp) == CONV_OK ? CONV_VARIANT_TC_PHASE : CONV_VARIANT_TC_GATHER;
+    if (plan_phase(P, sms, pp) == CONV_OK) return CONV_VARIANT_TC_PHASE;
+    // the staged kernel from 16 channels a group up ((4,32^3,65)->65: 0.153
+    // against 0.531 ms; 21 channels: 0.0193 against 0.0201); below that its
+    // fixed per-slot cost loses to the gather kernel (3 channels: 0.0170
+    // against 0.0087 ms)
+    StArgs sa;
+    int c;
+    size_t sm;
+    return P.Cg >= 16 && plan_staged(P, sms, sa, c, sm) == CONV_OK ? CONV_VARIANT_TC_STAGED : CONV_VARIANT_TC_GATHER;
   }
   if (P.Og % 64 == 0 && P.Og % 256 != 0 && P.kH >= 2) {
     TcPlan hp;
@@ -1906,6 +2029,7 @@ int run(const Problem& P, const void* x, const void* w, void* y, int variant, cu
   if (variant == CONV_VARIANT_DEPTHWISE) return launch_dw(P, x, w, y, st, sms);
   if (variant == CONV_VARIANT_DEPTHWISE_DIRECT) return launch_dw_direct(P, x, w, y, st);
   if (variant == CONV_VARIANT_TC_TMA_PHASES) return launch_tconv(P, x, w, y, st, dev, sms);
+  if (variant == CONV_VARIANT_TC_STAGED) return launch_staged(P, x, w, y, st, dev, sms);
   TcPlan plan;
   rc = plan_tc(P, variant, sms, plan);
   if (rc != CONV_OK) return rc;
@@ -2145,7 +2269,7 @@ int conv_fwd_ex(const void* x, const void* w, void* y, int N, int D, int H, int 
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_PHASES) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_STAGED) return CONV_EINVAL;
   if (variant == CONV_VARIANT_TC_TMA_PHASES) return CONV_EUNSUPPORTED;  // transposed convolutions only
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -2225,7 +2349,7 @@ int conv_transpose(const void* x, const void* w, void* y, int N, int D, int H, i
   if (rc != CONV_OK) return rc;
   rc = check_pointers(P, x, w, y);
   if (rc != CONV_OK) return rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_PHASES) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_STAGED) return CONV_EINVAL;
   return run(P, x, w, y, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -2245,7 +2369,7 @@ namespace {
 
 int plan_problem(const Problem& P, int variant, int* bn, int* stages, int* ctas) {
   int rc;
-  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_TMA_PHASES) return CONV_EINVAL;
+  if (variant < CONV_VARIANT_AUTO || variant > CONV_VARIANT_TC_STAGED) return CONV_EINVAL;
   int dev, sms = 148;
   if (current_device(dev) == CONV_OK) device_sms(dev, sms);
   if (variant == CONV_VARIANT_AUTO) variant = choose_variant(P, sms);
@@ -2277,6 +2401,17 @@ int plan_problem(const Problem& P, int variant, int* bn, int* stages, int* ctas)
     if (rc != CONV_OK) return rc;
     if (bn) *bn = ta.BN;
     if (stages) *stages = ta.stages;
+    if (ctas) *ctas = c;
+    return variant;
+  }
+  if (variant == CONV_VARIANT_TC_STAGED) {
+    StArgs sa;
+    int c;
+    size_t sm;
+    rc = plan_staged(P, sms, sa, c, sm);
+    if (rc != CONV_OK) return rc;
+    if (bn) *bn = kStBlockW * sa.tile_h;
+    if (stages) *stages = sa.stages;
     if (ctas) *ctas = c;
     return variant;
   }

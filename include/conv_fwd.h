@@ -106,11 +106,18 @@ enum {
                                    through an mbarrier ring (DEPTHWISE_DIRECT where the slabs do
                                    not fit); the automatic choice for these shapes */
   CONV_VARIANT_DEPTHWISE_DIRECT = 11, /* depthwise, loads straight from global memory */
-  CONV_VARIANT_TC_TMA_PHASES = 12  /* conv_transpose only: one stride-1 implicit GEMM per
+  CONV_VARIANT_TC_TMA_PHASES = 12, /* conv_transpose only: one stride-1 implicit GEMM per
                                    sub-pixel phase on tcgen05 CTA pairs, A by TMA im2col of
                                    the undilated input, B straight from w as MN-major tiles
                                    (f16/bf16, dilation 1, Cin/G % 64 == 0, Cout/G % 128 == 0,
                                    strides <= 8, a geometry inside the TMA im2col limits) */
+  CONV_VARIANT_TC_STAGED = 13     /* any channel count (the path for C*2 % 16 != 0): builder
+                                   warps realign, per (kd, 16-channel chunk), the input
+                                   region of an up-to-32 x 8 output block and the matching
+                                   weights into unswizzled K-major shared-memory tiles that
+                                   every (kh, kw) tap reads as a descriptor view; tcgen05
+                                   MMA M = 128 output channels, N = the block's pixels
+                                   (f16/bf16, groups 1, stride 1, O <= 128, no flip) */
 };
 
 /* Output extents.  stride/pad/dil: 3 ints (d, h, w).  out: 3 ints (Do, Ho, Wo).

@@ -95,7 +95,7 @@ def test_flip_and_side_padding_arguments(C):
     assert ex(i3(0, -1, 0), 0) == -1           # negative high-side pad
     assert ex(i3(0, 1, 1), 2) == -1            # flip is 0 or 1
     assert ex(i3(0, 1, 1), 0, 9) == -2         # dtype
-    assert ex(i3(0, 1, 1), 0, 1, 13) == -1     # unknown variant
+    assert ex(i3(0, 1, 1), 0, 1, 14) == -1     # unknown variant
     assert ex(i3(0, 1, 1), 0, 1, 12) == -7     # the transposed-convolution phase kernel: not a forward variant
     # flip keeps the phase-packed kernel (its B rows are built from the mirrored filter)
     stem = (2, 1, 32, 32, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")
@@ -139,7 +139,7 @@ def test_invalid_arguments_rejected_on_host(C):
     big = 1 << 30
     assert call(X, Wt, Y, big, big, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, None) == -1
     # unknown variant
-    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 13, None) == -1
+    assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, 14, None) == -1
     assert L.conv_fwd_variant(X, Wt, Y, 1, 1, 4, 4, 16, 16, 1, 3, 3, s, p, d, 1, 1, -2, None) == -1
 
 
@@ -150,7 +150,7 @@ def test_strerror_covers_codes(C):
 
 
 def test_variant_plan(C):
-    plan = lambda *a: C.plan(*a)
+    plan = lambda *a, **k: C.plan(*a, **k)
     v, bn, st, _ = plan(64, 1, 56, 56, 256, 256, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16")
     assert v == C.VARIANT_TC_TMA_PAIR and bn == 256 and st >= 2
     v, bn, _, _ = plan(1, 1, 56, 56, 64, 64, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "f16")
@@ -184,13 +184,20 @@ def test_variant_plan(C):
     # ... unless a condition fails (W*C*2 not a multiple of 16; Wo not a multiple of P)
     assert plan(2, 1, 16, 15, 3, 64, (1, 7, 7), (1, 2, 2), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
     assert plan(2, 1, 16, 24, 3, 64, (1, 7, 7), (1, 3, 3), (0, 3, 3), (1, 1, 1), 1, "bf16")[0] == C.VARIANT_TC_GATHER
-    v, bn, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
-    assert v == C.VARIANT_TC_GATHER and bn == 96
+    # unaligned channels at stride 1: the staged kernel, 16 x 8 output blocks (Ho = 16)
+    v, bn, st, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
+    assert v == C.VARIANT_TC_STAGED and bn == 128 and st >= 2
+    # ... but the gather kernel past its conditions (O > 128; groups; flip)
+    v, bn, _, _ = plan(4, 16, 16, 16, 65, 130, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
+    assert v == C.VARIANT_TC_GATHER
+    assert plan(2, 4, 8, 8, 42, 42, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 2, "f16")[0] == C.VARIANT_TC_GATHER
+    assert plan(2, 4, 8, 8, 21, 21, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16",
+                flip=1)[0] == C.VARIANT_TC_GATHER
     v, _, _, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f32")
     assert v == C.VARIANT_SIMT
-    # 3-D with pad beyond the rank-5 im2col corner range goes to the gather kernel
+    # 3-D with pad beyond the rank-5 im2col corner range goes to the staged kernel
     v, _, _, _ = plan(1, 40, 8, 8, 64, 64, (3, 3, 3), (1, 1, 1), (17, 1, 1), (1, 1, 1), 1, "f16")
-    assert v == C.VARIANT_TC_GATHER
+    assert v == C.VARIANT_TC_STAGED
     # channel chunks of 32 and 16
     assert plan(2, 64, 64, 64, 32, 256, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA_PAIR
     assert plan(2, 64, 64, 64, 32, 384, (1, 1, 1), (1, 1, 1), (0, 0, 0), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_TMA
@@ -250,7 +257,7 @@ def test_explicit_variant_plan(C):
     tall = (1, 1, 200, 32, 16, 16, (1, 5, 3), (1, 1, 1), (0, 140, 1), (1, 70, 1), 16)
     assert C.plan(*tall, "f16")[:3] == (C.VARIANT_DEPTHWISE, 8, 1)  # the direct form's 8 channels
     with pytest.raises(C.ConvError) as e:
-        C.plan(*g3, "bf16", 13)
+        C.plan(*g3, "bf16", 14)
     assert e.value.code == -1
     with pytest.raises(C.ConvError) as e:   # the transposed-convolution phase kernel
         C.plan(*g3, "bf16", C.VARIANT_TC_TMA_PHASES)

@@ -35,7 +35,7 @@ def _geom(wl):
 
 
 @pytest.mark.parametrize("variant", ["TC_GATHER", "TC_TMA", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T",
-                                     "TC_HALO_T", "TC_HALO_T_PAIR", "TC_PHASE", "DEPTHWISE"])
+                                     "TC_HALO_T", "TC_HALO_T_PAIR", "TC_PHASE", "DEPTHWISE", "TC_STAGED"])
 def test_injected_stall_times_out_and_recovers(variant):
     v = getattr(C, "VARIANT_" + variant)
     O = {"TC_TMA_T": 128, "TC_HALO_T": 128, "TC_HALO_T_PAIR": 256}.get(variant, 64)

@@ -66,7 +66,19 @@ def variants_for(wl):
         vs.append(C.VARIANT_TC_HALO_T_PAIR)
     if phase_applies(wl):
         vs.append(C.VARIANT_TC_PHASE)
+    if staged_applies(wl):
+        vs.append(C.VARIANT_TC_STAGED)
     return vs
+
+
+def staged_applies(wl):
+    """The staged kernel's conditions (one group, stride 1, O <= 128, its
+    pipeline slots fit in shared memory), as the library plans them."""
+    try:
+        return C.plan(wl.N, wl.D, wl.H, wl.W, wl.C, wl.O, wl.k, wl.stride, wl.pad, wl.dil, wl.groups, wl.dtype,
+                      C.VARIANT_TC_STAGED)[0] == C.VARIANT_TC_STAGED
+    except C.ConvError:
+        return False
 
 
 def depthwise_applies(wl):
@@ -107,6 +119,16 @@ SMALL = [
     WL.case(1, 6, 7, 8, 64, 128, (1, 3, 3), pad=(0, 1, 1), name="3d_k133"),
     WL.case(1, 5, 6, 5, 32, 64, (3, 3, 3), pad=(1, 1, 1), name="3d_c32"),
     WL.case(1, 4, 5, 6, 65, 65, (3, 3, 3), pad=(1, 1, 1), name="3d_c65"),
+    # the staged kernel: odd channel counts and chunk tails (C = 1, 5, 100),
+    # O = 1 and 128, block heights that do not divide Ho, blocks past W,
+    # dilation inside the staged region, even filters, empty depth planes,
+    # filters other than 3 x 3 (taps looped at run time)
+    WL.case(2, 3, 11, 13, 5, 7, (3, 3, 3), pad=(1, 2, 1), dil=(1, 2, 1), name="st_c5_o7_dil"),
+    WL.case(1, 2, 9, 19, 100, 128, (1, 3, 3), pad=(0, 1, 1), name="st_c100_o128"),
+    WL.case(2, 1, 6, 9, 1, 1, (1, 3, 3), pad=(0, 1, 1), name="st_c1_o1"),
+    WL.case(1, 1, 37, 10, 13, 40, (1, 5, 3), pad=(0, 2, 1), name="st_ho37_k53"),
+    WL.case(3, 2, 7, 21, 24, 24, (2, 2, 2), pad=(1, 0, 1), name="st_k222_w_edge"),
+    WL.case(1, 5, 6, 7, 9, 33, (3, 3, 3), pad=(3, 1, 1), name="st_empty_depth_planes"),
     WL.case(2, 4, 5, 6, 3, 32, (3, 3, 3), pad=(1, 1, 1), name="3d_c3"),
     WL.case(1, 7, 6, 9, 16, 16, (2, 3, 2), (2, 2, 1), (1, 0, 2), (2, 1, 3), name="3d_mixed"),
     WL.case(1, 1, 8, 8, 8, 8, (1, 3, 3), (1, 3, 3), (0, 3, 3), (1, 3, 3), name="s3_d3_p3"),
@@ -215,7 +237,7 @@ FLIP_PAD = [
 ]
 
 ALL_VARIANTS = ["SIMT", "TC_TMA", "TC_GATHER", "TC_TMA_PAIR", "TC_HALO", "TC_HALO_PAIR", "TC_TMA_T", "TC_HALO_T",
-                "TC_HALO_T_PAIR", "TC_PHASE", "DEPTHWISE", "DEPTHWISE_DIRECT"]
+                "TC_HALO_T_PAIR", "TC_PHASE", "DEPTHWISE", "DEPTHWISE_DIRECT", "TC_STAGED"]
 
 
 def run_gpu_ex(x, w, wl, pad_hi, flip, variant, guard=64):
