@@ -30,9 +30,9 @@
 // end of the weight area) and land in accumulator lanes the epilogue never
 // stores.
 //
-// Roles: 16 builder warps (every builder thread waits on the slot's `empty`
+// Roles: 20 builder warps (every builder thread waits on the slot's `empty`
 // barrier, fills its share, fences the async proxy and arrives on `full`),
-// one MMA-issuing thread (warp 16), four epilogue warps (17..20, tensor-memory
+// one MMA-issuing thread (warp 20), four epilogue warps (21..24, tensor-memory
 // lane quarter warp & 3) that convert 32-column chunks and store y with
 // 16-bit stores (y's rows are O*2 bytes apart, not a TMA stride).  Two
 // accumulators of 256 columns; every wait is bounded.
@@ -48,11 +48,11 @@
 
 namespace convfwd {
 
-// The builders are latency-bound: 8, 12 and 16 warps took 0.205, 0.176 and
-// 0.153 ms on (4,32^3,65)->65.
-constexpr int kStBuilderWarps = 16;
+// The builders are latency-bound: 8, 12, 16 and 20 warps took 0.205, 0.176,
+// 0.152 and 0.148 ms on (4,32^3,65)->65.
+constexpr int kStBuilderWarps = 20;
 constexpr int kStBuilders = 32 * kStBuilderWarps;
-constexpr int kStMmaWarp = kStBuilderWarps;         // warp 16
+constexpr int kStMmaWarp = kStBuilderWarps;         // warp 20
 constexpr int kStThreads = 32 * (kStBuilderWarps + 1 + 4);
 constexpr uint32_t kStAGroupBytes = 256;           // 8 weight rows x 16 channels (two 128-byte halves)
 constexpr uint32_t kStAccStride = 256;              // tensor-memory columns per accumulator
@@ -187,7 +187,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-constexpr int kStBatch = 4;  // units a builder thread has in flight
+constexpr int kStBatch = 3;  // units a builder thread has in flight
 
 // Builder thread `bt`'s share of one pipeline slot: the region of depth tap kd
 // and channel chunk cc for block t (units 0 .. 2*Hr*Wr-1: pixel u/2, channel
