@@ -137,9 +137,12 @@ int conv_out_dims(int D, int H, int W, int kD, int kH, int kW,
  * else TC_TMA_T when there are at least as many 256-pixel tiles as SMs;
  * otherwise TC_TMA_PAIR (or TC_TMA when there are fewer 256-row output tiles
  * than SM pairs); otherwise TC_PHASE where its conditions hold, else
- * TC_GATHER.  Depthwise problems (groups = C = O, C*elem % 16 == 0), of any
- * type, run DEPTHWISE.  TC_HALO, TC_HALO_PAIR and
- * TC_HALO_T_PAIR run only when requested through conv_fwd_variant. */
+ * TC_STAGED from 16 channels a group up where it plans, else TC_GATHER.
+ * Depthwise problems (groups = C = O, C*elem % 16 == 0), of any type, run
+ * DEPTHWISE.  TC_HALO, TC_HALO_PAIR and TC_HALO_T_PAIR run only when
+ * requested through conv_fwd_variant.  Every kernel is launched with
+ * programmatic stream serialization and waits for the previous kernel on the
+ * stream before it touches global memory: results are those of stream order. */
 int conv_fwd(const void* x, const void* w, void* y,
              int N, int D, int H, int W, int C, int O,
              int kD, int kH, int kW,
@@ -169,7 +172,8 @@ int conv_fwd_ex(const void* x, const void* w, void* y,
  * need C/G % 16 == 0 and a geometry inside the TMA im2col limits, TC_TMA_T
  * also O/G % 128 == 0; TC_HALO and TC_HALO_PAIR need stride 1 and
  * C/G % 32 == 0; TC_HALO_T also O/G % 64 == 0, TC_HALO_T_PAIR
- * O/G % 256 == 0). */
+ * O/G % 256 == 0; TC_STAGED needs one group, stride 1, O <= 128, no flip
+ * and two pipeline slots in shared memory). */
 int conv_fwd_variant(const void* x, const void* w, void* y,
                      int N, int D, int H, int W, int C, int O,
                      int kD, int kH, int kW,
