@@ -187,6 +187,22 @@ def test_variant_plan(C):
     # unaligned channels at stride 1: the staged kernel, 16 x 8 output blocks (Ho = 16)
     v, bn, st, _ = plan(4, 16, 16, 16, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_STAGED and bn == 128 and st >= 2
+    # (4,32^3,65)->65: 32 x 8 blocks, two slots beside the staged input and weight rows
+    v, bn, st, ct = plan(4, 32, 32, 32, 65, 65, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
+    assert v == C.VARIANT_TC_STAGED and bn == 256 and st == 2 and ct == 148
+    # 21 channels: the staged kernel too; 3 channels: the gather kernel (faster there)
+    assert plan(4, 16, 16, 16, 21, 21, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_STAGED
+    assert plan(4, 16, 16, 16, 3, 32, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")[0] == C.VARIANT_TC_GATHER
+    # the staged kernel on request: Ho = 9 takes 12-row blocks (the fewest padded rows, ties to
+    # the taller block); stride 2, O > 128 and two groups are refused
+    assert plan(1, 1, 9, 9, 3, 8, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "bf16",
+                C.VARIANT_TC_STAGED)[:2] == (C.VARIANT_TC_STAGED, 96)
+    for args in [(1, 1, 16, 16, 21, 21, (1, 3, 3), (1, 2, 2), (0, 1, 1), (1, 1, 1), 1, "f16"),
+                 (1, 1, 16, 16, 21, 130, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 1, "f16"),
+                 (1, 1, 16, 16, 42, 42, (1, 3, 3), (1, 1, 1), (0, 1, 1), (1, 1, 1), 2, "f16")]:
+        with pytest.raises(C.ConvError) as e:
+            plan(*args, C.VARIANT_TC_STAGED)
+        assert e.value.code == -7
     # ... but the gather kernel past its conditions (O > 128; groups; flip)
     v, bn, _, _ = plan(4, 16, 16, 16, 65, 130, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), 1, "f16")
     assert v == C.VARIANT_TC_GATHER
