@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <numeric>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -1379,6 +1380,36 @@ int launch_tconv(const Problem& P, const void* x, const void* w, void* y, cudaSt
 // input.  The block height is the multiple of 4 up to 32 that wastes the
 // fewest rows of Ho (ties to the taller block); the pipeline takes as many
 // slots (weights of the kH*kW taps + two region planes) as shared memory holds.
+// Raw mode: 16-byte shared-memory wavefronts of one pass of the builders'
+// region loads when region unit q reads pixel (q * stride) mod (Hr*Wr), from
+// rows rx_row bytes apart with pixels 2C bytes apart: per 8-lane phase of a
+// warp, the most distinct 128-byte lines that fall in one 16-byte bank group.
+long long staged_region_wavefronts(int C, int Hr, int Wr, long long rx_row, int stride) {
+  const int npix = Hr * Wr, nB = 2 * npix;
+  long long total = 0;
+  for (int base = 0; base < nB; base += 8) {
+    for (int half = 0; half < 2; ++half) {
+      long long line[8][8];
+      int nl[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int l = 0; l < 8 && base + l < nB; ++l) {
+        const int u = base + l, kk = u & 1;
+        const int pix = static_cast<int>((static_cast<long long>(u >> 1) * stride) % npix);
+        const int r = pix / Wr, c = pix - r * Wr;
+        const long long src = r * rx_row + 2LL * (static_cast<long long>(c) * C + kk * 8);
+        const long long blk = (src >> 4) + half;
+        const int g = static_cast<int>(blk & 7);
+        bool seen = false;
+        for (int k = 0; k < nl[g]; ++k) seen = seen || line[g][k] == (blk >> 3);
+        if (!seen) line[g][nl[g]++] = blk >> 3;
+      }
+      int worst = 0;
+      for (int g = 0; g < 8; ++g) worst = std::max(worst, nl[g]);
+      total += worst;
+    }
+  }
+  return total;
+}
+
 int plan_staged(const Problem& P, int sms, StArgs& a, int& ctas, size_t& smem) {
   if (P.dtype == CONV_F32 || P.G != 1 || P.flip || !plain_input(P)) return CONV_EUNSUPPORTED;
   if (P.s[0] != 1 || P.s[1] != 1 || P.s[2] != 1 || P.O > 128) return CONV_EUNSUPPORTED;
@@ -1429,6 +1460,20 @@ int plan_staged(const Problem& P, int sms, StArgs& a, int& ctas, size_t& smem) {
   a.tiles_w = static_cast<int>(tiles_w);
   a.total_tiles = static_cast<int>(total);
   a.nc16 = (P.C + 15) / 16;
+  // raw mode: the pixel stride whose region loads take the fewest wavefronts
+  // (ties to 1): 13 for 65 channels (10-pixel rows), 1 for 21 or 3
+  a.pix_stride = 1;
+  if (raw) {
+    long long best_w = staged_region_wavefronts(P.C, static_cast<int>(Hr), static_cast<int>(Wr), rx_row, 1);
+    for (int st : {3, 5, 7, 9, 11, 13, 15, 17}) {
+      if (std::gcd(static_cast<long long>(st), Hr * Wr) != 1) continue;
+      const long long wv = staged_region_wavefronts(P.C, static_cast<int>(Hr), static_cast<int>(Wr), rx_row, st);
+      if (wv < best_w) {
+        best_w = wv;
+        a.pix_stride = st;
+      }
+    }
+  }
   a.Hr = static_cast<int>(Hr);
   a.Wr = static_cast<int>(Wr);
   a.plane_bytes = static_cast<uint32_t>(plane);

@@ -75,6 +75,9 @@ struct StArgs {
   int tile_h;            // output rows of a block (N = 8 * tile_h)
   int tiles_h, tiles_w, total_tiles;
   int nc16;              // 16-channel chunks: ceil(C / 16)
+  int pix_stride;        // raw mode: region unit q packs pixel (q * pix_stride) mod (Hr*Wr), a stride
+                         // coprime to Hr*Wr chosen on the host to spread the builders' shared-memory
+                         // reads over the banks
   int Hr, Wr;            // staged region rows / columns
   uint32_t plane_bytes;  // Hr * Wr * 16
   uint32_t tap_bytes;    // one tap's weights in a slot: ceil(O/8) 8-row groups
@@ -323,7 +326,7 @@ __device__ __forceinline__ void st_pre_raw(const StArgs& a, const StTile& t, int
     pr.base[i] = 0u;
     pr.dst[i] = 0u;
     if (u < nB) {
-      const int kk = u & 1, pix = u >> 1;
+      const int kk = u & 1, pix = static_cast<int>((static_cast<long long>(u >> 1) * a.pix_stride) % (a.Hr * a.Wr));
       const int r = pix / a.Wr, c = pix - r * a.Wr;
       const int ih = t.h0 - a.ph + r, iw = t.w0 - a.pw + c;
       pr.used |= 1u << i;
