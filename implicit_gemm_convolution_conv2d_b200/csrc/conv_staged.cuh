@@ -4,9 +4,9 @@
 // O <= 128, one group.
 //
 // The product is issued transposed, y^T[o, m] = sum_k W[o, k] X[m, k]: MMA
-// M = 128 output-channel rows, N = 8 * tile_h
-// output pixels, a block of tile_h x 8 pixels (h x w) of one (n, od) output
-// plane, as in the transposed halo kernel.
+// M = 128 output-channel rows, N = 8 * tile_h output pixels, a block of
+// tile_h x 8 pixels (h x w) of one (n, od) output plane, as in the transposed
+// halo kernel.
 //
 // Operands live in shared memory in the canonical K-major layout WITHOUT
 // swizzle: a core matrix is 8 rows x 16 bytes (8 channels), its rows 16 bytes
@@ -380,8 +380,9 @@ __device__ __forceinline__ void st_pack_pre(const StArgs& a, const StPre& pr, in
 // KH, KW: the filter's height and width when compiled in (3 x 3: the view
 // offsets are computed once and the tap loop is unrolled), 0 for any size.
 // RAW: the builders stage each (block, kd)'s input rows and weights in shared
-// memory first (st_stage_raw) and pack the slots from there (st_pack_raw);
-// otherwise they pack straight from global memory (st_build).
+// memory first (st_stage_raw), decode their units once for that pair
+// (st_pre_raw) and pack its slots from there (st_pack_pre); otherwise they
+// pack straight from global memory (st_build).
 template <bool BF16, int KH, int KW, bool RAW>
 __global__ void __launch_bounds__(kStThreads, 1) conv_fwd_tc_staged_kernel(const StArgs a) {
   extern __shared__ uint8_t smem_raw[];
