@@ -95,7 +95,8 @@ def measured_peaks():
 
 
 # Device and host source files each kernel variant's behaviour depends on: a
-# traffic record taken with ncu stays valid while these files are unchanged.
+# traffic record taken with ncu stays valid while these files are unchanged. Each
+# set holds every local header its headers include.
 _COMMON_SRC = ["conv_fwd.cu", "ptx.cuh", "conv_tc.cuh", "launch.cuh"]
 KERNEL_SOURCES = {
     "tcgen05_tma_im2col": _COMMON_SRC,
@@ -106,15 +107,15 @@ KERNEL_SOURCES = {
     "tcgen05_tma_halo_pair": _COMMON_SRC + ["conv_halo.cuh"],
     "tcgen05_tma_halo_t": _COMMON_SRC + ["conv_halo.cuh", "conv_tct.cuh", "conv_halo_t.cuh"],
     "tcgen05_tma_halo_t_pair": _COMMON_SRC + ["conv_halo.cuh", "conv_tct.cuh", "conv_halo_t.cuh"],
-    "tcgen05_tma_phase": _COMMON_SRC + ["conv_phase.cuh"],
+    "tcgen05_tma_phase": _COMMON_SRC + ["conv_tct.cuh", "conv_phase.cuh"],
     "simt_ffma": ["conv_fwd.cu", "conv_simt.cuh", "ptx.cuh", "launch.cuh"],
     "depthwise_tma": _COMMON_SRC + ["conv_simt.cuh", "conv_dw.cuh"],
-    "depthwise_direct": ["conv_fwd.cu", "conv_simt.cuh", "conv_dw.cuh", "ptx.cuh", "launch.cuh"],
+    "depthwise_direct": ["conv_fwd.cu", "conv_simt.cuh", "conv_dw.cuh", "conv_tc.cuh", "ptx.cuh", "launch.cuh"],
     "simt_wgrad": ["conv_wgrad.cu", "conv_wgrad.cuh", "conv_simt.cuh", "ptx.cuh", "launch.cuh"],
     "tcgen05_tma_phases_pair": _COMMON_SRC + ["conv_tconv.cuh"],
     "tcgen05_staged_t": _COMMON_SRC + ["conv_tct.cuh", "conv_staged.cuh"],
-    "tcgen05_wgrad_pair": ["conv_fwd.cu", "conv_wgrad.cu", "conv_wgrad.cuh", "conv_wgrad_tc.cuh", "conv_tc.cuh",
-                           "ptx.cuh", "launch.cuh"],
+    "tcgen05_wgrad_pair": ["conv_fwd.cu", "conv_wgrad.cu", "conv_wgrad.cuh", "conv_wgrad_tc.cuh", "conv_simt.cuh",
+                           "conv_tc.cuh", "ptx.cuh", "launch.cuh"],
 }
 
 

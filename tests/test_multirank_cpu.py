@@ -108,6 +108,25 @@ def test_kernel_source_sets_cover_every_kernel():
         assert len(bench.kernel_source_hash(name)) == 12
 
 
+def test_kernel_source_sets_are_closed_under_includes():
+    """A kernel's traffic record must go stale when any header its code pulls in
+    changes: every local header included by a header of the set is in the set
+    (the two .cu files, which include every kernel, are the host side and are
+    not followed)."""
+    import re
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = os.path.join(ROOT, "implicit_gemm_convolution_conv2d_b200", "csrc")
+    for name, files in bench.KERNEL_SOURCES.items():
+        for f in files:
+            if not f.endswith(".cuh"):
+                continue
+            with open(os.path.join(csrc, f)) as fh:
+                for inc in re.findall(r'^#include "([^"]+\.cuh)"', fh.read(), re.M):
+                    assert inc in files, (name, f, inc)
+
+
 def test_transposed_and_weight_gradient_counters():
     """A transposed convolution counts the FLOPs of the forward pass it is the
     adjoint of (2 x its input pixels x Cin x taps x Cout/G); the weight
