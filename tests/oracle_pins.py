@@ -369,6 +369,7 @@ _T_GEOMS = [
     (1, 5, 6, 7, 4, 6, (3, 3, 3), (2, 1, 2), (1, 1, 0), (1, 2, 1), 2),
     (1, 1, 9, 8, 6, 3, (1, 4, 4), (1, 2, 3), (0, 1, 2), (1, 1, 1), 3),
     (2, 1, 5, 5, 2, 2, (1, 2, 2), (1, 2, 2), (0, 0, 0), (1, 1, 1), 1),
+    (1, 4, 6, 9, 4, 4, (2, 2, 3), (1, 2, 1), (1, 0, 2), (2, 1, 2), 2),
 ]
 
 

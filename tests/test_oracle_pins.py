@@ -113,6 +113,18 @@ MUTATIONS = {
     "wgrad_tap_sign": [(r"int64_t iw = \(int64_t\)ow \* t->s\[2\] - t->p\[2\] \+ \(int64_t\)kw \* t->d\[2\];",
                         "int64_t iw = (int64_t)ow * t->s[2] - t->p[2] - (int64_t)kw * t->d[2];")],
     "padding_not_zero": [(r"if \(ih < 0 \|\| ih >= sh->H\) continue;", "if (ih < 0 || ih >= sh->H) ih = ih < 0 ? 0 : sh->H - 1;")],
+    "transpose_dilation_dropped": [(r"src_index\(qw, kw, t->s\[2\], t->p\[2\], t->d\[2\], t->W\)",
+                                    "src_index(qw, kw, t->s[2], t->p[2], 1, t->W)")],
+    "transpose_group_offset_dropped": [(r"\* t->Ci \+ \(int64_t\)g \* Cig;", "* t->Ci;")],
+    "transpose_output_padding_ignored": [(r"\(int64_t\)d \* \(k - 1\) \+ 1 \+ op;", "(int64_t)d * (k - 1) + 1;")],
+    "transpose_last_input_row_dropped": [(r"return num < in \? num : -1;", "return num < in - 1 ? num : -1;")],
+    "transpose_magnitude_signed": [(r"mag \+= fabs\(v\);", "mag += v;")],
+    "wgrad_dilation_dropped": [(r"\+ \(int64_t\)kh \* t->d\[1\];", "+ (int64_t)kh;")],
+    "wgrad_stride_wrong_dim": [(r"\(int64_t\)oh \* t->s\[1\]", "(int64_t)oh * t->s[2]")],
+    "wgrad_group_offset_dropped": [(r"\(int64_t\)g \* Cg \+ c\];", "c];")],
+    "wgrad_magnitude_signed": [(r"mag \+= fabs\(gy \* xv\);", "mag += gy * xv;")],
+    "wgrad_taps_transposed": [(r"int64_t q = \(\(\(\(int64_t\)o \* kD \+ kd\) \* t->kH \+ kh\) \* t->kW \+ kw\) \* Cg \+ c;",
+                               "int64_t q = ((((int64_t)o * kD + kd) * t->kW + kw) * t->kH + kh) * Cg + c;")],
 }
 
 
