@@ -125,6 +125,15 @@ MUTATIONS = {
     "wgrad_magnitude_signed": [(r"mag \+= fabs\(gy \* xv\);", "mag += gy * xv;")],
     "wgrad_taps_transposed": [(r"int64_t q = \(\(\(\(int64_t\)o \* kD \+ kd\) \* t->kH \+ kh\) \* t->kW \+ kw\) \* Cg \+ c;",
                                "int64_t q = ((((int64_t)o * kD + kd) * t->kW + kw) * t->kH + kh) * Cg + c;")],
+    "dilation_dropped_depth": [(r"\+ \(int64_t\)kd \* sh->d\[0\];", "+ (int64_t)kd;")],
+    "stride_height_from_width": [(r"\(int64_t\)oh \* sh->s\[1\]", "(int64_t)oh * sh->s[2]")],
+    "pad_depth_sign": [(r"\(int64_t\)od \* sh->s\[0\] - sh->p\[0\]", "(int64_t)od * sh->s[0] + sh->p[0]")],
+    "extent_ceil": [(r"return num / s \+ 1;", "return (num + s - 1) / s + 1;")],
+    "decoder_sign_dropped": [(r"return sign \? -v : v;", "return v;")],
+    "f16_subnormal_scale": [(r"ldexp\(\(double\)m, -24\)", "ldexp((double)m, -25)")],
+    "encoder_truncates": [(r"double r = rint\(a / q\);", "double r = floor(a / q);")],
+    "encoder_subnormal_quantum_dropped": [(r"if \(E < emin\) E = emin;", "")],
+    "encoder_overflow_late": [(r"if \(rv >= ldexp\(1\.0, emax \+ 1\)\)", "if (rv >= ldexp(1.0, emax + 2))")],
 }
 
 
@@ -143,6 +152,8 @@ def _build_mutant(name, edits, tmp_path):
 
 
 def _codec_pins(orc):
+    """The decoders over a stride of all bit patterns and the encoders on edge
+    values, against NumPy (binary16) and torch (bfloat16)."""
     bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
     f16 = np.array([orc.lib.oracle_f16_to_f64(int(b)) for b in bits[::7]])
     ref = bits[::7].view(np.float16).astype(np.float64)
@@ -152,6 +163,13 @@ def _codec_pins(orc):
     refb = torch.from_numpy(bits[::7].astype(np.int16)).view(torch.bfloat16).double().numpy()
     okb = np.isnan(refb)
     assert np.array_equal(bf[~okb], refb[~okb])
+    v = _edge_values()
+    e16 = np.array([orc.lib.oracle_f64_to_f16_rn(float(a)) for a in v], dtype=np.uint16)
+    with np.errstate(over="ignore"):
+        assert np.array_equal(e16, v.astype(np.float16).view(np.uint16))
+    v32 = v.astype(np.float32)
+    eb = np.array([orc.lib.oracle_f64_to_bf16_rn(float(a)) for a in v32.astype(np.float64)], dtype=np.uint16)
+    assert np.array_equal(eb, torch.from_numpy(v32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
