@@ -35,7 +35,11 @@
  * gradient (conv_wgrad), each documented at its declaration below.
  *
  * Ownership: the caller owns every buffer.  conv_fwd allocates nothing, does
- * not synchronise, and returns after queueing its work on `stream`.
+ * not synchronise, and returns after queueing its work on `stream`.  Kernels
+ * may read x and w in whole aligned 16-byte blocks: the block holding a
+ * tensor's last element can be read in full, up to 14 bytes past the tensor's
+ * end but never past that block (which, 16-byte aligned, cannot cross a page);
+ * those bytes never reach y.  Nothing is written outside y.
  * Thread safety: calls may come from several host threads.
  *
  * Errors: every entry point returns CONV_OK (0) or a negative code and never
