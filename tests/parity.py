@@ -30,6 +30,8 @@ def compare(y_gpu, y_ref, s_ref, dtype):
     y = y.reshape(-1)
     y_ref = np.asarray(y_ref, np.float64).reshape(-1)
     s_ref = np.asarray(s_ref, np.float64).reshape(-1)
+    if not (y.size == y_ref.size == s_ref.size):
+        raise ValueError(f"element counts differ: result {y.size}, oracle {y_ref.size}, magnitudes {s_ref.size}")
     rel, ab = TOL[dtype]
     tol = rel * s_ref + ab
     err = np.abs(y - y_ref)
