@@ -160,3 +160,14 @@ def test_reference_arm_loads_only_the_oracle():
     assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
     assert "cpu_model" in line["cpu_baseline"]
     assert maps == {"oracle": True, "product": False}
+    # the rest of the line's contract
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "e2e", "cpu_baseline"):
+        assert key in line, key
+    assert line["value"] > 0 and line["ms_per_step"] > 0 and line["steps"] == 1 and line["warmup"] >= 3
+    assert line["higher_is_better"] is True and line["unit"] == "TFLOP/s" and line["vs_baseline"] is None
+    assert line["config"]["workload"] == "conv2d_f16_n1_56x56_c64_o64_k3" and "sample" in line["config"]
+    cb = line["cpu_baseline"]
+    assert cb["value"] == line["value"] and cb["unit"] == line["unit"] and cb["cores"] >= 1 and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
