@@ -57,3 +57,15 @@ def test_nvidia_smi_lines():
     assert [(x[0], x[1], x[2]) for x in s.samples] == [
         (1965.0, 1965.0, 0), (1800.0, 1965.0, R["sw_power_cap"]),
         (1200.0, 1965.0, R["hw_slowdown"] | R["hw_thermal_slowdown"])]
+
+
+def test_peaks_measured_file_or_labelled_fallback(tmp_path, monkeypatch):
+    """The roofline's denominators: the driver's measured file when present
+    (labelled "measured"), else the pool's earlier measurement (6.65 TB/s copy,
+    1.59 PFLOP/s bf16 burst), labelled "fallback"."""
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    d, src = bench.measured_peaks()
+    assert src == "fallback" and d["hbm_gbs"] == 6650.0 and d["bf16_tflops"] == 1590.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6542.7, "bf16_tflops": 1628.3}')
+    d, src = bench.measured_peaks()
+    assert src == "measured" and d == {"hbm_gbs": 6542.7, "bf16_tflops": 1628.3}
